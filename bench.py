@@ -1,0 +1,487 @@
+#!/usr/bin/env python3
+"""Benchmark of the gated-delta-rule prefill / decode kernels on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--chunk 64|16] [--no-extras]
+
+A step is one gdn_prefill call over one batch of the workload (default
+prefill_b1_h16_t512: one 512-token sequence, 16 heads, head dim 128 -- the
+single-sequence, scalar-gate, 512-token setting of the ROCmFPX gated-delta-net
+prefill note, bittide.aicompass.dev article d2880479, opening post).  Inputs
+are synthetic, seeded, resident in HBM before timing.  L2 (126 MB) is flushed
+by writing a 256 MiB buffer before every timed step; each step is timed with
+CUDA events on the launching stream, and the sum over K steps is the timed
+total.  With N > 1 (torchrun) every rank runs its own independent batch (weak
+scaling, no collective on the data path) and the max over ranks is reported.
+
+Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
+on the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gated_deltanet_linear_20_b200 import inputs as gin  # noqa: E402
+
+METRIC = "GDN prefill tokens/s and decode state GB/s at 1 B200; % of roofline"
+D = 128
+L2_FLUSH_BYTES = 256 << 20
+STATE_BYTES = D * D * 4
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PREFILL_SOURCES = ["gated_deltanet_linear_20_b200/csrc/gdn_prefill.cu",
+                   "gated_deltanet_linear_20_b200/csrc/sm100.cuh"]
+DECODE_SOURCES = ["gated_deltanet_linear_20_b200/csrc/gdn_decode.cu"]
+
+
+# ------------------------------------------------------------------ algorithmic work
+def prefill_bytes(B, T, H, has_s0):
+    """q, k, v bf16 + g, beta fp32 + o fp32 per token-head, plus the final state
+    (and the initial state when one is read)."""
+    per_token_head = 3 * D * 2 + 2 * 4 + D * 4          # 1288 B
+    return B * T * H * per_token_head + B * H * STATE_BYTES * (2 if has_s0 else 1)
+
+
+def prefill_flops(B, T, H, C=64):
+    """Chunk GEMM FLOPs of the chunked form: 6 D^2 + 10 C D per token-head,
+    always counted at C = 64 so the chunk size cannot inflate it."""
+    return B * T * H * (6 * D * D + 10 * C * D)
+
+
+def decode_bytes(B, H):
+    """Per step: the fp32 state read and written once, plus q, k, v, g, beta, o."""
+    return B * H * (2 * STATE_BYTES + 3 * D * 2 + 2 * 4 + D * 4)
+
+
+def decode_state_bytes(B, H):
+    return B * H * 2 * STATE_BYTES
+
+
+# ------------------------------------------------------------------ helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(key, paths):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            rec = json.load(f).get(key)
+    except Exception:
+        return None
+    if not rec or rec.get("kernel_sha") != source_sha(paths):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]),
+                                 hw=f[5], hwt=f[6], swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        smax = max(r["smax"] for r in rows)
+        busy = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = sorted({name for r in rows for name, key in
+                          (("hw_slowdown", "hw"), ("hw_thermal_slowdown", "hwt"),
+                           ("sw_thermal_slowdown", "swt"), ("sw_power_cap", "pcap"))
+                          if r[key].lower() == "active"})
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy), "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    """Max of a float over all ranks (every rank gets it)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(fn, steps, warmup, flush, stream):
+    """W untimed warm-up steps, then K steps each bracketed by CUDA events on
+    `stream` with an L2 flush before (outside) each.  Returns per-step ms."""
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for s, e in evs:
+        flush()
+        s.record(stream)
+        fn()
+        e.record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in evs]
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, world, rank, local):
+    from gated_deltanet_linear_20_b200 import gdn
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = gin.WORKLOADS[args.workload]
+    if w.is_decode:
+        raise SystemExit("--workload must be a prefill workload (decode is measured as an extra)")
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush = lambda: flush_buf.fill_(1.0)
+
+    d = gin.workload_inputs(w, seed=1000 + rank, device=str(dev))
+    B, T, H = w.B, w.T, w.H
+    o = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
+    S_T = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    call = lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
+                               chunk=args.chunk, o=o, S_T=S_T)
+
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        step_ms = time_steps(call, args.steps, args.warmup, flush, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = B * T
+    value = tokens_per_step * world * args.steps / (total_ms / 1e3)
+
+    nbytes = prefill_bytes(B, T, H, d["S0"] is not None)
+    launch_ms = statistics.mean(step_ms)  # one kernel launch per step
+    achieved = nbytes / (launch_ms / 1e3) / 1e9
+    flops = prefill_flops(B, T, H)
+    traffic = committed_traffic(f"{args.workload}/chunk{args.chunk}", PREFILL_SOURCES)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6.65 TB/s",
+                "algorithmic_bytes_per_launch": nbytes,
+                "tensor": {"achieved_tflops": round(flops / (launch_ms / 1e3) / 1e12, 2),
+                           "peak_tflops": peaks["bf16_tflops"],
+                           "frac": round(flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+                           "flops_per_launch": flops}}
+
+    # end to end through the public API: pinned host inputs -> device -> prefill -> host
+    host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in d.items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    s_host = torch.empty(S_T.shape, dtype=S_T.dtype, pin_memory=True)
+    dev_in = {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in host.items()}
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                dev_in[k].copy_(v, non_blocking=True)
+        gdn.prefill(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"], dev_in["beta"],
+                    dev_in["S0"], chunk=args.chunk, o=o, S_T=S_T)
+        o_host.copy_(o, non_blocking=True)
+        s_host.copy_(S_T, non_blocking=True)
+
+    barrier(world)
+    e2e_ms = time_steps(e2e_step, args.steps, args.warmup, flush, stream)
+    barrier(world)
+    e2e_total = max_over_ranks(sum(e2e_ms), world)
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = o_host.numel() * 4 + s_host.numel() * 4
+    e2e = {"value": round(tokens_per_step * world * args.steps / (e2e_total / 1e3), 1),
+           "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    extras = None
+    if not args.no_extras:
+        extras = run_extras(args, dev, stream, flush, peaks, rank)
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline(w, budget_s=args.cpu_seconds)
+
+    clocks = clk.summary()
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; q,k L2-normalised bf16, v bf16, g=logsigmoid, beta=sigmoid)",
+            "config": {"workload": args.workload, "B": B, "T": T, "H": H, "Dk": D, "Dv": D,
+                       "chunk": args.chunk, "tokens_per_step_per_gpu": tokens_per_step,
+                       "l2": "flushed (256 MiB write) before every timed step",
+                       "parallelism": f"dp{world} (independent batches, no collective)"},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps,
+            "clocks": clocks, "cpu_baseline": cpu, "impl": "ours"}
+    if extras is not None:
+        line["extras"] = extras
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_extras(args, dev, stream, flush, peaks, rank):
+    """Other measured workloads reported beside the headline: chunk 16 on the
+    headline workload, the batched decode step, and the large prefill."""
+    from gated_deltanet_linear_20_b200 import gdn
+    out = {}
+    steps = max(3, min(args.steps, 10))
+    # chunk 16 on the headline workload
+    w = gin.WORKLOADS[args.workload]
+    d = gin.workload_inputs(w, seed=1000 + rank, device=str(dev))
+    other = 16 if args.chunk == 64 else 64
+    ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
+                                        chunk=other), steps, 3, flush, stream)
+    t = statistics.mean(ms)
+    out[f"{args.workload}/chunk{other}"] = {
+        "tokens_per_s": round(w.B * w.T / (t / 1e3), 1), "ms": round(t, 5),
+        "hbm_frac": round(prefill_bytes(w.B, w.T, w.H, d["S0"] is not None) / (t / 1e3) / 1e9
+                          / peaks["hbm_gbs"], 4)}
+    del d
+    # decode: L2 flushed before every step (headline) and 256 back-to-back steps (L2-warm)
+    wd = gin.WORKLOADS["decode_b64_h16"]
+    dd = gin.workload_inputs(wd, seed=2000 + rank, device=str(dev))
+    S = dd["S"].clone()
+    o = torch.empty((wd.B, wd.H, D), dtype=torch.float32, device=dev)
+    it = [0]
+
+    def dstep():
+        i = it[0] % wd.decode_steps
+        gdn.decode_step(dd["q"][i], dd["k"][i], dd["v"][i], dd["g"][i], dd["beta"][i], S, o=o)
+        it[0] += 1
+    ms = time_steps(dstep, 64, 5, flush, stream)
+    t = statistics.mean(ms)
+    sb = decode_state_bytes(wd.B, wd.H)
+    gbs = sb / (t / 1e3) / 1e9
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(wd.decode_steps):
+        dstep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_warm = e0.elapsed_time(e1) / wd.decode_steps
+    traffic = committed_traffic("decode_b64_h16", DECODE_SOURCES)
+    out["decode_b64_h16"] = {
+        "state_GB_per_s": round(gbs, 1), "us_per_step": round(t * 1e3, 3),
+        "roofline": {"bound": "hbm", "achieved": round(decode_bytes(wd.B, wd.H) / (t / 1e3) / 1e9, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(decode_bytes(wd.B, wd.H) / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "traffic": traffic},
+        "l2": "flushed before every step",
+        "back_to_back_256_steps": {"us_per_step": round(t_warm * 1e3, 3),
+                                   "state_GB_per_s": round(sb / (t_warm / 1e3) / 1e9, 1),
+                                   "l2": "warm: the 64 MiB state fits in the 126 MB L2"}}
+    del dd, S
+    # large prefill (inputs 1.6 GB > L2)
+    wl = gin.WORKLOADS["prefill_b4_h32_t32768"]
+    dl = gin.workload_inputs(wl, seed=3000 + rank, device=str(dev))
+    ol = torch.empty((wl.B, wl.T, wl.H, D), dtype=torch.float32, device=dev)
+    sl = torch.empty((wl.B, wl.H, D, D), dtype=torch.float32, device=dev)
+    ms = time_steps(lambda: gdn.prefill(dl["q"], dl["k"], dl["v"], dl["g"], dl["beta"], None,
+                                        chunk=64, o=ol, S_T=sl), 3, 2, flush, stream)
+    t = statistics.mean(ms)
+    nb = prefill_bytes(wl.B, wl.T, wl.H, False)
+    fl = prefill_flops(wl.B, wl.T, wl.H)
+    out["prefill_b4_h32_t32768/chunk64"] = {
+        "tokens_per_s": round(wl.B * wl.T / (t / 1e3), 1), "ms": round(t, 4),
+        "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                     "traffic": committed_traffic("prefill_b4_h32_t32768/chunk64", PREFILL_SOURCES)},
+        "tensor_frac": round(fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
+    del dl, ol, sl
+    torch.cuda.empty_cache()
+    return out
+
+
+# ------------------------------------------------------------------ the oracle (CPU)
+def cpu_baseline(w, budget_s=10.0):
+    """The fp64 oracle as it stands, on the host cores, over a bounded sample of
+    the workload: whole batches while they fit the budget, else a subset of
+    chains.  Returns tokens/s (token-heads / H, so comparable to the GPU line)."""
+    import oracle
+    d = gin.workload_inputs(w, seed=1000)
+    chains = w.B * w.H
+    t0 = time.perf_counter()
+    oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=[0])
+    one_chain = time.perf_counter() - t0
+    cores = oracle.num_threads()
+    per_pass = one_chain * chains / max(1, min(cores, chains))
+    if per_pass <= budget_s:
+        passes, done, t0 = 0, 0.0, time.perf_counter()
+        while True:
+            oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+            passes += 1
+            done = time.perf_counter() - t0
+            if done > budget_s / 2 or passes >= 50:
+                break
+        tokens = w.B * w.T * passes
+        sample = f"{passes} full pass(es) of {args_name(w)} ({chains} chains x {w.T} tokens)"
+    else:
+        n = max(1, min(chains, cores))
+        ids = list(range(n))
+        t0 = time.perf_counter()
+        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=ids)
+        done = time.perf_counter() - t0
+        tokens = w.T * n / w.H
+        sample = f"{n} of {chains} chains of {args_name(w)} ({w.T} tokens each)"
+    return {"value": round(tokens / done, 2), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle", "sample": sample, "seconds": round(done, 3)}
+
+
+def args_name(w):
+    return w.name
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = gin.WORKLOADS[args.workload]
+    import oracle
+    d = gin.workload_inputs(w, seed=1000)
+    chains = w.B * w.H
+    cores = oracle.num_threads()
+    t0 = time.perf_counter()
+    oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=[0])
+    per_chain = time.perf_counter() - t0
+    # each step: as many chains as fit ~2 s of host time (the whole batch when it does)
+    n = chains if per_chain * chains / max(1, min(cores, chains)) <= 2.0 else \
+        max(1, min(chains, int(2.0 * cores / max(per_chain, 1e-6))))
+    ids = None if n == chains else list(range(n))
+    for _ in range(args.warmup):
+        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=ids)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=ids)
+    total = time.perf_counter() - t0
+    tokens_per_step = w.T * n / w.H
+    value = tokens_per_step * args.steps / total
+    sample = (f"full batch of {w.name} per step" if ids is None else
+              f"{n} of {chains} chains of {w.name} per step ({w.T} tokens each)")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "Dk": D, "Dv": D,
+                       "chunk": args.chunk, "parallelism": "host cores (OpenMP over chains)"},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_b1_h16_t512",
+                    choices=[k for k, v in gin.WORKLOADS.items() if not v.is_decode])
+    ap.add_argument("--chunk", type=int, default=64, choices=[16, 64])
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,26 @@
+"""Gated delta rule (gated DeltaNet) prefill and decode for NVIDIA B200 (sm_100a).
+
+The compute lives in ``libgdn_b200.so`` (hand-written CUDA, C ABI declared in
+``include/gdn.h``); ``gdn.py`` is a thin ctypes binding that only marshals
+torch tensors and the current CUDA stream into that ABI.  There is no CPU
+fallback: calling into the binding without the built library raises.
+
+    from gated_deltanet_linear_20_b200 import prefill, decode_step
+    o, S_T = prefill(q, k, v, g, beta, S0=None, chunk=64)
+    o = decode_step(q, k, v, g, beta, S)       # S updated in place
+
+The binding is imported lazily so that ``inputs`` (the seeded input
+generator) can be used without loading the CUDA library.
+"""
+from __future__ import annotations
+
+__all__ = ["prefill", "decode_step", "abi_version", "status_str", "query_status",
+           "GDNError"]
+
+
+def __getattr__(name):
+    if name in ("prefill", "decode_step", "abi_version", "status_str", "query_status",
+                "GDNError", "prefill_host", "library_path"):
+        import importlib
+        return getattr(importlib.import_module(__name__ + ".gdn"), name)
+    raise AttributeError(name)

@@ -1,0 +1,164 @@
+// C-ABI entry points of libgdn_b200.so (declared in include/gdn.h): argument
+// validation, TMA descriptor encoding on the host, launches on the caller's
+// stream.  No device memory is allocated here and no state is kept between
+// calls except the cached driver entry point of cuTensorMapEncodeTiled.
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gdn_internal.h"
+
+namespace {
+
+constexpr int kHeadDim = 128;
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// The current device must be an sm_100 part (the only architecture built).
+int check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_LAUNCH;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return GDN_ERR_LAUNCH;
+  if (major != 10 || minor != 0) return GDN_ERR_UNSUPPORTED;
+  return GDN_OK;
+}
+
+// 4-D view [B][T][H][128] of a bf16 activation; box = `box_inner` features x
+// 64 tokens of one head.  Tokens past T read as zeros.
+bool encode_act(CUtensorMap* map, const void* base, int B, int T, int H, int box_inner,
+                CUtensorMapSwizzle swz) {
+  auto enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {cuuint64_t(kHeadDim), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(kHeadDim) * 2, cuuint64_t(H) * kHeadDim * 2,
+                                 cuuint64_t(T) * H * kHeadDim * 2};
+  const cuuint32_t box[4] = {cuuint32_t(box_inner), 1, 64, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+const char* gdn_status_str(int code) {
+  switch (code) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_NULL: return "a required pointer is NULL";
+    case GDN_ERR_ALIGN: return "misaligned pointer (q/k/v/o/S need 16 bytes, g/beta 4 bytes)";
+    case GDN_ERR_SHAPE: return "negative size or problem larger than 2^31-1 elements";
+    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims must be 128, chunk 16 or 64, device sm_100)";
+    case GDN_ERR_ALIAS: return "output overlaps an input";
+    case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
+    case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+    default: return "unknown status code";
+  }
+}
+
+int gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
+                int chunk, int* status, void* stream) {
+  if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
+  const long long chains = (long long)B * H;
+  const long long act = chains * T * kHeadDim;
+  if (act > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  if (chains == 0) return GDN_OK;
+  if (!S_T) return GDN_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
+  if (!aligned(S_T, 16) || (S0 && !aligned(S0, 16))) return GDN_ERR_ALIGN;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+                !aligned(g, 4) || !aligned(beta, 4)))
+    return GDN_ERR_ALIGN;
+  const size_t act_bf16 = size_t(act) * 2, act_f32 = size_t(act) * 4;
+  const size_t gate_bytes = size_t(chains) * T * 4, state_bytes = size_t(chains) * kHeadDim * kHeadDim * 4;
+  if (T > 0 && (overlaps(o, act_f32, q, act_bf16) || overlaps(o, act_f32, k, act_bf16) ||
+                overlaps(o, act_f32, v, act_bf16) || overlaps(o, act_f32, g, gate_bytes) ||
+                overlaps(o, act_f32, beta, gate_bytes) || overlaps(o, act_f32, S0, state_bytes) ||
+                overlaps(o, act_f32, S_T, state_bytes)))
+    return GDN_ERR_ALIAS;
+  if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+
+  gdn::PrefillArgs a{g, beta, S0, o, S_T, B, T, H, status};
+  CUtensorMap tq{}, tk{}, tv{};
+  if (T > 0) {
+    if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return GDN_ERR_LAUNCH;
+  }
+  return gdn::launch_prefill(tq, tk, tv, a, chunk, static_cast<cudaStream_t>(stream)) == 0
+             ? GDN_OK
+             : GDN_ERR_LAUNCH;
+}
+
+int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, float* S, float* o, int B, int H, int Dk, int Dv,
+                    int* status, void* stream) {
+  (void)status;  // the decode kernel has no device-side waits
+  if (B < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (Dk != kHeadDim || Dv != kHeadDim) return GDN_ERR_UNSUPPORTED;
+  const long long heads = (long long)B * H;
+  if (heads * kHeadDim * kHeadDim > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  if (heads == 0) return GDN_OK;
+  if (!q || !k || !v || !g || !beta || !S || !o) return GDN_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(S, 16) ||
+      !aligned(o, 16) || !aligned(g, 4) || !aligned(beta, 4))
+    return GDN_ERR_ALIGN;
+  const size_t vec_bf16 = size_t(heads) * kHeadDim * 2, vec_f32 = size_t(heads) * kHeadDim * 4;
+  const size_t state_bytes = size_t(heads) * kHeadDim * kHeadDim * 4, gate_bytes = size_t(heads) * 4;
+  if (overlaps(o, vec_f32, q, vec_bf16) || overlaps(o, vec_f32, k, vec_bf16) ||
+      overlaps(o, vec_f32, v, vec_bf16) || overlaps(o, vec_f32, g, gate_bytes) ||
+      overlaps(o, vec_f32, beta, gate_bytes) || overlaps(o, vec_f32, S, state_bytes) ||
+      overlaps(S, state_bytes, q, vec_bf16) || overlaps(S, state_bytes, k, vec_bf16) ||
+      overlaps(S, state_bytes, v, vec_bf16) || overlaps(S, state_bytes, g, gate_bytes) ||
+      overlaps(S, state_bytes, beta, gate_bytes))
+    return GDN_ERR_ALIAS;
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+  gdn::DecodeArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H};
+  return gdn::launch_decode(a, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
+}
+
+int gdn_query_status(const int* status_dev, void* stream) {
+  if (!status_dev) return GDN_ERR_NULL;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN_ERR_LAUNCH;
+  int v = 0;
+  if (cudaMemcpy(&v, status_dev, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GDN_ERR_LAUNCH;
+  return v;
+}
+
+}  // extern "C"

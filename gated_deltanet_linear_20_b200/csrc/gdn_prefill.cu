@@ -1,0 +1,590 @@
+// Chunked gated-delta-rule prefill for sm_100a: TMA-staged bf16 tiles,
+// tcgen05 MMAs accumulating in tensor memory, fp32 state carried across
+// chunks.
+//
+// Recurrence (per sequence b, head h; S in R^{Dv x Dk}):
+//   S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t.
+// The ROCmFPX gated-delta-net prefill note (bittide.aicompass.dev article
+// d2880479, opening post) moves this prefill from one token at a time to
+// 16-token chunks with the state in F32 accumulators, scalar gate, head dim
+// 128; here chunks of 16 or 64 tokens run on the 5th-generation tensor cores.
+//
+// Chunked form used (derived from the recurrence; tokens i, j of one chunk,
+// S_c the state entering it, gamma = inclusive cumulative sum of g inside the
+// chunk, Gamma = exp(gamma), Dec_ij = exp(gamma_i - gamma_j)):
+//   A     = strict_tril(diag(beta) K K^T .* Dec)          (chunk x chunk)
+//   T     = (I + A)^{-1}                                  (unit lower triangular)
+//   X^T   = V^T diag(beta) - diag-cols(beta Gamma) (S_c K^T)        (Dv x chunk)
+//   Dl^T  = X^T T^T                                       (the delta-rule residuals)
+//   O^T   = diag-cols(Gamma) (S_c Q^T) + Dl^T Mq^T,  Mq = tril(Q K^T .* Dec)
+//   S_out = Gamma_last S_c + Dl^T diag(exp(gamma_last - gamma)) K
+//
+// One CTA (128 threads = one warpgroup) owns one (b, h) chain and walks its
+// tokens in tiles of 64 (one TMA tile); with chunk = 16 each tile holds four
+// chunks, processed in order.  Thread t owns TMEM lane t, i.e. state row t
+// (the Dv index) in every Dv-indexed product.  The fp32 state lives in the
+// threads' registers; the tensor core sees it as a bf16 hi/lo pair in TMEM
+// (the A operand of the S-dependent products).  Every operand derived inside
+// the kernel (S, X, T, the residuals, Mq) is fed to the MMA as hi + lo bf16
+// parts (hi = bf16(x), lo = bf16(x - hi)) so the products keep ~16 bits of
+// mantissa; q, k and v are exact bf16 inputs.
+//
+// Tensor memory (512 columns, fp32 unless noted):
+//   [  0,128) U   : state update Dl^T diag(.) K                  (lane dv, col dk)
+//   [128,192) SHI : S hi as bf16 pairs (A operand)               (lane dv, col dk/2)
+//   [192,256) SLO : S lo
+//   [256,384) ZQ  : [S K^T | S Q^T]                              (lane dv, col token)
+//   [384,448) PD  : [K;Q] K^T (lanes 0..127 = rows of [K;Q]), later Dl^T
+//   [448,512) OI  : Dl^T Mq^T                                    (lane dv, col token)
+#include "gdn_internal.h"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int NT = 64;  // tokens per TMA tile
+constexpr int NTHREADS = 128;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_U = 0, TM_SHI = 128, TM_SLO = 192, TM_ZQ = 256, TM_PD = 384, TM_OI = 448;
+
+// Shared memory map (offsets from a 1024-byte aligned base).
+constexpr uint32_t SM_KQ0 = 0;        // 32 KB: [K dk0-63 | Q dk0-63 | K dk64-127 | Q dk64-127]
+constexpr uint32_t SM_KQ1 = 32768;    //        each a 64-row x 128-byte SW128 box
+constexpr uint32_t SM_V0 = 65536;     // 16 KB: V tile [64 tokens][128] bf16, unswizzled
+constexpr uint32_t SM_V1 = 81920;
+constexpr uint32_t SM_MQH = 98304;    // 8 KB: Mq rows i, K-major SW128 (64 x 64 bf16)
+constexpr uint32_t SM_MQL = 106496;
+constexpr uint32_t SM_TH = 114688;    // 8 KB: T rows i (64 x 64)
+constexpr uint32_t SM_TL = 122880;
+constexpr uint32_t SM_XH = 131072;    // 16 KB: X^T rows dv (128 x 64); reused for the
+constexpr uint32_t SM_XL = 147456;    //        decay-scaled residuals once X is consumed
+constexpr uint32_t SM_DH = 163840;    // 16 KB: Dl^T rows dv (128 x 64)
+constexpr uint32_t SM_DL = 180224;
+constexpr uint32_t SM_AT = 196608;    // 16 KB: A^T fp32 [64][64] for the triangular solve
+constexpr uint32_t SM_MISC = 212992;  // gates, barriers, TMEM slot
+constexpr uint32_t MISC_G = 0, MISC_B = 256, MISC_GAM2 = 512, MISC_GAM = 768, MISC_BG = 1024,
+                   MISC_DF = 1280, MISC_GC = 1536, MISC_BAR = 1600, MISC_TMEM = 1632,
+                   MISC_ABORT = 1636;
+constexpr uint32_t SMEM_USED = SM_MISC + 2048;
+constexpr uint32_t TILE_TX_BYTES = 4 * 8192 + 16384;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
+
+constexpr float LOG2E = 1.4426950408889634f;
+
+// Byte offset of 16-byte chunk `c` (8 bf16 along K) of row `r` in a K-major
+// SW128 tile whose rows are 128 bytes and whose 8-row groups are 1024 B apart.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + (((c ^ r) & 7) << 4));
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+// Splits 8 floats into hi/lo bf16 and stores them as chunk `c` of row `r` in two tiles.
+__device__ __forceinline__ void store_split8(uint32_t hi_tile, uint32_t lo_tile, int r, int c,
+                                             const float* x) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat16 h0, l0, h1, l1;
+    split_bf16(x[2 * e], h0, l0);
+    split_bf16(x[2 * e + 1], h1, l1);
+    h[e] = pack_bf16x2(h0, h1);
+    l[e] = pack_bf16x2(l0, l1);
+  }
+  const uint32_t off = sw128_off(r, c);
+  st_shared_v4(hi_tile + off, h[0], h[1], h[2], h[3]);
+  st_shared_v4(lo_tile + off, l[0], l[1], l[2], l[3]);
+}
+
+// Writes the hi/lo bf16 split of the fp32 state row (this thread's lane) into
+// the SHI / SLO tensor-memory columns (two bf16 per 32-bit column).
+__device__ __forceinline__ void store_state_split(uint32_t tlane, const float (&S)[D]) {
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      __nv_bfloat16 h0, l0, h1, l1;
+      split_bf16(S[32 * g + 2 * e], h0, l0);
+      split_bf16(S[32 * g + 2 * e + 1], h1, l1);
+      hi[e] = pack_bf16x2(h0, h1);
+      lo[e] = pack_bf16x2(l0, l1);
+    }
+    tmem_st16(tlane + TM_SHI + 16 * g, hi);
+    tmem_st16(tlane + TM_SLO + 16 * g, lo);
+  }
+}
+
+struct Flow {
+  uint32_t mma_bar;
+  uint32_t mma_phase;
+  volatile int* abort_flag;
+  int* status;
+  // All threads wait for the last commit; a wait that gives up flags the CTA.
+  __device__ __forceinline__ void wait_mma() {
+    if (!mbar_wait_bounded(mma_bar, mma_phase, WAIT_LIMIT_NS)) fail();
+    mma_phase ^= 1u;
+    tc_fence_after();
+  }
+  __device__ __forceinline__ void fail() {
+    *abort_flag = 1;
+    if (status) atomicExch(status, GDN_ERR_DEVICE_TIMEOUT);
+  }
+};
+
+template <int C>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillArgs p) {
+  static_assert(C == 16 || C == 64, "chunk must be 16 or 64");
+  constexpr int NSUB = NT / C;  // chunks per TMA tile
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int chain = blockIdx.x;
+  const int b = chain / p.H;
+  const int h = chain - b * p.H;
+  const int T = p.T, H = p.H;
+
+  float* s_g = reinterpret_cast<float*>(sm + SM_MISC + MISC_G);
+  float* s_b = reinterpret_cast<float*>(sm + SM_MISC + MISC_B);
+  float* s_gam2 = reinterpret_cast<float*>(sm + SM_MISC + MISC_GAM2);
+  float* s_Gam = reinterpret_cast<float*>(sm + SM_MISC + MISC_GAM);
+  float* s_bG = reinterpret_cast<float*>(sm + SM_MISC + MISC_BG);
+  float* s_df = reinterpret_cast<float*>(sm + SM_MISC + MISC_DF);
+  float* s_GC = reinterpret_cast<float*>(sm + SM_MISC + MISC_GC);
+  const uint32_t bar_tma0 = sb + SM_MISC + MISC_BAR;
+  const uint32_t bar_mma = bar_tma0 + 16;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + SM_MISC + MISC_TMEM);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + SM_MISC + MISC_ABORT);
+  const float* AT = reinterpret_cast<const float*>(sm + SM_AT);
+
+  if (tid == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    mbar_init(bar_tma0, 1);
+    mbar_init(bar_tma0 + 8, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    *s_abort = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(s_tmem), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t tlane = tmem + (uint32_t(warp * 32) << 16);  // this warp's lane quarter
+
+  Flow flow{bar_mma, 0u, s_abort, p.status};
+  const int ntiles = (T + NT - 1) / NT;
+  int tma_issued = 0;  // tiles whose TMA was issued (thread 0's view)
+  int tma_done = 0;    // tiles whose TMA completion was observed
+
+  auto issue_tile = [&](int c) {
+    const int st = c & 1;
+    const uint32_t kq = sb + (st ? SM_KQ1 : SM_KQ0);
+    const uint32_t vt = sb + (st ? SM_V1 : SM_V0);
+    const uint32_t bar = bar_tma0 + 8 * st;
+    mbar_arrive_expect_tx(bar, TILE_TX_BYTES);
+    tma_load_4d(kq + 0, &tm_k, bar, 0, h, c * NT, b);
+    tma_load_4d(kq + 8192, &tm_q, bar, 0, h, c * NT, b);
+    tma_load_4d(kq + 16384, &tm_k, bar, 64, h, c * NT, b);
+    tma_load_4d(kq + 24576, &tm_q, bar, 64, h, c * NT, b);
+    tma_load_4d(vt, &tm_v, bar, 0, h, c * NT, b);
+  };
+
+  // ---- initial state: row dv = tid of S0 (or zeros), kept in fp32 registers
+  float S[D];
+  const int dv = tid;
+  if (p.S0 != nullptr) {
+    const float4* src =
+        reinterpret_cast<const float4*>(p.S0 + (size_t(chain) * D + dv) * D);
+#pragma unroll
+    for (int q4 = 0; q4 < D / 4; ++q4) {
+      const float4 x = __ldg(src + q4);
+      S[4 * q4] = x.x;
+      S[4 * q4 + 1] = x.y;
+      S[4 * q4 + 2] = x.z;
+      S[4 * q4 + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < D; ++e) S[e] = 0.f;
+  }
+  store_state_split(tlane, S);
+  tc_fence_before();
+
+  float g_next = 0.f, b_next = 0.f;
+  if (tid < NT && tid < T) {
+    const size_t gi = (size_t(b) * T + tid) * H + h;
+    g_next = __ldg(p.g + gi);
+    b_next = __ldg(p.beta + gi);
+  }
+  if (tid == 0 && ntiles > 0) {
+    issue_tile(0);
+    tma_issued = 1;
+  }
+
+  for (int c = 0; c < ntiles; ++c) {
+    const int st = c & 1;
+    const int t0 = c * NT;
+    const uint32_t kq = sb + (st ? SM_KQ1 : SM_KQ0);
+    const uint8_t* vtile = sm + (st ? SM_V1 : SM_V0);
+
+    // ---- gates of this tile; prefetch the next tile (gates to registers, q/k/v by TMA)
+    if (tid < NT) {
+      s_g[tid] = g_next;
+      s_b[tid] = b_next;
+      g_next = 0.f;
+      b_next = 0.f;
+      const int t = t0 + NT + tid;
+      if (t < T) {
+        const size_t gi = (size_t(b) * T + t) * H + h;
+        g_next = __ldg(p.g + gi);
+        b_next = __ldg(p.beta + gi);
+      }
+    }
+    if (tid == 0 && c + 1 < ntiles) {
+      issue_tile(c + 1);
+      tma_issued = c + 2;
+    }
+    __syncthreads();
+    if (tid < NT) {  // gamma (log2 units), inclusive within the chunk
+      const int cs = (tid / C) * C;
+      float acc = 0.f;
+      for (int t = cs; t <= tid; ++t) acc += s_g[t];
+      s_gam2[tid] = acc * LOG2E;
+    }
+    __syncthreads();
+    if (tid < NT) {
+      const int last = (tid / C) * C + C - 1;
+      const float gi = s_gam2[tid], gl = s_gam2[last];
+      const float G = exp2f(gi);
+      s_Gam[tid] = G;
+      s_bG[tid] = s_b[tid] * G;
+      s_df[tid] = exp2f(gl - gi);
+      if (tid == last) s_GC[tid / C] = exp2f(gl);
+    }
+    if (mbar_wait_bounded(bar_tma0 + 8 * st, (c >> 1) & 1, WAIT_LIMIT_NS))
+      tma_done = c + 1;
+    else
+      flow.fail();
+    __syncthreads();
+    if (*s_abort) goto teardown;
+
+    // ---- P = [K; Q] K^T : M=128 (rows of [K;Q]), N=64 (tokens j), K=128 (dk)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 64, 0, 0, 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+        mma_ss(tmem + TM_PD, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(kq + off, 16, 1024), id,
+               kk > 0);
+      }
+      mma_commit(bar_mma);
+    }
+    flow.wait_mma();
+
+    // ---- masks and decays: rows 0..63 -> A^T (fp32, for the solve); rows 64..127 -> Mq
+    {
+      const int i = tid & (NT - 1);
+      const int cs = (i / C) * C;
+      const float gi = s_gam2[i];
+      const float bi = s_b[i];
+      float* ATw = reinterpret_cast<float*>(sm + SM_AT);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float P[16];
+        tmem_ld16(tlane + TM_PD + 16 * q, P);
+        if (tid < NT) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int j = 16 * q + e;
+            const bool keep = (j >= cs) && (j < i);
+            const float a = bi * exp2f(gi - s_gam2[j]) * P[e];
+            ATw[j * NT + i] = keep ? a : 0.f;
+          }
+        } else {
+          float m[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int j = 16 * q + e;
+            const bool keep = (j >= cs) && (j <= i);
+            const float x = exp2f(gi - s_gam2[j]) * P[e];
+            m[e] = keep ? x : 0.f;
+          }
+          store_split8(sb + SM_MQH, sb + SM_MQL, i, 2 * q, m);
+          store_split8(sb + SM_MQH, sb + SM_MQL, i, 2 * q + 1, m + 8);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- T = (I + A)^{-1}: thread r < 64 forms row r by back substitution,
+    //      x_j = [j == r] - sum_{i>j} x_i A_ij, over its chunk's block.
+    if (tid < NT) {
+      const int r = tid;
+      const int base = (r / C) * C;
+      const int rr = r - base;
+      float x[C];
+#pragma unroll
+      for (int j = 0; j < C; ++j) x[j] = 0.f;
+#pragma unroll
+      for (int j = C - 1; j >= 0; --j) {
+        float acc = (j == rr) ? 1.f : 0.f;
+        const float* row = AT + (base + j) * NT + base;
+#pragma unroll
+        for (int i4 = ((j + 1) & ~3); i4 < C; i4 += 4) {
+          const float4 a = *reinterpret_cast<const float4*>(row + i4);
+          acc = fmaf(-x[i4], a.x, acc);
+          acc = fmaf(-x[i4 + 1], a.y, acc);
+          acc = fmaf(-x[i4 + 2], a.z, acc);
+          acc = fmaf(-x[i4 + 3], a.w, acc);
+        }
+        x[j] = acc;
+      }
+      // nonzero entries sit in columns [base, base + C) of row r
+#pragma unroll
+      for (int rc = 0; rc < C / 8; ++rc) store_split8(sb + SM_TH, sb + SM_TL, r, base / 8 + rc, x + 8 * rc);
+      if constexpr (C < NT) {
+        const float zero8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ch = 0; ch < NT / 8; ++ch)
+          if (ch < base / 8 || ch >= (base + C) / 8) store_split8(sb + SM_TH, sb + SM_TL, r, ch, zero8);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+#pragma unroll 1
+    for (int s = 0; s < NSUB; ++s) {
+      // ---- [Z | Y] = S_c [K | Q]^T : M=128 (dv), N=2C, K=128 (dk); A = S hi, then S lo
+      if (tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t a0 = tmem + (part ? TM_SLO : TM_SHI);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            const uint32_t acc = (part | kk) ? 1u : 0u;
+            if constexpr (C == 64) {
+              mma_ts(tmem + TM_ZQ, a0 + kk * 8, sdesc_sw128(kq + off, 16, 1024),
+                     idesc_bf16(128, 128, 0, 0, 0), acc);
+            } else {
+              const uint32_t rows = 2048u * s;
+              mma_ts(tmem + TM_ZQ + 16 * s, a0 + kk * 8, sdesc_sw128(kq + off + rows, 16, 1024),
+                     idesc_bf16(128, 16, 0, 0, 0), acc);
+              mma_ts(tmem + TM_ZQ + 64 + 16 * s, a0 + kk * 8,
+                     sdesc_sw128(kq + 8192 + off + rows, 16, 1024), idesc_bf16(128, 16, 0, 0, 0),
+                     acc);
+            }
+          }
+        }
+        mma_commit(bar_mma);
+      }
+      flow.wait_mma();
+
+      // ---- X^T[dv][n] = beta_n V[n][dv] - beta_n Gamma_n Z[dv][n]  (hi/lo -> SMEM)
+      {
+        const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(vtile);
+#pragma unroll
+        for (int q = 0; q < C / 16; ++q) {
+          float Z[16];
+          tmem_ld16(tlane + TM_ZQ + (C == 64 ? 16 * q : 16 * s), Z);
+          float x[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int n = C * s + 16 * q + e;
+            x[e] = s_b[n] * __bfloat162float(V[n * D + dv]) - s_bG[n] * Z[e];
+          }
+          const int ch = (C * s + 16 * q) / 8;
+          store_split8(sb + SM_XH, sb + SM_XL, dv, ch, x);
+          store_split8(sb + SM_XH, sb + SM_XL, dv, ch + 1, x + 8);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+
+      // ---- Dl^T = X^T T^T : M=128 (dv), N=C (i), K=C (n); 3 hi/lo products
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
+        const uint32_t trow = uint32_t(C * s / 8) * 1024u;
+#pragma unroll
+        for (int part = 0; part < 3; ++part) {
+          const uint32_t xa = sb + (part == 2 ? SM_XL : SM_XH);
+          const uint32_t tb = sb + (part == 1 ? SM_TL : SM_TH) + trow;
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks) {
+            const uint32_t kb = uint32_t(C * s + 16 * ks) * 2u;
+            mma_ss(tmem + TM_PD + C * s, sdesc_sw128(xa + kb, 16, 1024),
+                   sdesc_sw128(tb + kb, 16, 1024), id, (part | ks) ? 1u : 0u);
+          }
+        }
+        mma_commit(bar_mma);
+      }
+      flow.wait_mma();
+
+      // ---- residuals: Dl (for the output) and Dl * exp(gamma_last - gamma) (for the state)
+#pragma unroll
+      for (int q = 0; q < C / 16; ++q) {
+        float d[16];
+        tmem_ld16(tlane + TM_PD + C * s + 16 * q, d);
+        float dt[16];
+        const int n0 = C * s + 16 * q;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) dt[e] = d[e] * s_df[n0 + e];
+        store_split8(sb + SM_DH, sb + SM_DL, dv, n0 / 8, d);
+        store_split8(sb + SM_DH, sb + SM_DL, dv, n0 / 8 + 1, d + 8);
+        store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8, dt);
+        store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8 + 1, dt + 8);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+
+      // ---- O_intra = Dl^T Mq^T (N=C) and U = Dl~^T K (N=128, B = K tile MN-major)
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
+        const uint32_t mrow = uint32_t(C * s / 8) * 1024u;
+#pragma unroll
+        for (int part = 0; part < 3; ++part) {
+          const uint32_t da = sb + (part == 2 ? SM_DL : SM_DH);
+          const uint32_t mb = sb + (part == 1 ? SM_MQL : SM_MQH) + mrow;
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks) {
+            const uint32_t kb = uint32_t(C * s + 16 * ks) * 2u;
+            mma_ss(tmem + TM_OI + C * s, sdesc_sw128(da + kb, 16, 1024),
+                   sdesc_sw128(mb + kb, 16, 1024), id, (part | ks) ? 1u : 0u);
+          }
+        }
+        const uint32_t idu = idesc_bf16(128, 128, 0, 1, 0);
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t da = sb + (part ? SM_XL : SM_XH);
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks) {
+            const int tok = C * s + 16 * ks;
+            mma_ss(tmem + TM_U, sdesc_sw128(da + uint32_t(tok) * 2u, 16, 1024),
+                   sdesc_sw128(kq + uint32_t(tok) * 128u, 16384, 1024), idu,
+                   (part | ks) ? 1u : 0u);
+          }
+        }
+        mma_commit(bar_mma);
+      }
+      flow.wait_mma();
+
+      // ---- S <- Gamma_last S + U (fp32 registers); refresh the hi/lo copy in TMEM
+      {
+        const float gc = s_GC[s];
+#pragma unroll
+        for (int q = 0; q < D / 16; ++q) {
+          float u[16];
+          tmem_ld16(tlane + TM_U + 16 * q, u);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) S[16 * q + e] = fmaf(gc, S[16 * q + e], u[e]);
+        }
+        store_state_split(tlane, S);
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (*s_abort) goto teardown;
+    }
+
+    // ---- o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] for the valid tokens of the tile
+    {
+      float* orow = p.o + ((size_t(b) * T + t0) * H + h) * D + dv;
+      const size_t tstride = size_t(H) * D;
+#pragma unroll
+      for (int q = 0; q < NT / 16; ++q) {
+        float y[16], oi[16];
+        tmem_ld16x2(tlane + TM_ZQ + 64 + 16 * q, y, tlane + TM_OI + 16 * q, oi);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int n = 16 * q + e;
+          if (t0 + n < T) orow[size_t(n) * tstride] = fmaf(s_Gam[n], y[e], oi[e]);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  if (!*s_abort) {
+    float4* dst = reinterpret_cast<float4*>(p.S_T + (size_t(chain) * D + dv) * D);
+#pragma unroll
+    for (int q4 = 0; q4 < D / 4; ++q4)
+      dst[q4] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
+  }
+
+teardown:
+  // An aborted CTA may still have a TMA tile in flight: wait for it (bounded)
+  // before the shared memory goes away.
+  if (tid == 0 && *s_abort) {
+    for (int c = tma_done; c < tma_issued; ++c)
+      mbar_wait_bounded(bar_tma0 + 8 * (c & 1), (c >> 1) & 1, WAIT_LIMIT_NS / 4);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// T == 0: S_T = S0 (or zeros); nothing else to do.
+__global__ void copy_state_kernel(const float* __restrict__ S0, float* __restrict__ S_T,
+                                  size_t n4) {
+  const size_t i = size_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (S0) v = reinterpret_cast<const float4*>(S0)[i];
+  reinterpret_cast<float4*>(S_T)[i] = v;
+}
+
+}  // namespace
+
+int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                   const PrefillArgs& a, int chunk, cudaStream_t stream) {
+  const int chains = a.B * a.H;
+  if (chains == 0) return 0;
+  if (a.T == 0) {
+    const size_t n4 = size_t(chains) * D * D / 4;
+    if (a.S0 == a.S_T) return 0;
+    copy_state_kernel<<<unsigned((n4 + 255) / 256), 256, 0, stream>>>(a.S0, a.S_T, n4);
+    return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  }
+  const uint32_t smem = SMEM_USED + 1024;
+  cudaError_t err;
+  if (chunk == 64) {
+    err = cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(smem));
+    if (err != cudaSuccess) return -1;
+    prefill_kernel<64><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, a);
+  } else {
+    err = cudaFuncSetAttribute(prefill_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               int(smem));
+    if (err != cudaSuccess) return -1;
+    prefill_kernel<16><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, a);
+  }
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace gdn

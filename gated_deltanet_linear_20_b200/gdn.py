@@ -1,0 +1,167 @@
+"""ctypes binding of libgdn_b200.so (C ABI in include/gdn.h).
+
+Argument marshalling only: checks dtypes, shapes, devices and contiguity,
+allocates outputs with torch, and passes raw device pointers plus the current
+CUDA stream to the library.  Every step of the computation runs in the
+library's CUDA kernels; there is no fallback.  Importing this module without
+the built library raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libgdn_b200.so")
+
+if not os.path.exists(library_path):
+    raise ImportError(f"{library_path} is missing: build it with "
+                      "`python -m gated_deltanet_linear_20_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(library_path)
+_vp, _ci = ctypes.c_void_p, ctypes.c_int
+_lib.gdn_abi_version.argtypes = []
+_lib.gdn_abi_version.restype = _ci
+_lib.gdn_status_str.argtypes = [_ci]
+_lib.gdn_status_str.restype = ctypes.c_char_p
+_lib.gdn_prefill.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, _vp]
+_lib.gdn_prefill.restype = _ci
+_lib.gdn_decode_step.argtypes = [_vp] * 7 + [_ci] * 4 + [_vp, _vp]
+_lib.gdn_decode_step.restype = _ci
+_lib.gdn_query_status.argtypes = [_vp, _vp]
+_lib.gdn_query_status.restype = _ci
+
+ABI_VERSION = 1
+if _lib.gdn_abi_version() != ABI_VERSION:
+    raise ImportError(f"libgdn_b200.so ABI {_lib.gdn_abi_version()} != binding ABI {ABI_VERSION}")
+
+# status codes (include/gdn.h)
+GDN_OK = 0
+GDN_ERR_NULL = -1
+GDN_ERR_ALIGN = -2
+GDN_ERR_SHAPE = -3
+GDN_ERR_UNSUPPORTED = -4
+GDN_ERR_ALIAS = -5
+GDN_ERR_LAUNCH = -6
+GDN_ERR_DEVICE_TIMEOUT = -7
+
+
+class GDNError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_str(code)} (code {code})")
+
+
+def abi_version() -> int:
+    return int(_lib.gdn_abi_version())
+
+
+def status_str(code: int) -> str:
+    return _lib.gdn_status_str(int(code)).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple, device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+            beta: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64, *,
+            o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
+            status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Chunked prefill: returns (o [B,T,H,Dv] fp32, S_T [B,H,Dv,Dk] fp32).
+
+    q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g, beta [B,T,H] fp32; S0 [B,H,Dv,Dk]
+    fp32 or None (zeros); chunk 16 or 64.  Launches on the current stream.
+    ``o`` / ``S_T`` may be given preallocated (``S_T`` may be ``S0``)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B,T,H,Dk]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn.prefill runs on CUDA tensors only (no CPU path)")
+    _check(q, "q", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(k, "k", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(v, "v", torch.bfloat16, (B, T, H, Dv), dev)
+    _check(g, "g", torch.float32, (B, T, H), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, Dv, Dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
+    if S_T is None:
+        S_T = torch.empty((B, H, Dv, Dk), dtype=torch.float32, device=dev)
+    _check(S_T, "S_T", torch.float32, (B, H, Dv, Dk), dev)
+    if status is not None:
+        _check(status, "status", torch.int32, (1,), dev)
+    rc = _lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                          _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(status),
+                          _stream_handle(dev))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_prefill")
+    return o, S_T
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One decode step; S [B,H,Dv,Dk] fp32 is updated in place.  Returns o [B,H,Dv] fp32.
+
+    q, k [B,H,Dk] bf16; v [B,H,Dv] bf16; g, beta [B,H] fp32."""
+    if q.dim() != 3:
+        raise ValueError("q must be [B,H,Dk]")
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn.decode_step runs on CUDA tensors only (no CPU path)")
+    _check(q, "q", torch.bfloat16, (B, H, Dk), dev)
+    _check(k, "k", torch.bfloat16, (B, H, Dk), dev)
+    _check(v, "v", torch.bfloat16, (B, H, Dv), dev)
+    _check(g, "g", torch.float32, (B, H), dev)
+    _check(beta, "beta", torch.float32, (B, H), dev)
+    _check(S, "S", torch.float32, (B, H, Dv, Dk), dev)
+    if o is None:
+        o = torch.empty((B, H, Dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.float32, (B, H, Dv), dev)
+    rc = _lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                              B, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_decode_step")
+    return o
+
+
+def query_status(status: torch.Tensor) -> int:
+    """Synchronises the current stream and returns the device status word."""
+    return int(_lib.gdn_query_status(_ptr(status), _stream_handle(status.device)))
+
+
+def raw_prefill(*args) -> int:
+    """Direct call of the C entry point with raw integers/pointers (tests use it
+    to exercise argument validation without any tensor)."""
+    return int(_lib.gdn_prefill(*args))
+
+
+def raw_decode_step(*args) -> int:
+    return int(_lib.gdn_decode_step(*args))

@@ -1,0 +1,117 @@
+/*
+ * gdn.h -- C ABI of libgdn_b200.so: the gated delta rule (gated DeltaNet
+ * linear attention) on NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For every sequence b and head h independently, with the
+ * state S in R^{Dv x Dk}:
+ *
+ *     alpha_t = exp(g_t)
+ *     S_t     = alpha_t * S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t     = S_t q_t
+ *
+ * This is the recurrence of the linear-attention layers of the hybrid
+ * Qwen 3.5 models.  The ROCmFPX gated-delta-net prefill note
+ * (bittide.aicompass.dev article d2880479, opening post) describes its prefill
+ * in this setting: a scalar gate per token and head, head dim 128, one
+ * sequence per call, 16-token chunks, and the state held in F32 accumulators.
+ * Its decode step is the per-layer recurrence fused into the Megakernel of the
+ * Lucebox contribution guide (discosf.com/news/5165879, section 4, "CUDA/HIP
+ * kernel optimisation: the Megakernel example").
+ *
+ * Layouts.  Every array is dense and row-major (last index fastest):
+ *     q, k      [B][T][H][Dk]   bf16
+ *     v         [B][T][H][Dv]   bf16
+ *     g, beta   [B][T][H]       fp32   (g is the natural log of alpha)
+ *     S0, S_T   [B][H][Dv][Dk]  fp32   (row i of S is contiguous in Dk)
+ *     o         [B][T][H][Dv]   fp32
+ * The decode step drops the T index.  q and k are used as given: callers
+ * normalise or scale them beforehand if their model does so.
+ *
+ * Ownership and execution.  All pointers are DEVICE pointers owned by the
+ * caller.  The library allocates no device memory, keeps no state between
+ * calls and is safe to call from several host threads.  Work is enqueued on
+ * `stream` (a cudaStream_t; NULL means the legacy default stream) and the call
+ * returns before it completes.  S_T may be the same buffer as S0 (each chain
+ * reads its S0 before writing its S_T); o must not overlap any input.
+ *
+ * Errors.  A negative return value means nothing was launched:
+ *     GDN_ERR_NULL         a required pointer is NULL
+ *     GDN_ERR_ALIGN        q/k/v/o/S pointers must be 16-byte aligned, g/beta 4-byte
+ *     GDN_ERR_SHAPE        a size is negative or the problem exceeds 2^31-1 elements
+ *     GDN_ERR_UNSUPPORTED  Dk != 128, Dv != 128, chunk not in {16, 64}, or the
+ *                          current device is not compute capability 10.0
+ *     GDN_ERR_ALIAS        o overlaps an input or the state
+ *     GDN_ERR_LAUNCH       the CUDA launch (or a CUDA runtime query) failed
+ * Device-side waits are bounded: if one gives up, the kernel writes
+ * GDN_ERR_DEVICE_TIMEOUT to *status (when status is non-NULL), releases its
+ * tensor memory and returns; read it with gdn_query_status.  The kernels never
+ * trap and never print.
+ */
+#ifndef GDN_B200_H_
+#define GDN_B200_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_ABI_VERSION 1
+
+enum gdn_status_code {
+  GDN_OK = 0,
+  GDN_ERR_NULL = -1,
+  GDN_ERR_ALIGN = -2,
+  GDN_ERR_SHAPE = -3,
+  GDN_ERR_UNSUPPORTED = -4,
+  GDN_ERR_ALIAS = -5,
+  GDN_ERR_LAUNCH = -6,
+  GDN_ERR_DEVICE_TIMEOUT = -7
+};
+
+/* Returns GDN_ABI_VERSION of the built library; callers compare it with the
+ * header they compiled against and refuse to proceed on a mismatch. */
+int gdn_abi_version(void);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char* gdn_status_str(int code);
+
+/* Chunked prefill over T tokens (the chunked form of the recurrence above; the
+ * ROCmFPX gated-delta-net prefill note, opening post, motivates chunking).
+ *   q, k, v, g, beta : inputs as laid out above (device)
+ *   S0   : initial state, or NULL for zeros (device)
+ *   o    : output, written for every t < T (device)
+ *   S_T  : final state, written (device; may equal S0)
+ *   B, T, H : batch, tokens per sequence, heads; B*H == 0 or T == 0 are valid
+ *             (T == 0 only writes S_T = S0, or zeros)
+ *   Dk, Dv  : head dims; both must be 128
+ *   chunk   : 16 or 64 -- tokens per chunk of the chunked form; the result is
+ *             the same recurrence either way (up to rounding)
+ *   status  : optional device int; a bounded device wait that gives up stores
+ *             GDN_ERR_DEVICE_TIMEOUT there (it is never cleared by the library)
+ *   stream  : cudaStream_t to launch on
+ * Returns GDN_OK after enqueueing, or a negative gdn_status_code. */
+int gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
+                int chunk, int* status, void* stream);
+
+/* One decode step for B sequences (the recurrence above with T = 1), the state
+ * read and written in place (the Megakernel decode of the Lucebox contribution
+ * guide, section 4, is where this step runs once per layer and token).
+ *   q, k [B][H][Dk] bf16; v [B][H][Dv] bf16; g, beta [B][H] fp32 (device)
+ *   S    [B][H][Dv][Dk] fp32, updated in place (device)
+ *   o    [B][H][Dv] fp32, written (device)
+ *   Dk, Dv must be 128; B*H == 0 is a no-op.
+ * status and stream as for gdn_prefill.  Returns GDN_OK or a negative code. */
+int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, float* S, float* o, int B, int H, int Dk, int Dv,
+                    int* status, void* stream);
+
+/* Synchronises `stream`, then reads the device status word written by the
+ * kernels.  Returns GDN_OK, GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_NULL (status_dev is
+ * NULL) or GDN_ERR_LAUNCH (the synchronisation or copy failed). */
+int gdn_query_status(const int* status_dev, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_B200_H_ */

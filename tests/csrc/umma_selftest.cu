@@ -1,0 +1,131 @@
+// Test-only kernel: runs one tcgen05.mma configuration of the kinds the
+// prefill kernel uses on a single 128x128 tile and writes the fp32 result, so
+// that descriptor encodings, operand majors, A-from-tensor-memory, sub-block
+// offsets and operand negation can each be checked against a host matmul.
+//
+// Modes (A is [128 m][128 k] bf16 row-major; D is [128 m][128 n] fp32):
+//   0: D = A B^T, B [128 n][128 k] K-major (SW128), N = 128
+//   1: D = A B,   B [128 k][128 n] MN-major (SW128, two 64-column blocks), N = 128
+//   2: D = A B^T with A read from tensor memory (bf16 pairs per column), N = 128
+//   3: D[:, 0:16] = A[:, 16:32] B[32:48, 16:32]^T (one K=16 step, N=16, offsets in both)
+//   4: D = 1 - A B^T (D preset to 1 by tcgen05.st, A negated in the instruction)
+//   5: D[:, 0:64] = A B[0:64]^T, N = 64
+#include <cstdint>
+
+#include "sm100.cuh"
+
+using namespace gdn::sm100;
+
+namespace {
+
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+  return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + (((c ^ r) & 7) << 4));
+}
+
+__global__ void __launch_bounds__(128, 1)
+    umma_selftest_kernel(const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ B,
+                         float* __restrict__ Dout, int mode, int* status) {
+  extern __shared__ uint8_t raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  const uint32_t sa = sb, sbB = sb + 32768;  // A: 2 boxes x 16 KB; B: 2 boxes x 16 KB
+  const uint32_t bar = sb + 65536;
+  uint32_t* slot = reinterpret_cast<uint32_t*>(sm + 65536 + 16);
+  const int tid = threadIdx.x, warp = tid >> 5;
+
+  // A row tid -> K-major SW128, two boxes of 64 k
+  for (int c = 0; c < 16; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(A + tid * 128 + c * 8);
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(sa + (c >> 3) * 16384 + sw_off(tid, c & 7)),
+                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+  }
+  // B row tid: K-major ([n][k]) or MN-major ([k][n], rows are k, two 64-n blocks)
+  for (int c = 0; c < 16; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(B + tid * 128 + c * 8);
+    asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(sbB + (c >> 3) * 16384 + sw_off(tid, c & 7)),
+                 "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+  }
+  fence_proxy_async_smem();
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *slot;
+  const uint32_t tlane = tmem + (uint32_t(warp * 32) << 16);
+  const uint32_t TD = 0, TA = 256;
+
+  if (mode == 2) {  // A row tid -> TMEM columns TA.. as bf16 pairs
+    for (int g = 0; g < 4; ++g) {
+      uint32_t u[16];
+      for (int e = 0; e < 16; ++e)
+        u[e] = *reinterpret_cast<const uint32_t*>(A + tid * 128 + 32 * g + 2 * e);
+      tmem_st16(tlane + TA + 16 * g, u);
+    }
+  }
+  if (mode == 4) {
+    uint32_t one[16];
+    for (int e = 0; e < 16; ++e) one[e] = __float_as_uint(1.f);
+    for (int g = 0; g < 8; ++g) tmem_st16(tlane + TD + 16 * g, one);
+  }
+  tc_fence_before();
+  __syncthreads();
+
+  if (tid == 0) {
+    tc_fence_after();
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+      const uint64_t ad = sdesc_sw128(sa + off, 16, 1024);
+      if (mode == 0) {
+        mma_ss(tmem + TD, ad, sdesc_sw128(sbB + off, 16, 1024), idesc_bf16(128, 128, 0, 0, 0), kk > 0);
+      } else if (mode == 1) {
+        // B rows are k: 16 k per step = 2 row groups of 1024 B; k >= 64 lives in rows 64.. of
+        // the same 64-n block (rows 0..127 of each block), blocks 16 KB apart.
+        mma_ss(tmem + TD, ad, sdesc_sw128(sbB + kk * 2048, 16384, 1024), idesc_bf16(128, 128, 0, 1, 0), kk > 0);
+      } else if (mode == 2) {
+        mma_ts(tmem + TD, tmem + TA + kk * 8, sdesc_sw128(sbB + off, 16, 1024), idesc_bf16(128, 128, 0, 0, 0), kk > 0);
+      } else if (mode == 3) {
+        if (kk == 1)
+          mma_ss(tmem + TD, sdesc_sw128(sa + 32, 16, 1024), sdesc_sw128(sbB + 4096 + 32, 16, 1024),
+                 idesc_bf16(128, 16, 0, 0, 0), 0);
+      } else if (mode == 4) {
+        mma_ss(tmem + TD, ad, sdesc_sw128(sbB + off, 16, 1024), idesc_bf16(128, 128, 0, 0, 1), 1);
+      } else if (mode == 5) {
+        mma_ss(tmem + TD, ad, sdesc_sw128(sbB + off, 16, 1024), idesc_bf16(128, 64, 0, 0, 0), kk > 0);
+      }
+    }
+    mma_commit(bar);
+  }
+  if (!mbar_wait_bounded(bar, 0, 1000000000ull)) {
+    if (tid == 0) atomicExch(status, -7);
+  }
+  tc_fence_after();
+  for (int g = 0; g < 8; ++g) {
+    float r[16];
+    tmem_ld16(tlane + TD + 16 * g, r);
+    for (int e = 0; e < 16; ++e) Dout[tid * 128 + 16 * g + e] = r[e];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace
+
+extern "C" int umma_selftest(const void* A, const void* B, float* D, int mode, int* status,
+                             void* stream) {
+  const int smem = 65536 + 1024 + 64;
+  if (cudaFuncSetAttribute(umma_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return -1;
+  umma_selftest_kernel<<<1, 128, smem, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(A), static_cast<const __nv_bfloat16*>(B), D, mode, status);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}

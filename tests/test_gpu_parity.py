@@ -1,0 +1,242 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded inputs.
+
+Tolerance (the contract for fp32-accumulated outputs and final state):
+relative Frobenius error <= 2e-3 and max-abs error <= 1e-2 x RMS(reference),
+applied to o and to S_T.  The kernel feeds every derived operand to the
+tensor core as a bf16 hi/lo pair (about 16 significant bits), so its error is
+expected far below that; DESIGN_REL additionally guards that margin so a lost
+lo term cannot hide behind the contract.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_linear_20_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+REL_FRO = 2e-3
+MAXABS_FRAC = 1e-2
+DESIGN_REL = 1e-4
+
+DEV = "cuda:0"
+
+
+def _gdn():
+    from gated_deltanet_linear_20_b200 import gdn
+    return gdn
+
+
+def errors(got, ref):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    rel = np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300)
+    rms = np.sqrt(np.mean(ref * ref)) if ref.size else 0.0
+    mx = np.abs(got - ref).max() / max(rms, 1e-300) if ref.size else 0.0
+    return float(rel), float(mx)
+
+
+def assert_parity(got, ref, what, design=True):
+    rel, mx = errors(got, ref)
+    assert np.isfinite(got).all(), f"{what}: non-finite values"
+    assert rel <= REL_FRO and mx <= MAXABS_FRAC, f"{what}: rel_fro={rel:.3e} maxabs/rms={mx:.3e}"
+    if design:
+        assert rel <= DESIGN_REL, f"{what}: rel_fro={rel:.3e} above the hi/lo design margin"
+
+
+def to_dev(d):
+    return {k: (v.to(DEV) if v is not None else None) for k, v in d.items()}
+
+
+def gpu_prefill(d, chunk, S0=True):
+    dd = to_dev(d)
+    o, S_T = _gdn().prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
+                            dd["S0"] if S0 else None, chunk=chunk)
+    torch.cuda.synchronize()
+    return o.cpu().numpy(), S_T.cpu().numpy()
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_tiny_b1_h2_t64(chunk):
+    w = inputs.WORKLOADS["tiny_b1_h2_t64"]
+    d = inputs.workload_inputs(w, seed=0)
+    o, S_T = gpu_prefill(d, chunk)
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o, ro, "o")
+    assert_parity(S_T, rS, "S_T")
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+@pytest.mark.parametrize("T", [1, 15, 16, 17, 63, 64, 65, 100, 130, 200])
+def test_ragged_lengths(T, chunk):
+    d = inputs.prefill_inputs(2, T, 3, seed=T, s0_std=0.05)
+    o, S_T = gpu_prefill(d, chunk)
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o, ro, f"o T={T}")
+    assert_parity(S_T, rS, f"S_T T={T}")
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_prefill_b1_h16_t512(chunk):
+    w = inputs.WORKLOADS["prefill_b1_h16_t512"]
+    d = inputs.workload_inputs(w, seed=0)
+    o, S_T = gpu_prefill(d, chunk)
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o, ro, "o")
+    assert_parity(S_T, rS, "S_T")
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_prefill_b1_h16_t4096_carried_state(chunk):
+    w = inputs.WORKLOADS["prefill_b1_h16_t4096_s0"]
+    d = inputs.workload_inputs(w, seed=0)
+    o, S_T = gpu_prefill(d, chunk)
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o, ro, "o")
+    assert_parity(S_T, rS, "S_T")
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_prefill_b4_h32_t32768_sampled_chains(chunk):
+    """Full-size workload in the benchmark's launch configuration; the oracle
+    recomputes a sample of (b, h) chains one by one."""
+    w = inputs.WORKLOADS["prefill_b4_h32_t32768"]
+    d = inputs.workload_inputs(w, seed=0, device=DEV)
+    o, S_T = _gdn().prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
+    torch.cuda.synchronize()
+    for (b, h) in [(0, 0), (1, 17), (3, 31)]:
+        sl = lambda x: x[b:b + 1, :, h:h + 1].cpu()
+        ro, rS = oracle.prefill(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["g"]), sl(d["beta"]), None)
+        assert_parity(o[b, :, h].cpu().numpy(), ro[0, :, 0], f"o chain ({b},{h})")
+        assert_parity(S_T[b, h].cpu().numpy(), rS[0, 0], f"S_T chain ({b},{h})")
+    del d, o, S_T
+    torch.cuda.empty_cache()
+
+
+def test_decode_b64_h16_256_steps_sampled_sequences():
+    """256 in-place decode steps of the full batch on the GPU; sequences 0, 21,
+    42, 63 (all 16 heads) checked against the oracle at every step."""
+    w = inputs.WORKLOADS["decode_b64_h16"]
+    d = inputs.workload_inputs(w, seed=0)
+    dd = to_dev(d)
+    S = dd["S"].clone()
+    bsel = [0, 21, 42, 63]
+    S_ref = d["S"][bsel].double().numpy()
+    gdn = _gdn()
+    worst = 0.0
+    for t in range(w.decode_steps):
+        o = gdn.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["g"][t], dd["beta"][t], S)
+        ro, S_ref = oracle.decode_step(d["q"][t][bsel], d["k"][t][bsel], d["v"][t][bsel],
+                                       d["g"][t][bsel], d["beta"][t][bsel], S_ref)
+        got = o[bsel].cpu().numpy()
+        assert_parity(got, ro, f"o step {t}")
+        worst = max(worst, errors(got, ro)[0])
+    assert_parity(S[bsel].cpu().numpy(), S_ref, "S after 256 steps")
+
+
+def test_decode_equals_prefill_t1():
+    d = inputs.prefill_inputs(3, 1, 5, seed=7, s0_std=0.1)
+    dd = to_dev(d)
+    gdn = _gdn()
+    o_p, S_p = gdn.prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"], chunk=64)
+    S = dd["S0"].clone()
+    o_d = gdn.decode_step(dd["q"][:, 0], dd["k"][:, 0], dd["v"][:, 0], dd["g"][:, 0], dd["beta"][:, 0], S)
+    torch.cuda.synchronize()
+    assert_parity(o_d.cpu().numpy(), o_p[:, 0].cpu().numpy(), "decode vs prefill o")
+    assert_parity(S.cpu().numpy(), S_p.cpu().numpy(), "decode vs prefill S")
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_split_carry(chunk):
+    d = to_dev(inputs.prefill_inputs(1, 300, 4, seed=11, s0_std=0.05))
+    gdn = _gdn()
+    o, S_T = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
+    t1 = 130
+    cut = lambda x, a, b: x[:, a:b].contiguous()
+    o1, S1 = gdn.prefill(cut(d["q"], 0, t1), cut(d["k"], 0, t1), cut(d["v"], 0, t1),
+                         cut(d["g"], 0, t1), cut(d["beta"], 0, t1), d["S0"], chunk=chunk)
+    o2, S2 = gdn.prefill(cut(d["q"], t1, 300), cut(d["k"], t1, 300), cut(d["v"], t1, 300),
+                         cut(d["g"], t1, 300), cut(d["beta"], t1, 300), S1, chunk=chunk)
+    torch.cuda.synchronize()
+    assert_parity(torch.cat([o1, o2], 1).cpu().numpy(), o.cpu().numpy(), "split o")
+    assert_parity(S2.cpu().numpy(), S_T.cpu().numpy(), "split S_T")
+
+
+def test_chunk16_agrees_with_chunk64():
+    d = inputs.prefill_inputs(2, 257, 3, seed=5, s0_std=0.05)
+    o64, S64 = gpu_prefill(d, 64)
+    o16, S16 = gpu_prefill(d, 16)
+    assert_parity(o16, o64, "o chunk16 vs 64")
+    assert_parity(S16, S64, "S chunk16 vs 64")
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_bitwise_deterministic(chunk):
+    d = to_dev(inputs.prefill_inputs(2, 333, 4, seed=3, s0_std=0.02))
+    gdn = _gdn()
+    a = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
+    b = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_zero_length_and_empty_batch():
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(2, 0, 3, seed=1, s0_std=0.1))
+    o, S_T = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=64)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and torch.equal(S_T, d["S0"])
+    o, S_T = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None, chunk=16)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(S_T) == 0
+    e = to_dev(inputs.prefill_inputs(0, 10, 3, seed=1))
+    o, S_T = gdn.prefill(e["q"], e["k"], e["v"], e["g"], e["beta"], None, chunk=64)
+    assert o.numel() == 0 and S_T.numel() == 0
+
+
+def test_in_place_state_and_status_word():
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(1, 150, 2, seed=2, s0_std=0.1))
+    o_ref, S_ref = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=64)
+    S = d["S0"].clone()
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_out = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], S, chunk=64, S_T=S, status=status)
+    assert gdn.query_status(status) == 0
+    assert S_out.data_ptr() == S.data_ptr()
+    assert torch.equal(S, S_ref) and torch.equal(o, o_ref)
+
+
+def test_invariants_on_gpu():
+    """beta = 0, g = 0 keeps S0; beta = 1 with exactly unit keys writes v (q = k)."""
+    gdn = _gdn()
+    d = inputs.prefill_inputs(1, 96, 2, seed=4, s0_std=0.1)
+    d["beta"].zero_()
+    d["g"].zero_()
+    o, S_T = gpu_prefill(d, 64)
+    assert_parity(S_T, d["S0"].double().numpy(), "S unchanged", design=False)
+    ro = np.einsum("bhij,bthj->bthi", d["S0"].double().numpy(), d["q"].double().numpy())
+    assert_parity(o, ro, "o = S0 q")
+    rng = np.random.default_rng(4)
+    k = np.zeros((1, 96, 2, 128), np.float32)
+    for idx in np.ndindex(1, 96, 2):
+        pos = rng.choice(128, 4, replace=False)
+        k[idx][pos] = rng.choice([-0.5, 0.5], 4)
+    e = inputs.prefill_inputs(1, 96, 2, seed=5)
+    e["k"] = torch.from_numpy(k).to(torch.bfloat16)
+    e["q"] = e["k"].clone()
+    e["beta"].fill_(1.0)
+    o, _ = gpu_prefill(e, 64, S0=False)
+    assert_parity(o, e["v"].double().numpy(), "beta=1 writes v", design=False)
+
+
+def test_rejects_unsupported_head_dim_on_gpu():
+    gdn = _gdn()
+    q = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16, device=DEV)
+    g = torch.zeros(1, 8, 1, device=DEV)
+    with pytest.raises(gdn.GDNError) as e:
+        gdn.prefill(q, q, q, g, g)
+    assert e.value.code == gdn.GDN_ERR_UNSUPPORTED
