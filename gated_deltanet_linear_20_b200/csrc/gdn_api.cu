@@ -48,19 +48,20 @@ int check_device() {
   return GDN_OK;
 }
 
-// 4-D view [B][T][H][128] of a bf16 activation; box = `box_inner` features x
-// 64 tokens of one head.  Tokens past T read as zeros.
+// 4-D view [B][T][H][128] of an activation (bf16 input or fp32 output); box =
+// `box_inner` features x 64 tokens of one head.  Loads of tokens past T read
+// zeros; stores past T are dropped.
 bool encode_act(CUtensorMap* map, const void* base, int B, int T, int H, int box_inner,
-                CUtensorMapSwizzle swz) {
+                CUtensorMapSwizzle swz, CUtensorMapDataType dtype, int esize) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[4] = {cuuint64_t(kHeadDim), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
-  const cuuint64_t strides[3] = {cuuint64_t(kHeadDim) * 2, cuuint64_t(H) * kHeadDim * 2,
-                                 cuuint64_t(T) * H * kHeadDim * 2};
+  const cuuint64_t strides[3] = {cuuint64_t(kHeadDim) * esize, cuuint64_t(H) * kHeadDim * esize,
+                                 cuuint64_t(T) * H * kHeadDim * esize};
   const cuuint32_t box[4] = {cuuint32_t(box_inner), 1, 64, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -111,14 +112,17 @@ int gdn_prefill(const void* q, const void* k, const void* v, const float* g, con
   if (dev_ok != GDN_OK) return dev_ok;
 
   gdn::PrefillArgs a{g, beta, S0, o, S_T, B, T, H, status};
-  CUtensorMap tq{}, tk{}, tv{};
+  CUtensorMap tq{}, tk{}, tv{}, to{};
   if (T > 0) {
-    if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
+        !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
+        !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2) ||
+        !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4))
       return GDN_ERR_LAUNCH;
   }
-  return gdn::launch_prefill(tq, tk, tv, a, chunk, static_cast<cudaStream_t>(stream)) == 0
+  return gdn::launch_prefill(tq, tk, tv, to, a, chunk, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK
              : GDN_ERR_LAUNCH;
 }
