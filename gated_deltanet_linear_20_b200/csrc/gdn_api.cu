@@ -112,17 +112,15 @@ int gdn_prefill(const void* q, const void* k, const void* v, const float* g, con
   if (dev_ok != GDN_OK) return dev_ok;
 
   gdn::PrefillArgs a{g, beta, S0, o, S_T, B, T, H, status};
-  CUtensorMap tq{}, tk{}, tv{}, to{};
+  CUtensorMap tq{}, tk{}, tv{};
   if (T > 0) {
     const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
         !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
-        !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2) ||
-        !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4))
+        !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2))
       return GDN_ERR_LAUNCH;
   }
-  return gdn::launch_prefill(tq, tk, tv, to, a, chunk, static_cast<cudaStream_t>(stream)) == 0
+  return gdn::launch_prefill(tq, tk, tv, a, chunk, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK
              : GDN_ERR_LAUNCH;
 }

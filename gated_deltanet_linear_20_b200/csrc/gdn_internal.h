@@ -32,7 +32,7 @@ struct DecodeArgs {
 
 // Both return 0 on success, -1 when the launch failed.
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const CUtensorMap& to, const PrefillArgs& a, int chunk, cudaStream_t stream);
+                   const PrefillArgs& a, int chunk, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
 }  // namespace gdn

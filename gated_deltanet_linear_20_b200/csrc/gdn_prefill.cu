@@ -1,6 +1,7 @@
 // Chunked gated-delta-rule prefill for sm_100a: TMA-staged bf16 tiles,
 // tcgen05 MMAs accumulating in tensor memory, fp32 state carried across
-// chunks in tensor memory.
+// chunks in tensor memory, warp-specialised so that the work of consecutive
+// tiles overlaps.
 //
 // Recurrence (per sequence b, head h; S in R^{Dv x Dk}):
 //   S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t.
@@ -20,11 +21,20 @@
 //   S_out = Gamma_last S_c + Dl^T diag(exp(gamma_last - gamma)) K
 //
 // One CTA of 512 threads owns one (b, h) chain and walks its tokens in tiles
-// of 64 (one TMA tile); with chunk = 16 each tile holds four chunks, processed
-// in order.  Warp w reads TMEM lane quarter (w % 4) -- state rows, i.e. the Dv
-// index, 32 (w % 4) .. +31 -- and column quarter (w / 4) of every tile it
-// touches, so each epilogue is spread over 16 warps.  The fp32 state lives in tensor
-// memory, pre-multiplied by the decay of the chunk about to update it, so the
+// of 64 (one TMA tile); with chunk = 16 each tile holds four chunks.  The
+// warps split into three roles that run concurrently and hand off through
+// mbarriers:
+//   * chain  (warps 0-3 and 12-15, 256 threads): everything that depends on
+//     the state -- S_c [K;Q]^T, X, Dl = X T^T, the output and state-update
+//     products and their epilogues -- for tile c;
+//   * K side (warps 4-7): the state-independent work of tile c+1 -- gates,
+//     [K;Q] K^T, the masks and decays, the triangular solve -- handing T and
+//     Mq to the chain once the chain has finished with tile c's;
+//   * output (warps 8-11): o of tile c from tensor memory to HBM while the
+//     chain starts tile c+1.
+// Warp w reads TMEM lane quarter (w % 4); the two chain warpgroups split the
+// columns of each tile in halves.  The fp32 state lives in tensor memory,
+// pre-multiplied by the decay of the chunk about to update it, so the
 // state-update MMA accumulates straight into it; the tensor core reads the
 // state as a bf16 hi/lo pair, also in tensor memory.  Every operand derived
 // inside the kernel (S, X, T, the residuals, Mq) is fed to the MMA as hi + lo
@@ -35,8 +45,9 @@
 //   [  0,128) S   : state, scaled by the next chunk's total decay  (lane dv, col dk)
 //   [128,192) SHI : S hi as bf16 pairs (A operand)                 (lane dv, col dk/2)
 //   [192,256) SLO : S lo
-//   [256,384) ZQ  : [S K^T | S Q^T]                                (lane dv, col token)
-//   [384,448) PD  : [K;Q] K^T (lanes 0..127 = rows of [K;Q]), later Dl^T
+//   [256,320) Z   : S K^T, then Dl^T                               (lane dv, col token)
+//   [320,384) Y   : S Q^T                                          (lane dv, col token)
+//   [384,448) P   : [K;Q] K^T (lanes = rows of [K;Q]; K side only)
 //   [448,512) OI  : Dl^T Mq^T                                      (lane dv, col token)
 #include "gdn_internal.h"
 #include "sm100.cuh"
@@ -49,40 +60,52 @@ using namespace sm100;
 constexpr int D = 128;
 constexpr int NT = 64;  // tokens per TMA tile
 constexpr int NTHREADS = 512;
+constexpr int CHAIN_THREADS = 256, SIDE_THREADS = 128, OUT_THREADS = 128;
+constexpr int BAR_CHAIN = 1, BAR_SIDE = 2, BAR_OUT = 3, BAR_SCAN = 4;  // named barriers
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TM_S = 0, TM_SHI = 128, TM_SLO = 192, TM_ZQ = 256, TM_PD = 384, TM_OI = 448;
+constexpr uint32_t TM_S = 0, TM_SHI = 128, TM_SLO = 192, TM_Z = 256, TM_Y = 320, TM_P = 384,
+                   TM_OI = 448;
 
 // Shared memory map (offsets from a 1024-byte aligned base).
 constexpr uint32_t SM_KQ0 = 0;        // 32 KB: [K dk0-63 | Q dk0-63 | K dk64-127 | Q dk64-127]
 constexpr uint32_t SM_KQ1 = 32768;    //        each a 64-row x 128-byte SW128 box
-constexpr uint32_t SM_V0 = 65536;     // 16 KB: V tile [64 tokens][128] bf16, unswizzled
-constexpr uint32_t SM_V1 = 81920;
-constexpr uint32_t SM_MQH = 98304;    // 8 KB: Mq rows i, K-major SW128 (64 x 64 bf16)
-constexpr uint32_t SM_MQL = 106496;
-constexpr uint32_t SM_TH = 114688;    // 8 KB: T rows i (64 x 64)
-constexpr uint32_t SM_TL = 122880;
-constexpr uint32_t SM_XH = 131072;    // 16 KB: X^T rows dv (128 x 64); then the decay-scaled
-constexpr uint32_t SM_XL = 147456;    //        residuals; at the end of a tile, the o tile
-constexpr uint32_t SM_DH = 163840;    // 16 KB: Dl^T rows dv (128 x 64)
-constexpr uint32_t SM_DL = 180224;
-// The triangular solve runs while the X / Dl regions are idle and borrows them:
+constexpr uint32_t SM_V = 65536;      // 16 KB: V tile [64 tokens][128] bf16, unswizzled
+constexpr uint32_t SM_MQH = 81920;    // 8 KB: Mq rows i, K-major SW128 (64 x 64 bf16)
+constexpr uint32_t SM_MQL = 90112;
+constexpr uint32_t SM_TH = 98304;     // 8 KB: T rows i (64 x 64)
+constexpr uint32_t SM_TL = 106496;
+constexpr uint32_t SM_XH = 114688;    // 16 KB: X^T rows dv (128 x 64), then the
+constexpr uint32_t SM_XL = 131072;    //        decay-scaled residuals
+constexpr uint32_t SM_DH = 147456;    // 16 KB: Dl^T rows dv (128 x 64)
+constexpr uint32_t SM_DL = 163840;
 constexpr int APAD = 68;                      // row pitch (floats): conflict-free float4 rows
 constexpr uint32_t SOLVE_MAT = 64 * APAD * 4; // 17408 B
-constexpr uint32_t SM_A = SM_XH;              // A   fp32 [64][APAD]
-constexpr uint32_t SM_TF = SM_A + SOLVE_MAT;  // T   fp32 [64][APAD]
+constexpr uint32_t SM_A = 180224;             // A  fp32 [64][APAD] (K side)
+constexpr uint32_t SM_TF = SM_A + SOLVE_MAT;  // T  fp32 [64][APAD] (K side)
 constexpr uint32_t SM_E = SM_TF + SOLVE_MAT;  // block products fp32 [3][16][16]
-constexpr uint32_t SM_O = SM_XH;              // o tile fp32 [64 tokens][128] (32 KB)
-constexpr uint32_t SM_MISC = 196608;  // gates, barriers, TMEM slot
-constexpr uint32_t MISC_G = 0, MISC_B = 256, MISC_GAM2 = 512, MISC_GAM = 768, MISC_BG = 1024,
-                   MISC_DF = 1280, MISC_GC = 1536, MISC_GCN = 1552, MISC_PART = 1560,
-                   MISC_BAR = 1600, MISC_TMEM = 1632, MISC_ABORT = 1636;
-constexpr uint32_t SMEM_USED = SM_MISC + 2048;
-static_assert(SM_E + 3 * 256 * 4 <= SM_DL + 16384, "solve scratch must stay inside the X/Dl regions");
-static_assert(SM_O + 64 * 128 * 4 <= SM_DH, "o tile must stay inside the X region");
-static_assert(SM_DL + 16384 <= SM_MISC, "tiles overlap the misc area");
-constexpr uint32_t TILE_TX_BYTES = 4 * 8192 + 16384;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
+constexpr uint32_t SM_GATES = SM_E + 3072;    // 3 gate buffers (tile c uses c % 3)
+constexpr uint32_t GATE_BYTES = 1536;
+constexpr uint32_t G_GAM2 = 0, G_B = 256, G_BG = 512, G_DF = 768, G_GAM = 1024, G_GC = 1280;
+constexpr uint32_t SM_BAR = SM_GATES + 3 * GATE_BYTES;
+constexpr uint32_t SM_MISC = SM_BAR + 256;    // TMEM slot, abort flags, scan scratch, counters
+constexpr uint32_t SMEM_USED = SM_MISC + 256;
+static_assert(SM_A >= SM_DL + 16384, "K-side scratch overlaps the residual tiles");
+static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 
+// mbarriers (8 bytes each, offsets inside SM_BAR)
+constexpr uint32_t B_FULL0 = 0, B_FULL1 = 8, B_VFULL = 16, B_PFULL = 24, B_GFULL0 = 32,
+                   B_GFULL1 = 40, B_TMFULL = 48, B_TMFREE = 56, B_ZQ = 64, B_DL = 72, B_OU = 80,
+                   B_OUTFULL = 88, B_OUTFREE = 96;
+constexpr int NUM_BARS = 13;
+// misc slots (offsets inside SM_MISC)
+constexpr uint32_t M_TMEM = 0, M_ABORT = 4, M_PART = 8, M_KQ_ISSUED = 12, M_KQ_SEEN = 16,
+                   M_V_ISSUED = 20, M_V_SEEN = 24, M_FLAG_CHAIN = 32, M_FLAG_SIDE = 40,
+                   M_FLAG_OUT = 48;  // two verdict slots per role
+static_assert(M_FLAG_OUT + 8 <= 256, "misc slots");
+
+constexpr uint32_t KQ_TX_BYTES = 4 * 8192;
+constexpr uint32_t V_TX_BYTES = 16384;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr float LOG2E = 1.4426950408889634f;
 
 // Byte offset of 16-byte chunk `c` (8 bf16 along K) of row `r` in a K-major
@@ -101,104 +124,111 @@ __device__ __forceinline__ void store_split8(uint32_t hi_tile, uint32_t lo_tile,
                                              const float* x) {
   uint32_t h[4], l[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    __nv_bfloat16 h0, l0, h1, l1;
-    split_bf16(x[2 * e], h0, l0);
-    split_bf16(x[2 * e + 1], h1, l1);
-    h[e] = pack_bf16x2(h0, h1);
-    l[e] = pack_bf16x2(l0, l1);
-  }
+  for (int e = 0; e < 4; ++e) split2_bf16(x[2 * e], x[2 * e + 1], h[e], l[e]);
   const uint32_t off = sw128_off(r, c);
   st_shared_v4(hi_tile + off, h[0], h[1], h[2], h[3]);
   st_shared_v4(lo_tile + off, l[0], l[1], l[2], l[3]);
 }
-
-// Splits 4 floats into hi/lo bf16 and stores them as the 8-byte half `hf` of
-// chunk `c` of row `r` in two tiles.
-__device__ __forceinline__ void store_split4(uint32_t hi_tile, uint32_t lo_tile, int r, int c,
-                                             int hf, const float* x) {
-  __nv_bfloat16 h0, l0, h1, l1, h2, l2, h3, l3;
-  split_bf16(x[0], h0, l0);
-  split_bf16(x[1], h1, l1);
-  split_bf16(x[2], h2, l2);
-  split_bf16(x[3], h3, l3);
-  const uint32_t off = sw128_off(r, c) + 8u * hf;
-  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(hi_tile + off), "r"(pack_bf16x2(h0, h1)),
-               "r"(pack_bf16x2(h2, h3))
-               : "memory");
-  asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(lo_tile + off), "r"(pack_bf16x2(l0, l1)),
-               "r"(pack_bf16x2(l2, l3))
-               : "memory");
-}
-
 // Splits 32 consecutive state values (columns 32q..32q+31 of this lane's row)
 // into bf16 hi/lo pairs and stores them to SHI / SLO.
 __device__ __forceinline__ void store_state_split32(uint32_t tlane, int q, const float (&v)[32]) {
   uint32_t hi[16], lo[16];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) {
-    __nv_bfloat16 h0, l0, h1, l1;
-    split_bf16(v[2 * e], h0, l0);
-    split_bf16(v[2 * e + 1], h1, l1);
-    hi[e] = pack_bf16x2(h0, h1);
-    lo[e] = pack_bf16x2(l0, l1);
-  }
+  for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
   tmem_st16x2(tlane + TM_SHI + 16 * q, hi, tlane + TM_SLO + 16 * q, lo);
 }
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
 
-struct Flow {
-  uint32_t mma_bar;
-  uint32_t mma_phase;
-  volatile int* abort_flag;
+// Shared state of one CTA.
+struct Ctx {
+  uint8_t* sm;
+  uint32_t sb;        // shared-window address of sm
+  uint32_t tmem;      // TMEM base (lane 0, column 0)
   int* status;
-  // All threads wait for the last commit; a wait that gives up flags the CTA.
-  __device__ __forceinline__ void wait_mma() {
-    if (!mbar_wait_bounded(mma_bar, mma_phase, WAIT_LIMIT_NS)) fail();
-    mma_phase ^= 1u;
-    tc_fence_after();
+  volatile int* abort_flag;
+  __device__ __forceinline__ uint32_t bar(uint32_t off) const { return sb + SM_BAR + off; }
+  __device__ __forceinline__ float* gates(int c) const {
+    return reinterpret_cast<float*>(sm + SM_GATES + (c % 3) * GATE_BYTES);
   }
-  __device__ __forceinline__ void fail() {
+  __device__ __forceinline__ volatile int* misc(uint32_t off) const {
+    return reinterpret_cast<volatile int*>(sm + SM_MISC + off);
+  }
+  __device__ __forceinline__ void fail() const {
     *abort_flag = 1;
     if (status) atomicExch(status, GDN_ERR_DEVICE_TIMEOUT);
   }
 };
 
-// Sum of g over the first chunk of a tile held by threads 0..63 (one value
-// each, zero past T), i.e. the log-decay of that chunk.  Threads 0..63 call it;
-// the result lands in *out.  C == 64 uses `part` as a two-warp scratch slot.
-template <int C>
-__device__ __forceinline__ void first_chunk_logdecay(int tid, float g, float* part, float* out) {
-  float x = (tid < C) ? g : 0.f;
-  constexpr int W = C < 32 ? C : 32;
-#pragma unroll
-  for (int off = W / 2; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off, W);
-  if constexpr (C == 64) {
-    if (tid == 32) *part = x;
-    asm volatile("bar.sync 1, 64;" ::: "memory");  // warps 0 and 1 only
-    if (tid == 0) *out = x + *part;
-  } else {
-    if (tid == 0) *out = x;
+// Role-wide agreement on whether to go on.  The role leader decides (after a
+// bounded wait on an mbarrier phase, in wait()), writes the verdict to one of
+// two slots, and the role meets at its named barrier; every thread then reads
+// the same verdict, so the whole role takes the same path.  The slots
+// alternate: a slot is rewritten only two agreements later, after every
+// thread has passed the barrier of the agreement in between.
+struct RoleSync {
+  int bar_id, nthreads;
+  uint32_t flag_off;
+  bool leader;
+  int n;  // agreements so far (identical in every thread of the role)
+  __device__ __forceinline__ bool agree(const Ctx& x, bool leader_ok) {
+    volatile int* slot = x.misc(flag_off + 4u * (n & 1));
+    ++n;
+    if (leader) *slot = leader_ok ? 0 : 1;
+    named_bar(bar_id, nthreads);
+    const bool ok = (*slot == 0);
+    tc_fence_after();
+    return ok;
   }
+  // Leader waits (bounded) for the given phase parity of `bar`.
+  __device__ __forceinline__ bool wait(const Ctx& x, uint32_t bar, uint32_t parity) {
+    bool ok = true;
+    if (leader) {
+      ok = (*x.abort_flag == 0) && mbar_wait_bounded(bar, parity, WAIT_LIMIT_NS);
+      if (!ok) x.fail();
+    }
+    return agree(x, ok);
+  }
+  __device__ __forceinline__ bool check(const Ctx& x) {
+    return agree(x, !leader || *x.abort_flag == 0);
+  }
+};
+
+__device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
+                                         int c, int h, int b) {
+  const uint32_t kq = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
+  const uint32_t bar = x.bar((c & 1) ? B_FULL1 : B_FULL0);
+  mbar_arrive_expect_tx(bar, KQ_TX_BYTES);
+  tma_load_4d(kq + 0, tk, bar, 0, h, c * NT, b);
+  tma_load_4d(kq + 8192, tq, bar, 0, h, c * NT, b);
+  tma_load_4d(kq + 16384, tk, bar, 64, h, c * NT, b);
+  tma_load_4d(kq + 24576, tq, bar, 64, h, c * NT, b);
+  *x.misc(M_KQ_ISSUED) = c + 1;
+}
+__device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b) {
+  const uint32_t bar = x.bar(B_VFULL);
+  mbar_arrive_expect_tx(bar, V_TX_BYTES);
+  tma_load_4d(x.sb + SM_V, tv, bar, 0, h, c * NT, b);
+  *x.misc(M_V_ISSUED) = c + 1;
 }
 
 // One distance-d sweep of the blocked inverse of (I + A), 64 x 64 in 16 x 16
 // blocks (diagonal blocks already inverted in Tf):
 //   E_p     = sum_{K=J}^{I-1} A_{I,K} T_{K,J}        (I = J + d, p = J)
 //   T_{I,J} = -T_{I,I} E_p
-// Each thread owns a 1 x 4 strip of outputs so one A load and one float4 T
-// load feed four FMAs; all loop bounds are compile-time.
+// A thread owns 1 x 4 strips of outputs; all loop bounds are compile-time.
 template <int d>
-__device__ __forceinline__ void solve_offdiag(int tid, const float* sA, float* sTf, float* sE) {
+__device__ __forceinline__ void solve_offdiag(int kt, const float* sA, float* sTf, float* sE) {
   constexpr int NSTRIP = (4 - d) * 64;  // (4-d) block pairs x 16 rows x 4 strips
-  if (tid < NSTRIP) {
-    const int pp = tid >> 6, r = (tid >> 2) & 15, c4 = tid & 3;
+#pragma unroll
+  for (int st = kt; st < NSTRIP; st += SIDE_THREADS) {
+    const int pp = st >> 6, r = (st >> 2) & 15, c4 = st & 3;
     const float* arow = sA + ((pp + d) * 16 + r) * APAD + pp * 16;
     const float* tcol = sTf + (pp * 16) * APAD + pp * 16 + 4 * c4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < 16 * d; ++k) {
       const float a = arow[k];
-      const float4 t = *reinterpret_cast<const float4*>(tcol + k * APAD);
+      const float4 t = ld4(tcol + k * APAD);
       acc.x = fmaf(a, t.x, acc.x);
       acc.y = fmaf(a, t.y, acc.y);
       acc.z = fmaf(a, t.z, acc.z);
@@ -206,9 +236,10 @@ __device__ __forceinline__ void solve_offdiag(int tid, const float* sA, float* s
     }
     *reinterpret_cast<float4*>(sE + pp * 256 + r * 16 + 4 * c4) = acc;
   }
-  __syncthreads();
-  if (tid < NSTRIP) {
-    const int pp = tid >> 6, r = (tid >> 2) & 15, c4 = tid & 3;
+  named_bar(BAR_SIDE, SIDE_THREADS);
+#pragma unroll
+  for (int st = kt; st < NSTRIP; st += SIDE_THREADS) {
+    const int pp = st >> 6, r = (st >> 2) & 15, c4 = st & 3;
     const int I = pp + d;
     const float* trow = sTf + (I * 16 + r) * APAD + I * 16;
     const float* e = sE + pp * 256 + 4 * c4;
@@ -216,7 +247,7 @@ __device__ __forceinline__ void solve_offdiag(int tid, const float* sA, float* s
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       const float a = trow[k];
-      const float4 t = *reinterpret_cast<const float4*>(e + k * 16);
+      const float4 t = ld4(e + k * 16);
       acc.x = fmaf(a, t.x, acc.x);
       acc.y = fmaf(a, t.y, acc.y);
       acc.z = fmaf(a, t.z, acc.z);
@@ -225,247 +256,145 @@ __device__ __forceinline__ void solve_offdiag(int tid, const float* sA, float* s
     *reinterpret_cast<float4*>(sTf + (I * 16 + r) * APAD + pp * 16 + 4 * c4) =
         make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
   }
-  __syncthreads();
+  named_bar(BAR_SIDE, SIDE_THREADS);
 }
 
+// ============================================================== K side
+// Per tile c: gates(c) -> [K;Q] K^T -> masks / decays -> T = (I + A)^{-1};
+// then, once the chain has released tile c-1's T and Mq, writes T(c), Mq(c).
 template <int C>
-__global__ void __launch_bounds__(NTHREADS, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                   const PrefillArgs p) {
-  static_assert(C == 16 || C == 64, "chunk must be 16 or 64");
-  constexpr int NSUB = NT / C;  // chunks per TMA tile
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(sm);
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lq = warp & 3;                  // TMEM lane quarter
-  const int cg = warp >> 2;                 // column quarter
-  const int row = lq * 32 + (tid & 31);     // TMEM lane: Dv row, or row of [K;Q]
-  const int chain = blockIdx.x;
-  const int b = chain / p.H;
-  const int h = chain - b * p.H;
+__device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
+                           const CUtensorMap* tv, const PrefillArgs& p, int b, int h, int ntiles) {
+  const int kt = threadIdx.x - 128;        // 0..127
+  const int lq = (threadIdx.x >> 5) & 3;
+  const int row = kt;                      // TMEM lane == row of [K;Q]
+  const bool leader = (kt == 0);
+  const uint32_t tlane = x.tmem + (uint32_t(lq * 32) << 16);
   const int T = p.T, H = p.H;
+  float* sA = reinterpret_cast<float*>(x.sm + SM_A);
+  float* sTf = reinterpret_cast<float*>(x.sm + SM_TF);
+  float* sE = reinterpret_cast<float*>(x.sm + SM_E);
+  volatile float* s_part = reinterpret_cast<volatile float*>(x.misc(M_PART));
+  RoleSync rs{BAR_SIDE, SIDE_THREADS, M_FLAG_SIDE, leader, 0};
 
-  float* s_g = reinterpret_cast<float*>(sm + SM_MISC + MISC_G);
-  float* s_b = reinterpret_cast<float*>(sm + SM_MISC + MISC_B);
-  float* s_gam2 = reinterpret_cast<float*>(sm + SM_MISC + MISC_GAM2);
-  float* s_Gam = reinterpret_cast<float*>(sm + SM_MISC + MISC_GAM);
-  float* s_bG = reinterpret_cast<float*>(sm + SM_MISC + MISC_BG);
-  float* s_df = reinterpret_cast<float*>(sm + SM_MISC + MISC_DF);
-  float* s_GC = reinterpret_cast<float*>(sm + SM_MISC + MISC_GC);    // per chunk of this tile
-  float* s_GCn = reinterpret_cast<float*>(sm + SM_MISC + MISC_GCN);  // first chunk, next tile
-  float* s_part = reinterpret_cast<float*>(sm + SM_MISC + MISC_PART);
-  const uint32_t bar_tma0 = sb + SM_MISC + MISC_BAR;
-  const uint32_t bar_mma = bar_tma0 + 16;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + SM_MISC + MISC_TMEM);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(sm + SM_MISC + MISC_ABORT);
-  float* sA = reinterpret_cast<float*>(sm + SM_A);
-  float* sTf = reinterpret_cast<float*>(sm + SM_TF);
-  float* sE = reinterpret_cast<float*>(sm + SM_E);
-  float* sO = reinterpret_cast<float*>(sm + SM_O);
-
-  if (tid == 0) {
-    prefetch_tmap(&tm_q);
-    prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
-    prefetch_tmap(&tm_o);
-    mbar_init(bar_tma0, 1);
-    mbar_init(bar_tma0 + 8, 1);
-    mbar_init(bar_mma, 1);
-    fence_mbar_init();
-    *s_abort = 0;
+  if (leader) {
+    issue_kq(x, tq, tk, 0, h, b);
+    if (ntiles > 1) issue_kq(x, tq, tk, 1, h, b);
+    issue_v(x, tv, 0, h, b);
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(s_tmem), TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *s_tmem;
-  const uint32_t tlane = tmem + (uint32_t(lq * 32) << 16);  // this warp's lane quarter
-
-  Flow flow{bar_mma, 0u, s_abort, p.status};
-  const int ntiles = (T + NT - 1) / NT;
-  int tma_issued = 0;  // tiles whose TMA was issued (thread 0's view)
-  int tma_done = 0;    // tiles whose TMA completion was observed
-  const int dv = row;
-
-  auto issue_tile = [&](int c) {
-    const int st = c & 1;
-    const uint32_t kq = sb + (st ? SM_KQ1 : SM_KQ0);
-    const uint32_t vt = sb + (st ? SM_V1 : SM_V0);
-    const uint32_t bar = bar_tma0 + 8 * st;
-    mbar_arrive_expect_tx(bar, TILE_TX_BYTES);
-    tma_load_4d(kq + 0, &tm_k, bar, 0, h, c * NT, b);
-    tma_load_4d(kq + 8192, &tm_q, bar, 0, h, c * NT, b);
-    tma_load_4d(kq + 16384, &tm_k, bar, 64, h, c * NT, b);
-    tma_load_4d(kq + 24576, &tm_q, bar, 64, h, c * NT, b);
-    tma_load_4d(vt, &tm_v, bar, 0, h, c * NT, b);
-  };
-
-  // ---- gates of tile 0; the first TMA tile
   float g_next = 0.f, b_next = 0.f;
-  if (tid < NT && tid < T) {
-    const size_t gi = (size_t(b) * T + tid) * H + h;
+  if (kt < NT && kt < T) {
+    const size_t gi = (size_t(b) * T + kt) * H + h;
     g_next = __ldg(p.g + gi);
     b_next = __ldg(p.beta + gi);
   }
-  if (tid == 0) {
-    issue_tile(0);
-    tma_issued = 1;
-  }
-
-  // ---- initial state (row dv = tid of S0, or zeros): hi/lo copy, and the
-  //      fp32 copy pre-scaled by the decay of the first chunk
-  if (tid < NT) first_chunk_logdecay<C>(tid, g_next, s_part, s_GCn);
-  __syncthreads();
-  {
-    const float gc0 = exp2f(*s_GCn * LOG2E);
-    const float4* src = p.S0 ? reinterpret_cast<const float4*>(p.S0 + (size_t(chain) * D + dv) * D)
-                             : nullptr;
-    float v[32];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float4 x = src ? __ldg(src + 8 * cg + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-      v[4 * e] = x.x;
-      v[4 * e + 1] = x.y;
-      v[4 * e + 2] = x.z;
-      v[4 * e + 3] = x.w;
-    }
-    store_state_split32(tlane, cg, v);
-    uint32_t u[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gc0 * v[e]);
-    tmem_st32(tlane + TM_S + 32 * cg, u);
-  }
-  tc_fence_before();
 
   for (int c = 0; c < ntiles; ++c) {
-    const int st = c & 1;
     const int t0 = c * NT;
-    const uint32_t kq = sb + (st ? SM_KQ1 : SM_KQ0);
-    const uint8_t* vtile = sm + (st ? SM_V1 : SM_V0);
-    const bool last_tile = (c + 1 == ntiles);
-
-    // ---- gates of this tile (inclusive in-chunk scan); prefetch the next tile
-    float g_cur = 0.f;
-    if (tid < NT) {
-      g_cur = g_next;
-      s_g[tid] = g_next;
-      s_b[tid] = b_next;
+    float* G = x.gates(c);
+    // ---- gates of tile c: inclusive in-chunk scan of g, decays
+    if (kt < NT) {
+      float gc = g_next;
+      const float bc = b_next;
       g_next = 0.f;
       b_next = 0.f;
-      const int t = t0 + NT + tid;
+      const int t = t0 + NT + kt;
       if (t < T) {
         const size_t gi = (size_t(b) * T + t) * H + h;
         g_next = __ldg(p.g + gi);
         b_next = __ldg(p.beta + gi);
       }
       constexpr int W = C < 32 ? C : 32;
-      const int ln = tid & 31;
+      const int ln = kt & 31;
 #pragma unroll
       for (int off = 1; off < W; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, g_cur, off, W);
-        if ((ln & (W - 1)) >= off) g_cur += y;
+        const float y = __shfl_up_sync(0xffffffffu, gc, off, W);
+        if ((ln & (W - 1)) >= off) gc += y;
       }
       if constexpr (C == 64) {
-        if (tid == 31) *s_part = g_cur;
+        if (kt == 31) *s_part = gc;
+        named_bar(BAR_SCAN, 64);
+        if (kt >= 32) gc += *s_part;
       }
+      G[G_GAM2 / 4 + kt] = gc * LOG2E;
+      G[G_B / 4 + kt] = bc;
     }
-    if (tid == 0 && c + 1 < ntiles) {
-      issue_tile(c + 1);
-      tma_issued = c + 2;
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    if (kt < NT) {
+      const int last = (kt / C) * C + C - 1;
+      const float gi = G[G_GAM2 / 4 + kt], gl = G[G_GAM2 / 4 + last];
+      const float Gm = fast_exp2(gi);
+      G[G_GAM / 4 + kt] = Gm;
+      G[G_BG / 4 + kt] = G[G_B / 4 + kt] * Gm;
+      G[G_DF / 4 + kt] = fast_exp2(gl - gi);
+      if (kt == last) G[G_GC / 4 + kt / C] = fast_exp2(gl);
     }
-    __syncthreads();
-    if (tid < NT) {
-      if constexpr (C == 64) {
-        if (tid >= 32) g_cur += *s_part;
-      }
-      s_gam2[tid] = g_cur * LOG2E;
-    }
-    __syncthreads();
-    if (tid < NT) {
-      const int last = (tid / C) * C + C - 1;
-      const float gi = s_gam2[tid], gl = s_gam2[last];
-      const float G = exp2f(gi);
-      s_Gam[tid] = G;
-      s_bG[tid] = s_b[tid] * G;
-      s_df[tid] = exp2f(gl - gi);
-      if (tid == last) s_GC[tid / C] = exp2f(gl);
-    }
-    if (mbar_wait_bounded(bar_tma0 + 8 * st, (c >> 1) & 1, WAIT_LIMIT_NS))
-      tma_done = c + 1;
-    else
-      flow.fail();
-    __syncthreads();
-    if (*s_abort) goto teardown;
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    if (leader) mbar_arrive(x.bar((c & 1) ? B_GFULL1 : B_GFULL0));
 
     // ---- P = [K; Q] K^T : M=128 (rows of [K;Q]), N=64 (tokens j), K=128 (dk)
-    if (tid == 0) {
-      tc_fence_after();
+    if (!rs.wait(x, x.bar((c & 1) ? B_FULL1 : B_FULL0), (c >> 1) & 1)) break;
+    if (leader) {
+      *x.misc(M_KQ_SEEN) = c + 1;
+      const uint32_t kq = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
       const uint32_t id = idesc_bf16(128, 64, 0, 0, 0);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_ss(tmem + TM_PD, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(kq + off, 16, 1024), id,
+        mma_ss(x.tmem + TM_P, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(kq + off, 16, 1024), id,
                kk > 0);
       }
-      mma_commit(bar_mma);
+      mma_commit(x.bar(B_PFULL));
     }
-    flow.wait_mma();
+    if (!rs.wait(x, x.bar(B_PFULL), c & 1)) break;
 
-    // ---- masks and decays: rows 0..63 -> A (fp32, for the solve); rows 64..127 -> Mq
-    {
-      const int i = row & (NT - 1);
+    // ---- masks and decays, rows 0..63 of P: A = strict_tril(beta_i Dec_ij (k_i . k_j))
+    if (row < NT) {
+      const int i = row;
       const int cs = (i / C) * C;
-      const float gi = s_gam2[i];
-      const float bi = s_b[i];
-      float P[16];
-      tmem_ld16(tlane + TM_PD + 16 * cg, P);
-      float m[16];
+      const float gi = G[G_GAM2 / 4 + i];
+      const float bi = G[G_B / 4 + i];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int j = 16 * cg + e;
-        const bool keep = (j >= cs) && (row < NT ? (j < i) : (j <= i));
-        const float x = exp2f(gi - s_gam2[j]) * P[e];
-        m[e] = keep ? (row < NT ? bi * x : x) : 0.f;
-      }
-      if (row < NT) {
-        float4* dst = reinterpret_cast<float4*>(sA + i * APAD + 16 * cg);
+      for (int half = 0; half < 2; ++half) {
+        float P[32];
+        tmem_ld32(tlane + TM_P + 32 * half, P);
+        float4* dst = reinterpret_cast<float4*>(sA + i * APAD + 32 * half);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = make_float4(m[4 * e], m[4 * e + 1], m[4 * e + 2], m[4 * e + 3]);
-      } else {
-        store_split8(sb + SM_MQH, sb + SM_MQL, i, 2 * cg, m);
-        store_split8(sb + SM_MQH, sb + SM_MQL, i, 2 * cg + 1, m + 8);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 gj = ld4(G + G_GAM2 / 4 + 32 * half + 4 * e4);
+          const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+          float m[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 32 * half + 4 * e4 + e;
+            const float v = bi * fast_exp2(gi - gjv[e]) * P[4 * e4 + e];
+            m[e] = (j >= cs && j < i) ? v : 0.f;
+          }
+          dst[e4] = make_float4(m[0], m[1], m[2], m[3]);
+        }
       }
     }
-    fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    named_bar(BAR_SIDE, SIDE_THREADS);
 
     // ---- T = (I + A)^{-1}, blocked in 16 x 16 blocks.
-    //  (1) diagonal blocks: thread r < 64 forms row r of its block's inverse,
+    //  (1) diagonal blocks: lane r < 64 forms row r of its block's inverse,
     //      x (I + A_bb) = e_r, right-looking: x_i is final once every row
     //      below it has been subtracted, then x_i A_i,j leaves each acc_j (j < i);
-    //  (2) with chunk 64, the off-diagonal blocks by distance d = 1..3:
-    //      T_{I,J} = -T_{I,I} sum_{K=J}^{I-1} A_{I,K} T_{K,J}.
-    if (tid < NT) {
-      const int r = tid, bb = r >> 4, rr = r & 15, base = bb * 16;
+    //  (2) with chunk 64, the off-diagonal blocks by distance d = 1..3.
+    if (kt < NT) {
+      const int r = kt, bb = r >> 4, rr = r & 15, base = bb * 16;
       float acc[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) acc[j] = (j == rr) ? 1.f : 0.f;
 #pragma unroll
       for (int i = 15; i > 0; --i) {
         const float xi = acc[i];
-        const float4* arow = reinterpret_cast<const float4*>(sA + (base + i) * APAD + base);
+        const float* arow = sA + (base + i) * APAD + base;
 #pragma unroll
         for (int j4 = 0; j4 < 4; ++j4) {
           if (4 * j4 < i) {
-            const float4 a = arow[j4];
+            const float4 a = ld4(arow + 4 * j4);
             if (4 * j4 + 0 < i) acc[4 * j4 + 0] = fmaf(-xi, a.x, acc[4 * j4 + 0]);
             if (4 * j4 + 1 < i) acc[4 * j4 + 1] = fmaf(-xi, a.y, acc[4 * j4 + 1]);
             if (4 * j4 + 2 < i) acc[4 * j4 + 2] = fmaf(-xi, a.z, acc[4 * j4 + 2]);
@@ -483,130 +412,244 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         trow[q4] = v;
       }
     }
-    __syncthreads();
+    named_bar(BAR_SIDE, SIDE_THREADS);
     if constexpr (C == 64) {
-      solve_offdiag<1>(tid, sA, sTf, sE);
-      solve_offdiag<2>(tid, sA, sTf, sE);
-      solve_offdiag<3>(tid, sA, sTf, sE);
+      solve_offdiag<1>(kt, sA, sTf, sE);
+      solve_offdiag<2>(kt, sA, sTf, sE);
+      solve_offdiag<3>(kt, sA, sTf, sE);
     }
-    // T (fp32) -> hi/lo bf16 K-major tiles; eight threads per row, one chunk each
-    store_split8(sb + SM_TH, sb + SM_TL, tid >> 3, tid & 7, sTf + (tid >> 3) * APAD + 8 * (tid & 7));
-    fence_proxy_async_smem();
-    __syncthreads();
 
-#pragma unroll 1
-    for (int s = 0; s < NSUB; ++s) {
-      // ---- [Z | Y] = S_c [K | Q]^T : M=128 (dv), N=2C, K=128 (dk); A = S hi, then S lo
-      if (tid == 0) {
-        tc_fence_after();
+    // ---- hand T(c), Mq(c) to the chain once it is done with tile c-1's
+    if (c > 0 && !rs.wait(x, x.bar(B_TMFREE), (c - 1) & 1)) break;
+    if (row < NT) {
+      // T row r (fp32) -> hi/lo bf16, K-major rows
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t a0 = tmem + (part ? TM_SLO : TM_SHI);
+      for (int c8 = 0; c8 < 8; ++c8)
+        store_split8(x.sb + SM_TH, x.sb + SM_TL, row, c8, sTf + row * APAD + 8 * c8);
+    } else {
+      // Mq row i = tril(Dec_ij (q_i . k_j)), from rows 64..127 of P
+      const int i = row - NT;
+      const int cs = (i / C) * C;
+      const float gi = G[G_GAM2 / 4 + i];
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            const uint32_t acc = (part | kk) ? 1u : 0u;
-            if constexpr (C == 64) {
-              mma_ts(tmem + TM_ZQ, a0 + kk * 8, sdesc_sw128(kq + off, 16, 1024),
-                     idesc_bf16(128, 128, 0, 0, 0), acc);
-            } else {
-              const uint32_t rows = 2048u * s;
-              mma_ts(tmem + TM_ZQ + 16 * s, a0 + kk * 8, sdesc_sw128(kq + off + rows, 16, 1024),
-                     idesc_bf16(128, 16, 0, 0, 0), acc);
-              mma_ts(tmem + TM_ZQ + 64 + 16 * s, a0 + kk * 8,
-                     sdesc_sw128(kq + 8192 + off + rows, 16, 1024), idesc_bf16(128, 16, 0, 0, 0),
-                     acc);
-            }
+      for (int half = 0; half < 2; ++half) {
+        float P[32];
+        tmem_ld32(tlane + TM_P + 32 * half, P);
+        float m[32];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 gj = ld4(G + G_GAM2 / 4 + 32 * half + 4 * e4);
+          const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 32 * half + 4 * e4 + e;
+            const float v = fast_exp2(gi - gjv[e]) * P[4 * e4 + e];
+            m[4 * e4 + e] = (j >= cs && j <= i) ? v : 0.f;
           }
         }
-        mma_commit(bar_mma);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          store_split8(x.sb + SM_MQH, x.sb + SM_MQL, i, 4 * half + c8, m + 8 * c8);
       }
-      flow.wait_mma();
+    }
+    fence_proxy_async_smem();
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    if (leader) mbar_arrive(x.bar(B_TMFULL));
+  }
+}
+
+// ============================================================== chain
+template <int C>
+__device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
+                           const CUtensorMap* tv, const PrefillArgs& p, int chain, int b, int h,
+                           int ntiles) {
+  constexpr int NSUB = NT / C;
+  constexpr int NC = C / 2;  // columns of a chunk per chain thread
+  const int warp = threadIdx.x >> 5;
+  const int lq = warp & 3;
+  const int ch = (warp >= 12) ? 1 : 0;      // column half
+  const int dv = lq * 32 + (threadIdx.x & 31);
+  const bool leader = (threadIdx.x == 0);
+  const uint32_t tlane = x.tmem + (uint32_t(lq * 32) << 16);
+  const uint32_t sb = x.sb;
+  RoleSync rs{BAR_CHAIN, CHAIN_THREADS, M_FLAG_CHAIN, leader, 0};
+
+  // ---- initial state (row dv of S0, or zeros): hi/lo copy, and the fp32 copy
+  //      pre-scaled by the decay of the first chunk
+  if (!rs.wait(x, x.bar(B_GFULL0), 0)) return;
+  {
+    const float gc0 = x.gates(0)[G_GC / 4];
+    const float4* src =
+        p.S0 ? reinterpret_cast<const float4*>(p.S0 + (size_t(chain) * D + dv) * D) : nullptr;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int qq = 2 * ch + q;  // 32-column group
+      float v[32];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float4 a = src ? __ldg(src + 8 * qq + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[4 * e] = a.x;
+        v[4 * e + 1] = a.y;
+        v[4 * e + 2] = a.z;
+        v[4 * e + 3] = a.w;
+      }
+      store_state_split32(tlane, qq, v);
+      uint32_t u[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gc0 * v[e]);
+      tmem_st32(tlane + TM_S + 32 * qq, u);
+    }
+  }
+  tc_fence_before();
+  named_bar(BAR_CHAIN, CHAIN_THREADS);
+
+  uint32_t sc = 0;  // chunks processed (phase of the per-chunk MMA barriers)
+  for (int c = 0; c < ntiles; ++c) {
+    const uint32_t kq = sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
+    const float* G = x.gates(c);
+    const bool last_tile = (c + 1 == ntiles);
+#pragma unroll 1
+    for (int s = 0; s < NSUB; ++s, ++sc) {
+      // ---- [Z | Y] = S_c [K | Q]^T : M=128 (dv), N=2C, K=128 (dk); A = S hi, then S lo
+      if (leader) {
+        bool ok = true;
+        if (s == 0) {
+          ok = mbar_wait_bounded(x.bar((c & 1) ? B_FULL1 : B_FULL0), (c >> 1) & 1, WAIT_LIMIT_NS);
+          if (ok && c > 0) ok = mbar_wait_bounded(x.bar(B_OUTFREE), (c - 1) & 1, WAIT_LIMIT_NS);
+        }
+        if (!ok) x.fail();
+        if (ok && !*x.abort_flag) {
+          tc_fence_after();
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {
+            const uint32_t a0 = x.tmem + (part ? TM_SLO : TM_SHI);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+              const uint32_t acc = (part | kk) ? 1u : 0u;
+              if constexpr (C == 64) {
+                mma_ts(x.tmem + TM_Z, a0 + kk * 8, sdesc_sw128(kq + off, 16, 1024),
+                       idesc_bf16(128, 128, 0, 0, 0), acc);
+              } else {
+                const uint32_t rows = 2048u * s;
+                mma_ts(x.tmem + TM_Z + 16 * s, a0 + kk * 8, sdesc_sw128(kq + off + rows, 16, 1024),
+                       idesc_bf16(128, 16, 0, 0, 0), acc);
+                mma_ts(x.tmem + TM_Y + 16 * s, a0 + kk * 8,
+                       sdesc_sw128(kq + 8192 + off + rows, 16, 1024), idesc_bf16(128, 16, 0, 0, 0),
+                       acc);
+              }
+            }
+          }
+          mma_commit(x.bar(B_ZQ));
+        }
+      }
+      if (!rs.wait(x, x.bar(B_ZQ), sc & 1)) return;
+      if (s == 0) {
+        if (!rs.wait(x, x.bar((c & 1) ? B_GFULL1 : B_GFULL0), (c >> 1) & 1)) return;
+        if (!rs.wait(x, x.bar(B_VFULL), c & 1)) return;
+        if (leader) *x.misc(M_V_SEEN) = c + 1;
+      }
 
       // ---- X^T[dv][n] = beta_n V[n][dv] - beta_n Gamma_n Z[dv][n]  (hi/lo -> SMEM)
       {
-        const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(vtile);
-        if constexpr (C == 64) {
-          const int n0 = 16 * cg;
-          float Z[16];
-          tmem_ld16(tlane + TM_ZQ + n0, Z);
-          float x[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int n = n0 + e;
-            x[e] = fmaf(s_b[n], __bfloat162float(V[n * D + dv]), -s_bG[n] * Z[e]);
-          }
-          store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8, x);
-          store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8 + 1, x + 8);
+        const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(x.sm + SM_V);
+        const int n0 = C * s + NC * ch;
+        float z[NC];
+        if constexpr (NC == 32) {
+          tmem_ld32(tlane + TM_Z + n0, z);
         } else {
-          const int n0 = 16 * s + 4 * cg;
-          float Z[4];
-          tmem_ld4(tlane + TM_ZQ + n0, Z);
-          float x[4];
+          float za[4], zb[4];
+          tmem_ld4(tlane + TM_Z + n0, za);
+          tmem_ld4(tlane + TM_Z + n0 + 4, zb);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int n = n0 + e;
-            x[e] = fmaf(s_b[n], __bfloat162float(V[n * D + dv]), -s_bG[n] * Z[e]);
+            z[e] = za[e];
+            z[4 + e] = zb[e];
           }
-          store_split4(sb + SM_XH, sb + SM_XL, dv, n0 / 8, (n0 / 4) & 1, x);
         }
+        float xv[NC];
+#pragma unroll
+        for (int e4 = 0; e4 < NC / 4; ++e4) {
+          const float4 bb = ld4(G + G_B / 4 + n0 + 4 * e4);
+          const float4 bg = ld4(G + G_BG / 4 + n0 + 4 * e4);
+          const float bv[4] = {bb.x, bb.y, bb.z, bb.w};
+          const float gv[4] = {bg.x, bg.y, bg.z, bg.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int n = n0 + 4 * e4 + e;
+            xv[4 * e4 + e] = fmaf(bv[e], __bfloat162float(V[n * D + dv]), -gv[e] * z[4 * e4 + e]);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < NC / 8; ++e) store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8 + e, xv + 8 * e);
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      __syncthreads();
+      named_bar(BAR_CHAIN, CHAIN_THREADS);
+      if (leader && s == NSUB - 1 && !last_tile) issue_v(x, tv, c + 1, h, b);  // V(c) fully read
 
       // ---- Dl^T = X^T T^T : M=128 (dv), N=C (i), K=C (n); 3 hi/lo products
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
-        const uint32_t trow = uint32_t(C * s / 8) * 1024u;
+      if (leader) {
+        bool ok = true;
+        if (s == 0) ok = mbar_wait_bounded(x.bar(B_TMFULL), c & 1, WAIT_LIMIT_NS);
+        if (!ok) x.fail();
+        if (ok && !*x.abort_flag) {
+          tc_fence_after();
+          const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
+          const uint32_t trow = uint32_t(C * s / 8) * 1024u;
 #pragma unroll
-        for (int part = 0; part < 3; ++part) {
-          const uint32_t xa = sb + (part == 2 ? SM_XL : SM_XH);
-          const uint32_t tb = sb + (part == 1 ? SM_TL : SM_TH) + trow;
+          for (int part = 0; part < 3; ++part) {
+            const uint32_t xa = sb + (part == 2 ? SM_XL : SM_XH);
+            const uint32_t tb = sb + (part == 1 ? SM_TL : SM_TH) + trow;
 #pragma unroll
-          for (int ks = 0; ks < C / 16; ++ks) {
-            const uint32_t kb = uint32_t(C * s + 16 * ks) * 2u;
-            mma_ss(tmem + TM_PD + C * s, sdesc_sw128(xa + kb, 16, 1024),
-                   sdesc_sw128(tb + kb, 16, 1024), id, (part | ks) ? 1u : 0u);
+            for (int ks = 0; ks < C / 16; ++ks) {
+              const uint32_t kb = uint32_t(C * s + 16 * ks) * 2u;
+              mma_ss(x.tmem + TM_Z + C * s, sdesc_sw128(xa + kb, 16, 1024),
+                     sdesc_sw128(tb + kb, 16, 1024), id, (part | ks) ? 1u : 0u);
+            }
           }
+          mma_commit(x.bar(B_DL));
         }
-        mma_commit(bar_mma);
       }
-      flow.wait_mma();
+      if (!rs.wait(x, x.bar(B_DL), sc & 1)) return;
 
       // ---- residuals: Dl (for the output) and Dl * exp(gamma_last - gamma) (for the state)
       {
-        if constexpr (C == 64) {
-          const int n0 = 16 * cg;
-          float d[16];
-          tmem_ld16(tlane + TM_PD + n0, d);
-          float dt[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) dt[e] = d[e] * s_df[n0 + e];
-          store_split8(sb + SM_DH, sb + SM_DL, dv, n0 / 8, d);
-          store_split8(sb + SM_DH, sb + SM_DL, dv, n0 / 8 + 1, d + 8);
-          store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8, dt);
-          store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8 + 1, dt + 8);
+        const int n0 = C * s + NC * ch;
+        float d[NC];
+        if constexpr (NC == 32) {
+          tmem_ld32(tlane + TM_Z + n0, d);
         } else {
-          const int n0 = 16 * s + 4 * cg;
-          float d[4];
-          tmem_ld4(tlane + TM_PD + n0, d);
-          float dt[4];
+          float da[4], db[4];
+          tmem_ld4(tlane + TM_Z + n0, da);
+          tmem_ld4(tlane + TM_Z + n0 + 4, db);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dt[e] = d[e] * s_df[n0 + e];
-          store_split4(sb + SM_DH, sb + SM_DL, dv, n0 / 8, (n0 / 4) & 1, d);
-          store_split4(sb + SM_XH, sb + SM_XL, dv, n0 / 8, (n0 / 4) & 1, dt);
+          for (int e = 0; e < 4; ++e) {
+            d[e] = da[e];
+            d[4 + e] = db[e];
+          }
         }
-        // log-decay of the next tile's first chunk (its gates arrived long ago)
-        if (s == NSUB - 1 && !last_tile && tid < NT) first_chunk_logdecay<C>(tid, g_next, s_part, s_GCn);
+        float dt[NC];
+#pragma unroll
+        for (int e4 = 0; e4 < NC / 4; ++e4) {
+          const float4 f = ld4(G + G_DF / 4 + n0 + 4 * e4);
+          dt[4 * e4 + 0] = d[4 * e4 + 0] * f.x;
+          dt[4 * e4 + 1] = d[4 * e4 + 1] * f.y;
+          dt[4 * e4 + 2] = d[4 * e4 + 2] * f.z;
+          dt[4 * e4 + 3] = d[4 * e4 + 3] * f.w;
+        }
+#pragma unroll
+        for (int e = 0; e < NC / 8; ++e) {
+          store_split8(sb + SM_DH, sb + SM_DL, dv, n0 / 8 + e, d + 8 * e);
+          store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8 + e, dt + 8 * e);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      __syncthreads();
+      named_bar(BAR_CHAIN, CHAIN_THREADS);
 
       // ---- O_intra = Dl^T Mq^T (N=C) and S += Dl~^T K (N=128, B = K tile MN-major)
-      if (tid == 0) {
+      if (leader && !*x.abort_flag) {
         tc_fence_after();
         const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
         const uint32_t mrow = uint32_t(C * s / 8) * 1024u;
@@ -617,7 +660,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int ks = 0; ks < C / 16; ++ks) {
             const uint32_t kb = uint32_t(C * s + 16 * ks) * 2u;
-            mma_ss(tmem + TM_OI + C * s, sdesc_sw128(da + kb, 16, 1024),
+            mma_ss(x.tmem + TM_OI + C * s, sdesc_sw128(da + kb, 16, 1024),
                    sdesc_sw128(mb + kb, 16, 1024), id, (part | ks) ? 1u : 0u);
           }
         }
@@ -628,72 +671,153 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
           for (int ks = 0; ks < C / 16; ++ks) {
             const int tok = C * s + 16 * ks;
-            mma_ss(tmem + TM_S, sdesc_sw128(da + uint32_t(tok) * 2u, 16, 1024),
+            mma_ss(x.tmem + TM_S, sdesc_sw128(da + uint32_t(tok) * 2u, 16, 1024),
                    sdesc_sw128(kq + uint32_t(tok) * 128u, 16384, 1024), idu, 1u);
           }
         }
-        mma_commit(bar_mma);
+        mma_commit(x.bar(B_OU));
+        if (s == NSUB - 1) {
+          mma_commit(x.bar(B_TMFREE));   // T(c), Mq(c) consumed
+          mma_commit(x.bar(B_OUTFULL));  // Y(c), O_intra(c) complete
+        }
       }
-      flow.wait_mma();
+      if (!rs.wait(x, x.bar(B_OU), sc & 1)) return;
+      if (leader && s == NSUB - 1 && c + 2 < ntiles) issue_kq(x, tq, tk, c + 2, h, b);  // KQ(c) read
 
       // ---- S_out now sits in TMEM: refresh its hi/lo copy, and pre-scale it by
       //      the next chunk's decay (or store it as S_T after the last chunk)
       {
         const bool final_chunk = last_tile && (s == NSUB - 1);
-        const float gnext = (s + 1 < NSUB) ? s_GC[s + 1] : exp2f(*s_GCn * LOG2E);
-        float v[32];
-        tmem_ld32(tlane + TM_S + 32 * cg, v);
-        store_state_split32(tlane, cg, v);
-        if (final_chunk) {
-          float4* dst = reinterpret_cast<float4*>(p.S_T + (size_t(chain) * D + dv) * D + 32 * cg);
+        float gnext = 0.f;
+        if (s + 1 < NSUB) {
+          gnext = G[G_GC / 4 + s + 1];
+        } else if (!last_tile) {
+          if (!rs.wait(x, x.bar(((c + 1) & 1) ? B_GFULL1 : B_GFULL0), ((c + 1) >> 1) & 1)) return;
+          gnext = x.gates(c + 1)[G_GC / 4];
+        }
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-        } else {
-          uint32_t u[32];
+        for (int q = 0; q < 2; ++q) {
+          const int qq = 2 * ch + q;
+          float v[32];
+          tmem_ld32(tlane + TM_S + 32 * qq, v);
+          store_state_split32(tlane, qq, v);
+          if (final_chunk) {
+            float4* dst = reinterpret_cast<float4*>(p.S_T + (size_t(chain) * D + dv) * D + 32 * qq);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v[e]);
-          tmem_st32(tlane + TM_S + 32 * cg, u);
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          } else {
+            uint32_t u[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v[e]);
+            tmem_st32(tlane + TM_S + 32 * qq, u);
+          }
         }
       }
       tc_fence_before();
-      __syncthreads();
-      if (*s_abort) goto teardown;
+      if (!rs.check(x)) return;
     }
-
-    // ---- o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t]: staged in SMEM, one TMA store
-    {
-      const int n0 = 16 * cg;
-      float y[16], oi[16];
-      tmem_ld16x2(tlane + TM_ZQ + 64 + n0, y, tlane + TM_OI + n0, oi);
-#pragma unroll
-      for (int e = 0; e < 16; ++e) sO[(n0 + e) * D + dv] = fmaf(s_Gam[n0 + e], y[e], oi[e]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
-      tma_store_4d(&tm_o, sb + SM_O, 0, h, t0, b);  // rows past T are clipped by the TMA unit
-      bulk_commit();
-      bulk_wait_read0();  // the o tile region is rewritten by the next tile's solve
-    }
-    __syncthreads();
   }
+}
 
-teardown:
-  // An aborted CTA may still have a TMA tile in flight: wait for it (bounded)
-  // before the shared memory goes away.
-  if (tid == 0) {
-    bulk_wait0();
-    if (*s_abort) {
-      for (int c = tma_done; c < tma_issued; ++c)
-        mbar_wait_bounded(bar_tma0 + 8 * (c & 1), (c >> 1) & 1, WAIT_LIMIT_NS / 4);
+// ============================================================== output
+// o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] of tile c, straight to HBM
+// (each warp store is 32 consecutive floats of one token row).
+__device__ void output_role(const Ctx& x, const PrefillArgs& p, int b, int h, int ntiles) {
+  const int ot = threadIdx.x - 256;
+  const int lq = (threadIdx.x >> 5) & 3;
+  const int dv = lq * 32 + (threadIdx.x & 31);
+  const bool leader = (ot == 0);
+  const uint32_t tlane = x.tmem + (uint32_t(lq * 32) << 16);
+  const int T = p.T, H = p.H;
+  RoleSync rs{BAR_OUT, OUT_THREADS, M_FLAG_OUT, leader, 0};
+  const size_t tstride = size_t(H) * D;
+  for (int c = 0; c < ntiles; ++c) {
+    if (!rs.wait(x, x.bar(B_OUTFULL), c & 1)) return;
+    const float* G = x.gates(c);
+    const int t0 = c * NT;
+    const int nvalid = min(NT, T - t0);
+    float* orow = p.o + ((size_t(b) * T + t0) * H + h) * D + dv;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float y[32], oi[32];
+      tmem_ld32(tlane + TM_Y + 32 * q, y);
+      tmem_ld32(tlane + TM_OI + 32 * q, oi);
+#pragma unroll
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 gm = ld4(G + G_GAM / 4 + 32 * q + 4 * e4);
+        const float gv[4] = {gm.x, gm.y, gm.z, gm.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int n = 32 * q + 4 * e4 + e;
+          if (n < nvalid) orow[size_t(n) * tstride] = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
+        }
+      }
     }
+    tc_fence_before();
+    named_bar(BAR_OUT, OUT_THREADS);
+    if (leader) mbar_arrive(x.bar(B_OUTFREE));  // Y and O_intra may be overwritten
+  }
+}
+
+template <int C>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const PrefillArgs p) {
+  static_assert(C == 16 || C == 64, "chunk must be 16 or 64");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int chain = blockIdx.x;
+  const int b = chain / p.H;
+  const int h = chain - b * p.H;
+  const int ntiles = (p.T + NT - 1) / NT;
+
+  Ctx x;
+  x.sm = sm;
+  x.sb = smem_u32(sm);
+  x.status = p.status;
+  x.abort_flag = reinterpret_cast<volatile int*>(sm + SM_MISC + M_ABORT);
+  if (tid == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    for (int i = 0; i < NUM_BARS; ++i) mbar_init(x.sb + SM_BAR + 8 * i, 1);
+    fence_mbar_init();
+    for (int i = 0; i < 16; ++i) reinterpret_cast<volatile int*>(sm + SM_MISC)[i] = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(sm + SM_MISC + M_TMEM), TMEM_COLS);
+    tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+  x.tmem = *reinterpret_cast<volatile uint32_t*>(sm + SM_MISC + M_TMEM);
+
+  if (warp < 4 || warp >= 12)
+    chain_role<C>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
+  else if (warp < 8)
+    kside_role<C>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
+  else
+    output_role(x, p, b, h, ntiles);
+
+  tc_fence_before();
+  __syncthreads();
+  // An aborted CTA may still have TMA loads in flight: wait for them (bounded)
+  // before the shared memory is released.
+  if (tid == 0 && *x.abort_flag) {
+    const int kq_issued = *x.misc(M_KQ_ISSUED), kq_seen = *x.misc(M_KQ_SEEN);
+    for (int c = kq_seen; c < kq_issued; ++c)
+      mbar_wait_bounded(x.bar((c & 1) ? B_FULL1 : B_FULL0), (c >> 1) & 1, WAIT_LIMIT_NS / 4);
+    const int v_issued = *x.misc(M_V_ISSUED), v_seen = *x.misc(M_V_SEEN);
+    if (v_issued > v_seen) mbar_wait_bounded(x.bar(B_VFULL), (v_issued - 1) & 1, WAIT_LIMIT_NS / 4);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(x.tmem, TMEM_COLS);
 }
 
 // T == 0: S_T = S0 (or zeros); nothing else to do.
@@ -709,7 +833,7 @@ __global__ void copy_state_kernel(const float* __restrict__ S0, float* __restric
 }  // namespace
 
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const CUtensorMap& to, const PrefillArgs& a, int chunk, cudaStream_t stream) {
+                   const PrefillArgs& a, int chunk, cudaStream_t stream) {
   const int chains = a.B * a.H;
   if (chains == 0) return 0;
   if (a.T == 0) {
@@ -724,12 +848,12 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     err = cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                int(smem));
     if (err != cudaSuccess) return -1;
-    prefill_kernel<64><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, a);
+    prefill_kernel<64><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, a);
   } else {
     err = cudaFuncSetAttribute(prefill_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                int(smem));
     if (err != cudaSuccess) return -1;
-    prefill_kernel<16><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, a);
+    prefill_kernel<16><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, a);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
