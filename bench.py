@@ -104,7 +104,8 @@ def committed_traffic(key, paths):
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons with nvidia-smi (logged to a
+    temporary file, which survives the sampler being terminated) while running."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -113,30 +114,37 @@ class ClockSampler:
         self.gpu_index = gpu_index
         self.proc = None
         self.lines = []
+        self.path = None
 
     def __enter__(self):
+        import tempfile
         try:
+            fd, self.path = tempfile.mkstemp(prefix="gdn_clocks_", suffix=".csv")
+            os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
+                 "--format=csv,noheader,nounits", "-lms", "50", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)  # let the first samples land before the timed work starts
         except Exception:
             self.proc = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.1)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self.path:
+            try:
+                with open(self.path) as f:
+                    self.lines = [ln.strip() for ln in f if ln.strip()]
+                os.unlink(self.path)
+            except Exception:
+                pass
 
     def summary(self):
         rows = []
@@ -231,8 +239,8 @@ def run_ours(args, world, rank, local):
 
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        step_ms = time_steps(call, args.steps, args.warmup, flush, stream)
+    clk = ClockSampler(local).__enter__()
+    step_ms = time_steps(call, args.steps, args.warmup, flush, stream)
     torch.cuda.synchronize()
     barrier(world)
     total_ms = max_over_ranks(sum(step_ms), world)
@@ -282,6 +290,7 @@ def run_ours(args, world, rank, local):
     extras = None
     if not args.no_extras:
         extras = run_extras(args, dev, stream, flush, peaks, rank)
+    clk.__exit__(None, None, None)
 
     cpu = None
     if rank == 0 and world == 1:

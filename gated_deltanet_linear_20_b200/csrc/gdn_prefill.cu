@@ -695,24 +695,40 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           if (!rs.wait(x, x.bar(((c + 1) & 1) ? B_GFULL1 : B_GFULL0), ((c + 1) >> 1) & 1)) return;
           gnext = x.gates(c + 1)[G_GC / 4];
         }
+        // one pass over this thread's 64 columns: both loads, then all stores, one wait
+        float v0[32], v1[32];
+        tmem_ld32x2(tlane + TM_S + 64 * ch, v0, tlane + TM_S + 64 * ch + 32, v1);
+        {
+          uint32_t hi[16], lo[16];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int qq = 2 * ch + q;
-          float v[32];
-          tmem_ld32(tlane + TM_S + 32 * qq, v);
-          store_state_split32(tlane, qq, v);
-          if (final_chunk) {
-            float4* dst = reinterpret_cast<float4*>(p.S_T + (size_t(chain) * D + dv) * D + 32 * qq);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-          } else {
-            uint32_t u[32];
-#pragma unroll
-            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v[e]);
-            tmem_st32(tlane + TM_S + 32 * qq, u);
-          }
+          for (int e = 0; e < 16; ++e) split2_bf16(v0[2 * e], v0[2 * e + 1], hi[e], lo[e]);
+          tmem_st16_nowait(tlane + TM_SHI + 32 * ch, hi);
+          tmem_st16_nowait(tlane + TM_SLO + 32 * ch, lo);
         }
+        {
+          uint32_t hi[16], lo[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) split2_bf16(v1[2 * e], v1[2 * e + 1], hi[e], lo[e]);
+          tmem_st16_nowait(tlane + TM_SHI + 32 * ch + 16, hi);
+          tmem_st16_nowait(tlane + TM_SLO + 32 * ch + 16, lo);
+        }
+        if (final_chunk) {
+          float4* dst = reinterpret_cast<float4*>(p.S_T + (size_t(chain) * D + dv) * D + 64 * ch);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            dst[e] = make_float4(v0[4 * e], v0[4 * e + 1], v0[4 * e + 2], v0[4 * e + 3]);
+            dst[8 + e] = make_float4(v1[4 * e], v1[4 * e + 1], v1[4 * e + 2], v1[4 * e + 3]);
+          }
+        } else {
+          uint32_t u[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v0[e]);
+          tmem_st32_nowait(tlane + TM_S + 64 * ch, u);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v1[e]);
+          tmem_st32_nowait(tlane + TM_S + 64 * ch + 32, u);
+        }
+        tmem_wait_st();
       }
       tc_fence_before();
       if (!rs.check(x)) return;
@@ -738,25 +754,26 @@ __device__ void output_role(const Ctx& x, const PrefillArgs& p, int b, int h, in
     const int t0 = c * NT;
     const int nvalid = min(NT, T - t0);
     float* orow = p.o + ((size_t(b) * T + t0) * H + h) * D + dv;
+    float o[NT];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       float y[32], oi[32];
-      tmem_ld32(tlane + TM_Y + 32 * q, y);
-      tmem_ld32(tlane + TM_OI + 32 * q, oi);
+      tmem_ld32x2(tlane + TM_Y + 32 * q, y, tlane + TM_OI + 32 * q, oi);
 #pragma unroll
       for (int e4 = 0; e4 < 8; ++e4) {
         const float4 gm = ld4(G + G_GAM / 4 + 32 * q + 4 * e4);
-        const float gv[4] = {gm.x, gm.y, gm.z, gm.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int n = 32 * q + 4 * e4 + e;
-          if (n < nvalid) orow[size_t(n) * tstride] = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
-        }
+        o[32 * q + 4 * e4 + 0] = fmaf(gm.x, y[4 * e4 + 0], oi[4 * e4 + 0]);
+        o[32 * q + 4 * e4 + 1] = fmaf(gm.y, y[4 * e4 + 1], oi[4 * e4 + 1]);
+        o[32 * q + 4 * e4 + 2] = fmaf(gm.z, y[4 * e4 + 2], oi[4 * e4 + 2]);
+        o[32 * q + 4 * e4 + 3] = fmaf(gm.w, y[4 * e4 + 3], oi[4 * e4 + 3]);
       }
     }
     tc_fence_before();
     named_bar(BAR_OUT, OUT_THREADS);
     if (leader) mbar_arrive(x.bar(B_OUTFREE));  // Y and O_intra may be overwritten
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+      if (n < nvalid) orow[size_t(n) * tstride] = o[n];
   }
 }
 
