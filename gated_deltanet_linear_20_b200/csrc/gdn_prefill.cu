@@ -27,13 +27,13 @@
 //   * chain  (warps 0-3 and 12-15, 256 threads): everything that depends on
 //     the state -- S_c [K;Q]^T, X, Dl = X T^T, the output and state-update
 //     products and their epilogues -- for tile c;
-//   * K side (warps 4-7): the state-independent work of tile c+1 -- gates,
-//     [K;Q] K^T, the masks and decays, the triangular solve -- handing T and
-//     Mq to the chain once the chain has finished with tile c's;
-//   * output (warps 8-11): o of tile c from tensor memory to HBM while the
-//     chain starts tile c+1.
-// Warp w reads TMEM lane quarter (w % 4); the two chain warpgroups split the
-// columns of each tile in halves.  The fp32 state lives in tensor memory,
+//   * side (warps 4-11, 256 threads): the state-independent work of tile c+1
+//     -- gates, [K;Q] K^T, the masks and decays, the triangular solve --
+//     handing T and Mq to the chain once the chain has finished with tile
+//     c's, and draining o of tile c from tensor memory to HBM as soon as the
+//     chain has produced it.
+// Warp w reads TMEM lane quarter (w % 4); the two warpgroups of each role
+// split the columns of each tile in halves.  The fp32 state lives in tensor memory,
 // pre-multiplied by the decay of the chunk about to update it, so the
 // state-update MMA accumulates straight into it; the tensor core reads the
 // state as a bf16 hi/lo pair, also in tensor memory.  Every operand derived
@@ -60,8 +60,8 @@ using namespace sm100;
 constexpr int D = 128;
 constexpr int NT = 64;  // tokens per TMA tile
 constexpr int NTHREADS = 512;
-constexpr int CHAIN_THREADS = 256, SIDE_THREADS = 128, OUT_THREADS = 128;
-constexpr int BAR_CHAIN = 1, BAR_SIDE = 2, BAR_OUT = 3, BAR_SCAN = 4;  // named barriers
+constexpr int CHAIN_THREADS = 256, SIDE_THREADS = 256;
+constexpr int BAR_CHAIN = 1, BAR_SIDE = 2, BAR_SCAN = 3;  // named barriers
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S = 0, TM_SHI = 128, TM_SLO = 192, TM_Z = 256, TM_Y = 320, TM_P = 384,
                    TM_OI = 448;
@@ -82,26 +82,36 @@ constexpr int APAD = 68;                      // row pitch (floats): conflict-fr
 constexpr uint32_t SOLVE_MAT = 64 * APAD * 4; // 17408 B
 constexpr uint32_t SM_A = 180224;             // A  fp32 [64][APAD] (K side)
 constexpr uint32_t SM_TF = SM_A + SOLVE_MAT;  // T  fp32 [64][APAD] (K side)
-constexpr uint32_t SM_E = SM_TF + SOLVE_MAT;  // block products fp32 [3][16][16]
-constexpr uint32_t SM_GATES = SM_E + 3072;    // 3 gate buffers (tile c uses c % 3)
+constexpr uint32_t SM_AT = SM_TF + SOLVE_MAT; // T_II A_IK blocks fp32 [6][16][16] (K side)
+constexpr uint32_t SM_GATES = SM_AT + 6144;   // gate buffers (tile c uses c % GATE_BUFS)
 constexpr uint32_t GATE_BYTES = 1536;
+// The side role writes tile c's gates after the chain released tile c-3
+// (tm_free); the chain's last reader of tile c-4's buffer (the o drain) runs
+// before it starts tile c-3's MMAs, so four buffers never overlap a reader.
+constexpr int GATE_BUFS = 4;
 constexpr uint32_t G_GAM2 = 0, G_B = 256, G_BG = 512, G_DF = 768, G_GAM = 1024, G_GC = 1280;
-constexpr uint32_t SM_BAR = SM_GATES + 3 * GATE_BYTES;
+constexpr uint32_t SM_BAR = SM_GATES + GATE_BUFS * GATE_BYTES;
 constexpr uint32_t SM_MISC = SM_BAR + 256;    // TMEM slot, abort flags, scan scratch, counters
 constexpr uint32_t SMEM_USED = SM_MISC + 256;
 static_assert(SM_A >= SM_DL + 16384, "K-side scratch overlaps the residual tiles");
 static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 
 // mbarriers (8 bytes each, offsets inside SM_BAR)
-constexpr uint32_t B_FULL0 = 0, B_FULL1 = 8, B_VFULL = 16, B_PFULL = 24, B_GFULL0 = 32,
-                   B_GFULL1 = 40, B_TMFULL = 48, B_TMFREE = 56, B_ZQ = 64, B_DL = 72, B_OU = 80,
-                   B_OUTFULL = 88, B_OUTFREE = 96;
+// The gates of tile c are signalled on B_GFULL + 8 (c % 4): the side role can
+// finish the gates of tile c + 2 before the chain has waited for tile c's, so
+// two barriers with parity waits could alias; four cannot (tile c + 4 needs
+// the chain to have finished tile c + 2).
+constexpr uint32_t B_FULL0 = 0, B_FULL1 = 8, B_VFULL = 16, B_PFULL = 24, B_TMFULL = 32,
+                   B_TMFREE = 40, B_ZQ = 48, B_DL = 56, B_OU = 64, B_GFULL = 72;
 constexpr int NUM_BARS = 13;
+__device__ __forceinline__ uint32_t gfull_off(int c) { return B_GFULL + 8u * uint32_t(c & 3); }
+__device__ __forceinline__ uint32_t gfull_parity(int c) { return uint32_t(c >> 2) & 1u; }
 // misc slots (offsets inside SM_MISC)
 constexpr uint32_t M_TMEM = 0, M_ABORT = 4, M_PART = 8, M_KQ_ISSUED = 12, M_KQ_SEEN = 16,
-                   M_V_ISSUED = 20, M_V_SEEN = 24, M_FLAG_CHAIN = 32, M_FLAG_SIDE = 40,
-                   M_FLAG_OUT = 48;  // two verdict slots per role
-static_assert(M_FLAG_OUT + 8 <= 256, "misc slots");
+                   M_V_ISSUED = 20, M_V_SEEN = 24, M_FLAG_CHAIN = 32,
+                   M_FLAG_SIDE = 40;  // two verdict slots per role
+static_assert(M_FLAG_SIDE + 8 <= 256, "misc slots");
+static_assert(8 * NUM_BARS <= 256, "barrier slots");
 
 constexpr uint32_t KQ_TX_BYTES = 4 * 8192;
 constexpr uint32_t V_TX_BYTES = 16384;
@@ -148,7 +158,7 @@ struct Ctx {
   volatile int* abort_flag;
   __device__ __forceinline__ uint32_t bar(uint32_t off) const { return sb + SM_BAR + off; }
   __device__ __forceinline__ float* gates(int c) const {
-    return reinterpret_cast<float*>(sm + SM_GATES + (c % 3) * GATE_BYTES);
+    return reinterpret_cast<float*>(sm + SM_GATES + (c % GATE_BUFS) * GATE_BYTES);
   }
   __device__ __forceinline__ volatile int* misc(uint32_t off) const {
     return reinterpret_cast<volatile int*>(sm + SM_MISC + off);
@@ -211,69 +221,171 @@ __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int
   *x.misc(M_V_ISSUED) = c + 1;
 }
 
-// One distance-d sweep of the blocked inverse of (I + A), 64 x 64 in 16 x 16
-// blocks (diagonal blocks already inverted in Tf):
-//   E_p     = sum_{K=J}^{I-1} A_{I,K} T_{K,J}        (I = J + d, p = J)
-//   T_{I,J} = -T_{I,I} E_p
-// A thread owns 1 x 4 strips of outputs; all loop bounds are compile-time.
+// Off-diagonal blocks of T = (I + A)^{-1}, 64 x 64 in 16 x 16 blocks, once the
+// diagonal blocks T_II are in Tf.  With At_IK = T_II A_IK (K < I), block row I
+// of (I + A) T = I gives
+//   T_IJ = -sum_{K=J}^{I-1} At_IK T_KJ            (I > J),
+// computed by distance d = I - J = 1, 2, 3 after one pass that forms all six
+// At blocks.  A thread owns 1 x 4 strips of outputs; each dot product is split
+// over two accumulators; all loop bounds are compile-time.
+__device__ __forceinline__ int at_index(int I, int K) { return (I * (I - 1)) / 2 + K; }  // 0..5
+
+__device__ __forceinline__ void solve_at_blocks(int kt, const float* sA, const float* sTf, float* sAt) {
+  // 6 blocks x 16 rows x 4 strips = 384 strips
+#pragma unroll
+  for (int st = kt; st < 384; st += SIDE_THREADS) {
+    const int blk = st >> 6, r = (st >> 2) & 15, c4 = st & 3;
+    const int I = blk < 1 ? 1 : (blk < 3 ? 2 : 3);
+    const int K = blk - at_index(I, 0);
+    const float* trow = sTf + (I * 16 + r) * APAD + I * 16;        // T_II row r
+    const float* acol = sA + (I * 16) * APAD + K * 16 + 4 * c4;     // A_IK rows m, cols 4c4..
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+#pragma unroll
+    for (int m = 0; m < 16; m += 2) {
+      const float t0 = trow[m], t1 = trow[m + 1];
+      const float4 x0 = ld4(acol + m * APAD), x1 = ld4(acol + (m + 1) * APAD);
+      a0.x = fmaf(t0, x0.x, a0.x); a0.y = fmaf(t0, x0.y, a0.y);
+      a0.z = fmaf(t0, x0.z, a0.z); a0.w = fmaf(t0, x0.w, a0.w);
+      a1.x = fmaf(t1, x1.x, a1.x); a1.y = fmaf(t1, x1.y, a1.y);
+      a1.z = fmaf(t1, x1.z, a1.z); a1.w = fmaf(t1, x1.w, a1.w);
+    }
+    *reinterpret_cast<float4*>(sAt + blk * 256 + r * 16 + 4 * c4) =
+        make_float4(a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w);
+  }
+}
+
 template <int d>
-__device__ __forceinline__ void solve_offdiag(int kt, const float* sA, float* sTf, float* sE) {
-  constexpr int NSTRIP = (4 - d) * 64;  // (4-d) block pairs x 16 rows x 4 strips
+__device__ __forceinline__ void solve_distance(int kt, const float* sAt, float* sTf) {
+  constexpr int NSTRIP = (4 - d) * 64;
 #pragma unroll
   for (int st = kt; st < NSTRIP; st += SIDE_THREADS) {
-    const int pp = st >> 6, r = (st >> 2) & 15, c4 = st & 3;
-    const float* arow = sA + ((pp + d) * 16 + r) * APAD + pp * 16;
-    const float* tcol = sTf + (pp * 16) * APAD + pp * 16 + 4 * c4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int J = st >> 6, r = (st >> 2) & 15, c4 = st & 3;
+    const int I = J + d;
+    float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
 #pragma unroll
-    for (int k = 0; k < 16 * d; ++k) {
-      const float a = arow[k];
-      const float4 t = ld4(tcol + k * APAD);
-      acc.x = fmaf(a, t.x, acc.x);
-      acc.y = fmaf(a, t.y, acc.y);
-      acc.z = fmaf(a, t.z, acc.z);
-      acc.w = fmaf(a, t.w, acc.w);
+    for (int K = J; K < I; ++K) {
+      const float* atrow = sAt + at_index(I, K) * 256 + r * 16;      // At_IK row r
+      const float* tcol = sTf + (K * 16) * APAD + J * 16 + 4 * c4;    // T_KJ rows, cols 4c4..
+#pragma unroll
+      for (int m = 0; m < 16; m += 2) {
+        const float t0 = atrow[m], t1 = atrow[m + 1];
+        const float4 x0 = ld4(tcol + m * APAD), x1 = ld4(tcol + (m + 1) * APAD);
+        a0.x = fmaf(t0, x0.x, a0.x); a0.y = fmaf(t0, x0.y, a0.y);
+        a0.z = fmaf(t0, x0.z, a0.z); a0.w = fmaf(t0, x0.w, a0.w);
+        a1.x = fmaf(t1, x1.x, a1.x); a1.y = fmaf(t1, x1.y, a1.y);
+        a1.z = fmaf(t1, x1.z, a1.z); a1.w = fmaf(t1, x1.w, a1.w);
+      }
     }
-    *reinterpret_cast<float4*>(sE + pp * 256 + r * 16 + 4 * c4) = acc;
+    *reinterpret_cast<float4*>(sTf + (I * 16 + r) * APAD + J * 16 + 4 * c4) =
+        make_float4(-(a0.x + a1.x), -(a0.y + a1.y), -(a0.z + a1.z), -(a0.w + a1.w));
   }
-  named_bar(BAR_SIDE, SIDE_THREADS);
-#pragma unroll
-  for (int st = kt; st < NSTRIP; st += SIDE_THREADS) {
-    const int pp = st >> 6, r = (st >> 2) & 15, c4 = st & 3;
-    const int I = pp + d;
-    const float* trow = sTf + (I * 16 + r) * APAD + I * 16;
-    const float* e = sE + pp * 256 + 4 * c4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float a = trow[k];
-      const float4 t = ld4(e + k * 16);
-      acc.x = fmaf(a, t.x, acc.x);
-      acc.y = fmaf(a, t.y, acc.y);
-      acc.z = fmaf(a, t.z, acc.z);
-      acc.w = fmaf(a, t.w, acc.w);
-    }
-    *reinterpret_cast<float4*>(sTf + (I * 16 + r) * APAD + pp * 16 + 4 * c4) =
-        make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-  }
-  named_bar(BAR_SIDE, SIDE_THREADS);
 }
 
 // ============================================================== K side
-// Per tile c: gates(c) -> [K;Q] K^T -> masks / decays -> T = (I + A)^{-1};
-// then, once the chain has released tile c-1's T and Mq, writes T(c), Mq(c).
+// Per tile c: [K;Q] K^T -> masks / decays -> T = (I + A)^{-1}; the next
+// tile's [K;Q] K^T is issued as soon as this tile's P has been read, and the
+// next tile's gates are formed before waiting for the chain; then, once the
+// chain has released tile c-1's T and Mq, writes T(c), Mq(c).
+template <int C>
+__device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, float& g_next,
+                                           float& b_next, const PrefillArgs& p, int b, int h,
+                                           volatile float* s_part) {
+  // inclusive in-chunk scan of g over tile c (threads kt < 64), decays
+  float* G = x.gates(c);
+  const int H = p.H;
+  if (kt < NT) {
+    float gc = g_next;
+    const float bc = b_next;
+    g_next = 0.f;
+    b_next = 0.f;
+    const int t = (c + 1) * NT + kt;
+    if (t < T) {
+      const size_t gi = (size_t(b) * T + t) * H + h;
+      g_next = __ldg(p.g + gi);
+      b_next = __ldg(p.beta + gi);
+    }
+    constexpr int W = C < 32 ? C : 32;
+    const int ln = kt & 31;
+#pragma unroll
+    for (int off = 1; off < W; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, gc, off, W);
+      if ((ln & (W - 1)) >= off) gc += y;
+    }
+    if constexpr (C == 64) {
+      if (kt == 31) *s_part = gc;
+      named_bar(BAR_SCAN, 64);
+      if (kt >= 32) gc += *s_part;
+    }
+    G[G_GAM2 / 4 + kt] = gc * LOG2E;
+    G[G_B / 4 + kt] = bc;
+  }
+  named_bar(BAR_SIDE, SIDE_THREADS);
+  if (kt < NT) {
+    const int last = (kt / C) * C + C - 1;
+    const float gi = G[G_GAM2 / 4 + kt], gl = G[G_GAM2 / 4 + last];
+    const float Gm = fast_exp2(gi);
+    G[G_GAM / 4 + kt] = Gm;
+    G[G_BG / 4 + kt] = G[G_B / 4 + kt] * Gm;
+    G[G_DF / 4 + kt] = fast_exp2(gl - gi);
+    if (kt == last) G[G_GC / 4 + kt / C] = fast_exp2(gl);
+  }
+  named_bar(BAR_SIDE, SIDE_THREADS);
+  if (kt == 0) mbar_arrive(x.bar(gfull_off(c)));
+}
+
+__device__ __forceinline__ void issue_p(const Ctx& x, int c) {
+  const uint32_t kq = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
+  const uint32_t id = idesc_bf16(128, 64, 0, 0, 0);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    mma_ss(x.tmem + TM_P, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(kq + off, 16, 1024), id,
+           kk > 0);
+  }
+  mma_commit(x.bar(B_PFULL));
+}
+
+// o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] of tile c, this thread's 32
+// tokens (32 hf .. 32 hf + 31) of lane `dv`, 16 at a time, straight to HBM
+// (each warp store writes 32 consecutive floats of one token row).
+__device__ __forceinline__ void output_drain(const Ctx& x, const PrefillArgs& p, uint32_t tlane,
+                                             int b, int h, int dv, int hf, int c) {
+  const float* G = x.gates(c);
+  const int t0 = c * NT + 32 * hf;
+  const int nvalid = min(32, p.T - t0);
+  float* orow = p.o + ((size_t(b) * p.T + t0) * p.H + h) * D + dv;
+  const size_t tstride = size_t(p.H) * D;
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    float y[16], oi[16];
+    tmem_ld16x2(tlane + TM_Y + 32 * hf + 16 * q, y, tlane + TM_OI + 32 * hf + 16 * q, oi);
+#pragma unroll
+    for (int e4 = 0; e4 < 4; ++e4) {
+      const float4 gm = ld4(G + G_GAM / 4 + 32 * hf + 16 * q + 4 * e4);
+      const float gv[4] = {gm.x, gm.y, gm.z, gm.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int n = 16 * q + 4 * e4 + e;
+        if (n < nvalid) orow[size_t(n) * tstride] = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
+      }
+    }
+  }
+}
+
 template <int C>
 __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, const PrefillArgs& p, int b, int h, int ntiles) {
-  const int kt = threadIdx.x - 128;        // 0..127
-  const int lq = (threadIdx.x >> 5) & 3;
-  const int row = kt;                      // TMEM lane == row of [K;Q]
+  const int kt = threadIdx.x - 128;        // 0..255
+  const int warp = threadIdx.x >> 5;
+  const int lq = warp & 3;
+  const int hf = (warp >= 8) ? 1 : 0;      // column half
+  const int row = lq * 32 + (threadIdx.x & 31);  // TMEM lane: row of [K;Q], or Dv row
   const bool leader = (kt == 0);
   const uint32_t tlane = x.tmem + (uint32_t(lq * 32) << 16);
-  const int T = p.T, H = p.H;
+  const int T = p.T;
   float* sA = reinterpret_cast<float*>(x.sm + SM_A);
   float* sTf = reinterpret_cast<float*>(x.sm + SM_TF);
-  float* sE = reinterpret_cast<float*>(x.sm + SM_E);
+  float* sAt = reinterpret_cast<float*>(x.sm + SM_AT);
   volatile float* s_part = reinterpret_cast<volatile float*>(x.misc(M_PART));
   RoleSync rs{BAR_SIDE, SIDE_THREADS, M_FLAG_SIDE, leader, 0};
 
@@ -284,104 +396,66 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
   float g_next = 0.f, b_next = 0.f;
   if (kt < NT && kt < T) {
-    const size_t gi = (size_t(b) * T + kt) * H + h;
+    const size_t gi = (size_t(b) * T + kt) * p.H + h;
     g_next = __ldg(p.g + gi);
     b_next = __ldg(p.beta + gi);
   }
+  side_gates<C>(x, kt, 0, T, g_next, b_next, p, b, h, s_part);
+  if (!rs.wait(x, x.bar(B_FULL0), 0)) return;
+  if (leader) {
+    *x.misc(M_KQ_SEEN) = 1;
+    issue_p(x, 0);
+  }
+  int p_issued = 1;  // tiles whose P MMA was issued (leader's view)
+  float mq[32];      // this thread's half row of Mq (lanes 64..127)
 
   for (int c = 0; c < ntiles; ++c) {
-    const int t0 = c * NT;
-    float* G = x.gates(c);
-    // ---- gates of tile c: inclusive in-chunk scan of g, decays
-    if (kt < NT) {
-      float gc = g_next;
-      const float bc = b_next;
-      g_next = 0.f;
-      b_next = 0.f;
-      const int t = t0 + NT + kt;
-      if (t < T) {
-        const size_t gi = (size_t(b) * T + t) * H + h;
-        g_next = __ldg(p.g + gi);
-        b_next = __ldg(p.beta + gi);
-      }
-      constexpr int W = C < 32 ? C : 32;
-      const int ln = kt & 31;
-#pragma unroll
-      for (int off = 1; off < W; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, gc, off, W);
-        if ((ln & (W - 1)) >= off) gc += y;
-      }
-      if constexpr (C == 64) {
-        if (kt == 31) *s_part = gc;
-        named_bar(BAR_SCAN, 64);
-        if (kt >= 32) gc += *s_part;
-      }
-      G[G_GAM2 / 4 + kt] = gc * LOG2E;
-      G[G_B / 4 + kt] = bc;
-    }
-    named_bar(BAR_SIDE, SIDE_THREADS);
-    if (kt < NT) {
-      const int last = (kt / C) * C + C - 1;
-      const float gi = G[G_GAM2 / 4 + kt], gl = G[G_GAM2 / 4 + last];
-      const float Gm = fast_exp2(gi);
-      G[G_GAM / 4 + kt] = Gm;
-      G[G_BG / 4 + kt] = G[G_B / 4 + kt] * Gm;
-      G[G_DF / 4 + kt] = fast_exp2(gl - gi);
-      if (kt == last) G[G_GC / 4 + kt / C] = fast_exp2(gl);
-    }
-    named_bar(BAR_SIDE, SIDE_THREADS);
-    if (leader) mbar_arrive(x.bar((c & 1) ? B_GFULL1 : B_GFULL0));
+    const float* G = x.gates(c);
+    if (!rs.wait(x, x.bar(B_PFULL), c & 1)) return;
 
-    // ---- P = [K; Q] K^T : M=128 (rows of [K;Q]), N=64 (tokens j), K=128 (dk)
-    if (!rs.wait(x, x.bar((c & 1) ? B_FULL1 : B_FULL0), (c >> 1) & 1)) break;
-    if (leader) {
-      *x.misc(M_KQ_SEEN) = c + 1;
-      const uint32_t kq = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
-      const uint32_t id = idesc_bf16(128, 64, 0, 0, 0);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-        mma_ss(x.tmem + TM_P, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(kq + off, 16, 1024), id,
-               kk > 0);
-      }
-      mma_commit(x.bar(B_PFULL));
-    }
-    if (!rs.wait(x, x.bar(B_PFULL), c & 1)) break;
-
-    // ---- masks and decays, rows 0..63 of P: A = strict_tril(beta_i Dec_ij (k_i . k_j))
-    if (row < NT) {
-      const int i = row;
+    // ---- masks and decays of P(c), columns 32 hf ..: rows 0..63 -> A =
+    //      strict_tril(beta_i Dec_ij k_i.k_j) (fp32, for the solve); rows 64..127
+    //      -> Mq = tril(Dec_ij q_i.k_j) (registers)
+    {
+      const int i = row & (NT - 1);
       const int cs = (i / C) * C;
       const float gi = G[G_GAM2 / 4 + i];
-      const float bi = G[G_B / 4 + i];
+      const float bi = (row < NT) ? G[G_B / 4 + i] : 1.f;
+      float P[32];
+      tmem_ld32(tlane + TM_P + 32 * hf, P);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float P[32];
-        tmem_ld32(tlane + TM_P + 32 * half, P);
-        float4* dst = reinterpret_cast<float4*>(sA + i * APAD + 32 * half);
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 gj = ld4(G + G_GAM2 / 4 + 32 * hf + 4 * e4);
+        const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+        float m[4];
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 gj = ld4(G + G_GAM2 / 4 + 32 * half + 4 * e4);
-          const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
-          float m[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 32 * half + 4 * e4 + e;
-            const float v = bi * fast_exp2(gi - gjv[e]) * P[4 * e4 + e];
-            m[e] = (j >= cs && j < i) ? v : 0.f;
-          }
-          dst[e4] = make_float4(m[0], m[1], m[2], m[3]);
+        for (int e = 0; e < 4; ++e) {
+          const int j = 32 * hf + 4 * e4 + e;
+          const float v = bi * fast_exp2(gi - gjv[e]) * P[4 * e4 + e];
+          m[e] = (j >= cs && (row < NT ? j < i : j <= i)) ? v : 0.f;
+          mq[4 * e4 + e] = m[e];
         }
+        if (row < NT)
+          *reinterpret_cast<float4*>(sA + i * APAD + 32 * hf + 4 * e4) =
+              make_float4(m[0], m[1], m[2], m[3]);
       }
     }
     tc_fence_before();
     named_bar(BAR_SIDE, SIDE_THREADS);
+    // P(c) has been read: start P(c+1) now if its tile has landed
+    if (leader && c + 1 < ntiles && p_issued == c + 1 &&
+        mbar_try_wait(x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1)) {
+      tc_fence_after();
+      *x.misc(M_KQ_SEEN) = c + 2;
+      issue_p(x, c + 1);
+      p_issued = c + 2;
+    }
 
     // ---- T = (I + A)^{-1}, blocked in 16 x 16 blocks.
-    //  (1) diagonal blocks: lane r < 64 forms row r of its block's inverse,
+    //  (1) diagonal blocks: thread r < 64 forms row r of its block's inverse,
     //      x (I + A_bb) = e_r, right-looking: x_i is final once every row
     //      below it has been subtracted, then x_i A_i,j leaves each acc_j (j < i);
-    //  (2) with chunk 64, the off-diagonal blocks by distance d = 1..3.
+    //  (2) with chunk 64: At_IK = T_II A_IK, then T_IJ = -sum_K At_IK T_KJ by distance.
     if (kt < NT) {
       const int r = kt, bb = r >> 4, rr = r & 15, base = bb * 16;
       float acc[16];
@@ -414,47 +488,43 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
     }
     named_bar(BAR_SIDE, SIDE_THREADS);
     if constexpr (C == 64) {
-      solve_offdiag<1>(kt, sA, sTf, sE);
-      solve_offdiag<2>(kt, sA, sTf, sE);
-      solve_offdiag<3>(kt, sA, sTf, sE);
+      solve_at_blocks(kt, sA, sTf, sAt);
+      named_bar(BAR_SIDE, SIDE_THREADS);
+      solve_distance<1>(kt, sAt, sTf);
+      named_bar(BAR_SIDE, SIDE_THREADS);
+      solve_distance<2>(kt, sAt, sTf);
+      named_bar(BAR_SIDE, SIDE_THREADS);
+      solve_distance<3>(kt, sAt, sTf);
+      named_bar(BAR_SIDE, SIDE_THREADS);
     }
 
+    // ---- gates of the next tile, while the chain is still on tile c-1 / c
+    if (c + 1 < ntiles) side_gates<C>(x, kt, c + 1, T, g_next, b_next, p, b, h, s_part);
+
     // ---- hand T(c), Mq(c) to the chain once it is done with tile c-1's
-    if (c > 0 && !rs.wait(x, x.bar(B_TMFREE), (c - 1) & 1)) break;
+    if (c > 0 && !rs.wait(x, x.bar(B_TMFREE), (c - 1) & 1)) return;
     if (row < NT) {
-      // T row r (fp32) -> hi/lo bf16, K-major rows
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        store_split8(x.sb + SM_TH, x.sb + SM_TL, row, c8, sTf + row * APAD + 8 * c8);
+      for (int c8 = 0; c8 < 4; ++c8)
+        store_split8(x.sb + SM_TH, x.sb + SM_TL, row, 4 * hf + c8, sTf + row * APAD + 32 * hf + 8 * c8);
     } else {
-      // Mq row i = tril(Dec_ij (q_i . k_j)), from rows 64..127 of P
-      const int i = row - NT;
-      const int cs = (i / C) * C;
-      const float gi = G[G_GAM2 / 4 + i];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float P[32];
-        tmem_ld32(tlane + TM_P + 32 * half, P);
-        float m[32];
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 gj = ld4(G + G_GAM2 / 4 + 32 * half + 4 * e4);
-          const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 32 * half + 4 * e4 + e;
-            const float v = fast_exp2(gi - gjv[e]) * P[4 * e4 + e];
-            m[4 * e4 + e] = (j >= cs && j <= i) ? v : 0.f;
-          }
-        }
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-          store_split8(x.sb + SM_MQH, x.sb + SM_MQL, i, 4 * half + c8, m + 8 * c8);
-      }
+      for (int c8 = 0; c8 < 4; ++c8)
+        store_split8(x.sb + SM_MQH, x.sb + SM_MQL, row - NT, 4 * hf + c8, mq + 8 * c8);
     }
     fence_proxy_async_smem();
     named_bar(BAR_SIDE, SIDE_THREADS);
     if (leader) mbar_arrive(x.bar(B_TMFULL));
+
+    // ---- P(c+1), if it could not be started early
+    if (c + 1 < ntiles) {
+      if (!rs.wait(x, x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1)) return;
+      if (leader && p_issued == c + 1) {
+        *x.misc(M_KQ_SEEN) = c + 2;
+        issue_p(x, c + 1);
+        p_issued = c + 2;
+      }
+    }
   }
 }
 
@@ -476,7 +546,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
 
   // ---- initial state (row dv of S0, or zeros): hi/lo copy, and the fp32 copy
   //      pre-scaled by the decay of the first chunk
-  if (!rs.wait(x, x.bar(B_GFULL0), 0)) return;
+  if (!rs.wait(x, x.bar(gfull_off(0)), gfull_parity(0))) return;
   {
     const float gc0 = x.gates(0)[G_GC / 4];
     const float4* src =
@@ -515,7 +585,6 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         bool ok = true;
         if (s == 0) {
           ok = mbar_wait_bounded(x.bar((c & 1) ? B_FULL1 : B_FULL0), (c >> 1) & 1, WAIT_LIMIT_NS);
-          if (ok && c > 0) ok = mbar_wait_bounded(x.bar(B_OUTFREE), (c - 1) & 1, WAIT_LIMIT_NS);
         }
         if (!ok) x.fail();
         if (ok && !*x.abort_flag) {
@@ -545,7 +614,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       }
       if (!rs.wait(x, x.bar(B_ZQ), sc & 1)) return;
       if (s == 0) {
-        if (!rs.wait(x, x.bar((c & 1) ? B_GFULL1 : B_GFULL0), (c >> 1) & 1)) return;
+        if (!rs.wait(x, x.bar(gfull_off(c)), gfull_parity(c))) return;
         if (!rs.wait(x, x.bar(B_VFULL), c & 1)) return;
         if (leader) *x.misc(M_V_SEEN) = c + 1;
       }
@@ -676,13 +745,15 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           }
         }
         mma_commit(x.bar(B_OU));
-        if (s == NSUB - 1) {
-          mma_commit(x.bar(B_TMFREE));   // T(c), Mq(c) consumed
-          mma_commit(x.bar(B_OUTFULL));  // Y(c), O_intra(c) complete
-        }
+        if (s == NSUB - 1) mma_commit(x.bar(B_TMFREE));  // T(c), Mq(c) consumed
       }
       if (!rs.wait(x, x.bar(B_OU), sc & 1)) return;
       if (leader && s == NSUB - 1 && c + 2 < ntiles) issue_kq(x, tq, tk, c + 2, h, b);  // KQ(c) read
+
+      // ---- o of the whole tile is complete after its last chunk: o[t][dv] =
+      //      Gamma_t Y[dv][t] + O_intra[dv][t], this thread's 32 tokens to HBM
+      //      (loads first; the stores drain while the chain moves on)
+      if (s == NSUB - 1) output_drain(x, p, tlane, b, h, dv, ch, c);
 
       // ---- S_out now sits in TMEM: refresh its hi/lo copy, and pre-scale it by
       //      the next chunk's decay (or store it as S_T after the last chunk)
@@ -692,88 +763,36 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         if (s + 1 < NSUB) {
           gnext = G[G_GC / 4 + s + 1];
         } else if (!last_tile) {
-          if (!rs.wait(x, x.bar(((c + 1) & 1) ? B_GFULL1 : B_GFULL0), ((c + 1) >> 1) & 1)) return;
+          if (!rs.wait(x, x.bar(gfull_off(c + 1)), gfull_parity(c + 1))) return;
           gnext = x.gates(c + 1)[G_GC / 4];
         }
-        // one pass over this thread's 64 columns: both loads, then all stores, one wait
-        float v0[32], v1[32];
-        tmem_ld32x2(tlane + TM_S + 64 * ch, v0, tlane + TM_S + 64 * ch + 32, v1);
-        {
-          uint32_t hi[16], lo[16];
+        // this thread's 64 columns, 32 at a time: load, split, store hi / lo /
+        // pre-scaled fp32 in one waited group (or S_T to HBM after the last chunk)
 #pragma unroll
-          for (int e = 0; e < 16; ++e) split2_bf16(v0[2 * e], v0[2 * e + 1], hi[e], lo[e]);
-          tmem_st16_nowait(tlane + TM_SHI + 32 * ch, hi);
-          tmem_st16_nowait(tlane + TM_SLO + 32 * ch, lo);
-        }
-        {
-          uint32_t hi[16], lo[16];
+        for (int q = 0; q < 2; ++q) {
+          const int col = 64 * ch + 32 * q;
+          float v[32];
+          tmem_ld32(tlane + TM_S + col, v);
+          uint32_t hi[16], lo[16], u[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) split2_bf16(v1[2 * e], v1[2 * e + 1], hi[e], lo[e]);
-          tmem_st16_nowait(tlane + TM_SHI + 32 * ch + 16, hi);
-          tmem_st16_nowait(tlane + TM_SLO + 32 * ch + 16, lo);
-        }
-        if (final_chunk) {
-          float4* dst = reinterpret_cast<float4*>(p.S_T + (size_t(chain) * D + dv) * D + 64 * ch);
+          for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
+          if (final_chunk) {
+            tmem_st16x2(tlane + TM_SHI + col / 2, hi, tlane + TM_SLO + col / 2, lo);
+            float4* dst = reinterpret_cast<float4*>(p.S_T + (size_t(chain) * D + dv) * D + col);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            dst[e] = make_float4(v0[4 * e], v0[4 * e + 1], v0[4 * e + 2], v0[4 * e + 3]);
-            dst[8 + e] = make_float4(v1[4 * e], v1[4 * e + 1], v1[4 * e + 2], v1[4 * e + 3]);
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v[e]);
+            tmem_st_state(tlane + TM_SHI + col / 2, hi, tlane + TM_SLO + col / 2, lo,
+                          tlane + TM_S + col, u);
           }
-        } else {
-          uint32_t u[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v0[e]);
-          tmem_st32_nowait(tlane + TM_S + 64 * ch, u);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v1[e]);
-          tmem_st32_nowait(tlane + TM_S + 64 * ch + 32, u);
         }
-        tmem_wait_st();
       }
       tc_fence_before();
       if (!rs.check(x)) return;
     }
-  }
-}
-
-// ============================================================== output
-// o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] of tile c, straight to HBM
-// (each warp store is 32 consecutive floats of one token row).
-__device__ void output_role(const Ctx& x, const PrefillArgs& p, int b, int h, int ntiles) {
-  const int ot = threadIdx.x - 256;
-  const int lq = (threadIdx.x >> 5) & 3;
-  const int dv = lq * 32 + (threadIdx.x & 31);
-  const bool leader = (ot == 0);
-  const uint32_t tlane = x.tmem + (uint32_t(lq * 32) << 16);
-  const int T = p.T, H = p.H;
-  RoleSync rs{BAR_OUT, OUT_THREADS, M_FLAG_OUT, leader, 0};
-  const size_t tstride = size_t(H) * D;
-  for (int c = 0; c < ntiles; ++c) {
-    if (!rs.wait(x, x.bar(B_OUTFULL), c & 1)) return;
-    const float* G = x.gates(c);
-    const int t0 = c * NT;
-    const int nvalid = min(NT, T - t0);
-    float* orow = p.o + ((size_t(b) * T + t0) * H + h) * D + dv;
-    float o[NT];
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      float y[32], oi[32];
-      tmem_ld32x2(tlane + TM_Y + 32 * q, y, tlane + TM_OI + 32 * q, oi);
-#pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 gm = ld4(G + G_GAM / 4 + 32 * q + 4 * e4);
-        o[32 * q + 4 * e4 + 0] = fmaf(gm.x, y[4 * e4 + 0], oi[4 * e4 + 0]);
-        o[32 * q + 4 * e4 + 1] = fmaf(gm.y, y[4 * e4 + 1], oi[4 * e4 + 1]);
-        o[32 * q + 4 * e4 + 2] = fmaf(gm.z, y[4 * e4 + 2], oi[4 * e4 + 2]);
-        o[32 * q + 4 * e4 + 3] = fmaf(gm.w, y[4 * e4 + 3], oi[4 * e4 + 3]);
-      }
-    }
-    tc_fence_before();
-    named_bar(BAR_OUT, OUT_THREADS);
-    if (leader) mbar_arrive(x.bar(B_OUTFREE));  // Y and O_intra may be overwritten
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-      if (n < nvalid) orow[size_t(n) * tstride] = o[n];
   }
 }
 
@@ -816,10 +835,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   if (warp < 4 || warp >= 12)
     chain_role<C>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
-  else if (warp < 8)
-    kside_role<C>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
   else
-    output_role(x, p, b, h, ntiles);
+    kside_role<C>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
 
   tc_fence_before();
   __syncthreads();

@@ -151,7 +151,9 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
       : "r"(taddr)
       : "memory");
 }
-// Two 16-column loads in flight together, then one wait.
+// Two 16-column loads in flight together, then one wait.  The outputs are
+// early-clobber: the first load writes its registers asynchronously, so none
+// of them may share a register with the second load's address operand.
 __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, float (&a)[16], uint32_t tb,
                                             float (&b)[16]) {
   uint32_t* u = reinterpret_cast<uint32_t*>(a);
@@ -162,11 +164,11 @@ __device__ __forceinline__ void tmem_ld16x2(uint32_t ta, float (&a)[16], uint32_
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
       "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
-        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
-        "=r"(u[14]), "=r"(u[15]), "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]),
-        "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-        "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "=&r"(u[0]), "=&r"(u[1]), "=&r"(u[2]), "=&r"(u[3]), "=&r"(u[4]), "=&r"(u[5]), "=&r"(u[6]),
+        "=&r"(u[7]), "=&r"(u[8]), "=&r"(u[9]), "=&r"(u[10]), "=&r"(u[11]), "=&r"(u[12]), "=&r"(u[13]),
+        "=&r"(u[14]), "=&r"(u[15]), "=&r"(v[0]), "=&r"(v[1]), "=&r"(v[2]), "=&r"(v[3]), "=&r"(v[4]),
+        "=&r"(v[5]), "=&r"(v[6]), "=&r"(v[7]), "=&r"(v[8]), "=&r"(v[9]), "=&r"(v[10]), "=&r"(v[11]),
+        "=&r"(v[12]), "=&r"(v[13]), "=&r"(v[14]), "=&r"(v[15])
       : "r"(ta), "r"(tb)
       : "memory");
 }
@@ -210,31 +212,36 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&u)[32
       "r"(u[29]), "r"(u[30]), "r"(u[31])
       : "memory");
 }
-// 32-column store without a wait: the source registers are read when the
-// instruction issues; a later tcgen05.wait::st (tmem_wait_st) orders the
-// stored data before tensor-core reads or other threads' TMEM accesses.
-__device__ __forceinline__ void tmem_st32_nowait(uint32_t taddr, const uint32_t (&u)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
-      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]),
-      "r"(u[15]), "r"(u[16]), "r"(u[17]), "r"(u[18]), "r"(u[19]), "r"(u[20]), "r"(u[21]),
-      "r"(u[22]), "r"(u[23]), "r"(u[24]), "r"(u[25]), "r"(u[26]), "r"(u[27]), "r"(u[28]),
-      "r"(u[29]), "r"(u[30]), "r"(u[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st16_nowait(uint32_t taddr, const uint32_t (&u)[16]) {
+// One state-epilogue store group: 16 columns of hi, 16 of lo and 32 of fp32,
+// waited on inside the same statement -- a TMEM store may still be reading
+// its source registers until tcgen05.wait::st, so no source register may be
+// reused before the wait.
+__device__ __forceinline__ void tmem_st_state(uint32_t t_hi, const uint32_t (&hi)[16],
+                                              uint32_t t_lo, const uint32_t (&lo)[16],
+                                              uint32_t t_s, const uint32_t (&u)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
-      "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]),
-      "r"(u[15])
+      "{%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%1], "
+      "{%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%2], "
+      "{%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,"
+      "%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64,%65,%66};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(t_hi),
+      "r"(t_lo), "r"(t_s), "r"(hi[0]), "r"(hi[1]), "r"(hi[2]), "r"(hi[3]), "r"(hi[4]),
+      "r"(hi[5]), "r"(hi[6]), "r"(hi[7]), "r"(hi[8]), "r"(hi[9]), "r"(hi[10]), "r"(hi[11]),
+      "r"(hi[12]), "r"(hi[13]), "r"(hi[14]), "r"(hi[15]), "r"(lo[0]), "r"(lo[1]), "r"(lo[2]),
+      "r"(lo[3]), "r"(lo[4]), "r"(lo[5]), "r"(lo[6]), "r"(lo[7]), "r"(lo[8]), "r"(lo[9]),
+      "r"(lo[10]), "r"(lo[11]), "r"(lo[12]), "r"(lo[13]), "r"(lo[14]), "r"(lo[15]), "r"(u[0]),
+      "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
+      "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15]),
+      "r"(u[16]), "r"(u[17]), "r"(u[18]), "r"(u[19]), "r"(u[20]), "r"(u[21]), "r"(u[22]),
+      "r"(u[23]), "r"(u[24]), "r"(u[25]), "r"(u[26]), "r"(u[27]), "r"(u[28]), "r"(u[29]),
+      "r"(u[30]), "r"(u[31])
       : "memory");
 }
-// Two 32-column loads in flight together, then one wait.
+// Two 32-column loads in flight together, then one wait (early-clobber
+// outputs, as for tmem_ld16x2).
 __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, float (&a)[32], uint32_t tb,
                                             float (&b)[32]) {
   uint32_t* u = reinterpret_cast<uint32_t*>(a);
@@ -247,16 +254,16 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, float (&a)[32], uint32_
       "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
       "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
-        "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
-        "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]),
-        "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]), "=r"(u[25]),
-        "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31]),
-        "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
-        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
-        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "=&r"(u[0]), "=&r"(u[1]), "=&r"(u[2]), "=&r"(u[3]), "=&r"(u[4]), "=&r"(u[5]), "=&r"(u[6]),
+        "=&r"(u[7]), "=&r"(u[8]), "=&r"(u[9]), "=&r"(u[10]), "=&r"(u[11]), "=&r"(u[12]), "=&r"(u[13]),
+        "=&r"(u[14]), "=&r"(u[15]), "=&r"(u[16]), "=&r"(u[17]), "=&r"(u[18]), "=&r"(u[19]),
+        "=&r"(u[20]), "=&r"(u[21]), "=&r"(u[22]), "=&r"(u[23]), "=&r"(u[24]), "=&r"(u[25]),
+        "=&r"(u[26]), "=&r"(u[27]), "=&r"(u[28]), "=&r"(u[29]), "=&r"(u[30]), "=&r"(u[31]),
+        "=&r"(v[0]), "=&r"(v[1]), "=&r"(v[2]), "=&r"(v[3]), "=&r"(v[4]), "=&r"(v[5]), "=&r"(v[6]),
+        "=&r"(v[7]), "=&r"(v[8]), "=&r"(v[9]), "=&r"(v[10]), "=&r"(v[11]), "=&r"(v[12]), "=&r"(v[13]),
+        "=&r"(v[14]), "=&r"(v[15]), "=&r"(v[16]), "=&r"(v[17]), "=&r"(v[18]), "=&r"(v[19]),
+        "=&r"(v[20]), "=&r"(v[21]), "=&r"(v[22]), "=&r"(v[23]), "=&r"(v[24]), "=&r"(v[25]),
+        "=&r"(v[26]), "=&r"(v[27]), "=&r"(v[28]), "=&r"(v[29]), "=&r"(v[30]), "=&r"(v[31])
       : "r"(ta), "r"(tb)
       : "memory");
 }

@@ -52,11 +52,20 @@ def to_dev(d):
     return {k: (v.to(DEV) if v is not None else None) for k, v in d.items()}
 
 
+def checked_prefill(q, k, v, g, beta, S0, chunk, **kw):
+    """gdn.prefill with a device status word, which must stay 0 (no bounded
+    device wait gave up)."""
+    gdn = _gdn()
+    status = torch.zeros(1, dtype=torch.int32, device=q.device)
+    out = gdn.prefill(q, k, v, g, beta, S0, chunk=chunk, status=status, **kw)
+    assert gdn.query_status(status) == 0, "a device-side wait timed out"
+    return out
+
+
 def gpu_prefill(d, chunk, S0=True):
     dd = to_dev(d)
-    o, S_T = _gdn().prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
-                            dd["S0"] if S0 else None, chunk=chunk)
-    torch.cuda.synchronize()
+    o, S_T = checked_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
+                             dd["S0"] if S0 else None, chunk)
     return o.cpu().numpy(), S_T.cpu().numpy()
 
 
@@ -106,8 +115,7 @@ def test_prefill_b4_h32_t32768_sampled_chains(chunk):
     recomputes a sample of (b, h) chains one by one."""
     w = inputs.WORKLOADS["prefill_b4_h32_t32768"]
     d = inputs.workload_inputs(w, seed=0, device=DEV)
-    o, S_T = _gdn().prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
-    torch.cuda.synchronize()
+    o, S_T = checked_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk)
     for (b, h) in [(0, 0), (1, 17), (3, 31)]:
         sl = lambda x: x[b:b + 1, :, h:h + 1].cpu()
         ro, rS = oracle.prefill(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["g"]), sl(d["beta"]), None)
@@ -115,6 +123,18 @@ def test_prefill_b4_h32_t32768_sampled_chains(chunk):
         assert_parity(S_T[b, h].cpu().numpy(), rS[0, 0], f"S_T chain ({b},{h})")
     del d, o, S_T
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+@pytest.mark.parametrize("g_mean", [0.0, 2.0])
+def test_long_sequence_few_chains(chunk, g_mean):
+    """2048 tokens on two chains: the chain and side warps drift furthest apart
+    when few CTAs share the GPU, which is where hand-off bugs between tiles show."""
+    d = inputs.prefill_inputs(1, 2048, 2, seed=21, g_mean=g_mean)
+    o, S_T = gpu_prefill(d, chunk, S0=False)
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None)
+    assert_parity(o, ro, f"o g_mean={g_mean}")
+    assert_parity(S_T, rS, f"S_T g_mean={g_mean}")
 
 
 def test_decode_b64_h16_256_steps_sampled_sequences():
@@ -154,7 +174,7 @@ def test_decode_equals_prefill_t1():
 def test_split_carry(chunk):
     d = to_dev(inputs.prefill_inputs(1, 300, 4, seed=11, s0_std=0.05))
     gdn = _gdn()
-    o, S_T = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
+    o, S_T = checked_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk)
     t1 = 130
     cut = lambda x, a, b: x[:, a:b].contiguous()
     o1, S1 = gdn.prefill(cut(d["q"], 0, t1), cut(d["k"], 0, t1), cut(d["v"], 0, t1),
