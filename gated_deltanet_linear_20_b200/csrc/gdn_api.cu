@@ -4,6 +4,7 @@
 // calls except the cached driver entry point of cuTensorMapEncodeTiled.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -36,15 +37,40 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return a0 < b0 + nb && b0 < a0 + na;
 }
 
+// Per-device facts queried once: compute capability and multiprocessor count.
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  std::atomic<int> state{0};  // 0 unknown, 1 known
+  int cc_major = 0, cc_minor = 0, sms = 0;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_device_mutex;
+
+int device_info(const DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return GDN_ERR_LAUNCH;
+  if (dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
+  DeviceInfo& d = g_devices[dev];
+  if (d.state.load(std::memory_order_acquire) == 0) {
+    std::lock_guard<std::mutex> lock(g_device_mutex);
+    if (d.state.load(std::memory_order_relaxed) == 0) {
+      if (cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return GDN_ERR_LAUNCH;
+      d.state.store(1, std::memory_order_release);
+    }
+  }
+  *out = &d;
+  return GDN_OK;
+}
+
 // The current device must be an sm_100 part (the only architecture built).
 int check_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_LAUNCH;
-  int major = 0, minor = 0;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return GDN_ERR_LAUNCH;
-  if (major != 10 || minor != 0) return GDN_ERR_UNSUPPORTED;
+  const DeviceInfo* d = nullptr;
+  const int rc = device_info(&d);
+  if (rc != GDN_OK) return rc;
+  if (d->cc_major != 10 || d->cc_minor != 0) return GDN_ERR_UNSUPPORTED;
   return GDN_OK;
 }
 
@@ -65,29 +91,58 @@ bool encode_act(CUtensorMap* map, const void* base, int B, int T, int H, int box
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-extern "C" {
-
-int gdn_abi_version(void) { return GDN_ABI_VERSION; }
-
-const char* gdn_status_str(int code) {
-  switch (code) {
-    case GDN_OK: return "ok";
-    case GDN_ERR_NULL: return "a required pointer is NULL";
-    case GDN_ERR_ALIGN: return "misaligned pointer (q/k/v/o/S need 16 bytes, g/beta 4 bytes)";
-    case GDN_ERR_SHAPE: return "negative size or problem larger than 2^31-1 elements";
-    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims must be 128, chunk 16 or 64, device sm_100)";
-    case GDN_ERR_ALIAS: return "output overlaps an input";
-    case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
-    case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
-    default: return "unknown status code";
-  }
+int num_sms(int* sms) {
+  const DeviceInfo* d = nullptr;
+  const int rc = device_info(&d);
+  if (rc != GDN_OK) return rc;
+  *sms = d->sms;
+  return GDN_OK;
 }
 
-int gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
-                int chunk, int* status, void* stream) {
+// Segmented schedule for B*H chains of T tokens on `sms` multiprocessors (one
+// prefill CTA per SM).  A chain cut into n segments of L tiles costs 2n - 1 CTAs
+// in the first launch, which must fit in one wave; its time is modelled, in
+// units of one tile of the single-pass kernel (about 8 us), as
+//     single pass:  tiles
+//     n segments :  1.2 L + 0.4 (n - 1) + 0.6
+// (a segment tile also pays its share of the second launch; each chained
+// segment end costs one 128 x 128 x 128 product there; plus one launch), and
+// the cheapest n is taken.
+struct SegPlan {
+  int nseg, seg_tiles;
+  size_t ws_bytes, off_R, off_F;
+};
+SegPlan plan_segments(int B, int T, int H, int sms) {
+  const long long chains = (long long)B * H;
+  const int tiles = (T + 63) / 64;
+  SegPlan best{1, tiles, 0, 0, 0};
+  if (chains <= 0 || tiles < 2 || sms <= 0) return best;
+  const long long nmax = (sms / chains + 1) / 2;
+  double best_cost = tiles;
+  for (long long n = 2; n <= nmax && n <= tiles; ++n) {
+    const int L = int((tiles + n - 1) / n);
+    const int nn = (tiles + L - 1) / L;  // segments actually used
+    const double cost = 1.2 * L + 0.4 * (nn - 1) + 0.6;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best.nseg = nn;
+      best.seg_tiles = L;
+    }
+  }
+  if (best.nseg > 1) {
+    const size_t f_bytes = size_t(chains) * T * kHeadDim * 4;
+    const size_t mats = size_t(chains) * best.nseg * kHeadDim * kHeadDim * 4;
+    best.off_R = (f_bytes + 255) & ~size_t(255);
+    best.off_F = best.off_R + mats;
+    best.ws_bytes = best.off_F + mats;
+  }
+  return best;
+}
+
+int prefill_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                 const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
+                 int chunk, void* ws, size_t ws_bytes, bool allow_segments, int* status,
+                 void* stream) {
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
   const long long chains = (long long)B * H;
@@ -111,7 +166,26 @@ int gdn_prefill(const void* q, const void* k, const void* v, const float* g, con
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
 
-  gdn::PrefillArgs a{g, beta, S0, o, S_T, B, T, H, status};
+  gdn::PrefillArgs a{g, beta, S0, o, S_T, B, T, H, status, 1, (T + 63) / 64, nullptr, nullptr, nullptr};
+  if (allow_segments && T > 0) {
+    int sms = 0;
+    if (num_sms(&sms) != GDN_OK) return GDN_ERR_LAUNCH;
+    const SegPlan plan = plan_segments(B, T, H, sms);
+    if (plan.nseg > 1) {
+      if (!ws || !aligned(ws, 256) || ws_bytes < plan.ws_bytes) return GDN_ERR_WORKSPACE;
+      const void* args[] = {q, k, v, g, beta, S0, o, S_T};
+      const size_t sizes[] = {act_bf16, act_bf16, act_bf16, gate_bytes, gate_bytes, state_bytes,
+                              act_f32, state_bytes};
+      for (int i = 0; i < 8; ++i)
+        if (overlaps(ws, plan.ws_bytes, args[i], sizes[i])) return GDN_ERR_ALIAS;
+      uint8_t* base = static_cast<uint8_t*>(ws);
+      a.nseg = plan.nseg;
+      a.seg_tiles = plan.seg_tiles;
+      a.ws_f = reinterpret_cast<float*>(base);
+      a.ws_R = reinterpret_cast<float*>(base + plan.off_R);
+      a.ws_F = reinterpret_cast<float*>(base + plan.off_F);
+    }
+  }
   CUtensorMap tq{}, tk{}, tv{};
   if (T > 0) {
     const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -120,9 +194,82 @@ int gdn_prefill(const void* q, const void* k, const void* v, const float* g, con
         !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2))
       return GDN_ERR_LAUNCH;
   }
-  return gdn::launch_prefill(tq, tk, tv, a, chunk, static_cast<cudaStream_t>(stream)) == 0
-             ? GDN_OK
-             : GDN_ERR_LAUNCH;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (gdn::launch_prefill(tq, tk, tv, a, chunk, st) != 0) return GDN_ERR_LAUNCH;
+  if (a.nseg > 1 && gdn::launch_segment_fix(a, st) != 0) return GDN_ERR_LAUNCH;
+  return GDN_OK;
+}
+
+}  // namespace
+
+namespace gdn {
+bool ensure_smem_attr(const void* func, int slot, int bytes) {
+  static std::atomic<uint64_t> done[8];  // bit d: device d, per kernel slot
+  int dev = 0;
+  if (slot < 0 || slot >= 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return false;
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done[slot].load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done[slot].fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
+}  // namespace gdn
+
+extern "C" {
+
+int gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+const char* gdn_status_str(int code) {
+  switch (code) {
+    case GDN_OK: return "ok";
+    case GDN_ERR_NULL: return "a required pointer is NULL";
+    case GDN_ERR_ALIGN: return "misaligned pointer (q/k/v/o/S need 16 bytes, g/beta 4 bytes)";
+    case GDN_ERR_SHAPE: return "negative size or problem larger than 2^31-1 elements";
+    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims must be 128, chunk 16 or 64, device sm_100)";
+    case GDN_ERR_ALIAS: return "output overlaps an input";
+    case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
+    case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+    case GDN_ERR_WORKSPACE: return "workspace NULL, not 256-byte aligned, or smaller than gdn_prefill_workspace_bytes";
+    default: return "unknown status code";
+  }
+}
+
+int gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
+                int chunk, int* status, void* stream) {
+  return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, nullptr, 0, false,
+                      status, stream);
+}
+
+size_t gdn_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk) {
+  if (B < 0 || T < 0 || H < 0 || Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64))
+    return 0;
+  const long long chains = (long long)B * H;
+  if (chains == 0 || chains * T * kHeadDim > 0x7fffffffLL) return 0;
+  int sms = 0;
+  if (num_sms(&sms) != GDN_OK) return 0;
+  return plan_segments(B, T, H, sms).ws_bytes;
+}
+
+int gdn_prefill_schedule(int B, int T, int H, int num_sms, int* nseg, int* seg_tiles,
+                         size_t* ws_bytes) {
+  if (!nseg || !seg_tiles || !ws_bytes) return GDN_ERR_NULL;
+  if (B < 0 || T < 0 || H < 0 || num_sms < 0) return GDN_ERR_SHAPE;
+  const SegPlan plan = plan_segments(B, T, H, num_sms);
+  *nseg = plan.nseg;
+  *seg_tiles = plan.seg_tiles;
+  *ws_bytes = plan.ws_bytes;
+  return GDN_OK;
+}
+
+int gdn_prefill_ws(const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, const float* S0, float* o, float* S_T, int B, int T, int H,
+                   int Dk, int Dv, int chunk, void* workspace, size_t workspace_bytes,
+                   int* status, void* stream) {
+  return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, workspace,
+                      workspace_bytes, true, status, stream);
 }
 
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,

@@ -17,6 +17,17 @@ struct PrefillArgs {
   float* S_T;
   int B, T, H;
   int* status;      // may be null
+  // Segmented schedule.  nseg == 1: one CTA walks each chain from S0 to S_T.
+  // nseg > 1: the tiles of a chain are cut into nseg segments of seg_tiles
+  // tiles (the last may be shorter); the first pass runs, per segment k, an
+  // "R" CTA (start from S0 for k = 0, else from zero; writes o and the end
+  // state R_k) and, for k >= 1, an "F" CTA (start from the identity with
+  // v = 0; writes f_t = F q_t like o and the transfer matrix F_k); the second
+  // pass chains S_k+1 = S_k F_k + R_k and adds S_k f_t to o.
+  int nseg, seg_tiles;
+  float* ws_f;      // f_t of the F CTAs, laid out like o            [B][T][H][128]
+  float* ws_R;      // end state of each R CTA                         [B*H][nseg][128][128]
+  float* ws_F;      // transfer matrix of each F CTA (slot 0 unused)   [B*H][nseg][128][128]
 };
 
 struct DecodeArgs {
@@ -30,9 +41,15 @@ struct DecodeArgs {
   int B, H;
 };
 
+// Sets the dynamic shared-memory limit of `func` to `bytes` once per device
+// (slot: a small per-kernel index); returns false if the attribute call failed.
+bool ensure_smem_attr(const void* func, int slot, int bytes);
+
 // Both return 0 on success, -1 when the launch failed.
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const PrefillArgs& a, int chunk, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
+// Second pass of the segmented schedule (a.nseg > 1).
+int launch_segment_fix(const PrefillArgs& a, cudaStream_t stream);
 
 }  // namespace gdn

@@ -118,27 +118,6 @@ constexpr uint32_t V_TX_BYTES = 16384;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr float LOG2E = 1.4426950408889634f;
 
-// Byte offset of 16-byte chunk `c` (8 bf16 along K) of row `r` in a K-major
-// SW128 tile whose rows are 128 bytes and whose 8-row groups are 1024 B apart.
-__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
-  return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + (((c ^ r) & 7) << 4));
-}
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
-                                             uint32_t d) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
-               "r"(d)
-               : "memory");
-}
-// Splits 8 floats into hi/lo bf16 and stores them as chunk `c` of row `r` in two tiles.
-__device__ __forceinline__ void store_split8(uint32_t hi_tile, uint32_t lo_tile, int r, int c,
-                                             const float* x) {
-  uint32_t h[4], l[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) split2_bf16(x[2 * e], x[2 * e + 1], h[e], l[e]);
-  const uint32_t off = sw128_off(r, c);
-  st_shared_v4(hi_tile + off, h[0], h[1], h[2], h[3]);
-  st_shared_v4(lo_tile + off, l[0], l[1], l[2], l[3]);
-}
 // Splits 32 consecutive state values (columns 32q..32q+31 of this lane's row)
 // into bf16 hi/lo pairs and stores them to SHI / SLO.
 __device__ __forceinline__ void store_state_split32(uint32_t tlane, int q, const float (&v)[32]) {
@@ -156,6 +135,12 @@ struct Ctx {
   uint32_t tmem;      // TMEM base (lane 0, column 0)
   int* status;
   volatile int* abort_flag;
+  int tb;              // first tile (of the chain) this CTA walks
+  bool vzero;          // v taken as zero (transfer-matrix CTA of the segmented schedule)
+  bool s0_identity;    // start from the identity instead of s0src / zeros
+  const float* s0src;  // start state of this chain [128][128], or null
+  float* odst;         // destination of o-like outputs, laid out like o
+  float* sdst;         // destination of the end state [128][128]
   __device__ __forceinline__ uint32_t bar(uint32_t off) const { return sb + SM_BAR + off; }
   __device__ __forceinline__ float* gates(int c) const {
     return reinterpret_cast<float*>(sm + SM_GATES + (c % GATE_BUFS) * GATE_BYTES);
@@ -208,16 +193,17 @@ __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, co
   const uint32_t kq = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
   const uint32_t bar = x.bar((c & 1) ? B_FULL1 : B_FULL0);
   mbar_arrive_expect_tx(bar, KQ_TX_BYTES);
-  tma_load_4d(kq + 0, tk, bar, 0, h, c * NT, b);
-  tma_load_4d(kq + 8192, tq, bar, 0, h, c * NT, b);
-  tma_load_4d(kq + 16384, tk, bar, 64, h, c * NT, b);
-  tma_load_4d(kq + 24576, tq, bar, 64, h, c * NT, b);
+  const int t0 = (x.tb + c) * NT;
+  tma_load_4d(kq + 0, tk, bar, 0, h, t0, b);
+  tma_load_4d(kq + 8192, tq, bar, 0, h, t0, b);
+  tma_load_4d(kq + 16384, tk, bar, 64, h, t0, b);
+  tma_load_4d(kq + 24576, tq, bar, 64, h, t0, b);
   *x.misc(M_KQ_ISSUED) = c + 1;
 }
 __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b) {
   const uint32_t bar = x.bar(B_VFULL);
   mbar_arrive_expect_tx(bar, V_TX_BYTES);
-  tma_load_4d(x.sb + SM_V, tv, bar, 0, h, c * NT, b);
+  tma_load_4d(x.sb + SM_V, tv, bar, 0, h, (x.tb + c) * NT, b);
   *x.misc(M_V_ISSUED) = c + 1;
 }
 
@@ -298,7 +284,7 @@ __device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, f
     const float bc = b_next;
     g_next = 0.f;
     b_next = 0.f;
-    const int t = (c + 1) * NT + kt;
+    const int t = (x.tb + c + 1) * NT + kt;
     if (t < T) {
       const size_t gi = (size_t(b) * T + t) * H + h;
       g_next = __ldg(p.g + gi);
@@ -351,9 +337,9 @@ __device__ __forceinline__ void issue_p(const Ctx& x, int c) {
 __device__ __forceinline__ void output_drain(const Ctx& x, const PrefillArgs& p, uint32_t tlane,
                                              int b, int h, int dv, int hf, int c) {
   const float* G = x.gates(c);
-  const int t0 = c * NT + 32 * hf;
+  const int t0 = (x.tb + c) * NT + 32 * hf;
   const int nvalid = min(32, p.T - t0);
-  float* orow = p.o + ((size_t(b) * p.T + t0) * p.H + h) * D + dv;
+  float* orow = x.odst + ((size_t(b) * p.T + t0) * p.H + h) * D + dv;
   const size_t tstride = size_t(p.H) * D;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
@@ -392,11 +378,11 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   if (leader) {
     issue_kq(x, tq, tk, 0, h, b);
     if (ntiles > 1) issue_kq(x, tq, tk, 1, h, b);
-    issue_v(x, tv, 0, h, b);
+    if (!x.vzero) issue_v(x, tv, 0, h, b);
   }
   float g_next = 0.f, b_next = 0.f;
-  if (kt < NT && kt < T) {
-    const size_t gi = (size_t(b) * T + kt) * p.H + h;
+  if (kt < NT && x.tb * NT + kt < T) {
+    const size_t gi = (size_t(b) * T + x.tb * NT + kt) * p.H + h;
     g_next = __ldg(p.g + gi);
     b_next = __ldg(p.beta + gi);
   }
@@ -549,8 +535,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   if (!rs.wait(x, x.bar(gfull_off(0)), gfull_parity(0))) return;
   {
     const float gc0 = x.gates(0)[G_GC / 4];
-    const float4* src =
-        p.S0 ? reinterpret_cast<const float4*>(p.S0 + (size_t(chain) * D + dv) * D) : nullptr;
+    const float4* src = x.s0src ? reinterpret_cast<const float4*>(x.s0src + size_t(dv) * D) : nullptr;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int qq = 2 * ch + q;  // 32-column group
@@ -562,6 +547,10 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         v[4 * e + 1] = a.y;
         v[4 * e + 2] = a.z;
         v[4 * e + 3] = a.w;
+      }
+      if (x.s0_identity) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = (32 * qq + e == dv) ? 1.f : 0.f;
       }
       store_state_split32(tlane, qq, v);
       uint32_t u[32];
@@ -615,8 +604,10 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       if (!rs.wait(x, x.bar(B_ZQ), sc & 1)) return;
       if (s == 0) {
         if (!rs.wait(x, x.bar(gfull_off(c)), gfull_parity(c))) return;
-        if (!rs.wait(x, x.bar(B_VFULL), c & 1)) return;
-        if (leader) *x.misc(M_V_SEEN) = c + 1;
+        if (!x.vzero) {
+          if (!rs.wait(x, x.bar(B_VFULL), c & 1)) return;
+          if (leader) *x.misc(M_V_SEEN) = c + 1;
+        }
       }
 
       // ---- X^T[dv][n] = beta_n V[n][dv] - beta_n Gamma_n Z[dv][n]  (hi/lo -> SMEM)
@@ -646,7 +637,8 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int n = n0 + 4 * e4 + e;
-            xv[4 * e4 + e] = fmaf(bv[e], __bfloat162float(V[n * D + dv]), -gv[e] * z[4 * e4 + e]);
+            const float vn = x.vzero ? 0.f : __bfloat162float(V[n * D + dv]);
+            xv[4 * e4 + e] = fmaf(bv[e], vn, -gv[e] * z[4 * e4 + e]);
           }
         }
 #pragma unroll
@@ -655,7 +647,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar(BAR_CHAIN, CHAIN_THREADS);
-      if (leader && s == NSUB - 1 && !last_tile) issue_v(x, tv, c + 1, h, b);  // V(c) fully read
+      if (leader && s == NSUB - 1 && !last_tile && !x.vzero) issue_v(x, tv, c + 1, h, b);  // V(c) read
 
       // ---- Dl^T = X^T T^T : M=128 (dv), N=C (i), K=C (n); 3 hi/lo products
       if (leader) {
@@ -778,7 +770,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
           if (final_chunk) {
             tmem_st16x2(tlane + TM_SHI + col / 2, hi, tlane + TM_SLO + col / 2, lo);
-            float4* dst = reinterpret_cast<float4*>(p.S_T + (size_t(chain) * D + dv) * D + col);
+            float4* dst = reinterpret_cast<float4*>(x.sdst + size_t(dv) * D + col);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
@@ -806,16 +798,39 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                            ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
-  const int chain = blockIdx.x;
+  const int total_tiles = (p.T + NT - 1) / NT;
+  // CTA -> (chain, segment, kind); see PrefillArgs
+  int chain = blockIdx.x, seg = 0;
+  bool frun = false;
+  if (p.nseg > 1) {
+    const int per = 2 * p.nseg - 1;
+    chain = blockIdx.x / per;
+    const int j = blockIdx.x - chain * per;
+    frun = j >= p.nseg;
+    seg = frun ? j - p.nseg + 1 : j;
+  }
   const int b = chain / p.H;
   const int h = chain - b * p.H;
-  const int ntiles = (p.T + NT - 1) / NT;
+  const size_t cstate = size_t(chain) * D * D;
 
   Ctx x;
   x.sm = sm;
   x.sb = smem_u32(sm);
   x.status = p.status;
   x.abort_flag = reinterpret_cast<volatile int*>(sm + SM_MISC + M_ABORT);
+  x.tb = 0;
+  x.vzero = frun;
+  x.s0_identity = frun;
+  x.s0src = (seg == 0 && p.S0) ? p.S0 + cstate : nullptr;
+  x.odst = frun ? p.ws_f : p.o;
+  int ntiles = total_tiles;
+  if (p.nseg > 1) {
+    x.tb = seg * p.seg_tiles;
+    ntiles = min(p.seg_tiles, total_tiles - x.tb);
+    x.sdst = (frun ? p.ws_F : p.ws_R) + (size_t(chain) * p.nseg + seg) * D * D;
+  } else {
+    x.sdst = p.S_T + cstate;
+  }
   if (tid == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
@@ -877,17 +892,13 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   }
   const uint32_t smem = SMEM_USED + 1024;
-  cudaError_t err;
+  const int ctas = a.nseg > 1 ? chains * (2 * a.nseg - 1) : chains;
   if (chunk == 64) {
-    err = cudaFuncSetAttribute(prefill_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(smem));
-    if (err != cudaSuccess) return -1;
-    prefill_kernel<64><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, a);
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<64>), 0, int(smem))) return -1;
+    prefill_kernel<64><<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, a);
   } else {
-    err = cudaFuncSetAttribute(prefill_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               int(smem));
-    if (err != cudaSuccess) return -1;
-    prefill_kernel<16><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, a);
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<16>), 1, int(smem))) return -1;
+    prefill_kernel<16><<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, a);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

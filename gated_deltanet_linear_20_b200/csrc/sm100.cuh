@@ -372,5 +372,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 a, __nv_bfloat16 b
   return uint32_t(__bfloat16_as_ushort(a)) | (uint32_t(__bfloat16_as_ushort(b)) << 16);
 }
 
+// ---------------------------------------------------------------- SW128 tiles in shared memory
+// Byte offset of 16-byte chunk `c` (8 bf16) of row `r` in a 128-byte-swizzled
+// tile whose rows are 128 bytes and whose 8-row groups are 1024 B apart (the
+// layout TMA writes with SWIZZLE_128B; rows run along M/N for a K-major operand,
+// along K for an MN-major one).
+__device__ __forceinline__ uint32_t sw128_off(int r, int c) {
+  return uint32_t((r >> 3) * 1024 + (r & 7) * 128 + (((c ^ r) & 7) << 4));
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+// Splits 8 floats into hi/lo bf16 and stores them as chunk `c` of row `r` in two tiles.
+__device__ __forceinline__ void store_split8(uint32_t hi_tile, uint32_t lo_tile, int r, int c,
+                                             const float* x) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) split2_bf16(x[2 * e], x[2 * e + 1], h[e], l[e]);
+  const uint32_t off = sw128_off(r, c);
+  st_shared_v4(hi_tile + off, h[0], h[1], h[2], h[3]);
+  st_shared_v4(lo_tile + off, l[0], l[1], l[2], l[3]);
+}
 }  // namespace sm100
 }  // namespace gdn

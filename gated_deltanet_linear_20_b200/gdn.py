@@ -29,12 +29,18 @@ _lib.gdn_status_str.argtypes = [_ci]
 _lib.gdn_status_str.restype = ctypes.c_char_p
 _lib.gdn_prefill.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, _vp]
 _lib.gdn_prefill.restype = _ci
+_lib.gdn_prefill_workspace_bytes.argtypes = [_ci] * 6
+_lib.gdn_prefill_workspace_bytes.restype = ctypes.c_size_t
+_lib.gdn_prefill_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, ctypes.c_size_t, _vp, _vp]
+_lib.gdn_prefill_ws.restype = _ci
+_lib.gdn_prefill_schedule.argtypes = [_ci] * 4 + [_vp, _vp, _vp]
+_lib.gdn_prefill_schedule.restype = _ci
 _lib.gdn_decode_step.argtypes = [_vp] * 7 + [_ci] * 4 + [_vp, _vp]
 _lib.gdn_decode_step.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
-ABI_VERSION = 1
+ABI_VERSION = 2
 if _lib.gdn_abi_version() != ABI_VERSION:
     raise ImportError(f"libgdn_b200.so ABI {_lib.gdn_abi_version()} != binding ABI {ABI_VERSION}")
 
@@ -47,6 +53,7 @@ GDN_ERR_UNSUPPORTED = -4
 GDN_ERR_ALIAS = -5
 GDN_ERR_LAUNCH = -6
 GDN_ERR_DEVICE_TIMEOUT = -7
+GDN_ERR_WORKSPACE = -8
 
 
 class GDNError(RuntimeError):
@@ -84,15 +91,36 @@ def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple, device)
         raise ValueError(f"{name} must be contiguous")
 
 
+def workspace_bytes(B: int, T: int, H: int, chunk: int = 64, Dk: int = 128, Dv: int = 128) -> int:
+    """Bytes of workspace gdn_prefill_ws needs on the current device (0: single pass)."""
+    return int(_lib.gdn_prefill_workspace_bytes(B, T, H, Dk, Dv, int(chunk)))
+
+
+def schedule(B: int, T: int, H: int, num_sms: int) -> Tuple[int, int, int]:
+    """(segments per chain, tiles per segment, workspace bytes) that gdn_prefill_ws
+    picks on a device with ``num_sms`` multiprocessors."""
+    n, L, ws = ctypes.c_int(), ctypes.c_int(), ctypes.c_size_t()
+    rc = _lib.gdn_prefill_schedule(B, T, H, num_sms, ctypes.byref(n), ctypes.byref(L),
+                                   ctypes.byref(ws))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_prefill_schedule")
+    return n.value, L.value, ws.value
+
+
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
             beta: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64, *,
             o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
-            status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+            status: Optional[torch.Tensor] = None, segmented: bool = True,
+            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Chunked prefill: returns (o [B,T,H,Dv] fp32, S_T [B,H,Dv,Dk] fp32).
 
     q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g, beta [B,T,H] fp32; S0 [B,H,Dv,Dk]
     fp32 or None (zeros); chunk 16 or 64.  Launches on the current stream.
-    ``o`` / ``S_T`` may be given preallocated (``S_T`` may be ``S0``)."""
+    ``o`` / ``S_T`` may be given preallocated (``S_T`` may be ``S0``).
+    ``segmented`` calls gdn_prefill_ws, which cuts chains into segments walked
+    in parallel when they are too few to fill the GPU; its workspace is
+    ``workspace`` (a uint8 CUDA tensor) or a fresh torch allocation.  With
+    ``segmented=False`` it calls gdn_prefill (one pass per chain)."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape
@@ -115,11 +143,27 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     _check(S_T, "S_T", torch.float32, (B, H, Dv, Dk), dev)
     if status is not None:
         _check(status, "status", torch.int32, (1,), dev)
-    rc = _lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                          _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(status),
-                          _stream_handle(dev))
+    if not segmented:
+        rc = _lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                              _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(status),
+                              _stream_handle(dev))
+        if rc != GDN_OK:
+            raise GDNError(rc, "gdn_prefill")
+        return o, S_T
+    if workspace is None:
+        with torch.cuda.device(dev):
+            need = workspace_bytes(B, T, H, chunk, Dk, Dv)
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is not None:
+        if workspace.dtype != torch.uint8 or workspace.device != dev or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous uint8 tensor on the inputs' device")
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    rc = _lib.gdn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                             _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(workspace),
+                             ctypes.c_size_t(ws_bytes), _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
-        raise GDNError(rc, "gdn_prefill")
+        raise GDNError(rc, "gdn_prefill_ws")
     return o, S_T
 
 
@@ -161,6 +205,10 @@ def raw_prefill(*args) -> int:
     """Direct call of the C entry point with raw integers/pointers (tests use it
     to exercise argument validation without any tensor)."""
     return int(_lib.gdn_prefill(*args))
+
+
+def raw_prefill_ws(*args) -> int:
+    return int(_lib.gdn_prefill_ws(*args))
 
 
 def raw_decode_step(*args) -> int:

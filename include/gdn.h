@@ -42,6 +42,8 @@
  *                          current device is not compute capability 10.0
  *     GDN_ERR_ALIAS        o overlaps an input or the state
  *     GDN_ERR_LAUNCH       the CUDA launch (or a CUDA runtime query) failed
+ *     GDN_ERR_WORKSPACE    gdn_prefill_ws: workspace NULL, misaligned (256 B) or
+ *                          smaller than gdn_prefill_workspace_bytes asked for
  * Device-side waits are bounded: if one gives up, the kernel writes
  * GDN_ERR_DEVICE_TIMEOUT to *status (when status is non-NULL), releases its
  * tensor memory and returns; read it with gdn_query_status.  The kernels never
@@ -50,11 +52,13 @@
 #ifndef GDN_B200_H_
 #define GDN_B200_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 1
+#define GDN_ABI_VERSION 2
 
 enum gdn_status_code {
   GDN_OK = 0,
@@ -64,7 +68,8 @@ enum gdn_status_code {
   GDN_ERR_UNSUPPORTED = -4,
   GDN_ERR_ALIAS = -5,
   GDN_ERR_LAUNCH = -6,
-  GDN_ERR_DEVICE_TIMEOUT = -7
+  GDN_ERR_DEVICE_TIMEOUT = -7,
+  GDN_ERR_WORKSPACE = -8
 };
 
 /* Returns GDN_ABI_VERSION of the built library; callers compare it with the
@@ -92,6 +97,44 @@ const char* gdn_status_str(int code);
 int gdn_prefill(const void* q, const void* k, const void* v, const float* g, const float* beta,
                 const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
                 int chunk, int* status, void* stream);
+
+/* Workspace, in bytes, that gdn_prefill_ws needs for this problem on the
+ * current device (the schedule depends on its multiprocessor count), or 0 when
+ * it would run the single-pass schedule of gdn_prefill.  Invalid arguments
+ * give 0 too; gdn_prefill_ws then reports them. */
+size_t gdn_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk);
+
+/* The schedule gdn_prefill_ws picks for B*H chains of T tokens on a device
+ * with num_sms multiprocessors (no device is touched): *nseg segments per chain
+ * (1: the single pass of gdn_prefill) of *seg_tiles 64-token tiles each (the
+ * last may be shorter), needing *ws_bytes of workspace.  Returns GDN_OK, or
+ * GDN_ERR_SHAPE for negative sizes, GDN_ERR_NULL for a NULL output pointer. */
+int gdn_prefill_schedule(int B, int T, int H, int num_sms, int* nseg, int* seg_tiles,
+                         size_t* ws_bytes);
+
+/* gdn_prefill with a caller-provided device workspace, which lets chains that
+ * are too few to fill the GPU be cut into segments walked in parallel.  The
+ * pages have no such schedule; it follows from the recurrence itself: over a
+ * stretch of tokens the state is affine in the state the stretch starts from,
+ *     S_t = S_start F_t + R_t,   o_t = S_start (F_t q_t) + o_t^R,
+ * with F_t the ordered product of the factors alpha_s (I - beta_s k_s k_s^T)
+ * and R_t, o_t^R the state and output from a zero start.  A first launch
+ * walks every segment from zero (and, for each segment after the first, from
+ * the identity with v = 0, which yields F and F q_t); a second launch chains
+ * the segment-end states and adds S_start F_t q_t to o.  The result is the
+ * same recurrence up to rounding.
+ *   workspace       : device memory of at least gdn_prefill_workspace_bytes
+ *                     (same sizes, same current device), 256-byte aligned,
+ *                     overlapping no argument; may be NULL when that is 0.
+ *                     Its contents on entry do not matter and are left
+ *                     unspecified; two calls in flight must not share it.
+ *   workspace_bytes : its size
+ * Every other argument, and the results, as for gdn_prefill.  Returns GDN_OK,
+ * GDN_ERR_WORKSPACE, or another negative code as for gdn_prefill. */
+int gdn_prefill_ws(const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, const float* S0, float* o, float* S_T, int B, int T, int H,
+                   int Dk, int Dv, int chunk, void* workspace, size_t workspace_bytes,
+                   int* status, void* stream);
 
 /* One decode step for B sequences (the recurrence above with T = 1), the state
  * read and written in place (the Megakernel decode of the Lucebox contribution

@@ -30,7 +30,8 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("gdn_prefill", "gdn_decode_step", "gdn_abi_version", "gdn_status_str",
+    for n in ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_workspace_bytes",
+              "gdn_prefill_schedule", "gdn_decode_step", "gdn_abi_version", "gdn_status_str",
               "gdn_query_status"):
         assert n in names
 
@@ -46,8 +47,8 @@ def test_library_exports_every_declared_symbol(gdn):
 
 
 def test_abi_version_and_status_strings(gdn):
-    assert gdn.abi_version() == 1
-    for code in range(-7, 1):
+    assert gdn.abi_version() == 2
+    for code in range(-8, 1):
         s = gdn.status_str(code)
         assert s and s != "unknown status code"
     assert gdn.status_str(12345) == "unknown status code"
@@ -82,6 +83,68 @@ def test_prefill_rejects_bad_arguments(gdn, over, code):
 def test_prefill_empty_batch_is_a_noop(gdn):
     assert gdn.raw_prefill(*prefill_args(B=0, q=None, k=None, o=None, S_T=None)) == 0
     assert gdn.raw_prefill(*prefill_args(H=0)) == 0
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(B=-1), -3), (dict(Dk=64), -4), (dict(chunk=32), -4), (dict(q=None), -1),
+    (dict(q=P + 8), -2), (dict(o=P + 0x10000000 + 0x100), -5),
+], ids=lambda x: str(x))
+def test_prefill_ws_rejects_bad_arguments_like_prefill(gdn, over, code):
+    a = prefill_args(**over)
+    assert gdn.raw_prefill_ws(*(a[:14] + [None, 0] + a[14:])) == code
+
+
+def test_prefill_ws_empty_batch_is_a_noop(gdn):
+    a = prefill_args(B=0, q=None, k=None, o=None, S_T=None)
+    assert gdn.raw_prefill_ws(*(a[:14] + [None, 0] + a[14:])) == 0
+
+
+def test_workspace_query_is_zero_without_a_device_or_for_bad_sizes(gdn):
+    import torch
+    assert gdn.workspace_bytes(1, 512, 16, chunk=32) == 0
+    assert gdn.workspace_bytes(-1, 512, 16) == 0
+    if not torch.cuda.is_available():
+        assert gdn.workspace_bytes(1, 512, 16) == 0
+
+
+def plan_cost(tiles, n, L):
+    # the time model documented with the planner (units: one single-pass tile)
+    return tiles if n == 1 else 1.2 * L + 0.4 * (n - 1) + 0.6
+
+
+@pytest.mark.parametrize("B,T,H,expect", [
+    (1, 64, 2, (1, 1)),           # one tile: nothing to cut
+    (1, 512, 16, (4, 2)),         # 16 chains x 8 tiles: 4 segments of 2 tiles
+    (1, 4096, 16, (5, 13)),       # 16 chains x 64 tiles: 2*5-1 = 9 CTAs per chain
+    (4, 32768, 32, (1, 512)),     # 128 chains already fill the GPU
+    (1, 100, 16, (1, 2)),         # 2 tiles: segmenting does not pay
+])
+def test_schedule_of_the_benchmark_shapes(gdn, B, T, H, expect):
+    n, L, ws = gdn.schedule(B, T, H, 148)
+    assert (n, L) == expect
+    tiles = (T + 63) // 64
+    if n == 1:
+        assert ws == 0 and L == tiles
+    else:
+        assert (n - 1) * L < tiles <= n * L               # every segment is non-empty
+        assert B * H * (2 * n - 1) <= 148                 # first launch fits in one wave
+        f_bytes = B * T * H * 128 * 4
+        assert ws == ((f_bytes + 255) // 256) * 256 + 2 * B * H * n * 128 * 128 * 4
+        # the planner took the cheapest admissible segment count
+        nmax = (148 // (B * H) + 1) // 2
+        costs = []
+        for m in range(1, min(nmax, tiles) + 1):
+            Lm = -(-tiles // m)
+            mm = -(-tiles // Lm)
+            costs.append(plan_cost(tiles, mm, Lm))
+        assert abs(plan_cost(tiles, n, L) - min(costs)) < 1e-9
+
+
+def test_schedule_rejects_bad_sizes(gdn):
+    with pytest.raises(gdn.GDNError):
+        gdn.schedule(-1, 64, 1, 148)
+    assert gdn.schedule(1, 512, 16, 0)[0] == 1     # no multiprocessor count: single pass
+    assert gdn.schedule(0, 512, 16, 148)[0] == 1
 
 
 def decode_args(**over):

@@ -62,11 +62,16 @@ def checked_prefill(q, k, v, g, beta, S0, chunk, **kw):
     return out
 
 
-def gpu_prefill(d, chunk, S0=True):
+def gpu_prefill(d, chunk, S0=True, segmented=True):
     dd = to_dev(d)
     o, S_T = checked_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"],
-                             dd["S0"] if S0 else None, chunk)
+                             dd["S0"] if S0 else None, chunk, segmented=segmented)
     return o.cpu().numpy(), S_T.cpu().numpy()
+
+
+# gdn_prefill (one pass per chain) and gdn_prefill_ws (segments in parallel when
+# the chains are too few to fill the GPU)
+ENTRY = pytest.mark.parametrize("segmented", [False, True], ids=["single", "segmented"])
 
 
 @pytest.mark.parametrize("chunk", [64, 16])
@@ -79,31 +84,34 @@ def test_tiny_b1_h2_t64(chunk):
     assert_parity(S_T, rS, "S_T")
 
 
+@ENTRY
 @pytest.mark.parametrize("chunk", [64, 16])
 @pytest.mark.parametrize("T", [1, 15, 16, 17, 63, 64, 65, 100, 130, 200])
-def test_ragged_lengths(T, chunk):
+def test_ragged_lengths(T, chunk, segmented):
     d = inputs.prefill_inputs(2, T, 3, seed=T, s0_std=0.05)
-    o, S_T = gpu_prefill(d, chunk)
+    o, S_T = gpu_prefill(d, chunk, segmented=segmented)
     ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
     assert_parity(o, ro, f"o T={T}")
     assert_parity(S_T, rS, f"S_T T={T}")
 
 
+@ENTRY
 @pytest.mark.parametrize("chunk", [64, 16])
-def test_prefill_b1_h16_t512(chunk):
+def test_prefill_b1_h16_t512(chunk, segmented):
     w = inputs.WORKLOADS["prefill_b1_h16_t512"]
     d = inputs.workload_inputs(w, seed=0)
-    o, S_T = gpu_prefill(d, chunk)
+    o, S_T = gpu_prefill(d, chunk, segmented=segmented)
     ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
     assert_parity(o, ro, "o")
     assert_parity(S_T, rS, "S_T")
 
 
+@ENTRY
 @pytest.mark.parametrize("chunk", [64, 16])
-def test_prefill_b1_h16_t4096_carried_state(chunk):
+def test_prefill_b1_h16_t4096_carried_state(chunk, segmented):
     w = inputs.WORKLOADS["prefill_b1_h16_t4096_s0"]
     d = inputs.workload_inputs(w, seed=0)
-    o, S_T = gpu_prefill(d, chunk)
+    o, S_T = gpu_prefill(d, chunk, segmented=segmented)
     ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
     assert_parity(o, ro, "o")
     assert_parity(S_T, rS, "S_T")
@@ -125,16 +133,68 @@ def test_prefill_b4_h32_t32768_sampled_chains(chunk):
     torch.cuda.empty_cache()
 
 
+@ENTRY
 @pytest.mark.parametrize("chunk", [64, 16])
 @pytest.mark.parametrize("g_mean", [0.0, 2.0])
-def test_long_sequence_few_chains(chunk, g_mean):
+def test_long_sequence_few_chains(chunk, g_mean, segmented):
     """2048 tokens on two chains: the chain and side warps drift furthest apart
     when few CTAs share the GPU, which is where hand-off bugs between tiles show."""
     d = inputs.prefill_inputs(1, 2048, 2, seed=21, g_mean=g_mean)
-    o, S_T = gpu_prefill(d, chunk, S0=False)
+    o, S_T = gpu_prefill(d, chunk, S0=False, segmented=segmented)
     ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None)
     assert_parity(o, ro, f"o g_mean={g_mean}")
     assert_parity(S_T, rS, f"S_T g_mean={g_mean}")
+
+
+@pytest.mark.parametrize("B,T,H,s0", [
+    (1, 1000, 1, 0.05),    # one chain, 16 tiles: 8 segments of 2 tiles (7 chained ends)
+    (1, 577, 3, 0.0),      # ragged last segment (one token in its last tile)
+    (2, 700, 4, 0.1),      # 8 chains
+    (1, 256, 37, 0.02),    # 37 chains: 2 segments of 2 tiles
+])
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_segmented_schedule_shapes(B, T, H, s0, chunk):
+    gdn = _gdn()
+    n, L, ws = gdn.schedule(B, T, H, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert n > 1, "shape meant to be segmented"
+    assert gdn.workspace_bytes(B, T, H, chunk) == ws
+    d = inputs.prefill_inputs(B, T, H, seed=T + H, s0_std=s0)
+    o, S_T = gpu_prefill(d, chunk, S0=s0 > 0)
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"] if s0 > 0 else None)
+    assert_parity(o, ro, f"o {n}x{L}")
+    assert_parity(S_T, rS, f"S_T {n}x{L}")
+
+
+def test_segmented_in_place_state_deterministic_and_caller_workspace():
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(1, 640, 4, seed=9, s0_std=0.05))
+    assert gdn.workspace_bytes(1, 640, 4) > 0
+    o_ref, S_ref = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    # S_T == S0 in place, with a caller-owned workspace reused twice
+    ws = torch.empty(gdn.workspace_bytes(1, 640, 4), dtype=torch.uint8, device=DEV)
+    for _ in range(2):
+        S = d["S0"].clone()
+        o, _ = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], S, S_T=S, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(S, S_ref) and torch.equal(o, o_ref)
+
+
+def test_segmented_workspace_errors():
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(1, 640, 4, seed=9))
+    need = gdn.workspace_bytes(1, 640, 4)
+    with pytest.raises(gdn.GDNError) as e:
+        gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                    workspace=torch.empty(need - 256, dtype=torch.uint8, device=DEV))
+    assert e.value.code == gdn.GDN_ERR_WORKSPACE
+    big = torch.empty(need + 512, dtype=torch.uint8, device=DEV)
+    with pytest.raises(gdn.GDNError) as e:
+        gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], workspace=big[16:])
+    assert e.value.code == gdn.GDN_ERR_WORKSPACE
+    o = big[:1 * 640 * 4 * 128 * 4].view(torch.float32).view(1, 640, 4, 128)
+    with pytest.raises(gdn.GDNError) as e:
+        gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], o=o, workspace=big)
+    assert e.value.code == gdn.GDN_ERR_ALIAS
 
 
 def test_decode_b64_h16_256_steps_sampled_sequences():
@@ -170,17 +230,21 @@ def test_decode_equals_prefill_t1():
     assert_parity(S.cpu().numpy(), S_p.cpu().numpy(), "decode vs prefill S")
 
 
+@ENTRY
 @pytest.mark.parametrize("chunk", [64, 16])
-def test_split_carry(chunk):
+def test_split_carry(chunk, segmented):
     d = to_dev(inputs.prefill_inputs(1, 300, 4, seed=11, s0_std=0.05))
     gdn = _gdn()
-    o, S_T = checked_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk)
+    o, S_T = checked_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk,
+                             segmented=segmented)
     t1 = 130
     cut = lambda x, a, b: x[:, a:b].contiguous()
     o1, S1 = gdn.prefill(cut(d["q"], 0, t1), cut(d["k"], 0, t1), cut(d["v"], 0, t1),
-                         cut(d["g"], 0, t1), cut(d["beta"], 0, t1), d["S0"], chunk=chunk)
+                         cut(d["g"], 0, t1), cut(d["beta"], 0, t1), d["S0"], chunk=chunk,
+                         segmented=segmented)
     o2, S2 = gdn.prefill(cut(d["q"], t1, 300), cut(d["k"], t1, 300), cut(d["v"], t1, 300),
-                         cut(d["g"], t1, 300), cut(d["beta"], t1, 300), S1, chunk=chunk)
+                         cut(d["g"], t1, 300), cut(d["beta"], t1, 300), S1, chunk=chunk,
+                         segmented=segmented)
     torch.cuda.synchronize()
     assert_parity(torch.cat([o1, o2], 1).cpu().numpy(), o.cpu().numpy(), "split o")
     assert_parity(S2.cpu().numpy(), S_T.cpu().numpy(), "split S_T")
@@ -194,12 +258,13 @@ def test_chunk16_agrees_with_chunk64():
     assert_parity(S16, S64, "S chunk16 vs 64")
 
 
+@ENTRY
 @pytest.mark.parametrize("chunk", [64, 16])
-def test_bitwise_deterministic(chunk):
+def test_bitwise_deterministic(chunk, segmented):
     d = to_dev(inputs.prefill_inputs(2, 333, 4, seed=3, s0_std=0.02))
     gdn = _gdn()
-    a = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
-    b = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
+    a = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk, segmented=segmented)
+    b = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk, segmented=segmented)
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
