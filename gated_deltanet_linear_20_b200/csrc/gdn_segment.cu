@@ -28,45 +28,100 @@ constexpr int NTHREADS = 256;
 // Shared memory (offsets from a 1024-byte aligned base).  Each 128 x 128 bf16
 // operand is two 16 KB SW128 blocks of 128 rows x 64 columns (block h holds
 // columns 64h .. 64h+63): rows are M for the state (K-major A) and K for the
-// transfer matrix (MN-major B).  The f tile is two 8 KB blocks of 64 token rows.
+// transfer matrix (MN-major B).  The f tile (two 8 KB blocks of 64 token rows,
+// K-major B) reuses the transfer-matrix blocks once the chained products are
+// done.  The staging buffer receives fp32 rows by cp.async (row pitch 528 B,
+// so that eight consecutive rows read as float4 hit distinct banks): one
+// 128-row matrix, or two 64-row f tiles.
 constexpr uint32_t SS_HI = 0, SS_LO = 32768;
 constexpr uint32_t SF_HI = 65536, SF_LO = 98304;
-constexpr uint32_t SQ_HI = 131072, SQ_LO = 147456;
-constexpr uint32_t SM_BAR = 163840;  // one mbarrier (MMA completion) + verdict slot
+constexpr uint32_t SQ_HI = SF_HI, SQ_LO = SF_HI + 16384;
+constexpr uint32_t PITCH = 528;                  // bytes per staged fp32 row
+constexpr uint32_t SSTAGE = 131072;
+constexpr uint32_t STAGE_TILE = 64 * PITCH;      // one staged f tile
+constexpr uint32_t SM_BAR = SSTAGE + 128 * PITCH;  // mbarrier, verdict, TMEM slot
 constexpr uint32_t SMEM_USED = SM_BAR + 64;
+static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t TM_ACC = 0, TM_O = 128;  // 128-column state product, 64-column o tile
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
-// Thread t of the CTA converts row t/2, columns 64 (t%2) .. +63 of a row-major
-// 128 x 128 fp32 matrix into the hi/lo bf16 pair of SW128 blocks.  All loads
-// are issued before the first shared store (the stores are ordered asm, which
-// would otherwise serialise one global latency per chunk).
-__device__ __forceinline__ void load_split_matrix(const float* __restrict__ src, uint32_t hi,
-                                                  uint32_t lo) {
-  const int r = threadIdx.x >> 1, hf = threadIdx.x & 1;
-  const float4* row = reinterpret_cast<const float4*>(src + size_t(r) * D + 64 * hf);
-  float4 a[16];
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Row-major 128 x 128 fp32 matrix -> staging buffer (asynchronous; 16 chunks
+// of 16 B per thread, consecutive threads on consecutive chunks).
+__device__ __forceinline__ void stage_matrix(uint32_t stage, const float* __restrict__ src) {
 #pragma unroll
-  for (int i = 0; i < 16; ++i) a[i] = __ldg(row + i);
+  for (int i = 0; i < 16; ++i) {
+    const int c = threadIdx.x + NTHREADS * i;  // chunk: row c / 32, 16-byte column c % 32
+    cp_async16(stage + uint32_t(c >> 5) * PITCH + uint32_t(c & 31) * 16u, src + 4 * c);
+  }
+  cp_async_commit();
+}
+
+// f_t rows of the tokens t0 .. t0+63 of chain (b, h) -> one staged tile
+// (tokens at or past T are skipped; the split zeroes them).
+__device__ __forceinline__ void stage_f_tile(uint32_t stage, const PrefillArgs& p, int b, int h,
+                                             int t0) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = threadIdx.x + NTHREADS * i;  // chunk: token row c / 32, column c % 32
+    const int t = t0 + (c >> 5);
+    if (t < p.T)
+      cp_async16(stage + uint32_t(c >> 5) * PITCH + uint32_t(c & 31) * 16u,
+                 p.ws_f + ((size_t(b) * p.T + t) * p.H + h) * D + 4 * (c & 31));
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ float4 lds4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+// Staged 128 x 128 matrix -> hi/lo SW128 blocks.  Thread t: row t % 128,
+// columns 64 (t / 128) ..; eight consecutive threads read eight rows.
+__device__ __forceinline__ void split_staged_matrix(uint32_t stage, uint32_t hi, uint32_t lo) {
+  const int r = threadIdx.x & 127, hf = threadIdx.x >> 7;
+  const uint32_t row = stage + uint32_t(r) * PITCH + uint32_t(hf) * 256u;
 #pragma unroll
   for (int c8 = 0; c8 < 8; ++c8) {
-    const float x[8] = {a[2 * c8].x, a[2 * c8].y, a[2 * c8].z, a[2 * c8].w,
-                        a[2 * c8 + 1].x, a[2 * c8 + 1].y, a[2 * c8 + 1].z, a[2 * c8 + 1].w};
+    const float4 a = lds4(row + 32u * c8), b = lds4(row + 32u * c8 + 16u);
+    const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     store_split8(hi + 16384u * hf, lo + 16384u * hf, r, c8, x);
   }
 }
 
-// 32 consecutive floats of row `row`, columns 64 hf + 32 q .., as registers.
-__device__ __forceinline__ void load_row32(const float* __restrict__ p, float (&v)[32]) {
+// Staged f tile -> hi/lo K-major blocks (rows = tokens).  Thread t: token row
+// t % 64, features 32 (t / 64) ..; rows at or past T become zeros.
+__device__ __forceinline__ void split_staged_f(uint32_t stage, uint32_t hi, uint32_t lo, int nrows) {
+  const int r = threadIdx.x & 63, qd = threadIdx.x >> 6;
+  const uint32_t row = stage + uint32_t(r) * PITCH + uint32_t(qd) * 128u;
+  const uint32_t blk = 8192u * uint32_t(qd >> 1);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(p) + e);
-    v[4 * e] = a.x;
-    v[4 * e + 1] = a.y;
-    v[4 * e + 2] = a.z;
-    v[4 * e + 3] = a.w;
+  for (int c8 = 0; c8 < 4; ++c8) {
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+    if (r < nrows) {
+      a = lds4(row + 32u * c8);
+      b = lds4(row + 32u * c8 + 16u);
+    }
+    const float x[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    store_split8(hi + blk, lo + blk, r, 4 * (qd & 1) + c8, x);
   }
+}
+
+// 64 consecutive floats as registers (16 independent loads).
+__device__ __forceinline__ void load_row64(const float* __restrict__ p, float4 (&v)[16]) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) v[e] = __ldg(reinterpret_cast<const float4*>(p) + e);
 }
 
 struct Fix {
@@ -133,6 +188,8 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   const size_t mat = size_t(D) * D;
   const float* R = p.ws_R + size_t(chain) * p.nseg * mat;
   const float* F = p.ws_F + size_t(chain) * p.nseg * mat;
+  const bool last = (k == p.nseg - 1);
+  const int nprod = last ? k : k - 1;  // chained products S_j F_j, j = 1 .. nprod
 
   Fix f;
   f.sb = smem_u32(sm);
@@ -140,16 +197,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   f.verdict = reinterpret_cast<volatile int*>(sm + SM_BAR + 8);
   f.status = p.status;
   f.phase = 0;
-  if (tid == 0) {
-    mbar_init(f.bar, 1);
-    fence_mbar_init();
+  const uint32_t stage = f.sb + SSTAGE;
+
+  // Prologue: R_0 (= S_1) through registers while F_1 streams into staging.
+  {
+    float4 r0[16];
+    load_row64(R + size_t(tid & 127) * D + 64 * (tid >> 7), r0);
+    if (nprod >= 1) stage_matrix(stage, F + mat);
+    if (tid == 0) {
+      mbar_init(f.bar, 1);
+      fence_mbar_init();
+    }
+    if (warp == 0) {
+      tmem_alloc(smem_u32(sm + SM_BAR + 16), TMEM_COLS);
+      tmem_relinquish();
+    }
+    const int r = tid & 127, hf = tid >> 7;
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+      const float x[8] = {r0[2 * c8].x, r0[2 * c8].y, r0[2 * c8].z, r0[2 * c8].w,
+                          r0[2 * c8 + 1].x, r0[2 * c8 + 1].y, r0[2 * c8 + 1].z, r0[2 * c8 + 1].w};
+      store_split8(f.sb + SS_HI + 16384u * hf, f.sb + SS_LO + 16384u * hf, r, c8, x);
+    }
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(sm + SM_BAR + 16), TMEM_COLS);
-    tmem_relinquish();
-  }
-  // S_1 = R_0
-  load_split_matrix(R, f.sb + SS_HI, f.sb + SS_LO);
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -162,28 +232,36 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   const uint32_t tlane = f.tmem + (uint32_t((warp & 3) * 32) << 16);
   bool ok = true;
 
-  // S_{j+1} = S_j F_j + R_j for j = 1 .. k-1 (and j = k into S_T when k is last)
-  const bool last = (k == p.nseg - 1);
-  for (int j = 1; ok && j <= (last ? k : k - 1); ++j) {
-    load_split_matrix(F + j * mat, f.sb + SF_HI, f.sb + SF_LO);
+  // S_{j+1} = S_j F_j + R_j for j = 1 .. k-1; for the last segment also
+  // S_k F_k, kept in TMEM for S_T.  F_{j+1} streams in during product j.
+  for (int j = 1; ok && j <= nprod; ++j) {
+    cp_async_wait_all();
+    __syncthreads();                                   // F_j staged by every thread
+    split_staged_matrix(stage, f.sb + SF_HI, f.sb + SF_LO);
     fence_proxy_async_smem();
-    __syncthreads();
+    __syncthreads();                                   // staging free, SF ready
     if (tid == 0) {
       tc_fence_after();
       issue_state_product(f, f.tmem + TM_ACC);
       mma_commit(f.bar);
     }
+    if (j < nprod) stage_matrix(stage, F + (j + 1) * mat);
+    float4 rj[16];
+    if (j < k) load_row64(R + j * mat + size_t(row) * D + 64 * hf, rj);
     ok = f.wait_mma();
-    if (!ok) break;
-    if (j == k) break;  // the S_T product stays in TMEM until the o tiles are done
-    const float* rrow = R + j * mat + size_t(row) * D + 64 * hf;
+    if (!ok || j == k) break;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      float v[32], r[32];
-      load_row32(rrow + 32 * q, r);
+      float v[32];
       tmem_ld32(tlane + TM_ACC + 64 * hf + 32 * q, v);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] += r[e];
+      for (int e = 0; e < 8; ++e) {
+        const float4 a = rj[8 * q + e];
+        v[4 * e] += a.x;
+        v[4 * e + 1] += a.y;
+        v[4 * e + 2] += a.z;
+        v[4 * e + 3] += a.w;
+      }
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8)
         store_split8(f.sb + SS_HI + 16384u * hf, f.sb + SS_LO + 16384u * hf, row, 4 * q + c8,
@@ -194,73 +272,61 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
     __syncthreads();
   }
 
-  // o_t += S_k f_t over the tokens of segment k, 64 at a time
+  // o_t += S_k f_t over the tokens of segment k, 64 at a time; tile i + 1
+  // streams into the other staging half while tile i is multiplied.
   const int total_tiles = (p.T + NT - 1) / NT;
   const int tb = k * p.seg_tiles;
   const int te = min(total_tiles, tb + p.seg_tiles);
+  if (ok && tb < te) stage_f_tile(stage, p, b, h, tb * NT);
   for (int c = tb; ok && c < te; ++c) {
-    {
-      // thread -> token r = tid / 4, 32 features 32 (tid % 4) ..
-      const int r = tid >> 2, qd = tid & 3;
-      const int t = c * NT + r;
-      const float4* src =
-          reinterpret_cast<const float4*>(p.ws_f + ((size_t(b) * p.T + t) * p.H + h) * D + 32 * qd);
-      const uint32_t blk = 8192u * uint32_t(qd >> 1);
-      float x[32];
-      if (t < p.T) {
-        load_row32(reinterpret_cast<const float*>(src), x);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = 0.f;
-      }
-#pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8)
-        store_split8(f.sb + SQ_HI + blk, f.sb + SQ_LO + blk, r, 4 * (qd & 1) + c8, x + 8 * c8);
-    }
+    const uint32_t st = stage + uint32_t((c - tb) & 1) * STAGE_TILE;
+    cp_async_wait_all();
+    __syncthreads();                                   // tile c staged
+    split_staged_f(st, f.sb + SQ_HI, f.sb + SQ_LO, min(NT, p.T - c * NT));
     fence_proxy_async_smem();
-    tc_fence_before();
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
       issue_output_product(f, f.tmem + TM_O);
       mma_commit(f.bar);
     }
+    if (c + 1 < te) stage_f_tile(stage + uint32_t((c + 1 - tb) & 1) * STAGE_TILE, p, b, h, (c + 1) * NT);
+    // this thread: lane dv = row, tokens 32 hf .. 32 hf + 31 of the tile; the
+    // loads of o go out before the wait
+    const int t0 = c * NT + 32 * hf;
+    const int nvalid = min(32, p.T - t0);
+    float* orow = p.o + ((size_t(b) * p.T + t0) * p.H + h) * D + row;
+    const size_t ts = size_t(p.H) * D;
+    float cur[32];
+#pragma unroll
+    for (int n = 0; n < 32; ++n) cur[n] = (n < nvalid) ? orow[n * ts] : 0.f;
     ok = f.wait_mma();
     if (!ok) break;
-    {
-      // this thread: lane dv = row, tokens 32 hf .. 32 hf + 31 of the tile
-      // all 32 loads of o first, then the stores (one global latency, not 32)
-      const int t0 = c * NT + 32 * hf;
-      const int nvalid = min(32, p.T - t0);
-      float* orow = p.o + ((size_t(b) * p.T + t0) * p.H + h) * D + row;
-      const size_t ts = size_t(p.H) * D;
-      float cur[32];
+    float v[32];
+    tmem_ld32(tlane + TM_O + 32 * hf, v);
 #pragma unroll
-      for (int n = 0; n < 32; ++n) cur[n] = (n < nvalid) ? orow[n * ts] : 0.f;
-      float v[32];
-      tmem_ld32(tlane + TM_O + 32 * hf, v);
-#pragma unroll
-      for (int n = 0; n < 32; ++n)
-        if (n < nvalid) orow[n * ts] = cur[n] + v[n];
-    }
+    for (int n = 0; n < 32; ++n)
+      if (n < nvalid) orow[n * ts] = cur[n] + v[n];
     tc_fence_before();
     __syncthreads();
   }
+  cp_async_wait_all();
 
   // S_T = S_k F_k + R_k (the product is already in TMEM)
   if (ok && last) {
-    const float* rrow = R + k * mat + size_t(row) * D + 64 * hf;
+    float4 rk[16];
+    load_row64(R + k * mat + size_t(row) * D + 64 * hf, rk);
     float* dst = p.S_T + size_t(chain) * mat + size_t(row) * D + 64 * hf;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      float v[32], r[32];
-      load_row32(rrow + 32 * q, r);
+      float v[32];
       tmem_ld32(tlane + TM_ACC + 64 * hf + 32 * q, v);
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
+      for (int e = 0; e < 8; ++e) {
+        const float4 a = rk[8 * q + e];
         reinterpret_cast<float4*>(dst + 32 * q)[e] =
-            make_float4(v[4 * e] + r[4 * e], v[4 * e + 1] + r[4 * e + 1],
-                        v[4 * e + 2] + r[4 * e + 2], v[4 * e + 3] + r[4 * e + 3]);
+            make_float4(v[4 * e] + a.x, v[4 * e + 1] + a.y, v[4 * e + 2] + a.z, v[4 * e + 3] + a.w);
+      }
     }
   }
   tc_fence_before();
