@@ -11,6 +11,9 @@
 
 #include "gdn_internal.h"
 
+// Built-in scratch of gdn_prefill_static_ws (no allocation anywhere).
+static __device__ __align__(256) unsigned char g_static_ws[GDN_STATIC_WORKSPACE_BYTES];
+
 namespace {
 
 constexpr int kHeadDim = 128;
@@ -200,6 +203,25 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   return GDN_OK;
 }
 
+// Device address of the built-in scratch per device (looked up once, on the
+// first call on that device).
+void* g_static_ws_addr[kMaxDevices];
+std::mutex g_static_ws_mutex;
+
+int static_workspace(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return GDN_ERR_LAUNCH;
+  if (dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (!g_static_ws_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) return GDN_ERR_LAUNCH;
+    g_static_ws_addr[dev] = p;
+  }
+  *out = g_static_ws_addr[dev];
+  return GDN_OK;
+}
+
 }  // namespace
 
 namespace gdn {
@@ -232,6 +254,7 @@ const char* gdn_status_str(int code) {
     case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
     case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
     case GDN_ERR_WORKSPACE: return "workspace NULL, not 256-byte aligned, or smaller than gdn_prefill_workspace_bytes";
+    case GDN_ERR_STATIC_WORKSPACE_LIMIT: return "problem needs more scratch than the built-in GDN_STATIC_WORKSPACE_BYTES (16 MiB); use gdn_prefill_ws";
     default: return "unknown status code";
   }
 }
@@ -270,6 +293,34 @@ int gdn_prefill_ws(const void* q, const void* k, const void* v, const float* g,
                    int* status, void* stream) {
   return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, workspace,
                       workspace_bytes, true, status, stream);
+}
+
+int gdn_prefill_static_ws(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* S0, float* o, float* S_T, int B,
+                          int T, int H, int Dk, int Dv, int chunk, int* status, void* stream) {
+  // the shape checks of prefill_impl come first, so that bad arguments get
+  // their own codes rather than the limit
+  if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
+  const long long chains = (long long)B * H;
+  if (chains * T * kHeadDim > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL)
+    return GDN_ERR_SHAPE;
+  if (chains == 0 || T == 0)
+    return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, nullptr, 0, false,
+                        status, stream);
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+  int sms = 0;
+  if (num_sms(&sms) != GDN_OK) return GDN_ERR_LAUNCH;
+  const SegPlan plan = plan_segments(B, T, H, sms);
+  if (plan.ws_bytes > GDN_STATIC_WORKSPACE_BYTES) return GDN_ERR_STATIC_WORKSPACE_LIMIT;
+  void* ws = nullptr;
+  if (plan.ws_bytes > 0) {
+    const int rc = static_workspace(&ws);
+    if (rc != GDN_OK) return rc;
+  }
+  return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, ws,
+                      ws ? size_t(GDN_STATIC_WORKSPACE_BYTES) : 0, true, status, stream);
 }
 
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,

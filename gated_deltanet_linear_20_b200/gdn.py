@@ -33,6 +33,8 @@ _lib.gdn_prefill_workspace_bytes.argtypes = [_ci] * 6
 _lib.gdn_prefill_workspace_bytes.restype = ctypes.c_size_t
 _lib.gdn_prefill_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, ctypes.c_size_t, _vp, _vp]
 _lib.gdn_prefill_ws.restype = _ci
+_lib.gdn_prefill_static_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, _vp]
+_lib.gdn_prefill_static_ws.restype = _ci
 _lib.gdn_prefill_schedule.argtypes = [_ci] * 4 + [_vp, _vp, _vp]
 _lib.gdn_prefill_schedule.restype = _ci
 _lib.gdn_decode_step.argtypes = [_vp] * 7 + [_ci] * 4 + [_vp, _vp]
@@ -54,6 +56,8 @@ GDN_ERR_ALIAS = -5
 GDN_ERR_LAUNCH = -6
 GDN_ERR_DEVICE_TIMEOUT = -7
 GDN_ERR_WORKSPACE = -8
+GDN_ERR_STATIC_WORKSPACE_LIMIT = -9
+STATIC_WORKSPACE_BYTES = 16 << 20  # GDN_STATIC_WORKSPACE_BYTES
 
 
 class GDNError(RuntimeError):
@@ -164,6 +168,41 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                              ctypes.c_size_t(ws_bytes), _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_prefill_ws")
+    return o, S_T
+
+
+def prefill_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                   beta: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64, *,
+                   o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """gdn_prefill_static_ws: the segmented schedule on the library's built-in
+    16 MiB device scratch (no allocation).  Calls that may overlap on a device
+    race on that scratch; larger problems raise GDNError(GDN_ERR_STATIC_WORKSPACE_LIMIT)."""
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn.prefill_static runs on CUDA tensors only (no CPU path)")
+    _check(q, "q", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(k, "k", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(v, "v", torch.bfloat16, (B, T, H, Dv), dev)
+    _check(g, "g", torch.float32, (B, T, H), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, Dv, Dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
+    if S_T is None:
+        S_T = torch.empty((B, H, Dv, Dk), dtype=torch.float32, device=dev)
+    _check(S_T, "S_T", torch.float32, (B, H, Dv, Dk), dev)
+    if status is not None:
+        _check(status, "status", torch.int32, (1,), dev)
+    rc = _lib.gdn_prefill_static_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                    _ptr(o), _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(status),
+                                    _stream_handle(dev))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_prefill_static_ws")
     return o, S_T
 
 

@@ -44,6 +44,8 @@
  *     GDN_ERR_LAUNCH       the CUDA launch (or a CUDA runtime query) failed
  *     GDN_ERR_WORKSPACE    gdn_prefill_ws: workspace NULL, misaligned (256 B) or
  *                          smaller than gdn_prefill_workspace_bytes asked for
+ *     GDN_ERR_STATIC_WORKSPACE_LIMIT  gdn_prefill_static_ws: the problem needs more
+ *                          scratch than GDN_STATIC_WORKSPACE_BYTES
  * Device-side waits are bounded: if one gives up, the kernel writes
  * GDN_ERR_DEVICE_TIMEOUT to *status (when status is non-NULL), releases its
  * tensor memory and returns; read it with gdn_query_status.  The kernels never
@@ -69,8 +71,12 @@ enum gdn_status_code {
   GDN_ERR_ALIAS = -5,
   GDN_ERR_LAUNCH = -6,
   GDN_ERR_DEVICE_TIMEOUT = -7,
-  GDN_ERR_WORKSPACE = -8
+  GDN_ERR_WORKSPACE = -8,
+  GDN_ERR_STATIC_WORKSPACE_LIMIT = -9
 };
+
+/* Size of the library's built-in device scratch used by gdn_prefill_static_ws. */
+#define GDN_STATIC_WORKSPACE_BYTES (16u << 20)
 
 /* Returns GDN_ABI_VERSION of the built library; callers compare it with the
  * header they compiled against and refuse to proceed on a mismatch. */
@@ -135,6 +141,26 @@ int gdn_prefill_ws(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, const float* S0, float* o, float* S_T, int B, int T, int H,
                    int Dk, int Dv, int chunk, void* workspace, size_t workspace_bytes,
                    int* status, void* stream);
+
+/* gdn_prefill_ws without any caller workspace and without any device
+ * allocation: the scratch is a file-scope device array of the library of
+ * GDN_STATIC_WORKSPACE_BYTES (16 MiB).  The pages have no counterpart; it
+ * exists for callers that may not allocate.
+ *   Problems whose schedule needs more scratch than that (see
+ *   gdn_prefill_workspace_bytes; the single-pass schedule needs none) are
+ *   rejected with GDN_ERR_STATIC_WORKSPACE_LIMIT before anything is launched.
+ *   The scratch needs no zeroing: every byte read is written earlier in the
+ *   same call.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   stream capture.
+ *   All calls on a device share the one array: calls whose executions
+ *   overlap (other streams, other host threads) race on it and must be
+ *   serialised by the caller.
+ * Arguments, results and other errors as for gdn_prefill. */
+int gdn_prefill_static_ws(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* S0, float* o, float* S_T, int B,
+                          int T, int H, int Dk, int Dv, int chunk, int* status, void* stream);
 
 /* One decode step for B sequences (the recurrence above with T = 1), the state
  * read and written in place (the Megakernel decode of the Lucebox contribution

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(gdn):
 
 def test_abi_version_and_status_strings(gdn):
     assert gdn.abi_version() == 2
-    for code in range(-8, 1):
+    for code in range(-9, 1):
         s = gdn.status_str(code)
         assert s and s != "unknown status code"
     assert gdn.status_str(12345) == "unknown status code"
