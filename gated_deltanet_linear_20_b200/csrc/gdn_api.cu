@@ -189,16 +189,20 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
       a.ws_F = reinterpret_cast<float*>(base + plan.off_F);
     }
   }
-  CUtensorMap tq{}, tk{}, tv{};
+  CUtensorMap tq{}, tk{}, tv{}, to{}, tf{};
   if (T > 0) {
-    const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
         !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
-        !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2))
+        !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2) ||
+        !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4))
+      return GDN_ERR_LAUNCH;
+    tf = to;
+    if (a.nseg > 1 && !encode_act(&tf, a.ws_f, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4))
       return GDN_ERR_LAUNCH;
   }
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (gdn::launch_prefill(tq, tk, tv, a, chunk, st) != 0) return GDN_ERR_LAUNCH;
+  if (gdn::launch_prefill(tq, tk, tv, to, tf, a, chunk, st) != 0) return GDN_ERR_LAUNCH;
   if (a.nseg > 1 && gdn::launch_segment_fix(a, st) != 0) return GDN_ERR_LAUNCH;
   return GDN_OK;
 }

@@ -46,8 +46,11 @@ struct DecodeArgs {
 bool ensure_smem_attr(const void* func, int slot, int bytes);
 
 // Both return 0 on success, -1 when the launch failed.
+// tq, tk, tv: bf16 inputs; to: o, tf: the f output of the transfer-matrix
+// CTAs (ws_f; equal to `to` without segments) -- fp32, box 64 tokens x 128.
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const PrefillArgs& a, int chunk, cudaStream_t stream);
+                   const CUtensorMap& to, const CUtensorMap& tf, const PrefillArgs& a, int chunk,
+                   cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Second pass of the segmented schedule (a.nseg > 1).
 int launch_segment_fix(const PrefillArgs& a, cudaStream_t stream);

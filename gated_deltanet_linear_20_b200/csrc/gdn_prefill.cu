@@ -82,8 +82,11 @@ constexpr int APAD = 68;                      // row pitch (floats): conflict-fr
 constexpr uint32_t SOLVE_MAT = 64 * APAD * 4; // 17408 B
 constexpr uint32_t SM_A = 180224;             // A  fp32 [64][APAD] (K side)
 constexpr uint32_t SM_TF = SM_A + SOLVE_MAT;  // T  fp32 [64][APAD] (K side)
-constexpr uint32_t SM_AT = SM_TF + SOLVE_MAT; // T_II A_IK blocks fp32 [6][16][16] (K side)
-constexpr uint32_t SM_GATES = SM_AT + 6144;   // gate buffers (tile c uses c % GATE_BUFS)
+// T_II A_IK blocks fp32 [6][16][AT_PITCH] (K side); the 20-float row pitch puts the
+// eight rows a warp reads at once in eight distinct banks
+constexpr int AT_PITCH = 20, AT_BLOCK = 16 * AT_PITCH;
+constexpr uint32_t SM_AT = SM_TF + SOLVE_MAT;
+constexpr uint32_t SM_GATES = SM_AT + 6 * AT_BLOCK * 4;  // gate buffers (tile c uses c % GATE_BUFS)
 constexpr uint32_t GATE_BYTES = 1536;
 // The side role writes tile c's gates after the chain released tile c-3
 // (tm_free); the chain's last reader of tile c-4's buffer (the o drain) runs
@@ -140,6 +143,7 @@ struct Ctx {
   bool s0_identity;    // start from the identity instead of s0src / zeros
   const float* s0src;  // start state of this chain [128][128], or null
   float* odst;         // destination of o-like outputs, laid out like o
+  const CUtensorMap* tmo;  // TMA view of odst: [B][T][H][128] fp32, box 64 tokens x 128
   float* sdst;         // destination of the end state [128][128]
   __device__ __forceinline__ uint32_t bar(uint32_t off) const { return sb + SM_BAR + off; }
   __device__ __forceinline__ float* gates(int c) const {
@@ -235,7 +239,7 @@ __device__ __forceinline__ void solve_at_blocks(int kt, const float* sA, const f
       a1.x = fmaf(t1, x1.x, a1.x); a1.y = fmaf(t1, x1.y, a1.y);
       a1.z = fmaf(t1, x1.z, a1.z); a1.w = fmaf(t1, x1.w, a1.w);
     }
-    *reinterpret_cast<float4*>(sAt + blk * 256 + r * 16 + 4 * c4) =
+    *reinterpret_cast<float4*>(sAt + blk * AT_BLOCK + r * AT_PITCH + 4 * c4) =
         make_float4(a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w);
   }
 }
@@ -250,7 +254,7 @@ __device__ __forceinline__ void solve_distance(int kt, const float* sAt, float* 
     float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
 #pragma unroll
     for (int K = J; K < I; ++K) {
-      const float* atrow = sAt + at_index(I, K) * 256 + r * 16;      // At_IK row r
+      const float* atrow = sAt + at_index(I, K) * AT_BLOCK + r * AT_PITCH;  // At_IK row r
       const float* tcol = sTf + (K * 16) * APAD + J * 16 + 4 * c4;    // T_KJ rows, cols 4c4..
 #pragma unroll
       for (int m = 0; m < 16; m += 2) {
@@ -331,16 +335,16 @@ __device__ __forceinline__ void issue_p(const Ctx& x, int c) {
   mma_commit(x.bar(B_PFULL));
 }
 
-// o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] of tile c, this thread's 32
-// tokens (32 hf .. 32 hf + 31) of lane `dv`, 16 at a time, straight to HBM
-// (each warp store writes 32 consecutive floats of one token row).
-__device__ __forceinline__ void output_drain(const Ctx& x, const PrefillArgs& p, uint32_t tlane,
-                                             int b, int h, int dv, int hf, int c) {
+// o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] of tile c.  This thread's 32
+// tokens (32 hf ..) of lane dv go into an fp32 [64 tokens][128] tile in the
+// X^T region, which is free between the state update and the next X epilogue;
+// the leader then stores the tile with TMA (tokens at or past T are dropped by
+// the copy) and waits for the copy to have read the tile before X^T is written
+// again.
+__device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b, int h, int dv,
+                                             int hf, int c, bool leader) {
   const float* G = x.gates(c);
-  const int t0 = (x.tb + c) * NT + 32 * hf;
-  const int nvalid = min(32, p.T - t0);
-  float* orow = x.odst + ((size_t(b) * p.T + t0) * p.H + h) * D + dv;
-  const size_t tstride = size_t(p.H) * D;
+  float* so = reinterpret_cast<float*>(x.sm + SM_XH) + dv;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     float y[16], oi[16];
@@ -351,10 +355,16 @@ __device__ __forceinline__ void output_drain(const Ctx& x, const PrefillArgs& p,
       const float gv[4] = {gm.x, gm.y, gm.z, gm.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int n = 16 * q + 4 * e4 + e;
-        if (n < nvalid) orow[size_t(n) * tstride] = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
+        const int n = 32 * hf + 16 * q + 4 * e4 + e;  // token within the tile
+        so[n * D] = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
       }
     }
+  }
+  fence_proxy_async_smem();
+  named_bar(BAR_CHAIN, CHAIN_THREADS);
+  if (leader) {
+    tma_store_4d(x.tmo, x.sb + SM_XH, 0, h, (x.tb + c) * NT, b);
+    bulk_commit();
   }
 }
 
@@ -514,6 +524,26 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
+// Z = S_c K^T (into TM_Z) and/or Y = S_c Q^T (into TM_Y) for chunk s of the
+// tile in `kq`: A = the bf16 hi / lo state pair in TMEM, B = K or Q rows.
+template <int C>
+__device__ __forceinline__ void issue_zq(const Ctx& x, uint32_t kq, int s, bool z, bool y) {
+  const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
+  const uint32_t rows = 2048u * uint32_t(s);  // C rows of 128 B per chunk (C = 16)
+#pragma unroll
+  for (int part = 0; part < 2; ++part) {
+    const uint32_t a0 = x.tmem + (part ? TM_SLO : TM_SHI);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32 + rows;
+      const uint32_t acc = (part | kk) ? 1u : 0u;
+      if (z) mma_ts(x.tmem + TM_Z + C * s, a0 + kk * 8, sdesc_sw128(kq + off, 16, 1024), id, acc);
+      if (y)
+        mma_ts(x.tmem + TM_Y + C * s, a0 + kk * 8, sdesc_sw128(kq + 8192 + off, 16, 1024), id, acc);
+    }
+  }
+}
+
 // ============================================================== chain
 template <int C>
 __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
@@ -569,7 +599,8 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
     const bool last_tile = (c + 1 == ntiles);
 #pragma unroll 1
     for (int s = 0; s < NSUB; ++s, ++sc) {
-      // ---- [Z | Y] = S_c [K | Q]^T : M=128 (dv), N=2C, K=128 (dk); A = S hi, then S lo
+      // ---- Z = S_c K^T and Y = S_c Q^T : M=128 (dv), N=C each, K=128 (dk); A = S hi,
+      //      then S lo
       if (leader) {
         bool ok = true;
         if (s == 0) {
@@ -578,36 +609,25 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         if (!ok) x.fail();
         if (ok && !*x.abort_flag) {
           tc_fence_after();
-#pragma unroll
-          for (int part = 0; part < 2; ++part) {
-            const uint32_t a0 = x.tmem + (part ? TM_SLO : TM_SHI);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              const uint32_t acc = (part | kk) ? 1u : 0u;
-              if constexpr (C == 64) {
-                mma_ts(x.tmem + TM_Z, a0 + kk * 8, sdesc_sw128(kq + off, 16, 1024),
-                       idesc_bf16(128, 128, 0, 0, 0), acc);
-              } else {
-                const uint32_t rows = 2048u * s;
-                mma_ts(x.tmem + TM_Z + 16 * s, a0 + kk * 8, sdesc_sw128(kq + off + rows, 16, 1024),
-                       idesc_bf16(128, 16, 0, 0, 0), acc);
-                mma_ts(x.tmem + TM_Y + 16 * s, a0 + kk * 8,
-                       sdesc_sw128(kq + 8192 + off + rows, 16, 1024), idesc_bf16(128, 16, 0, 0, 0),
-                       acc);
-              }
-            }
-          }
+          issue_zq<C>(x, kq, s, true, true);
           mma_commit(x.bar(B_ZQ));
         }
       }
-      if (!rs.wait(x, x.bar(B_ZQ), sc & 1)) return;
-      if (s == 0) {
-        if (!rs.wait(x, x.bar(gfull_off(c)), gfull_parity(c))) return;
-        if (!x.vzero) {
-          if (!rs.wait(x, x.bar(B_VFULL), c & 1)) return;
-          if (leader) *x.misc(M_V_SEEN) = c + 1;
+      // one agreement: Z is in TMEM and, at a tile's first chunk, its gates and V are in
+      {
+        bool ok = true;
+        if (leader) {
+          bulk_wait_read0();  // the previous tile's o store has read the X^T region
+          ok = (*x.abort_flag == 0) && mbar_wait_bounded(x.bar(B_ZQ), sc & 1, WAIT_LIMIT_NS);
+          if (ok && s == 0)
+            ok = mbar_wait_bounded(x.bar(gfull_off(c)), gfull_parity(c), WAIT_LIMIT_NS);
+          if (ok && s == 0 && !x.vzero) {
+            ok = mbar_wait_bounded(x.bar(B_VFULL), c & 1, WAIT_LIMIT_NS);
+            if (ok) *x.misc(M_V_SEEN) = c + 1;
+          }
+          if (!ok) x.fail();
         }
+        if (!rs.agree(x, ok)) return;
       }
 
       // ---- X^T[dv][n] = beta_n V[n][dv] - beta_n Gamma_n Z[dv][n]  (hi/lo -> SMEM)
@@ -744,8 +764,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
 
       // ---- o of the whole tile is complete after its last chunk: o[t][dv] =
       //      Gamma_t Y[dv][t] + O_intra[dv][t], this thread's 32 tokens to HBM
-      //      (loads first; the stores drain while the chain moves on)
-      if (s == NSUB - 1) output_drain(x, p, tlane, b, h, dv, ch, c);
+      if (s == NSUB - 1) output_drain(x, tlane, b, h, dv, ch, c, leader);
 
       // ---- S_out now sits in TMEM: refresh its hi/lo copy, and pre-scale it by
       //      the next chunk's decay (or store it as S_T after the last chunk)
@@ -791,7 +810,8 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
 template <int C>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const PrefillArgs p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                   const __grid_constant__ CUtensorMap tm_f, const PrefillArgs p) {
   static_assert(C == 16 || C == 64, "chunk must be 16 or 64");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -823,6 +843,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   x.s0_identity = frun;
   x.s0src = (seg == 0 && p.S0) ? p.S0 + cstate : nullptr;
   x.odst = frun ? p.ws_f : p.o;
+  x.tmo = frun ? &tm_f : &tm_o;
   int ntiles = total_tiles;
   if (p.nseg > 1) {
     x.tb = seg * p.seg_tiles;
@@ -835,6 +856,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
+    prefetch_tmap(x.tmo);
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(x.sb + SM_BAR + 8 * i, 1);
     fence_mbar_init();
     for (int i = 0; i < 16; ++i) reinterpret_cast<volatile int*>(sm + SM_MISC)[i] = 0;
@@ -853,6 +875,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   else
     kside_role<C>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
 
+  if (tid == 0) bulk_wait0();  // the chain leader's o stores have completed
   tc_fence_before();
   __syncthreads();
   // An aborted CTA may still have TMA loads in flight: wait for them (bounded)
@@ -882,7 +905,8 @@ __global__ void copy_state_kernel(const float* __restrict__ S0, float* __restric
 }  // namespace
 
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                   const PrefillArgs& a, int chunk, cudaStream_t stream) {
+                   const CUtensorMap& to, const CUtensorMap& tf, const PrefillArgs& a, int chunk,
+                   cudaStream_t stream) {
   const int chains = a.B * a.H;
   if (chains == 0) return 0;
   if (a.T == 0) {
@@ -895,10 +919,10 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   const int ctas = a.nseg > 1 ? chains * (2 * a.nseg - 1) : chains;
   if (chunk == 64) {
     if (!ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<64>), 0, int(smem))) return -1;
-    prefill_kernel<64><<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, a);
+    prefill_kernel<64><<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, to, tf, a);
   } else {
     if (!ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<16>), 1, int(smem))) return -1;
-    prefill_kernel<16><<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, a);
+    prefill_kernel<16><<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, to, tf, a);
   }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
