@@ -45,6 +45,7 @@ STATE_BYTES = D * D * 4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 PREFILL_SOURCES = ["gated_deltanet_linear_20_b200/csrc/gdn_prefill.cu",
                    "gated_deltanet_linear_20_b200/csrc/gdn_segment.cu",
+                   "gated_deltanet_linear_20_b200/csrc/gdn_api.cu",
                    "gated_deltanet_linear_20_b200/csrc/sm100.cuh"]
 DECODE_SOURCES = ["gated_deltanet_linear_20_b200/csrc/gdn_decode.cu"]
 
@@ -92,8 +93,8 @@ def source_sha(paths):
 
 
 def committed_traffic(key, paths):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    """DRAM bytes per step (every launch of the step) from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
     try:
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
             rec = json.load(f).get(key)
@@ -101,7 +102,7 @@ def committed_traffic(key, paths):
         return None
     if not rec or rec.get("kernel_sha") != source_sha(paths):
         return None
-    return rec.get("dram_bytes_per_launch")
+    return rec.get("dram_bytes_per_step")
 
 
 class ClockSampler:
@@ -485,6 +486,37 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+PROFILE_CASES = {
+    # name: (workload, chunk, calls) -- untimed calls for ncu captures
+    "decode": ("decode_b64_h16", None, 5),
+    "prefill_b4_h32_t2048": (None, 64, 3),   # the large prefill's structure on 2048 tokens
+    "headline": ("prefill_b1_h16_t512", 64, 3),
+}
+
+
+def run_profile_case(name):
+    """A few untimed calls of one case on cuda:0, for ncu captures (never a
+    bench number)."""
+    from gated_deltanet_linear_20_b200 import gdn
+    dev = torch.device("cuda", 0)
+    wname, chunk, calls = PROFILE_CASES[name]
+    if name == "decode":
+        w = gin.WORKLOADS[wname]
+        d = gin.workload_inputs(w, seed=0, device=str(dev))
+        S = d["S"].clone()
+        for i in range(calls):
+            gdn.decode_step(d["q"][i], d["k"][i], d["v"][i], d["g"][i], d["beta"][i], S)
+    else:
+        if wname is None:
+            d = gin.prefill_inputs(4, 2048, 32, seed=0, g_mean=2.0, device=str(dev))
+        else:
+            d = gin.workload_inputs(gin.WORKLOADS[wname], seed=0, device=str(dev))
+        for _ in range(calls):
+            gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "calls": calls}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -496,7 +528,12 @@ def main(argv=None):
     ap.add_argument("--chunk", type=int, default=64, choices=[16, 64])
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="run a few untimed calls of one case for an ncu capture, then exit")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup()
