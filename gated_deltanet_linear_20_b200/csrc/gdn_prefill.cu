@@ -324,13 +324,12 @@ __device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, f
 }
 
 __device__ __forceinline__ void issue_p(const Ctx& x, int c) {
-  const uint32_t kq = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
+  const uint64_t d0 = sdesc_sw128(x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0), 16, 1024);
   const uint32_t id = idesc_bf16(128, 64, 0, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    mma_ss(x.tmem + TM_P, sdesc_sw128(kq + off, 16, 1024), sdesc_sw128(kq + off, 16, 1024), id,
-           kk > 0);
+    const uint64_t d = sdesc_add(d0, (kk >> 2) * 16384 + (kk & 3) * 32);
+    mma_ss(x.tmem + TM_P, d, d, id, kk > 0);
   }
   mma_commit(x.bar(B_PFULL));
 }
@@ -524,22 +523,29 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
-// Z = S_c K^T (into TM_Z) and/or Y = S_c Q^T (into TM_Y) for chunk s of the
-// tile in `kq`: A = the bf16 hi / lo state pair in TMEM, B = K or Q rows.
+// Z = S_c K^T (into TM_Z) and Y = S_c Q^T (into TM_Y) for chunk s of the tile
+// in `kq`: A = the bf16 hi / lo state pair in TMEM, B = K and Q rows.  With
+// chunk 64 the K and Q rows of the tile are adjacent (64 + 64 rows) and Y sits
+// right after Z in TMEM, so one N = 128 MMA per step computes both.
 template <int C>
-__device__ __forceinline__ void issue_zq(const Ctx& x, uint32_t kq, int s, bool z, bool y) {
-  const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
-  const uint32_t rows = 2048u * uint32_t(s);  // C rows of 128 B per chunk (C = 16)
+__device__ __forceinline__ void issue_zq(const Ctx& x, uint32_t kq, int s) {
+  // C rows of 128 B per chunk (C = 16)
+  const uint64_t d0 = sdesc_sw128(kq + 2048u * uint32_t(s), 16, 1024);
 #pragma unroll
   for (int part = 0; part < 2; ++part) {
     const uint32_t a0 = x.tmem + (part ? TM_SLO : TM_SHI);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32 + rows;
+      const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
       const uint32_t acc = (part | kk) ? 1u : 0u;
-      if (z) mma_ts(x.tmem + TM_Z + C * s, a0 + kk * 8, sdesc_sw128(kq + off, 16, 1024), id, acc);
-      if (y)
-        mma_ts(x.tmem + TM_Y + C * s, a0 + kk * 8, sdesc_sw128(kq + 8192 + off, 16, 1024), id, acc);
+      if constexpr (C == 64) {
+        static_assert(TM_Y == TM_Z + 64, "Y follows Z");
+        mma_ts(x.tmem + TM_Z, a0 + kk * 8, sdesc_add(d0, off), idesc_bf16(128, 128, 0, 0, 0), acc);
+      } else {
+        const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
+        mma_ts(x.tmem + TM_Z + C * s, a0 + kk * 8, sdesc_add(d0, off), id, acc);
+        mma_ts(x.tmem + TM_Y + C * s, a0 + kk * 8, sdesc_add(d0, off + 8192), id, acc);
+      }
     }
   }
 }
@@ -609,7 +615,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         if (!ok) x.fail();
         if (ok && !*x.abort_flag) {
           tc_fence_after();
-          issue_zq<C>(x, kq, s, true, true);
+          issue_zq<C>(x, kq, s);
           mma_commit(x.bar(B_ZQ));
         }
       }
@@ -677,16 +683,17 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         if (ok && !*x.abort_flag) {
           tc_fence_after();
           const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
+          const uint64_t d0 = sdesc_sw128(sb + uint32_t(C * s) * 2u, 16, 1024);  // chunk's K offset
           const uint32_t trow = uint32_t(C * s / 8) * 1024u;
 #pragma unroll
           for (int part = 0; part < 3; ++part) {
-            const uint32_t xa = sb + (part == 2 ? SM_XL : SM_XH);
-            const uint32_t tb = sb + (part == 1 ? SM_TL : SM_TH) + trow;
+            const uint32_t xa = part == 2 ? SM_XL : SM_XH;
+            const uint32_t tb = (part == 1 ? SM_TL : SM_TH) + trow;
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
-              const uint32_t kb = uint32_t(C * s + 16 * ks) * 2u;
-              mma_ss(x.tmem + TM_Z + C * s, sdesc_sw128(xa + kb, 16, 1024),
-                     sdesc_sw128(tb + kb, 16, 1024), id, (part | ks) ? 1u : 0u);
+              const uint32_t kb = uint32_t(16 * ks) * 2u;
+              mma_ss(x.tmem + TM_Z + C * s, sdesc_add(d0, xa + kb), sdesc_add(d0, tb + kb), id,
+                     (part | ks) ? 1u : 0u);
             }
           }
           mma_commit(x.bar(B_DL));
@@ -733,27 +740,28 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       if (leader && !*x.abort_flag) {
         tc_fence_after();
         const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
+        const uint64_t d0 = sdesc_sw128(sb + uint32_t(C * s) * 2u, 16, 1024);  // chunk's K offset
         const uint32_t mrow = uint32_t(C * s / 8) * 1024u;
 #pragma unroll
         for (int part = 0; part < 3; ++part) {
-          const uint32_t da = sb + (part == 2 ? SM_DL : SM_DH);
-          const uint32_t mb = sb + (part == 1 ? SM_MQL : SM_MQH) + mrow;
+          const uint32_t da = part == 2 ? SM_DL : SM_DH;
+          const uint32_t mb = (part == 1 ? SM_MQL : SM_MQH) + mrow;
 #pragma unroll
           for (int ks = 0; ks < C / 16; ++ks) {
-            const uint32_t kb = uint32_t(C * s + 16 * ks) * 2u;
-            mma_ss(x.tmem + TM_OI + C * s, sdesc_sw128(da + kb, 16, 1024),
-                   sdesc_sw128(mb + kb, 16, 1024), id, (part | ks) ? 1u : 0u);
+            const uint32_t kb = uint32_t(16 * ks) * 2u;
+            mma_ss(x.tmem + TM_OI + C * s, sdesc_add(d0, da + kb), sdesc_add(d0, mb + kb), id,
+                   (part | ks) ? 1u : 0u);
           }
         }
         const uint32_t idu = idesc_bf16(128, 128, 0, 1, 0);
+        const uint64_t dk = sdesc_sw128(kq + uint32_t(C * s) * 128u, 16384, 1024);  // K rows, MN-major
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-          const uint32_t da = sb + (part ? SM_XL : SM_XH);
+          const uint32_t da = part ? SM_XL : SM_XH;
 #pragma unroll
           for (int ks = 0; ks < C / 16; ++ks) {
-            const int tok = C * s + 16 * ks;
-            mma_ss(x.tmem + TM_S, sdesc_sw128(da + uint32_t(tok) * 2u, 16, 1024),
-                   sdesc_sw128(kq + uint32_t(tok) * 128u, 16384, 1024), idu, 1u);
+            mma_ss(x.tmem + TM_S, sdesc_add(d0, da + uint32_t(16 * ks) * 2u),
+                   sdesc_add(dk, uint32_t(16 * ks) * 128u), idu, 1u);
           }
         }
         mma_commit(x.bar(B_OU));

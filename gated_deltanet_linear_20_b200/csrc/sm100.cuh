@@ -345,6 +345,14 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
          (uint64_t(2) << 61);
 }
 
+// Descriptor of (the address of `desc`) + `bytes`: the start address sits in
+// the low 14 bits as addr >> 4, and shared-memory addresses stay below 256 KB,
+// so the sum never carries into the next field.  Lets unrolled MMA loops build
+// one descriptor per operand and add immediate offsets.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+  return desc + uint64_t(bytes >> 4);
+}
+
 // ---------------------------------------------------------------- bf16 helpers
 // Splits x into hi + lo with hi = bf16(x) and lo = bf16(x - hi) (both round to
 // nearest even); hi + lo carries ~16 significant bits of x.
