@@ -25,25 +25,27 @@ using namespace sm100;
 constexpr int D = 128;
 constexpr int NT = 64;
 constexpr int NTHREADS = 256;
-// Shared memory (offsets from a 1024-byte aligned base).  Each 128 x 128 bf16
-// operand is two 16 KB SW128 blocks of 128 rows x 64 columns (block h holds
-// columns 64h .. 64h+63): rows are M for the state (K-major A) and K for the
-// transfer matrix (MN-major B).  The f tile (two 8 KB blocks of 64 token rows,
-// K-major B) reuses the transfer-matrix blocks once the chained products are
-// done.  The staging buffer receives fp32 rows by cp.async (row pitch 528 B,
-// so that eight consecutive rows read as float4 hit distinct banks): one
-// 128-row matrix, or two 64-row f tiles.
-constexpr uint32_t SS_HI = 0, SS_LO = 32768;
-constexpr uint32_t SF_HI = 65536, SF_LO = 98304;
+// The chained state S lives in tensor memory as a bf16 hi/lo pair (the A
+// operand of every product, lane = row).  Shared memory (offsets from a
+// 1024-byte aligned base):
+//   F hi/lo: the transfer matrix as the MN-major B operand, two 16 KB SW128
+//     blocks each (block h: columns 64h .. 64h+63, rows = K); the f tile (two
+//     8 KB blocks of 64 token rows, K-major B) reuses it once the products are done;
+//   two fp32 staging buffers filled by cp.async (row pitch 528 B, so that eight
+//   consecutive rows read as float4 hit distinct banks): one for the next
+//   transfer matrix (or two f tiles), one for R_j and finally S_T.
+constexpr uint32_t SF_HI = 0, SF_LO = 32768;
 constexpr uint32_t SQ_HI = SF_HI, SQ_LO = SF_HI + 16384;
 constexpr uint32_t PITCH = 528;                  // bytes per staged fp32 row
-constexpr uint32_t SSTAGE = 131072;
+constexpr uint32_t STAGE_BYTES = 128 * PITCH;
+constexpr uint32_t SSTAGE = 65536;               // F_{j+1}, then f tiles
 constexpr uint32_t STAGE_TILE = 64 * PITCH;      // one staged f tile
-constexpr uint32_t SM_BAR = SSTAGE + 128 * PITCH;  // mbarrier, verdict, TMEM slot
+constexpr uint32_t RSTAGE = SSTAGE + STAGE_BYTES;  // R_j, then S_T
+constexpr uint32_t SM_BAR = RSTAGE + STAGE_BYTES;  // mbarrier, verdict, TMEM slot
 constexpr uint32_t SMEM_USED = SM_BAR + 64;
 static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
-constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t TM_ACC = 0, TM_O = 128;  // 128-column state product, 64-column o tile
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_ACC = 0, TM_SHI = 128, TM_SLO = 192, TM_O = 256;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -51,6 +53,9 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all_but_one() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
 
 // Row-major 128 x 128 fp32 matrix -> staging buffer (asynchronous; 16 chunks
 // of 16 B per thread, consecutive threads on consecutive chunks).
@@ -86,9 +91,14 @@ __device__ __forceinline__ float4 lds4(uint32_t addr) {
                : "memory");
   return v;
 }
+__device__ __forceinline__ void sts4(uint32_t addr, float4 v) {
+  st_shared_v4(addr, __float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z),
+               __float_as_uint(v.w));
+}
 
-// Staged 128 x 128 matrix -> hi/lo SW128 blocks.  Thread t: row t % 128,
-// columns 64 (t / 128) ..; eight consecutive threads read eight rows.
+// Staged 128 x 128 matrix -> hi/lo SW128 blocks (the MN-major B operand).
+// Thread t: row t % 128, columns 64 (t / 128) ..; eight consecutive threads
+// read eight rows.
 __device__ __forceinline__ void split_staged_matrix(uint32_t stage, uint32_t hi, uint32_t lo) {
   const int r = threadIdx.x & 127, hf = threadIdx.x >> 7;
   const uint32_t row = stage + uint32_t(r) * PITCH + uint32_t(hf) * 256u;
@@ -118,10 +128,18 @@ __device__ __forceinline__ void split_staged_f(uint32_t stage, uint32_t hi, uint
   }
 }
 
-// 64 consecutive floats as registers (16 independent loads).
-__device__ __forceinline__ void load_row64(const float* __restrict__ p, float4 (&v)[16]) {
+// 32 staged floats of row `row` starting at column `col` (epilogue mapping:
+// lane = row, so eight consecutive lanes read eight rows).
+__device__ __forceinline__ void lds_row32(uint32_t stage, int row, int col, float (&v)[32]) {
+  const uint32_t a = stage + uint32_t(row) * PITCH + uint32_t(col) * 4u;
 #pragma unroll
-  for (int e = 0; e < 16; ++e) v[e] = __ldg(reinterpret_cast<const float4*>(p) + e);
+  for (int e = 0; e < 8; ++e) {
+    const float4 x = lds4(a + 16u * e);
+    v[4 * e] = x.x;
+    v[4 * e + 1] = x.y;
+    v[4 * e + 2] = x.z;
+    v[4 * e + 3] = x.w;
+  }
 }
 
 struct Fix {
@@ -144,36 +162,43 @@ struct Fix {
   }
 };
 
-// acc (TMEM, lane = row of S, column = column of F) = S F.  A = S (K-major),
-// B = F (MN-major: K rows of 128 B, N blocks 16 KB apart).
+// acc (TMEM, lane = row of S, column = column of F) = S F.  A = S hi / lo in
+// TMEM, B = F (MN-major: K rows of 128 B, N blocks 16 KB apart).
 __device__ __forceinline__ void issue_state_product(const Fix& f, uint32_t acc) {
   const uint32_t id = idesc_bf16(128, 128, 0, 1, 0);
+  const uint64_t d0 = sdesc_sw128(f.sb, 16384, 1024);
 #pragma unroll
   for (int part = 0; part < 3; ++part) {
-    const uint32_t a = f.sb + (part == 2 ? SS_LO : SS_HI);
-    const uint32_t bm = f.sb + (part == 1 ? SF_LO : SF_HI);
+    const uint32_t a = f.tmem + (part == 2 ? TM_SLO : TM_SHI);
+    const uint32_t bm = part == 1 ? SF_LO : SF_HI;
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      mma_ss(acc, sdesc_sw128(a + (kk >> 2) * 16384u + (kk & 3) * 32u, 16, 1024),
-             sdesc_sw128(bm + kk * 2048u, 16384, 1024), id, (part | kk) ? 1u : 0u);
-    }
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ts(acc, a + 8u * kk, sdesc_add(d0, bm + kk * 2048u), id, (part | kk) ? 1u : 0u);
   }
 }
 
 // acc (TMEM, lane = dv, column = token of the tile) = S f^T.  B = f tile (K-major).
 __device__ __forceinline__ void issue_output_product(const Fix& f, uint32_t acc) {
   const uint32_t id = idesc_bf16(128, 64, 0, 0, 0);
+  const uint64_t d0 = sdesc_sw128(f.sb, 16, 1024);
 #pragma unroll
   for (int part = 0; part < 3; ++part) {
-    const uint32_t a = f.sb + (part == 2 ? SS_LO : SS_HI);
-    const uint32_t bm = f.sb + (part == 1 ? SQ_LO : SQ_HI);
+    const uint32_t a = f.tmem + (part == 2 ? TM_SLO : TM_SHI);
+    const uint32_t bm = part == 1 ? SQ_LO : SQ_HI;
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t ko = (kk & 3) * 32u;
-      mma_ss(acc, sdesc_sw128(a + (kk >> 2) * 16384u + ko, 16, 1024),
-             sdesc_sw128(bm + (kk >> 2) * 8192u + ko, 16, 1024), id, (part | kk) ? 1u : 0u);
-    }
+    for (int kk = 0; kk < 8; ++kk)
+      mma_ts(acc, a + 8u * kk, sdesc_add(d0, bm + (kk >> 2) * 8192u + (kk & 3) * 32u), id,
+             (part | kk) ? 1u : 0u);
   }
+}
+
+// Writes 32 consecutive state values (columns col .. col+31 of this lane's row)
+// as bf16 hi/lo pairs into the state's TMEM columns.
+__device__ __forceinline__ void store_state32(uint32_t tlane, int col, const float (&v)[32]) {
+  uint32_t hi[16], lo[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
+  tmem_st16x2(tlane + TM_SHI + col / 2, hi, tlane + TM_SLO + col / 2, lo);
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillArgs p) {
@@ -190,6 +215,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   const float* F = p.ws_F + size_t(chain) * p.nseg * mat;
   const bool last = (k == p.nseg - 1);
   const int nprod = last ? k : k - 1;  // chained products S_j F_j, j = 1 .. nprod
+  // R_j is added after product j for j < k, and after the last product (j = k)
+  // of the last segment, where it completes S_T
+  auto need_r = [&](int j) { return j < k || (last && j == k); };
 
   Fix f;
   f.sb = smem_u32(sm);
@@ -197,32 +225,22 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   f.verdict = reinterpret_cast<volatile int*>(sm + SM_BAR + 8);
   f.status = p.status;
   f.phase = 0;
-  const uint32_t stage = f.sb + SSTAGE;
+  const uint32_t stage = f.sb + SSTAGE, rstage = f.sb + RSTAGE;
 
-  // Prologue: R_0 (= S_1) through registers while F_1 streams into staging.
-  {
-    float4 r0[16];
-    load_row64(R + size_t(tid & 127) * D + 64 * (tid >> 7), r0);
-    if (nprod >= 1) stage_matrix(stage, F + mat);
-    if (tid == 0) {
-      mbar_init(f.bar, 1);
-      fence_mbar_init();
-    }
-    if (warp == 0) {
-      tmem_alloc(smem_u32(sm + SM_BAR + 16), TMEM_COLS);
-      tmem_relinquish();
-    }
-    const int r = tid & 127, hf = tid >> 7;
-#pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-      const float x[8] = {r0[2 * c8].x, r0[2 * c8].y, r0[2 * c8].z, r0[2 * c8].w,
-                          r0[2 * c8 + 1].x, r0[2 * c8 + 1].y, r0[2 * c8 + 1].z, r0[2 * c8 + 1].w};
-      store_split8(f.sb + SS_HI + 16384u * hf, f.sb + SS_LO + 16384u * hf, r, c8, x);
-    }
+  // Prologue: R_0 (= S_1) and F_1 stream into the two staging buffers.
+  stage_matrix(rstage, R);
+  if (nprod >= 1) stage_matrix(stage, F + mat);
+  if (tid == 0) {
+    mbar_init(f.bar, 1);
+    fence_mbar_init();
   }
-  fence_proxy_async_smem();
+  if (warp == 0) {
+    tmem_alloc(smem_u32(sm + SM_BAR + 16), TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (nprod >= 1) cp_async_wait_all_but_one(); else cp_async_wait_all();
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // R_0 staged, TMEM allocated
   tc_fence_after();
   f.tmem = *reinterpret_cast<volatile uint32_t*>(sm + SM_BAR + 16);
 
@@ -230,13 +248,23 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   // accumulators, and the column half `hf`.
   const int row = (warp & 3) * 32 + lane, hf = warp >> 2;
   const uint32_t tlane = f.tmem + (uint32_t((warp & 3) * 32) << 16);
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    float v[32];
+    lds_row32(rstage, row, 64 * hf + 32 * q, v);
+    store_state32(tlane, 64 * hf + 32 * q, v);
+  }
+  tc_fence_before();
+  __syncthreads();  // S_1 in TMEM; the R staging buffer is free
+  if (need_r(1)) stage_matrix(rstage, R + mat);
   bool ok = true;
 
   // S_{j+1} = S_j F_j + R_j for j = 1 .. k-1; for the last segment also
-  // S_k F_k, kept in TMEM for S_T.  F_{j+1} streams in during product j.
+  // S_k F_k, kept in TMEM for S_T.  F_{j+1} streams in during product j, and
+  // R_{j+1} during the epilogue of product j + 1's predecessor.
   for (int j = 1; ok && j <= nprod; ++j) {
     cp_async_wait_all();
-    __syncthreads();                                   // F_j staged by every thread
+    __syncthreads();                                   // F_j and R_j staged
     split_staged_matrix(stage, f.sb + SF_HI, f.sb + SF_LO);
     fence_proxy_async_smem();
     __syncthreads();                                   // staging free, SF ready
@@ -246,30 +274,20 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
       mma_commit(f.bar);
     }
     if (j < nprod) stage_matrix(stage, F + (j + 1) * mat);
-    float4 rj[16];
-    if (j < k) load_row64(R + j * mat + size_t(row) * D + 64 * hf, rj);
     ok = f.wait_mma();
     if (!ok || j == k) break;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      float v[32];
+      float v[32], r[32];
+      lds_row32(rstage, row, 64 * hf + 32 * q, r);
       tmem_ld32(tlane + TM_ACC + 64 * hf + 32 * q, v);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float4 a = rj[8 * q + e];
-        v[4 * e] += a.x;
-        v[4 * e + 1] += a.y;
-        v[4 * e + 2] += a.z;
-        v[4 * e + 3] += a.w;
-      }
-#pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8)
-        store_split8(f.sb + SS_HI + 16384u * hf, f.sb + SS_LO + 16384u * hf, row, 4 * q + c8,
-                     v + 8 * c8);
+      for (int e = 0; e < 32; ++e) v[e] += r[e];
+      store_state32(tlane, 64 * hf + 32 * q, v);
     }
-    fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    __syncthreads();                                   // S_{j+1} in TMEM; R staging free
+    if (need_r(j + 1)) stage_matrix(rstage, R + (j + 1) * mat);
   }
 
   // o_t += S_k f_t over the tokens of segment k, 64 at a time; tile i + 1
@@ -311,22 +329,29 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
     __syncthreads();
   }
   cp_async_wait_all();
+  __syncthreads();  // R_k staged (last segment)
 
-  // S_T = S_k F_k + R_k (the product is already in TMEM)
+  // S_T = S_k F_k + R_k (the product is in TMEM): each thread adds its part in
+  // the R staging buffer, then the CTA copies the buffer out row by row.
   if (ok && last) {
-    float4 rk[16];
-    load_row64(R + k * mat + size_t(row) * D + 64 * hf, rk);
-    float* dst = p.S_T + size_t(chain) * mat + size_t(row) * D + 64 * hf;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      float v[32];
-      tmem_ld32(tlane + TM_ACC + 64 * hf + 32 * q, v);
+      const int col = 64 * hf + 32 * q;
+      float v[32], r[32];
+      lds_row32(rstage, row, col, r);
+      tmem_ld32(tlane + TM_ACC + col, v);
+      const uint32_t a = rstage + uint32_t(row) * PITCH + uint32_t(col) * 4u;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float4 a = rk[8 * q + e];
-        reinterpret_cast<float4*>(dst + 32 * q)[e] =
-            make_float4(v[4 * e] + a.x, v[4 * e + 1] + a.y, v[4 * e + 2] + a.z, v[4 * e + 3] + a.w);
-      }
+      for (int e = 0; e < 8; ++e)
+        sts4(a + 16u * e, make_float4(v[4 * e] + r[4 * e], v[4 * e + 1] + r[4 * e + 1],
+                                      v[4 * e + 2] + r[4 * e + 2], v[4 * e + 3] + r[4 * e + 3]));
+    }
+    __syncthreads();
+    float4* dst = reinterpret_cast<float4*>(p.S_T + size_t(chain) * mat);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int c = tid + NTHREADS * i;  // chunk: row c / 32, 16-byte column c % 32
+      dst[c] = lds4(rstage + uint32_t(c >> 5) * PITCH + uint32_t(c & 31) * 16u);
     }
   }
   tc_fence_before();
