@@ -97,6 +97,7 @@ constexpr uint32_t SM_BAR = SM_GATES + GATE_BUFS * GATE_BYTES;
 constexpr uint32_t SM_MISC = SM_BAR + 256;    // TMEM slot, abort flags, scan scratch, counters
 constexpr uint32_t SMEM_USED = SM_MISC + 256;
 static_assert(SM_A >= SM_DL + 16384, "K-side scratch overlaps the residual tiles");
+static_assert(SM_DL + 16384 - SM_XH == 65536, "X^T and Dl^T tiles form the 64 KB end-state staging area");
 static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 
 // mbarriers (8 bytes each, offsets inside SM_BAR)
@@ -785,23 +786,44 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           if (!rs.wait(x, x.bar(gfull_off(c + 1)), gfull_parity(c + 1))) return;
           gnext = x.gates(c + 1)[G_GC / 4];
         }
-        // this thread's 64 columns, 32 at a time: load, split, store hi / lo /
-        // pre-scaled fp32 in one waited group (or S_T to HBM after the last chunk)
+        if (final_chunk) {
+          // the end state goes out through the X^T / Dl^T region (64 KB, free once
+          // the o store has read it): rows of 512 B whose 16-byte chunks are
+          // XOR-swizzled by the row, then copied out row by row
+          if (leader) bulk_wait_read0();
+          named_bar(BAR_CHAIN, CHAIN_THREADS);
+          const uint32_t stg = sb + SM_XH;
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int col = 64 * ch + 32 * q;
-          float v[32];
-          tmem_ld32(tlane + TM_S + col, v);
-          uint32_t hi[16], lo[16], u[32];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
-          if (final_chunk) {
-            tmem_st16x2(tlane + TM_SHI + col / 2, hi, tlane + TM_SLO + col / 2, lo);
-            float4* dst = reinterpret_cast<float4*>(x.sdst + size_t(dv) * D + col);
+          for (int q = 0; q < 2; ++q) {
+            const int col = 64 * ch + 32 * q;
+            float v[32];
+            tmem_ld32(tlane + TM_S + col, v);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-          } else {
+              st_shared_v4(stg + uint32_t(dv) * 512u + uint32_t(((col / 4 + e) ^ (dv & 7)) * 16),
+                           __float_as_uint(v[4 * e]), __float_as_uint(v[4 * e + 1]),
+                           __float_as_uint(v[4 * e + 2]), __float_as_uint(v[4 * e + 3]));
+          }
+          named_bar(BAR_CHAIN, CHAIN_THREADS);
+          float4* dst = reinterpret_cast<float4*>(x.sdst);
+          const int ct = ch * 128 + dv;  // 0 .. 255 over the chain role
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int cidx = ct + CHAIN_THREADS * i;  // 16-byte chunk: row cidx / 32, column cidx % 32
+            const int r = cidx >> 5, j = cidx & 31;
+            dst[cidx] = *reinterpret_cast<const float4*>(x.sm + SM_XH + r * 512 + ((j ^ (r & 7)) * 16));
+          }
+        } else {
+          // this thread's 64 columns, 32 at a time: load, split, store hi / lo /
+          // pre-scaled fp32 in one waited group
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int col = 64 * ch + 32 * q;
+            float v[32];
+            tmem_ld32(tlane + TM_S + col, v);
+            uint32_t hi[16], lo[16], u[32];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(gnext * v[e]);
             tmem_st_state(tlane + TM_SHI + col / 2, hi, tlane + TM_SLO + col / 2, lo,
@@ -878,6 +900,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   x.tmem = *reinterpret_cast<volatile uint32_t*>(sm + SM_MISC + M_TMEM);
 
+  // a dependent launch (the segment fix) may begin its set-up now; it waits
+  // for this grid to complete before it reads anything this grid writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp < 4 || warp >= 12)
     chain_role<C>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
   else

@@ -227,9 +227,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   f.phase = 0;
   const uint32_t stage = f.sb + SSTAGE, rstage = f.sb + RSTAGE;
 
-  // Prologue: R_0 (= S_1) and F_1 stream into the two staging buffers.
-  stage_matrix(rstage, R);
-  if (nprod >= 1) stage_matrix(stage, F + mat);
+  // Prologue: set-up first (this grid may be launched before the first pass
+  // has finished), then wait for the first pass and stream R_0 (= S_1) and F_1
+  // into the two staging buffers.
   if (tid == 0) {
     mbar_init(f.bar, 1);
     fence_mbar_init();
@@ -238,6 +238,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
     tmem_alloc(smem_u32(sm + SM_BAR + 16), TMEM_COLS);
     tmem_relinquish();
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  stage_matrix(rstage, R);
+  if (nprod >= 1) stage_matrix(stage, F + mat);
   if (nprod >= 1) cp_async_wait_all_but_one(); else cp_async_wait_all();
   tc_fence_before();
   __syncthreads();  // R_0 staged, TMEM allocated
@@ -262,9 +265,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   // S_{j+1} = S_j F_j + R_j for j = 1 .. k-1; for the last segment also
   // S_k F_k, kept in TMEM for S_T.  F_{j+1} streams in during product j, and
   // R_{j+1} during the epilogue of product j + 1's predecessor.
+  // cp.async groups complete in commit order: F_j was committed before R_j,
+  // and R_j before F_{j+1}.
   for (int j = 1; ok && j <= nprod; ++j) {
-    cp_async_wait_all();
-    __syncthreads();                                   // F_j and R_j staged
+    if (need_r(j)) cp_async_wait_all_but_one(); else cp_async_wait_all();
+    __syncthreads();                                   // F_j staged (R_j may be in flight)
     split_staged_matrix(stage, f.sb + SF_HI, f.sb + SF_LO);
     fence_proxy_async_smem();
     __syncthreads();                                   // staging free, SF ready
@@ -274,7 +279,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
       mma_commit(f.bar);
     }
     if (j < nprod) stage_matrix(stage, F + (j + 1) * mat);
-    ok = f.wait_mma();
+    if (j < k) {                                       // R_j staged (F_{j+1} may be in flight)
+      if (j < nprod) cp_async_wait_all_but_one(); else cp_async_wait_all();
+    }
+    ok = f.wait_mma();                                 // (its barrier publishes R_j)
     if (!ok || j == k) break;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -367,8 +375,19 @@ int launch_segment_fix(const PrefillArgs& a, cudaStream_t stream) {
   const int ctas = a.B * a.H * (a.nseg - 1);
   const uint32_t smem = SMEM_USED + 1024;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(segment_fix_kernel), 2, int(smem))) return -1;
-  segment_fix_kernel<<<ctas, NTHREADS, smem, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+  // programmatic dependent launch: the kernel's set-up overlaps the end of the
+  // first pass; griddepcontrol.wait inside orders every access to its outputs
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(ctas));
+  cfg.blockDim = dim3(NTHREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, segment_fix_kernel, a) == cudaSuccess ? 0 : -1;
 }
 
 }  // namespace gdn
