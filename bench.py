@@ -386,6 +386,19 @@ def run_extras(args, dev, stream, flush, peaks, rank):
                                    "state_GB_per_s": round(sb / (t_warm / 1e3) / 1e9, 1),
                                    "l2": "warm: the 64 MiB state fits in the 126 MB L2"}}
     del dd, S
+    # a 4-token burst per sequence in one call (state read and written once)
+    dt = gin.prefill_inputs(wd.B, 4, wd.H, seed=2500 + rank, s0_std=0.02, device=str(dev))
+    S4 = dt["S0"].clone()
+    o4 = torch.empty((wd.B, 4, wd.H, D), dtype=torch.float32, device=dev)
+    ms = time_steps(lambda: gdn.decode_tokens(dt["q"], dt["k"], dt["v"], dt["g"], dt["beta"], S4,
+                                              o=o4), 32, 5, flush, stream)
+    t4 = statistics.mean(ms)
+    out["decode_b64_h16_t4"] = {
+        "us_per_call": round(t4 * 1e3, 3), "tokens_per_s": round(wd.B * 4 / (t4 / 1e3), 1),
+        "state_GB_per_s": round(sb / (t4 / 1e3) / 1e9, 1),
+        "l2": "flushed before every call",
+        "note": "4 tokens per sequence per call; the state crosses HBM once per call"}
+    del dt, S4, o4
     # large prefill (inputs 1.6 GB > L2)
     wl = gin.WORKLOADS["prefill_b4_h32_t32768"]
     dl = gin.workload_inputs(wl, seed=3000 + rank, device=str(dev))

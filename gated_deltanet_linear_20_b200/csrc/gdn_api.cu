@@ -330,18 +330,26 @@ int gdn_prefill_static_ws(const void* q, const void* k, const void* v, const flo
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                     const float* beta, float* S, float* o, int B, int H, int Dk, int Dv,
                     int* status, void* stream) {
+  return gdn_decode_tokens(q, k, v, g, beta, S, o, B, 1, H, Dk, Dv, status, stream);
+}
+
+int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
+                      int* status, void* stream) {
   (void)status;  // the decode kernel has no device-side waits
-  if (B < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (B < 0 || H < 0 || T < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim) return GDN_ERR_UNSUPPORTED;
   const long long heads = (long long)B * H;
-  if (heads * kHeadDim * kHeadDim > 0x7fffffffLL) return GDN_ERR_SHAPE;
-  if (heads == 0) return GDN_OK;
+  if (heads * kHeadDim * kHeadDim > 0x7fffffffLL || heads * T * kHeadDim > 0x7fffffffLL)
+    return GDN_ERR_SHAPE;
+  if (heads == 0 || T == 0) return GDN_OK;
   if (!q || !k || !v || !g || !beta || !S || !o) return GDN_ERR_NULL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(S, 16) ||
       !aligned(o, 16) || !aligned(g, 4) || !aligned(beta, 4))
     return GDN_ERR_ALIGN;
-  const size_t vec_bf16 = size_t(heads) * kHeadDim * 2, vec_f32 = size_t(heads) * kHeadDim * 4;
-  const size_t state_bytes = size_t(heads) * kHeadDim * kHeadDim * 4, gate_bytes = size_t(heads) * 4;
+  const size_t toks = size_t(heads) * T;
+  const size_t vec_bf16 = toks * kHeadDim * 2, vec_f32 = toks * kHeadDim * 4;
+  const size_t state_bytes = size_t(heads) * kHeadDim * kHeadDim * 4, gate_bytes = toks * 4;
   if (overlaps(o, vec_f32, q, vec_bf16) || overlaps(o, vec_f32, k, vec_bf16) ||
       overlaps(o, vec_f32, v, vec_bf16) || overlaps(o, vec_f32, g, gate_bytes) ||
       overlaps(o, vec_f32, beta, gate_bytes) || overlaps(o, vec_f32, S, state_bytes) ||
@@ -352,7 +360,7 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
   gdn::DecodeArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H};
+                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H, T};
   return gdn::launch_decode(a, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
 }
 

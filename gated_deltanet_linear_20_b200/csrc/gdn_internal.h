@@ -39,6 +39,7 @@ struct DecodeArgs {
   float* S;
   float* o;
   int B, H;
+  int T;  // tokens per sequence in this call (q, k, v, g, beta, o laid out [B][T][H])
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device

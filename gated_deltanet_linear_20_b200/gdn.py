@@ -39,6 +39,8 @@ _lib.gdn_prefill_schedule.argtypes = [_ci] * 4 + [_vp, _vp, _vp]
 _lib.gdn_prefill_schedule.restype = _ci
 _lib.gdn_decode_step.argtypes = [_vp] * 7 + [_ci] * 4 + [_vp, _vp]
 _lib.gdn_decode_step.restype = _ci
+_lib.gdn_decode_tokens.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp]
+_lib.gdn_decode_tokens.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
@@ -235,6 +237,36 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     return o
 
 
+def decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                  beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
+                  status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """T decode tokens per sequence in one call; S [B,H,Dv,Dk] fp32 is updated in
+    place (read and written once).  Returns o [B,T,H,Dv] fp32.
+
+    q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g, beta [B,T,H] fp32."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B,T,H,Dk]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn.decode_tokens runs on CUDA tensors only (no CPU path)")
+    _check(q, "q", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(k, "k", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(v, "v", torch.bfloat16, (B, T, H, Dv), dev)
+    _check(g, "g", torch.float32, (B, T, H), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    _check(S, "S", torch.float32, (B, H, Dv, Dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
+    rc = _lib.gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_decode_tokens")
+    return o
+
+
 def query_status(status: torch.Tensor) -> int:
     """Synchronises the current stream and returns the device status word."""
     return int(_lib.gdn_query_status(_ptr(status), _stream_handle(status.device)))
@@ -248,6 +280,10 @@ def raw_prefill(*args) -> int:
 
 def raw_prefill_ws(*args) -> int:
     return int(_lib.gdn_prefill_ws(*args))
+
+
+def raw_decode_tokens(*args) -> int:
+    return int(_lib.gdn_decode_tokens(*args))
 
 
 def raw_decode_step(*args) -> int:

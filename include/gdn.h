@@ -174,6 +174,22 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                     const float* beta, float* S, float* o, int B, int H, int Dk, int Dv,
                     int* status, void* stream);
 
+/* T decode tokens per sequence in one call (T = 1 is gdn_decode_step): the
+ * recurrence above applied to tokens 1..T in order, starting from S and
+ * leaving S_T in S.  The state is read once and written once, so a short burst
+ * costs one state round trip instead of T: e.g. the block of drafted tokens
+ * that speculative decoding verifies at once (the DFlash contribution guide,
+ * discosf.com/news/4742660, opening section: block drafts for speculative
+ * decoding).  For long T, gdn_prefill is faster.
+ *   q, k [B][T][H][Dk] bf16; v [B][T][H][Dv] bf16; g, beta [B][T][H] fp32 (device)
+ *   S    [B][H][Dv][Dk] fp32, updated in place (device)
+ *   o    [B][T][H][Dv] fp32, written (device)
+ *   Dk, Dv must be 128; B*H == 0 or T == 0 is a no-op.
+ * status and stream as for gdn_prefill.  Returns GDN_OK or a negative code. */
+int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
+                      int* status, void* stream);
+
 /* Synchronises `stream`, then reads the device status word written by the
  * kernels.  Returns GDN_OK, GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_NULL (status_dev is
  * NULL) or GDN_ERR_LAUNCH (the synchronisation or copy failed). */

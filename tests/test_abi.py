@@ -31,8 +31,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_workspace_bytes",
-              "gdn_prefill_schedule", "gdn_decode_step", "gdn_abi_version", "gdn_status_str",
-              "gdn_query_status"):
+              "gdn_prefill_schedule", "gdn_decode_step", "gdn_decode_tokens", "gdn_abi_version",
+              "gdn_status_str", "gdn_query_status"):
         assert n in names
 
 
@@ -161,6 +161,29 @@ def decode_args(**over):
 ], ids=lambda x: str(x))
 def test_decode_rejects_bad_arguments(gdn, over, code):
     assert gdn.raw_decode_step(*decode_args(**over)) == code
+
+
+def decode_tokens_args(**over):
+    a = dict(q=P, k=P + 0x1000000, v=P + 0x2000000, g=P + 0x3000000, beta=P + 0x3100000,
+             S=P + 0x4000000, o=P + 0x8000000, B=2, T=4, H=3, Dk=128, Dv=128, status=None,
+             stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "g", "beta", "S", "o", "B", "T", "H", "Dk", "Dv",
+                           "status", "stream")]
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(T=-1), -3), (dict(B=-1), -3), (dict(Dv=64), -4), (dict(k=None), -1),
+    (dict(o=P + 0x8000004), -2), (dict(o=P + 0x4000000 + 64), -5),
+    (dict(v=P + 0x4000000 + 4096), -5),     # v overlaps the state
+], ids=lambda x: str(x))
+def test_decode_tokens_rejects_bad_arguments(gdn, over, code):
+    assert gdn.raw_decode_tokens(*decode_tokens_args(**over)) == code
+
+
+def test_decode_tokens_empty_is_a_noop(gdn):
+    assert gdn.raw_decode_tokens(*decode_tokens_args(T=0)) == 0
+    assert gdn.raw_decode_tokens(*decode_tokens_args(B=0)) == 0
 
 
 def test_decode_empty_batch_is_a_noop(gdn):

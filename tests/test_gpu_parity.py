@@ -218,6 +218,47 @@ def test_decode_b64_h16_256_steps_sampled_sequences():
     assert_parity(S[bsel].cpu().numpy(), S_ref, "S after 256 steps")
 
 
+@pytest.mark.parametrize("T", [1, 2, 3, 8, 16, 33])
+def test_decode_tokens_against_oracle(T):
+    """T tokens per sequence in one call, state in place: o at every token and
+    the state after the burst against the oracle run from the same state."""
+    d = inputs.prefill_inputs(4, T, 8, seed=40 + T, s0_std=0.05)
+    dd = to_dev(d)
+    gdn = _gdn()
+    S = dd["S0"].clone()
+    o = gdn.decode_tokens(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], S)
+    torch.cuda.synchronize()
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o T={T}")
+    assert_parity(S.cpu().numpy(), rS, f"S T={T}")
+
+
+def test_decode_tokens_equals_repeated_steps():
+    """A burst of 5 equals 5 single steps (the same per-token arithmetic, summed
+    in another order by the burst kernel), and a burst of 1 is the step."""
+    d = to_dev(inputs.prefill_inputs(3, 5, 4, seed=77, s0_std=0.05))
+    gdn = _gdn()
+    S1 = d["S0"].clone()
+    o1 = gdn.decode_tokens(d["q"], d["k"], d["v"], d["g"], d["beta"], S1)
+    S2 = d["S0"].clone()
+    o2 = [gdn.decode_step(d["q"][:, t].contiguous(), d["k"][:, t].contiguous(),
+                          d["v"][:, t].contiguous(), d["g"][:, t].contiguous(),
+                          d["beta"][:, t].contiguous(), S2) for t in range(5)]
+    torch.cuda.synchronize()
+    assert_parity(S1.cpu().numpy(), S2.cpu().numpy(), "burst vs steps, S")
+    assert_parity(o1.cpu().numpy(), torch.stack(o2, 1).cpu().numpy(), "burst vs steps, o")
+    S3 = d["S0"].clone()
+    o3 = gdn.decode_tokens(d["q"][:, :1].contiguous(), d["k"][:, :1].contiguous(),
+                           d["v"][:, :1].contiguous(), d["g"][:, :1].contiguous(),
+                           d["beta"][:, :1].contiguous(), S3)
+    S4 = d["S0"].clone()
+    o4 = gdn.decode_step(d["q"][:, 0].contiguous(), d["k"][:, 0].contiguous(),
+                         d["v"][:, 0].contiguous(), d["g"][:, 0].contiguous(),
+                         d["beta"][:, 0].contiguous(), S4)
+    torch.cuda.synchronize()
+    assert torch.equal(S3, S4) and torch.equal(o3[:, 0], o4)
+
+
 def test_decode_equals_prefill_t1():
     d = inputs.prefill_inputs(3, 1, 5, seed=7, s0_std=0.1)
     dd = to_dev(d)
