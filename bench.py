@@ -30,6 +30,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -336,8 +337,10 @@ def run_extras(args, dev, stream, flush, peaks, rank):
     w = gin.WORKLOADS[args.workload]
     d = gin.workload_inputs(w, seed=1000 + rank, device=str(dev))
     other = 16 if args.chunk == 64 else 64
+    ws = torch.empty(max(gdn.workspace_bytes(w.B, w.T, w.H, other), 1), dtype=torch.uint8,
+                     device=dev)
     ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
-                                        chunk=other), steps, 3, flush, stream)
+                                        chunk=other, workspace=ws), steps, 3, flush, stream)
     t = statistics.mean(ms)
     out[f"{args.workload}/chunk{other}"] = {
         "tokens_per_s": round(w.B * w.T / (t / 1e3), 1), "ms": round(t, 5),
@@ -350,7 +353,7 @@ def run_extras(args, dev, stream, flush, peaks, rank):
         t = statistics.mean(ms)
         out[f"{args.workload}/chunk{c}/single_pass"] = {
             "tokens_per_s": round(w.B * w.T / (t / 1e3), 1), "ms": round(t, 5)}
-    del d
+    del d, ws
     # decode: L2 flushed before every step (headline) and 256 back-to-back steps (L2-warm)
     wd = gin.WORKLOADS["decode_b64_h16"]
     dd = gin.workload_inputs(wd, seed=2000 + rank, device=str(dev))
@@ -399,6 +402,25 @@ def run_extras(args, dev, stream, flush, peaks, rank):
         "l2": "flushed before every call",
         "note": "4 tokens per sequence per call; the state crosses HBM once per call"}
     del dt, S4, o4
+    # packed sequences of mixed lengths (one pass per sequence and head)
+    rng = np.random.default_rng(4000 + rank)
+    lens = rng.integers(64, 2049, size=32)
+    seqs = [gin.prefill_inputs(1, int(L), 16, seed=4100 + 37 * rank + i, device=str(dev))
+            for i, L in enumerate(lens)]
+    cat = lambda key: torch.cat([d[key][0] for d in seqs], 0)
+    pk = {key: cat(key) for key in ("q", "k", "v", "g", "beta")}
+    del seqs
+    cu = torch.tensor([0] + np.cumsum(lens).tolist(), dtype=torch.int32, device=dev)
+    ms = time_steps(lambda: gdn.prefill_varlen(pk["q"], pk["k"], pk["v"], pk["g"], pk["beta"], cu),
+                    steps, 3, flush, stream)
+    t = statistics.mean(ms)
+    ntok = int(lens.sum())
+    nb = prefill_bytes(1, ntok, 16, False) + (len(lens) - 1) * 16 * 65536
+    out["prefill_varlen_32seq_h16"] = {
+        "tokens": ntok, "lengths": "32 sequences, seeded uniform 64..2048",
+        "tokens_per_s": round(ntok / (t / 1e3), 1), "ms": round(t, 4),
+        "hbm_frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+    del pk, cu
     # large prefill (inputs 1.6 GB > L2)
     wl = gin.WORKLOADS["prefill_b4_h32_t32768"]
     dl = gin.workload_inputs(wl, seed=3000 + rank, device=str(dev))

@@ -169,7 +169,9 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
 
-  gdn::PrefillArgs a{g, beta, S0, o, S_T, B, T, H, status, 1, (T + 63) / 64, nullptr, nullptr, nullptr};
+  gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     B,      T,
+                     H,      status, 1,      (T + 63) / 64, nullptr, nullptr, nullptr,
+                     nullptr};
   if (allow_segments && T > 0) {
     int sms = 0;
     if (num_sms(&sms) != GDN_OK) return GDN_ERR_LAUNCH;
@@ -297,6 +299,53 @@ int gdn_prefill_ws(const void* q, const void* k, const void* v, const float* g,
                    int* status, void* stream) {
   return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, workspace,
                       workspace_bytes, true, status, stream);
+}
+
+int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* S0, float* o, float* S_T,
+                       const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
+                       int chunk, int* status, void* stream) {
+  if (N < 0 || total_T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
+  const long long chains = (long long)N * H;
+  const long long act = (long long)total_T * H * kHeadDim;
+  if (act > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  if (chains == 0) return GDN_OK;
+  if (!S_T || !cu_seqlens) return GDN_ERR_NULL;
+  if (total_T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
+  if (!aligned(S_T, 16) || (S0 && !aligned(S0, 16)) || !aligned(cu_seqlens, 4)) return GDN_ERR_ALIGN;
+  if (total_T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+                      !aligned(g, 4) || !aligned(beta, 4)))
+    return GDN_ERR_ALIGN;
+  const size_t act_bf16 = size_t(act) * 2, act_f32 = size_t(act) * 4;
+  const size_t gate_bytes = size_t(total_T) * H * 4;
+  const size_t state_bytes = size_t(chains) * kHeadDim * kHeadDim * 4, cu_bytes = size_t(N + 1) * 4;
+  if (total_T > 0 && (overlaps(o, act_f32, q, act_bf16) || overlaps(o, act_f32, k, act_bf16) ||
+                      overlaps(o, act_f32, v, act_bf16) || overlaps(o, act_f32, g, gate_bytes) ||
+                      overlaps(o, act_f32, beta, gate_bytes) || overlaps(o, act_f32, S0, state_bytes) ||
+                      overlaps(o, act_f32, S_T, state_bytes) || overlaps(o, act_f32, cu_seqlens, cu_bytes)))
+    return GDN_ERR_ALIAS;
+  if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
+  if (overlaps(S_T, state_bytes, cu_seqlens, cu_bytes)) return GDN_ERR_ALIAS;
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+
+  // B = N chains of sequences, T = total_T: the views are [1][total_T][H][128]
+  gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
+                     H,      status, 1,      (total_T + 63) / 64, nullptr, nullptr, nullptr,
+                     cu_seqlens};
+  CUtensorMap tq{}, tk{}, tv{}, to{};
+  const int Tv = total_T > 0 ? total_T : 1;  // a valid (never read) view when every sequence is empty
+  const void* qv = total_T > 0 ? q : S_T;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (!encode_act(&tq, qv, 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
+      !encode_act(&tk, total_T > 0 ? k : S_T, 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
+      !encode_act(&tv, total_T > 0 ? v : S_T, 1, Tv, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2) ||
+      !encode_act(&to, total_T > 0 ? static_cast<const void*>(o) : S_T, 1, Tv, H, 128,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4))
+    return GDN_ERR_LAUNCH;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return gdn::launch_prefill(tq, tk, tv, to, to, a, chunk, st) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
 }
 
 int gdn_prefill_static_ws(const void* q, const void* k, const void* v, const float* g,

@@ -28,6 +28,10 @@ struct PrefillArgs {
   float* ws_f;      // f_t of the F CTAs, laid out like o            [B][T][H][128]
   float* ws_R;      // end state of each R CTA                         [B*H][nseg][128][128]
   float* ws_F;      // transfer matrix of each F CTA (slot 0 unused)   [B*H][nseg][128][128]
+  // Packed sequences (or null): B sequences of lengths cu[n+1] - cu[n] packed
+  // along T (the views then have one batch entry); chain n H + h walks
+  // tokens [cu[n], cu[n+1]).
+  const int* cu_seqlens;
 };
 
 struct DecodeArgs {

@@ -138,8 +138,11 @@ struct Ctx {
   uint32_t sb;        // shared-window address of sm
   uint32_t tmem;      // TMEM base (lane 0, column 0)
   int* status;
+  int H;
   volatile int* abort_flag;
-  int tb;              // first tile (of the chain) this CTA walks
+  int tok0;            // token coordinate (in the TMA views) of this CTA's first tile
+  int tend;            // first token coordinate past this CTA's sequence: padding from there on
+  int tmap;            // token extent of the TMA views (T, or the packed total)
   bool vzero;          // v taken as zero (transfer-matrix CTA of the segmented schedule)
   bool s0_identity;    // start from the identity instead of s0src / zeros
   const float* s0src;  // start state of this chain [128][128], or null
@@ -198,7 +201,7 @@ __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, co
   const uint32_t kq = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
   const uint32_t bar = x.bar((c & 1) ? B_FULL1 : B_FULL0);
   mbar_arrive_expect_tx(bar, KQ_TX_BYTES);
-  const int t0 = (x.tb + c) * NT;
+  const int t0 = x.tok0 + c * NT;
   tma_load_4d(kq + 0, tk, bar, 0, h, t0, b);
   tma_load_4d(kq + 8192, tq, bar, 0, h, t0, b);
   tma_load_4d(kq + 16384, tk, bar, 64, h, t0, b);
@@ -208,7 +211,7 @@ __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, co
 __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b) {
   const uint32_t bar = x.bar(B_VFULL);
   mbar_arrive_expect_tx(bar, V_TX_BYTES);
-  tma_load_4d(x.sb + SM_V, tv, bar, 0, h, (x.tb + c) * NT, b);
+  tma_load_4d(x.sb + SM_V, tv, bar, 0, h, x.tok0 + c * NT, b);
   *x.misc(M_V_ISSUED) = c + 1;
 }
 
@@ -289,8 +292,8 @@ __device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, f
     const float bc = b_next;
     g_next = 0.f;
     b_next = 0.f;
-    const int t = (x.tb + c + 1) * NT + kt;
-    if (t < T) {
+    const int t = x.tok0 + (c + 1) * NT + kt;
+    if (t < x.tend) {  // tokens past the sequence are padding: g = beta = 0, an exact identity
       const size_t gi = (size_t(b) * T + t) * H + h;
       g_next = __ldg(p.g + gi);
       b_next = __ldg(p.beta + gi);
@@ -335,6 +338,18 @@ __device__ __forceinline__ void issue_p(const Ctx& x, int c) {
   mma_commit(x.bar(B_PFULL));
 }
 
+// Copies rows 0 .. nvalid-1 of the staged fp32 o tile (rows of 128 floats) to
+// dst (row r at dst + r H 128), thread ct of the chain role taking every
+// CHAIN_THREADS-th 16-byte chunk.  Kept out of line: it runs only for the last
+// tile of a packed sequence.
+__device__ __noinline__ void store_partial_tile(const float4* src, float* dst, int H, int nvalid,
+                                                int ct) {
+  for (int i = ct; i < nvalid * (D / 4); i += CHAIN_THREADS) {
+    const int r = i / (D / 4), j = i % (D / 4);
+    reinterpret_cast<float4*>(dst + size_t(r) * H * D)[j] = src[i];
+  }
+}
+
 // o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] of tile c.  This thread's 32
 // tokens (32 hf ..) of lane dv go into an fp32 [64 tokens][128] tile in the
 // X^T region, which is free between the state update and the next X epilogue;
@@ -362,9 +377,19 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
   }
   fence_proxy_async_smem();
   named_bar(BAR_CHAIN, CHAIN_THREADS);
-  if (leader) {
-    tma_store_4d(x.tmo, x.sb + SM_XH, 0, h, (x.tb + c) * NT, b);
-    bulk_commit();
+  const int ts = x.tok0 + c * NT;
+  if (ts + NT <= x.tend || x.tend == x.tmap) {
+    // whole tile, or the view's own end clips it
+    if (leader) {
+      tma_store_4d(x.tmo, x.sb + SM_XH, 0, h, ts, b);
+      bulk_commit();
+    }
+  } else {
+    // last tile of a packed sequence: the rows past it belong to the next
+    // sequence, so only the valid rows are copied out
+    store_partial_tile(reinterpret_cast<const float4*>(x.sm + SM_XH),
+                       x.odst + ((size_t(b) * x.tmap + ts) * x.H + h) * D, x.H, x.tend - ts,
+                       hf * 128 + dv);
   }
 }
 
@@ -391,8 +416,8 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
     if (!x.vzero) issue_v(x, tv, 0, h, b);
   }
   float g_next = 0.f, b_next = 0.f;
-  if (kt < NT && x.tb * NT + kt < T) {
-    const size_t gi = (size_t(b) * T + x.tb * NT + kt) * p.H + h;
+  if (kt < NT && x.tok0 + kt < x.tend) {
+    const size_t gi = (size_t(b) * T + x.tok0 + kt) * p.H + h;
     g_next = __ldg(p.g + gi);
     b_next = __ldg(p.beta + gi);
   }
@@ -859,7 +884,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     frun = j >= p.nseg;
     seg = frun ? j - p.nseg + 1 : j;
   }
-  const int b = chain / p.H;
+  int b = chain / p.H;
   const int h = chain - b * p.H;
   const size_t cstate = size_t(chain) * D * D;
 
@@ -867,17 +892,40 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   x.sm = sm;
   x.sb = smem_u32(sm);
   x.status = p.status;
+  x.H = p.H;
   x.abort_flag = reinterpret_cast<volatile int*>(sm + SM_MISC + M_ABORT);
-  x.tb = 0;
+  x.tok0 = 0;
+  x.tend = p.T;
+  x.tmap = p.T;
+  int ntiles = total_tiles;
+  if (p.cu_seqlens) {
+    // packed sequences: chain = n H + h walks tokens [cu[n], cu[n+1]) of views with B = 1
+    const int start = __ldg(p.cu_seqlens + b), end = __ldg(p.cu_seqlens + b + 1);
+    if (start < 0 || end < start || end > p.T) {
+      if (tid == 0 && p.status) atomicExch(p.status, GDN_ERR_SHAPE);
+      return;
+    }
+    x.tok0 = start;
+    x.tend = end;
+    b = 0;
+    ntiles = (end - start + NT - 1) / NT;
+    if (ntiles == 0) {  // empty sequence: S_T = S0 (or zeros)
+      const float4* src = p.S0 ? reinterpret_cast<const float4*>(p.S0 + cstate) : nullptr;
+      float4* dst = reinterpret_cast<float4*>(p.S_T + cstate);
+      for (int i = tid; i < D * D / 4; i += NTHREADS)
+        dst[i] = src ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      return;
+    }
+  }
   x.vzero = frun;
   x.s0_identity = frun;
   x.s0src = (seg == 0 && p.S0) ? p.S0 + cstate : nullptr;
   x.odst = frun ? p.ws_f : p.o;
   x.tmo = frun ? &tm_f : &tm_o;
-  int ntiles = total_tiles;
   if (p.nseg > 1) {
-    x.tb = seg * p.seg_tiles;
-    ntiles = min(p.seg_tiles, total_tiles - x.tb);
+    const int tb = seg * p.seg_tiles;
+    x.tok0 = tb * NT;
+    ntiles = min(p.seg_tiles, total_tiles - tb);
     x.sdst = (frun ? p.ws_F : p.ws_R) + (size_t(chain) * p.nseg + seg) * D * D;
   } else {
     x.sdst = p.S_T + cstate;

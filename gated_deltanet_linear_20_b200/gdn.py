@@ -33,6 +33,8 @@ _lib.gdn_prefill_workspace_bytes.argtypes = [_ci] * 6
 _lib.gdn_prefill_workspace_bytes.restype = ctypes.c_size_t
 _lib.gdn_prefill_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, ctypes.c_size_t, _vp, _vp]
 _lib.gdn_prefill_ws.restype = _ci
+_lib.gdn_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 6 + [_vp, _vp]
+_lib.gdn_prefill_varlen.restype = _ci
 _lib.gdn_prefill_static_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, _vp]
 _lib.gdn_prefill_static_ws.restype = _ci
 _lib.gdn_prefill_schedule.argtypes = [_ci] * 4 + [_vp, _vp, _vp]
@@ -173,6 +175,48 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     return o, S_T
 
 
+def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                   beta: torch.Tensor, cu_seqlens: torch.Tensor, S0: Optional[torch.Tensor] = None,
+                   chunk: int = 64, *, o: Optional[torch.Tensor] = None,
+                   S_T: Optional[torch.Tensor] = None,
+                   status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Prefill of N packed sequences: q, k [total_T,H,Dk] bf16; v [total_T,H,Dv] bf16;
+    g, beta [total_T,H] fp32; cu_seqlens int32 [N+1] on the device (offsets of
+    the sequences).  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,Dk] fp32)."""
+    if q.dim() != 3:
+        raise ValueError("q must be [total_T,H,Dk]")
+    total_T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn.prefill_varlen runs on CUDA tensors only (no CPU path)")
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be [N+1]")
+    N = cu_seqlens.numel() - 1
+    _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+    _check(q, "q", torch.bfloat16, (total_T, H, Dk), dev)
+    _check(k, "k", torch.bfloat16, (total_T, H, Dk), dev)
+    _check(v, "v", torch.bfloat16, (total_T, H, Dv), dev)
+    _check(g, "g", torch.float32, (total_T, H), dev)
+    _check(beta, "beta", torch.float32, (total_T, H), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (N, H, Dv, Dk), dev)
+    if o is None:
+        o = torch.empty((total_T, H, Dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.float32, (total_T, H, Dv), dev)
+    if S_T is None:
+        S_T = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=dev)
+    _check(S_T, "S_T", torch.float32, (N, H, Dv, Dk), dev)
+    if status is not None:
+        _check(status, "status", torch.int32, (1,), dev)
+    rc = _lib.gdn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                 _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk, Dv, int(chunk),
+                                 _ptr(status), _stream_handle(dev))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_prefill_varlen")
+    return o, S_T
+
+
 def prefill_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                    beta: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64, *,
                    o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
@@ -276,6 +320,10 @@ def raw_prefill(*args) -> int:
     """Direct call of the C entry point with raw integers/pointers (tests use it
     to exercise argument validation without any tensor)."""
     return int(_lib.gdn_prefill(*args))
+
+
+def raw_prefill_varlen(*args) -> int:
+    return int(_lib.gdn_prefill_varlen(*args))
 
 
 def raw_prefill_ws(*args) -> int:

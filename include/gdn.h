@@ -110,6 +110,27 @@ int gdn_prefill(const void* q, const void* k, const void* v, const float* g, con
  * give 0 too; gdn_prefill_ws then reports them. */
 size_t gdn_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chunk);
 
+/* Prefill of N sequences of different lengths packed along the token axis
+ * (no padding between them): sequence n is tokens cu_seqlens[n] ..
+ * cu_seqlens[n+1]-1 of the packed arrays.  The recurrence and its chunked form
+ * are those of gdn_prefill, per sequence and head; the pages' prefill note
+ * works on one sequence at a time, and packing is how a serving batch arrives.
+ *   q, k [total_T][H][Dk] bf16; v [total_T][H][Dv] bf16; g, beta [total_T][H]
+ *   fp32; o [total_T][H][Dv] fp32 (device)
+ *   S0, S_T [N][H][Dv][Dk] fp32 (S0 may be NULL; S_T may equal S0) (device)
+ *   cu_seqlens : device int[N+1], cu_seqlens[0] = 0, non-decreasing,
+ *                cu_seqlens[N] = total_T.  A sequence whose offsets are out of
+ *                order or past total_T is detected on the device: GDN_ERR_SHAPE
+ *                goes to *status and that sequence's outputs are not written.
+ *                Empty sequences are allowed (S_T = S0, or zeros).
+ *   N, total_T, H : sequences, packed tokens, heads.  One pass per (sequence,
+ *                head); the segmented schedule of gdn_prefill_ws is not used.
+ * chunk, status, stream and the other rules as for gdn_prefill. */
+int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* S0, float* o, float* S_T,
+                       const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
+                       int chunk, int* status, void* stream);
+
 /* The schedule gdn_prefill_ws picks for B*H chains of T tokens on a device
  * with num_sms multiprocessors (no device is touched): *nseg segments per chain
  * (1: the single pass of gdn_prefill) of *seg_tiles 64-token tiles each (the

@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_workspace_bytes",
+    for n in ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_varlen", "gdn_prefill_workspace_bytes",
               "gdn_prefill_schedule", "gdn_decode_step", "gdn_decode_tokens", "gdn_abi_version",
               "gdn_status_str", "gdn_query_status"):
         assert n in names
@@ -145,6 +145,30 @@ def test_schedule_rejects_bad_sizes(gdn):
         gdn.schedule(-1, 64, 1, 148)
     assert gdn.schedule(1, 512, 16, 0)[0] == 1     # no multiprocessor count: single pass
     assert gdn.schedule(0, 512, 16, 148)[0] == 1
+
+
+def varlen_args(**over):
+    a = dict(q=P, k=P + 0x10000000, v=P + 0x20000000, g=P + 0x30000000, beta=P + 0x31000000,
+             S0=None, o=P + 0x40000000, S_T=P + 0x50000000, cu=P + 0x60000000, N=3, total_T=200,
+             H=2, Dk=128, Dv=128, chunk=64, status=None, stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "g", "beta", "S0", "o", "S_T", "cu", "N", "total_T",
+                           "H", "Dk", "Dv", "chunk", "status", "stream")]
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(N=-1), -3), (dict(total_T=-1), -3), (dict(Dk=64), -4), (dict(chunk=8), -4),
+    (dict(cu=None), -1), (dict(S_T=None), -1), (dict(q=None), -1),
+    (dict(cu=P + 0x60000002), -2), (dict(o=P + 0x40000008), -2),
+    (dict(o=P + 0x60000000 - 64), -5),          # o runs into cu_seqlens
+    (dict(S_T=P + 0x60000000 - 64 * 1024), -5),  # S_T runs into cu_seqlens
+], ids=lambda x: str(x))
+def test_prefill_varlen_rejects_bad_arguments(gdn, over, code):
+    assert gdn.raw_prefill_varlen(*varlen_args(**over)) == code
+
+
+def test_prefill_varlen_no_sequences_is_a_noop(gdn):
+    assert gdn.raw_prefill_varlen(*varlen_args(N=0, q=None, S_T=None)) == 0
 
 
 def decode_args(**over):

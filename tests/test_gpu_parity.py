@@ -197,6 +197,66 @@ def test_segmented_workspace_errors():
     assert e.value.code == gdn.GDN_ERR_ALIAS
 
 
+def packed(lengths, H, seed, s0_std=None, g_mean=0.0):
+    """Packed inputs of sequences of the given lengths: per-sequence draws of
+    the seeded generator, concatenated along tokens."""
+    seqs = [inputs.prefill_inputs(1, L, H, seed=seed + i, g_mean=g_mean, s0_std=s0_std)
+            for i, L in enumerate(lengths)]
+    cat = lambda key: torch.cat([d[key][0] for d in seqs], 0)
+    S0 = torch.cat([d["S0"] for d in seqs], 0) if s0_std else None
+    cu = torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32)
+    return seqs, dict(q=cat("q"), k=cat("k"), v=cat("v"), g=cat("g"), beta=cat("beta"), S0=S0, cu=cu)
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+@pytest.mark.parametrize("s0", [None, 0.05])
+def test_varlen_packed_sequences(chunk, s0):
+    """Packed sequences of mixed lengths (empty, 1 token, ragged, tile-aligned),
+    each against the oracle run on that sequence alone."""
+    lengths = [130, 0, 1, 64, 200, 17, 63, 65]
+    H = 3
+    seqs, pk = packed(lengths, H, seed=90, s0_std=s0)
+    gdn = _gdn()
+    dd = to_dev(pk)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"], dd["S0"],
+                                chunk=chunk, status=status)
+    assert gdn.query_status(status) == 0
+    o, S_T = o.cpu().numpy(), S_T.cpu().numpy()
+    cu = pk["cu"].numpy()
+    for n, d in enumerate(seqs):
+        ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+        if lengths[n]:
+            assert_parity(o[cu[n]:cu[n + 1]], ro[0], f"o seq {n} (len {lengths[n]})")
+        assert_parity(S_T[n], rS[0], f"S_T seq {n} (len {lengths[n]})") if (s0 or lengths[n]) else \
+            np.testing.assert_array_equal(S_T[n], 0.0)
+
+
+def test_varlen_equal_lengths_match_the_dense_call():
+    """Equal lengths packed = the dense [B][T][H] call, bitwise (the same CTAs
+    on the same tiles; only the token coordinates differ)."""
+    B, T, H = 3, 150, 4
+    d = to_dev(inputs.prefill_inputs(B, T, H, seed=8, s0_std=0.05))
+    gdn = _gdn()
+    o1, S1 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], segmented=False)
+    cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=DEV)
+    flat = lambda x: x.reshape(B * T, *x.shape[2:]).contiguous()
+    o2, S2 = gdn.prefill_varlen(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["g"]),
+                                flat(d["beta"]), cu, d["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(o1.reshape(B * T, H, 128), o2) and torch.equal(S1, S2)
+
+
+def test_varlen_bad_offsets_are_reported_on_the_device():
+    _, pk = packed([40, 40], 2, seed=3)
+    gdn = _gdn()
+    dd = to_dev(pk)
+    bad = torch.tensor([0, 50, 30], dtype=torch.int32, device=DEV)  # out of order
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gdn.prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], bad, status=status)
+    assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
+
+
 def test_decode_b64_h16_256_steps_sampled_sequences():
     """256 in-place decode steps of the full batch on the GPU; sequences 0, 21,
     42, 63 (all 16 heads) checked against the oracle at every step."""
