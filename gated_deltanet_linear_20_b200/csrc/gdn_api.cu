@@ -171,7 +171,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
 
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     B,      T,
                      H,      status, 1,      (T + 63) / 64, nullptr, nullptr, nullptr,
-                     nullptr};
+                     nullptr, nullptr, 0,      0};
   if (allow_segments && T > 0) {
     int sms = 0;
     if (num_sms(&sms) != GDN_OK) return GDN_ERR_LAUNCH;
@@ -304,9 +304,11 @@ int gdn_prefill_ws(const void* q, const void* k, const void* v, const float* g,
 int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
                        const float* beta, const float* S0, float* o, float* S_T,
                        const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
-                       int chunk, int* status, void* stream) {
-  if (N < 0 || total_T < 0 || H < 0) return GDN_ERR_SHAPE;
+                       int chunk, float* snaps, int snap_every, int n_snaps, int* status,
+                       void* stream) {
+  if (N < 0 || total_T < 0 || H < 0 || n_snaps < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
+  if (snaps && (snap_every <= 0 || snap_every % 64 != 0)) return GDN_ERR_UNSUPPORTED;
   const long long chains = (long long)N * H;
   const long long act = (long long)total_T * H * kHeadDim;
   if (act > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL) return GDN_ERR_SHAPE;
@@ -327,13 +329,24 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
     return GDN_ERR_ALIAS;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
   if (overlaps(S_T, state_bytes, cu_seqlens, cu_bytes)) return GDN_ERR_ALIAS;
+  if (snaps) {
+    const size_t snap_bytes = size_t(n_snaps) * H * kHeadDim * kHeadDim * 4;
+    if (!aligned(snaps, 16)) return GDN_ERR_ALIGN;
+    if ((total_T > 0 && overlaps(snaps, snap_bytes, o, act_f32)) ||
+        overlaps(snaps, snap_bytes, S_T, state_bytes) || overlaps(snaps, snap_bytes, S0, state_bytes) ||
+        overlaps(snaps, snap_bytes, cu_seqlens, cu_bytes) ||
+        (total_T > 0 && (overlaps(snaps, snap_bytes, q, act_bf16) || overlaps(snaps, snap_bytes, k, act_bf16) ||
+                         overlaps(snaps, snap_bytes, v, act_bf16) || overlaps(snaps, snap_bytes, g, gate_bytes) ||
+                         overlaps(snaps, snap_bytes, beta, gate_bytes))))
+      return GDN_ERR_ALIAS;
+  }
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
 
   // B = N chains of sequences, T = total_T: the views are [1][total_T][H][128]
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
                      H,      status, 1,      (total_T + 63) / 64, nullptr, nullptr, nullptr,
-                     cu_seqlens};
+                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0};
   CUtensorMap tq{}, tk{}, tv{}, to{};
   const int Tv = total_T > 0 ? total_T : 1;  // a valid (never read) view when every sequence is empty
   const void* qv = total_T > 0 ? q : S_T;

@@ -32,6 +32,12 @@ struct PrefillArgs {
   // along T (the views then have one batch entry); chain n H + h walks
   // tokens [cu[n], cu[n+1]).
   const int* cu_seqlens;
+  // State snapshots (packed sequences only; snaps == null: none): the state
+  // after every snap_every tokens (a multiple of 64) of each sequence, at
+  // snaps[(k_n + j) H + h] with k_n = sum over earlier sequences m of
+  // len_m / snap_every; n_snaps slots in all.
+  float* snaps;
+  int snap_every, n_snaps;
 };
 
 struct DecodeArgs {

@@ -113,8 +113,10 @@ __device__ __forceinline__ uint32_t gfull_parity(int c) { return uint32_t(c >> 2
 // misc slots (offsets inside SM_MISC)
 constexpr uint32_t M_TMEM = 0, M_ABORT = 4, M_PART = 8, M_KQ_ISSUED = 12, M_KQ_SEEN = 16,
                    M_V_ISSUED = 20, M_V_SEEN = 24, M_FLAG_CHAIN = 32,
-                   M_FLAG_SIDE = 40;  // two verdict slots per role
-static_assert(M_FLAG_SIDE + 8 <= 256, "misc slots");
+                   M_FLAG_SIDE = 40,  // two verdict slots per role
+                   M_SNAP_TILES = 48,  // tiles between state snapshots (0: none)
+                   M_SNAP_PTR = 56;    // this chain's first snapshot slot (8 bytes)
+static_assert(M_SNAP_PTR + 8 <= 64, "misc slots (the first 64 bytes are cleared at start)");
 static_assert(8 * NUM_BARS <= 256, "barrier slots");
 
 constexpr uint32_t KQ_TX_BYTES = 4 * 8192;
@@ -549,6 +551,33 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
+// Copies columns col0 .. col0+63 of this lane's state row (fp32, TMEM) to
+// dst_row + col0.  Out of line: it runs only at snapshot tile ends.
+__device__ __noinline__ void snapshot_row(uint32_t tlane, int col0, float* dst_row) {
+#pragma unroll 1
+  for (int q = 0; q < 2; ++q) {
+    float v[32];
+    tmem_ld32(tlane + TM_S + col0 + 32 * q, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      reinterpret_cast<float4*>(dst_row + col0 + 32 * q)[e] =
+          make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+  }
+}
+
+// Copies the staged 128 x 128 fp32 state (rows of 512 B, 16-byte chunks
+// XOR-swizzled by the row) to dst, row by row: chain thread ct takes every
+// CHAIN_THREADS-th chunk.
+__device__ __noinline__ void copy_staged_state(const uint8_t* stg, float* dst, int ct) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll 4
+  for (int i = 0; i < 16; ++i) {
+    const int cidx = ct + CHAIN_THREADS * i;  // 16-byte chunk: row cidx / 32, column cidx % 32
+    const int r = cidx >> 5, j = cidx & 31;
+    d4[cidx] = *reinterpret_cast<const float4*>(stg + r * 512 + ((j ^ (r & 7)) * 16));
+  }
+}
+
 // Z = S_c K^T (into TM_Z) and Y = S_c Q^T (into TM_Y) for chunk s of the tile
 // in `kq`: A = the bf16 hi / lo state pair in TMEM, B = K and Q rows.  With
 // chunk 64 the K and Q rows of the tile are adjacent (64 + 64 rows) and Y sits
@@ -830,15 +859,24 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
                            __float_as_uint(v[4 * e + 2]), __float_as_uint(v[4 * e + 3]));
           }
           named_bar(BAR_CHAIN, CHAIN_THREADS);
-          float4* dst = reinterpret_cast<float4*>(x.sdst);
-          const int ct = ch * 128 + dv;  // 0 .. 255 over the chain role
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int cidx = ct + CHAIN_THREADS * i;  // 16-byte chunk: row cidx / 32, column cidx % 32
-            const int r = cidx >> 5, j = cidx & 31;
-            dst[cidx] = *reinterpret_cast<const float4*>(x.sm + SM_XH + r * 512 + ((j ^ (r & 7)) * 16));
+          copy_staged_state(x.sm + SM_XH, x.sdst, ch * 128 + dv);
+          const int stiles = *x.misc(M_SNAP_TILES);
+          if (stiles && (x.tend - x.tok0) % (stiles * NT) == 0) {
+            // the sequence ends on a snapshot boundary: its last snapshot is S_T
+            float* snap = *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR);
+            copy_staged_state(x.sm + SM_XH,
+                              snap + size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * D * D,
+                              ch * 128 + dv);
           }
         } else {
+          // at a snapshot tile end, the state itself first goes to its slot
+          if (s == NSUB - 1) {
+            const int stiles = *x.misc(M_SNAP_TILES);
+            if (stiles && (c + 1) % stiles == 0) {
+              float* snap = *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR);
+              snapshot_row(tlane, 64 * ch, snap + (size_t((c + 1) / stiles - 1) * x.H * D + dv) * D);
+            }
+          }
           // this thread's 64 columns, 32 at a time: load, split, store hi / lo /
           // pre-scaled fp32 in one waited group
 #pragma unroll
@@ -938,6 +976,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(x.sb + SM_BAR + 8 * i, 1);
     fence_mbar_init();
     for (int i = 0; i < 16; ++i) reinterpret_cast<volatile int*>(sm + SM_MISC)[i] = 0;
+    if (p.snaps && p.cu_seqlens) {
+      // first snapshot slot of this sequence: one per snap_every tokens of
+      // every earlier sequence
+      const int n = chain / p.H;
+      int base = 0;
+      for (int m = 0; m < n; ++m)
+        base += (__ldg(p.cu_seqlens + m + 1) - __ldg(p.cu_seqlens + m)) / p.snap_every;
+      if (base + (x.tend - x.tok0) / p.snap_every > p.n_snaps) {  // too few slots
+        if (p.status) atomicExch(p.status, GDN_ERR_SHAPE);
+      } else {
+        *reinterpret_cast<float* volatile*>(sm + SM_MISC + M_SNAP_PTR) =
+            p.snaps + (size_t(base) * p.H + h) * D * D;
+        *x.misc(M_SNAP_TILES) = p.snap_every / NT;
+      }
+    }
   }
   if (warp == 0) {
     tmem_alloc(smem_u32(sm + SM_MISC + M_TMEM), TMEM_COLS);

@@ -33,7 +33,7 @@ _lib.gdn_prefill_workspace_bytes.argtypes = [_ci] * 6
 _lib.gdn_prefill_workspace_bytes.restype = ctypes.c_size_t
 _lib.gdn_prefill_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, ctypes.c_size_t, _vp, _vp]
 _lib.gdn_prefill_ws.restype = _ci
-_lib.gdn_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 6 + [_vp, _vp]
+_lib.gdn_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 6 + [_vp, _ci, _ci, _vp, _vp]
 _lib.gdn_prefill_varlen.restype = _ci
 _lib.gdn_prefill_static_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, _vp]
 _lib.gdn_prefill_static_ws.restype = _ci
@@ -46,7 +46,7 @@ _lib.gdn_decode_tokens.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
-ABI_VERSION = 2
+ABI_VERSION = 3
 if _lib.gdn_abi_version() != ABI_VERSION:
     raise ImportError(f"libgdn_b200.so ABI {_lib.gdn_abi_version()} != binding ABI {ABI_VERSION}")
 
@@ -178,11 +178,16 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
 def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                    beta: torch.Tensor, cu_seqlens: torch.Tensor, S0: Optional[torch.Tensor] = None,
                    chunk: int = 64, *, o: Optional[torch.Tensor] = None,
-                   S_T: Optional[torch.Tensor] = None,
-                   status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+                   S_T: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                   snap_every: int = 0,
+                   snaps: Optional[torch.Tensor] = None):
     """Prefill of N packed sequences: q, k [total_T,H,Dk] bf16; v [total_T,H,Dv] bf16;
     g, beta [total_T,H] fp32; cu_seqlens int32 [N+1] on the device (offsets of
-    the sequences).  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,Dk] fp32)."""
+    the sequences).  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,Dk] fp32).
+    With ``snap_every`` (a multiple of 64) it also returns the state snapshots
+    [n_snaps,H,Dv,Dk] (after every snap_every tokens of each sequence, sequence
+    by sequence); ``snaps`` may be given preallocated, else its size is read
+    from cu_seqlens (one device-to-host copy)."""
     if q.dim() != 3:
         raise ValueError("q must be [total_T,H,Dk]")
     total_T, H, Dk = q.shape
@@ -209,12 +214,23 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     _check(S_T, "S_T", torch.float32, (N, H, Dv, Dk), dev)
     if status is not None:
         _check(status, "status", torch.int32, (1,), dev)
+    n_snaps = 0
+    if snap_every:
+        if snaps is None:
+            lens = (cu_seqlens[1:] - cu_seqlens[:-1]).cpu()
+            n_snaps = int((lens // int(snap_every)).sum())
+            snaps = torch.empty((n_snaps, H, Dv, Dk), dtype=torch.float32, device=dev)
+        n_snaps = snaps.shape[0]
+        _check(snaps, "snaps", torch.float32, (n_snaps, H, Dv, Dk), dev)
+    else:
+        snaps = None
     rc = _lib.gdn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
                                  _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk, Dv, int(chunk),
-                                 _ptr(status), _stream_handle(dev))
+                                 _ptr(snaps), int(snap_every), n_snaps, _ptr(status),
+                                 _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_prefill_varlen")
-    return o, S_T
+    return (o, S_T) if snaps is None else (o, S_T, snaps)
 
 
 def prefill_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,

@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 2
+#define GDN_ABI_VERSION 3
 
 enum gdn_status_code {
   GDN_OK = 0,
@@ -125,11 +125,22 @@ size_t gdn_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chun
  *                Empty sequences are allowed (S_T = S0, or zeros).
  *   N, total_T, H : sequences, packed tokens, heads.  One pass per (sequence,
  *                head); the segmented schedule of gdn_prefill_ws is not used.
+ *   snaps      : optional device fp32 output (NULL: none) of state snapshots,
+ *                for prefix caching and for rolling back speculated tokens:
+ *                the state after tokens j*snap_every of sequence n (j = 1 ..
+ *                len_n / snap_every; the last one equals S_T when len_n is a
+ *                multiple) goes to snaps[(k_n + j - 1) H + h][Dv][Dk], where k_n
+ *                = sum over m < n of len_m / snap_every.
+ *   snap_every : a positive multiple of 64 when snaps is given, else ignored
+ *   n_snaps    : slots in snaps (sum over all n of len_n / snap_every); a
+ *                sequence whose slots would pass it gets none, and
+ *                GDN_ERR_SHAPE goes to *status.
  * chunk, status, stream and the other rules as for gdn_prefill. */
 int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
                        const float* beta, const float* S0, float* o, float* S_T,
                        const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
-                       int chunk, int* status, void* stream);
+                       int chunk, float* snaps, int snap_every, int n_snaps, int* status,
+                       void* stream);
 
 /* The schedule gdn_prefill_ws picks for B*H chains of T tokens on a device
  * with num_sms multiprocessors (no device is touched): *nseg segments per chain

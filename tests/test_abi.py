@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(gdn):
 
 
 def test_abi_version_and_status_strings(gdn):
-    assert gdn.abi_version() == 2
+    assert gdn.abi_version() == 3
     for code in range(-9, 1):
         s = gdn.status_str(code)
         assert s and s != "unknown status code"
@@ -150,10 +150,12 @@ def test_schedule_rejects_bad_sizes(gdn):
 def varlen_args(**over):
     a = dict(q=P, k=P + 0x10000000, v=P + 0x20000000, g=P + 0x30000000, beta=P + 0x31000000,
              S0=None, o=P + 0x40000000, S_T=P + 0x50000000, cu=P + 0x60000000, N=3, total_T=200,
-             H=2, Dk=128, Dv=128, chunk=64, status=None, stream=None)
+             H=2, Dk=128, Dv=128, chunk=64, snaps=None, snap_every=0, n_snaps=0, status=None,
+             stream=None)
     a.update(over)
     return [a[k] for k in ("q", "k", "v", "g", "beta", "S0", "o", "S_T", "cu", "N", "total_T",
-                           "H", "Dk", "Dv", "chunk", "status", "stream")]
+                           "H", "Dk", "Dv", "chunk", "snaps", "snap_every", "n_snaps", "status",
+                           "stream")]
 
 
 @pytest.mark.parametrize("over,code", [
@@ -162,6 +164,11 @@ def varlen_args(**over):
     (dict(cu=P + 0x60000002), -2), (dict(o=P + 0x40000008), -2),
     (dict(o=P + 0x60000000 - 64), -5),          # o runs into cu_seqlens
     (dict(S_T=P + 0x60000000 - 64 * 1024), -5),  # S_T runs into cu_seqlens
+    (dict(snaps=P + 0x70000000, snap_every=100, n_snaps=2), -4),   # not a multiple of 64
+    (dict(snaps=P + 0x70000000, snap_every=0, n_snaps=2), -4),
+    (dict(snaps=P + 0x70000008, snap_every=64, n_snaps=2), -2),
+    (dict(snaps=P + 0x50000000, snap_every=64, n_snaps=2), -5),    # snapshots over S_T
+    (dict(n_snaps=-1), -3),
 ], ids=lambda x: str(x))
 def test_prefill_varlen_rejects_bad_arguments(gdn, over, code):
     assert gdn.raw_prefill_varlen(*varlen_args(**over)) == code

@@ -247,6 +247,36 @@ def test_varlen_equal_lengths_match_the_dense_call():
     assert torch.equal(o1.reshape(B * T, H, 128), o2) and torch.equal(S1, S2)
 
 
+@pytest.mark.parametrize("snap_every", [64, 128])
+def test_varlen_state_snapshots(snap_every):
+    """Snapshots after every snap_every tokens of each sequence equal the final
+    state of the oracle run on that prefix."""
+    lengths = [200, 64, 0, 129, 256]
+    H = 2
+    seqs, pk = packed(lengths, H, seed=55, s0_std=0.05)
+    gdn = _gdn()
+    dd = to_dev(pk)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T, snaps = gdn.prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"],
+                                       dd["S0"], status=status, snap_every=snap_every)
+    assert gdn.query_status(status) == 0
+    assert snaps.shape[0] == sum(L // snap_every for L in lengths)
+    snaps = snaps.cpu().numpy()
+    slot = 0
+    for n, d in enumerate(seqs):
+        for j in range(1, lengths[n] // snap_every + 1):
+            t = j * snap_every
+            cut = lambda x: x[:, :t]
+            _, rS = oracle.prefill(cut(d["q"]), cut(d["k"]), cut(d["v"]), cut(d["g"]), cut(d["beta"]),
+                                   d["S0"])
+            assert_parity(snaps[slot], rS[0], f"snapshot {j} of seq {n} (t={t})")
+            slot += 1
+    # the dense outputs are unchanged by the snapshots
+    o2, S2 = gdn.prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"], dd["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(o.cpu(), o2.cpu()) and torch.equal(S_T.cpu(), S2.cpu())
+
+
 def test_varlen_bad_offsets_are_reported_on_the_device():
     _, pk = packed([40, 40], 2, seed=3)
     gdn = _gdn()
