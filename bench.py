@@ -202,9 +202,16 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
+HOST_SLACK_CYCLES = 60_000  # ~30 us of device-side wait queued after each flush
+
+
 def time_steps(fn, steps, warmup, flush, stream):
     """W untimed warm-up steps, then K steps each bracketed by CUDA events on
-    `stream` with an L2 flush before (outside) each.  Returns per-step ms."""
+    `stream` with an L2 flush before (outside) each.  After the flush a short
+    device-side sleep (also outside the events) keeps the GPU busy while the
+    host enqueues the step, so host launch latency cannot show up as idle time
+    between the events; the host path is what `e2e` measures.  Returns
+    per-step ms."""
     for _ in range(warmup):
         flush()
         fn()
@@ -213,6 +220,7 @@ def time_steps(fn, steps, warmup, flush, stream):
            for _ in range(steps)]
     for s, e in evs:
         flush()
+        torch.cuda._sleep(HOST_SLACK_CYCLES)
         s.record(stream)
         fn()
         e.record(stream)
@@ -318,6 +326,10 @@ def run_ours(args, world, rank, local):
                        "schedule": {"segments_per_chain": nseg, "tiles_per_segment": seg_tiles,
                                     "workspace_bytes": ws_bytes},
                        "l2": "flushed (256 MiB write) before every timed step",
+                       "timing": ("CUDA events around each step on its stream; before each "
+                                  "step, outside the events: the L2 flush, then a ~30 us "
+                                  "device-side sleep so host enqueue latency is not device "
+                                  "time (the host path is in e2e)"),
                        "parallelism": f"dp{world} (independent batches, no collective)"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps * launches_per_step,
             "clocks": clocks, "cpu_baseline": cpu, "impl": "ours"}
@@ -339,8 +351,11 @@ def run_extras(args, dev, stream, flush, peaks, rank):
     other = 16 if args.chunk == 64 else 64
     ws = torch.empty(max(gdn.workspace_bytes(w.B, w.T, w.H, other), 1), dtype=torch.uint8,
                      device=dev)
+    oc = torch.empty((w.B, w.T, w.H, D), dtype=torch.float32, device=dev)
+    sc = torch.empty((w.B, w.H, D, D), dtype=torch.float32, device=dev)
     ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
-                                        chunk=other, workspace=ws), steps, 3, flush, stream)
+                                        chunk=other, workspace=ws, o=oc, S_T=sc), steps, 3, flush,
+                    stream)
     t = statistics.mean(ms)
     out[f"{args.workload}/chunk{other}"] = {
         "tokens_per_s": round(w.B * w.T / (t / 1e3), 1), "ms": round(t, 5),
@@ -349,11 +364,12 @@ def run_extras(args, dev, stream, flush, peaks, rank):
     # the single-pass schedule (gdn_prefill) on the headline workload, both chunks
     for c in (args.chunk, other):
         ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
-                                            chunk=c, segmented=False), steps, 3, flush, stream)
+                                            chunk=c, segmented=False, o=oc, S_T=sc), steps, 3,
+                        flush, stream)
         t = statistics.mean(ms)
         out[f"{args.workload}/chunk{c}/single_pass"] = {
             "tokens_per_s": round(w.B * w.T / (t / 1e3), 1), "ms": round(t, 5)}
-    del d, ws
+    del d, ws, oc, sc
     # decode: L2 flushed before every step (headline) and 256 back-to-back steps (L2-warm)
     wd = gin.WORKLOADS["decode_b64_h16"]
     dd = gin.workload_inputs(wd, seed=2000 + rank, device=str(dev))
