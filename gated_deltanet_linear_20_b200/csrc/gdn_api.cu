@@ -4,6 +4,7 @@
 // calls except the cached driver entry point of cuTensorMapEncodeTiled.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -114,11 +115,12 @@ int num_sms(int* sms) {
 struct SegPlan {
   int nseg, seg_tiles;
   size_t ws_bytes, off_R, off_F;
+  int fix_parts;  // CTAs per segment in the second launch (splitting its o correction)
 };
 SegPlan plan_segments(int B, int T, int H, int sms) {
   const long long chains = (long long)B * H;
   const int tiles = (T + 63) / 64;
-  SegPlan best{1, tiles, 0, 0, 0};
+  SegPlan best{1, tiles, 0, 0, 0, 1};
   if (chains <= 0 || tiles < 2 || sms <= 0) return best;
   const long long nmax = (sms / chains + 1) / 2;
   double best_cost = tiles;
@@ -133,6 +135,11 @@ SegPlan plan_segments(int B, int T, int H, int sms) {
     }
   }
   if (best.nseg > 1) {
+    // the second launch may split each segment's o correction over a few CTAs
+    // as long as it stays within one wave
+    const long long fix_ctas = chains * (best.nseg - 1);
+    best.fix_parts = int(std::max<long long>(1, std::min<long long>(best.seg_tiles, sms / fix_ctas)));
+    best.fix_parts = std::min(best.fix_parts, 4);
     const size_t f_bytes = size_t(chains) * T * kHeadDim * 4;
     const size_t mats = size_t(chains) * best.nseg * kHeadDim * kHeadDim * 4;
     best.off_R = (f_bytes + 255) & ~size_t(255);
@@ -170,7 +177,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   if (dev_ok != GDN_OK) return dev_ok;
 
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     B,      T,
-                     H,      status, 1,      (T + 63) / 64, nullptr, nullptr, nullptr,
+                     H,      status, 1,      (T + 63) / 64, 1, nullptr, nullptr, nullptr,
                      nullptr, nullptr, 0,      0};
   if (allow_segments && T > 0) {
     int sms = 0;
@@ -186,6 +193,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
       uint8_t* base = static_cast<uint8_t*>(ws);
       a.nseg = plan.nseg;
       a.seg_tiles = plan.seg_tiles;
+      a.fix_parts = plan.fix_parts;
       a.ws_f = reinterpret_cast<float*>(base);
       a.ws_R = reinterpret_cast<float*>(base + plan.off_R);
       a.ws_F = reinterpret_cast<float*>(base + plan.off_F);
@@ -345,7 +353,7 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
 
   // B = N chains of sequences, T = total_T: the views are [1][total_T][H][128]
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
-                     H,      status, 1,      (total_T + 63) / 64, nullptr, nullptr, nullptr,
+                     H,      status, 1,      (total_T + 63) / 64, 1, nullptr, nullptr, nullptr,
                      cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0};
   CUtensorMap tq{}, tk{}, tv{}, to{};
   const int Tv = total_T > 0 ? total_T : 1;  // a valid (never read) view when every sequence is empty

@@ -25,6 +25,7 @@ struct PrefillArgs {
   // v = 0; writes f_t = F q_t like o and the transfer matrix F_k); the second
   // pass chains S_k+1 = S_k F_k + R_k and adds S_k f_t to o.
   int nseg, seg_tiles;
+  int fix_parts;    // CTAs sharing the o correction of one segment in the second pass
   float* ws_f;      // f_t of the F CTAs, laid out like o            [B][T][H][128]
   float* ws_R;      // end state of each R CTA                         [B*H][nseg][128][128]
   float* ws_F;      // transfer matrix of each F CTA (slot 0 unused)   [B*H][nseg][128][128]

@@ -206,14 +206,17 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nk = p.nseg - 1;
-  const int chain = blockIdx.x / nk;
-  const int k = blockIdx.x - chain * nk + 1;  // segment 1 .. nseg-1
+  // CTA -> (chain, segment k >= 1, part of the segment's o correction)
+  const int per = (p.nseg - 1) * p.fix_parts;
+  const int chain = blockIdx.x / per;
+  const int rem = blockIdx.x - chain * per;
+  const int k = rem / p.fix_parts + 1;  // segment 1 .. nseg-1
+  const int part = rem - (k - 1) * p.fix_parts;
   const int b = chain / p.H, h = chain - b * p.H;
   const size_t mat = size_t(D) * D;
   const float* R = p.ws_R + size_t(chain) * p.nseg * mat;
   const float* F = p.ws_F + size_t(chain) * p.nseg * mat;
-  const bool last = (k == p.nseg - 1);
+  const bool last = (k == p.nseg - 1) && part == 0;  // this CTA also forms S_T
   const int nprod = last ? k : k - 1;  // chained products S_j F_j, j = 1 .. nprod
   // R_j is added after product j for j < k, and after the last product (j = k)
   // of the last segment, where it completes S_T
@@ -301,8 +304,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
   // o_t += S_k f_t over the tokens of segment k, 64 at a time; tile i + 1
   // streams into the other staging half while tile i is multiplied.
   const int total_tiles = (p.T + NT - 1) / NT;
-  const int tb = k * p.seg_tiles;
-  const int te = min(total_tiles, tb + p.seg_tiles);
+  const int sb0 = k * p.seg_tiles, se0 = min(total_tiles, sb0 + p.seg_tiles);
+  const int per_part = (se0 - sb0 + p.fix_parts - 1) / p.fix_parts;
+  const int tb = min(se0, sb0 + part * per_part);
+  const int te = min(se0, tb + per_part);
   if (ok && tb < te) stage_f_tile(stage, p, b, h, tb * NT);
   for (int c = tb; ok && c < te; ++c) {
     const uint32_t st = stage + uint32_t((c - tb) & 1) * STAGE_TILE;
@@ -372,7 +377,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) segment_fix_kernel(const PrefillA
 
 int launch_segment_fix(const PrefillArgs& a, cudaStream_t stream) {
   if (a.nseg <= 1) return 0;
-  const int ctas = a.B * a.H * (a.nseg - 1);
+  const int ctas = a.B * a.H * (a.nseg - 1) * a.fix_parts;
   const uint32_t smem = SMEM_USED + 1024;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(segment_fix_kernel), 2, int(smem))) return -1;
   // programmatic dependent launch: the kernel's set-up overlaps the end of the
