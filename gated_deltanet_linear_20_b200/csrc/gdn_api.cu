@@ -149,10 +149,24 @@ SegPlan plan_segments(int B, int T, int H, int sms) {
   return best;
 }
 
+// Reads the options (NULL: defaults); false if they are invalid.
+bool read_options(const gdn_options* opts, int* qk_norm, float* q_scale) {
+  *qk_norm = 0;
+  *q_scale = 1.f;
+  if (!opts) return true;
+  if (opts->size < int(sizeof(gdn_options))) return false;
+  *qk_norm = opts->qk_l2norm ? 1 : 0;
+  *q_scale = opts->q_scale;
+  return opts->q_scale == opts->q_scale;  // not NaN
+}
+
 int prefill_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
                  const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
                  int chunk, void* ws, size_t ws_bytes, bool allow_segments, int* status,
-                 void* stream) {
+                 void* stream, const gdn_options* opts = nullptr) {
+  int qk_norm = 0;
+  float q_scale = 1.f;
+  if (!read_options(opts, &qk_norm, &q_scale)) return GDN_ERR_UNSUPPORTED;
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
   const long long chains = (long long)B * H;
@@ -178,7 +192,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
 
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     B,      T,
                      H,      status, 1,      (T + 63) / 64, 1, nullptr, nullptr, nullptr,
-                     nullptr, nullptr, 0,      0};
+                     nullptr, nullptr, 0,      0, qk_norm, q_scale};
   if (allow_segments && T > 0) {
     int sms = 0;
     if (num_sms(&sms) != GDN_OK) return GDN_ERR_LAUNCH;
@@ -290,6 +304,15 @@ size_t gdn_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chun
   return plan_segments(B, T, H, sms).ws_bytes;
 }
 
+int gdn_prefill_ex(const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, const float* S0, float* o, float* S_T, int B, int T, int H,
+                   int Dk, int Dv, int chunk, void* workspace, size_t workspace_bytes,
+                   const gdn_options* opts, int* status, void* stream) {
+  // without a workspace: the single pass of gdn_prefill
+  return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, workspace,
+                      workspace_bytes, workspace != nullptr, status, stream, opts);
+}
+
 int gdn_prefill_schedule(int B, int T, int H, int num_sms, int* nseg, int* seg_tiles,
                          size_t* ws_bytes) {
   if (!nseg || !seg_tiles || !ws_bytes) return GDN_ERR_NULL;
@@ -354,7 +377,7 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
   // B = N chains of sequences, T = total_T: the views are [1][total_T][H][128]
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
                      H,      status, 1,      (total_T + 63) / 64, 1, nullptr, nullptr, nullptr,
-                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0};
+                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, 0, 1.f};
   CUtensorMap tq{}, tk{}, tv{}, to{};
   const int Tv = total_T > 0 ? total_T : 1;  // a valid (never read) view when every sequence is empty
   const void* qv = total_T > 0 ? q : S_T;
@@ -406,7 +429,16 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
 int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                       int* status, void* stream) {
-  (void)status;  // the decode kernel has no device-side waits
+  return gdn_decode_ex(q, k, v, g, beta, S, o, B, T, H, Dk, Dv, nullptr, status, stream);
+}
+
+int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
+                  const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
+                  const gdn_options* opts, int* status, void* stream) {
+  (void)status;  // the decode kernels have no device-side waits
+  int qk_norm = 0;
+  float q_scale = 1.f;
+  if (!read_options(opts, &qk_norm, &q_scale)) return GDN_ERR_UNSUPPORTED;
   if (B < 0 || H < 0 || T < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim) return GDN_ERR_UNSUPPORTED;
   const long long heads = (long long)B * H;
@@ -430,7 +462,7 @@ int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* 
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
   gdn::DecodeArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H, T};
+                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H, T, qk_norm, q_scale};
   return gdn::launch_decode(a, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
 }
 

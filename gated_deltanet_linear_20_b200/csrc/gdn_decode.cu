@@ -63,7 +63,9 @@ __device__ __forceinline__ Tok load_tok(const DecodeArgs& a, size_t tok, int c0,
   return t;
 }
 
-// Burst kernel (T > 1): eight lanes per row.
+// Burst kernel (T > 1): eight lanes per row.  PRE: q / k normalisation or a q
+// scale is requested (a separate instantiation keeps the plain one lean).
+template <bool PRE>
 __global__ void __launch_bounds__(WARPS * 32) decode_burst_kernel(const DecodeArgs a) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -95,6 +97,28 @@ __global__ void __launch_bounds__(WARPS * 32) decode_burst_kernel(const DecodeAr
     bf16x8_to_float(cur.v, v);
     const float alpha = expf(cur.g);
     const float beta = cur.beta;
+    if (PRE && a.qk_norm) {  // x^ = x / sqrt(sum x^2 + 1e-6) over Dk (8 lanes of the row)
+      float kk = 0.f, qq = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        kk = fmaf(k[e], k[e], kk);
+        qq = fmaf(q[e], q[e], qq);
+      }
+#pragma unroll
+      for (int off = 1; off < 8; off <<= 1) {
+        kk += __shfl_xor_sync(0xffffffffu, kk, off);
+        qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      }
+      const float kn = rsqrtf(kk + 1e-6f), qn = rsqrtf(qq + 1e-6f) * a.q_scale;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        k[e] *= kn;
+        q[e] *= qn;
+      }
+    } else if (PRE) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) q[e] *= a.q_scale;
+    }
 
     float kq = 0.f, sk[RG], sq[RG];
 #pragma unroll
@@ -147,6 +171,7 @@ __device__ __forceinline__ float dot44(const float4& a, const float4& b) {
   return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
 }
 
+template <bool PRE>
 __global__ void __launch_bounds__(WARPS * 32) decode_step_kernel(const DecodeArgs a) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -162,11 +187,24 @@ __global__ void __launch_bounds__(WARPS * 32) decode_step_kernel(const DecodeArg
 #pragma unroll 1
   for (int t = 0; t < a.T; ++t) {
     const size_t tok = (size_t(b) * a.T + t) * a.H + h;  // [B][T][H] index of (b, t, h)
-    const float4 k4 = bf16x4_to_float4(*reinterpret_cast<const uint2*>(a.k + tok * D + 4 * lane));
-    const float4 q4 = bf16x4_to_float4(*reinterpret_cast<const uint2*>(a.q + tok * D + 4 * lane));
+    float4 k4 = bf16x4_to_float4(*reinterpret_cast<const uint2*>(a.k + tok * D + 4 * lane));
+    float4 q4 = bf16x4_to_float4(*reinterpret_cast<const uint2*>(a.q + tok * D + 4 * lane));
     const uint4 vraw = *reinterpret_cast<const uint4*>(a.v + tok * D + row0);
     const float alpha = expf(a.g[tok]);
     const float beta = a.beta[tok];
+    if (PRE && a.qk_norm) {  // x^ = x / sqrt(sum x^2 + 1e-6) over Dk (the whole warp)
+      float kk = dot44(k4, k4), qq = dot44(q4, q4);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        kk += __shfl_xor_sync(0xffffffffu, kk, off);
+        qq += __shfl_xor_sync(0xffffffffu, qq, off);
+      }
+      const float kn = rsqrtf(kk + 1e-6f), qn = rsqrtf(qq + 1e-6f) * a.q_scale;
+      k4 = make_float4(k4.x * kn, k4.y * kn, k4.z * kn, k4.w * kn);
+      q4 = make_float4(q4.x * qn, q4.y * qn, q4.z * qn, q4.w * qn);
+    } else if (PRE) {
+      q4 = make_float4(q4.x * a.q_scale, q4.y * a.q_scale, q4.z * a.q_scale, q4.w * a.q_scale);
+    }
 
     float kq = dot44(k4, q4);
 #pragma unroll
@@ -208,10 +246,19 @@ __global__ void __launch_bounds__(WARPS * 32) decode_step_kernel(const DecodeArg
 int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const long long heads = (long long)a.B * a.H;
   if (heads == 0) return 0;
-  if (a.T == 1)
-    decode_step_kernel<<<unsigned(heads * CTAS_PER_HEAD), WARPS * 32, 0, stream>>>(a);
-  else
-    decode_burst_kernel<<<unsigned(heads * CTAS_PER_HEAD), WARPS * 32, 0, stream>>>(a);
+  const unsigned grid = unsigned(heads * CTAS_PER_HEAD);
+  const bool pre = a.qk_norm || a.q_scale != 1.f;
+  if (a.T == 1) {
+    if (pre)
+      decode_step_kernel<true><<<grid, WARPS * 32, 0, stream>>>(a);
+    else
+      decode_step_kernel<false><<<grid, WARPS * 32, 0, stream>>>(a);
+  } else {
+    if (pre)
+      decode_burst_kernel<true><<<grid, WARPS * 32, 0, stream>>>(a);
+    else
+      decode_burst_kernel<false><<<grid, WARPS * 32, 0, stream>>>(a);
+  }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -39,6 +39,10 @@ struct PrefillArgs {
   // len_m / snap_every; n_snaps slots in all.
   float* snaps;
   int snap_every, n_snaps;
+  // q and k L2-normalised per token and head inside the kernel (nonzero), q
+  // multiplied by q_scale afterwards (1: unchanged).  Set explicitly.
+  int qk_norm;
+  float q_scale;
 };
 
 struct DecodeArgs {
@@ -51,6 +55,8 @@ struct DecodeArgs {
   float* o;
   int B, H;
   int T;  // tokens per sequence in this call (q, k, v, g, beta, o laid out [B][T][H])
+  int qk_norm;    // as in PrefillArgs
+  float q_scale;
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device

@@ -87,12 +87,18 @@ constexpr uint32_t SM_TF = SM_A + SOLVE_MAT;  // T  fp32 [64][APAD] (K side)
 constexpr int AT_PITCH = 20, AT_BLOCK = 16 * AT_PITCH;
 constexpr uint32_t SM_AT = SM_TF + SOLVE_MAT;
 constexpr uint32_t SM_GATES = SM_AT + 6 * AT_BLOCK * 4;  // gate buffers (tile c uses c % GATE_BUFS)
-constexpr uint32_t GATE_BYTES = 1536;
+constexpr uint32_t GATE_BYTES = 1808;
 // The side role writes tile c's gates after the chain released tile c-3
 // (tm_free); the chain's last reader of tile c-4's buffer (the o drain) runs
 // before it starts tile c-3's MMAs, so four buffers never overlap a reader.
 constexpr int GATE_BUFS = 4;
-constexpr uint32_t G_GAM2 = 0, G_B = 256, G_BG = 512, G_DF = 768, G_GAM = 1024, G_GC = 1280;
+// per-token arrays of a gate buffer (64 floats each; G_GC: one float per chunk):
+//   gamma (log2), beta, beta Gamma |k|^-1, exp(gamma_last - gamma) |k|^-1,
+//   Gamma q_scale |q|^-1, |k|^-1, q_scale |q|^-1, Gamma_last per chunk
+// (the |.|^-1 factors are 1 without in-kernel normalisation)
+constexpr uint32_t G_GAM2 = 0, G_B = 256, G_BG = 512, G_DF = 768, G_GAM = 1024, G_KN = 1280,
+                   G_QN = 1536, G_GC = 1792;
+static_assert(GATE_BYTES % 16 == 0 && G_GC + 16 <= GATE_BYTES, "gate buffer layout");
 constexpr uint32_t SM_BAR = SM_GATES + GATE_BUFS * GATE_BYTES;
 constexpr uint32_t SM_MISC = SM_BAR + 256;    // TMEM slot, abort flags, scan scratch, counters
 constexpr uint32_t SMEM_USED = SM_MISC + 256;
@@ -282,7 +288,48 @@ __device__ __forceinline__ void solve_distance(int kt, const float* sAt, float* 
 // tile's [K;Q] K^T is issued as soon as this tile's P has been read, and the
 // next tile's gates are formed before waiting for the chain; then, once the
 // chain has released tile c-1's T and Mq, writes T(c), Mq(c).
-template <int C>
+// |k_j|^-1 and q_scale |q_i|^-1 of tile c into its gate buffer (all side
+// threads; with normalisation off, just 1 and q_scale).  Thread t sums the
+// squares of half a row of [K; Q] (64 bf16 in one 128-byte SW128 row: the
+// chunk order of the swizzle does not matter for a sum) and the two halves
+// meet by a shuffle.  x^ = x / sqrt(sum x^2 + 1e-6).
+__device__ __forceinline__ void side_norms(const Ctx& x, int kt, int c, const PrefillArgs& p) {
+  float* G = x.gates(c);
+  if (!p.qk_norm) {
+    if (kt < NT) {
+      G[G_KN / 4 + kt] = 1.f;
+      G[G_QN / 4 + kt] = p.q_scale;
+    }
+    return;
+  }
+  const int r = kt >> 1, hf = kt & 1;  // row of [K; Q] (0..63 K, 64..127 Q), dk half
+  const int rr = r & (NT - 1);
+  const uint32_t row = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0) + (r < NT ? 0u : 8192u) +
+                       (hf ? 16384u : 0u) + uint32_t(rr >> 3) * 1024u + uint32_t(rr & 7) * 128u;
+  float ss = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch) {
+    uint32_t w[4];
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                 : "r"(row + 16u * ch));
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+    }
+  }
+  ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+  if (hf == 0) {
+    const float inv = rsqrtf(ss + 1e-6f);
+    if (r < NT)
+      G[G_KN / 4 + rr] = inv;
+    else
+      G[G_QN / 4 + rr] = inv * p.q_scale;
+  }
+}
+
+template <int C, bool PRE>
 __device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, float& g_next,
                                            float& b_next, const PrefillArgs& p, int b, int h,
                                            volatile float* s_part) {
@@ -320,9 +367,16 @@ __device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, f
     const int last = (kt / C) * C + C - 1;
     const float gi = G[G_GAM2 / 4 + kt], gl = G[G_GAM2 / 4 + last];
     const float Gm = fast_exp2(gi);
-    G[G_GAM / 4 + kt] = Gm;
-    G[G_BG / 4 + kt] = G[G_B / 4 + kt] * Gm;
-    G[G_DF / 4 + kt] = fast_exp2(gl - gi);
+    if constexpr (PRE) {  // fold |k|^-1 and q_scale |q|^-1
+      const float kn = G[G_KN / 4 + kt];
+      G[G_GAM / 4 + kt] = Gm * G[G_QN / 4 + kt];
+      G[G_BG / 4 + kt] = G[G_B / 4 + kt] * Gm * kn;
+      G[G_DF / 4 + kt] = fast_exp2(gl - gi) * kn;
+    } else {
+      G[G_GAM / 4 + kt] = Gm;
+      G[G_BG / 4 + kt] = G[G_B / 4 + kt] * Gm;
+      G[G_DF / 4 + kt] = fast_exp2(gl - gi);
+    }
     if (kt == last) G[G_GC / 4 + kt / C] = fast_exp2(gl);
   }
   named_bar(BAR_SIDE, SIDE_THREADS);
@@ -395,7 +449,7 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
   }
 }
 
-template <int C>
+template <int C, bool PRE>
 __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, const PrefillArgs& p, int b, int h, int ntiles) {
   const int kt = threadIdx.x - 128;        // 0..255
@@ -423,7 +477,12 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
     g_next = __ldg(p.g + gi);
     b_next = __ldg(p.beta + gi);
   }
-  side_gates<C>(x, kt, 0, T, g_next, b_next, p, b, h, s_part);
+  if constexpr (PRE) {
+    if (p.qk_norm && !rs.wait(x, x.bar(B_FULL0), 0)) return;  // the norms read tile 0
+    side_norms(x, kt, 0, p);
+    named_bar(BAR_SIDE, SIDE_THREADS);
+  }
+  side_gates<C, PRE>(x, kt, 0, T, g_next, b_next, p, b, h, s_part);
   if (!rs.wait(x, x.bar(B_FULL0), 0)) return;
   if (leader) {
     *x.misc(M_KQ_SEEN) = 1;
@@ -443,18 +502,26 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       const int i = row & (NT - 1);
       const int cs = (i / C) * C;
       const float gi = G[G_GAM2 / 4 + i];
-      const float bi = (row < NT) ? G[G_B / 4 + i] : 1.f;
+      // row factor: beta_i (|k_i|^-1) for A, 1 (q_scale |q_i|^-1) for Mq
+      float bi = (row < NT) ? G[G_B / 4 + i] : 1.f;
+      if constexpr (PRE) bi = (row < NT) ? bi * G[G_KN / 4 + i] : G[G_QN / 4 + i];
       float P[32];
       tmem_ld32(tlane + TM_P + 32 * hf, P);
 #pragma unroll
       for (int e4 = 0; e4 < 8; ++e4) {
         const float4 gj = ld4(G + G_GAM2 / 4 + 32 * hf + 4 * e4);
         const float gjv[4] = {gj.x, gj.y, gj.z, gj.w};
+        float knv[4] = {1.f, 1.f, 1.f, 1.f};
+        if constexpr (PRE) {
+          const float4 kj = ld4(G + G_KN / 4 + 32 * hf + 4 * e4);
+          knv[0] = kj.x; knv[1] = kj.y; knv[2] = kj.z; knv[3] = kj.w;
+        }
         float m[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = 32 * hf + 4 * e4 + e;
-          const float v = bi * fast_exp2(gi - gjv[e]) * P[4 * e4 + e];
+          float v = bi * fast_exp2(gi - gjv[e]) * P[4 * e4 + e];
+          if constexpr (PRE) v *= knv[e];
           m[e] = (j >= cs && (row < NT ? j < i : j <= i)) ? v : 0.f;
           mq[4 * e4 + e] = m[e];
         }
@@ -521,8 +588,17 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       named_bar(BAR_SIDE, SIDE_THREADS);
     }
 
-    // ---- gates of the next tile, while the chain is still on tile c-1 / c
-    if (c + 1 < ntiles) side_gates<C>(x, kt, c + 1, T, g_next, b_next, p, b, h, s_part);
+    // ---- gates of the next tile, while the chain is still on tile c-1 / c (with
+    //      normalisation they need the tile's norms, hence the tile itself)
+    if (c + 1 < ntiles) {
+      if constexpr (PRE) {
+        if (p.qk_norm && !rs.wait(x, x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1))
+          return;
+        side_norms(x, kt, c + 1, p);
+        named_bar(BAR_SIDE, SIDE_THREADS);
+      }
+      side_gates<C, PRE>(x, kt, c + 1, T, g_next, b_next, p, b, h, s_part);
+    }
 
     // ---- hand T(c), Mq(c) to the chain once it is done with tile c-1's
     if (c > 0 && !rs.wait(x, x.bar(B_TMFREE), (c - 1) & 1)) return;
@@ -900,7 +976,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
-template <int C>
+template <int C, bool PRE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -1007,7 +1083,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp < 4 || warp >= 12)
     chain_role<C>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
   else
-    kside_role<C>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
+    kside_role<C, PRE>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
 
   if (tid == 0) bulk_wait0();  // the chain leader's o stores have completed
   tc_fence_before();
@@ -1051,13 +1127,18 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   }
   const uint32_t smem = SMEM_USED + 1024;
   const int ctas = a.nseg > 1 ? chains * (2 * a.nseg - 1) : chains;
-  if (chunk == 64) {
-    if (!ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<64>), 0, int(smem))) return -1;
-    prefill_kernel<64><<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, to, tf, a);
-  } else {
-    if (!ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<16>), 1, int(smem))) return -1;
-    prefill_kernel<16><<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, to, tf, a);
-  }
+  const bool pre = a.qk_norm || a.q_scale != 1.f;  // fused q / k pre-steps requested
+  auto go = [&](auto kernel, int slot) {
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(kernel), slot, int(smem))) return false;
+    kernel<<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, to, tf, a);
+    return true;
+  };
+  bool ok;
+  if (chunk == 64)
+    ok = pre ? go(prefill_kernel<64, true>, 3) : go(prefill_kernel<64, false>, 0);
+  else
+    ok = pre ? go(prefill_kernel<16, true>, 4) : go(prefill_kernel<16, false>, 1);
+  if (!ok) return -1;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

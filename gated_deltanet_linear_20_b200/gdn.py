@@ -35,6 +35,21 @@ _lib.gdn_prefill_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, ctypes.c_size_t, _v
 _lib.gdn_prefill_ws.restype = _ci
 _lib.gdn_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 6 + [_vp, _ci, _ci, _vp, _vp]
 _lib.gdn_prefill_varlen.restype = _ci
+class Options(ctypes.Structure):
+    """gdn_options (include/gdn.h)."""
+    _fields_ = [("size", ctypes.c_int), ("qk_l2norm", ctypes.c_int), ("q_scale", ctypes.c_float)]
+
+
+def _options(qk_l2norm: bool, q_scale: float):
+    if not qk_l2norm and q_scale == 1.0:
+        return None
+    return ctypes.byref(Options(ctypes.sizeof(Options), int(bool(qk_l2norm)), float(q_scale)))
+
+
+_lib.gdn_prefill_ex.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, ctypes.c_size_t, _vp, _vp, _vp]
+_lib.gdn_prefill_ex.restype = _ci
+_lib.gdn_decode_ex.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp, _vp]
+_lib.gdn_decode_ex.restype = _ci
 _lib.gdn_prefill_static_ws.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, _vp]
 _lib.gdn_prefill_static_ws.restype = _ci
 _lib.gdn_prefill_schedule.argtypes = [_ci] * 4 + [_vp, _vp, _vp]
@@ -46,7 +61,7 @@ _lib.gdn_decode_tokens.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
-ABI_VERSION = 3
+ABI_VERSION = 4
 if _lib.gdn_abi_version() != ABI_VERSION:
     raise ImportError(f"libgdn_b200.so ABI {_lib.gdn_abi_version()} != binding ABI {ABI_VERSION}")
 
@@ -119,7 +134,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
             beta: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64, *,
             o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
             status: Optional[torch.Tensor] = None, segmented: bool = True,
-            workspace: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+            workspace: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
+            q_scale: float = 1.0) -> Tuple[torch.Tensor, torch.Tensor]:
     """Chunked prefill: returns (o [B,T,H,Dv] fp32, S_T [B,H,Dv,Dk] fp32).
 
     q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g, beta [B,T,H] fp32; S0 [B,H,Dv,Dk]
@@ -128,7 +144,9 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     ``segmented`` calls gdn_prefill_ws, which cuts chains into segments walked
     in parallel when they are too few to fill the GPU; its workspace is
     ``workspace`` (a uint8 CUDA tensor) or a fresh torch allocation.  With
-    ``segmented=False`` it calls gdn_prefill (one pass per chain)."""
+    ``segmented=False`` it calls gdn_prefill (one pass per chain).
+    ``qk_l2norm`` / ``q_scale`` (gdn_options) normalise q and k per token and
+    head and scale q inside the kernel (gdn_prefill_ex)."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape
@@ -151,10 +169,16 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     _check(S_T, "S_T", torch.float32, (B, H, Dv, Dk), dev)
     if status is not None:
         _check(status, "status", torch.int32, (1,), dev)
+    opts = _options(qk_l2norm, q_scale)
     if not segmented:
-        rc = _lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                              _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(status),
-                              _stream_handle(dev))
+        if opts is None:
+            rc = _lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                  _ptr(o), _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(status),
+                                  _stream_handle(dev))
+        else:
+            rc = _lib.gdn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                     _ptr(o), _ptr(S_T), B, T, H, Dk, Dv, int(chunk), None,
+                                     ctypes.c_size_t(0), opts, _ptr(status), _stream_handle(dev))
         if rc != GDN_OK:
             raise GDNError(rc, "gdn_prefill")
         return o, S_T
@@ -167,9 +191,16 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
         if workspace.dtype != torch.uint8 or workspace.device != dev or not workspace.is_contiguous():
             raise ValueError("workspace must be a contiguous uint8 tensor on the inputs' device")
     ws_bytes = 0 if workspace is None else workspace.numel()
-    rc = _lib.gdn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                             _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(workspace),
-                             ctypes.c_size_t(ws_bytes), _ptr(status), _stream_handle(dev))
+    if opts is None:
+        rc = _lib.gdn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                 _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(workspace),
+                                 ctypes.c_size_t(ws_bytes), _ptr(status), _stream_handle(dev))
+    else:
+        # workspace is None only when the schedule is the single pass, which is
+        # what gdn_prefill_ex runs for a NULL workspace
+        rc = _lib.gdn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                 _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(workspace),
+                                 ctypes.c_size_t(ws_bytes), opts, _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_prefill_ws")
     return o, S_T
@@ -270,7 +301,8 @@ def prefill_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                 beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
-                status: Optional[torch.Tensor] = None) -> torch.Tensor:
+                status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
+                q_scale: float = 1.0) -> torch.Tensor:
     """One decode step; S [B,H,Dv,Dk] fp32 is updated in place.  Returns o [B,H,Dv] fp32.
 
     q, k [B,H,Dk] bf16; v [B,H,Dv] bf16; g, beta [B,H] fp32."""
@@ -290,8 +322,13 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     if o is None:
         o = torch.empty((B, H, Dv), dtype=torch.float32, device=dev)
     _check(o, "o", torch.float32, (B, H, Dv), dev)
-    rc = _lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
-                              B, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    opts = _options(qk_l2norm, q_scale)
+    if opts is None:
+        rc = _lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                  B, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    else:
+        rc = _lib.gdn_decode_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                B, 1, H, Dk, Dv, opts, _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_decode_step")
     return o
@@ -299,7 +336,8 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
 
 def decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                   beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
-                  status: Optional[torch.Tensor] = None) -> torch.Tensor:
+                  status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
+                  q_scale: float = 1.0) -> torch.Tensor:
     """T decode tokens per sequence in one call; S [B,H,Dv,Dk] fp32 is updated in
     place (read and written once).  Returns o [B,T,H,Dv] fp32.
 
@@ -320,8 +358,13 @@ def decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     if o is None:
         o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
     _check(o, "o", torch.float32, (B, T, H, Dv), dev)
-    rc = _lib.gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
-                                B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    opts = _options(qk_l2norm, q_scale)
+    if opts is None:
+        rc = _lib.gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
+                                    _ptr(o), B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    else:
+        rc = _lib.gdn_decode_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                B, T, H, Dk, Dv, opts, _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_decode_tokens")
     return o
@@ -336,6 +379,14 @@ def raw_prefill(*args) -> int:
     """Direct call of the C entry point with raw integers/pointers (tests use it
     to exercise argument validation without any tensor)."""
     return int(_lib.gdn_prefill(*args))
+
+
+def raw_prefill_ex(*args) -> int:
+    return int(_lib.gdn_prefill_ex(*args))
+
+
+def raw_decode_ex(*args) -> int:
+    return int(_lib.gdn_decode_ex(*args))
 
 
 def raw_prefill_varlen(*args) -> int:

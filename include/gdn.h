@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 3
+#define GDN_ABI_VERSION 4
 
 enum gdn_status_code {
   GDN_OK = 0,
@@ -77,6 +77,21 @@ enum gdn_status_code {
 
 /* Size of the library's built-in device scratch used by gdn_prefill_static_ws. */
 #define GDN_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/* Optional pre-steps fused into the kernels (gdn_prefill_ex, gdn_decode_ex).
+ *   size      : sizeof(gdn_options) (a smaller value is rejected)
+ *   qk_l2norm : nonzero: q and k are L2-normalised per token and head before
+ *               use, x^ = x / sqrt(sum_d x_d^2 + 1e-6), in fp32 from the bf16
+ *               inputs.  The hybrid models normalise q and k before this layer;
+ *               fusing it saves a pass over q and k (the inputs are read once).
+ *   q_scale   : q is multiplied by this after the normalisation (1: unchanged;
+ *               e.g. Dk^-1/2).
+ * NULL options mean qk_l2norm = 0, q_scale = 1. */
+typedef struct gdn_options {
+  int size;
+  int qk_l2norm;
+  float q_scale;
+} gdn_options;
 
 /* Returns GDN_ABI_VERSION of the built library; callers compare it with the
  * header they compiled against and refuse to proceed on a mismatch. */
@@ -141,6 +156,14 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
                        const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
                        int chunk, float* snaps, int snap_every, int n_snaps, int* status,
                        void* stream);
+
+/* gdn_prefill_ws with options (gdn_options above; NULL = none); with a NULL
+ * workspace it runs the single pass of gdn_prefill.  Invalid options (size
+ * too small, q_scale NaN) return GDN_ERR_UNSUPPORTED. */
+int gdn_prefill_ex(const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, const float* S0, float* o, float* S_T, int B, int T, int H,
+                   int Dk, int Dv, int chunk, void* workspace, size_t workspace_bytes,
+                   const gdn_options* opts, int* status, void* stream);
 
 /* The schedule gdn_prefill_ws picks for B*H chains of T tokens on a device
  * with num_sms multiprocessors (no device is touched): *nseg segments per chain
@@ -221,6 +244,11 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
 int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                       int* status, void* stream);
+
+/* gdn_decode_tokens with options (gdn_options; NULL = none). */
+int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
+                  const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
+                  const gdn_options* opts, int* status, void* stream);
 
 /* Synchronises `stream`, then reads the device status word written by the
  * kernels.  Returns GDN_OK, GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_NULL (status_dev is

@@ -31,7 +31,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_varlen", "gdn_prefill_workspace_bytes",
-              "gdn_prefill_schedule", "gdn_decode_step", "gdn_decode_tokens", "gdn_abi_version",
+              "gdn_prefill_schedule", "gdn_prefill_ex", "gdn_decode_step", "gdn_decode_tokens",
+              "gdn_decode_ex", "gdn_abi_version",
               "gdn_status_str", "gdn_query_status"):
         assert n in names
 
@@ -47,7 +48,7 @@ def test_library_exports_every_declared_symbol(gdn):
 
 
 def test_abi_version_and_status_strings(gdn):
-    assert gdn.abi_version() == 3
+    assert gdn.abi_version() == 4
     for code in range(-9, 1):
         s = gdn.status_str(code)
         assert s and s != "unknown status code"
@@ -176,6 +177,25 @@ def test_prefill_varlen_rejects_bad_arguments(gdn, over, code):
 
 def test_prefill_varlen_no_sequences_is_a_noop(gdn):
     assert gdn.raw_prefill_varlen(*varlen_args(N=0, q=None, S_T=None)) == 0
+
+
+def test_options_struct_matches_the_header(gdn):
+    import ctypes as ct
+    text = open(HEADER).read()
+    assert "typedef struct gdn_options" in text
+    assert ct.sizeof(gdn.Options) == 12
+    assert [f[0] for f in gdn.Options._fields_] == ["size", "qk_l2norm", "q_scale"]
+
+
+def test_invalid_options_are_rejected(gdn):
+    import ctypes as ct
+    short = gdn.Options(4, 1, 1.0)                     # size smaller than the struct
+    nan = gdn.Options(ct.sizeof(gdn.Options), 0, float("nan"))
+    for opts in (short, nan):
+        a = prefill_args()
+        assert gdn.raw_prefill_ex(*(a[:14] + [None, 0, ct.byref(opts)] + a[14:])) == -4
+        d = decode_tokens_args()
+        assert gdn.raw_decode_ex(*(d[:12] + [ct.byref(opts)] + d[12:])) == -4
 
 
 def decode_args(**over):

@@ -287,6 +287,74 @@ def test_varlen_bad_offsets_are_reported_on_the_device():
     assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
 
 
+def raw_qk(d, seed):
+    """Un-normalised q, k (each token-head row scaled by a random factor in
+    [0.2, 5]) and their fp64 L2-normalised versions."""
+    rng = np.random.default_rng(seed)
+    out = {}
+    for key in ("q", "k"):
+        x = d[key].double()
+        scale = torch.from_numpy(rng.uniform(0.2, 5.0, size=x.shape[:-1] + (1,)))
+        raw = (x * scale).to(torch.bfloat16)
+        r64 = raw.double()
+        out[key] = raw
+        out[key + "_n"] = (r64 / torch.sqrt((r64 * r64).sum(-1, keepdim=True) + 1e-6))
+    return out
+
+
+@pytest.mark.parametrize("segmented", [False, True], ids=["single", "segmented"])
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_fused_qk_l2norm_and_q_scale(chunk, segmented):
+    """q / k L2 normalisation and the q scale fused into the kernel equal the
+    oracle run on inputs normalised in fp64 beforehand."""
+    d = inputs.prefill_inputs(1, 300, 6, seed=61, s0_std=0.05)
+    r = raw_qk(d, 62)
+    qs = 128 ** -0.5
+    gdn = _gdn()
+    dd = to_dev(d)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.prefill(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], dd["S0"],
+                         chunk=chunk, segmented=segmented, qk_l2norm=True, q_scale=qs, status=status)
+    assert gdn.query_status(status) == 0
+    ro, rS = oracle.prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"], d["beta"],
+                            d["S0"])
+    assert_parity(o.cpu().numpy(), ro, "o (fused norm)")
+    assert_parity(S_T.cpu().numpy(), rS, "S_T (fused norm)")
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_fused_qk_l2norm_in_decode(T):
+    d = inputs.prefill_inputs(4, T, 8, seed=70 + T, s0_std=0.05)
+    r = raw_qk(d, 71)
+    qs = 0.5
+    gdn = _gdn()
+    dd = to_dev(d)
+    S = dd["S0"].clone()
+    o = gdn.decode_tokens(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], S,
+                          qk_l2norm=True, q_scale=qs)
+    torch.cuda.synchronize()
+    ro, rS = oracle.prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"], d["beta"],
+                            d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o T={T}")
+    assert_parity(S.cpu().numpy(), rS, f"S T={T}")
+
+
+def test_default_options_are_bitwise_the_plain_call():
+    import ctypes as ct
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(2, 200, 3, seed=12, s0_std=0.02))
+    o1, S1 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], segmented=False)
+    o2 = torch.empty_like(o1)
+    S2 = torch.empty_like(S1)
+    opts = gdn.Options(ct.sizeof(gdn.Options), 0, 1.0)
+    rc = gdn.raw_prefill_ex(*[ct.c_void_p(t.data_ptr()) for t in (d["q"], d["k"], d["v"], d["g"],
+                                                                    d["beta"], d["S0"], o2, S2)],
+                            2, 200, 3, 128, 128, 64, None, ct.c_size_t(0), ct.byref(opts), None,
+                            ct.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert rc == 0 and torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
 def test_decode_b64_h16_256_steps_sampled_sequences():
     """256 in-place decode steps of the full batch on the GPU; sequences 0, 21,
     42, 63 (all 16 heads) checked against the oracle at every step."""
