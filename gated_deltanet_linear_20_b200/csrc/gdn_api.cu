@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <cstddef>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -150,13 +151,16 @@ SegPlan plan_segments(int B, int T, int H, int sms) {
 }
 
 // Reads the options (NULL: defaults); false if they are invalid.
-bool read_options(const gdn_options* opts, int* qk_norm, float* q_scale) {
+bool read_options(const gdn_options* opts, int* qk_norm, float* q_scale, int* o_bf16) {
   *qk_norm = 0;
   *q_scale = 1.f;
+  *o_bf16 = 0;
   if (!opts) return true;
-  if (opts->size < int(sizeof(gdn_options))) return false;
+  // a struct from before o_bf16 existed ends at it: o stays fp32
+  if (opts->size < int(offsetof(gdn_options, o_bf16))) return false;
   *qk_norm = opts->qk_l2norm ? 1 : 0;
   *q_scale = opts->q_scale;
+  if (opts->size >= int(sizeof(gdn_options))) *o_bf16 = opts->o_bf16 ? 1 : 0;
   return opts->q_scale == opts->q_scale;  // not NaN
 }
 
@@ -164,9 +168,10 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
                  const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
                  int chunk, void* ws, size_t ws_bytes, bool allow_segments, int* status,
                  void* stream, const gdn_options* opts = nullptr) {
-  int qk_norm = 0;
+  int qk_norm = 0, o_bf16 = 0;
   float q_scale = 1.f;
-  if (!read_options(opts, &qk_norm, &q_scale)) return GDN_ERR_UNSUPPORTED;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
+  if (o_bf16) allow_segments = false;  // the segment fix accumulates o in fp32
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
   const long long chains = (long long)B * H;
@@ -179,7 +184,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
                 !aligned(g, 4) || !aligned(beta, 4)))
     return GDN_ERR_ALIGN;
-  const size_t act_bf16 = size_t(act) * 2, act_f32 = size_t(act) * 4;
+  const size_t act_bf16 = size_t(act) * 2, act_f32 = size_t(act) * (o_bf16 ? 2 : 4);  // o bytes
   const size_t gate_bytes = size_t(chains) * T * 4, state_bytes = size_t(chains) * kHeadDim * kHeadDim * 4;
   if (T > 0 && (overlaps(o, act_f32, q, act_bf16) || overlaps(o, act_f32, k, act_bf16) ||
                 overlaps(o, act_f32, v, act_bf16) || overlaps(o, act_f32, g, gate_bytes) ||
@@ -192,7 +197,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
 
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     B,      T,
                      H,      status, 1,      (T + 63) / 64, 1, nullptr, nullptr, nullptr,
-                     nullptr, nullptr, 0,      0, qk_norm, q_scale};
+                     nullptr, nullptr, 0,      0, qk_norm, q_scale, o_bf16};
   if (allow_segments && T > 0) {
     int sms = 0;
     if (num_sms(&sms) != GDN_OK) return GDN_ERR_LAUNCH;
@@ -219,7 +224,8 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
     if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
         !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
         !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2) ||
-        !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4))
+        !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, o_bf16 ? bf : f32,
+                    o_bf16 ? 2 : 4))
       return GDN_ERR_LAUNCH;
     tf = to;
     if (a.nseg > 1 && !encode_act(&tf, a.ws_f, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4))
@@ -254,9 +260,9 @@ int static_workspace(void** out) {
 
 namespace gdn {
 bool ensure_smem_attr(const void* func, int slot, int bytes) {
-  static std::atomic<uint64_t> done[8];  // bit d: device d, per kernel slot
+  static std::atomic<uint64_t> done[16];  // bit d: device d, per kernel slot
   int dev = 0;
-  if (slot < 0 || slot >= 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+  if (slot < 0 || slot >= 16 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return false;
   const uint64_t bit = uint64_t(1) << dev;
   if (done[slot].load(std::memory_order_acquire) & bit) return true;
@@ -377,7 +383,7 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
   // B = N chains of sequences, T = total_T: the views are [1][total_T][H][128]
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
                      H,      status, 1,      (total_T + 63) / 64, 1, nullptr, nullptr, nullptr,
-                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, 0, 1.f};
+                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, 0, 1.f, 0};
   CUtensorMap tq{}, tk{}, tv{}, to{};
   const int Tv = total_T > 0 ? total_T : 1;  // a valid (never read) view when every sequence is empty
   const void* qv = total_T > 0 ? q : S_T;
@@ -436,9 +442,9 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
                   const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                   const gdn_options* opts, int* status, void* stream) {
   (void)status;  // the decode kernels have no device-side waits
-  int qk_norm = 0;
+  int qk_norm = 0, o_bf16 = 0;
   float q_scale = 1.f;
-  if (!read_options(opts, &qk_norm, &q_scale)) return GDN_ERR_UNSUPPORTED;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
   if (B < 0 || H < 0 || T < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim) return GDN_ERR_UNSUPPORTED;
   const long long heads = (long long)B * H;
@@ -450,7 +456,7 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
       !aligned(o, 16) || !aligned(g, 4) || !aligned(beta, 4))
     return GDN_ERR_ALIGN;
   const size_t toks = size_t(heads) * T;
-  const size_t vec_bf16 = toks * kHeadDim * 2, vec_f32 = toks * kHeadDim * 4;
+  const size_t vec_bf16 = toks * kHeadDim * 2, vec_f32 = toks * kHeadDim * (o_bf16 ? 2 : 4);  // o bytes
   const size_t state_bytes = size_t(heads) * kHeadDim * kHeadDim * 4, gate_bytes = toks * 4;
   if (overlaps(o, vec_f32, q, vec_bf16) || overlaps(o, vec_f32, k, vec_bf16) ||
       overlaps(o, vec_f32, v, vec_bf16) || overlaps(o, vec_f32, g, gate_bytes) ||
@@ -462,7 +468,8 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
   gdn::DecodeArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H, T, qk_norm, q_scale};
+                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H, T, qk_norm, q_scale,
+                    o_bf16};
   return gdn::launch_decode(a, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
 }
 

@@ -147,7 +147,14 @@ __global__ void __launch_bounds__(WARPS * 32) decode_burst_kernel(const DecodeAr
         s[i][e].z = fmaf(alpha, s[i][e].z, d * k[4 * e + 2]);
         s[i][e].w = fmaf(alpha, s[i][e].w, d * k[4 * e + 3]);
       }
-      if ((lane & 7) == 0) a.o[tok * D + row0 + 4 * i + sub] = fmaf(alpha, sq[i], d * kq);
+      if ((lane & 7) == 0) {
+        const float ov = fmaf(alpha, sq[i], d * kq);
+        const size_t oi = tok * D + row0 + 4 * i + sub;
+        if (a.o_bf16)
+          reinterpret_cast<__nv_bfloat16*>(a.o)[oi] = __float2bfloat16_rn(ov);
+        else
+          a.o[oi] = ov;
+      }
     }
     cur = nxt;
   }
@@ -235,7 +242,12 @@ __global__ void __launch_bounds__(WARPS * 32) decode_step_kernel(const DecodeArg
       const float o = fmaf(alpha, sq[r], d * kq);
       if (lane == r) o_mine = o;
     }
-    if (lane < ROWS_PER_WARP) a.o[tok * D + row0 + lane] = o_mine;
+    if (lane < ROWS_PER_WARP) {
+      if (a.o_bf16)
+        reinterpret_cast<__nv_bfloat16*>(a.o)[tok * D + row0 + lane] = __float2bfloat16_rn(o_mine);
+      else
+        a.o[tok * D + row0 + lane] = o_mine;
+    }
   }
 #pragma unroll
   for (int r = 0; r < ROWS_PER_WARP; ++r) __stcs(srow + r * (D / 4), s[r]);

@@ -43,6 +43,7 @@ struct PrefillArgs {
   // multiplied by q_scale afterwards (1: unchanged).  Set explicitly.
   int qk_norm;
   float q_scale;
+  int o_bf16;  // o is bf16 (same layout); single-pass schedule only
 };
 
 struct DecodeArgs {
@@ -57,6 +58,7 @@ struct DecodeArgs {
   int T;  // tokens per sequence in this call (q, k, v, g, beta, o laid out [B][T][H])
   int qk_norm;    // as in PrefillArgs
   float q_scale;
+  int o_bf16;     // o is bf16 (same layout)
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device

@@ -412,10 +412,13 @@ __device__ __noinline__ void store_partial_tile(const float4* src, float* dst, i
 // the leader then stores the tile with TMA (tokens at or past T are dropped by
 // the copy) and waits for the copy to have read the tile before X^T is written
 // again.
+// OBF: o is bf16 (tile rows of 256 B, stored through a bf16 view).
+template <bool OBF>
 __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b, int h, int dv,
                                              int hf, int c, bool leader) {
   const float* G = x.gates(c);
   float* so = reinterpret_cast<float*>(x.sm + SM_XH) + dv;
+  __nv_bfloat16* so16 = reinterpret_cast<__nv_bfloat16*>(x.sm + SM_XH) + dv;
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     float y[16], oi[16];
@@ -427,7 +430,11 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int n = 32 * hf + 16 * q + 4 * e4 + e;  // token within the tile
-        so[n * D] = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
+        const float ov = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
+        if constexpr (OBF)
+          so16[n * D] = __float2bfloat16_rn(ov);
+        else
+          so[n * D] = ov;
       }
     }
   }
@@ -440,9 +447,9 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
       tma_store_4d(x.tmo, x.sb + SM_XH, 0, h, ts, b);
       bulk_commit();
     }
-  } else {
-    // last tile of a packed sequence: the rows past it belong to the next
-    // sequence, so only the valid rows are copied out
+  } else if constexpr (!OBF) {
+    // last tile of a packed sequence (packed calls take fp32 o only): the rows
+    // past it belong to the next sequence, so only the valid rows are copied out
     store_partial_tile(reinterpret_cast<const float4*>(x.sm + SM_XH),
                        x.odst + ((size_t(b) * x.tmap + ts) * x.H + h) * D, x.H, x.tend - ts,
                        hf * 128 + dv);
@@ -682,7 +689,7 @@ __device__ __forceinline__ void issue_zq(const Ctx& x, uint32_t kq, int s) {
 }
 
 // ============================================================== chain
-template <int C>
+template <int C, bool OBF>
 __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, const PrefillArgs& p, int chain, int b, int h,
                            int ntiles) {
@@ -903,7 +910,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
 
       // ---- o of the whole tile is complete after its last chunk: o[t][dv] =
       //      Gamma_t Y[dv][t] + O_intra[dv][t], this thread's 32 tokens to HBM
-      if (s == NSUB - 1) output_drain(x, tlane, b, h, dv, ch, c, leader);
+      if (s == NSUB - 1) output_drain<OBF>(x, tlane, b, h, dv, ch, c, leader);
 
       // ---- S_out now sits in TMEM: refresh its hi/lo copy, and pre-scale it by
       //      the next chunk's decay (or store it as S_T after the last chunk)
@@ -976,7 +983,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
-template <int C, bool PRE>
+template <int C, bool PRE, bool OBF>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -1081,7 +1088,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // for this grid to complete before it reads anything this grid writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp < 4 || warp >= 12)
-    chain_role<C>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
+    chain_role<C, OBF>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
   else
     kside_role<C, PRE>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
 
@@ -1133,11 +1140,19 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
     kernel<<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, to, tf, a);
     return true;
   };
+  const bool obf = a.o_bf16 != 0;
   bool ok;
-  if (chunk == 64)
-    ok = pre ? go(prefill_kernel<64, true>, 3) : go(prefill_kernel<64, false>, 0);
-  else
-    ok = pre ? go(prefill_kernel<16, true>, 4) : go(prefill_kernel<16, false>, 1);
+  if (chunk == 64) {
+    if (obf)
+      ok = pre ? go(prefill_kernel<64, true, true>, 5) : go(prefill_kernel<64, false, true>, 6);
+    else
+      ok = pre ? go(prefill_kernel<64, true, false>, 3) : go(prefill_kernel<64, false, false>, 0);
+  } else {
+    if (obf)
+      ok = pre ? go(prefill_kernel<16, true, true>, 7) : go(prefill_kernel<16, false, true>, 8);
+    else
+      ok = pre ? go(prefill_kernel<16, true, false>, 4) : go(prefill_kernel<16, false, false>, 1);
+  }
   if (!ok) return -1;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }

@@ -37,13 +37,15 @@ _lib.gdn_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 6 + [_vp, _ci, _ci, _vp, 
 _lib.gdn_prefill_varlen.restype = _ci
 class Options(ctypes.Structure):
     """gdn_options (include/gdn.h)."""
-    _fields_ = [("size", ctypes.c_int), ("qk_l2norm", ctypes.c_int), ("q_scale", ctypes.c_float)]
+    _fields_ = [("size", ctypes.c_int), ("qk_l2norm", ctypes.c_int), ("q_scale", ctypes.c_float),
+                ("o_bf16", ctypes.c_int)]
 
 
-def _options(qk_l2norm: bool, q_scale: float):
-    if not qk_l2norm and q_scale == 1.0:
+def _options(qk_l2norm: bool, q_scale: float, o_bf16: bool = False):
+    if not qk_l2norm and q_scale == 1.0 and not o_bf16:
         return None
-    return ctypes.byref(Options(ctypes.sizeof(Options), int(bool(qk_l2norm)), float(q_scale)))
+    return ctypes.byref(Options(ctypes.sizeof(Options), int(bool(qk_l2norm)), float(q_scale),
+                                int(bool(o_bf16))))
 
 
 _lib.gdn_prefill_ex.argtypes = [_vp] * 8 + [_ci] * 6 + [_vp, ctypes.c_size_t, _vp, _vp, _vp]
@@ -61,7 +63,7 @@ _lib.gdn_decode_tokens.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
-ABI_VERSION = 4
+ABI_VERSION = 5
 if _lib.gdn_abi_version() != ABI_VERSION:
     raise ImportError(f"libgdn_b200.so ABI {_lib.gdn_abi_version()} != binding ABI {ABI_VERSION}")
 
@@ -135,8 +137,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
             o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
             status: Optional[torch.Tensor] = None, segmented: bool = True,
             workspace: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
-            q_scale: float = 1.0) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Chunked prefill: returns (o [B,T,H,Dv] fp32, S_T [B,H,Dv,Dk] fp32).
+            q_scale: float = 1.0, o_bf16: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Chunked prefill: returns (o [B,T,H,Dv] fp32 or bf16, S_T [B,H,Dv,Dk] fp32).
 
     q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g, beta [B,T,H] fp32; S0 [B,H,Dv,Dk]
     fp32 or None (zeros); chunk 16 or 64.  Launches on the current stream.
@@ -146,7 +148,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     ``workspace`` (a uint8 CUDA tensor) or a fresh torch allocation.  With
     ``segmented=False`` it calls gdn_prefill (one pass per chain).
     ``qk_l2norm`` / ``q_scale`` (gdn_options) normalise q and k per token and
-    head and scale q inside the kernel (gdn_prefill_ex)."""
+    head and scale q inside the kernel (gdn_prefill_ex).  ``o_bf16`` makes o
+    bf16 (the fp32 value rounded to nearest even); it runs the single pass."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape
@@ -161,16 +164,17 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     _check(beta, "beta", torch.float32, (B, T, H), dev)
     if S0 is not None:
         _check(S0, "S0", torch.float32, (B, H, Dv, Dk), dev)
+    o_dtype = torch.bfloat16 if o_bf16 else torch.float32
     if o is None:
-        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
-    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
+        o = torch.empty((B, T, H, Dv), dtype=o_dtype, device=dev)
+    _check(o, "o", o_dtype, (B, T, H, Dv), dev)
     if S_T is None:
         S_T = torch.empty((B, H, Dv, Dk), dtype=torch.float32, device=dev)
     _check(S_T, "S_T", torch.float32, (B, H, Dv, Dk), dev)
     if status is not None:
         _check(status, "status", torch.int32, (1,), dev)
-    opts = _options(qk_l2norm, q_scale)
-    if not segmented:
+    opts = _options(qk_l2norm, q_scale, o_bf16)
+    if not segmented or o_bf16:
         if opts is None:
             rc = _lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
                                   _ptr(o), _ptr(S_T), B, T, H, Dk, Dv, int(chunk), _ptr(status),
@@ -302,8 +306,9 @@ def prefill_static(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                 beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
                 status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
-                q_scale: float = 1.0) -> torch.Tensor:
-    """One decode step; S [B,H,Dv,Dk] fp32 is updated in place.  Returns o [B,H,Dv] fp32.
+                q_scale: float = 1.0, o_bf16: bool = False) -> torch.Tensor:
+    """One decode step; S [B,H,Dv,Dk] fp32 is updated in place.  Returns o [B,H,Dv]
+    (fp32, or bf16 with ``o_bf16``).
 
     q, k [B,H,Dk] bf16; v [B,H,Dv] bf16; g, beta [B,H] fp32."""
     if q.dim() != 3:
@@ -319,10 +324,11 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     _check(g, "g", torch.float32, (B, H), dev)
     _check(beta, "beta", torch.float32, (B, H), dev)
     _check(S, "S", torch.float32, (B, H, Dv, Dk), dev)
+    o_dtype = torch.bfloat16 if o_bf16 else torch.float32
     if o is None:
-        o = torch.empty((B, H, Dv), dtype=torch.float32, device=dev)
-    _check(o, "o", torch.float32, (B, H, Dv), dev)
-    opts = _options(qk_l2norm, q_scale)
+        o = torch.empty((B, H, Dv), dtype=o_dtype, device=dev)
+    _check(o, "o", o_dtype, (B, H, Dv), dev)
+    opts = _options(qk_l2norm, q_scale, o_bf16)
     if opts is None:
         rc = _lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
                                   B, H, Dk, Dv, _ptr(status), _stream_handle(dev))
@@ -337,9 +343,10 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
 def decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                   beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
                   status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
-                  q_scale: float = 1.0) -> torch.Tensor:
+                  q_scale: float = 1.0, o_bf16: bool = False) -> torch.Tensor:
     """T decode tokens per sequence in one call; S [B,H,Dv,Dk] fp32 is updated in
-    place (read and written once).  Returns o [B,T,H,Dv] fp32.
+    place (read and written once).  Returns o [B,T,H,Dv] (fp32, or bf16 with
+    ``o_bf16``).
 
     q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g, beta [B,T,H] fp32."""
     if q.dim() != 4:
@@ -355,10 +362,11 @@ def decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     _check(g, "g", torch.float32, (B, T, H), dev)
     _check(beta, "beta", torch.float32, (B, T, H), dev)
     _check(S, "S", torch.float32, (B, H, Dv, Dk), dev)
+    o_dtype = torch.bfloat16 if o_bf16 else torch.float32
     if o is None:
-        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
-    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
-    opts = _options(qk_l2norm, q_scale)
+        o = torch.empty((B, T, H, Dv), dtype=o_dtype, device=dev)
+    _check(o, "o", o_dtype, (B, T, H, Dv), dev)
+    opts = _options(qk_l2norm, q_scale, o_bf16)
     if opts is None:
         rc = _lib.gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S),
                                     _ptr(o), B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))

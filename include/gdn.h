@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 4
+#define GDN_ABI_VERSION 5
 
 enum gdn_status_code {
   GDN_OK = 0,
@@ -86,11 +86,17 @@ enum gdn_status_code {
  *               fusing it saves a pass over q and k (the inputs are read once).
  *   q_scale   : q is multiplied by this after the normalisation (1: unchanged;
  *               e.g. Dk^-1/2).
- * NULL options mean qk_l2norm = 0, q_scale = 1. */
+ *   o_bf16    : nonzero: o is written as bf16 (same layout; the fp32 value
+ *               rounded to nearest even), halving its bytes.  A prefill with
+ *               it runs the single-pass schedule (no workspace is used).
+ * NULL options mean qk_l2norm = 0, q_scale = 1, o_bf16 = 0.  `size` is
+ * sizeof(gdn_options) as the caller compiled it: 12 (a struct without o_bf16)
+ * reads as o_bf16 = 0; anything below 12 is GDN_ERR_UNSUPPORTED. */
 typedef struct gdn_options {
   int size;
   int qk_l2norm;
   float q_scale;
+  int o_bf16;
 } gdn_options;
 
 /* Returns GDN_ABI_VERSION of the built library; callers compare it with the

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(gdn):
 
 
 def test_abi_version_and_status_strings(gdn):
-    assert gdn.abi_version() == 4
+    assert gdn.abi_version() == 5
     for code in range(-9, 1):
         s = gdn.status_str(code)
         assert s and s != "unknown status code"
@@ -183,8 +183,8 @@ def test_options_struct_matches_the_header(gdn):
     import ctypes as ct
     text = open(HEADER).read()
     assert "typedef struct gdn_options" in text
-    assert ct.sizeof(gdn.Options) == 12
-    assert [f[0] for f in gdn.Options._fields_] == ["size", "qk_l2norm", "q_scale"]
+    assert ct.sizeof(gdn.Options) == 16
+    assert [f[0] for f in gdn.Options._fields_] == ["size", "qk_l2norm", "q_scale", "o_bf16"]
 
 
 def test_invalid_options_are_rejected(gdn):
@@ -196,6 +196,27 @@ def test_invalid_options_are_rejected(gdn):
         assert gdn.raw_prefill_ex(*(a[:14] + [None, 0, ct.byref(opts)] + a[14:])) == -4
         d = decode_tokens_args()
         assert gdn.raw_decode_ex(*(d[:12] + [ct.byref(opts)] + d[12:])) == -4
+
+
+def test_bf16_o_overlap_uses_two_byte_elements(gdn):
+    """With o_bf16 o spans B*T*H*Dv*2 bytes: an o that would run into S_T as
+    fp32 (64 KiB) stops short of it as bf16 (32 KiB)."""
+    import ctypes as ct
+    o = P + 0x50000000 - 48 * 1024
+    a = prefill_args(o=o)
+    plain = gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 0)
+    half = gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 1)
+    assert gdn.raw_prefill_ex(*(a[:14] + [None, 0, ct.byref(plain)] + a[14:])) == -5
+    assert gdn.raw_prefill_ex(*(a[:14] + [None, 0, ct.byref(half)] + a[14:])) not in (0, -5)
+
+
+def test_options_without_o_bf16_field_are_accepted(gdn):
+    """A 12-byte struct (before o_bf16) reads as o_bf16 = 0: the fp32 overlap
+    rule applies, so the call fails on the overlap and not on the size."""
+    import ctypes as ct
+    a = prefill_args(o=P + 0x50000000 - 48 * 1024)
+    old = gdn.Options(12, 0, 1.0, 1)   # the trailing o_bf16 lies past `size`: ignored
+    assert gdn.raw_prefill_ex(*(a[:14] + [None, 0, ct.byref(old)] + a[14:])) == -5
 
 
 def decode_args(**over):

@@ -355,6 +355,62 @@ def test_default_options_are_bitwise_the_plain_call():
     assert rc == 0 and torch.equal(o1, o2) and torch.equal(S1, S2)
 
 
+@pytest.mark.parametrize("pre", [False, True], ids=["plain", "qknorm"])
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_bf16_o_is_the_fp32_o_rounded(chunk, pre):
+    """o_bf16 stores the same fp32 o rounded to nearest even: bit for bit the
+    fp32 call's o cast to bf16, with an identical end state.  T = 300 leaves a
+    ragged last tile; a segmented request runs the single pass."""
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(2, 300, 5, seed=81, s0_std=0.05))
+    kw = dict(qk_l2norm=True, q_scale=0.25) if pre else {}
+    o32, S32 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk,
+                           segmented=False, **kw)
+    for seg in (False, True):
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        o16, S16 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chunk=chunk,
+                               segmented=seg, o_bf16=True, status=status, **kw)
+        assert gdn.query_status(status) == 0
+        assert o16.dtype == torch.bfloat16
+        assert torch.equal(o16, o32.to(torch.bfloat16)), f"segmented={seg}"
+        assert torch.equal(S16, S32), f"segmented={seg}"
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_bf16_o_in_decode(T):
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(8, T, 16, seed=90 + T, s0_std=0.05))
+    S32 = d["S0"].clone()
+    S16 = d["S0"].clone()
+    if T == 1:
+        sq = {n: d[n][:, 0] for n in ("q", "k", "v", "g", "beta")}
+        o32 = gdn.decode_step(sq["q"], sq["k"], sq["v"], sq["g"], sq["beta"], S32)
+        o16 = gdn.decode_step(sq["q"], sq["k"], sq["v"], sq["g"], sq["beta"], S16, o_bf16=True)
+    else:
+        o32 = gdn.decode_tokens(d["q"], d["k"], d["v"], d["g"], d["beta"], S32)
+        o16 = gdn.decode_tokens(d["q"], d["k"], d["v"], d["g"], d["beta"], S16, o_bf16=True)
+    torch.cuda.synchronize()
+    assert o16.dtype == torch.bfloat16
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(S16, S32)
+
+
+def test_bf16_o_full_size_against_the_oracle():
+    """B1 H16 T512 with bf16 o: the oracle's fp64 o rounded to bf16 agrees to
+    the rounding step (one bf16 ulp) plus the fp32 path's tolerance."""
+    gdn = _gdn()
+    d = inputs.workload_inputs(inputs.WORKLOADS["prefill_b1_h16_t512"], seed=0)
+    dd = to_dev(d)
+    o16, S = gdn.prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"], o_bf16=True)
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(S.cpu().numpy(), rS, "S_T (bf16 o call)")
+    got = o16.float().cpu().numpy().astype(np.float64)
+    ref = np.asarray(ro, dtype=np.float64)
+    ulp = np.abs(ref) * 2.0 ** -7            # one bf16 ulp at |ref| (8 significant bits)
+    rms = float(np.sqrt(np.mean(ref ** 2)))
+    assert np.all(np.abs(got - ref) <= ulp + 1e-2 * rms)
+
+
 def test_decode_b64_h16_256_steps_sampled_sequences():
     """256 in-place decode steps of the full batch on the GPU; sequences 0, 21,
     42, 63 (all 16 heads) checked against the oracle at every step."""
