@@ -13,6 +13,8 @@ What is computed (per sequence b and head h, independently), in fp64:
     o_t     = S_t q_t
 
 This is the gated delta rule of the hybrid Qwen 3.5 linear-attention layers.
+``kda_prefill`` is the per-channel-gate variant (KDA): alpha_t becomes a vector
+over Dk, applied as S_{t-1} diag(alpha_t) in place of alpha_t S_{t-1}.
 The ROCmFPX gated-delta-net prefill note (bittide.aicompass.dev article
 d2880479, opening post) fixes its setting -- scalar gate per token and head,
 head dim 128, single-sequence prefill, state in F32 accumulators -- but prints
@@ -61,6 +63,8 @@ def _load():
         lib.oracle_gdn_prefill_chains_f64.restype = ci
         lib.oracle_gdn_decode_step_f64.argtypes = [fp, fp, fp, fp, fp, dp, dp, ci, ci, ci, ci]
         lib.oracle_gdn_decode_step_f64.restype = ci
+        lib.oracle_kda_prefill_f64.argtypes = [fp, fp, fp, fp, fp, fp, dp, dp, ci, ci, ci, ci, ci]
+        lib.oracle_kda_prefill_f64.restype = ci
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ci
         _lib = lib
@@ -147,3 +151,28 @@ def decode_step(q, k, v, g, beta, S):
     if rc != 0:
         raise RuntimeError(f"oracle decode failed with code {rc}")
     return o, S
+
+
+def kda_prefill(q, k, v, g, beta, S0=None):
+    """Per-channel gate (KDA): alpha_t = exp(g_t) over Dk,
+    S_t = S_{t-1} diag(alpha_t)(I - beta_t k_t k_t^T) + beta_t v_t k_t^T, o_t = S_t q_t.
+
+    q, k: [B,T,H,Dk]; v: [B,T,H,Dv]; g: [B,T,H,Dk]; beta: [B,T,H]; S0: [B,H,Dv,Dk]
+    or None.  Returns (o [B,T,H,Dv], S_T [B,H,Dv,Dk]) as float64 numpy arrays.
+    """
+    q, k, v, g, beta, S0 = (_f32(t) for t in (q, k, v, g, beta, S0))
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    assert k.shape == (B, T, H, Dk) and v.shape == (B, T, H, Dv)
+    assert g.shape == (B, T, H, Dk) and beta.shape == (B, T, H)
+    assert S0 is None or S0.shape == (B, H, Dv, Dk)
+    o = np.empty((B, T, H, Dv), np.float64)
+    S_T = np.empty((B, H, Dv, Dk), np.float64)
+    rc = _load().oracle_kda_prefill_f64(_ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float),
+                                        _ptr(v, ctypes.c_float), _ptr(g, ctypes.c_float),
+                                        _ptr(beta, ctypes.c_float), _ptr(S0, ctypes.c_float),
+                                        _ptr(o, ctypes.c_double), _ptr(S_T, ctypes.c_double),
+                                        B, T, H, Dk, Dv)
+    if rc != 0:
+        raise RuntimeError(f"oracle KDA prefill failed with code {rc}")
+    return o, S_T

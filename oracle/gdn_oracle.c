@@ -185,6 +185,91 @@ int oracle_gdn_decode_step_f64(const float *q, const float *k, const float *v,
     return failed ? -2 : 0;
 }
 
+/* ------------------------------------------------------------------------
+ * Per-channel gate (KDA, the "next" variant the ROCmFPX gated-delta-net
+ * prefill note names among the cases its fused kernel did not cover).  The
+ * scalar gate becomes one decay per key channel, applied where the scalar one
+ * is:
+ *
+ *     alpha_t = exp(g_t)                       (a vector over Dk)
+ *     S_t     = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t     = S_t q_t
+ *
+ * evaluated, as above, in the product form term by term:
+ *     u       = S_{t-1} diag(alpha_t) k_t                          (Dv vector)
+ *     S_t[i][j] = alpha_t[j] S_{t-1}[i][j] - beta_t u[i] k_t[j] + beta_t v_t[i] k_t[j]
+ *
+ * g is [B][T][H][Dk] (natural-log decays, fp32); everything else is laid out
+ * as for the scalar gate.
+ */
+static void kda_step(double *S, const float *qt, const float *kt, const float *vt,
+                     const float *gt, double bt, double *ot, int Dk, int Dv, double *u,
+                     double *a) {
+    for (int j = 0; j < Dk; ++j) a[j] = exp((double)gt[j]);
+    /* u = S_{t-1} diag(alpha) k */
+    for (int i = 0; i < Dv; ++i) {
+        double acc = 0.0;
+        const double *Si = S + (int64_t)i * Dk;
+        for (int j = 0; j < Dk; ++j) acc += Si[j] * a[j] * (double)kt[j];
+        u[i] = acc;
+    }
+    for (int i = 0; i < Dv; ++i) {
+        double *Si = S + (int64_t)i * Dk;
+        const double vi = (double)vt[i];
+        for (int j = 0; j < Dk; ++j) {
+            const double kj = (double)kt[j];
+            Si[j] = a[j] * Si[j] - bt * u[i] * kj + bt * vi * kj;
+        }
+    }
+    for (int i = 0; i < Dv; ++i) {
+        double acc = 0.0;
+        const double *Si = S + (int64_t)i * Dk;
+        for (int j = 0; j < Dk; ++j) acc += Si[j] * (double)qt[j];
+        ot[i] = acc;
+    }
+}
+
+int oracle_kda_prefill_f64(const float *q, const float *k, const float *v,
+                           const float *g, const float *beta, const float *S0,
+                           double *o, double *S_T, int B, int T, int H,
+                           int Dk, int Dv) {
+    if (B < 0 || T < 0 || H < 0 || Dk <= 0 || Dv <= 0) return -1;
+    const int chains = B * H;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *S = (double *)malloc(sizeof(double) * (size_t)Dv * (size_t)Dk);
+        double *u = (double *)malloc(sizeof(double) * (size_t)Dv);
+        double *a = (double *)malloc(sizeof(double) * (size_t)Dk);
+        if (!S || !u || !a) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+#pragma omp for schedule(dynamic, 1)
+            for (int c = 0; c < chains; ++c) {
+                const int b = c / H, h = c % H;
+                const int64_t s_off = ((int64_t)b * H + h) * (int64_t)Dv * Dk;
+                if (S0) {
+                    for (int64_t e = 0; e < (int64_t)Dv * Dk; ++e) S[e] = (double)S0[s_off + e];
+                } else {
+                    memset(S, 0, sizeof(double) * (size_t)Dv * (size_t)Dk);
+                }
+                for (int t = 0; t < T; ++t) {
+                    const int64_t gi = ((int64_t)b * T + t) * H + h;
+                    kda_step(S, q + idx4(b, t, h, 0, T, H, Dk), k + idx4(b, t, h, 0, T, H, Dk),
+                             v + idx4(b, t, h, 0, T, H, Dv), g + idx4(b, t, h, 0, T, H, Dk),
+                             (double)beta[gi], o + idx4(b, t, h, 0, T, H, Dv), Dk, Dv, u, a);
+                }
+                if (S_T) memcpy(S_T + s_off, S, sizeof(double) * (size_t)Dv * (size_t)Dk);
+            }
+        }
+        free(S);
+        free(u);
+        free(a);
+    }
+    return failed ? -2 : 0;
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
