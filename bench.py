@@ -74,6 +74,23 @@ def decode_state_bytes(B, H):
     return B * H * 2 * STATE_BYTES
 
 
+# per-channel gate (KDA): g is a vector of D fp32 per token-head
+KDA_TOKEN_HEAD_BYTES = 3 * D * 2 + D * 4 + 4 + D * 4   # q, k, v bf16 + g + beta + o = 1796 B
+KDA_OPS_PER_TOKEN_HEAD = 4 * D * D   # per state element: decay, two dot-product FMAs, update FMA
+FP32_LANES_PER_SM = 128
+SM_MAX_MHZ = 1965.0                   # clocks.max.sm of the B200
+
+
+def kda_prefill_bytes(B, T, H, has_s0):
+    return B * T * H * KDA_TOKEN_HEAD_BYTES + B * H * STATE_BYTES * (2 if has_s0 else 1)
+
+
+def alu_peak_tops(dev):
+    """FP32 lane operations per second at the maximum SM clock: SMs x 128 lanes x clock."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return sms * FP32_LANES_PER_SM * SM_MAX_MHZ * 1e6 / 1e12
+
+
 # ------------------------------------------------------------------ helpers
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -456,6 +473,60 @@ def run_extras(args, dev, stream, flush, peaks, rank):
         "tensor_frac": round(fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
     del dl, ol, sl
     torch.cuda.empty_cache()
+    out.update(run_kda_extras(dev, stream, flush, peaks, rank, steps))
+    return out
+
+
+def run_kda_extras(dev, stream, flush, peaks, rank, steps):
+    """The per-channel-gate (KDA) kernel: the headline shape, a large batch, and
+    the batched decode step.  Its work is fp32 lane arithmetic (4 operations per
+    state element and token), so the roofline is the SMs' FP32 lanes at the
+    maximum clock; the HBM fraction is reported beside it."""
+    from gated_deltanet_linear_20_b200 import gdn
+    out = {}
+    peak_ops = alu_peak_tops(dev)
+    for (B, T, H, g_mean, n) in ((1, 512, 16, 0.0, steps), (4, 8192, 32, 2.0, 3)):
+        d = gin.kda_inputs(B, T, H, seed=5000 + rank, g_mean=g_mean, device=str(dev))
+        o = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
+        sT = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+        ms = time_steps(lambda: gdn.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None,
+                                                o=o, S_T=sT), n, 3, flush, stream)
+        t = statistics.mean(ms)
+        ops = B * T * H * KDA_OPS_PER_TOKEN_HEAD
+        nb = kda_prefill_bytes(B, T, H, False)
+        out[f"kda_prefill_b{B}_h{H}_t{T}"] = {
+            "tokens_per_s": round(B * T / (t / 1e3), 1), "ms": round(t, 5),
+            "roofline": {"bound": "alu", "achieved": round(ops / (t / 1e3) / 1e12, 3),
+                         "peak": round(peak_ops, 2), "unit": "Tops/s (fp32 lane ops)",
+                         "frac": round(ops / (t / 1e3) / 1e12 / peak_ops, 4),
+                         "peak_source": "SMs x 128 fp32 lanes x 1965 MHz"},
+            "hbm_frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+            "gate": f"per channel, logsigmoid(N({g_mean},1))"}
+        del d, o, sT
+    # decode: one token for 64 x 16 heads, state in place, L2 flushed per step
+    B, H = 64, 16
+    d = gin.kda_inputs(B, 8, H, seed=6000 + rank, s0_std=0.02, device=str(dev))
+    S = d["S0"].clone()
+    tok = [{key: d[key][:, i].contiguous() for key in ("q", "k", "v", "g", "beta")}
+           for i in range(8)]
+    o = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    it = [0]
+
+    def kstep():
+        x = tok[it[0] % 8]
+        gdn.kda_decode(x["q"], x["k"], x["v"], x["g"], x["beta"], S, o=o)
+        it[0] += 1
+    ms = time_steps(kstep, 32, 5, flush, stream)
+    t = statistics.mean(ms)
+    nb = B * H * (2 * STATE_BYTES + KDA_TOKEN_HEAD_BYTES)
+    out["kda_decode_b64_h16"] = {
+        "us_per_step": round(t * 1e3, 3),
+        "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
+        "l2": "flushed before every step"}
+    del d, S, o
+    torch.cuda.empty_cache()
     return out
 
 
@@ -542,6 +613,9 @@ PROFILE_CASES = {
     "decode": ("decode_b64_h16", None, 5),
     "prefill_b4_h32_t2048": (None, 64, 3),   # the large prefill's structure on 2048 tokens
     "headline": ("prefill_b1_h16_t512", 64, 3),
+    "kda_b1_h16_t512": (None, None, 3),       # per-channel gate, headline shape
+    "kda_b4_h32_t2048": (None, None, 3),      # per-channel gate, a large batch
+    "kda_decode": (None, None, 5),            # per-channel gate, B64 H16 one token
 }
 
 
@@ -551,7 +625,20 @@ def run_profile_case(name):
     from gated_deltanet_linear_20_b200 import gdn
     dev = torch.device("cuda", 0)
     wname, chunk, calls = PROFILE_CASES[name]
-    if name == "decode":
+    if name.startswith("kda"):
+        B, T, H = {"kda_b1_h16_t512": (1, 512, 16), "kda_b4_h32_t2048": (4, 2048, 32),
+                   "kda_decode": (64, calls, 16)}[name]
+        d = gin.kda_inputs(B, T, H, seed=0, g_mean=2.0 if B == 4 else 0.0,
+                           s0_std=0.02 if name == "kda_decode" else None, device=str(dev))
+        if name == "kda_decode":
+            S = d["S0"].clone()
+            for i in range(calls):
+                x = {key: d[key][:, i].contiguous() for key in ("q", "k", "v", "g", "beta")}
+                gdn.kda_decode(x["q"], x["k"], x["v"], x["g"], x["beta"], S)
+        else:
+            for _ in range(calls):
+                gdn.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None)
+    elif name == "decode":
         w = gin.WORKLOADS[wname]
         d = gin.workload_inputs(w, seed=0, device=str(dev))
         S = d["S"].clone()

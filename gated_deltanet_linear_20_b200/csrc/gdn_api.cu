@@ -473,6 +473,55 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
   return gdn::launch_decode(a, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
 }
 
+int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, const float* S0, float* o, float* S_T, int B, int T,
+                    int H, int Dk, int Dv, int* status, void* stream) {
+  (void)status;  // the kernel has no device-side waits
+  if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (Dk != kHeadDim || Dv != kHeadDim) return GDN_ERR_UNSUPPORTED;
+  const long long heads = (long long)B * H;
+  if (heads * kHeadDim * kHeadDim > 0x7fffffffLL || heads * T * kHeadDim > 0x7fffffffLL)
+    return GDN_ERR_SHAPE;
+  if (heads == 0) return GDN_OK;
+  if (!S_T) return GDN_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
+  if (!aligned(S_T, 16) || (S0 && !aligned(S0, 16))) return GDN_ERR_ALIGN;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
+                !aligned(o, 4) || !aligned(beta, 4)))
+    return GDN_ERR_ALIGN;
+  const size_t toks = size_t(heads) * T;
+  const size_t vec_bf16 = toks * kHeadDim * 2, vec_f32 = toks * kHeadDim * 4;
+  const size_t beta_bytes = toks * 4, state_bytes = size_t(heads) * kHeadDim * kHeadDim * 4;
+  if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
+  if (T > 0) {
+    const void* ins[5] = {q, k, v, g, beta};
+    const size_t in_bytes[5] = {vec_bf16, vec_bf16, vec_bf16, vec_f32, beta_bytes};
+    for (int i = 0; i < 5; ++i)
+      if (overlaps(o, vec_f32, ins[i], in_bytes[i]) || overlaps(S_T, state_bytes, ins[i], in_bytes[i]))
+        return GDN_ERR_ALIAS;
+    if (overlaps(o, vec_f32, S_T, state_bytes) || overlaps(o, vec_f32, S0, state_bytes))
+      return GDN_ERR_ALIAS;
+  } else if (S0 == S_T) {
+    return GDN_OK;
+  }
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+  int sms = 0;
+  const int rc = num_sms(&sms);
+  if (rc != GDN_OK) return rc;
+  gdn::KdaArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                 static_cast<const __nv_bfloat16*>(v), g, beta, S0, S_T, o, B, H, T};
+  return gdn::launch_kda(a, sms, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
+}
+
+int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
+                   int* status, void* stream) {
+  if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
+  return gdn_kda_prefill(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, status, stream);
+}
+
 int gdn_query_status(const int* status_dev, void* stream) {
   if (!status_dev) return GDN_ERR_NULL;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN_ERR_LAUNCH;

@@ -61,6 +61,18 @@ struct DecodeArgs {
   int o_bf16;     // o is bf16 (same layout)
 };
 
+struct KdaArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const __nv_bfloat16* v;
+  const float* g;     // [B][T][H][128]: per-channel log decays
+  const float* beta;  // [B][T][H]
+  const float* S_in;  // [B][H][128][128] or null (zeros)
+  float* S_out;       // may equal S_in
+  float* o;           // [B][T][H][128]
+  int B, H, T;
+};
+
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device
 // (slot: a small per-kernel index); returns false if the attribute call failed.
 bool ensure_smem_attr(const void* func, int slot, int bytes);
@@ -74,5 +86,8 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Second pass of the segmented schedule (a.nseg > 1).
 int launch_segment_fix(const PrefillArgs& a, cudaStream_t stream);
+// Per-channel-gate recurrence; num_sms picks the rows per CTA.
+int launch_kda(const KdaArgs& a, int num_sms, cudaStream_t stream);
+int kda_rows_per_cta(long long heads, int num_sms);
 
 }  // namespace gdn

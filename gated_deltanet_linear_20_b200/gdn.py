@@ -60,10 +60,14 @@ _lib.gdn_decode_step.argtypes = [_vp] * 7 + [_ci] * 4 + [_vp, _vp]
 _lib.gdn_decode_step.restype = _ci
 _lib.gdn_decode_tokens.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp]
 _lib.gdn_decode_tokens.restype = _ci
+_lib.gdn_kda_prefill.argtypes = [_vp] * 8 + [_ci] * 5 + [_vp, _vp]
+_lib.gdn_kda_prefill.restype = _ci
+_lib.gdn_kda_decode.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp]
+_lib.gdn_kda_decode.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
-ABI_VERSION = 5
+ABI_VERSION = 6
 if _lib.gdn_abi_version() != ABI_VERSION:
     raise ImportError(f"libgdn_b200.so ABI {_lib.gdn_abi_version()} != binding ABI {ABI_VERSION}")
 
@@ -383,6 +387,77 @@ def query_status(status: torch.Tensor) -> int:
     return int(_lib.gdn_query_status(_ptr(status), _stream_handle(status.device)))
 
 
+def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                beta: torch.Tensor, S0: Optional[torch.Tensor] = None, *,
+                o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-channel-gate (KDA) prefill: returns (o [B,T,H,Dv] fp32, S_T [B,H,Dv,Dk] fp32).
+
+    q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g [B,T,H,Dk] fp32 (log decay per key
+    channel); beta [B,T,H] fp32; S0 [B,H,Dv,Dk] fp32 or None (zeros).  ``S_T``
+    may be ``S0`` (in place).  Launches on the current stream."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B,T,H,Dk]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn.kda_prefill runs on CUDA tensors only (no CPU path)")
+    _check(q, "q", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(k, "k", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(v, "v", torch.bfloat16, (B, T, H, Dv), dev)
+    _check(g, "g", torch.float32, (B, T, H, Dk), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (B, H, Dv, Dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
+    if S_T is None:
+        S_T = torch.empty((B, H, Dv, Dk), dtype=torch.float32, device=dev)
+    _check(S_T, "S_T", torch.float32, (B, H, Dv, Dk), dev)
+    rc = _lib.gdn_kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                              _ptr(S_T), B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_kda_prefill")
+    return o, S_T
+
+
+def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+               beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
+               status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per-channel-gate (KDA) decode; S [B,H,Dv,Dk] fp32 is updated in place.
+
+    One token: q, k [B,H,Dk], v [B,H,Dv], g [B,H,Dk], beta [B,H] -> o [B,H,Dv].
+    T tokens: the same with a T axis after B ([B,T,H,...]) -> o [B,T,H,Dv]."""
+    one = q.dim() == 3
+    if one:
+        q, k, v, g, beta = (x.unsqueeze(1) for x in (q, k, v, g, beta))
+        if o is not None:
+            o = o.unsqueeze(1)
+    if q.dim() != 4:
+        raise ValueError("q must be [B,H,Dk] or [B,T,H,Dk]")
+    B, T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn.kda_decode runs on CUDA tensors only (no CPU path)")
+    _check(q, "q", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(k, "k", torch.bfloat16, (B, T, H, Dk), dev)
+    _check(v, "v", torch.bfloat16, (B, T, H, Dv), dev)
+    _check(g, "g", torch.float32, (B, T, H, Dk), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    _check(S, "S", torch.float32, (B, H, Dv, Dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
+    rc = _lib.gdn_kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                             B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_kda_decode")
+    return o[:, 0] if one else o
+
+
 def raw_prefill(*args) -> int:
     """Direct call of the C entry point with raw integers/pointers (tests use it
     to exercise argument validation without any tensor)."""
@@ -411,3 +486,11 @@ def raw_decode_tokens(*args) -> int:
 
 def raw_decode_step(*args) -> int:
     return int(_lib.gdn_decode_step(*args))
+
+
+def raw_kda_prefill(*args) -> int:
+    return int(_lib.gdn_kda_prefill(*args))
+
+
+def raw_kda_decode(*args) -> int:
+    return int(_lib.gdn_kda_decode(*args))

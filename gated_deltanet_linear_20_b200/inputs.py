@@ -130,6 +130,50 @@ def _prefill_inputs_torch(B, T, H, Dk, Dv, seed, g_mean, s0_std, device):
     return out
 
 
+def kda_inputs(B: int, T: int, H: int, Dk: int = 128, Dv: int = 128, *, seed: int = 0,
+               g_mean: float = 0.0, s0_std: Optional[float] = None,
+               device: str = "cpu") -> dict:
+    """Draw one batch for the per-channel gate (KDA).  The recipe of
+    ``prefill_inputs`` with one gate draw per key channel: g [B,T,H,Dk] fp32 =
+    logsigmoid(N(g_mean, 1)).  Draw order q, k, v, g_raw, beta_raw, S0."""
+    if str(device).startswith("cuda"):
+        gen = torch.Generator(device=device)
+        gen.manual_seed(seed)
+        out = {}
+        for name, D in (("q", Dk), ("k", Dk)):
+            x = torch.randn((B, T, H, D), generator=gen, device=device, dtype=torch.float32)
+            out[name] = (x / torch.sqrt((x * x).sum(-1, keepdim=True))).to(torch.bfloat16)
+            del x
+        out["v"] = torch.randn((B, T, H, Dv), generator=gen, device=device,
+                               dtype=torch.float32).to(torch.bfloat16)
+        g_raw = torch.randn((B, T, H, Dk), generator=gen, device=device,
+                            dtype=torch.float64) + g_mean
+        out["g"] = torch.nn.functional.logsigmoid(g_raw).to(torch.float32)
+        del g_raw
+        b_raw = torch.randn((B, T, H), generator=gen, device=device, dtype=torch.float64)
+        out["beta"] = torch.sigmoid(b_raw).to(torch.float32)
+        out["S0"] = None
+        if s0_std is not None:
+            out["S0"] = torch.randn((B, H, Dv, Dk), generator=gen, device=device,
+                                    dtype=torch.float32) * s0_std
+        return out
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, H, Dk), dtype=np.float32)
+    k = rng.standard_normal((B, T, H, Dk), dtype=np.float32)
+    v = rng.standard_normal((B, T, H, Dv), dtype=np.float32)
+    g_raw = rng.standard_normal((B, T, H, Dk), dtype=np.float32) + np.float32(g_mean)
+    b_raw = rng.standard_normal((B, T, H), dtype=np.float32)
+    S0 = None
+    if s0_std is not None:
+        S0 = torch.from_numpy((rng.standard_normal((B, H, Dv, Dk), dtype=np.float32)
+                               * np.float32(s0_std)).astype(np.float32))
+    return dict(q=_l2norm_bf16_np(q), k=_l2norm_bf16_np(k),
+                v=torch.from_numpy(v).to(torch.bfloat16),
+                g=torch.from_numpy(_logsigmoid64(g_raw).astype(np.float32)),
+                beta=torch.from_numpy(_sigmoid64(b_raw).astype(np.float32)),
+                S0=S0)
+
+
 def decode_inputs(B: int, H: int, steps: int, Dk: int = 128, Dv: int = 128, *, seed: int = 0,
                   g_mean: float = 0.0, s0_std: float = 0.02, device: str = "cpu") -> dict:
     """Draw ``steps`` decode steps up front.  q, k [steps,B,H,Dk] bf16;

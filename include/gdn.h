@@ -60,7 +60,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 5
+#define GDN_ABI_VERSION 6
 
 enum gdn_status_code {
   GDN_OK = 0,
@@ -255,6 +255,35 @@ int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* 
 int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
                   const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                   const gdn_options* opts, int* status, void* stream);
+
+/* Delta rule with a per-channel gate (KDA): alpha_t = exp(g_t) is a vector
+ * over the key channels, applied where the scalar gate is (the variant that the
+ * ROCmFPX gated-delta-net prefill note, bittide.aicompass.dev article
+ * d2880479, lists among the cases its fused kernel left to the old path):
+ *     S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t
+ * for t = 1..T of each of the B*H chains, in fp32, token by token.
+ *   q, k [B][T][H][Dk] bf16; v [B][T][H][Dv] bf16 (device, 16-byte aligned)
+ *   g    [B][T][H][Dk] fp32, natural-log decays (device, 16-byte aligned;
+ *        g > 0 is accepted and grows the state)
+ *   beta [B][T][H] fp32 (device)
+ *   S0   [B][H][Dv][Dk] fp32 or NULL (zeros); S_T written, same layout; S_T
+ *        may be S0 (in place) but may not partly overlap it (16-byte aligned)
+ *   o    [B][T][H][Dv] fp32, written (device); may not overlap any other array
+ *   Dk, Dv must be 128.  B*H == 0 is a no-op; T == 0 copies S0 (or zeros) to S_T.
+ * status is accepted for symmetry (no device-side waits; never written) and
+ * stream is a cudaStream_t.  Returns GDN_OK or a negative code; nothing is
+ * launched on an error. */
+int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
+                    const float* beta, const float* S0, float* o, float* S_T, int B, int T,
+                    int H, int Dk, int Dv, int* status, void* stream);
+
+/* gdn_kda_prefill with the state updated in place: T tokens per sequence
+ * starting from S and leaving S_T in S (T = 1: one decode step).  Arguments as
+ * for gdn_kda_prefill with S0 = S_T = S. */
+int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
+                   const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
+                   int* status, void* stream);
 
 /* Synchronises `stream`, then reads the device status word written by the
  * kernels.  Returns GDN_OK, GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_NULL (status_dev is

@@ -32,7 +32,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("gdn_prefill", "gdn_prefill_ws", "gdn_prefill_varlen", "gdn_prefill_workspace_bytes",
               "gdn_prefill_schedule", "gdn_prefill_ex", "gdn_decode_step", "gdn_decode_tokens",
-              "gdn_decode_ex", "gdn_abi_version",
+              "gdn_decode_ex", "gdn_kda_prefill", "gdn_kda_decode", "gdn_abi_version",
               "gdn_status_str", "gdn_query_status"):
         assert n in names
 
@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(gdn):
 
 
 def test_abi_version_and_status_strings(gdn):
-    assert gdn.abi_version() == 5
+    assert gdn.abi_version() == 6
     for code in range(-9, 1):
         s = gdn.status_str(code)
         assert s and s != "unknown status code"
@@ -279,3 +279,57 @@ def test_tensor_binding_refuses_cpu_tensors(gdn):
         gdn.prefill(q, q, q, g, g)
     with pytest.raises(ValueError):
         gdn.decode_step(q[:, 0], q[:, 0], q[:, 0], g[:, 0], g[:, 0], torch.zeros(1, 1, 128, 128))
+
+
+# ---------------------------------------------------------------------------- KDA entry points
+
+def kda_args(**over):
+    # B=1 T=64 H=2: q/k/v 32 KiB each, g 64 KiB, o 64 KiB, state 128 KiB
+    a = dict(q=P, k=P + 0x1000000, v=P + 0x2000000, g=P + 0x3000000, beta=P + 0x3100000,
+             S0=P + 0x4000000, o=P + 0x5000000, S_T=P + 0x6000000, B=1, T=64, H=2, Dk=128,
+             Dv=128, status=None, stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "g", "beta", "S0", "o", "S_T", "B", "T", "H", "Dk",
+                           "Dv", "status", "stream")]
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(B=-1), -3), (dict(T=-1), -3), (dict(Dk=64), -4), (dict(Dv=256), -4),
+    (dict(S_T=None), -1), (dict(q=None), -1), (dict(g=None), -1), (dict(o=None), -1),
+    (dict(g=P + 0x3000004), -2),                  # g rows are copied in 16-byte pieces
+    (dict(S_T=P + 0x6000008), -2), (dict(o=P + 0x5000002), -2),
+    (dict(S0=P + 0x6000000 + 0x1000), -5),        # S0 partly overlaps S_T
+    (dict(o=P + 0x3000000 + 0x100), -5),           # o over g
+    (dict(S_T=P + 0x2000000 + 0x40), -5),          # S_T over v
+    (dict(o=P + 0x6000000 - 0x100), -5),           # o runs into S_T
+], ids=lambda x: str(x))
+def test_kda_prefill_rejects_bad_arguments(gdn, over, code):
+    assert gdn.raw_kda_prefill(*kda_args(**over)) == code
+
+
+def test_kda_no_op_shapes_return_ok_without_a_device(gdn):
+    assert gdn.raw_kda_prefill(*kda_args(B=0)) == 0
+    assert gdn.raw_kda_prefill(*kda_args(H=0, q=None, S_T=None)) == 0
+    # T = 0 in place has nothing to do; T = 0 to another buffer copies (needs the device)
+    assert gdn.raw_kda_prefill(*kda_args(T=0, S0=P + 0x6000000)) == 0
+    assert gdn.raw_kda_prefill(*kda_args(T=0)) not in (0, -1, -2, -3, -4, -5)
+
+
+def test_kda_in_place_state_is_accepted_by_validation(gdn):
+    """S0 == S_T is the decode form: validation passes it (the call then fails
+    only for want of a device)."""
+    rc = gdn.raw_kda_prefill(*kda_args(S0=P + 0x6000000))
+    assert rc not in (-1, -2, -3, -4, -5)
+
+
+def test_kda_decode_argument_checks(gdn):
+    d = dict(q=P, k=P + 0x1000000, v=P + 0x2000000, g=P + 0x3000000, beta=P + 0x3100000,
+             S=P + 0x4000000, o=P + 0x5000000, B=4, T=1, H=2, Dk=128, Dv=128, status=None,
+             stream=None)
+    order = ("q", "k", "v", "g", "beta", "S", "o", "B", "T", "H", "Dk", "Dv", "status", "stream")
+    call = lambda **o: gdn.raw_kda_decode(*[{**d, **o}[k] for k in order])
+    assert call(S=None) == -1
+    assert call(B=-2) == -3
+    assert call(Dk=256) == -4
+    assert call(o=P + 0x4000000 + 0x10) == -5      # o inside the state
+    assert call(B=0) == 0
