@@ -474,6 +474,54 @@ def run_extras(args, dev, stream, flush, peaks, rank):
     del dl, ol, sl
     torch.cuda.empty_cache()
     out.update(run_kda_extras(dev, stream, flush, peaks, rank, steps))
+    out.update(run_head_dim_extras(dev, stream, flush, peaks, rank, steps))
+    return out
+
+
+def run_head_dim_extras(dev, stream, flush, peaks, rank, steps):
+    """Scalar gate at head dims other than 128 x 128 (the row-parallel fp32
+    kernel): the 16-head, 512-token prefill and the batched decode step."""
+    from gated_deltanet_linear_20_b200 import gdn
+    out = {}
+    peak_ops = alu_peak_tops(dev)
+    for dk, dv in ((64, 64), (256, 256), (128, 256)):
+        d = gin.prefill_inputs(1, 512, 16, dk, dv, seed=7000 + rank, device=str(dev))
+        o = torch.empty((1, 512, 16, dv), dtype=torch.float32, device=dev)
+        sT = torch.empty((1, 16, dv, dk), dtype=torch.float32, device=dev)
+        ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None,
+                                            o=o, S_T=sT), steps, 3, flush, stream)
+        t = statistics.mean(ms)
+        ops = 512 * 16 * 4 * dk * dv
+        out[f"prefill_b1_h16_t512_dk{dk}_dv{dv}"] = {
+            "tokens_per_s": round(512 / (t / 1e3), 1), "ms": round(t, 5),
+            "roofline": {"bound": "alu", "achieved": round(ops / (t / 1e3) / 1e12, 3),
+                         "peak": round(peak_ops, 2), "unit": "Tops/s (fp32 lane ops)",
+                         "frac": round(ops / (t / 1e3) / 1e12 / peak_ops, 4)}}
+        del d, o, sT
+    for dk, dv in ((256, 256), (64, 64)):
+        B, H = 64, 16
+        d = gin.prefill_inputs(B, 4, H, dk, dv, seed=7500 + rank, s0_std=0.02, device=str(dev))
+        S = d["S0"].clone()
+        tok = [{key: d[key][:, i].contiguous() for key in ("q", "k", "v", "g", "beta")}
+               for i in range(4)]
+        o = torch.empty((B, H, dv), dtype=torch.float32, device=dev)
+        it = [0]
+
+        def dstep():
+            x = tok[it[0] % 4]
+            gdn.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], S, o=o)
+            it[0] += 1
+        ms = time_steps(dstep, 32, 5, flush, stream)
+        t = statistics.mean(ms)
+        nb = B * H * (2 * dk * dv * 4 + 2 * dk * 2 + dv * 2 + 8 + dv * 4)
+        out[f"decode_b64_h16_dk{dk}_dv{dv}"] = {
+            "us_per_step": round(t * 1e3, 3), "state_MiB": B * H * dk * dv * 4 / 2**20,
+            "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
+            "l2": "flushed before every step"}
+        del d, S, o, tok
+    torch.cuda.empty_cache()
     return out
 
 

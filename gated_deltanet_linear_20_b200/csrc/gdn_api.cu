@@ -164,6 +164,52 @@ bool read_options(const gdn_options* opts, int* qk_norm, float* q_scale, int* o_
   return opts->q_scale == opts->q_scale;  // not NaN
 }
 
+// The row-parallel fp32 kernel: the per-channel gate at every supported head
+// dim, and the scalar gate at head dims other than 128 x 128.  g is [B][T][H][Dk]
+// with vector_gate, else [B][T][H].  S_T may be S0 (in place).
+int rows_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
+              const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
+              bool vector_gate, void* stream) {
+  if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (!gdn::rows_head_dims_ok(Dk, Dv)) return GDN_ERR_UNSUPPORTED;
+  const long long heads = (long long)B * H;
+  if (heads * Dk * Dv > 0x7fffffffLL || heads * T * (Dk > Dv ? Dk : Dv) > 0x7fffffffLL)
+    return GDN_ERR_SHAPE;
+  if (heads == 0) return GDN_OK;
+  if (!S_T) return GDN_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
+  if (!aligned(S_T, 16) || (S0 && !aligned(S0, 16))) return GDN_ERR_ALIGN;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+                !aligned(g, vector_gate ? 16 : 4) || !aligned(o, 4) || !aligned(beta, 4)))
+    return GDN_ERR_ALIGN;
+  const size_t toks = size_t(heads) * T;
+  const size_t qk_bytes = toks * Dk * 2, v_bytes = toks * Dv * 2, o_bytes = toks * Dv * 4;
+  const size_t g_bytes = toks * (vector_gate ? Dk : 1) * 4, beta_bytes = toks * 4;
+  const size_t state_bytes = size_t(heads) * Dk * Dv * 4;
+  if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
+  if (T > 0) {
+    const void* ins[5] = {q, k, v, g, beta};
+    const size_t in_bytes[5] = {qk_bytes, qk_bytes, v_bytes, g_bytes, beta_bytes};
+    for (int i = 0; i < 5; ++i)
+      if (overlaps(o, o_bytes, ins[i], in_bytes[i]) || overlaps(S_T, state_bytes, ins[i], in_bytes[i]))
+        return GDN_ERR_ALIAS;
+    if (overlaps(o, o_bytes, S_T, state_bytes) || overlaps(o, o_bytes, S0, state_bytes))
+      return GDN_ERR_ALIAS;
+  } else if (S0 == S_T) {
+    return GDN_OK;
+  }
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+  int sms = 0;
+  const int rc = num_sms(&sms);
+  if (rc != GDN_OK) return rc;
+  gdn::RowArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                 static_cast<const __nv_bfloat16*>(v), g, beta, S0, S_T, o, B, H, T, Dv};
+  return gdn::launch_rows(a, Dk, vector_gate, sms, static_cast<cudaStream_t>(stream)) == 0
+             ? GDN_OK
+             : GDN_ERR_LAUNCH;
+}
+
 int prefill_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
                  const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
                  int chunk, void* ws, size_t ws_bytes, bool allow_segments, int* status,
@@ -173,7 +219,12 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
   if (o_bf16) allow_segments = false;  // the segment fix accumulates o in fp32
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
-  if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
+  if (chunk != 16 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+  if (Dk != kHeadDim || Dv != kHeadDim) {
+    // other head dims: the row kernel (no chunking, no workspace, no fused options)
+    if (qk_norm || q_scale != 1.f || o_bf16) return GDN_ERR_UNSUPPORTED;
+    return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, false, stream);
+  }
   const long long chains = (long long)B * H;
   const long long act = chains * T * kHeadDim;
   if (act > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL) return GDN_ERR_SHAPE;
@@ -260,9 +311,9 @@ int static_workspace(void** out) {
 
 namespace gdn {
 bool ensure_smem_attr(const void* func, int slot, int bytes) {
-  static std::atomic<uint64_t> done[16];  // bit d: device d, per kernel slot
+  static std::atomic<uint64_t> done[64];  // bit d: device d, per kernel slot
   int dev = 0;
-  if (slot < 0 || slot >= 16 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+  if (slot < 0 || slot >= 64 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return false;
   const uint64_t bit = uint64_t(1) << dev;
   if (done[slot].load(std::memory_order_acquire) & bit) return true;
@@ -404,7 +455,10 @@ int gdn_prefill_static_ws(const void* q, const void* k, const void* v, const flo
   // the shape checks of prefill_impl come first, so that bad arguments get
   // their own codes rather than the limit
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
-  if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
+  if (chunk != 16 && chunk != 64) return GDN_ERR_UNSUPPORTED;
+  if (Dk != kHeadDim || Dv != kHeadDim)  // the row kernel needs no scratch
+    return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, nullptr, 0, false,
+                        status, stream);
   const long long chains = (long long)B * H;
   if (chains * T * kHeadDim > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL)
     return GDN_ERR_SHAPE;
@@ -446,7 +500,13 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
   float q_scale = 1.f;
   if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
   if (B < 0 || H < 0 || T < 0) return GDN_ERR_SHAPE;
-  if (Dk != kHeadDim || Dv != kHeadDim) return GDN_ERR_UNSUPPORTED;
+  if (Dk != kHeadDim || Dv != kHeadDim) {
+    // other head dims: the row kernel with the state in place (no fused options)
+    if (!gdn::rows_head_dims_ok(Dk, Dv) || qk_norm || q_scale != 1.f || o_bf16)
+      return GDN_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
+    return rows_impl(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, false, stream);
+  }
   const long long heads = (long long)B * H;
   if (heads * kHeadDim * kHeadDim > 0x7fffffffLL || heads * T * kHeadDim > 0x7fffffffLL)
     return GDN_ERR_SHAPE;
@@ -477,41 +537,7 @@ int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
                     const float* beta, const float* S0, float* o, float* S_T, int B, int T,
                     int H, int Dk, int Dv, int* status, void* stream) {
   (void)status;  // the kernel has no device-side waits
-  if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
-  if (Dk != kHeadDim || Dv != kHeadDim) return GDN_ERR_UNSUPPORTED;
-  const long long heads = (long long)B * H;
-  if (heads * kHeadDim * kHeadDim > 0x7fffffffLL || heads * T * kHeadDim > 0x7fffffffLL)
-    return GDN_ERR_SHAPE;
-  if (heads == 0) return GDN_OK;
-  if (!S_T) return GDN_ERR_NULL;
-  if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
-  if (!aligned(S_T, 16) || (S0 && !aligned(S0, 16))) return GDN_ERR_ALIGN;
-  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
-                !aligned(o, 4) || !aligned(beta, 4)))
-    return GDN_ERR_ALIGN;
-  const size_t toks = size_t(heads) * T;
-  const size_t vec_bf16 = toks * kHeadDim * 2, vec_f32 = toks * kHeadDim * 4;
-  const size_t beta_bytes = toks * 4, state_bytes = size_t(heads) * kHeadDim * kHeadDim * 4;
-  if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
-  if (T > 0) {
-    const void* ins[5] = {q, k, v, g, beta};
-    const size_t in_bytes[5] = {vec_bf16, vec_bf16, vec_bf16, vec_f32, beta_bytes};
-    for (int i = 0; i < 5; ++i)
-      if (overlaps(o, vec_f32, ins[i], in_bytes[i]) || overlaps(S_T, state_bytes, ins[i], in_bytes[i]))
-        return GDN_ERR_ALIAS;
-    if (overlaps(o, vec_f32, S_T, state_bytes) || overlaps(o, vec_f32, S0, state_bytes))
-      return GDN_ERR_ALIAS;
-  } else if (S0 == S_T) {
-    return GDN_OK;
-  }
-  const int dev_ok = check_device();
-  if (dev_ok != GDN_OK) return dev_ok;
-  int sms = 0;
-  const int rc = num_sms(&sms);
-  if (rc != GDN_OK) return rc;
-  gdn::KdaArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                 static_cast<const __nv_bfloat16*>(v), g, beta, S0, S_T, o, B, H, T};
-  return gdn::launch_kda(a, sms, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
+  return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, true, stream);
 }
 
 int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,

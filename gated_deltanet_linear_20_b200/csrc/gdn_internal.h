@@ -61,16 +61,17 @@ struct DecodeArgs {
   int o_bf16;     // o is bf16 (same layout)
 };
 
-struct KdaArgs {
-  const __nv_bfloat16* q;
+// Row-parallel fp32 kernel (any supported head dims; scalar or per-channel gate).
+struct RowArgs {
+  const __nv_bfloat16* q;  // [B][T][H][Dk]
   const __nv_bfloat16* k;
-  const __nv_bfloat16* v;
-  const float* g;     // [B][T][H][128]: per-channel log decays
-  const float* beta;  // [B][T][H]
-  const float* S_in;  // [B][H][128][128] or null (zeros)
-  float* S_out;       // may equal S_in
-  float* o;           // [B][T][H][128]
-  int B, H, T;
+  const __nv_bfloat16* v;  // [B][T][H][Dv]
+  const float* g;          // [B][T][H][Dk] (per-channel gate) or [B][T][H]
+  const float* beta;       // [B][T][H]
+  const float* S_in;       // [B][H][Dv][Dk] or null (zeros)
+  float* S_out;            // may equal S_in
+  float* o;                // [B][T][H][Dv]
+  int B, H, T, Dv;
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device
@@ -86,8 +87,10 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Second pass of the segmented schedule (a.nseg > 1).
 int launch_segment_fix(const PrefillArgs& a, cudaStream_t stream);
-// Per-channel-gate recurrence; num_sms picks the rows per CTA.
-int launch_kda(const KdaArgs& a, int num_sms, cudaStream_t stream);
-int kda_rows_per_cta(long long heads, int num_sms);
+// Row-parallel recurrence (Dk, Dv in {64, 128, 256}); num_sms picks the rows
+// per CTA.  Returns 0, or -1 when the dims are unsupported or the launch failed.
+int launch_rows(const RowArgs& a, int Dk, bool vector_gate, int num_sms, cudaStream_t stream);
+int rows_per_cta(long long heads, int Dv, int num_sms);
+bool rows_head_dims_ok(int Dk, int Dv);
 
 }  // namespace gdn

@@ -1,0 +1,370 @@
+// Row-parallel fp32 recurrence: every head dim the chunked tensor-core kernel
+// does not cover (Dk, Dv in {64, 128, 256}, Dk != Dv included; the ROCmFPX
+// gated-delta-net prefill note, bittide.aicompass.dev article d2880479, lists
+// other head dims among the cases its fused kernel left to the old path), and
+// the per-channel gate (KDA, listed there too) at every head dim.
+//
+//   S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t,
+//
+// with alpha_t = exp(g_t) a vector over the Dk key channels (per-channel gate)
+// or the same scalar on every channel (the gated delta rule).  S in R^{Dv x Dk}
+// is stored [Dv][Dk].  Row i of S (a value channel) evolves on its own given
+// the token's k, q, alpha and beta:
+//   s'  = s o alpha                  (the decay, column by column)
+//   d   = beta (v_i - s' . k)        (delta-rule residual)
+//   s  <- s' + d k
+//   o_i = s . q = s' . q + d (k . q)
+// so the rows are split over warps and CTAs and each row walks the tokens in
+// fp32 registers, in the order of the recurrence: one kernel for prefill
+// (S0 -> S_T) and decode (S in place).
+//
+// Layout of a CTA: 4 warps; a warp holds RG groups of 4 rows; the 8 lanes of a
+// row hold the float4 column blocks j, j+8, j+16, .. (j = lane % 8, Dk/32
+// blocks), so the lanes of a row touch 128 contiguous bytes per access, in
+// global and in shared memory alike, and a dot product reduces over 8 lanes.
+// Tokens are staged NT at a time with cp.async into a double buffer (k, q, g,
+// this CTA's v rows, beta); one cooperative pass per chunk turns them into
+// fp32 k, q, alpha = exp(g) and k . q in shared memory, so each exp is taken
+// once per CTA and not once per row.  A single token (decode) skips the
+// staging: each lane reads its blocks straight from global memory.
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int WARPS = 4;
+constexpr int THREADS = WARPS * 32;
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ float dot44(const float4& a, const float4& b) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+__device__ __forceinline__ float4 bf16x4(uint2 raw) {
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ float4 mul4(const float4& s, const float4& a) {
+  return make_float4(s.x * a.x, s.y * a.y, s.z * a.z, s.w * a.w);
+}
+__device__ __forceinline__ float4 mul4(const float4& s, float a) {
+  return make_float4(s.x * a, s.y * a, s.z * a, s.w * a);
+}
+__device__ __forceinline__ float4 fma4(float d, const float4& k, const float4& s) {
+  return make_float4(fmaf(d, k.x, s.x), fmaf(d, k.y, s.y), fmaf(d, k.z, s.z), fmaf(d, k.w, s.w));
+}
+constexpr int round16(int x) { return (x + 15) / 16 * 16; }
+
+// Sum of v[0..N) by pairs (a tree, so that the partial dot products do not
+// form one long dependency chain).
+template <int N>
+__device__ __forceinline__ float tree_sum(const float (&v)[N]) {
+  if constexpr (N == 1) {
+    return v[0];
+  } else {
+    float h[(N + 1) / 2];
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) h[i] = v[2 * i] + v[2 * i + 1];
+    if constexpr (N % 2) h[N / 2] = v[N - 1];
+    return tree_sum<(N + 1) / 2>(h);
+  }
+}
+
+template <int DK, bool VG, int RG>
+struct Shape {
+  static constexpr int MB = DK / 32;                  // float4 column blocks per lane
+  static constexpr int NT = (VG ? 1536 : 2048) / DK;  // tokens per staged chunk
+  static constexpr int ROWS_PER_WARP = 4 * RG;
+  static constexpr int ROWS_PER_CTA = WARPS * ROWS_PER_WARP;  // 16 or 32
+  // staging buffer (cp.async target), bytes
+  static constexpr int R_K = 0;
+  static constexpr int R_Q = R_K + NT * DK * 2;
+  static constexpr int R_G = R_Q + NT * DK * 2;
+  static constexpr int R_V = R_G + round16(VG ? NT * DK * 4 : NT * 4);
+  static constexpr int R_B = R_V + NT * ROWS_PER_CTA * 2;
+  static constexpr int R_BYTES = round16(R_B + NT * 4);
+  // converted chunk, bytes
+  static constexpr int C_K = 2 * R_BYTES;
+  static constexpr int C_Q = C_K + NT * DK * 4;
+  static constexpr int C_A = C_Q + NT * DK * 4;
+  static constexpr int C_KQ = C_A + round16(VG ? NT * DK * 4 : NT * 4);
+  static constexpr int SMEM = C_KQ + NT * 4;
+  static_assert(DK % 32 == 0 && (NT * DK * 2) % 16 == 0, "16-byte staging pieces");
+};
+
+template <int DK, bool VG, int RG>
+__device__ __forceinline__ void stage_chunk(const RowArgs& a, uint8_t* buf, int b, int h, int t0,
+                                            int n, int vrow0) {
+  using S = Shape<DK, VG, RG>;
+  const int tid = threadIdx.x;
+  const uint32_t base = smem_addr(buf);
+  auto tok = [&](int j) { return (size_t(b) * a.T + t0 + j) * a.H + h; };  // [B][T][H] index
+  constexpr int KP = DK / 8;  // 16-byte pieces of a bf16 row of k or q
+  for (int p = tid; p < n * KP; p += THREADS) {
+    const int j = p / KP, c = p % KP;
+    const size_t e = tok(j) * DK + c * 8;
+    cp16(base + S::R_K + j * DK * 2 + c * 16, a.k + e);
+    cp16(base + S::R_Q + j * DK * 2 + c * 16, a.q + e);
+  }
+  if constexpr (VG) {
+    constexpr int GP = DK / 4;  // 16-byte pieces of an fp32 gate row
+    for (int p = tid; p < n * GP; p += THREADS) {
+      const int j = p / GP, c = p % GP;
+      cp16(base + S::R_G + j * DK * 4 + c * 16, a.g + tok(j) * DK + c * 4);
+    }
+  } else {
+    for (int p = tid; p < n; p += THREADS) cp4(base + S::R_G + p * 4, a.g + tok(p));
+  }
+  constexpr int VP = S::ROWS_PER_CTA / 8;  // this CTA's v rows: 2 or 4 pieces per token
+  for (int p = tid; p < n * VP; p += THREADS) {
+    const int j = p / VP, c = p % VP;
+    cp16(base + S::R_V + j * S::ROWS_PER_CTA * 2 + c * 16, a.v + tok(j) * a.Dv + vrow0 + c * 8);
+  }
+  for (int p = tid; p < n; p += THREADS) cp4(base + S::R_B + p * 4, a.beta + tok(p));
+  cp_commit();
+}
+
+// One token on this lane's rows.  kk, qq: k and q blocks; aa: the decay
+// blocks (per-channel gate) or aa[0].x the decay (scalar gate); kq: k . q, or
+// a lane's partial of it when KQ_PARTIAL (reduced here with sk and sq).
+template <int DK, bool VG, int RG, bool KQ_PARTIAL>
+__device__ __forceinline__ void apply_token(float4 (&s)[RG][DK / 32], const float4 (&kk)[DK / 32],
+                                            const float4 (&qq)[DK / 32],
+                                            const float4 (&aa)[VG ? DK / 32 : 1], float kq,
+                                            float beta, const float (&v)[RG], float (&o)[RG]) {
+  constexpr int MB = DK / 32;
+  float sk[RG], sq[RG];
+#pragma unroll
+  for (int i = 0; i < RG; ++i) {
+    float pk[MB], pq[MB];
+#pragma unroll
+    for (int m = 0; m < MB; ++m) {
+      s[i][m] = VG ? mul4(s[i][m], aa[m]) : mul4(s[i][m], aa[0].x);
+      pk[m] = dot44(s[i][m], kk[m]);
+      pq[m] = dot44(s[i][m], qq[m]);
+    }
+    sk[i] = tree_sum(pk);
+    sq[i] = tree_sum(pq);
+  }
+#pragma unroll
+  for (int off = 1; off < 8; off <<= 1) {
+#pragma unroll
+    for (int i = 0; i < RG; ++i) {
+      sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], off);
+      sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], off);
+    }
+    if constexpr (KQ_PARTIAL) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+  }
+#pragma unroll
+  for (int i = 0; i < RG; ++i) {
+    const float d = beta * (v[i] - sk[i]);
+#pragma unroll
+    for (int m = 0; m < MB; ++m) s[i][m] = fma4(d, kk[m], s[i][m]);
+    o[i] = fmaf(d, kq, sq[i]);
+  }
+}
+
+// DIRECT: a single token per chain (decode), read straight from global memory.
+template <int DK, bool VG, int RG, bool DIRECT>
+__global__ void __launch_bounds__(THREADS) rows_kernel(const RowArgs a) {
+  using S = Shape<DK, VG, RG>;
+  constexpr int MB = S::MB;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ctas_per_head = a.Dv / S::ROWS_PER_CTA;
+  const int head = blockIdx.x / ctas_per_head;  // b * H + h
+  const int b = head / a.H, h = head - b * a.H;
+  const int vrow0 = (blockIdx.x % ctas_per_head) * S::ROWS_PER_CTA;
+  const int j8 = lane & 7, sub = lane >> 3;
+  const int wrow = warp * S::ROWS_PER_WARP + sub;  // this lane's first row within the CTA
+
+  // rows vrow0 + wrow + 4 i, column blocks j8 + 8 m
+  float4 s[RG][MB];
+  const size_t srow = (size_t(head) * a.Dv + vrow0 + wrow) * DK;
+  if (a.S_in) {
+    const float4* src = reinterpret_cast<const float4*>(a.S_in + srow);
+#pragma unroll
+    for (int i = 0; i < RG; ++i)
+#pragma unroll
+      for (int m = 0; m < MB; ++m) s[i][m] = __ldcs(src + i * DK + j8 + 8 * m);  // +4 rows
+  } else {
+#pragma unroll
+    for (int i = 0; i < RG; ++i)
+#pragma unroll
+      for (int m = 0; m < MB; ++m) s[i][m] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+
+  if constexpr (DIRECT) {
+#pragma unroll 1
+    for (int t = 0; t < a.T; ++t) {
+      const size_t tok = (size_t(b) * a.T + t) * a.H + h;
+      float4 kk[MB], qq[MB], aa[VG ? MB : 1];
+      float kq = 0.f;
+#pragma unroll
+      for (int m = 0; m < MB; ++m) {
+        kk[m] = bf16x4(*reinterpret_cast<const uint2*>(a.k + tok * DK + 4 * (j8 + 8 * m)));
+        qq[m] = bf16x4(*reinterpret_cast<const uint2*>(a.q + tok * DK + 4 * (j8 + 8 * m)));
+        kq += dot44(kk[m], qq[m]);
+        if constexpr (VG) {
+          const float4 gv = *reinterpret_cast<const float4*>(a.g + tok * DK + 4 * (j8 + 8 * m));
+          aa[m] = make_float4(expf(gv.x), expf(gv.y), expf(gv.z), expf(gv.w));
+        }
+      }
+      if constexpr (!VG) aa[0].x = expf(a.g[tok]);
+      float v[RG], o[RG];
+#pragma unroll
+      for (int i = 0; i < RG; ++i) v[i] = __bfloat162float(a.v[tok * a.Dv + vrow0 + wrow + 4 * i]);
+      apply_token<DK, VG, RG, true>(s, kk, qq, aa, kq, a.beta[tok], v, o);
+      if (j8 == 0) {
+#pragma unroll
+        for (int i = 0; i < RG; ++i) a.o[tok * a.Dv + vrow0 + wrow + 4 * i] = o[i];
+      }
+    }
+  } else {
+    const int nch = (a.T + S::NT - 1) / S::NT;
+    if (nch > 0) stage_chunk<DK, VG, RG>(a, smem, b, h, 0, min(S::NT, a.T), vrow0);
+    const float4* ck = reinterpret_cast<const float4*>(smem + S::C_K);
+    const float4* cq = reinterpret_cast<const float4*>(smem + S::C_Q);
+    const float* caf = reinterpret_cast<const float*>(smem + S::C_A);
+    const float* ckq = reinterpret_cast<const float*>(smem + S::C_KQ);
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+      const int t0 = c * S::NT, n = min(S::NT, a.T - t0);
+      uint8_t* raw = smem + (c & 1) * S::R_BYTES;
+      if (c + 1 < nch) {
+        stage_chunk<DK, VG, RG>(a, smem + ((c + 1) & 1) * S::R_BYTES, b, h, t0 + S::NT,
+                                min(S::NT, a.T - t0 - S::NT), vrow0);
+        cp_wait<1>();
+      } else {
+        cp_wait<0>();
+      }
+      __syncthreads();
+      // convert: warp w takes tokens w, w+4, ..; lane l columns CPL l .. CPL l + CPL - 1
+      constexpr int CPL = DK / 32, PAIRS = CPL / 2;
+      for (int j = warp; j < n; j += WARPS) {
+        const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(raw + S::R_K + j * DK * 2);
+        const __nv_bfloat162* qr = reinterpret_cast<const __nv_bfloat162*>(raw + S::R_Q + j * DK * 2);
+        float2* kc = reinterpret_cast<float2*>(smem + S::C_K) + j * DK / 2;
+        float2* qc = reinterpret_cast<float2*>(smem + S::C_Q) + j * DK / 2;
+        float kq = 0.f;
+#pragma unroll
+        for (int e = 0; e < PAIRS; ++e) {
+          const float2 kf = __bfloat1622float2(kr[lane * PAIRS + e]);
+          const float2 qf = __bfloat1622float2(qr[lane * PAIRS + e]);
+          kc[lane * PAIRS + e] = kf;
+          qc[lane * PAIRS + e] = qf;
+          kq = fmaf(kf.x, qf.x, fmaf(kf.y, qf.y, kq));
+          if constexpr (VG) {
+            const float2 gv = reinterpret_cast<const float2*>(raw + S::R_G + j * DK * 4)[lane * PAIRS + e];
+            reinterpret_cast<float2*>(smem + S::C_A)[j * DK / 2 + lane * PAIRS + e] =
+                make_float2(expf(gv.x), expf(gv.y));
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+        if (lane == 0) {
+          reinterpret_cast<float*>(smem + S::C_KQ)[j] = kq;
+          if constexpr (!VG)
+            reinterpret_cast<float*>(smem + S::C_A)[j] =
+                expf(reinterpret_cast<const float*>(raw + S::R_G)[j]);
+        }
+      }
+      __syncthreads();
+
+      const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(raw + S::R_V);
+      const float* rb = reinterpret_cast<const float*>(raw + S::R_B);
+#pragma unroll 1
+      for (int j = 0; j < n; ++j) {
+        float4 kk[MB], qq[MB], aa[VG ? MB : 1];
+#pragma unroll
+        for (int m = 0; m < MB; ++m) {
+          kk[m] = ck[j * DK / 4 + j8 + 8 * m];
+          qq[m] = cq[j * DK / 4 + j8 + 8 * m];
+          if constexpr (VG) aa[m] = reinterpret_cast<const float4*>(caf)[j * DK / 4 + j8 + 8 * m];
+        }
+        if constexpr (!VG) aa[0].x = caf[j];
+        float v[RG], o[RG];
+#pragma unroll
+        for (int i = 0; i < RG; ++i) v[i] = __bfloat162float(rv[j * S::ROWS_PER_CTA + wrow + 4 * i]);
+        apply_token<DK, VG, RG, false>(s, kk, qq, aa, ckq[j], rb[j], v, o);
+        if (j8 == 0) {
+          const size_t orow = ((size_t(b) * a.T + t0 + j) * a.H + h) * a.Dv + vrow0 + wrow;
+#pragma unroll
+          for (int i = 0; i < RG; ++i) a.o[orow + 4 * i] = o[i];
+        }
+      }
+      __syncthreads();  // the converted chunk and this staging buffer are reused
+    }
+  }
+
+  float4* dst = reinterpret_cast<float4*>(a.S_out + srow);
+#pragma unroll
+  for (int i = 0; i < RG; ++i)
+#pragma unroll
+    for (int m = 0; m < MB; ++m) __stcs(dst + i * DK + j8 + 8 * m, s[i][m]);
+}
+
+template <int DK, bool VG, int RG, bool DIRECT>
+bool launch_one(const RowArgs& a, long long heads, cudaStream_t stream) {
+  using S = Shape<DK, VG, RG>;
+  const int smem = DIRECT ? 0 : S::SMEM;
+  const int slot = 16 + (DK == 64 ? 0 : DK == 128 ? 8 : 16) + (VG ? 4 : 0) + (RG - 1) * 2 + DIRECT;
+  auto kern = &rows_kernel<DK, VG, RG, DIRECT>;
+  if (smem > 48 * 1024 && !ensure_smem_attr(reinterpret_cast<const void*>(kern), slot, smem))
+    return false;
+  kern<<<unsigned(heads * (a.Dv / S::ROWS_PER_CTA)), THREADS, smem, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess;
+}
+
+template <int DK, bool VG>
+bool launch_dk(const RowArgs& a, long long heads, bool rg1, cudaStream_t stream) {
+  const bool direct = a.T == 1;
+  if (rg1)
+    return direct ? launch_one<DK, VG, 1, true>(a, heads, stream)
+                  : launch_one<DK, VG, 1, false>(a, heads, stream);
+  return direct ? launch_one<DK, VG, 2, true>(a, heads, stream)
+                : launch_one<DK, VG, 2, false>(a, heads, stream);
+}
+
+}  // namespace
+
+int rows_per_cta(long long heads, int Dv, int num_sms) {
+  // 16 rows per CTA while every CTA still gets an SM of its own (the chains
+  // are few: spread them); 32 rows per CTA otherwise, which halves the staging
+  // and conversion work per row
+  return heads * (Dv / 16) <= num_sms ? 16 : 32;
+}
+
+bool rows_head_dims_ok(int Dk, int Dv) {
+  auto ok = [](int d) { return d == 64 || d == 128 || d == 256; };
+  return ok(Dk) && ok(Dv);
+}
+
+int launch_rows(const RowArgs& a, int Dk, bool vector_gate, int num_sms, cudaStream_t stream) {
+  const long long heads = (long long)a.B * a.H;
+  if (heads == 0) return 0;
+  if (!rows_head_dims_ok(Dk, a.Dv)) return -1;
+  const bool rg1 = rows_per_cta(heads, a.Dv, num_sms) == 16;
+  bool ok;
+  if (Dk == 64)
+    ok = vector_gate ? launch_dk<64, true>(a, heads, rg1, stream) : launch_dk<64, false>(a, heads, rg1, stream);
+  else if (Dk == 128)
+    ok = vector_gate ? launch_dk<128, true>(a, heads, rg1, stream) : launch_dk<128, false>(a, heads, rg1, stream);
+  else
+    ok = vector_gate ? launch_dk<256, true>(a, heads, rg1, stream) : launch_dk<256, false>(a, heads, rg1, stream);
+  return ok ? 0 : -1;
+}
+
+}  // namespace gdn

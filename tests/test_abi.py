@@ -69,7 +69,7 @@ def prefill_args(**over):
 
 @pytest.mark.parametrize("over,code", [
     (dict(B=-1), -3), (dict(T=-5), -3), (dict(H=-2), -3),
-    (dict(Dk=64), -4), (dict(Dv=256), -4), (dict(chunk=32), -4), (dict(chunk=0), -4),
+    (dict(Dk=96), -4), (dict(Dv=512), -4), (dict(chunk=32), -4), (dict(chunk=0), -4),
     (dict(q=None), -1), (dict(o=None), -1), (dict(S_T=None), -1), (dict(g=None), -1),
     (dict(q=P + 8), -2), (dict(o=P + 0x40000004), -2), (dict(g=P + 0x30000002), -2),
     (dict(S0=P + 0x60000008), -2),
@@ -87,7 +87,7 @@ def test_prefill_empty_batch_is_a_noop(gdn):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(B=-1), -3), (dict(Dk=64), -4), (dict(chunk=32), -4), (dict(q=None), -1),
+    (dict(B=-1), -3), (dict(Dk=96), -4), (dict(chunk=32), -4), (dict(q=None), -1),
     (dict(q=P + 8), -2), (dict(o=P + 0x10000000 + 0x100), -5),
 ], ids=lambda x: str(x))
 def test_prefill_ws_rejects_bad_arguments_like_prefill(gdn, over, code):
@@ -245,7 +245,7 @@ def decode_tokens_args(**over):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(T=-1), -3), (dict(B=-1), -3), (dict(Dv=64), -4), (dict(k=None), -1),
+    (dict(T=-1), -3), (dict(B=-1), -3), (dict(Dv=32), -4), (dict(k=None), -1),
     (dict(o=P + 0x8000004), -2), (dict(o=P + 0x4000000 + 64), -5),
     (dict(v=P + 0x4000000 + 4096), -5),     # v overlaps the state
 ], ids=lambda x: str(x))
@@ -294,7 +294,7 @@ def kda_args(**over):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(B=-1), -3), (dict(T=-1), -3), (dict(Dk=64), -4), (dict(Dv=256), -4),
+    (dict(B=-1), -3), (dict(T=-1), -3), (dict(Dk=96), -4), (dict(Dv=512), -4),
     (dict(S_T=None), -1), (dict(q=None), -1), (dict(g=None), -1), (dict(o=None), -1),
     (dict(g=P + 0x3000004), -2),                  # g rows are copied in 16-byte pieces
     (dict(S_T=P + 0x6000008), -2), (dict(o=P + 0x5000002), -2),
@@ -330,6 +330,41 @@ def test_kda_decode_argument_checks(gdn):
     call = lambda **o: gdn.raw_kda_decode(*[{**d, **o}[k] for k in order])
     assert call(S=None) == -1
     assert call(B=-2) == -3
-    assert call(Dk=256) == -4
+    assert call(Dk=100) == -4
     assert call(o=P + 0x4000000 + 0x10) == -5      # o inside the state
     assert call(B=0) == 0
+
+
+# ---------------------------------------------------------------------------- other head dims
+
+VALIDATION_CODES = (-1, -2, -3, -4, -5)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (256, 256), (128, 256), (64, 128), (256, 64)])
+def test_other_head_dims_pass_validation(gdn, dk, dv):
+    """Head dims 64, 128, 256 in any combination are accepted by gdn_prefill,
+    the decode entry points and the KDA ones (without a device the calls then
+    fail at the device check, not at validation)."""
+    assert gdn.raw_prefill(*prefill_args(Dk=dk, Dv=dv)) not in VALIDATION_CODES + (0,)
+    d = decode_args(Dk=dk, Dv=dv)
+    assert gdn.raw_decode_step(*d) not in VALIDATION_CODES + (0,)
+    assert gdn.raw_kda_prefill(*kda_args(Dk=dk, Dv=dv)) not in VALIDATION_CODES + (0,)
+    assert gdn.workspace_bytes(1, 4096, 16, 64, dk, dv) == 0 or (dk, dv) == (128, 128)
+
+
+def test_other_head_dims_reject_fused_options(gdn):
+    """The fused q/k norm, q scale and bf16 o exist on the 128 x 128 kernels only."""
+    import ctypes as ct
+    opts = gdn.Options(ct.sizeof(gdn.Options), 1, 1.0, 0)
+    a = prefill_args(Dk=64, Dv=64)
+    assert gdn.raw_prefill_ex(*(a[:14] + [None, 0, ct.byref(opts)] + a[14:])) == -4
+    d = decode_tokens_args(Dk=256, Dv=256)
+    assert gdn.raw_decode_ex(*(d[:12] + [ct.byref(opts)] + d[12:])) == -4
+
+
+def test_other_head_dims_size_the_overlap_checks(gdn):
+    """Byte extents follow Dk and Dv: with Dv = 256, an o that starts 32 KiB
+    before S_T (64 token-heads x 1 KiB) overlaps it; with Dv = 64 it does not."""
+    o = P + 0x50000000 - 0x8000
+    assert gdn.raw_prefill(*prefill_args(o=o, Dk=64, Dv=256)) == -5
+    assert gdn.raw_prefill(*prefill_args(o=o, Dk=64, Dv=64)) not in VALIDATION_CODES

@@ -1,0 +1,103 @@
+"""GPU parity at head dims other than 128 x 128 (64, 128, 256 in any
+combination, Dk != Dv included), through the same C entry points, against the
+fp64 oracles (which take any Dk, Dv).  These shapes run the row-parallel fp32
+kernel; the contract and the 1e-4 design margin are those of the other tests.
+"""
+from __future__ import annotations
+
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_linear_20_b200 import inputs
+from tests.test_gpu_parity import DEV, assert_parity, to_dev
+
+pytestmark = pytest.mark.gpu
+
+DIMS = [(64, 64), (256, 256), (128, 256), (256, 128), (64, 128), (128, 64), (64, 256)]
+
+
+def _gdn():
+    from gated_deltanet_linear_20_b200 import gdn
+    return gdn
+
+
+@pytest.mark.parametrize("dk,dv", DIMS, ids=lambda x: str(x))
+@pytest.mark.parametrize("BH", [(1, 3), (4, 16)], ids=["16rows", "32rows"])
+def test_prefill_other_head_dims(dk, dv, BH):
+    """Scalar gate through gdn.prefill (gdn_prefill_ws): T = 77 is not a
+    multiple of any staging chunk; S0 is carried in."""
+    B, H = BH
+    T = 77 if B == 1 else 33
+    d = inputs.prefill_inputs(B, T, H, dk, dv, seed=dk + dv + B, s0_std=0.05)
+    dd = to_dev(d)
+    o, S_T = _gdn().prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"])
+    torch.cuda.synchronize()
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o {dk}x{dv}")
+    assert_parity(S_T.cpu().numpy(), rS, f"S_T {dk}x{dv}")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (256, 256), (128, 256)], ids=lambda x: str(x))
+def test_long_prefill_other_head_dims(dk, dv):
+    d = inputs.prefill_inputs(1, 1024, 2, dk, dv, seed=3, g_mean=2.0, s0_std=0.02)
+    dd = to_dev(d)
+    o, S_T = _gdn().prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"], chunk=16,
+                            segmented=False)
+    torch.cuda.synchronize()
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o {dk}x{dv} T1024")
+    assert_parity(S_T.cpu().numpy(), rS, f"S_T {dk}x{dv} T1024")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (256, 256), (128, 256), (256, 64)], ids=lambda x: str(x))
+def test_decode_other_head_dims(dk, dv):
+    """Five single-token steps (the direct path) and a 3-token burst (the
+    staged path), the state in place, against the oracle over all 8 tokens."""
+    d = inputs.prefill_inputs(16, 8, 4, dk, dv, seed=dk * 3 + dv, s0_std=0.05)
+    dd = to_dev(d)
+    gdn = _gdn()
+    S = dd["S0"].clone()
+    step = lambda sl: [dd[key][:, sl].contiguous() for key in ("q", "k", "v", "g", "beta")]
+    outs = [gdn.decode_step(*step(t), S) for t in range(5)]
+    o3 = gdn.decode_tokens(*step(slice(5, 8)), S)
+    torch.cuda.synchronize()
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    o = torch.cat([torch.stack(outs, 1), o3], 1).cpu().numpy()
+    assert_parity(o, ro, f"o decode {dk}x{dv}")
+    assert_parity(S.cpu().numpy(), rS, f"S decode {dk}x{dv}")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (256, 256), (128, 64), (64, 256)], ids=lambda x: str(x))
+def test_kda_other_head_dims(dk, dv):
+    d = inputs.kda_inputs(2, 50, 3, dk, dv, seed=dk + 2 * dv, s0_std=0.05)
+    dd = to_dev(d)
+    gdn = _gdn()
+    o, S_T = gdn.kda_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"])
+    S = dd["S0"].clone()
+    o1 = gdn.kda_decode(*[dd[key][:, 0].contiguous() for key in ("q", "k", "v", "g", "beta")], S)
+    torch.cuda.synchronize()
+    ro, rS = oracle.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o kda {dk}x{dv}")
+    assert_parity(S_T.cpu().numpy(), rS, f"S_T kda {dk}x{dv}")
+    assert_parity(o1.cpu().numpy(), ro[:, 0], f"o kda decode {dk}x{dv}")
+
+
+def test_other_head_dims_in_place_and_deterministic():
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(2, 40, 3, 256, 64, seed=21, s0_std=0.05))
+    o1, S1 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    o2, S2 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    S_in = d["S0"].clone()
+    o3, S3 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], S_in, S_T=S_in)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    assert torch.equal(o3, o1) and torch.equal(S3, S1) and S3.data_ptr() == S_in.data_ptr()
+
+
+def test_other_head_dims_reject_fused_options_on_gpu():
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(1, 16, 2, 64, 64, seed=22))
+    with pytest.raises(gdn.GDNError) as e:
+        gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], qk_l2norm=True)
+    assert e.value.code == gdn.GDN_ERR_UNSUPPORTED

@@ -575,7 +575,7 @@ def test_invariants_on_gpu():
 
 def test_rejects_unsupported_head_dim_on_gpu():
     gdn = _gdn()
-    q = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16, device=DEV)
+    q = torch.zeros(1, 8, 1, 96, dtype=torch.bfloat16, device=DEV)
     g = torch.zeros(1, 8, 1, device=DEV)
     with pytest.raises(gdn.GDNError) as e:
         gdn.prefill(q, q, q, g, g)
