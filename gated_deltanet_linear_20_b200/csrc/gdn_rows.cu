@@ -18,10 +18,13 @@
 // fp32 registers, in the order of the recurrence: one kernel for prefill
 // (S0 -> S_T) and decode (S in place).
 //
-// Layout of a CTA: 4 warps; a warp holds RG groups of 4 rows; the 8 lanes of a
-// row hold the float4 column blocks j, j+8, j+16, .. (j = lane % 8, Dk/32
-// blocks), so the lanes of a row touch 128 contiguous bytes per access, in
-// global and in shared memory alike, and a dot product reduces over 8 lanes.
+// Layout of a CTA: 4 warps; LPR (8 or 16) lanes share a row, so a warp holds
+// 32/LPR rows per group and RG groups; the lanes of a row hold the float4
+// column blocks j, j+LPR, j+2 LPR, .. (j = lane % LPR, Dk/(4 LPR) blocks), so
+// they touch 128 or 256 contiguous bytes per access, in global and in shared
+// memory alike, and a dot product reduces over LPR lanes (LPR = 8 here: a
+// row's dot products take 3 shuffle steps).  Many chains take two row groups
+// per warp (fewer instructions per row), few take one (more SMs busy).
 // Tokens are staged NT at a time with cp.async into a double buffer (k, q, g,
 // this CTA's v rows, beta); one cooperative pass per chunk turns them into
 // fp32 k, q, alpha = exp(g) and k . q in shared memory, so each exp is taken
@@ -82,12 +85,13 @@ __device__ __forceinline__ float tree_sum(const float (&v)[N]) {
   }
 }
 
-template <int DK, bool VG, int RG>
+template <int DK, bool VG, int LPR, int RG>
 struct Shape {
-  static constexpr int MB = DK / 32;                  // float4 column blocks per lane
+  static constexpr int MB = DK / (4 * LPR);           // float4 column blocks per lane
+  static constexpr int RSTEP = 32 / LPR;              // rows per group in a warp
   static constexpr int NT = (VG ? 1536 : 2048) / DK;  // tokens per staged chunk
-  static constexpr int ROWS_PER_WARP = 4 * RG;
-  static constexpr int ROWS_PER_CTA = WARPS * ROWS_PER_WARP;  // 16 or 32
+  static constexpr int ROWS_PER_WARP = RSTEP * RG;
+  static constexpr int ROWS_PER_CTA = WARPS * ROWS_PER_WARP;  // 8, 16 or 32
   // staging buffer (cp.async target), bytes
   static constexpr int R_K = 0;
   static constexpr int R_Q = R_K + NT * DK * 2;
@@ -101,13 +105,12 @@ struct Shape {
   static constexpr int C_A = C_Q + NT * DK * 4;
   static constexpr int C_KQ = C_A + round16(VG ? NT * DK * 4 : NT * 4);
   static constexpr int SMEM = C_KQ + NT * 4;
-  static_assert(DK % 32 == 0 && (NT * DK * 2) % 16 == 0, "16-byte staging pieces");
+  static_assert(MB >= 1 && (NT * DK * 2) % 16 == 0, "16-byte staging pieces");
 };
 
-template <int DK, bool VG, int RG>
+template <typename S, int DK, bool VG>
 __device__ __forceinline__ void stage_chunk(const RowArgs& a, uint8_t* buf, int b, int h, int t0,
                                             int n, int vrow0) {
-  using S = Shape<DK, VG, RG>;
   const int tid = threadIdx.x;
   const uint32_t base = smem_addr(buf);
   auto tok = [&](int j) { return (size_t(b) * a.T + t0 + j) * a.H + h; };  // [B][T][H] index
@@ -127,7 +130,7 @@ __device__ __forceinline__ void stage_chunk(const RowArgs& a, uint8_t* buf, int 
   } else {
     for (int p = tid; p < n; p += THREADS) cp4(base + S::R_G + p * 4, a.g + tok(p));
   }
-  constexpr int VP = S::ROWS_PER_CTA / 8;  // this CTA's v rows: 2 or 4 pieces per token
+  constexpr int VP = S::ROWS_PER_CTA / 8;  // this CTA's v rows: 1, 2 or 4 pieces per token
   for (int p = tid; p < n * VP; p += THREADS) {
     const int j = p / VP, c = p % VP;
     cp16(base + S::R_V + j * S::ROWS_PER_CTA * 2 + c * 16, a.v + tok(j) * a.Dv + vrow0 + c * 8);
@@ -139,12 +142,11 @@ __device__ __forceinline__ void stage_chunk(const RowArgs& a, uint8_t* buf, int 
 // One token on this lane's rows.  kk, qq: k and q blocks; aa: the decay
 // blocks (per-channel gate) or aa[0].x the decay (scalar gate); kq: k . q, or
 // a lane's partial of it when KQ_PARTIAL (reduced here with sk and sq).
-template <int DK, bool VG, int RG, bool KQ_PARTIAL>
-__device__ __forceinline__ void apply_token(float4 (&s)[RG][DK / 32], const float4 (&kk)[DK / 32],
-                                            const float4 (&qq)[DK / 32],
-                                            const float4 (&aa)[VG ? DK / 32 : 1], float kq,
-                                            float beta, const float (&v)[RG], float (&o)[RG]) {
-  constexpr int MB = DK / 32;
+template <int MB, bool VG, int LPR, int RG, bool KQ_PARTIAL>
+__device__ __forceinline__ void apply_token(float4 (&s)[RG][MB], const float4 (&kk)[MB],
+                                            const float4 (&qq)[MB], const float4 (&aa)[VG ? MB : 1],
+                                            float kq, float beta, const float (&v)[RG],
+                                            float (&o)[RG]) {
   float sk[RG], sq[RG];
 #pragma unroll
   for (int i = 0; i < RG; ++i) {
@@ -159,7 +161,7 @@ __device__ __forceinline__ void apply_token(float4 (&s)[RG][DK / 32], const floa
     sq[i] = tree_sum(pq);
   }
 #pragma unroll
-  for (int off = 1; off < 8; off <<= 1) {
+  for (int off = 1; off < LPR; off <<= 1) {
 #pragma unroll
     for (int i = 0; i < RG; ++i) {
       sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], off);
@@ -177,20 +179,20 @@ __device__ __forceinline__ void apply_token(float4 (&s)[RG][DK / 32], const floa
 }
 
 // DIRECT: a single token per chain (decode), read straight from global memory.
-template <int DK, bool VG, int RG, bool DIRECT>
+template <int DK, bool VG, int LPR, int RG, bool DIRECT>
 __global__ void __launch_bounds__(THREADS) rows_kernel(const RowArgs a) {
-  using S = Shape<DK, VG, RG>;
-  constexpr int MB = S::MB;
+  using S = Shape<DK, VG, LPR, RG>;
+  constexpr int MB = S::MB, RS = S::RSTEP;
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ctas_per_head = a.Dv / S::ROWS_PER_CTA;
   const int head = blockIdx.x / ctas_per_head;  // b * H + h
   const int b = head / a.H, h = head - b * a.H;
   const int vrow0 = (blockIdx.x % ctas_per_head) * S::ROWS_PER_CTA;
-  const int j8 = lane & 7, sub = lane >> 3;
+  const int j8 = lane % LPR, sub = lane / LPR;
   const int wrow = warp * S::ROWS_PER_WARP + sub;  // this lane's first row within the CTA
 
-  // rows vrow0 + wrow + 4 i, column blocks j8 + 8 m
+  // rows vrow0 + wrow + RS i, column blocks j8 + LPR m
   float4 s[RG][MB];
   const size_t srow = (size_t(head) * a.Dv + vrow0 + wrow) * DK;
   if (a.S_in) {
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(THREADS) rows_kernel(const RowArgs a) {
 #pragma unroll
     for (int i = 0; i < RG; ++i)
 #pragma unroll
-      for (int m = 0; m < MB; ++m) s[i][m] = __ldcs(src + i * DK + j8 + 8 * m);  // +4 rows
+      for (int m = 0; m < MB; ++m) s[i][m] = __ldcs(src + i * RS * DK / 4 + j8 + LPR * m);
   } else {
 #pragma unroll
     for (int i = 0; i < RG; ++i)
@@ -214,27 +216,27 @@ __global__ void __launch_bounds__(THREADS) rows_kernel(const RowArgs a) {
       float kq = 0.f;
 #pragma unroll
       for (int m = 0; m < MB; ++m) {
-        kk[m] = bf16x4(*reinterpret_cast<const uint2*>(a.k + tok * DK + 4 * (j8 + 8 * m)));
-        qq[m] = bf16x4(*reinterpret_cast<const uint2*>(a.q + tok * DK + 4 * (j8 + 8 * m)));
+        kk[m] = bf16x4(*reinterpret_cast<const uint2*>(a.k + tok * DK + 4 * (j8 + LPR * m)));
+        qq[m] = bf16x4(*reinterpret_cast<const uint2*>(a.q + tok * DK + 4 * (j8 + LPR * m)));
         kq += dot44(kk[m], qq[m]);
         if constexpr (VG) {
-          const float4 gv = *reinterpret_cast<const float4*>(a.g + tok * DK + 4 * (j8 + 8 * m));
+          const float4 gv = *reinterpret_cast<const float4*>(a.g + tok * DK + 4 * (j8 + LPR * m));
           aa[m] = make_float4(expf(gv.x), expf(gv.y), expf(gv.z), expf(gv.w));
         }
       }
       if constexpr (!VG) aa[0].x = expf(a.g[tok]);
       float v[RG], o[RG];
 #pragma unroll
-      for (int i = 0; i < RG; ++i) v[i] = __bfloat162float(a.v[tok * a.Dv + vrow0 + wrow + 4 * i]);
-      apply_token<DK, VG, RG, true>(s, kk, qq, aa, kq, a.beta[tok], v, o);
+      for (int i = 0; i < RG; ++i) v[i] = __bfloat162float(a.v[tok * a.Dv + vrow0 + wrow + RS * i]);
+      apply_token<MB, VG, LPR, RG, true>(s, kk, qq, aa, kq, a.beta[tok], v, o);
       if (j8 == 0) {
 #pragma unroll
-        for (int i = 0; i < RG; ++i) a.o[tok * a.Dv + vrow0 + wrow + 4 * i] = o[i];
+        for (int i = 0; i < RG; ++i) a.o[tok * a.Dv + vrow0 + wrow + RS * i] = o[i];
       }
     }
   } else {
     const int nch = (a.T + S::NT - 1) / S::NT;
-    if (nch > 0) stage_chunk<DK, VG, RG>(a, smem, b, h, 0, min(S::NT, a.T), vrow0);
+    if (nch > 0) stage_chunk<S, DK, VG>(a, smem, b, h, 0, min(S::NT, a.T), vrow0);
     const float4* ck = reinterpret_cast<const float4*>(smem + S::C_K);
     const float4* cq = reinterpret_cast<const float4*>(smem + S::C_Q);
     const float* caf = reinterpret_cast<const float*>(smem + S::C_A);
@@ -244,41 +246,59 @@ __global__ void __launch_bounds__(THREADS) rows_kernel(const RowArgs a) {
       const int t0 = c * S::NT, n = min(S::NT, a.T - t0);
       uint8_t* raw = smem + (c & 1) * S::R_BYTES;
       if (c + 1 < nch) {
-        stage_chunk<DK, VG, RG>(a, smem + ((c + 1) & 1) * S::R_BYTES, b, h, t0 + S::NT,
-                                min(S::NT, a.T - t0 - S::NT), vrow0);
+        stage_chunk<S, DK, VG>(a, smem + ((c + 1) & 1) * S::R_BYTES, b, h, t0 + S::NT,
+                               min(S::NT, a.T - t0 - S::NT), vrow0);
         cp_wait<1>();
       } else {
         cp_wait<0>();
       }
       __syncthreads();
-      // convert: warp w takes tokens w, w+4, ..; lane l columns CPL l .. CPL l + CPL - 1
+      // convert: warp w takes tokens w, w+4, .. (all at once, so that their
+      // loads, exps and k . q reductions overlap); lane l columns CPL l ..
+      // (Dk = 256 takes one token at a time: its wider rows would spill)
       constexpr int CPL = DK / 32, PAIRS = CPL / 2;
-      for (int j = warp; j < n; j += WARPS) {
-        const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(raw + S::R_K + j * DK * 2);
-        const __nv_bfloat162* qr = reinterpret_cast<const __nv_bfloat162*>(raw + S::R_Q + j * DK * 2);
-        float2* kc = reinterpret_cast<float2*>(smem + S::C_K) + j * DK / 2;
-        float2* qc = reinterpret_cast<float2*>(smem + S::C_Q) + j * DK / 2;
-        float kq = 0.f;
+      constexpr int JPW = DK == 256 ? 1 : (S::NT + WARPS - 1) / WARPS;
+      for (int j0 = warp; j0 < n; j0 += WARPS * JPW) {
+        float kqp[JPW];
 #pragma unroll
-        for (int e = 0; e < PAIRS; ++e) {
-          const float2 kf = __bfloat1622float2(kr[lane * PAIRS + e]);
-          const float2 qf = __bfloat1622float2(qr[lane * PAIRS + e]);
-          kc[lane * PAIRS + e] = kf;
-          qc[lane * PAIRS + e] = qf;
-          kq = fmaf(kf.x, qf.x, fmaf(kf.y, qf.y, kq));
-          if constexpr (VG) {
-            const float2 gv = reinterpret_cast<const float2*>(raw + S::R_G + j * DK * 4)[lane * PAIRS + e];
-            reinterpret_cast<float2*>(smem + S::C_A)[j * DK / 2 + lane * PAIRS + e] =
-                make_float2(expf(gv.x), expf(gv.y));
+        for (int u = 0; u < JPW; ++u) {
+          const int j = j0 + WARPS * u;
+          kqp[u] = 0.f;
+          if (j < n) {
+            const __nv_bfloat162* kr = reinterpret_cast<const __nv_bfloat162*>(raw + S::R_K + j * DK * 2);
+            const __nv_bfloat162* qr = reinterpret_cast<const __nv_bfloat162*>(raw + S::R_Q + j * DK * 2);
+            float2* kc = reinterpret_cast<float2*>(smem + S::C_K) + j * DK / 2;
+            float2* qc = reinterpret_cast<float2*>(smem + S::C_Q) + j * DK / 2;
+#pragma unroll
+            for (int e = 0; e < PAIRS; ++e) {
+              const float2 kf = __bfloat1622float2(kr[lane * PAIRS + e]);
+              const float2 qf = __bfloat1622float2(qr[lane * PAIRS + e]);
+              kc[lane * PAIRS + e] = kf;
+              qc[lane * PAIRS + e] = qf;
+              kqp[u] = fmaf(kf.x, qf.x, fmaf(kf.y, qf.y, kqp[u]));
+              if constexpr (VG) {
+                const float2 gv = reinterpret_cast<const float2*>(raw + S::R_G + j * DK * 4)[lane * PAIRS + e];
+                reinterpret_cast<float2*>(smem + S::C_A)[j * DK / 2 + lane * PAIRS + e] =
+                    make_float2(expf(gv.x), expf(gv.y));
+              }
+            }
           }
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+          for (int u = 0; u < JPW; ++u) kqp[u] += __shfl_xor_sync(0xffffffffu, kqp[u], off);
         if (lane == 0) {
-          reinterpret_cast<float*>(smem + S::C_KQ)[j] = kq;
-          if constexpr (!VG)
-            reinterpret_cast<float*>(smem + S::C_A)[j] =
-                expf(reinterpret_cast<const float*>(raw + S::R_G)[j]);
+#pragma unroll
+          for (int u = 0; u < JPW; ++u) {
+            const int j = j0 + WARPS * u;
+            if (j < n) {
+              reinterpret_cast<float*>(smem + S::C_KQ)[j] = kqp[u];
+              if constexpr (!VG)
+                reinterpret_cast<float*>(smem + S::C_A)[j] =
+                    expf(reinterpret_cast<const float*>(raw + S::R_G)[j]);
+            }
+          }
         }
       }
       __syncthreads();
@@ -290,19 +310,19 @@ __global__ void __launch_bounds__(THREADS) rows_kernel(const RowArgs a) {
         float4 kk[MB], qq[MB], aa[VG ? MB : 1];
 #pragma unroll
         for (int m = 0; m < MB; ++m) {
-          kk[m] = ck[j * DK / 4 + j8 + 8 * m];
-          qq[m] = cq[j * DK / 4 + j8 + 8 * m];
-          if constexpr (VG) aa[m] = reinterpret_cast<const float4*>(caf)[j * DK / 4 + j8 + 8 * m];
+          kk[m] = ck[j * DK / 4 + j8 + LPR * m];
+          qq[m] = cq[j * DK / 4 + j8 + LPR * m];
+          if constexpr (VG) aa[m] = reinterpret_cast<const float4*>(caf)[j * DK / 4 + j8 + LPR * m];
         }
         if constexpr (!VG) aa[0].x = caf[j];
         float v[RG], o[RG];
 #pragma unroll
-        for (int i = 0; i < RG; ++i) v[i] = __bfloat162float(rv[j * S::ROWS_PER_CTA + wrow + 4 * i]);
-        apply_token<DK, VG, RG, false>(s, kk, qq, aa, ckq[j], rb[j], v, o);
+        for (int i = 0; i < RG; ++i) v[i] = __bfloat162float(rv[j * S::ROWS_PER_CTA + wrow + RS * i]);
+        apply_token<MB, VG, LPR, RG, false>(s, kk, qq, aa, ckq[j], rb[j], v, o);
         if (j8 == 0) {
           const size_t orow = ((size_t(b) * a.T + t0 + j) * a.H + h) * a.Dv + vrow0 + wrow;
 #pragma unroll
-          for (int i = 0; i < RG; ++i) a.o[orow + 4 * i] = o[i];
+          for (int i = 0; i < RG; ++i) a.o[orow + RS * i] = o[i];
         }
       }
       __syncthreads();  // the converted chunk and this staging buffer are reused
@@ -313,38 +333,39 @@ __global__ void __launch_bounds__(THREADS) rows_kernel(const RowArgs a) {
 #pragma unroll
   for (int i = 0; i < RG; ++i)
 #pragma unroll
-    for (int m = 0; m < MB; ++m) __stcs(dst + i * DK + j8 + 8 * m, s[i][m]);
+    for (int m = 0; m < MB; ++m) __stcs(dst + i * RS * DK / 4 + j8 + LPR * m, s[i][m]);
 }
 
-template <int DK, bool VG, int RG, bool DIRECT>
+template <int DK, bool VG, int LPR, int RG, bool DIRECT>
 bool launch_one(const RowArgs& a, long long heads, cudaStream_t stream) {
-  using S = Shape<DK, VG, RG>;
+  using S = Shape<DK, VG, LPR, RG>;
   const int smem = DIRECT ? 0 : S::SMEM;
-  const int slot = 16 + (DK == 64 ? 0 : DK == 128 ? 8 : 16) + (VG ? 4 : 0) + (RG - 1) * 2 + DIRECT;
-  auto kern = &rows_kernel<DK, VG, RG, DIRECT>;
-  if (smem > 48 * 1024 && !ensure_smem_attr(reinterpret_cast<const void*>(kern), slot, smem))
-    return false;
-  kern<<<unsigned(heads * (a.Dv / S::ROWS_PER_CTA)), THREADS, smem, stream>>>(a);
+  static_assert(S::SMEM <= 48 * 1024, "every shape stages within the default 48 KB");
+  rows_kernel<DK, VG, LPR, RG, DIRECT>
+      <<<unsigned(heads * (a.Dv / S::ROWS_PER_CTA)), THREADS, smem, stream>>>(a);
   return cudaGetLastError() == cudaSuccess;
 }
 
+template <int DK, bool VG, int LPR, int RG>
+bool launch_shape(const RowArgs& a, long long heads, cudaStream_t stream) {
+  return a.T == 1 ? launch_one<DK, VG, LPR, RG, true>(a, heads, stream)
+                  : launch_one<DK, VG, LPR, RG, false>(a, heads, stream);
+}
+
 template <int DK, bool VG>
-bool launch_dk(const RowArgs& a, long long heads, bool rg1, cudaStream_t stream) {
-  const bool direct = a.T == 1;
-  if (rg1)
-    return direct ? launch_one<DK, VG, 1, true>(a, heads, stream)
-                  : launch_one<DK, VG, 1, false>(a, heads, stream);
-  return direct ? launch_one<DK, VG, 2, true>(a, heads, stream)
-                : launch_one<DK, VG, 2, false>(a, heads, stream);
+bool launch_dk(const RowArgs& a, long long heads, int rows, cudaStream_t stream) {
+  if (rows == 16) return launch_shape<DK, VG, 8, 1>(a, heads, stream);
+  return launch_shape<DK, VG, 8, 2>(a, heads, stream);
 }
 
 }  // namespace
 
 int rows_per_cta(long long heads, int Dv, int num_sms) {
-  // 16 rows per CTA while every CTA still gets an SM of its own (the chains
-  // are few: spread them); 32 rows per CTA otherwise, which halves the staging
-  // and conversion work per row
-  return heads * (Dv / 16) <= num_sms ? 16 : 32;
+  // 32 rows per CTA (two row groups per warp: the fewest instructions per
+  // row) when that still gives every SM two CTAs; else 16 rows, which spreads
+  // few chains over more SMs.  (16 lanes a row, for twice the warps, measured
+  // no faster on few chains: each warp is bound by its own per-token latency.)
+  return heads * (Dv / 32) >= 2LL * num_sms ? 32 : 16;
 }
 
 bool rows_head_dims_ok(int Dk, int Dv) {
@@ -356,14 +377,14 @@ int launch_rows(const RowArgs& a, int Dk, bool vector_gate, int num_sms, cudaStr
   const long long heads = (long long)a.B * a.H;
   if (heads == 0) return 0;
   if (!rows_head_dims_ok(Dk, a.Dv)) return -1;
-  const bool rg1 = rows_per_cta(heads, a.Dv, num_sms) == 16;
+  const int rows = rows_per_cta(heads, a.Dv, num_sms);
   bool ok;
   if (Dk == 64)
-    ok = vector_gate ? launch_dk<64, true>(a, heads, rg1, stream) : launch_dk<64, false>(a, heads, rg1, stream);
+    ok = vector_gate ? launch_dk<64, true>(a, heads, rows, stream) : launch_dk<64, false>(a, heads, rows, stream);
   else if (Dk == 128)
-    ok = vector_gate ? launch_dk<128, true>(a, heads, rg1, stream) : launch_dk<128, false>(a, heads, rg1, stream);
+    ok = vector_gate ? launch_dk<128, true>(a, heads, rows, stream) : launch_dk<128, false>(a, heads, rows, stream);
   else
-    ok = vector_gate ? launch_dk<256, true>(a, heads, rg1, stream) : launch_dk<256, false>(a, heads, rg1, stream);
+    ok = vector_gate ? launch_dk<256, true>(a, heads, rows, stream) : launch_dk<256, false>(a, heads, rows, stream);
   return ok ? 0 : -1;
 }
 

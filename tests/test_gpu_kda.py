@@ -42,11 +42,12 @@ def test_kda_tiny_b1_h2_t64():
     _check(inputs.kda_inputs(1, 64, 2, seed=0), "B1 H2 T64")
 
 
-@pytest.mark.parametrize("T", [1, 15, 16, 17, 100])
-@pytest.mark.parametrize("BH", [(1, 4), (2, 16)], ids=["16rows", "32rows"])
-def test_kda_ragged_lengths_both_cta_shapes(T, BH):
-    """B*H = 4 runs 16 rows per CTA, B*H = 32 runs 32 rows per CTA (148 SMs);
-    T covers a single token, partial and exact 16-token chunks."""
+@pytest.mark.parametrize("T", [1, 11, 12, 13, 100])
+@pytest.mark.parametrize("BH", [(1, 4), (3, 16), (8, 16)], ids=["16rows_4heads", "16rows", "32rows"])
+def test_kda_ragged_lengths_all_cta_shapes(T, BH):
+    """On 148 SMs, B*H = 4 and 48 run 16 rows per CTA, 128 runs 32 rows per
+    CTA; T covers the direct single-token path, partial and exact 12-token
+    chunks (a warp converts up to 3 tokens of a chunk)."""
     B, H = BH
     _check(inputs.kda_inputs(B, T, H, seed=T, s0_std=0.05), f"B{B} H{H} T{T}")
 
