@@ -597,7 +597,7 @@ def cpu_baseline(w, budget_s=10.0):
             oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
             passes += 1
             done = time.perf_counter() - t0
-            if done > budget_s / 2 or passes >= 50:
+            if done >= budget_s:  # about budget_s of host work
                 break
         tokens = w.B * w.T * passes
         sample = f"{passes} full pass(es) of {args_name(w)} ({chains} chains x {w.T} tokens)"
