@@ -5,22 +5,27 @@ The compute lives in ``libgdn_b200.so`` (hand-written CUDA, C ABI declared in
 torch tensors and the current CUDA stream into that ABI.  There is no CPU
 fallback: calling into the binding without the built library raises.
 
-    from gated_deltanet_linear_20_b200 import prefill, decode_step
+    from gated_deltanet_linear_20_b200 import prefill, decode_step, kda_prefill
     o, S_T = prefill(q, k, v, g, beta, S0=None, chunk=64)
     o = decode_step(q, k, v, g, beta, S)       # S updated in place
+    o, S_T = kda_prefill(q, k, v, g_vec, beta)  # per-channel gate: g_vec [B,T,H,Dk]
+
+Head dims 64, 128 and 256 (Dk != Dv allowed) are accepted; 128 x 128 runs the
+chunked tensor-core kernel, the others the row-parallel fp32 kernel.
 
 The binding is imported lazily so that ``inputs`` (the seeded input
 generator) can be used without loading the CUDA library.
 """
 from __future__ import annotations
 
-__all__ = ["prefill", "decode_step", "abi_version", "status_str", "query_status",
-           "GDNError"]
+__all__ = ["prefill", "decode_step", "decode_tokens", "prefill_varlen", "kda_prefill",
+           "kda_decode", "abi_version", "status_str", "query_status", "GDNError"]
 
 
 def __getattr__(name):
-    if name in ("prefill", "decode_step", "abi_version", "status_str", "query_status",
-                "GDNError", "prefill_host", "library_path"):
+    if name in ("prefill", "decode_step", "decode_tokens", "prefill_varlen", "kda_prefill",
+                "kda_decode", "abi_version", "status_str", "query_status", "GDNError",
+                "library_path"):
         import importlib
         return getattr(importlib.import_module(__name__ + ".gdn"), name)
     raise AttributeError(name)

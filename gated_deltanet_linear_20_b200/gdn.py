@@ -153,7 +153,9 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     ``segmented=False`` it calls gdn_prefill (one pass per chain).
     ``qk_l2norm`` / ``q_scale`` (gdn_options) normalise q and k per token and
     head and scale q inside the kernel (gdn_prefill_ex).  ``o_bf16`` makes o
-    bf16 (the fp32 value rounded to nearest even); it runs the single pass."""
+    bf16 (the fp32 value rounded to nearest even); it runs the single pass.
+    Dk, Dv may each be 64, 128 or 256: other than 128 x 128 the row-parallel
+    fp32 kernel runs (chunk, segments and the fused options do not apply)."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape

@@ -114,7 +114,11 @@ const char* gdn_status_str(int code);
  *   S_T  : final state, written (device; may equal S0)
  *   B, T, H : batch, tokens per sequence, heads; B*H == 0 or T == 0 are valid
  *             (T == 0 only writes S_T = S0, or zeros)
- *   Dk, Dv  : head dims; both must be 128
+ *   Dk, Dv  : head dims, each 64, 128 or 256.  128 x 128 runs the chunked
+ *             tensor-core kernel; every other pair runs the row-parallel fp32
+ *             kernel (token by token, exact in the recurrence's order; chunk,
+ *             workspace and schedule do not apply to it).  Other values:
+ *             GDN_ERR_UNSUPPORTED
  *   chunk   : 16 or 64 -- tokens per chunk of the chunked form; the result is
  *             the same recurrence either way (up to rounding)
  *   status  : optional device int; a bounded device wait that gives up stores
@@ -156,7 +160,8 @@ size_t gdn_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chun
  *   n_snaps    : slots in snaps (sum over all n of len_n / snap_every); a
  *                sequence whose slots would pass it gets none, and
  *                GDN_ERR_SHAPE goes to *status.
- * chunk, status, stream and the other rules as for gdn_prefill. */
+ * Dk, Dv must be 128 (packed sequences run on the chunked tensor-core kernel
+ * only).  chunk, status, stream and the other rules as for gdn_prefill. */
 int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
                        const float* beta, const float* S0, float* o, float* S_T,
                        const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
@@ -165,7 +170,8 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
 
 /* gdn_prefill_ws with options (gdn_options above; NULL = none); with a NULL
  * workspace it runs the single pass of gdn_prefill.  Invalid options (size
- * too small, q_scale NaN) return GDN_ERR_UNSUPPORTED. */
+ * too small, q_scale NaN) return GDN_ERR_UNSUPPORTED, and so do non-default
+ * options at head dims other than 128 x 128. */
 int gdn_prefill_ex(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, const float* S0, float* o, float* S_T, int B, int T, int H,
                    int Dk, int Dv, int chunk, void* workspace, size_t workspace_bytes,
@@ -229,7 +235,8 @@ int gdn_prefill_static_ws(const void* q, const void* k, const void* v, const flo
  *   q, k [B][H][Dk] bf16; v [B][H][Dv] bf16; g, beta [B][H] fp32 (device)
  *   S    [B][H][Dv][Dk] fp32, updated in place (device)
  *   o    [B][H][Dv] fp32, written (device)
- *   Dk, Dv must be 128; B*H == 0 is a no-op.
+ *   Dk, Dv each 64, 128 or 256 (other than 128 x 128: the row-parallel kernel);
+ *   B*H == 0 is a no-op.
  * status and stream as for gdn_prefill.  Returns GDN_OK or a negative code. */
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                     const float* beta, float* S, float* o, int B, int H, int Dk, int Dv,
@@ -245,13 +252,15 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
  *   q, k [B][T][H][Dk] bf16; v [B][T][H][Dv] bf16; g, beta [B][T][H] fp32 (device)
  *   S    [B][H][Dv][Dk] fp32, updated in place (device)
  *   o    [B][T][H][Dv] fp32, written (device)
- *   Dk, Dv must be 128; B*H == 0 or T == 0 is a no-op.
+ *   Dk, Dv each 64, 128 or 256 (other than 128 x 128: the row-parallel kernel);
+ *   B*H == 0 or T == 0 is a no-op.
  * status and stream as for gdn_prefill.  Returns GDN_OK or a negative code. */
 int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                       int* status, void* stream);
 
-/* gdn_decode_tokens with options (gdn_options; NULL = none). */
+/* gdn_decode_tokens with options (gdn_options; NULL = none).  Non-default
+ * options need Dk = Dv = 128 (else GDN_ERR_UNSUPPORTED). */
 int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
                   const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                   const gdn_options* opts, int* status, void* stream);
@@ -270,7 +279,8 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
  *   S0   [B][H][Dv][Dk] fp32 or NULL (zeros); S_T written, same layout; S_T
  *        may be S0 (in place) but may not partly overlap it (16-byte aligned)
  *   o    [B][T][H][Dv] fp32, written (device); may not overlap any other array
- *   Dk, Dv must be 128.  B*H == 0 is a no-op; T == 0 copies S0 (or zeros) to S_T.
+ *   Dk, Dv each 64, 128 or 256.  B*H == 0 is a no-op; T == 0 copies S0 (or
+ *   zeros) to S_T.
  * status is accepted for symmetry (no device-side waits; never written) and
  * stream is a cudaStream_t.  Returns GDN_OK or a negative code; nothing is
  * launched on an error. */
