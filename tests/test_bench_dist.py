@@ -66,3 +66,7 @@ def test_algorithmic_work_figures():
     assert bench.prefill_bytes(1, 1, 1, True) == 1288 + 2 * 65536
     assert bench.prefill_flops(1, 1, 1) == 6 * 128 * 128 + 10 * 64 * 128 == 180224
     assert bench.decode_state_bytes(64, 16) == 134217728
+    # per-channel gate: g is a vector of 128 fp32 per token-head
+    assert bench.KDA_TOKEN_HEAD_BYTES == 3 * 256 + 512 + 4 + 512
+    assert bench.kda_prefill_bytes(1, 512, 16, False) == 512 * 16 * 1796 + 16 * 65536
+    assert bench.KDA_OPS_PER_TOKEN_HEAD == 4 * 128 * 128
