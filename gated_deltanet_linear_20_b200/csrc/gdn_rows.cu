@@ -18,13 +18,13 @@
 // fp32 registers, in the order of the recurrence: one kernel for prefill
 // (S0 -> S_T) and decode (S in place).
 //
-// Layout of a CTA: 4 warps; LPR (8 or 16) lanes share a row, so a warp holds
-// 32/LPR rows per group and RG groups; the lanes of a row hold the float4
-// column blocks j, j+LPR, j+2 LPR, .. (j = lane % LPR, Dk/(4 LPR) blocks), so
-// they touch 128 or 256 contiguous bytes per access, in global and in shared
-// memory alike, and a dot product reduces over LPR lanes (LPR = 8 here: a
-// row's dot products take 3 shuffle steps).  Many chains take two row groups
-// per warp (fewer instructions per row), few take one (more SMs busy).
+// Layout of a CTA: 4 warps; LPR lanes share a row (the launches use LPR = 8:
+// a row's dot products take 3 shuffle steps), so a warp holds 32/LPR rows per
+// group and RG groups; the lanes of a row hold the float4 column blocks j,
+// j+LPR, j+2 LPR, .. (j = lane % LPR, Dk/(4 LPR) blocks), so they touch 128
+// contiguous bytes per access, in global and in shared memory alike.  Many
+// chains take two row groups per warp (fewer instructions per row), few take
+// one (more SMs busy).
 // Tokens are staged NT at a time with cp.async into a double buffer (k, q, g,
 // this CTA's v rows, beta); one cooperative pass per chunk turns them into
 // fp32 k, q, alpha = exp(g) and the token-only scalars below in shared memory,
