@@ -478,6 +478,10 @@ def raw_prefill_varlen(*args) -> int:
     return int(_lib.gdn_prefill_varlen(*args))
 
 
+def raw_prefill_static_ws(*args) -> int:
+    return int(_lib.gdn_prefill_static_ws(*args))
+
+
 def raw_prefill_ws(*args) -> int:
     return int(_lib.gdn_prefill_ws(*args))
 

@@ -350,6 +350,14 @@ def test_other_head_dims_pass_validation(gdn, dk, dv):
     assert gdn.raw_decode_step(*d) not in VALIDATION_CODES + (0,)
     assert gdn.raw_kda_prefill(*kda_args(Dk=dk, Dv=dv)) not in VALIDATION_CODES + (0,)
     assert gdn.workspace_bytes(1, 4096, 16, 64, dk, dv) == 0 or (dk, dv) == (128, 128)
+    a = prefill_args(Dk=dk, Dv=dv)
+    assert gdn.raw_prefill_ws(*(a[:14] + [None, 0] + a[14:])) not in VALIDATION_CODES + (0,)
+    assert gdn.raw_prefill_static_ws(*a) not in VALIDATION_CODES + (0, -9)  # no scratch needed
+    t = decode_tokens_args(Dk=dk, Dv=dv)
+    assert gdn.raw_decode_tokens(*t) not in VALIDATION_CODES + (0,)
+    kd = [P, P + 0x1000000, P + 0x2000000, P + 0x3000000, P + 0x3100000, P + 0x4000000,
+          P + 0x5000000, 4, 2, 2, dk, dv, None, None]
+    assert gdn.raw_kda_decode(*kd) not in VALIDATION_CODES + (0,)
 
 
 def test_other_head_dims_reject_fused_options(gdn):
