@@ -290,3 +290,17 @@ def test_every_planted_kda_mistake_fails_a_pin(name):
         kda = _load_kda_from(so)
         results = {p.__name__: bool(p(kda)) for p in PINS}
     assert not all(results.values()), f"mutant {name} passed every pin: {results}"
+
+
+def test_empty_shapes():
+    """T = 0 leaves the state (S_T = S0, or zeros); B = 0 or H = 0 returns empty
+    arrays; both oracles agree on it."""
+    q, k, v, g, beta, S0 = _case(B=2, T=0, H=3, Dk=8, Dv=5, seed=17)
+    for f, gg in ((oracle.kda_prefill, g), (oracle.prefill, g[..., 0])):
+        o, S_T = f(q, k, v, gg, beta, S0)
+        assert o.shape == (2, 0, 3, 5) and np.array_equal(S_T, S0.astype(np.float64))
+        o, S_T = f(q, k, v, gg, beta, None)
+        assert not S_T.any()
+    q, k, v, g, beta, S0 = _case(B=0, T=4, H=3, Dk=8, Dv=5, seed=18)
+    o, S_T = oracle.kda_prefill(q, k, v, g, beta, S0)
+    assert o.shape == (0, 4, 3, 5) and S_T.shape == (0, 3, 5, 8)
