@@ -4,18 +4,21 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--chunk 64|16] [--no-extras]
 
-A step is one gdn_prefill call over one batch of the workload (default
-prefill_b1_h16_t512: one 512-token sequence, 16 heads, head dim 128 -- the
-single-sequence, scalar-gate, 512-token setting of the ROCmFPX gated-delta-net
-prefill note, bittide.aicompass.dev article d2880479, opening post).  Inputs
-are synthetic, seeded, resident in HBM before timing.  L2 (126 MB) is flushed
-by writing a 256 MiB buffer before every timed step; each step is timed with
-CUDA events on the launching stream, and the sum over K steps is the timed
-total.  With N > 1 (torchrun) every rank runs its own independent batch (weak
-scaling, no collective on the data path) and the max over ranks is reported.
+A step is one gdn_prefill call over one batch of the workload.  The default
+workload is the large batched prefill prefill_b4_h32_t32768 (B=4 sequences x
+H=32 heads x T=32768 tokens, head dim 128, scalar gate, chunk 64): the largest
+configuration on one GPU.  The 512-token single-sequence call of the ROCmFPX
+gated-delta-net prefill note (bittide.aicompass.dev article d2880479, opening
+post), the 4096-token prefill with a carried state, the batched decode step and
+the extensions are reported under ``extras``.  Inputs are synthetic, seeded,
+resident in HBM before timing.  L2 (126 MB) is flushed by writing a 256 MiB
+buffer before every timed step; each step is timed with CUDA events on the
+launching stream, and the sum over K steps is the timed total.  With N > 1
+(torchrun) every rank runs its own independent batch (weak scaling, no
+collective on the data path) and the max over ranks is reported.
 
 Prints ONE JSON line (rank 0).  ``--impl reference`` times the fp64 CPU oracle
-on the same workload instead (rank 0 only).
+on a bounded sample of the same workload instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -246,6 +249,66 @@ def time_steps(fn, steps, warmup, flush, stream):
 
 
 # ------------------------------------------------------------------ our arm
+def e2e_pipelined(call_part, host, dev_in, outs_dev, outs_host, nparts, steps, warmup, stream):
+    """End-to-end steps through the public API with the copies overlapped.
+
+    The batch is split into `nparts` parts along B.  Per step and part: the
+    pinned host inputs of the part go to the device on a copy stream, the part
+    is computed on `stream`, and its outputs go back to pinned host memory on a
+    second copy stream, so that the host-to-device copy of part j+1, the
+    compute of part j and the device-to-host copy of part j-1 overlap (and the
+    same across steps).  A part's input buffers are rewritten only after the
+    previous step's compute of that part, and its outputs only after the
+    previous step's copy-out.  Returns the mean ms per step over `steps`
+    timed steps (the device time from the first copy to the last copy-out)."""
+    dev = stream.device
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    comp_done = [torch.cuda.Event() for _ in range(nparts)]
+    out_done = [torch.cuda.Event() for _ in range(nparts)]
+    for j in range(nparts):
+        comp_done[j].record(stream)
+        out_done[j].record(stream)
+
+    def part_slices(t, j):
+        n = t.shape[0] // nparts
+        return t[j * n:(j + 1) * n]
+
+    def one_step():
+        for j in range(nparts):
+            s_in.wait_event(comp_done[j])
+            with torch.cuda.stream(s_in):
+                for key, hv in host.items():
+                    if hv is not None:
+                        part_slices(dev_in[key], j).copy_(part_slices(hv, j), non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(s_in)
+            stream.wait_event(ready)
+            stream.wait_event(out_done[j])
+            call_part(j)
+            comp_done[j].record(stream)
+            s_out.wait_event(comp_done[j])
+            with torch.cuda.stream(s_out):
+                for dv, hv in zip(outs_dev, outs_host):
+                    part_slices(hv, j).copy_(part_slices(dv, j), non_blocking=True)
+            out_done[j].record(s_out)
+
+    for _ in range(warmup):
+        one_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for _ in range(steps):
+        one_step()
+    for j in range(nparts):
+        stream.wait_event(out_done[j])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
 def run_ours(args, world, rank, local):
     from gated_deltanet_linear_20_b200 import gdn
     dev = torch.device("cuda", local)
@@ -257,14 +320,15 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     flush = lambda: flush_buf.fill_(1.0)
-
     d = gin.workload_inputs(w, seed=1000 + rank, device=str(dev))
     B, T, H = w.B, w.T, w.H
     o = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
     S_T = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     # gdn_prefill_ws: chains too few to fill the GPU are cut into segments that
-    # run in parallel (first pass + segment fix: two launches per step)
-    nseg, seg_tiles, ws_bytes = gdn.schedule(B, T, H, torch.cuda.get_device_properties(dev).multi_processor_count)
+    # run in parallel (first pass + segment fix: two launches per step); enough
+    # chains run in one pass (one launch per step)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    nseg, seg_tiles, ws_bytes = gdn.schedule(B, T, H, sms)
     ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
     launches_per_step = 2 if nseg > 1 else 1
     call = lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
@@ -290,39 +354,56 @@ def run_ours(args, world, rank, local):
     traffic = committed_traffic(f"{args.workload}/chunk{args.chunk}", PREFILL_SOURCES)
     roofline = {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": traffic, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                "traffic": traffic,
+                "traffic_is_lower_bound": True,
+                "traffic_note": ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
+                                 "step's launches: lines still dirty in L2 when a launch ends "
+                                 "(at most the 126 MB L2) are written back later and are not "
+                                 "counted, so this is a lower bound on the step's DRAM bytes"),
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6.65 TB/s",
                 "algorithmic_bytes_per_step": nbytes,
                 "scope": ("whole step: first pass + segment fix" if launches_per_step == 2
                           else "the single prefill launch of the step"),
                 "tensor": {"achieved_tflops": round(flops / (launch_ms / 1e3) / 1e12, 2),
                            "peak_tflops": peaks["bf16_tflops"],
+                           "peak_source": ("MEASURED_PEAKS.json bf16_tflops (burst: the kernel "
+                                           "is timed alone)"),
                            "frac": round(flops / (launch_ms / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
-                           "flops_per_step": flops}}
+                           "flops_per_step": flops,
+                           "flops_per_token_head": "6 D^2 + 10 C D at C = 64"}}
 
-    # end to end through the public API: pinned host inputs -> device -> prefill -> host
+    # end to end through the public API: pinned host inputs -> device -> prefill -> host,
+    # the copies of one part overlapping the compute of another
     host = {k: (v.cpu().pin_memory() if v is not None else None) for k, v in d.items()}
+    del d
     o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     s_host = torch.empty(S_T.shape, dtype=S_T.dtype, pin_memory=True)
     dev_in = {k: (torch.empty_like(v, device=dev) if v is not None else None) for k, v in host.items()}
+    nparts = B if B > 1 else 1
+    pb = B // nparts
+    ws_part = torch.empty(max(gdn.workspace_bytes(pb, T, H, args.chunk), 1), dtype=torch.uint8,
+                          device=dev)
 
-    def e2e_step():
-        for k, v in host.items():
-            if v is not None:
-                dev_in[k].copy_(v, non_blocking=True)
-        gdn.prefill(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["g"], dev_in["beta"],
-                    dev_in["S0"], chunk=args.chunk, o=o, S_T=S_T, workspace=ws)
-        o_host.copy_(o, non_blocking=True)
-        s_host.copy_(S_T, non_blocking=True)
+    def call_part(j):
+        sl = slice(j * pb, (j + 1) * pb)
+        gdn.prefill(dev_in["q"][sl], dev_in["k"][sl], dev_in["v"][sl], dev_in["g"][sl],
+                    dev_in["beta"][sl], None if dev_in["S0"] is None else dev_in["S0"][sl],
+                    chunk=args.chunk, o=o[sl], S_T=S_T[sl], workspace=ws_part)
 
     barrier(world)
-    e2e_ms = time_steps(e2e_step, args.steps, args.warmup, flush, stream)
+    e2e_ms = e2e_pipelined(call_part, host, dev_in, (o, S_T), (o_host, s_host), nparts,
+                           args.steps, args.warmup, stream)
     barrier(world)
-    e2e_total = max_over_ranks(sum(e2e_ms), world)
+    e2e_total = max_over_ranks(e2e_ms * args.steps, world)
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     d2h = o_host.numel() * 4 + s_host.numel() * 4
     e2e = {"value": round(tokens_per_step * world * args.steps / (e2e_total / 1e3), 1),
-           "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": round(e2e_ms, 4),
+           "pipeline": (f"{nparts} part(s) along B per step: host-to-device copy, prefill "
+                        "and device-to-host copy of different parts overlap on three streams")}
+    del host, dev_in, o_host, s_host
 
     extras = None
     if not args.no_extras:
@@ -339,7 +420,8 @@ def run_ours(args, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded; q,k L2-normalised bf16, v bf16, g=logsigmoid, beta=sigmoid)",
             "config": {"workload": args.workload, "B": B, "T": T, "H": H, "Dk": D, "Dv": D,
-                       "chunk": args.chunk, "tokens_per_step_per_gpu": tokens_per_step,
+                       "chunk": args.chunk, "g": f"logsigmoid(N({w.g_mean},1))",
+                       "tokens_per_step_per_gpu": tokens_per_step,
                        "schedule": {"segments_per_chain": nseg, "tiles_per_segment": seg_tiles,
                                     "workspace_bytes": ws_bytes},
                        "l2": "flushed (256 MiB write) before every timed step",
@@ -357,36 +439,42 @@ def run_ours(args, world, rank, local):
 
 
 def run_extras(args, dev, stream, flush, peaks, rank):
-    """Other measured workloads reported beside the headline: chunk 16 on the
-    headline workload, the batched decode step, and the large prefill."""
+    """Other measured workloads reported beside the headline: the other prefill
+    workloads (both chunks; the segmented and the single-pass schedule), the
+    batched decode step, a decode burst, packed sequences, the per-channel gate
+    and other head dims."""
     from gated_deltanet_linear_20_b200 import gdn
     out = {}
     steps = max(3, min(args.steps, 10))
-    # chunk 16 on the headline workload
-    w = gin.WORKLOADS[args.workload]
-    d = gin.workload_inputs(w, seed=1000 + rank, device=str(dev))
-    other = 16 if args.chunk == 64 else 64
-    ws = torch.empty(max(gdn.workspace_bytes(w.B, w.T, w.H, other), 1), dtype=torch.uint8,
-                     device=dev)
-    oc = torch.empty((w.B, w.T, w.H, D), dtype=torch.float32, device=dev)
-    sc = torch.empty((w.B, w.H, D, D), dtype=torch.float32, device=dev)
-    ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
-                                        chunk=other, workspace=ws, o=oc, S_T=sc), steps, 3, flush,
-                    stream)
-    t = statistics.mean(ms)
-    out[f"{args.workload}/chunk{other}"] = {
-        "tokens_per_s": round(w.B * w.T / (t / 1e3), 1), "ms": round(t, 5),
-        "hbm_frac": round(prefill_bytes(w.B, w.T, w.H, d["S0"] is not None) / (t / 1e3) / 1e9
-                          / peaks["hbm_gbs"], 4)}
-    # the single-pass schedule (gdn_prefill) on the headline workload, both chunks
-    for c in (args.chunk, other):
-        ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"],
-                                            chunk=c, segmented=False, o=oc, S_T=sc), steps, 3,
-                        flush, stream)
-        t = statistics.mean(ms)
-        out[f"{args.workload}/chunk{c}/single_pass"] = {
-            "tokens_per_s": round(w.B * w.T / (t / 1e3), 1), "ms": round(t, 5)}
-    del d, ws, oc, sc
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    for name, w in gin.WORKLOADS.items():
+        if w.is_decode or name == args.workload or w.T < 512:
+            continue
+        d = gin.workload_inputs(w, seed=1000 + rank, device=str(dev))
+        oc = torch.empty((w.B, w.T, w.H, D), dtype=torch.float32, device=dev)
+        sc = torch.empty((w.B, w.H, D, D), dtype=torch.float32, device=dev)
+        nb = prefill_bytes(w.B, w.T, w.H, d["S0"] is not None)
+        fl = prefill_flops(w.B, w.T, w.H)
+        n = steps if w.B * w.T * w.H <= (1 << 20) else 3
+        for c in (64, 16):
+            ws = torch.empty(max(gdn.workspace_bytes(w.B, w.T, w.H, c), 1), dtype=torch.uint8,
+                             device=dev)
+            nseg = gdn.schedule(w.B, w.T, w.H, sms)[0]
+            variants = [("", True)] + ([("/single_pass", False)] if nseg > 1 else [])
+            for suffix, seg in variants:
+                ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                                    d["S0"], chunk=c, segmented=seg, workspace=ws,
+                                                    o=oc, S_T=sc), n, 3, flush, stream)
+                t = statistics.mean(ms)
+                out[f"{name}/chunk{c}{suffix}"] = {
+                    "tokens_per_s": round(w.B * w.T / (t / 1e3), 1), "ms": round(t, 5),
+                    "schedule": (f"{nseg} segments per chain, two launches" if seg and nseg > 1
+                                 else "single pass, one launch"),
+                    "hbm_frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                    "tensor_frac": round(fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
+            del ws
+        del d, oc, sc
+        torch.cuda.empty_cache()
     # decode: L2 flushed before every step (headline) and 256 back-to-back steps (L2-warm)
     wd = gin.WORKLOADS["decode_b64_h16"]
     dd = gin.workload_inputs(wd, seed=2000 + rank, device=str(dev))
@@ -454,24 +542,6 @@ def run_extras(args, dev, stream, flush, peaks, rank):
         "tokens_per_s": round(ntok / (t / 1e3), 1), "ms": round(t, 4),
         "hbm_frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
     del pk, cu
-    # large prefill (inputs 1.6 GB > L2)
-    wl = gin.WORKLOADS["prefill_b4_h32_t32768"]
-    dl = gin.workload_inputs(wl, seed=3000 + rank, device=str(dev))
-    ol = torch.empty((wl.B, wl.T, wl.H, D), dtype=torch.float32, device=dev)
-    sl = torch.empty((wl.B, wl.H, D, D), dtype=torch.float32, device=dev)
-    ms = time_steps(lambda: gdn.prefill(dl["q"], dl["k"], dl["v"], dl["g"], dl["beta"], None,
-                                        chunk=64, o=ol, S_T=sl), 3, 2, flush, stream)
-    t = statistics.mean(ms)
-    nb = prefill_bytes(wl.B, wl.T, wl.H, False)
-    fl = prefill_flops(wl.B, wl.T, wl.H)
-    out["prefill_b4_h32_t32768/chunk64"] = {
-        "tokens_per_s": round(wl.B * wl.T / (t / 1e3), 1), "ms": round(t, 4),
-        "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
-                     "traffic": committed_traffic("prefill_b4_h32_t32768/chunk64", PREFILL_SOURCES)},
-        "tensor_frac": round(fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
-    del dl, ol, sl
     torch.cuda.empty_cache()
     out.update(run_kda_extras(dev, stream, flush, peaks, rank, steps))
     out.update(run_head_dim_extras(dev, stream, flush, peaks, rank, steps))
@@ -579,42 +649,41 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
 
 
 # ------------------------------------------------------------------ the oracle (CPU)
+ORACLE_SAMPLE_MAX_T = 8192  # tokens per sampled chain (bounds host memory and time)
+
+
+def oracle_sample(w, cores, seed=1000):
+    """A bounded sample of workload `w` for the oracle: min(cores, B*H) chains
+    (one per host core), each the first min(T, 8192) tokens, drawn with the
+    workload's own recipe (same distributions, gate mean and S0).  The
+    oracle's cost per token-head does not depend on T, so tokens/s from the
+    sample stands for the whole workload."""
+    n = max(1, min(cores, w.B * w.H))
+    Ts = min(w.T, ORACLE_SAMPLE_MAX_T)
+    d = gin.prefill_inputs(1, Ts, n, w.Dk, w.Dv, seed=seed, g_mean=w.g_mean, s0_std=w.s0_std)
+    desc = (f"{n} chain(s) x {Ts} tokens of {w.name}'s recipe "
+            f"(the full batch is {w.B * w.H} chains x {w.T} tokens)")
+    return d, n, Ts, desc
+
+
 def cpu_baseline(w, budget_s=10.0):
     """The fp64 oracle as it stands, on the host cores, over a bounded sample of
-    the workload: whole batches while they fit the budget, else a subset of
-    chains.  Returns tokens/s (token-heads / H, so comparable to the GPU line)."""
+    the workload (about `budget_s` of host work).  Returns tokens/s: sampled
+    token-heads per second / H, so comparable to the GPU line."""
     import oracle
-    d = gin.workload_inputs(w, seed=1000)
-    chains = w.B * w.H
-    t0 = time.perf_counter()
-    oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=[0])
-    one_chain = time.perf_counter() - t0
     cores = oracle.num_threads()
-    per_pass = one_chain * chains / max(1, min(cores, chains))
-    if per_pass <= budget_s:
-        passes, done, t0 = 0, 0.0, time.perf_counter()
-        while True:
-            oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
-            passes += 1
-            done = time.perf_counter() - t0
-            if done >= budget_s:  # about budget_s of host work
-                break
-        tokens = w.B * w.T * passes
-        sample = f"{passes} full pass(es) of {args_name(w)} ({chains} chains x {w.T} tokens)"
-    else:
-        n = max(1, min(chains, cores))
-        ids = list(range(n))
-        t0 = time.perf_counter()
-        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=ids)
+    d, n, Ts, desc = oracle_sample(w, cores)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+        passes += 1
         done = time.perf_counter() - t0
-        tokens = w.T * n / w.H
-        sample = f"{n} of {chains} chains of {args_name(w)} ({w.T} tokens each)"
+        if done >= budget_s:
+            break
+    tokens = n * Ts * passes / w.H
     return {"value": round(tokens / done, 2), "unit": "tokens/s", "cores": cores,
-            "kind": "oracle", "sample": sample, "seconds": round(done, 3)}
-
-
-def args_name(w):
-    return w.name
+            "kind": "oracle", "sample": f"{passes} pass(es) over {desc}",
+            "seconds": round(done, 3)}
 
 
 def run_reference(args, world, rank):
@@ -622,26 +691,17 @@ def run_reference(args, world, rank):
         return
     w = gin.WORKLOADS[args.workload]
     import oracle
-    d = gin.workload_inputs(w, seed=1000)
-    chains = w.B * w.H
     cores = oracle.num_threads()
-    t0 = time.perf_counter()
-    oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=[0])
-    per_chain = time.perf_counter() - t0
-    # each step: as many chains as fit ~2 s of host time (the whole batch when it does)
-    n = chains if per_chain * chains / max(1, min(cores, chains)) <= 2.0 else \
-        max(1, min(chains, int(2.0 * cores / max(per_chain, 1e-6))))
-    ids = None if n == chains else list(range(n))
+    d, n, Ts, desc = oracle_sample(w, cores)
     for _ in range(args.warmup):
-        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=ids)
+        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], chains=ids)
+        oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
     total = time.perf_counter() - t0
-    tokens_per_step = w.T * n / w.H
+    tokens_per_step = n * Ts / w.H
     value = tokens_per_step * args.steps / total
-    sample = (f"full batch of {w.name} per step" if ids is None else
-              f"{n} of {chains} chains of {w.name} per step ({w.T} tokens each)")
+    sample = f"each step: {desc}"
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
@@ -709,7 +769,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=30)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill_b1_h16_t512",
+    ap.add_argument("--workload", default="prefill_b4_h32_t32768",
                     choices=[k for k, v in gin.WORKLOADS.items() if not v.is_decode])
     ap.add_argument("--chunk", type=int, default=64, choices=[16, 64])
     ap.add_argument("--no-extras", action="store_true")

@@ -1,7 +1,9 @@
 // C-ABI entry points of libgdn_b200.so (declared in include/gdn.h): argument
 // validation, TMA descriptor encoding on the host, launches on the caller's
-// stream.  No device memory is allocated here and no state is kept between
-// calls except the cached driver entry point of cuTensorMapEncodeTiled.
+// stream.  No device memory is allocated here.  Between calls the library
+// keeps only host-side caches: the driver entry point of
+// cuTensorMapEncodeTiled, per-device facts (compute capability, SM count) and
+// which kernels already had their shared-memory limit raised on a device.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -243,6 +245,11 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
                 overlaps(o, act_f32, S_T, state_bytes)))
     return GDN_ERR_ALIAS;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
+  // one chain may write its S_T while another still reads its inputs
+  if (T > 0 && (overlaps(S_T, state_bytes, q, act_bf16) || overlaps(S_T, state_bytes, k, act_bf16) ||
+                overlaps(S_T, state_bytes, v, act_bf16) || overlaps(S_T, state_bytes, g, gate_bytes) ||
+                overlaps(S_T, state_bytes, beta, gate_bytes)))
+    return GDN_ERR_ALIAS;
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
 
@@ -288,22 +295,15 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   return GDN_OK;
 }
 
-// Device address of the built-in scratch per device (looked up once, on the
-// first call on that device).
-void* g_static_ws_addr[kMaxDevices];
-std::mutex g_static_ws_mutex;
-
+// Device address of the built-in scratch on the current device.  Looked up
+// on every call (a cheap table lookup once the module is loaded), so that the
+// address stays right after a device reset or in another context of the same
+// device.  The first lookup on a device may load the module there, which is
+// why the first call on a device should come before any stream capture.
 int static_workspace(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return GDN_ERR_LAUNCH;
-  if (dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-  if (!g_static_ws_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) return GDN_ERR_LAUNCH;
-    g_static_ws_addr[dev] = p;
-  }
-  *out = g_static_ws_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_ws) != cudaSuccess || !p) return GDN_ERR_LAUNCH;
+  *out = p;
   return GDN_OK;
 }
 
@@ -334,7 +334,7 @@ const char* gdn_status_str(int code) {
     case GDN_ERR_NULL: return "a required pointer is NULL";
     case GDN_ERR_ALIGN: return "misaligned pointer (q/k/v/o/S need 16 bytes, g/beta 4 bytes)";
     case GDN_ERR_SHAPE: return "negative size or problem larger than 2^31-1 elements";
-    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims must be 128, chunk 16 or 64, device sm_100)";
+    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options and packed sequences at 128 x 128 only; chunk 16 or 64; device sm_100)";
     case GDN_ERR_ALIAS: return "output overlaps an input";
     case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
     case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
@@ -417,6 +417,10 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
     return GDN_ERR_ALIAS;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
   if (overlaps(S_T, state_bytes, cu_seqlens, cu_bytes)) return GDN_ERR_ALIAS;
+  if (total_T > 0 && (overlaps(S_T, state_bytes, q, act_bf16) || overlaps(S_T, state_bytes, k, act_bf16) ||
+                      overlaps(S_T, state_bytes, v, act_bf16) || overlaps(S_T, state_bytes, g, gate_bytes) ||
+                      overlaps(S_T, state_bytes, beta, gate_bytes)))
+    return GDN_ERR_ALIAS;
   if (snaps) {
     const size_t snap_bytes = size_t(n_snaps) * H * kHeadDim * kHeadDim * 4;
     if (!aligned(snaps, 16)) return GDN_ERR_ALIGN;

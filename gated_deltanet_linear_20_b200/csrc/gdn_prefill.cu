@@ -1062,11 +1062,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (p.snaps && p.cu_seqlens) {
       // first snapshot slot of this sequence: one per snap_every tokens of
       // every earlier sequence
+      // every earlier sequence; an invalid earlier entry (its own CTAs report
+      // it) leaves this sequence without snapshots rather than with a slot
+      // index computed from garbage
       const int n = chain / p.H;
       int base = 0;
-      for (int m = 0; m < n; ++m)
-        base += (__ldg(p.cu_seqlens + m + 1) - __ldg(p.cu_seqlens + m)) / p.snap_every;
-      if (base + (x.tend - x.tok0) / p.snap_every > p.n_snaps) {  // too few slots
+      bool offsets_ok = true;
+      for (int m = 0; m < n; ++m) {
+        const int s0 = __ldg(p.cu_seqlens + m), s1 = __ldg(p.cu_seqlens + m + 1);
+        if (s0 < 0 || s1 < s0 || s1 > p.T) {
+          offsets_ok = false;
+          break;
+        }
+        base += (s1 - s0) / p.snap_every;
+      }
+      if (!offsets_ok || base < 0 || base + (x.tend - x.tok0) / p.snap_every > p.n_snaps) {
         if (p.status) atomicExch(p.status, GDN_ERR_SHAPE);
       } else {
         *reinterpret_cast<float* volatile*>(sm + SM_MISC + M_SNAP_PTR) =

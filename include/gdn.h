@@ -28,19 +28,23 @@
  * normalise or scale them beforehand if their model does so.
  *
  * Ownership and execution.  All pointers are DEVICE pointers owned by the
- * caller.  The library allocates no device memory, keeps no state between
- * calls and is safe to call from several host threads.  Work is enqueued on
+ * caller.  The library allocates no device memory and is safe to call from
+ * several host threads; between calls it keeps only host-side caches (per
+ * device: compute capability, SM count, kernel attributes already set).  Work is enqueued on
  * `stream` (a cudaStream_t; NULL means the legacy default stream) and the call
  * returns before it completes.  S_T may be the same buffer as S0 (each chain
- * reads its S0 before writing its S_T); o must not overlap any input.
+ * reads its S0 before writing its S_T); neither o nor S_T may overlap q, k, v,
+ * g or beta, and o may not overlap the state.
  *
  * Errors.  A negative return value means nothing was launched:
  *     GDN_ERR_NULL         a required pointer is NULL
  *     GDN_ERR_ALIGN        q/k/v/o/S pointers must be 16-byte aligned, g/beta 4-byte
  *     GDN_ERR_SHAPE        a size is negative or the problem exceeds 2^31-1 elements
- *     GDN_ERR_UNSUPPORTED  Dk != 128, Dv != 128, chunk not in {16, 64}, or the
- *                          current device is not compute capability 10.0
- *     GDN_ERR_ALIAS        o overlaps an input or the state
+ *     GDN_ERR_UNSUPPORTED  a head dim not in {64, 128, 256}; fused options or
+ *                          packed sequences at head dims other than 128 x 128;
+ *                          chunk not in {16, 64}; or the current device is not
+ *                          compute capability 10.0
+ *     GDN_ERR_ALIAS        o or S_T overlaps an input, or o overlaps the state
  *     GDN_ERR_LAUNCH       the CUDA launch (or a CUDA runtime query) failed
  *     GDN_ERR_WORKSPACE    gdn_prefill_ws: workspace NULL, misaligned (256 B) or
  *                          smaller than gdn_prefill_workspace_bytes asked for
@@ -158,8 +162,9 @@ size_t gdn_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chun
  *                = sum over m < n of len_m / snap_every.
  *   snap_every : a positive multiple of 64 when snaps is given, else ignored
  *   n_snaps    : slots in snaps (sum over all n of len_n / snap_every); a
- *                sequence whose slots would pass it gets none, and
- *                GDN_ERR_SHAPE goes to *status.
+ *                sequence whose slots would pass it, or that follows a
+ *                sequence with invalid offsets, gets none, and GDN_ERR_SHAPE
+ *                goes to *status.
  * Dk, Dv must be 128 (packed sequences run on the chunked tensor-core kernel
  * only).  chunk, status, stream and the other rules as for gdn_prefill. */
 int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
@@ -218,8 +223,9 @@ int gdn_prefill_ws(const void* q, const void* k, const void* v, const float* g,
  *   rejected with GDN_ERR_STATIC_WORKSPACE_LIMIT before anything is launched.
  *   The scratch needs no zeroing: every byte read is written earlier in the
  *   same call.
- *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress) and caches it; make that first call before any
+ *   Every call looks up the array's device address on the current device
+ *   (cudaGetSymbolAddress; cheap once the library's module is loaded there).
+ *   The first call on a device may load that module, so make it before any
  *   stream capture.
  *   All calls on a device share the one array: calls whose executions
  *   overlap (other streams, other host threads) race on it and must be

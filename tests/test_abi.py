@@ -75,6 +75,8 @@ def prefill_args(**over):
     (dict(S0=P + 0x60000008), -2),
     (dict(o=P + 0x10000000 + 0x100), -5),                # o overlaps k
     (dict(S0=P + 0x50000000 + 0x40), -5),                 # S0 partially overlaps S_T
+    (dict(S_T=P + 0x20000000 + 0x1000), -5),              # S_T overlaps v
+    (dict(S_T=P + 0x31000000 - 0x100), -5),               # S_T runs into beta
     (dict(B=1 << 16, T=1 << 16, H=1), -3),                # too many elements
 ], ids=lambda x: str(x))
 def test_prefill_rejects_bad_arguments(gdn, over, code):
@@ -165,6 +167,7 @@ def varlen_args(**over):
     (dict(cu=P + 0x60000002), -2), (dict(o=P + 0x40000008), -2),
     (dict(o=P + 0x60000000 - 64), -5),          # o runs into cu_seqlens
     (dict(S_T=P + 0x60000000 - 64 * 1024), -5),  # S_T runs into cu_seqlens
+    (dict(S_T=P + 0x10000000), -5),              # S_T over k
     (dict(snaps=P + 0x70000000, snap_every=100, n_snaps=2), -4),   # not a multiple of 64
     (dict(snaps=P + 0x70000000, snap_every=0, n_snaps=2), -4),
     (dict(snaps=P + 0x70000008, snap_every=64, n_snaps=2), -2),
