@@ -1,6 +1,6 @@
 """GPU check of the tcgen05 building blocks the prefill kernel relies on: each
-MMA form (K-major / MN-major SW128 descriptors, A from tensor memory, N=16
-sub-block with row and K offsets, negated A, N=64) on one 128x128 tile
+MMA form (K-major / MN-major SW128 descriptors for A and for B, A from tensor
+memory, N=16 sub-block with row and K offsets, negated A, N=64) on one 128x128 tile
 against a host matmul of the same bf16 inputs."""
 from __future__ import annotations
 
@@ -36,7 +36,7 @@ def test_selftest_library_builds():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4, 5])
+@pytest.mark.parametrize("mode", [0, 1, 2, 3, 4, 5, 6, 7, 8])
 def test_umma_forms(mode):
     lib = ctypes.CDLL(build_selftest())
     lib.umma_selftest.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]
@@ -61,7 +61,43 @@ def test_umma_forms(mode):
         ref, got = Af[:, 16:32] @ Bf[32:48, 16:32].T, D.double().cpu()[:, :16]
     elif mode == 4:
         ref, got = 1.0 - Af @ Bf.T, D.double().cpu()
-    else:
+    elif mode == 5:
         ref, got = Af @ Bf[:64].T, D.double().cpu()[:, :64]
+    elif mode == 6:
+        ref, got = Af.T @ Bf[:64].T, D.double().cpu()[:, :64]
+    elif mode == 7:
+        ref, got = Af[:64].T @ Bf[:64, :64].T, D.double().cpu()[:, :64]
+    else:
+        ref, got = Af @ Bf[:, :64], D.double().cpu()[:, :64]
     err = (got - ref).abs().max().item()
     assert err < 1e-3 * max(1.0, ref.abs().max().item()), f"mode {mode}: max err {err}"
+
+
+@pytest.mark.gpu
+def test_mma_issue_rate():
+    """Issue cost of tcgen05.mma from one thread (printed with -s): the kernel
+    design counts MMA instructions, not only FLOPs, so this records how long a
+    run of 128 MMAs of M = 128 and N = 32..256 takes to issue and to complete,
+    on one CTA and on one CTA per SM.  Checks only that every run completes."""
+    lib = ctypes.CDLL(build_selftest())
+    lib.umma_issue_probe.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 3
+    lib.umma_issue_probe.restype = ctypes.c_int
+    dev = torch.device("cuda:0")
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    out = torch.zeros(2 * sms, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    n = 128
+    for mode in range(8):
+        N = [64, 128, 256, 32][mode & 3]
+        for ctas in (1, sms):
+            for _ in range(2):  # the second run is the one recorded
+                rc = lib.umma_issue_probe(mode, n, ctas, out.data_ptr(), status.data_ptr(),
+                                          torch.cuda.current_stream().cuda_stream)
+                assert rc == 0
+            torch.cuda.synchronize()
+            assert int(status.item()) == 0
+            t = out.view(sms, 2)[:ctas].double().cpu().mean(0)
+            tflops = 128 * N * 16 * 2 * n / (t[1].item() * 1e-9) / 1e12
+            print(f"A from {'TMEM' if mode >= 4 else 'SMEM'} N={N:3d} CTAs={ctas:3d}: "
+                  f"issue {t[0].item() / n:.1f} ns/MMA, complete {t[1].item() / n:.1f} ns/MMA, "
+                  f"{tflops:.2f} TFLOP/s per SM")
