@@ -548,26 +548,55 @@ def run_extras(args, dev, stream, flush, peaks, rank):
     return out
 
 
+def prefill_bytes_dims(B, T, H, dk, dv, has_s0):
+    """q, k (Dk) and v (Dv) bf16, g, beta fp32, o (Dv) fp32 per token-head, plus the states."""
+    return B * T * H * (2 * dk * 2 + dv * 2 + 8 + dv * 4) + B * H * dk * dv * 4 * (2 if has_s0 else 1)
+
+
+def prefill_flops_dims(B, T, H, dk, dv, C=64):
+    """Chunk GEMM FLOPs per token-head at general head dims: S K^T, S Q^T and the
+    state update (6 Dk Dv), K K^T and Q K^T (4 C Dk), and the residual and
+    intra-chunk output products (6 C Dv); at Dk = Dv = D this is 6 D^2 + 10 C D."""
+    return B * T * H * (6 * dk * dv + 4 * C * dk + 6 * C * dv)
+
+
 def run_head_dim_extras(dev, stream, flush, peaks, rank, steps):
-    """Scalar gate at head dims other than 128 x 128 (the row-parallel fp32
-    kernel): the 16-head, 512-token prefill and the batched decode step."""
+    """Scalar gate at head dims other than 128 x 128: the 16-head, 512-token
+    prefill (Dk = 64 or 128: the chunked tensor-core kernel; Dk = 256: the
+    row-parallel fp32 kernel), a 4 x 32-head, 4096-token prefill at 128 x 256,
+    and the batched decode step (row kernel)."""
     from gated_deltanet_linear_20_b200 import gdn
     out = {}
     peak_ops = alu_peak_tops(dev)
-    for dk, dv in ((64, 64), (256, 256), (128, 256)):
-        d = gin.prefill_inputs(1, 512, 16, dk, dv, seed=7000 + rank, device=str(dev))
-        o = torch.empty((1, 512, 16, dv), dtype=torch.float32, device=dev)
-        sT = torch.empty((1, 16, dv, dk), dtype=torch.float32, device=dev)
+    for B, T, H, dk, dv in ((1, 512, 16, 64, 64), (1, 512, 16, 256, 256), (1, 512, 16, 128, 256),
+                            (1, 512, 16, 64, 128), (4, 4096, 32, 128, 256)):
+        d = gin.prefill_inputs(B, T, H, dk, dv, seed=7000 + rank, device=str(dev))
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+        sT = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
         ms = time_steps(lambda: gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None,
-                                            o=o, S_T=sT), steps, 3, flush, stream)
+                                            o=o, S_T=sT), steps if T <= 512 else 3, 3, flush, stream)
         t = statistics.mean(ms)
-        ops = 512 * 16 * 4 * dk * dv
-        out[f"prefill_b1_h16_t512_dk{dk}_dv{dv}"] = {
-            "tokens_per_s": round(512 / (t / 1e3), 1), "ms": round(t, 5),
-            "roofline": {"bound": "alu", "achieved": round(ops / (t / 1e3) / 1e12, 3),
-                         "peak": round(peak_ops, 2), "unit": "Tops/s (fp32 lane ops)",
-                         "frac": round(ops / (t / 1e3) / 1e12 / peak_ops, 4)}}
+        key = f"prefill_b{B}_h{H}_t{T}_dk{dk}_dv{dv}"
+        if dk == 256:
+            ops = B * T * H * 4 * dk * dv
+            out[key] = {
+                "tokens_per_s": round(B * T / (t / 1e3), 1), "ms": round(t, 5),
+                "kernel": "row-parallel fp32 (Dk = 256)",
+                "roofline": {"bound": "alu", "achieved": round(ops / (t / 1e3) / 1e12, 3),
+                             "peak": round(peak_ops, 2), "unit": "Tops/s (fp32 lane ops)",
+                             "frac": round(ops / (t / 1e3) / 1e12 / peak_ops, 4)}}
+        else:
+            nb = prefill_bytes_dims(B, T, H, dk, dv, False)
+            fl = prefill_flops_dims(B, T, H, dk, dv)
+            out[key] = {
+                "tokens_per_s": round(B * T / (t / 1e3), 1), "ms": round(t, 5),
+                "kernel": "chunked tcgen05, chunk 64" + (", two CTAs per chain" if dv == 256 else ""),
+                "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
+                "tensor_frac": round(fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"], 4)}
         del d, o, sT
+        torch.cuda.empty_cache()
     for dk, dv in ((256, 256), (64, 64)):
         B, H = 64, 16
         d = gin.prefill_inputs(B, 4, H, dk, dv, seed=7500 + rank, s0_std=0.02, device=str(dev))

@@ -81,16 +81,16 @@ int check_device() {
   return GDN_OK;
 }
 
-// 4-D view [B][T][H][128] of an activation (bf16 input or fp32 output); box =
-// `box_inner` features x 64 tokens of one head.  Loads of tokens past T read
-// zeros; stores past T are dropped.
+// 4-D view [B][T][H][F] of an activation (bf16 input or fp32 output, F its
+// feature dim); box = `box_inner` features x 64 tokens of one head.  Loads of
+// tokens past T read zeros; stores past T are dropped.
 bool encode_act(CUtensorMap* map, const void* base, int B, int T, int H, int box_inner,
-                CUtensorMapSwizzle swz, CUtensorMapDataType dtype, int esize) {
+                CUtensorMapSwizzle swz, CUtensorMapDataType dtype, int esize, int F = kHeadDim) {
   auto enc = get_encode_fn();
   if (!enc) return false;
-  const cuuint64_t dims[4] = {cuuint64_t(kHeadDim), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
-  const cuuint64_t strides[3] = {cuuint64_t(kHeadDim) * esize, cuuint64_t(H) * kHeadDim * esize,
-                                 cuuint64_t(T) * H * kHeadDim * esize};
+  const cuuint64_t dims[4] = {cuuint64_t(F), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(F) * esize, cuuint64_t(H) * F * esize,
+                                 cuuint64_t(T) * H * F * esize};
   const cuuint32_t box[4] = {cuuint32_t(box_inner), 1, 64, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
@@ -223,13 +223,16 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if (chunk != 16 && chunk != 64) return GDN_ERR_UNSUPPORTED;
   if (Dk != kHeadDim || Dv != kHeadDim) {
-    // other head dims: the row kernel (no chunking, no workspace, no fused options)
+    // other head dims: no fused options; Dk = 256 takes the row kernel (its fp32
+    // state and bf16 hi/lo copy alone would fill the 512 TMEM columns)
     if (qk_norm || q_scale != 1.f || o_bf16) return GDN_ERR_UNSUPPORTED;
-    return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, false, stream);
+    if (!gdn::rows_head_dims_ok(Dk, Dv)) return GDN_ERR_UNSUPPORTED;
+    if (Dk == 256) return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, false, stream);
+    allow_segments = false;  // the segmented schedule is built for 128 x 128 states
   }
   const long long chains = (long long)B * H;
-  const long long act = chains * T * kHeadDim;
-  if (act > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  const long long act = chains * T * (Dk > Dv ? Dk : Dv);
+  if (act > 0x7fffffffLL || chains * Dk * Dv > 0x7fffffffLL) return GDN_ERR_SHAPE;
   if (chains == 0) return GDN_OK;
   if (!S_T) return GDN_ERR_NULL;
   if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
@@ -237,25 +240,29 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
                 !aligned(g, 4) || !aligned(beta, 4)))
     return GDN_ERR_ALIGN;
-  const size_t act_bf16 = size_t(act) * 2, act_f32 = size_t(act) * (o_bf16 ? 2 : 4);  // o bytes
-  const size_t gate_bytes = size_t(chains) * T * 4, state_bytes = size_t(chains) * kHeadDim * kHeadDim * 4;
-  if (T > 0 && (overlaps(o, act_f32, q, act_bf16) || overlaps(o, act_f32, k, act_bf16) ||
-                overlaps(o, act_f32, v, act_bf16) || overlaps(o, act_f32, g, gate_bytes) ||
+  const size_t toks = size_t(chains) * T;
+  const size_t qk_bytes = toks * Dk * 2, v_bytes = toks * Dv * 2;
+  const size_t act_f32 = toks * Dv * (o_bf16 ? 2 : 4);  // o bytes
+  const size_t gate_bytes = toks * 4, state_bytes = size_t(chains) * Dk * Dv * 4;
+  if (T > 0 && (overlaps(o, act_f32, q, qk_bytes) || overlaps(o, act_f32, k, qk_bytes) ||
+                overlaps(o, act_f32, v, v_bytes) || overlaps(o, act_f32, g, gate_bytes) ||
                 overlaps(o, act_f32, beta, gate_bytes) || overlaps(o, act_f32, S0, state_bytes) ||
                 overlaps(o, act_f32, S_T, state_bytes)))
     return GDN_ERR_ALIAS;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
   // one chain may write its S_T while another still reads its inputs
-  if (T > 0 && (overlaps(S_T, state_bytes, q, act_bf16) || overlaps(S_T, state_bytes, k, act_bf16) ||
-                overlaps(S_T, state_bytes, v, act_bf16) || overlaps(S_T, state_bytes, g, gate_bytes) ||
+  if (T > 0 && (overlaps(S_T, state_bytes, q, qk_bytes) || overlaps(S_T, state_bytes, k, qk_bytes) ||
+                overlaps(S_T, state_bytes, v, v_bytes) || overlaps(S_T, state_bytes, g, gate_bytes) ||
                 overlaps(S_T, state_bytes, beta, gate_bytes)))
     return GDN_ERR_ALIAS;
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
 
+  const int dv_box = Dv < kHeadDim ? Dv : kHeadDim;
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     B,      T,
                      H,      status, 1,      (T + 63) / 64, 1, nullptr, nullptr, nullptr,
-                     nullptr, nullptr, 0,      0, qk_norm, q_scale, o_bf16};
+                     nullptr, nullptr, 0,      0, qk_norm, q_scale, o_bf16,
+                     Dk,     Dv,   Dv / dv_box, dv_box};
   if (allow_segments && T > 0) {
     int sms = 0;
     if (num_sms(&sms) != GDN_OK) return GDN_ERR_LAUNCH;
@@ -263,7 +270,7 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
     if (plan.nseg > 1) {
       if (!ws || !aligned(ws, 256) || ws_bytes < plan.ws_bytes) return GDN_ERR_WORKSPACE;
       const void* args[] = {q, k, v, g, beta, S0, o, S_T};
-      const size_t sizes[] = {act_bf16, act_bf16, act_bf16, gate_bytes, gate_bytes, state_bytes,
+      const size_t sizes[] = {qk_bytes, qk_bytes, v_bytes, gate_bytes, gate_bytes, state_bytes,
                               act_f32, state_bytes};
       for (int i = 0; i < 8; ++i)
         if (overlaps(ws, plan.ws_bytes, args[i], sizes[i])) return GDN_ERR_ALIAS;
@@ -279,11 +286,11 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   CUtensorMap tq{}, tk{}, tv{}, to{}, tf{};
   if (T > 0) {
     const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
-        !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
-        !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2) ||
-        !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, o_bf16 ? bf : f32,
-                    o_bf16 ? 2 : 4))
+    if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, Dk) ||
+        !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, Dk) ||
+        !encode_act(&tv, v, B, T, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv) ||
+        !encode_act(&to, o, B, T, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, o_bf16 ? bf : f32,
+                    o_bf16 ? 2 : 4, Dv))
       return GDN_ERR_LAUNCH;
     tf = to;
     if (a.nseg > 1 && !encode_act(&tf, a.ws_f, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4))
@@ -438,7 +445,8 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
   // B = N chains of sequences, T = total_T: the views are [1][total_T][H][128]
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
                      H,      status, 1,      (total_T + 63) / 64, 1, nullptr, nullptr, nullptr,
-                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, 0, 1.f, 0};
+                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, 0, 1.f, 0,
+                     kHeadDim, kHeadDim, 1, kHeadDim};
   CUtensorMap tq{}, tk{}, tv{}, to{};
   const int Tv = total_T > 0 ? total_T : 1;  // a valid (never read) view when every sequence is empty
   const void* qv = total_T > 0 ? q : S_T;
@@ -460,7 +468,7 @@ int gdn_prefill_static_ws(const void* q, const void* k, const void* v, const flo
   // their own codes rather than the limit
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if (chunk != 16 && chunk != 64) return GDN_ERR_UNSUPPORTED;
-  if (Dk != kHeadDim || Dv != kHeadDim)  // the row kernel needs no scratch
+  if (Dk != kHeadDim || Dv != kHeadDim)  // other head dims run one pass, which needs no scratch
     return prefill_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, chunk, nullptr, 0, false,
                         status, stream);
   const long long chains = (long long)B * H;

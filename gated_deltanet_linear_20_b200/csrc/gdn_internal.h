@@ -44,6 +44,11 @@ struct PrefillArgs {
   int qk_norm;
   float q_scale;
   int o_bf16;  // o is bf16 (same layout); single-pass schedule only
+  // Head dims: Dk (64 or 128) is the kernel's template parameter; Dv is 64,
+  // 128 or 256.  dv_ctas CTAs share a chain, each owning dv_box = min(Dv, 128)
+  // consecutive rows of its state (Dv = 256: two CTAs of 128 rows; Dv = 64:
+  // one CTA whose rows 64..127 stay zero).
+  int Dk, Dv, dv_ctas, dv_box;
 };
 
 struct DecodeArgs {

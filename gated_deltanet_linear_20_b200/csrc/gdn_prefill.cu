@@ -20,8 +20,12 @@
 //   O^T   = diag-cols(Gamma) (S_c Q^T) + Dl^T Mq^T,  Mq = tril(Q K^T .* Dec)
 //   S_out = Gamma_last S_c + Dl^T diag(exp(gamma_last - gamma)) K
 //
-// One CTA of 512 threads owns one (b, h) chain and walks its tokens in tiles
-// of 64 (one TMA tile); with chunk = 16 each tile holds four chunks.  The
+// One CTA of 512 threads owns one (b, h) chain (with Dv = 256, two CTAs own
+// 128 rows of its state each) and walks its tokens in tiles of 64 (one TMA
+// tile); with chunk = 16 each tile holds four chunks.  The key dimension Dk is
+// 64 or 128 (a template parameter: the K-dimension of the S products, the
+// state's TMEM columns and the K/Q boxes); the rows of the state a CTA owns are
+// the MMAs' M = 128 lanes (Dv = 64 keeps lanes 64..127 at zero).  The
 // warps split into three roles that run concurrently and hand off through
 // mbarriers:
 //   * chain  (warps 0-3 and 12-15, 256 threads): everything that depends on
@@ -41,7 +45,8 @@
 // bf16 parts (hi = bf16(x), lo = bf16(x - hi)) so the products keep ~16 bits
 // of mantissa; q, k and v are exact bf16 inputs.
 //
-// Tensor memory (512 columns, fp32 unless noted):
+// Tensor memory (512 columns, fp32 unless noted; with Dk = 64 the state uses
+// the first half of its ranges):
 //   [  0,128) S   : state, scaled by the next chunk's total decay  (lane dv, col dk)
 //   [128,192) SHI : S hi as bf16 pairs (A operand)                 (lane dv, col dk/2)
 //   [192,256) SLO : S lo
@@ -125,8 +130,9 @@ constexpr uint32_t M_TMEM = 0, M_ABORT = 4, M_PART = 8, M_KQ_ISSUED = 12, M_KQ_S
 static_assert(M_SNAP_PTR + 8 <= 64, "misc slots (the first 64 bytes are cleared at start)");
 static_assert(8 * NUM_BARS <= 256, "barrier slots");
 
-constexpr uint32_t KQ_TX_BYTES = 4 * 8192;
-constexpr uint32_t V_TX_BYTES = 16384;
+// K and Q of a tile: Dk / 64 boxes each of 64 tokens x 128 bytes
+template <int DK>
+constexpr uint32_t kq_tx_bytes() { return uint32_t(DK / 64) * 2u * 8192u; }
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -156,7 +162,8 @@ struct Ctx {
   const float* s0src;  // start state of this chain [128][128], or null
   float* odst;         // destination of o-like outputs, laid out like o
   const CUtensorMap* tmo;  // TMA view of odst: [B][T][H][128] fp32, box 64 tokens x 128
-  float* sdst;         // destination of the end state [128][128]
+  float* sdst;         // destination of the end state rows owned by this CTA
+  int dv0;             // first state row (value channel) owned by this CTA
   __device__ __forceinline__ uint32_t bar(uint32_t off) const { return sb + SM_BAR + off; }
   __device__ __forceinline__ float* gates(int c) const {
     return reinterpret_cast<float*>(sm + SM_GATES + (c % GATE_BUFS) * GATE_BYTES);
@@ -204,22 +211,27 @@ struct RoleSync {
   }
 };
 
+template <int DK>
 __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
                                          int c, int h, int b) {
   const uint32_t kq = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0);
   const uint32_t bar = x.bar((c & 1) ? B_FULL1 : B_FULL0);
-  mbar_arrive_expect_tx(bar, KQ_TX_BYTES);
+  mbar_arrive_expect_tx(bar, kq_tx_bytes<DK>());
   const int t0 = x.tok0 + c * NT;
   tma_load_4d(kq + 0, tk, bar, 0, h, t0, b);
   tma_load_4d(kq + 8192, tq, bar, 0, h, t0, b);
-  tma_load_4d(kq + 16384, tk, bar, 64, h, t0, b);
-  tma_load_4d(kq + 24576, tq, bar, 64, h, t0, b);
+  if constexpr (DK == 128) {
+    tma_load_4d(kq + 16384, tk, bar, 64, h, t0, b);
+    tma_load_4d(kq + 24576, tq, bar, 64, h, t0, b);
+  }
   *x.misc(M_KQ_ISSUED) = c + 1;
 }
+// V rows dv0 .. dv0 + DVB - 1 of the tile's 64 tokens ([64][DVB] bf16)
+template <int DVB>
 __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b) {
   const uint32_t bar = x.bar(B_VFULL);
-  mbar_arrive_expect_tx(bar, V_TX_BYTES);
-  tma_load_4d(x.sb + SM_V, tv, bar, 0, h, x.tok0 + c * NT, b);
+  mbar_arrive_expect_tx(bar, uint32_t(NT * DVB * 2));
+  tma_load_4d(x.sb + SM_V, tv, bar, x.dv0, h, x.tok0 + c * NT, b);
   *x.misc(M_V_ISSUED) = c + 1;
 }
 
@@ -383,11 +395,12 @@ __device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, f
   if (kt == 0) mbar_arrive(x.bar(gfull_off(c)));
 }
 
+template <int DK>
 __device__ __forceinline__ void issue_p(const Ctx& x, int c) {
   const uint64_t d0 = sdesc_sw128(x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0), 16, 1024);
   const uint32_t id = idesc_bf16(128, 64, 0, 0, 0);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
+  for (int kk = 0; kk < DK / 16; ++kk) {
     const uint64_t d = sdesc_add(d0, (kk >> 2) * 16384 + (kk & 3) * 32);
     mma_ss(x.tmem + TM_P, d, d, id, kk > 0);
   }
@@ -413,10 +426,12 @@ __device__ __noinline__ void store_partial_tile(const float4* src, float* dst, i
 // the copy) and waits for the copy to have read the tile before X^T is written
 // again.
 // OBF: o is bf16 (tile rows of 256 B, stored through a bf16 view).
-template <bool OBF>
+template <bool OBF, int DVB>
 __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b, int h, int dv,
                                              int hf, int c, bool leader) {
   const float* G = x.gates(c);
+  // staging tile [64 tokens][DVB]; with DVB = 64 lanes 64..127 hold zero rows
+  const bool own = DVB == D || dv < DVB;
   float* so = reinterpret_cast<float*>(x.sm + SM_XH) + dv;
   __nv_bfloat16* so16 = reinterpret_cast<__nv_bfloat16*>(x.sm + SM_XH) + dv;
 #pragma unroll
@@ -433,8 +448,8 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
         const float ov = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
         if constexpr (OBF)
           so16[n * D] = __float2bfloat16_rn(ov);
-        else
-          so[n * D] = ov;
+        else if (own)
+          so[n * DVB] = ov;
       }
     }
   }
@@ -444,7 +459,7 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
   if (ts + NT <= x.tend || x.tend == x.tmap) {
     // whole tile, or the view's own end clips it
     if (leader) {
-      tma_store_4d(x.tmo, x.sb + SM_XH, 0, h, ts, b);
+      tma_store_4d(x.tmo, x.sb + SM_XH, x.dv0, h, ts, b);
       bulk_commit();
     }
   } else if constexpr (!OBF) {
@@ -456,7 +471,7 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
   }
 }
 
-template <int C, bool PRE>
+template <int C, bool PRE, int DK, int DVB>
 __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, const PrefillArgs& p, int b, int h, int ntiles) {
   const int kt = threadIdx.x - 128;        // 0..255
@@ -474,9 +489,9 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   RoleSync rs{BAR_SIDE, SIDE_THREADS, M_FLAG_SIDE, leader, 0};
 
   if (leader) {
-    issue_kq(x, tq, tk, 0, h, b);
-    if (ntiles > 1) issue_kq(x, tq, tk, 1, h, b);
-    if (!x.vzero) issue_v(x, tv, 0, h, b);
+    issue_kq<DK>(x, tq, tk, 0, h, b);
+    if (ntiles > 1) issue_kq<DK>(x, tq, tk, 1, h, b);
+    if (!x.vzero) issue_v<DVB>(x, tv, 0, h, b);
   }
   float g_next = 0.f, b_next = 0.f;
   if (kt < NT && x.tok0 + kt < x.tend) {
@@ -493,7 +508,7 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   if (!rs.wait(x, x.bar(B_FULL0), 0)) return;
   if (leader) {
     *x.misc(M_KQ_SEEN) = 1;
-    issue_p(x, 0);
+    issue_p<DK>(x, 0);
   }
   int p_issued = 1;  // tiles whose P MMA was issued (leader's view)
   float mq[32];      // this thread's half row of Mq (lanes 64..127)
@@ -544,7 +559,7 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         mbar_try_wait(x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1)) {
       tc_fence_after();
       *x.misc(M_KQ_SEEN) = c + 2;
-      issue_p(x, c + 1);
+      issue_p<DK>(x, c + 1);
       p_issued = c + 2;
     }
 
@@ -627,7 +642,7 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       if (!rs.wait(x, x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1)) return;
       if (leader && p_issued == c + 1) {
         *x.misc(M_KQ_SEEN) = c + 2;
-        issue_p(x, c + 1);
+        issue_p<DK>(x, c + 1);
         p_issued = c + 2;
       }
     }
@@ -665,7 +680,7 @@ __device__ __noinline__ void copy_staged_state(const uint8_t* stg, float* dst, i
 // in `kq`: A = the bf16 hi / lo state pair in TMEM, B = K and Q rows.  With
 // chunk 64 the K and Q rows of the tile are adjacent (64 + 64 rows) and Y sits
 // right after Z in TMEM, so one N = 128 MMA per step computes both.
-template <int C>
+template <int C, int DK>
 __device__ __forceinline__ void issue_zq(const Ctx& x, uint32_t kq, int s) {
   // C rows of 128 B per chunk (C = 16)
   const uint64_t d0 = sdesc_sw128(kq + 2048u * uint32_t(s), 16, 1024);
@@ -673,7 +688,7 @@ __device__ __forceinline__ void issue_zq(const Ctx& x, uint32_t kq, int s) {
   for (int part = 0; part < 2; ++part) {
     const uint32_t a0 = x.tmem + (part ? TM_SLO : TM_SHI);
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
+    for (int kk = 0; kk < DK / 16; ++kk) {
       const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
       const uint32_t acc = (part | kk) ? 1u : 0u;
       if constexpr (C == 64) {
@@ -689,12 +704,14 @@ __device__ __forceinline__ void issue_zq(const Ctx& x, uint32_t kq, int s) {
 }
 
 // ============================================================== chain
-template <int C, bool OBF>
+template <int C, bool OBF, int DK, int DVB>
 __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, const PrefillArgs& p, int chain, int b, int h,
                            int ntiles) {
   constexpr int NSUB = NT / C;
-  constexpr int NC = C / 2;  // columns of a chunk per chain thread
+  constexpr int NC = C / 2;      // columns of a chunk per chain thread
+  constexpr int NQ = DK / 64;    // 32-column groups of the state per chain thread
+  constexpr int SCOLS = DK / 2;  // state columns per chain thread
   const int warp = threadIdx.x >> 5;
   const int lq = warp & 3;
   const int ch = (warp >= 12) ? 1 : 0;      // column half
@@ -704,15 +721,18 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   const uint32_t sb = x.sb;
   RoleSync rs{BAR_CHAIN, CHAIN_THREADS, M_FLAG_CHAIN, leader, 0};
 
-  // ---- initial state (row dv of S0, or zeros): hi/lo copy, and the fp32 copy
-  //      pre-scaled by the decay of the first chunk
+  // ---- initial state (row dv of S0, or zeros; rows past the CTA's own stay
+  //      zero): hi/lo copy, and the fp32 copy pre-scaled by the decay of the
+  //      first chunk
   if (!rs.wait(x, x.bar(gfull_off(0)), gfull_parity(0))) return;
   {
     const float gc0 = x.gates(0)[G_GC / 4];
-    const float4* src = x.s0src ? reinterpret_cast<const float4*>(x.s0src + size_t(dv) * D) : nullptr;
+    const float4* src = (x.s0src && (DVB == D || dv < DVB))
+                            ? reinterpret_cast<const float4*>(x.s0src + size_t(dv) * DK)
+                            : nullptr;
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int qq = 2 * ch + q;  // 32-column group
+    for (int q = 0; q < NQ; ++q) {
+      const int qq = NQ * ch + q;  // 32-column group
       float v[32];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -753,7 +773,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         if (!ok) x.fail();
         if (ok && !*x.abort_flag) {
           tc_fence_after();
-          issue_zq<C>(x, kq, s);
+          issue_zq<C, DK>(x, kq, s);
           mma_commit(x.bar(B_ZQ));
         }
       }
@@ -801,7 +821,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int n = n0 + 4 * e4 + e;
-            const float vn = x.vzero ? 0.f : __bfloat162float(V[n * D + dv]);
+            const float vn = (x.vzero || (DVB != D && dv >= DVB)) ? 0.f : __bfloat162float(V[n * DVB + dv]);
             xv[4 * e4 + e] = fmaf(bv[e], vn, -gv[e] * z[4 * e4 + e]);
           }
         }
@@ -811,7 +831,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar(BAR_CHAIN, CHAIN_THREADS);
-      if (leader && s == NSUB - 1 && !last_tile && !x.vzero) issue_v(x, tv, c + 1, h, b);  // V(c) read
+      if (leader && s == NSUB - 1 && !last_tile && !x.vzero) issue_v<DVB>(x, tv, c + 1, h, b);  // V(c) read
 
       // ---- Dl^T = X^T T^T : M=128 (dv), N=C (i), K=C (n); 3 hi/lo products
       if (leader) {
@@ -891,7 +911,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
                    (part | ks) ? 1u : 0u);
           }
         }
-        const uint32_t idu = idesc_bf16(128, 128, 0, 1, 0);
+        const uint32_t idu = idesc_bf16(128, DK, 0, 1, 0);
         const uint64_t dk = sdesc_sw128(kq + uint32_t(C * s) * 128u, 16384, 1024);  // K rows, MN-major
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
@@ -906,11 +926,11 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         if (s == NSUB - 1) mma_commit(x.bar(B_TMFREE));  // T(c), Mq(c) consumed
       }
       if (!rs.wait(x, x.bar(B_OU), sc & 1)) return;
-      if (leader && s == NSUB - 1 && c + 2 < ntiles) issue_kq(x, tq, tk, c + 2, h, b);  // KQ(c) read
+      if (leader && s == NSUB - 1 && c + 2 < ntiles) issue_kq<DK>(x, tq, tk, c + 2, h, b);  // KQ(c) read
 
       // ---- o of the whole tile is complete after its last chunk: o[t][dv] =
       //      Gamma_t Y[dv][t] + O_intra[dv][t], this thread's 32 tokens to HBM
-      if (s == NSUB - 1) output_drain<OBF>(x, tlane, b, h, dv, ch, c, leader);
+      if (s == NSUB - 1) output_drain<OBF, DVB>(x, tlane, b, h, dv, ch, c, leader);
 
       // ---- S_out now sits in TMEM: refresh its hi/lo copy, and pre-scale it by
       //      the next chunk's decay (or store it as S_T after the last chunk)
@@ -923,7 +943,26 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           if (!rs.wait(x, x.bar(gfull_off(c + 1)), gfull_parity(c + 1))) return;
           gnext = x.gates(c + 1)[G_GC / 4];
         }
-        if (final_chunk) {
+        if (final_chunk && (DK != D || DVB != D)) {
+          // other head dims: this thread's columns of its own row, straight to HBM
+          if (DVB == D || dv < DVB) {
+            float4* dst = reinterpret_cast<float4*>(x.sdst + size_t(dv) * DK + SCOLS * ch);
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+              float v[32];
+              tmem_ld32(tlane + TM_S + SCOLS * ch + 32 * q, v);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[8 * q + e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {  // keep the warp's TMEM loads convergent
+              float v[32];
+              tmem_ld32(tlane + TM_S + SCOLS * ch + 32 * q, v);
+            }
+          }
+        } else if (final_chunk) {
           // the end state goes out through the X^T / Dl^T region (64 KB, free once
           // the o store has read it): rows of 512 B whose 16-byte chunks are
           // XOR-swizzled by the row, then copied out row by row
@@ -960,11 +999,11 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
               snapshot_row(tlane, 64 * ch, snap + (size_t((c + 1) / stiles - 1) * x.H * D + dv) * D);
             }
           }
-          // this thread's 64 columns, 32 at a time: load, split, store hi / lo /
+          // this thread's DK / 2 columns, 32 at a time: load, split, store hi / lo /
           // pre-scaled fp32 in one waited group
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int col = 64 * ch + 32 * q;
+          for (int q = 0; q < NQ; ++q) {
+            const int col = SCOLS * ch + 32 * q;
             float v[32];
             tmem_ld32(tlane + TM_S + col, v);
             uint32_t hi[16], lo[16], u[32];
@@ -983,31 +1022,36 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
-template <int C, bool PRE, bool OBF>
+template <int C, bool PRE, bool OBF, int DK, int DVB>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                    const __grid_constant__ CUtensorMap tm_f, const PrefillArgs p) {
   static_assert(C == 16 || C == 64, "chunk must be 16 or 64");
+  static_assert(DK == 64 || DK == 128, "key dimension must be 64 or 128");
+  static_assert(DVB == 64 || DVB == 128, "a CTA owns 64 or 128 rows of the state");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int total_tiles = (p.T + NT - 1) / NT;
-  // CTA -> (chain, segment, kind); see PrefillArgs
-  int chain = blockIdx.x, seg = 0;
+  // CTA -> (chain, segment, kind, rows of the state); see PrefillArgs
+  const int dvpart = int(blockIdx.x) % p.dv_ctas;
+  const int cta = int(blockIdx.x) / p.dv_ctas;
+  int chain = cta, seg = 0;
   bool frun = false;
   if (p.nseg > 1) {
     const int per = 2 * p.nseg - 1;
-    chain = blockIdx.x / per;
-    const int j = blockIdx.x - chain * per;
+    chain = cta / per;
+    const int j = cta - chain * per;
     frun = j >= p.nseg;
     seg = frun ? j - p.nseg + 1 : j;
   }
   int b = chain / p.H;
   const int h = chain - b * p.H;
-  const size_t cstate = size_t(chain) * D * D;
+  const size_t cstate = size_t(chain) * p.Dv * DK;  // this chain's state
+  const int dv0 = dvpart * 128;                       // first row owned by this CTA
 
   Ctx x;
   x.sm = sm;
@@ -1018,6 +1062,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   x.tok0 = 0;
   x.tend = p.T;
   x.tmap = p.T;
+  x.dv0 = dv0;
   int ntiles = total_tiles;
   if (p.cu_seqlens) {
     // packed sequences: chain = n H + h walks tokens [cu[n], cu[n+1]) of views with B = 1
@@ -1040,7 +1085,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
   x.vzero = frun;
   x.s0_identity = frun;
-  x.s0src = (seg == 0 && p.S0) ? p.S0 + cstate : nullptr;
+  x.s0src = (seg == 0 && p.S0) ? p.S0 + cstate + size_t(dv0) * DK : nullptr;
   x.odst = frun ? p.ws_f : p.o;
   x.tmo = frun ? &tm_f : &tm_o;
   if (p.nseg > 1) {
@@ -1049,7 +1094,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     ntiles = min(p.seg_tiles, total_tiles - tb);
     x.sdst = (frun ? p.ws_F : p.ws_R) + (size_t(chain) * p.nseg + seg) * D * D;
   } else {
-    x.sdst = p.S_T + cstate;
+    x.sdst = p.S_T + cstate + size_t(dv0) * DK;
   }
   if (tid == 0) {
     prefetch_tmap(&tm_q);
@@ -1061,7 +1106,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = 0; i < 16; ++i) reinterpret_cast<volatile int*>(sm + SM_MISC)[i] = 0;
     if (p.snaps && p.cu_seqlens) {
       // first snapshot slot of this sequence: one per snap_every tokens of
-      // every earlier sequence
       // every earlier sequence; an invalid earlier entry (its own CTAs report
       // it) leaves this sequence without snapshots rather than with a slot
       // index computed from garbage
@@ -1098,9 +1142,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // for this grid to complete before it reads anything this grid writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp < 4 || warp >= 12)
-    chain_role<C, OBF>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
+    chain_role<C, OBF, DK, DVB>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
   else
-    kside_role<C, PRE>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
+    kside_role<C, PRE, DK, DVB>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
 
   if (tid == 0) bulk_wait0();  // the chain leader's o stores have completed
   tc_fence_before();
@@ -1137,13 +1181,13 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   const int chains = a.B * a.H;
   if (chains == 0) return 0;
   if (a.T == 0) {
-    const size_t n4 = size_t(chains) * D * D / 4;
+    const size_t n4 = size_t(chains) * a.Dv * a.Dk / 4;
     if (a.S0 == a.S_T) return 0;
     copy_state_kernel<<<unsigned((n4 + 255) / 256), 256, 0, stream>>>(a.S0, a.S_T, n4);
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   }
   const uint32_t smem = SMEM_USED + 1024;
-  const int ctas = a.nseg > 1 ? chains * (2 * a.nseg - 1) : chains;
+  const int ctas = (a.nseg > 1 ? chains * (2 * a.nseg - 1) : chains) * a.dv_ctas;
   const bool pre = a.qk_norm || a.q_scale != 1.f;  // fused q / k pre-steps requested
   auto go = [&](auto kernel, int slot) {
     if (!ensure_smem_attr(reinterpret_cast<const void*>(kernel), slot, int(smem))) return false;
@@ -1152,16 +1196,29 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   };
   const bool obf = a.o_bf16 != 0;
   bool ok;
-  if (chunk == 64) {
-    if (obf)
-      ok = pre ? go(prefill_kernel<64, true, true>, 5) : go(prefill_kernel<64, false, true>, 6);
+  if (a.Dk != D || a.Dv != D) {  // plain calls only: no fused options at other head dims
+    if (pre || obf) return -1;
+    const bool c64 = chunk == 64;
+    if (a.Dk == D)  // Dv = 64 (Dv = 256 runs the 128 x 128 kernel on two CTAs per chain)
+      ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 128, 128>, 0)
+                                : go(prefill_kernel<16, false, false, 128, 128>, 1))
+                         : (c64 ? go(prefill_kernel<64, false, false, 128, 64>, 9)
+                                : go(prefill_kernel<16, false, false, 128, 64>, 10));
     else
-      ok = pre ? go(prefill_kernel<64, true, false>, 3) : go(prefill_kernel<64, false, false>, 0);
+      ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 64, 128>, 11)
+                                : go(prefill_kernel<16, false, false, 64, 128>, 12))
+                         : (c64 ? go(prefill_kernel<64, false, false, 64, 64>, 13)
+                                : go(prefill_kernel<16, false, false, 64, 64>, 14));
+  } else if (chunk == 64) {
+    if (obf)
+      ok = pre ? go(prefill_kernel<64, true, true, 128, 128>, 5) : go(prefill_kernel<64, false, true, 128, 128>, 6);
+    else
+      ok = pre ? go(prefill_kernel<64, true, false, 128, 128>, 3) : go(prefill_kernel<64, false, false, 128, 128>, 0);
   } else {
     if (obf)
-      ok = pre ? go(prefill_kernel<16, true, true>, 7) : go(prefill_kernel<16, false, true>, 8);
+      ok = pre ? go(prefill_kernel<16, true, true, 128, 128>, 7) : go(prefill_kernel<16, false, true, 128, 128>, 8);
     else
-      ok = pre ? go(prefill_kernel<16, true, false>, 4) : go(prefill_kernel<16, false, false>, 1);
+      ok = pre ? go(prefill_kernel<16, true, false, 128, 128>, 4) : go(prefill_kernel<16, false, false, 128, 128>, 1);
   }
   if (!ok) return -1;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;

@@ -1,7 +1,10 @@
 """GPU parity at head dims other than 128 x 128 (64, 128, 256 in any
 combination, Dk != Dv included), through the same C entry points, against the
-fp64 oracles (which take any Dk, Dv).  These shapes run the row-parallel fp32
-kernel; the contract and the 1e-4 design margin are those of the other tests.
+fp64 oracles (which take any Dk, Dv).  Prefill with Dk = 64 or 128 runs the
+chunked tensor-core kernel (Dv = 256: two CTAs per chain, 128 state rows each;
+Dv = 64: one CTA with its upper 64 rows held at zero); Dk = 256, decode and
+the per-channel gate run the row-parallel fp32 kernel.  The contract and the
+1e-4 design margin are those of the other tests.
 """
 from __future__ import annotations
 
@@ -93,6 +96,60 @@ def test_other_head_dims_in_place_and_deterministic():
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
     assert torch.equal(o3, o1) and torch.equal(S3, S1) and S3.data_ptr() == S_in.data_ptr()
+
+
+TC_DIMS = [(64, 64), (64, 128), (64, 256), (128, 64), (128, 256)]
+
+
+@pytest.mark.parametrize("dk,dv", TC_DIMS, ids=lambda x: str(x))
+@pytest.mark.parametrize("chunk", [64, 16])
+@pytest.mark.parametrize("T", [1, 64, 130], ids=lambda t: f"T{t}")
+def test_tensor_core_head_dims_chunks_and_tails(dk, dv, chunk, T):
+    """The tensor-core shapes at both chunks, one token, one full tile and a
+    ragged third tile; S0 carried in; the device status word stays 0."""
+    gdn = _gdn()
+    d = inputs.prefill_inputs(2, T, 3, dk, dv, seed=dk + dv + T + chunk, s0_std=0.05)
+    dd = to_dev(d)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"], chunk=chunk,
+                         status=status)
+    assert gdn.query_status(status) == 0
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o {dk}x{dv} chunk {chunk} T {T}")
+    assert_parity(S_T.cpu().numpy(), rS, f"S_T {dk}x{dv} chunk {chunk} T {T}")
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 256), (64, 64)], ids=lambda x: str(x))
+def test_tensor_core_head_dims_in_place_deterministic_and_segmented_flag(dk, dv):
+    """The state updated in place (two CTAs write the two row halves of one
+    state when Dv = 256), bitwise run-to-run determinism, and the segmented
+    entry point (which runs the single pass at these dims) giving the same bits."""
+    gdn = _gdn()
+    d = to_dev(inputs.prefill_inputs(2, 200, 3, dk, dv, seed=31 + dk, s0_std=0.05))
+    o1, S1 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], segmented=False)
+    o2, S2 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], segmented=True)
+    S_in = d["S0"].clone()
+    o3, S3 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], S_in, S_T=S_in)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    assert torch.equal(o3, o1) and torch.equal(S3, S1) and S3.data_ptr() == S_in.data_ptr()
+
+
+def test_tensor_core_head_dims_many_chains_sampled():
+    """128 x 256 at B4 H32 T1024 (256 CTAs, two per chain), checked on sampled chains."""
+    gdn = _gdn()
+    B, T, H, dk, dv = 4, 1024, 32, 128, 256
+    d = inputs.prefill_inputs(B, T, H, dk, dv, seed=5, g_mean=2.0)
+    dd = to_dev(d)
+    o, S_T = gdn.prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], None)
+    torch.cuda.synchronize()
+    chains = [0, 37, 127]
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None, chains=chains)
+    o, S_T = o.cpu().numpy(), S_T.cpu().numpy()
+    for c in chains:
+        b, h = divmod(c, H)
+        assert_parity(o[b, :, h], ro[b, :, h], f"o chain {c}")
+        assert_parity(S_T[b, h], rS[b, h], f"S_T chain {c}")
 
 
 def test_other_head_dims_reject_fused_options_on_gpu():
