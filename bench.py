@@ -625,13 +625,13 @@ def run_head_dim_extras(dev, stream, flush, peaks, rank, steps):
 
 
 def run_kda_extras(dev, stream, flush, peaks, rank, steps):
-    """The per-channel-gate (KDA) kernel: the headline shape, a large batch, and
-    the batched decode step.  Its work is fp32 lane arithmetic (4 operations per
-    state element and token), so the roofline is the SMs' FP32 lanes at the
-    maximum clock; the HBM fraction is reported beside it."""
+    """The per-channel gate (KDA): prefill at 128 x 128 on the chunked
+    tensor-core kernel (32-token chunks; HBM roofline, with the tensor fraction
+    of the same chunk-GEMM FLOP count as the scalar gate beside it), at the
+    512-token single-sequence shape and a large batch; and the batched decode
+    step on the row kernel (HBM roofline)."""
     from gated_deltanet_linear_20_b200 import gdn
     out = {}
-    peak_ops = alu_peak_tops(dev)
     for (B, T, H, g_mean, n) in ((1, 512, 16, 0.0, steps), (4, 8192, 32, 2.0, 3)):
         d = gin.kda_inputs(B, T, H, seed=5000 + rank, g_mean=g_mean, device=str(dev))
         o = torch.empty((B, T, H, D), dtype=torch.float32, device=dev)
@@ -639,15 +639,16 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
         ms = time_steps(lambda: gdn.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None,
                                                 o=o, S_T=sT), n, 3, flush, stream)
         t = statistics.mean(ms)
-        ops = B * T * H * KDA_OPS_PER_TOKEN_HEAD
         nb = kda_prefill_bytes(B, T, H, False)
+        fl = prefill_flops(B, T, H)
         out[f"kda_prefill_b{B}_h{H}_t{T}"] = {
             "tokens_per_s": round(B * T / (t / 1e3), 1), "ms": round(t, 5),
-            "roofline": {"bound": "alu", "achieved": round(ops / (t / 1e3) / 1e12, 3),
-                         "peak": round(peak_ops, 2), "unit": "Tops/s (fp32 lane ops)",
-                         "frac": round(ops / (t / 1e3) / 1e12 / peak_ops, 4),
-                         "peak_source": "SMs x 128 fp32 lanes x 1965 MHz"},
-            "hbm_frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+            "kernel": "chunked tcgen05, chunk 32",
+            "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                         "bytes_per_token_head": KDA_TOKEN_HEAD_BYTES},
+            "tensor_frac": round(fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
             "gate": f"per channel, logsigmoid(N({g_mean},1))"}
         del d, o, sT
     # decode: one token for 64 x 16 heads, state in place, L2 flushed per step

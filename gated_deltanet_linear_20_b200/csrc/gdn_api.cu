@@ -82,16 +82,17 @@ int check_device() {
 }
 
 // 4-D view [B][T][H][F] of an activation (bf16 input or fp32 output, F its
-// feature dim); box = `box_inner` features x 64 tokens of one head.  Loads of
-// tokens past T read zeros; stores past T are dropped.
+// feature dim); box = `box_inner` features x `box_tokens` tokens of one head.
+// Loads of tokens past T read zeros; stores past T are dropped.
 bool encode_act(CUtensorMap* map, const void* base, int B, int T, int H, int box_inner,
-                CUtensorMapSwizzle swz, CUtensorMapDataType dtype, int esize, int F = kHeadDim) {
+                CUtensorMapSwizzle swz, CUtensorMapDataType dtype, int esize, int F = kHeadDim,
+                int box_tokens = 64) {
   auto enc = get_encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[4] = {cuuint64_t(F), cuuint64_t(H), cuuint64_t(T), cuuint64_t(B)};
   const cuuint64_t strides[3] = {cuuint64_t(F) * esize, cuuint64_t(H) * F * esize,
                                  cuuint64_t(T) * H * F * esize};
-  const cuuint32_t box[4] = {cuuint32_t(box_inner), 1, 64, 1};
+  const cuuint32_t box[4] = {cuuint32_t(box_inner), 1, cuuint32_t(box_tokens), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -548,16 +549,53 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
 int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
                     const float* beta, const float* S0, float* o, float* S_T, int B, int T,
                     int H, int Dk, int Dv, int* status, void* stream) {
-  (void)status;  // the kernel has no device-side waits
-  return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, true, stream);
+  // the row kernel validates every argument; at 128 x 128 with tokens to process
+  // the chunked tensor-core kernel runs instead (same validation first)
+  if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (Dk != kHeadDim || Dv != kHeadDim || T == 0 || (long long)B * H == 0)
+    return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, true, stream);
+  const long long chains = (long long)B * H;
+  if (chains * T * kHeadDim > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL)
+    return GDN_ERR_SHAPE;
+  if (!S_T || !q || !k || !v || !g || !beta || !o) return GDN_ERR_NULL;
+  if (!aligned(S_T, 16) || (S0 && !aligned(S0, 16)) || !aligned(q, 16) || !aligned(k, 16) ||
+      !aligned(v, 16) || !aligned(g, 16) || !aligned(o, 16) || !aligned(beta, 4))
+    return GDN_ERR_ALIGN;
+  const size_t toks = size_t(chains) * T;
+  const size_t act_bf16 = toks * kHeadDim * 2, o_bytes = toks * kHeadDim * 4;
+  const size_t g_bytes = toks * kHeadDim * 4, beta_bytes = toks * 4;
+  const size_t state_bytes = size_t(chains) * kHeadDim * kHeadDim * 4;
+  if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
+  const void* ins[5] = {q, k, v, g, beta};
+  const size_t in_bytes[5] = {act_bf16, act_bf16, act_bf16, g_bytes, beta_bytes};
+  for (int i = 0; i < 5; ++i)
+    if (overlaps(o, o_bytes, ins[i], in_bytes[i]) || overlaps(S_T, state_bytes, ins[i], in_bytes[i]))
+      return GDN_ERR_ALIAS;
+  if (overlaps(o, o_bytes, S_T, state_bytes) || overlaps(o, o_bytes, S0, state_bytes))
+    return GDN_ERR_ALIAS;
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+  CUtensorMap tq{}, tk{}, tv{}, to{};
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
+      !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
+      !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, kHeadDim, 32) ||
+      !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, kHeadDim, 32))
+    return GDN_ERR_LAUNCH;
+  gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status};
+  return gdn::launch_kda_prefill(tq, tk, tv, to, a, static_cast<cudaStream_t>(stream)) == 0
+             ? GDN_OK
+             : GDN_ERR_LAUNCH;
 }
 
 int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                    int* status, void* stream) {
+  (void)status;  // the row kernel has no device-side waits
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
-  return gdn_kda_prefill(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, status, stream);
+  // a few tokens per call: the row kernel streams the state once
+  return rows_impl(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, true, stream);
 }
 
 int gdn_query_status(const int* status_dev, void* stream) {

@@ -79,6 +79,16 @@ struct RowArgs {
   int B, H, T, Dv;
 };
 
+// Chunked per-channel-gate (KDA) prefill on the tensor cores, Dk = Dv = 128.
+struct KdaArgs {
+  const float* g;     // [B][T][H][128] natural-log decays per key channel
+  const float* beta;  // [B][T][H]
+  const float* S0;    // [B][H][128][128] or null (zeros)
+  float* S_T;         // may equal S0
+  int B, T, H;
+  int* status;        // may be null
+};
+
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device
 // (slot: a small per-kernel index); returns false if the attribute call failed.
 bool ensure_smem_attr(const void* func, int slot, int bytes);
@@ -89,6 +99,10 @@ bool ensure_smem_attr(const void* func, int slot, int bytes);
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& to, const CUtensorMap& tf, const PrefillArgs& a, int chunk,
                    cudaStream_t stream);
+// tq, tk: bf16 q, k boxes of 64 features x 32 tokens (SW128); tv: bf16 v, tv:
+// 128 x 32 unswizzled; to: fp32 o, 128 x 32.  T > 0 and B*H > 0.
+int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const KdaArgs& a, cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Second pass of the segmented schedule (a.nseg > 1).
 int launch_segment_fix(const PrefillArgs& a, cudaStream_t stream);

@@ -1,0 +1,739 @@
+// Chunked delta rule with a per-channel gate (KDA) on the 5th-generation tensor
+// cores (sm_100a): 32-token TMA tiles, tcgen05 MMAs accumulating in tensor
+// memory, the fp32 state carried from chunk to chunk in tensor memory.
+//
+// Recurrence (per sequence b, head h; S in R^{Dv x Dk}, Dk = Dv = 128; g_t a
+// vector of natural-log decays over the key channels):
+//   S_t = S_{t-1} diag(exp(g_t)) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t.
+// The ROCmFPX gated-delta-net prefill note (bittide.aicompass.dev article
+// d2880479, opening post) names KDA among the cases its chunked kernel left to
+// the per-token path; this kernel chunks it.
+//
+// Chunked form (tokens i, j of one chunk; S_c the state entering it;
+// gamma_i = inclusive cumulative sum of g inside the chunk, per channel, and
+// Lambda_i = exp(gamma_i); r = the chunk's middle token):
+//   K+ = K o Lambda,  Q+ = Q o Lambda                 (decayed from the chunk start)
+//   K' = K o Lambda / Lambda_r,  Q' = Q o Lambda / Lambda_r,  K'' = K o Lambda_r / Lambda
+//   A  = strict_tril(diag(beta) K' K''^T),   Mq = tril(Q' K''^T)   (r cancels)
+//   T  = (I + A)^{-1}
+//   X^T  = V^T diag(beta) - (S_c K+^T) diag(beta),   Dl^T = X^T T^T
+//   O^T  = S_c Q+^T + Dl^T Mq^T
+//   S'   = S_c diag(Lambda_last) + Dl^T (K o Lambda_last / Lambda)
+// The reference r keeps every factor of K', Q', K'' within exp(+-16 |g|) for a
+// 32-token chunk: exact while a channel's decay over 16 tokens stays above
+// e^-87 (the fp32 range); beyond that the exponents are clamped (no inf/NaN).
+//
+// One CTA of 512 threads owns one (b, h) chain; two roles hand off through
+// mbarriers:
+//   * chain (warps 0-3, 12-15): S_c [K+;Q+]^T, X, Dl = X T^T, the state update
+//     and the output product, their epilogues, and the o store;
+//   * side (warps 4-11), one chunk ahead: the gates (per-channel cumulative
+//     decays), the decayed operand tiles, [K';Q'] K''^T, masks, the triangular
+//     solve, and the hand-over of T, Mq and the chain's operand tiles.
+// Every operand derived in the kernel is fed to the tensor core as a bf16
+// hi/lo pair (hi = bf16(x), lo = bf16(x - hi)); products of two derived
+// operands take hi*hi + hi*lo + lo*hi.  Where a product has an exact A
+// operand or a free N dimension, the hi and lo of one operand are stacked
+// along N and the halves summed in the epilogue (fewer MMA instructions).
+//
+// Tensor memory (512 columns, fp32):
+//   [  0,128) S   : state, pre-scaled by the next chunk's decay (per column)
+//   [128,192) SHI : S hi (bf16 pairs)      [192,256) SLO : S lo
+//   [256,384) ZQ  : [Z | Y] of S hi x [K+;Q+] hi, then [Z | Y] of S hi x lo    (32 cols each)
+//   [384,448) P   : [K';Q'] x [K'' hi | K'' lo]   (lanes 0..63 used)
+//   [448,512) DO  : [Dl | Dl'] of X x [T hi | T lo], then [O | O'] of Dl x [Mq hi | Mq lo]
+#include "gdn_internal.h"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+
+constexpr int D = 128;
+constexpr int NT = 32;  // tokens per tile (= chunk)
+constexpr int NTHREADS = 512;
+constexpr int CHAIN_THREADS = 256, SIDE_THREADS = 256;
+constexpr int BAR_CHAIN = 1, BAR_SIDE = 2;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TM_S = 0, TM_SHI = 128, TM_SLO = 192, TM_ZQ = 256, TM_P = 384, TM_DO = 448;
+
+// Shared memory (offsets from a 1024-byte aligned base).  K-major SW128 tiles
+// have 128-byte rows (64 bf16 along K) in 8-row groups 1024 B apart.
+constexpr uint32_t SM_KQ = 0;          // raw [K dk0-63 | Q dk0-63 | K dk64-127 | Q dk64-127], 4 KB boxes
+constexpr uint32_t SM_V = 16384;       // raw V [32 tokens][128] bf16
+constexpr uint32_t SM_ZQB = 24576;     // [K+ hi; Q+ hi; K+ lo; Q+ lo] 128 rows, boxes dk0-63 / dk64-127 16 KB apart
+constexpr uint32_t SM_PA = 57344;      // [K'; Q'] hi (64 rows, boxes 8 KB apart), then lo at +16 KB
+constexpr uint32_t SM_PB = 90112;      // [K'' hi; K'' lo] 64 rows, boxes 8 KB apart
+constexpr uint32_t SM_KT = 106496;     // K~ = K o Lambda_last / Lambda, rows j, MN-major: hi (2 x 4 KB), lo at +8 KB
+constexpr uint32_t SM_XH = 122880;     // X^T hi rows dv (K = 32 tokens in the first 64 B of a row);
+constexpr uint32_t SM_XL = 139264;     //   X^T hi doubles as the fp32 [32][128] o staging tile
+constexpr uint32_t SM_DH = 155648;     // Dl^T hi / lo, rows dv
+constexpr uint32_t SM_DL = 172032;
+constexpr uint32_t SM_TM = 188416;     // [T hi; T lo] rows i (32 + 32), K = 32 tokens
+constexpr uint32_t SM_MQ = 196608;     // [Mq hi; Mq lo]
+constexpr int APAD = 36;               // solve row pitch (floats)
+constexpr uint32_t SM_A = 204800;      // A fp32 [32][APAD]
+constexpr uint32_t SM_TF = SM_A + 32 * APAD * 4;   // T fp32 [32][APAD]
+constexpr uint32_t SM_X = SM_TF + 32 * APAD * 4;   // exchange: per-quarter channel sums [4][128],
+                                                   // then the solve's [16][16] product
+constexpr uint32_t SM_GATES = SM_X + 4 * 128 * 4;
+constexpr uint32_t GATE_BYTES = 640;   // beta [32], Lambda_last [128]
+constexpr uint32_t G_B = 0, G_LC = 128;
+constexpr int GATE_BUFS = 4;
+constexpr uint32_t SM_BAR = SM_GATES + GATE_BUFS * GATE_BYTES;
+constexpr uint32_t SM_MISC = SM_BAR + 256;
+constexpr uint32_t SMEM_USED = SM_MISC + 256;
+static_assert(SM_ZQB % 1024 == 0 && SM_PA % 1024 == 0 && SM_PB % 1024 == 0 && SM_KT % 1024 == 0 &&
+                  SM_XH % 1024 == 0 && SM_DH % 1024 == 0 && SM_TM % 1024 == 0 && SM_MQ % 1024 == 0,
+              "SW128 tiles need 1024-byte alignment");
+// the M = 128 reads of the [K';Q'] tiles run 8 KB past each 64-row box: they
+// must stay inside this CTA's shared memory (the rows read there are unused)
+static_assert(SM_PA + 32768 + 8192 <= SM_KT, "P operand over-read stays in the operand region");
+static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
+
+// mbarriers (8 bytes each, offsets inside SM_BAR)
+constexpr uint32_t B_KQFULL = 0, B_VFULL = 8, B_P = 16, B_TMFULL = 24, B_TMFREE = 32,
+                   B_OPFULL = 40, B_OPFREE = 48, B_ZQ = 56, B_DL = 64, B_SU = 72, B_OI = 80,
+                   B_CLEAN0 = 88, B_CLEAN1 = 96, B_GFULL = 104;  // B_GFULL: 4 barriers
+constexpr int NUM_BARS = 17;
+static_assert(8 * NUM_BARS <= 256, "barrier slots");
+__device__ __forceinline__ uint32_t gfull_off(int c) { return B_GFULL + 8u * uint32_t(c & 3); }
+__device__ __forceinline__ uint32_t gfull_parity(int c) { return uint32_t(c >> 2) & 1u; }
+constexpr uint32_t M_TMEM = 0, M_ABORT = 4, M_KQ_ISSUED = 12, M_KQ_SEEN = 16, M_V_ISSUED = 20,
+                   M_V_SEEN = 24, M_FLAG_CHAIN = 32, M_FLAG_SIDE = 40;
+
+constexpr uint32_t KQ_TX_BYTES = 4 * 4096;
+constexpr uint32_t V_TX_BYTES = NT * D * 2;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
+constexpr float LOG2E = 1.4426950408889634f;
+constexpr float EXP2_CLAMP = 126.f;
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float exp2c(float x) {
+  return fast_exp2(fminf(fmaxf(x, -EXP2_CLAMP), EXP2_CLAMP));
+}
+// Byte offset of element (row r, column d) of a K-major SW128 tile whose
+// 64-column boxes are `box` bytes apart.
+__device__ __forceinline__ uint32_t kmaj_off(int r, int d, uint32_t box) {
+  return uint32_t(d >> 6) * box + sw128_off(r, (d & 63) >> 3) + uint32_t(d & 7) * 2u;
+}
+__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_shared_b32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+struct Ctx {
+  uint8_t* sm;
+  uint32_t sb;
+  uint32_t tmem;
+  int* status;
+  volatile int* abort_flag;
+  __device__ __forceinline__ uint32_t bar(uint32_t off) const { return sb + SM_BAR + off; }
+  __device__ __forceinline__ float* gates(int c) const {
+    return reinterpret_cast<float*>(sm + SM_GATES + (c % GATE_BUFS) * GATE_BYTES);
+  }
+  __device__ __forceinline__ volatile int* misc(uint32_t off) const {
+    return reinterpret_cast<volatile int*>(sm + SM_MISC + off);
+  }
+  __device__ __forceinline__ void fail() const {
+    *abort_flag = 1;
+    if (status) atomicExch(status, GDN_ERR_DEVICE_TIMEOUT);
+  }
+};
+
+// Role-wide agreement: the leader decides (after a bounded wait), every thread
+// of the role reads the verdict after the role's named barrier.  Called from
+// one site per agreement, so that the whole warp reaches the barrier together.
+struct RoleSync {
+  int bar_id, nthreads;
+  uint32_t flag_off;
+  bool leader;
+  int n;
+  __device__ __forceinline__ bool agree(const Ctx& x, bool leader_ok) {
+    volatile int* slot = x.misc(flag_off + 4u * (n & 1));
+    ++n;
+    if (leader) *slot = leader_ok ? 0 : 1;
+    named_bar(bar_id, nthreads);
+    const bool ok = (*slot == 0);
+    tc_fence_after();
+    return ok;
+  }
+  __device__ __forceinline__ bool wait(const Ctx& x, uint32_t bar, uint32_t parity) {
+    bool ok = true;
+    if (leader) {
+      ok = (*x.abort_flag == 0) && mbar_wait_bounded(bar, parity, WAIT_LIMIT_NS);
+      if (!ok) x.fail();
+    }
+    return agree(x, ok);
+  }
+};
+__device__ __forceinline__ bool lead_wait(const Ctx& x, uint32_t bar, uint32_t parity) {
+  if (*x.abort_flag) return false;
+  if (mbar_wait_bounded(bar, parity, WAIT_LIMIT_NS)) return true;
+  x.fail();
+  return false;
+}
+
+__device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
+                                         int c, int h, int b) {
+  const uint32_t bar = x.bar(B_KQFULL);
+  mbar_arrive_expect_tx(bar, KQ_TX_BYTES);
+  const int t0 = c * NT;
+  tma_load_4d(x.sb + SM_KQ + 0, tk, bar, 0, h, t0, b);
+  tma_load_4d(x.sb + SM_KQ + 4096, tq, bar, 0, h, t0, b);
+  tma_load_4d(x.sb + SM_KQ + 8192, tk, bar, 64, h, t0, b);
+  tma_load_4d(x.sb + SM_KQ + 12288, tq, bar, 64, h, t0, b);
+  *x.misc(M_KQ_ISSUED) = c + 1;
+}
+__device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b) {
+  const uint32_t bar = x.bar(B_VFULL);
+  mbar_arrive_expect_tx(bar, V_TX_BYTES);
+  tma_load_4d(x.sb + SM_V, tv, bar, 0, h, c * NT, b);
+  *x.misc(M_V_ISSUED) = c + 1;
+}
+
+// ============================================================== side role
+// Thread kt: channel pair cp = kt % 64 (channels 2cp, 2cp+1) and token quarter
+// qt = kt / 64 (tokens 8qt .. 8qt+7 of the tile) for the gates and operands;
+// TMEM lane quarter (warp % 4) and column half for the masks.
+__device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
+                          const KdaArgs& p, int b, int h, int ntiles) {
+  const int kt = threadIdx.x - 128;
+  const int warp = threadIdx.x >> 5;
+  const int lq = warp & 3;
+  const int hf = (warp >= 8) ? 1 : 0;
+  const bool leader = (kt == 0);
+  const uint32_t tlane = x.tmem + (uint32_t(lq * 32) << 16);
+  const uint32_t sb = x.sb;
+  const int cp = kt & 63, qt = kt >> 6;
+  const int d0 = 2 * cp;
+  float* sA = reinterpret_cast<float*>(x.sm + SM_A);
+  float* sT = reinterpret_cast<float*>(x.sm + SM_TF);
+  float* sX = reinterpret_cast<float*>(x.sm + SM_X);
+  RoleSync rs{BAR_SIDE, SIDE_THREADS, M_FLAG_SIDE, leader, 0};
+
+  for (int c = 0; c < ntiles; ++c) {
+    // ---- 1. gates: g of this thread's 8 tokens x 2 channels, cumulative sums
+    //      (log2 units) across the tile, beta, and Lambda_last per channel
+    float gm[8][2];
+    {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int tok = c * NT + 8 * qt + t;
+        float2 g2 = make_float2(0.f, 0.f);
+        if (tok < p.T) g2 = __ldg(reinterpret_cast<const float2*>(p.g + ((size_t(b) * p.T + tok) * p.H + h) * D + d0));
+        gm[t][0] = g2.x * LOG2E;
+        gm[t][1] = g2.y * LOG2E;
+      }
+#pragma unroll
+      for (int t = 1; t < 8; ++t) {
+        gm[t][0] += gm[t - 1][0];
+        gm[t][1] += gm[t - 1][1];
+      }
+      *reinterpret_cast<float2*>(sX + qt * 128 + d0) = make_float2(gm[7][0], gm[7][1]);
+      float* G = x.gates(c);
+      if (kt < NT) {
+        const int tok = c * NT + kt;
+        G[G_B / 4 + kt] = tok < p.T ? __ldg(p.beta + (size_t(b) * p.T + tok) * p.H + h) : 0.f;
+      }
+    }
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    float gref[2], glast[2];
+    {
+      float pre[2] = {0.f, 0.f}, tot[2] = {0.f, 0.f}, half[2] = {0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 s2 = *reinterpret_cast<const float2*>(sX + q * 128 + d0);
+        if (q < qt) { pre[0] += s2.x; pre[1] += s2.y; }
+        if (q < 2) { half[0] += s2.x; half[1] += s2.y; }
+        tot[0] += s2.x;
+        tot[1] += s2.y;
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        gm[t][0] += pre[0];
+        gm[t][1] += pre[1];
+      }
+      // reference: after token 15; last: after token 31
+      gref[0] = half[0]; gref[1] = half[1];
+      glast[0] = tot[0]; glast[1] = tot[1];
+      if (qt == 0) {
+        float* G = x.gates(c);
+        *reinterpret_cast<float2*>(G + G_LC / 4 + d0) = make_float2(exp2c(tot[0]), exp2c(tot[1]));
+      }
+    }
+    named_bar(BAR_SIDE, SIDE_THREADS);  // gates complete; the exchange area is free again
+    if (leader) mbar_arrive(x.bar(gfull_off(c)));
+
+    // ---- 2. the decayed operands of this thread's 8 tokens x 2 channels: the
+    //      P operands go to shared memory now; K+, Q+, K~ stay in registers
+    //      until the chain has released their tiles
+    float kp[8][2], qp[8][2], kt2[8][2];
+    {
+      if (!rs.wait(x, x.bar(B_KQFULL), c & 1)) return;
+      if (leader) *x.misc(M_KQ_SEEN) = c + 1;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int r = 8 * qt + t;
+        const uint32_t ko = SM_KQ + kmaj_off(r, d0, 8192u), qo = ko + 4096u;
+        const uint32_t kw = ld_shared_b32(sb + ko), qw = ld_shared_b32(sb + qo);
+        const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw));
+        const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw));
+        const float kv[2] = {kf.x, kf.y}, qv[2] = {qf.x, qf.y};
+        float k1[2], q1[2], k2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float ep = exp2c(gm[t][e] - gref[e]);   // Lambda_t / Lambda_r
+          const float em = exp2c(gref[e] - gm[t][e]);   // Lambda_r / Lambda_t
+          const float eplus = exp2c(gm[t][e]);          // Lambda_t (from the tile start)
+          const float etil = exp2c(glast[e] - gm[t][e]);  // Lambda_last / Lambda_t
+          k1[e] = kv[e] * ep;
+          q1[e] = qv[e] * ep;
+          k2[e] = kv[e] * em;
+          kp[t][e] = kv[e] * eplus;
+          qp[t][e] = qv[e] * eplus;
+          kt2[t][e] = kv[e] * etil;
+        }
+        uint32_t hi, lo;
+        split2_bf16(k1[0], k1[1], hi, lo);  // K' row r
+        st_shared_b32(sb + SM_PA + kmaj_off(r, d0, 8192u), hi);
+        st_shared_b32(sb + SM_PA + 16384u + kmaj_off(r, d0, 8192u), lo);
+        split2_bf16(q1[0], q1[1], hi, lo);  // Q' row 32 + r
+        st_shared_b32(sb + SM_PA + kmaj_off(32 + r, d0, 8192u), hi);
+        st_shared_b32(sb + SM_PA + 16384u + kmaj_off(32 + r, d0, 8192u), lo);
+        split2_bf16(k2[0], k2[1], hi, lo);  // K'' hi row r, lo row 32 + r
+        st_shared_b32(sb + SM_PB + kmaj_off(r, d0, 8192u), hi);
+        st_shared_b32(sb + SM_PB + kmaj_off(32 + r, d0, 8192u), lo);
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar(BAR_SIDE, SIDE_THREADS);  // the raw tile is read; the P operands are in place
+    // ---- 3. P = [K';Q'] [K'' hi | K'' lo]^T + [K';Q'] lo K'' hi^T  (M=128: rows 0..63 used)
+    {
+      bool ok = true;
+      if (leader) {
+        if (c + 1 < ntiles) issue_kq(x, tq, tk, c + 1, h, b);
+        tc_fence_after();
+        const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0), id32 = idesc_bf16(128, 32, 0, 0, 0);
+        const uint64_t da = sdesc_sw128(sb + SM_PA, 16, 1024), db = sdesc_sw128(sb + SM_PB, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+          mma_ss(x.tmem + TM_P, sdesc_add(da, off), sdesc_add(db, off), id64, kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+          mma_ss(x.tmem + TM_P, sdesc_add(da, 16384 + off), sdesc_add(db, off), id32, 1u);
+        }
+        mma_commit(x.bar(B_P));
+        ok = lead_wait(x, x.bar(B_P), c & 1);
+      }
+      if (!rs.agree(x, ok)) return;
+    }
+    // ---- 4. masks: rows 0..31 (K') -> A = strict_tril(beta_i P_ij) (fp32, for the
+    //      solve); rows 32..63 (Q') -> Mq = tril(P_ij) (registers); lanes 64..127 unused
+    float mq[16];
+    {
+      const float* G = x.gates(c);
+      if (lq < 2) {
+        float pa[16], pb[16];
+        tmem_ld16x2(tlane + TM_P + 16 * hf, pa, tlane + TM_P + 32 + 16 * hf, pb);
+        const int i = threadIdx.x & 31;
+        const float bi = (lq == 0) ? G[G_B / 4 + i] : 1.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int j = 16 * hf + e;
+          const float v = bi * (pa[e] + pb[e]);
+          mq[e] = (lq == 0 ? j < i : j <= i) ? v : 0.f;
+        }
+        if (lq == 0) {
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4)
+            *reinterpret_cast<float4*>(sA + i * APAD + 16 * hf + 4 * e4) =
+                make_float4(mq[4 * e4], mq[4 * e4 + 1], mq[4 * e4 + 2], mq[4 * e4 + 3]);
+        }
+      }
+    }
+    tc_fence_before();
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    // ---- 5. T = (I + A)^{-1}: 16 x 16 diagonal blocks by substitution, then
+    //      T_10 = -T_11 (A_10 T_00)
+    if (kt < NT) {
+      const int r = kt, bb = r >> 4, rr = r & 15, base = bb * 16;
+      float acc[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) acc[j] = (j == rr) ? 1.f : 0.f;
+#pragma unroll
+      for (int i = 15; i > 0; --i) {
+        const float xi = acc[i];
+        const float* arow = sA + (base + i) * APAD + base;
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+          if (4 * j4 < i) {
+            const float4 a = ld4(arow + 4 * j4);
+            if (4 * j4 + 0 < i) acc[4 * j4 + 0] = fmaf(-xi, a.x, acc[4 * j4 + 0]);
+            if (4 * j4 + 1 < i) acc[4 * j4 + 1] = fmaf(-xi, a.y, acc[4 * j4 + 1]);
+            if (4 * j4 + 2 < i) acc[4 * j4 + 2] = fmaf(-xi, a.z, acc[4 * j4 + 2]);
+            if (4 * j4 + 3 < i) acc[4 * j4 + 3] = fmaf(-xi, a.w, acc[4 * j4 + 3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if ((q4 >> 2) == bb)
+          v = make_float4(acc[4 * (q4 & 3)], acc[4 * (q4 & 3) + 1], acc[4 * (q4 & 3) + 2],
+                          acc[4 * (q4 & 3) + 3]);
+        *reinterpret_cast<float4*>(sT + r * APAD + 4 * q4) = v;
+      }
+    }
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    {
+      const int r = kt >> 4, cc = kt & 15;  // X[r][cc] = sum_k A[16 + r][k] T[k][cc]
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        a0 = fmaf(sA[(16 + r) * APAD + k], sT[k * APAD + cc], a0);
+        a1 = fmaf(sA[(16 + r) * APAD + k + 1], sT[(k + 1) * APAD + cc], a1);
+      }
+      sX[r * 16 + cc] = a0 + a1;
+    }
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    {
+      const int r = kt >> 4, cc = kt & 15;  // T[16 + r][cc] = -sum_k T[16 + r][16 + k] X[k][cc]
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < 16; k += 2) {
+        a0 = fmaf(sT[(16 + r) * APAD + 16 + k], sX[k * 16 + cc], a0);
+        a1 = fmaf(sT[(16 + r) * APAD + 17 + k], sX[(k + 1) * 16 + cc], a1);
+      }
+      sT[(16 + r) * APAD + cc] = -(a0 + a1);
+    }
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    // ---- 6. hand T and Mq to the chain once it is done with the previous tile's
+    //      (its output product, the last reader, has completed)
+    if (c > 0 && !rs.wait(x, x.bar(B_TMFREE), (c - 1) & 1)) return;
+    if (kt < 4 * NT) {  // T: row i = kt / 4, 8 columns each
+      const int i = kt >> 2, cc = kt & 3;
+      store_split8(sb + SM_TM, sb + SM_TM + 4096, i, cc, sT + i * APAD + 8 * cc);
+    }
+    if (lq == 1) {  // Mq row threadIdx % 32, columns 16 hf ..
+      const int i = threadIdx.x & 31;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) store_split8(sb + SM_MQ, sb + SM_MQ + 4096, i, 2 * hf + e, mq + 8 * e);
+    }
+    fence_proxy_async_smem();
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    if (leader) mbar_arrive(x.bar(B_TMFULL));
+    // ---- 7. the chain's operand tiles, once its state update of the previous
+    //      tile (the last reader of both) has completed: [K+;Q+] hi/lo and K~ hi/lo
+    if (c > 0 && !rs.wait(x, x.bar(B_OPFREE), (c - 1) & 1)) return;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int r = 8 * qt + t;
+      uint32_t hi, lo;
+      split2_bf16(kp[t][0], kp[t][1], hi, lo);
+      st_shared_b32(sb + SM_ZQB + kmaj_off(r, d0, 16384u), hi);
+      st_shared_b32(sb + SM_ZQB + kmaj_off(64 + r, d0, 16384u), lo);
+      split2_bf16(qp[t][0], qp[t][1], hi, lo);
+      st_shared_b32(sb + SM_ZQB + kmaj_off(32 + r, d0, 16384u), hi);
+      st_shared_b32(sb + SM_ZQB + kmaj_off(96 + r, d0, 16384u), lo);
+      split2_bf16(kt2[t][0], kt2[t][1], hi, lo);  // rows j, 64-column blocks 4 KB apart
+      st_shared_b32(sb + SM_KT + kmaj_off(r, d0, 4096u), hi);
+      st_shared_b32(sb + SM_KT + 8192u + kmaj_off(r, d0, 4096u), lo);
+    }
+    fence_proxy_async_smem();
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    if (leader) mbar_arrive(x.bar(B_OPFULL));
+  }
+}
+
+// ============================================================== chain role
+__device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMap* tmo,
+                           const KdaArgs& p, int chain, int b, int h, int ntiles) {
+  const int warp = threadIdx.x >> 5;
+  const int lq = warp & 3;
+  const int ch = (warp >= 12) ? 1 : 0;  // column half
+  const int dv = lq * 32 + (threadIdx.x & 31);
+  const bool leader = (threadIdx.x == 0);
+  const uint32_t tlane = x.tmem + (uint32_t(lq * 32) << 16);
+  const uint32_t sb = x.sb;
+  RoleSync rs{BAR_CHAIN, CHAIN_THREADS, M_FLAG_CHAIN, leader, 0};
+  const size_t cstate = size_t(chain) * D * D;
+
+  // ---- initial state (row dv of S0, or zeros): hi/lo copy, and the fp32 copy
+  //      pre-scaled, column by column, by the decay of the first tile
+  if (!rs.wait(x, x.bar(gfull_off(0)), gfull_parity(0))) return;
+  {
+    const float* LC = x.gates(0) + G_LC / 4;
+    const float4* src = p.S0 ? reinterpret_cast<const float4*>(p.S0 + cstate + size_t(dv) * D) : nullptr;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int col = 64 * ch + 32 * q;
+      float v[32];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float4 a = src ? __ldg(src + col / 4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[4 * e] = a.x; v[4 * e + 1] = a.y; v[4 * e + 2] = a.z; v[4 * e + 3] = a.w;
+      }
+      uint32_t hi[16], lo[16], u[32];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(LC[col + e] * v[e]);
+      tmem_st_state(tlane + TM_SHI + col / 2, hi, tlane + TM_SLO + col / 2, lo, tlane + TM_S + col, u);
+    }
+  }
+  tc_fence_before();
+  named_bar(BAR_CHAIN, CHAIN_THREADS);
+
+  for (int c = 0; c < ntiles; ++c) {
+    const float* G = x.gates(c);
+    const bool last = (c + 1 == ntiles);
+    const int n0 = 16 * ch;  // this thread's tokens of the tile
+    // ---- [Z|Y] = S_c [K+;Q+]^T: S hi x [hi rows; lo rows] (N=128), S lo x hi rows (N=64)
+    if (leader) {
+      if (lead_wait(x, x.bar(B_OPFULL), c & 1)) {
+        tc_fence_after();
+        const uint64_t db = sdesc_sw128(sb + SM_ZQB, 16, 1024);
+        const uint32_t id128 = idesc_bf16(128, 128, 0, 0, 0), id64 = idesc_bf16(128, 64, 0, 0, 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(x.tmem + TM_ZQ, x.tmem + TM_SHI + kk * 8,
+                 sdesc_add(db, (kk >> 2) * 16384 + (kk & 3) * 32), id128, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(x.tmem + TM_ZQ, x.tmem + TM_SLO + kk * 8,
+                 sdesc_add(db, (kk >> 2) * 16384 + (kk & 3) * 32), id64, 1u);
+        mma_commit(x.bar(B_ZQ));
+      }
+    }
+    // ---- X^T[dv][n] = beta_n (V[n][dv] - Z[dv][n]) (hi/lo -> shared memory)
+    {
+      bool ok = true;
+      if (leader) {
+        bulk_wait_read0();  // the previous tile's o store has read the staging tile
+        ok = lead_wait(x, x.bar(B_ZQ), c & 1) && lead_wait(x, x.bar(gfull_off(c)), gfull_parity(c)) &&
+             lead_wait(x, x.bar(B_VFULL), c & 1);
+        if (ok) *x.misc(M_V_SEEN) = c + 1;
+      }
+      if (!rs.agree(x, ok)) return;
+    }
+    {
+      float za[16], zb[16];
+      tmem_ld16x2(tlane + TM_ZQ + n0, za, tlane + TM_ZQ + 64 + n0, zb);
+      const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(x.sm + SM_V);
+      float xv[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int n = n0 + e;
+        xv[e] = G[G_B / 4 + n] * (__bfloat162float(V[n * D + dv]) - (za[e] + zb[e]));
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) store_split8(sb + SM_XH, sb + SM_XL, dv, 2 * ch + e, xv + 8 * e);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar(BAR_CHAIN, CHAIN_THREADS);
+    // ---- Dl^T = X^T T^T: X hi x [T hi; T lo] (N=64), X lo x T hi (N=32); K = 32
+    if (leader) {
+      if (!last) issue_v(x, tv, c + 1, h, b);  // V(c) has been read
+      if (lead_wait(x, x.bar(B_TMFULL), c & 1)) {
+        tc_fence_after();
+        const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0), id32 = idesc_bf16(128, 32, 0, 0, 0);
+        const uint64_t dt = sdesc_sw128(sb + SM_TM, 16, 1024);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          mma_ss(x.tmem + TM_DO, sdesc_sw128(sb + SM_XH + 32 * ks, 16, 1024), sdesc_add(dt, 32 * ks),
+                 id64, ks > 0);
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          mma_ss(x.tmem + TM_DO, sdesc_sw128(sb + SM_XL + 32 * ks, 16, 1024), sdesc_add(dt, 32 * ks),
+                 id32, 1u);
+        mma_commit(x.bar(B_DL));
+      }
+    }
+    if (!rs.wait(x, x.bar(B_DL), c & 1)) return;
+    {
+      float da[16], db2[16];
+      tmem_ld16x2(tlane + TM_DO + n0, da, tlane + TM_DO + 32 + n0, db2);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) da[e] += db2[e];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) store_split8(sb + SM_DH, sb + SM_DL, dv, 2 * ch + e, da + 8 * e);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar(BAR_CHAIN, CHAIN_THREADS);
+    // ---- S += Dl^T K~ (3 hi/lo products, N=128, B MN-major); then
+    //      O_intra = Dl^T Mq^T: Dl hi x [Mq hi; Mq lo] (N=64), Dl lo x Mq hi (N=32)
+    if (leader && !*x.abort_flag) {
+      tc_fence_after();
+      const uint32_t idu = idesc_bf16(128, 128, 0, 1, 0);
+#pragma unroll
+      for (int part = 0; part < 3; ++part) {
+        const uint32_t a = part == 2 ? SM_DL : SM_DH;
+        const uint32_t kb = part == 1 ? SM_KT + 8192 : SM_KT;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks)
+          mma_ss(x.tmem + TM_S, sdesc_sw128(sb + a + 32 * ks, 16, 1024),
+                 sdesc_sw128(sb + kb + 2048 * ks, 4096, 1024), idu, 1u);
+      }
+      mma_commit(x.bar(B_SU));
+      mma_commit(x.bar(B_OPFREE));  // [K+;Q+] (read by the first product) and K~ consumed
+      const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0), id32 = idesc_bf16(128, 32, 0, 0, 0);
+      const uint64_t dm = sdesc_sw128(sb + SM_MQ, 16, 1024);
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks)
+        mma_ss(x.tmem + TM_DO, sdesc_sw128(sb + SM_DH + 32 * ks, 16, 1024), sdesc_add(dm, 32 * ks), id64,
+               ks > 0);
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks)
+        mma_ss(x.tmem + TM_DO, sdesc_sw128(sb + SM_DL + 32 * ks, 16, 1024), sdesc_add(dm, 32 * ks), id32,
+               1u);
+      mma_commit(x.bar(B_OI));
+      mma_commit(x.bar(B_TMFREE));  // T and Mq consumed
+    }
+    // ---- o[t][dv] = Y[dv][t] + O_intra[dv][t] (both halves), staged fp32 in the
+    //      X^T hi region (free: the residual product has completed), one TMA store
+    if (!rs.wait(x, x.bar(B_OI), c & 1)) return;
+    {
+      float ya[16], yb[16], oa[16], ob[16];
+      tmem_ld16x2(tlane + TM_ZQ + 32 + n0, ya, tlane + TM_ZQ + 96 + n0, yb);
+      tmem_ld16x2(tlane + TM_DO + n0, oa, tlane + TM_DO + 32 + n0, ob);
+      float* so = reinterpret_cast<float*>(x.sm + SM_XH) + dv;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) so[(n0 + e) * D] = (ya[e] + yb[e]) + (oa[e] + ob[e]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_bar(BAR_CHAIN, CHAIN_THREADS);
+    if (leader) {
+      tma_store_4d(tmo, sb + SM_XH, 0, h, c * NT, b);
+      bulk_commit();
+    }
+    // ---- state epilogue: the update has completed (its commit preceded the
+    //      output product's); refresh hi/lo and pre-scale by the next tile's
+    //      decay per column, or store S_T
+    if (!rs.wait(x, x.bar(B_SU), c & 1)) return;
+    if (!last) {
+      if (!rs.wait(x, x.bar(gfull_off(c + 1)), gfull_parity(c + 1))) return;
+      const float* LC = x.gates(c + 1) + G_LC / 4;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int col = 64 * ch + 32 * q;
+        float v[32];
+        tmem_ld32(tlane + TM_S + col, v);
+        uint32_t hi[16], lo[16], u[32];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 l = ld4(LC + col + 4 * e4);
+          u[4 * e4 + 0] = __float_as_uint(l.x * v[4 * e4 + 0]);
+          u[4 * e4 + 1] = __float_as_uint(l.y * v[4 * e4 + 1]);
+          u[4 * e4 + 2] = __float_as_uint(l.z * v[4 * e4 + 2]);
+          u[4 * e4 + 3] = __float_as_uint(l.w * v[4 * e4 + 3]);
+        }
+        tmem_st_state(tlane + TM_SHI + col / 2, hi, tlane + TM_SLO + col / 2, lo, tlane + TM_S + col, u);
+      }
+      tc_fence_before();
+      named_bar(BAR_CHAIN, CHAIN_THREADS);
+    } else {
+      float4* dst = reinterpret_cast<float4*>(p.S_T + cstate + size_t(dv) * D + 64 * ch);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        float v[32];
+        tmem_ld32(tlane + TM_S + 64 * ch + 32 * q, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dst[8 * q + e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+      }
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    kda_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const KdaArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int chain = blockIdx.x;
+  const int b = chain / p.H, h = chain - (chain / p.H) * p.H;
+  const int ntiles = (p.T + NT - 1) / NT;
+
+  Ctx x;
+  x.sm = sm;
+  x.sb = smem_u32(sm);
+  x.status = p.status;
+  x.abort_flag = reinterpret_cast<volatile int*>(sm + SM_MISC + M_ABORT);
+  if (tid == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_o);
+    for (int i = 0; i < NUM_BARS; ++i) mbar_init(x.sb + SM_BAR + 8 * i, 1);
+    fence_mbar_init();
+    for (int i = 0; i < 16; ++i) reinterpret_cast<volatile int*>(sm + SM_MISC)[i] = 0;
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(sm + SM_MISC + M_TMEM), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  x.tmem = *reinterpret_cast<volatile uint32_t*>(sm + SM_MISC + M_TMEM);
+  if (tid == 0) {
+    issue_kq(x, &tm_q, &tm_k, 0, h, b);
+    issue_v(x, &tm_v, 0, h, b);
+  }
+  if (warp < 4 || warp >= 12)
+    chain_role(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
+  else
+    side_role(x, &tm_q, &tm_k, p, b, h, ntiles);
+
+  // each MMA-issuing thread waits (bounded) for its own products in flight
+  if (tid == 0 || tid == 128) {
+    const uint32_t bc = x.bar(tid == 0 ? B_CLEAN0 : B_CLEAN1);
+    mma_commit(bc);
+    mbar_wait_bounded(bc, 0, WAIT_LIMIT_NS / 4);
+  }
+  if (tid == 0) bulk_wait0();  // the o stores have completed
+  tc_fence_before();
+  __syncthreads();
+  // An aborted CTA may still have TMA loads in flight: wait for them (bounded)
+  // before the shared memory is released.
+  if (tid == 0 && *x.abort_flag) {
+    const int kq_issued = *x.misc(M_KQ_ISSUED), kq_seen = *x.misc(M_KQ_SEEN);
+    if (kq_issued > kq_seen) mbar_wait_bounded(x.bar(B_KQFULL), (kq_issued - 1) & 1, WAIT_LIMIT_NS / 4);
+    const int v_issued = *x.misc(M_V_ISSUED), v_seen = *x.misc(M_V_SEEN);
+    if (v_issued > v_seen) mbar_wait_bounded(x.bar(B_VFULL), (v_issued - 1) & 1, WAIT_LIMIT_NS / 4);
+  }
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(x.tmem, TMEM_COLS);
+}
+
+}  // namespace
+
+int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& to, const KdaArgs& a, cudaStream_t stream) {
+  const int chains = a.B * a.H;
+  if (chains == 0 || a.T == 0) return -1;
+  const uint32_t smem = SMEM_USED + 1024;
+  if (!ensure_smem_attr(reinterpret_cast<const void*>(kda_prefill_kernel), 15, int(smem))) return -1;
+  kda_prefill_kernel<<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, a);
+  return cudaGetLastError() == cudaSuccess ? 0 : -1;
+}
+
+}  // namespace gdn

@@ -277,7 +277,10 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
  * d2880479, lists among the cases its fused kernel left to the old path):
  *     S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
  *     o_t = S_t q_t
- * for t = 1..T of each of the B*H chains, in fp32, token by token.
+ * for t = 1..T of each of the B*H chains.  At Dk = Dv = 128 it runs chunked on
+ * the tensor cores (32-token chunks; every derived operand as a bf16 hi/lo
+ * pair; exact up to rounding while a key channel's decay over 16 tokens stays
+ * above e^-87, the fp32 range); other head dims run token by token in fp32.
  *   q, k [B][T][H][Dk] bf16; v [B][T][H][Dv] bf16 (device, 16-byte aligned)
  *   g    [B][T][H][Dk] fp32, natural-log decays (device, 16-byte aligned;
  *        g > 0 is accepted and grows the state)
@@ -287,16 +290,19 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
  *   o    [B][T][H][Dv] fp32, written (device); may not overlap any other array
  *   Dk, Dv each 64, 128 or 256.  B*H == 0 is a no-op; T == 0 copies S0 (or
  *   zeros) to S_T.
- * status is accepted for symmetry (no device-side waits; never written) and
+ * status: optional device int; the tensor-core path's bounded waits store
+ * GDN_ERR_DEVICE_TIMEOUT there if one gives up (the row kernel never writes it).
  * stream is a cudaStream_t.  Returns GDN_OK or a negative code; nothing is
  * launched on an error. */
 int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
                     const float* beta, const float* S0, float* o, float* S_T, int B, int T,
                     int H, int Dk, int Dv, int* status, void* stream);
 
-/* gdn_kda_prefill with the state updated in place: T tokens per sequence
- * starting from S and leaving S_T in S (T = 1: one decode step).  Arguments as
- * for gdn_kda_prefill with S0 = S_T = S. */
+/* The per-channel-gate recurrence with the state updated in place: T tokens
+ * per sequence starting from S and leaving S_T in S (T = 1: one decode step).
+ * Runs the row kernel at every head dim (a few tokens per call: the state is
+ * read and written once).  Arguments as for gdn_kda_prefill with
+ * S0 = S_T = S; status is never written. */
 int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                    int* status, void* stream);
