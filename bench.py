@@ -79,7 +79,6 @@ def decode_state_bytes(B, H):
 
 # per-channel gate (KDA): g is a vector of D fp32 per token-head
 KDA_TOKEN_HEAD_BYTES = 3 * D * 2 + D * 4 + 4 + D * 4   # q, k, v bf16 + g + beta + o = 1796 B
-KDA_OPS_PER_TOKEN_HEAD = 4 * D * D   # per state element: decay, two dot-product FMAs, update FMA
 FP32_LANES_PER_SM = 128
 SM_MAX_MHZ = 1965.0                   # clocks.max.sm of the B200
 
@@ -750,6 +749,7 @@ PROFILE_CASES = {
     # name: (workload, chunk, calls) -- untimed calls for ncu captures
     "decode": ("decode_b64_h16", None, 5),
     "prefill_b4_h32_t2048": (None, 64, 3),   # the large prefill's structure on 2048 tokens
+    "prefill_b4_h32_t8192": (None, 64, 3),   # the same on 8192 tokens (DRAM traffic, scaled by 4)
     "headline": ("prefill_b1_h16_t512", 64, 3),
     "kda_b1_h16_t512": (None, None, 3),       # per-channel gate, headline shape
     "kda_b4_h32_t2048": (None, None, 3),      # per-channel gate, a large batch
@@ -784,7 +784,8 @@ def run_profile_case(name):
             gdn.decode_step(d["q"][i], d["k"][i], d["v"][i], d["g"][i], d["beta"][i], S)
     else:
         if wname is None:
-            d = gin.prefill_inputs(4, 2048, 32, seed=0, g_mean=2.0, device=str(dev))
+            T = 8192 if name == "prefill_b4_h32_t8192" else 2048
+            d = gin.prefill_inputs(4, T, 32, seed=0, g_mean=2.0, device=str(dev))
         else:
             d = gin.workload_inputs(gin.WORKLOADS[wname], seed=0, device=str(dev))
         for _ in range(calls):
