@@ -50,10 +50,14 @@
 //   [  0,128) S   : state, scaled by the next chunk's total decay  (lane dv, col dk)
 //   [128,192) SHI : S hi as bf16 pairs (A operand)                 (lane dv, col dk/2)
 //   [192,256) SLO : S lo
-//   [256,320) Z   : S K^T, then Dl^T                               (lane dv, col token)
+//   [256,320) Z   : S K^T, then X^T as a bf16 hi/lo pair (the A operand of the
+//                   residual product), then Dl~^T as a hi/lo pair (the A
+//                   operand of the state update)              (lane dv, col token)
 //   [320,384) Y   : S Q^T                                          (lane dv, col token)
 //   [384,448) P   : [K;Q] K^T (lanes = rows of [K;Q]; K side only)
-//   [448,512) OI  : Dl^T Mq^T                                      (lane dv, col token)
+//   [448,512) OI  : Dl^T, then Dl^T Mq^T                           (lane dv, col token)
+// Reading the residual product's and the state update's A operands from tensor
+// memory halves their MMA issue cost against shared-memory operands.
 #include "gdn_internal.h"
 #include "sm100.cuh"
 
@@ -79,8 +83,8 @@ constexpr uint32_t SM_MQH = 81920;    // 8 KB: Mq rows i, K-major SW128 (64 x 64
 constexpr uint32_t SM_MQL = 90112;
 constexpr uint32_t SM_TH = 98304;     // 8 KB: T rows i (64 x 64)
 constexpr uint32_t SM_TL = 106496;
-constexpr uint32_t SM_XH = 114688;    // 16 KB: X^T rows dv (128 x 64), then the
-constexpr uint32_t SM_XL = 131072;    //        decay-scaled residuals
+constexpr uint32_t SM_XH = 114688;    // 32 KB staging: the fp32 o tile [64 tokens][128]
+constexpr uint32_t SM_XL = 131072;    //   (and, with the Dl^T tiles, the 64 KB end state)
 constexpr uint32_t SM_DH = 147456;    // 16 KB: Dl^T rows dv (128 x 64)
 constexpr uint32_t SM_DL = 163840;
 constexpr int APAD = 68;                      // row pitch (floats): conflict-free float4 rows
@@ -117,8 +121,16 @@ static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 // two barriers with parity waits could alias; four cannot (tile c + 4 needs
 // the chain to have finished tile c + 2).
 constexpr uint32_t B_FULL0 = 0, B_FULL1 = 8, B_VFULL = 16, B_PFULL = 24, B_TMFULL = 32,
-                   B_TMFREE = 40, B_ZQ = 48, B_DL = 56, B_OU = 64, B_GFULL = 72;
-constexpr int NUM_BARS = 13;
+                   B_TMFREE = 40, B_ZQ = 48, B_DL = 56, B_SU = 64, B_GFULL = 72, B_OI = 104,
+                   B_CLEAN0 = 112, B_CLEAN1 = 120, B_CLEAN2 = 128, B_CLEAN3 = 136;
+constexpr int NUM_BARS = 18;
+// MMA issuers: tcgen05.mma costs ~40-100 ns to issue from one thread, and
+// issuers in different warps proceed in parallel, so independent products are
+// issued by different threads: the chain leader (thread 0: [Z|Y], Dl, the
+// state update), a second chain thread (the output product) and, on the side,
+// a thread outside the solve's first phase ([K;Q] K^T).
+constexpr int OI_ISSUER = 384;   // warp 12, lane 0
+constexpr int P_ISSUER = 192;    // warp 6, lane 0 (side thread kt = 64)
 __device__ __forceinline__ uint32_t gfull_off(int c) { return B_GFULL + 8u * uint32_t(c & 3); }
 __device__ __forceinline__ uint32_t gfull_parity(int c) { return uint32_t(c >> 2) & 1u; }
 // misc slots (offsets inside SM_MISC)
@@ -145,6 +157,25 @@ __device__ __forceinline__ void store_state_split32(uint32_t tlane, int q, const
   tmem_st16x2(tlane + TM_SHI + 16 * q, hi, tlane + TM_SLO + 16 * q, lo);
 }
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+// N consecutive values of this thread's TMEM lane (a chunk's tokens) as bf16
+// hi/lo pairs: N/2 columns of hi at t_hi, N/2 of lo at t_lo (the layout an MMA
+// A operand read from tensor memory takes: lane = row, K packed 2 per column).
+template <int N>
+__device__ __forceinline__ void store_pairs_split(uint32_t t_hi, uint32_t t_lo, const float (&v)[N]) {
+  static_assert(N == 32 || N == 8, "a chunk half of 64 or 16 tokens");
+  if constexpr (N == 32) {
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
+    tmem_st16x2(t_hi, hi, t_lo, lo);
+  } else {
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
+    tmem_st4x2(t_hi, hi, t_lo, lo);
+  }
+}
 
 // Shared state of one CTA.
 struct Ctx {
@@ -506,11 +537,12 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
   side_gates<C, PRE>(x, kt, 0, T, g_next, b_next, p, b, h, s_part);
   if (!rs.wait(x, x.bar(B_FULL0), 0)) return;
-  if (leader) {
+  const bool p_iss = (threadIdx.x == P_ISSUER);
+  if (p_iss) {
     *x.misc(M_KQ_SEEN) = 1;
     issue_p<DK>(x, 0);
   }
-  int p_issued = 1;  // tiles whose P MMA was issued (leader's view)
+  int p_issued = 1;  // tiles whose P MMA was issued (the issuer's view)
   float mq[32];      // this thread's half row of Mq (lanes 64..127)
 
   for (int c = 0; c < ntiles; ++c) {
@@ -555,7 +587,7 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
     tc_fence_before();
     named_bar(BAR_SIDE, SIDE_THREADS);
     // P(c) has been read: start P(c+1) now if its tile has landed
-    if (leader && c + 1 < ntiles && p_issued == c + 1 &&
+    if (p_iss && c + 1 < ntiles && p_issued == c + 1 &&
         mbar_try_wait(x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1)) {
       tc_fence_after();
       *x.misc(M_KQ_SEEN) = c + 2;
@@ -640,7 +672,7 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
     // ---- P(c+1), if it could not be started early
     if (c + 1 < ntiles) {
       if (!rs.wait(x, x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1)) return;
-      if (leader && p_issued == c + 1) {
+      if (p_iss && p_issued == c + 1) {
         *x.misc(M_KQ_SEEN) = c + 2;
         issue_p<DK>(x, c + 1);
         p_issued = c + 2;
@@ -794,7 +826,9 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         if (!rs.agree(x, ok)) return;
       }
 
-      // ---- X^T[dv][n] = beta_n V[n][dv] - beta_n Gamma_n Z[dv][n]  (hi/lo -> SMEM)
+      // ---- X^T[dv][n] = beta_n V[n][dv] - beta_n Gamma_n Z[dv][n], as a hi/lo
+      //      pair into the chunk's Z columns once every thread has read its Z
+      //      (the A operand of the residual product, read from tensor memory)
       {
         const __nv_bfloat16* V = reinterpret_cast<const __nv_bfloat16*>(x.sm + SM_V);
         const int n0 = C * s + NC * ch;
@@ -825,15 +859,17 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
             xv[4 * e4 + e] = fmaf(bv[e], vn, -gv[e] * z[4 * e4 + e]);
           }
         }
-#pragma unroll
-        for (int e = 0; e < NC / 8; ++e) store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8 + e, xv + 8 * e);
+        named_bar(BAR_CHAIN, CHAIN_THREADS);  // every thread's Z columns have been read
+        store_pairs_split<NC>(tlane + TM_Z + C * s + NC * ch / 2, tlane + TM_Z + C * s + C / 2 + NC * ch / 2,
+                              xv);
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       named_bar(BAR_CHAIN, CHAIN_THREADS);
       if (leader && s == NSUB - 1 && !last_tile && !x.vzero) issue_v<DVB>(x, tv, c + 1, h, b);  // V(c) read
 
-      // ---- Dl^T = X^T T^T : M=128 (dv), N=C (i), K=C (n); 3 hi/lo products
+      // ---- Dl^T = X^T T^T : M=128 (dv), N=C (i), K=C (n); 3 hi/lo products, A (X)
+      //      from tensor memory, into the chunk's O_intra columns (free until its
+      //      output product)
       if (leader) {
         bool ok = true;
         if (s == 0) ok = mbar_wait_bounded(x.bar(B_TMFULL), c & 1, WAIT_LIMIT_NS);
@@ -845,30 +881,42 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           const uint32_t trow = uint32_t(C * s / 8) * 1024u;
 #pragma unroll
           for (int part = 0; part < 3; ++part) {
-            const uint32_t xa = part == 2 ? SM_XL : SM_XH;
+            const uint32_t xa = x.tmem + TM_Z + C * s + (part == 2 ? C / 2 : 0);
             const uint32_t tb = (part == 1 ? SM_TL : SM_TH) + trow;
 #pragma unroll
             for (int ks = 0; ks < C / 16; ++ks) {
               const uint32_t kb = uint32_t(16 * ks) * 2u;
-              mma_ss(x.tmem + TM_Z + C * s, sdesc_add(d0, xa + kb), sdesc_add(d0, tb + kb), id,
+              mma_ts(x.tmem + TM_OI + C * s, xa + 8 * ks, sdesc_add(d0, tb + kb), id,
                      (part | ks) ? 1u : 0u);
             }
           }
           mma_commit(x.bar(B_DL));
         }
       }
-      if (!rs.wait(x, x.bar(B_DL), sc & 1)) return;
+      {
+        // the previous chunk's output product (another issuer) must have read the
+        // Dl tiles before they are rewritten
+        bool ok = true;
+        if (leader) {
+          ok = (*x.abort_flag == 0) && mbar_wait_bounded(x.bar(B_DL), sc & 1, WAIT_LIMIT_NS);
+          if (ok && s > 0) ok = mbar_wait_bounded(x.bar(B_OI), (sc - 1) & 1, WAIT_LIMIT_NS);
+          if (!ok) x.fail();
+        }
+        if (!rs.agree(x, ok)) return;
+      }
 
-      // ---- residuals: Dl (for the output) and Dl * exp(gamma_last - gamma) (for the state)
+      // ---- residuals: Dl (for the output product: hi/lo into shared memory) and
+      //      Dl~ = Dl * exp(gamma_last - gamma) (for the state update: hi/lo into the
+      //      chunk's Z columns, whose X has been consumed)
       {
         const int n0 = C * s + NC * ch;
         float d[NC];
         if constexpr (NC == 32) {
-          tmem_ld32(tlane + TM_Z + n0, d);
+          tmem_ld32(tlane + TM_OI + n0, d);
         } else {
           float da[4], db[4];
-          tmem_ld4(tlane + TM_Z + n0, da);
-          tmem_ld4(tlane + TM_Z + n0 + 4, db);
+          tmem_ld4(tlane + TM_OI + n0, da);
+          tmem_ld4(tlane + TM_OI + n0 + 4, db);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             d[e] = da[e];
@@ -885,17 +933,32 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           dt[4 * e4 + 3] = d[4 * e4 + 3] * f.w;
         }
 #pragma unroll
-        for (int e = 0; e < NC / 8; ++e) {
-          store_split8(sb + SM_DH, sb + SM_DL, dv, n0 / 8 + e, d + 8 * e);
-          store_split8(sb + SM_XH, sb + SM_XL, dv, n0 / 8 + e, dt + 8 * e);
-        }
+        for (int e = 0; e < NC / 8; ++e) store_split8(sb + SM_DH, sb + SM_DL, dv, n0 / 8 + e, d + 8 * e);
+        store_pairs_split<NC>(tlane + TM_Z + C * s + NC * ch / 2, tlane + TM_Z + C * s + C / 2 + NC * ch / 2,
+                              dt);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar(BAR_CHAIN, CHAIN_THREADS);
 
-      // ---- O_intra = Dl^T Mq^T (N=C) and S += Dl~^T K (N=128, B = K tile MN-major)
+      // ---- S += Dl~^T K (N = Dk, B = K tile MN-major; the chain leader) and
+      //      O_intra = Dl^T Mq^T (N = C; a second issuer), committed separately:
+      //      the state epilogue waits for the update only
       if (leader && !*x.abort_flag) {
+        tc_fence_after();
+        const uint32_t idu = idesc_bf16(128, DK, 0, 1, 0);
+        const uint64_t dk = sdesc_sw128(kq + uint32_t(C * s) * 128u, 16384, 1024);  // K rows, MN-major
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          const uint32_t da = x.tmem + TM_Z + C * s + (part ? C / 2 : 0);  // Dl~ hi / lo (TMEM)
+#pragma unroll
+          for (int ks = 0; ks < C / 16; ++ks) {
+            mma_ts(x.tmem + TM_S, da + 8 * ks, sdesc_add(dk, uint32_t(16 * ks) * 128u), idu, 1u);
+          }
+        }
+        mma_commit(x.bar(B_SU));
+      }
+      if (threadIdx.x == OI_ISSUER && !*x.abort_flag) {
         tc_fence_after();
         const uint32_t id = idesc_bf16(128, C, 0, 0, 0);
         const uint64_t d0 = sdesc_sw128(sb + uint32_t(C * s) * 2u, 16, 1024);  // chunk's K offset
@@ -911,26 +974,17 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
                    (part | ks) ? 1u : 0u);
           }
         }
-        const uint32_t idu = idesc_bf16(128, DK, 0, 1, 0);
-        const uint64_t dk = sdesc_sw128(kq + uint32_t(C * s) * 128u, 16384, 1024);  // K rows, MN-major
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          const uint32_t da = part ? SM_XL : SM_XH;
-#pragma unroll
-          for (int ks = 0; ks < C / 16; ++ks) {
-            mma_ss(x.tmem + TM_S, sdesc_add(d0, da + uint32_t(16 * ks) * 2u),
-                   sdesc_add(dk, uint32_t(16 * ks) * 128u), idu, 1u);
-          }
-        }
-        mma_commit(x.bar(B_OU));
-        if (s == NSUB - 1) mma_commit(x.bar(B_TMFREE));  // T(c), Mq(c) consumed
+        mma_commit(x.bar(B_OI));
+        if (s == NSUB - 1) mma_commit(x.bar(B_TMFREE));  // T(c), Mq(c) consumed (Dl(c) waited)
       }
-      if (!rs.wait(x, x.bar(B_OU), sc & 1)) return;
+      if (!rs.wait(x, x.bar(B_SU), sc & 1)) return;
       if (leader && s == NSUB - 1 && c + 2 < ntiles) issue_kq<DK>(x, tq, tk, c + 2, h, b);  // KQ(c) read
 
-      // ---- o of the whole tile is complete after its last chunk: o[t][dv] =
-      //      Gamma_t Y[dv][t] + O_intra[dv][t], this thread's 32 tokens to HBM
-      if (s == NSUB - 1) output_drain<OBF, DVB>(x, tlane, b, h, dv, ch, c, leader);
+      // ---- the last tile: o first (its staging area then holds the end state)
+      if (last_tile && s == NSUB - 1) {
+        if (!rs.wait(x, x.bar(B_OI), sc & 1)) return;
+        output_drain<OBF, DVB>(x, tlane, b, h, dv, ch, c, leader);
+      }
 
       // ---- S_out now sits in TMEM: refresh its hi/lo copy, and pre-scale it by
       //      the next chunk's decay (or store it as S_T after the last chunk)
@@ -1015,6 +1069,14 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
                           tlane + TM_S + col, u);
           }
         }
+      }
+      // ---- o of the whole tile is complete after its last chunk's output
+      //      product: o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t], to HBM (before
+      //      the next tile's [Z|Y] product rewrites Y)
+      if (s == NSUB - 1 && !last_tile) {
+        tc_fence_before();
+        if (!rs.wait(x, x.bar(B_OI), sc & 1)) return;
+        output_drain<OBF, DVB>(x, tlane, b, h, dv, ch, c, leader);
       }
       tc_fence_before();
       if (!rs.check(x)) return;
@@ -1146,6 +1208,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   else
     kside_role<C, PRE, DK, DVB>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
 
+  // every MMA issuer waits (bounded) for its own products in flight
+  if (tid == 0 || tid == 128 || tid == OI_ISSUER || tid == P_ISSUER) {
+    const uint32_t bc = x.bar(tid == 0 ? B_CLEAN0 : tid == 128 ? B_CLEAN1 : tid == OI_ISSUER ? B_CLEAN2 : B_CLEAN3);
+    mma_commit(bc);
+    mbar_wait_bounded(bc, 0, WAIT_LIMIT_NS / 4);
+  }
   if (tid == 0) bulk_wait0();  // the chain leader's o stores have completed
   tc_fence_before();
   __syncthreads();

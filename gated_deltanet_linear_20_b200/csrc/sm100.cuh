@@ -283,6 +283,16 @@ __device__ __forceinline__ void tmem_st16x2(uint32_t ta, const uint32_t (&a)[16]
       "r"(b[14]), "r"(b[15])
       : "memory");
 }
+// Two 4-column stores (e.g. hi and lo halves), one wait.
+__device__ __forceinline__ void tmem_st4x2(uint32_t ta, const uint32_t (&a)[4], uint32_t tb,
+                                           const uint32_t (&b)[4]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%2,%3,%4,%5};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x4.b32 [%1], {%6,%7,%8,%9};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(ta), "r"(tb),
+      "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3])
+      : "memory");
+}
 // Store of 16 columns, waited on inside the same statement (the source
 // registers are free for reuse when it returns).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&u)[16]) {

@@ -144,10 +144,14 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 
-// Issue-rate probe: one thread issues n_mma tcgen05.mma (kind::f16, M = 128,
-// N = 32/64/128/256 by mode & 3, A from shared memory or, with mode >= 4, from
-// tensor memory) on zeroed operands and records, per CTA, the wall time of the
-// issue loop and the time until the products have completed (ns).
+// Issue-rate probe: tcgen05.mma (kind::f16, M = 128, N = 32/64/128/256 by
+// mode & 3) on zeroed operands; records, per CTA, the wall time of the issue
+// loop and the time until the products have completed (ns).
+//   mode & 4 : A from tensor memory (else shared memory)
+//   mode & 8 : consecutive MMAs rotate over 4 accumulators (N <= 128, A from
+//              shared memory) instead of all accumulating into one
+//   mode & 16: two threads (warps 0 and 1) each issue half of the MMAs, into
+//              accumulators 256 columns apart (N <= 128, A from shared memory)
 __global__ void __launch_bounds__(128, 1) umma_issue_kernel(int mode, int n_mma,
                                                              unsigned long long* out, int* status) {
   extern __shared__ uint8_t raw[];
@@ -160,6 +164,7 @@ __global__ void __launch_bounds__(128, 1) umma_issue_kernel(int mode, int n_mma,
   fence_proxy_async_smem();
   if (tid == 0) {
     mbar_init(bar, 1);
+    mbar_init(bar + 8, 1);  // the second issuer's completion
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -170,26 +175,34 @@ __global__ void __launch_bounds__(128, 1) umma_issue_kernel(int mode, int n_mma,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
-  if (tid == 0) {
+  const bool two = (mode & 16) != 0;
+  if (tid == 0 || (two && tid == 32)) {
     // A: 128 rows x 128 B at sb (K-major); B: up to 256 rows x 128 B at sb + 32 KB;
-    // D: TMEM columns 0 .. N-1; A from TMEM: columns 256 .. 319
+    // D: TMEM columns from 0 (rotating: 0, 128, 256, 384; second issuer: 256 ..);
+    // A from TMEM: columns 256 .. 319
     const uint64_t a = sdesc_sw128(sb, 16, 1024), b = sdesc_sw128(sb + 32768, 16, 1024);
     const int N = (mode & 3) == 0 ? 64 : (mode & 3) == 1 ? 128 : (mode & 3) == 2 ? 256 : 32;
     const uint32_t id = idesc_bf16(128, N, 0, 0, 0);
+    const uint32_t dbase = tmem + (tid == 32 ? 256u : 0u);
+    const int n = two ? n_mma / 2 : n_mma;
     const unsigned long long t0 = globaltimer_ns();
-    for (int i = 0; i < n_mma; ++i) {
+    for (int i = 0; i < n; ++i) {
       const uint32_t kk = i & 3;
-      if (mode >= 4)
-        mma_ts(tmem, tmem + 256 + kk * 8, sdesc_add(b, kk * 32), id, 1u);
+      if (mode & 4)
+        mma_ts(dbase, tmem + 256 + kk * 8, sdesc_add(b, kk * 32), id, 1u);
+      else if (mode & 8)
+        mma_ss(dbase + 128u * (i & 3), sdesc_add(a, kk * 32), sdesc_add(b, kk * 32), id, 1u);
       else
-        mma_ss(tmem, sdesc_add(a, kk * 32), sdesc_add(b, kk * 32), id, 1u);
+        mma_ss(dbase, sdesc_add(a, kk * 32), sdesc_add(b, kk * 32), id, 1u);
     }
     const unsigned long long t1 = globaltimer_ns();
-    mma_commit(bar);
-    if (!mbar_wait_bounded(bar, 0, 1000000000ull)) atomicExch(status, -7);
+    mma_commit(bar + (tid == 32 ? 8u : 0u));
+    if (!mbar_wait_bounded(bar + (tid == 32 ? 8u : 0u), 0, 1000000000ull)) atomicExch(status, -7);
     const unsigned long long t2 = globaltimer_ns();
-    out[2 * blockIdx.x] = t1 - t0;
-    out[2 * blockIdx.x + 1] = t2 - t0;
+    if (tid == 0) {
+      out[2 * blockIdx.x] = t1 - t0;
+      out[2 * blockIdx.x + 1] = t2 - t0;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -213,7 +226,8 @@ extern "C" int umma_selftest(const void* A, const void* B, float* D, int mode, i
 extern "C" int umma_issue_probe(int mode, int n_mma, int ctas, unsigned long long* out, int* status,
                                 void* stream) {
   const int smem = 65536 + 1024 + 64;
-  if (mode < 0 || mode > 7 || n_mma < 1 || ctas < 1 ||
+  if (mode < 0 || mode > 31 || ((mode & 24) && ((mode & 4) || (mode & 3) == 2)) || n_mma < 2 ||
+      ctas < 1 ||
       cudaFuncSetAttribute(umma_issue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
           cudaSuccess)
     return -1;

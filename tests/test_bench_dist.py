@@ -69,4 +69,7 @@ def test_algorithmic_work_figures():
     # per-channel gate: g is a vector of 128 fp32 per token-head
     assert bench.KDA_TOKEN_HEAD_BYTES == 3 * 256 + 512 + 4 + 512
     assert bench.kda_prefill_bytes(1, 512, 16, False) == 512 * 16 * 1796 + 16 * 65536
-    assert bench.KDA_OPS_PER_TOKEN_HEAD == 4 * 128 * 128
+    # general head dims reduce to the 128 x 128 figures
+    assert bench.prefill_bytes_dims(1, 512, 16, 128, 128, False) == bench.prefill_bytes(1, 512, 16, False)
+    assert bench.prefill_flops_dims(1, 1, 1, 128, 128) == bench.prefill_flops(1, 1, 1)
+    assert bench.prefill_bytes_dims(1, 1, 1, 64, 256, False) == 2 * 64 * 2 + 256 * 2 + 8 + 256 * 4 + 64 * 256 * 4

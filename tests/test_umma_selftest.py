@@ -75,10 +75,11 @@ def test_umma_forms(mode):
 
 @pytest.mark.gpu
 def test_mma_issue_rate():
-    """Issue cost of tcgen05.mma from one thread (printed with -s): the kernel
-    design counts MMA instructions, not only FLOPs, so this records how long a
-    run of 128 MMAs of M = 128 and N = 32..256 takes to issue and to complete,
-    on one CTA and on one CTA per SM.  Checks only that every run completes."""
+    """Issue cost of tcgen05.mma (printed with -s): the kernel design counts MMA
+    instructions, not only FLOPs, so this records how long a run of 128 MMAs of
+    M = 128 and N = 32..256 takes to issue and to complete, on one CTA and on
+    one CTA per SM; with one accumulator, with four rotating accumulators, and
+    split between two issuing warps.  Checks only that every run completes."""
     lib = ctypes.CDLL(build_selftest())
     lib.umma_issue_probe.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 3
     lib.umma_issue_probe.restype = ctypes.c_int
@@ -87,7 +88,8 @@ def test_mma_issue_rate():
     out = torch.zeros(2 * sms, dtype=torch.int64, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     n = 128
-    for mode in range(8):
+    modes = list(range(8)) + [8, 9, 11, 16, 17, 19]  # + rotating accumulators, two issuers
+    for mode in modes:
         N = [64, 128, 256, 32][mode & 3]
         for ctas in (1, sms):
             for _ in range(2):  # the second run is the one recorded
@@ -98,6 +100,7 @@ def test_mma_issue_rate():
             assert int(status.item()) == 0
             t = out.view(sms, 2)[:ctas].double().cpu().mean(0)
             tflops = 128 * N * 16 * 2 * n / (t[1].item() * 1e-9) / 1e12
-            print(f"A from {'TMEM' if mode >= 4 else 'SMEM'} N={N:3d} CTAs={ctas:3d}: "
+            kind = "two issuers" if mode & 16 else "4 accumulators" if mode & 8 else "one accumulator"
+            print(f"A from {'TMEM' if mode & 4 else 'SMEM'}, {kind}, N={N:3d} CTAs={ctas:3d}: "
                   f"issue {t[0].item() / n:.1f} ns/MMA, complete {t[1].item() / n:.1f} ns/MMA, "
                   f"{tflops:.2f} TFLOP/s per SM")
