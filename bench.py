@@ -247,6 +247,18 @@ def time_steps(fn, steps, warmup, flush, stream):
     return [s.elapsed_time(e) for s, e in evs]
 
 
+def copy_reference_us(state_bytes, dev, flush, stream, steps=32):
+    """A device-to-device copy of `state_bytes` (the state's read + write
+    traffic, without the kernel's arithmetic), timed with the same protocol as
+    the decode step it sits beside: the memory-system limit for that many
+    bytes after an L2 flush, fixed costs included."""
+    src = torch.empty(state_bytes // 4, dtype=torch.float32, device=dev)
+    dst = torch.empty_like(src)
+    t = statistics.mean(time_steps(lambda: dst.copy_(src), steps, 5, flush, stream))
+    del src, dst
+    return t * 1e3
+
+
 # ------------------------------------------------------------------ our arm
 def e2e_pipelined(call_part, host, dev_in, outs_dev, outs_host, nparts, steps, warmup, stream):
     """End-to-end steps through the public API with the copies overlapped.
@@ -498,6 +510,7 @@ def run_extras(args, dev, stream, flush, peaks, rank):
     torch.cuda.synchronize()
     t_warm = e0.elapsed_time(e1) / wd.decode_steps
     traffic = committed_traffic("decode_b64_h16", DECODE_SOURCES)
+    copy_us = copy_reference_us(wd.B * wd.H * STATE_BYTES, dev, flush, stream)
     out["decode_b64_h16"] = {
         "state_GB_per_s": round(gbs, 1), "us_per_step": round(t * 1e3, 3),
         "roofline": {"bound": "hbm", "achieved": round(decode_bytes(wd.B, wd.H) / (t / 1e3) / 1e9, 1),
@@ -505,6 +518,8 @@ def run_extras(args, dev, stream, flush, peaks, rank):
                      "frac": round(decode_bytes(wd.B, wd.H) / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                      "traffic": traffic},
         "l2": "flushed before every step",
+        "same_bytes_copy_us": round(copy_us, 3),
+        "frac_of_copy": round(copy_us / (t * 1e3), 4),
         "back_to_back_256_steps": {"us_per_step": round(t_warm * 1e3, 3),
                                    "state_GB_per_s": round(sb / (t_warm / 1e3) / 1e9, 1),
                                    "l2": "warm: the 64 MiB state fits in the 126 MB L2"}}
@@ -563,7 +578,8 @@ def run_head_dim_extras(dev, stream, flush, peaks, rank, steps):
     """Scalar gate at head dims other than 128 x 128: the 16-head, 512-token
     prefill (Dk = 64 or 128: the chunked tensor-core kernel; Dk = 256: the
     row-parallel fp32 kernel), a 4 x 32-head, 4096-token prefill at 128 x 256,
-    and the batched decode step (row kernel)."""
+    and the batched decode step (64 x 64: the streaming decode kernel; 256 x 256:
+    the row kernel)."""
     from gated_deltanet_linear_20_b200 import gdn
     out = {}
     peak_ops = alu_peak_tops(dev)
@@ -614,10 +630,14 @@ def run_head_dim_extras(dev, stream, flush, peaks, rank, steps):
         nb = B * H * (2 * dk * dv * 4 + 2 * dk * 2 + dv * 2 + 8 + dv * 4)
         out[f"decode_b64_h16_dk{dk}_dv{dv}"] = {
             "us_per_step": round(t * 1e3, 3), "state_MiB": B * H * dk * dv * 4 / 2**20,
+            "kernel": "streaming decode" if dk == 64 else "row-parallel fp32",
             "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
             "l2": "flushed before every step"}
+        copy_us = copy_reference_us(B * H * dk * dv * 4, dev, flush, stream)
+        out[f"decode_b64_h16_dk{dk}_dv{dv}"].update(
+            same_bytes_copy_us=round(copy_us, 3), frac_of_copy=round(copy_us / (t * 1e3), 4))
         del d, S, o, tok
     torch.cuda.empty_cache()
     return out
@@ -628,7 +648,8 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
     tensor-core kernel (32-token chunks; HBM roofline, with the tensor fraction
     of the same chunk-GEMM FLOP count as the scalar gate beside it), at the
     512-token single-sequence shape and a large batch; and the batched decode
-    step on the row kernel (HBM roofline)."""
+    step at 128 x 128 and 64 x 64 on the streaming decode kernel (HBM
+    roofline)."""
     from gated_deltanet_linear_20_b200 import gdn
     out = {}
     for (B, T, H, g_mean, n) in ((1, 512, 16, 0.0, steps), (4, 8192, 32, 2.0, 3)):
@@ -652,27 +673,33 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
         del d, o, sT
     # decode: one token for 64 x 16 heads, state in place, L2 flushed per step
     B, H = 64, 16
-    d = gin.kda_inputs(B, 8, H, seed=6000 + rank, s0_std=0.02, device=str(dev))
-    S = d["S0"].clone()
-    tok = [{key: d[key][:, i].contiguous() for key in ("q", "k", "v", "g", "beta")}
-           for i in range(8)]
-    o = torch.empty((B, H, D), dtype=torch.float32, device=dev)
-    it = [0]
+    for Dh in (D, 64):
+        d = gin.kda_inputs(B, 8, H, Dh, Dh, seed=6000 + rank, s0_std=0.02, device=str(dev))
+        S = d["S0"].clone()
+        tok = [{key: d[key][:, i].contiguous() for key in ("q", "k", "v", "g", "beta")}
+               for i in range(8)]
+        o = torch.empty((B, H, Dh), dtype=torch.float32, device=dev)
+        it = [0]
 
-    def kstep():
-        x = tok[it[0] % 8]
-        gdn.kda_decode(x["q"], x["k"], x["v"], x["g"], x["beta"], S, o=o)
-        it[0] += 1
-    ms = time_steps(kstep, 32, 5, flush, stream)
-    t = statistics.mean(ms)
-    nb = B * H * (2 * STATE_BYTES + KDA_TOKEN_HEAD_BYTES)
-    out["kda_decode_b64_h16"] = {
-        "us_per_step": round(t * 1e3, 3),
-        "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
-        "l2": "flushed before every step"}
-    del d, S, o
+        def kstep():
+            x = tok[it[0] % 8]
+            gdn.kda_decode(x["q"], x["k"], x["v"], x["g"], x["beta"], S, o=o)
+            it[0] += 1
+        ms = time_steps(kstep, 32, 5, flush, stream)
+        t = statistics.mean(ms)
+        # state read + written; q, k, v bf16; g fp32 per key channel; beta; o fp32
+        nb = B * H * (2 * Dh * Dh * 4 + 3 * Dh * 2 + Dh * 4 + 4 + Dh * 4)
+        key = "kda_decode_b64_h16" + ("" if Dh == D else f"_dk{Dh}_dv{Dh}")
+        out[key] = {
+            "us_per_step": round(t * 1e3, 3), "kernel": "streaming decode",
+            "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)},
+            "l2": "flushed before every step"}
+        copy_us = copy_reference_us(B * H * Dh * Dh * 4, dev, flush, stream)
+        out[key].update(same_bytes_copy_us=round(copy_us, 3),
+                        frac_of_copy=round(copy_us / (t * 1e3), 4))
+        del d, S, o, tok
     torch.cuda.empty_cache()
     return out
 

@@ -213,6 +213,37 @@ int rows_impl(const void* q, const void* k, const void* v, const float* g, const
              : GDN_ERR_LAUNCH;
 }
 
+// The streaming decode kernel (Dk = Dv = DH, 128 or 64), the state updated in
+// place.  vector_gate: g is [B][T][H][DH], else [B][T][H].  o_align: the
+// alignment the entry point documents for o.
+int decode_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                float* S, float* o, int B, int T, int H, int DH, int qk_norm, float q_scale,
+                int o_bf16, bool vector_gate, size_t o_align, void* stream) {
+  const long long heads = (long long)B * H;
+  if (heads * DH * DH > 0x7fffffffLL || heads * T * DH > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  if (heads == 0 || T == 0) return GDN_OK;
+  if (!q || !k || !v || !g || !beta || !S || !o) return GDN_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(S, 16) ||
+      !aligned(o, o_align) || !aligned(g, vector_gate ? 16 : 4) || !aligned(beta, 4))
+    return GDN_ERR_ALIGN;
+  const size_t toks = size_t(heads) * T;
+  const size_t vec_bf16 = toks * DH * 2, o_bytes = toks * DH * (o_bf16 ? 2 : 4);
+  const size_t state_bytes = size_t(heads) * DH * DH * 4;
+  const size_t g_bytes = toks * (vector_gate ? DH : 1) * 4, beta_bytes = toks * 4;
+  const void* ins[5] = {q, k, v, g, beta};
+  const size_t in_bytes[5] = {vec_bf16, vec_bf16, vec_bf16, g_bytes, beta_bytes};
+  for (int i = 0; i < 5; ++i)
+    if (overlaps(o, o_bytes, ins[i], in_bytes[i]) || overlaps(S, state_bytes, ins[i], in_bytes[i]))
+      return GDN_ERR_ALIAS;
+  if (overlaps(o, o_bytes, S, state_bytes)) return GDN_ERR_ALIAS;
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+  gdn::DecodeArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H, T, qk_norm, q_scale,
+                    o_bf16, vector_gate ? 1 : 0, DH};
+  return gdn::launch_decode(a, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
+}
+
 int prefill_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
                  const float* S0, float* o, float* S_T, int B, int T, int H, int Dk, int Dv,
                  int chunk, void* ws, size_t ws_bytes, bool allow_segments, int* status,
@@ -514,36 +545,17 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
   if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
   if (B < 0 || H < 0 || T < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim) {
-    // other head dims: the row kernel with the state in place (no fused options)
+    // other head dims: no fused options; 64 x 64 streams through the decode
+    // kernel, the rest through the row kernel, the state in place
     if (!gdn::rows_head_dims_ok(Dk, Dv) || qk_norm || q_scale != 1.f || o_bf16)
       return GDN_ERR_UNSUPPORTED;
     if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
+    if (Dk == 64 && Dv == 64)
+      return decode_impl(q, k, v, g, beta, S, o, B, T, H, 64, 0, 1.f, 0, false, 4, stream);
     return rows_impl(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, false, stream);
   }
-  const long long heads = (long long)B * H;
-  if (heads * kHeadDim * kHeadDim > 0x7fffffffLL || heads * T * kHeadDim > 0x7fffffffLL)
-    return GDN_ERR_SHAPE;
-  if (heads == 0 || T == 0) return GDN_OK;
-  if (!q || !k || !v || !g || !beta || !S || !o) return GDN_ERR_NULL;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(S, 16) ||
-      !aligned(o, 16) || !aligned(g, 4) || !aligned(beta, 4))
-    return GDN_ERR_ALIGN;
-  const size_t toks = size_t(heads) * T;
-  const size_t vec_bf16 = toks * kHeadDim * 2, vec_f32 = toks * kHeadDim * (o_bf16 ? 2 : 4);  // o bytes
-  const size_t state_bytes = size_t(heads) * kHeadDim * kHeadDim * 4, gate_bytes = toks * 4;
-  if (overlaps(o, vec_f32, q, vec_bf16) || overlaps(o, vec_f32, k, vec_bf16) ||
-      overlaps(o, vec_f32, v, vec_bf16) || overlaps(o, vec_f32, g, gate_bytes) ||
-      overlaps(o, vec_f32, beta, gate_bytes) || overlaps(o, vec_f32, S, state_bytes) ||
-      overlaps(S, state_bytes, q, vec_bf16) || overlaps(S, state_bytes, k, vec_bf16) ||
-      overlaps(S, state_bytes, v, vec_bf16) || overlaps(S, state_bytes, g, gate_bytes) ||
-      overlaps(S, state_bytes, beta, gate_bytes))
-    return GDN_ERR_ALIAS;
-  const int dev_ok = check_device();
-  if (dev_ok != GDN_OK) return dev_ok;
-  gdn::DecodeArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                    static_cast<const __nv_bfloat16*>(v), g, beta, S, o, B, H, T, qk_norm, q_scale,
-                    o_bf16};
-  return gdn::launch_decode(a, static_cast<cudaStream_t>(stream)) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
+  return decode_impl(q, k, v, g, beta, S, o, B, T, H, kHeadDim, qk_norm, q_scale, o_bf16, false,
+                     16, stream);
 }
 
 int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
@@ -591,10 +603,13 @@ int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
 int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                    int* status, void* stream) {
-  (void)status;  // the row kernel has no device-side waits
+  (void)status;  // the decode kernels have no device-side waits
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
-  // a few tokens per call: the row kernel streams the state once
+  // Dk = Dv = 128 or 64: the streaming decode kernel; other head dims: the row
+  // kernel (both read and write the state once per call)
+  if (Dk == Dv && (Dk == kHeadDim || Dk == 64))
+    return decode_impl(q, k, v, g, beta, S, o, B, T, H, Dk, 0, 1.f, 0, true, 4, stream);
   return rows_impl(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, true, stream);
 }
 

@@ -64,6 +64,8 @@ struct DecodeArgs {
   int qk_norm;    // as in PrefillArgs
   float q_scale;
   int o_bf16;     // o is bf16 (same layout)
+  int vector_gate;  // g is [B][T][H][Dk], one log decay per key channel (no fused options)
+  int head_dim;     // Dk = Dv: 128, or 64 (no fused options)
 };
 
 // Row-parallel fp32 kernel (any supported head dims; scalar or per-channel gate).

@@ -241,8 +241,8 @@ int gdn_prefill_static_ws(const void* q, const void* k, const void* v, const flo
  *   q, k [B][H][Dk] bf16; v [B][H][Dv] bf16; g, beta [B][H] fp32 (device)
  *   S    [B][H][Dv][Dk] fp32, updated in place (device)
  *   o    [B][H][Dv] fp32, written (device)
- *   Dk, Dv each 64, 128 or 256 (other than 128 x 128: the row-parallel kernel);
- *   B*H == 0 is a no-op.
+ *   Dk, Dv each 64, 128 or 256 (128 x 128 and 64 x 64: the streaming decode
+ *   kernel; other pairs: the row-parallel kernel); B*H == 0 is a no-op.
  * status and stream as for gdn_prefill.  Returns GDN_OK or a negative code. */
 int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
                     const float* beta, float* S, float* o, int B, int H, int Dk, int Dv,
@@ -258,8 +258,9 @@ int gdn_decode_step(const void* q, const void* k, const void* v, const float* g,
  *   q, k [B][T][H][Dk] bf16; v [B][T][H][Dv] bf16; g, beta [B][T][H] fp32 (device)
  *   S    [B][H][Dv][Dk] fp32, updated in place (device)
  *   o    [B][T][H][Dv] fp32, written (device)
- *   Dk, Dv each 64, 128 or 256 (other than 128 x 128: the row-parallel kernel);
- *   B*H == 0 or T == 0 is a no-op.
+ *   Dk, Dv each 64, 128 or 256 (128 x 128 and 64 x 64: the streaming decode
+ *   kernels; other pairs: the row-parallel kernel); B*H == 0 or T == 0 is a
+ *   no-op.
  * status and stream as for gdn_prefill.  Returns GDN_OK or a negative code. */
 int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
@@ -300,9 +301,11 @@ int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
 
 /* The per-channel-gate recurrence with the state updated in place: T tokens
  * per sequence starting from S and leaving S_T in S (T = 1: one decode step).
- * Runs the row kernel at every head dim (a few tokens per call: the state is
- * read and written once).  Arguments as for gdn_kda_prefill with
- * S0 = S_T = S; status is never written. */
+ * At 128 x 128 and 64 x 64 it runs the streaming decode kernel (the decay
+ * applied per key column of each state row in registers); other head dims run
+ * the row kernel.  Either reads and writes the state once per call.  Arguments
+ * as for gdn_kda_prefill with S0 = S_T = S, except that o needs only 4-byte
+ * alignment; status is never written. */
 int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                    int* status, void* stream);

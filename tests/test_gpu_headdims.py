@@ -2,8 +2,10 @@
 combination, Dk != Dv included), through the same C entry points, against the
 fp64 oracles (which take any Dk, Dv).  Prefill with Dk = 64 or 128 runs the
 chunked tensor-core kernel (Dv = 256: two CTAs per chain, 128 state rows each;
-Dv = 64: one CTA with its upper 64 rows held at zero); Dk = 256, decode and
-the per-channel gate run the row-parallel fp32 kernel.  The contract and the
+Dv = 64: one CTA with its upper 64 rows held at zero); decode at 64 x 64 runs
+the streaming decode kernel (two 256-byte rows per warp-wide load); Dk = 256,
+the other decode dims and the per-channel-gate prefill run the row-parallel
+fp32 kernel.  The contract and the
 1e-4 design margin are those of the other tests.
 """
 from __future__ import annotations
@@ -69,6 +71,29 @@ def test_decode_other_head_dims(dk, dv):
     o = torch.cat([torch.stack(outs, 1), o3], 1).cpu().numpy()
     assert_parity(o, ro, f"o decode {dk}x{dv}")
     assert_parity(S.cpu().numpy(), rS, f"S decode {dk}x{dv}")
+
+
+def test_decode_64_b64_h16_steps():
+    """The 64 x 64 decode at 64 x 16 heads: 6 single-token steps and a 3-token
+    burst on every head, the state in place, against the oracle; then the same
+    inputs again give the same bits."""
+    d = inputs.prefill_inputs(64, 9, 16, 64, 64, seed=64, s0_std=0.02)
+    dd = to_dev(d)
+    gdn = _gdn()
+    step = lambda sl: [dd[key][:, sl].contiguous() for key in ("q", "k", "v", "g", "beta")]
+
+    def run():
+        S = dd["S0"].clone()
+        outs = [gdn.decode_step(*step(t), S).unsqueeze(1) for t in range(6)]
+        outs.append(gdn.decode_tokens(*step(slice(6, 9)), S))
+        torch.cuda.synchronize()
+        return torch.cat(outs, 1), S
+    o, S = run()
+    ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, "o decode 64x64 B64 H16")
+    assert_parity(S.cpu().numpy(), rS, "S decode 64x64 B64 H16")
+    o2, S2 = run()
+    assert torch.equal(o, o2) and torch.equal(S, S2), "not bitwise run-to-run"
 
 
 @pytest.mark.parametrize("dk,dv", [(64, 64), (256, 256), (128, 64), (64, 256)], ids=lambda x: str(x))

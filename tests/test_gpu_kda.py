@@ -2,9 +2,10 @@
 the fp64 KDA oracle on the same seeded inputs.
 
 Prefill at Dk = Dv = 128 runs the chunked tensor-core kernel (32-token
-chunks, every derived operand as a bf16 hi/lo pair); decode and the other head
-dims run the row kernel, which walks the tokens in fp32 in the order of the
-recurrence.  The same contract as the scalar-gate path applies (relative
+chunks, every derived operand as a bf16 hi/lo pair); decode at Dk = Dv = 128
+or 64 runs the streaming decode kernel (the per-column decay applied to each
+state row in registers); the other head dims run the row kernel, which walks
+the tokens in fp32 in the order of the recurrence.  The same contract as the scalar-gate path applies (relative
 Frobenius <= 2e-3, max-abs <= 1e-2 x RMS on o and S_T), and the tighter 1e-4
 design margin is asserted too.
 """
@@ -95,6 +96,46 @@ def test_kda_decode_b64_h16_steps():
     o = torch.cat([torch.stack(outs, 1), o4], 1).cpu().numpy()
     assert_parity(o, ro, "o decode")
     assert_parity(S.cpu().numpy(), rS, "S decode")
+
+
+@pytest.mark.parametrize("D", [128, 64])
+@pytest.mark.parametrize("g_mean,label", [(-3.0, "strong"), (4.0, "weak"), (None, "growing")])
+def test_kda_decode_decay_strengths(D, g_mean, label):
+    """Decode at 128 x 128 and 64 x 64 with per-channel decays of several
+    strengths (and positive log decays, which grow the state): 3 single-token
+    steps, a 2-token and a 5-token burst, against the oracle over the 10
+    tokens."""
+    d = inputs.kda_inputs(8, 10, 5, D, D, seed=40 + D, s0_std=0.05,
+                          g_mean=g_mean if g_mean is not None else -3.0)
+    if g_mean is None:
+        d["g"] = (d["g"].abs() * 0.05).contiguous()
+    dd = to_dev(d)
+    gdn = _gdn()
+    S = dd["S0"].clone()
+    step = lambda sl: [dd[key][:, sl].contiguous() for key in ("q", "k", "v", "g", "beta")]
+    outs = [gdn.kda_decode(*step(t), S).unsqueeze(1) for t in range(3)]
+    outs.append(gdn.kda_decode(*step(slice(3, 5)), S))
+    outs.append(gdn.kda_decode(*step(slice(5, 10)), S))
+    torch.cuda.synchronize()
+    ro, rS = oracle.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(torch.cat(outs, 1).cpu().numpy(), ro, f"o kda decode {D} {label}")
+    assert_parity(S.cpu().numpy(), rS, f"S kda decode {D} {label}")
+
+
+def test_kda_decode_64_b64_h16_steps():
+    """The 64 x 64 decode at 64 x 16 heads: 6 single-token steps and a 2-token
+    burst on every head, against the oracle."""
+    d = inputs.kda_inputs(64, 8, 16, 64, 64, seed=17, s0_std=0.02)
+    dd = to_dev(d)
+    gdn = _gdn()
+    S = dd["S0"].clone()
+    step = lambda sl: [dd[key][:, sl].contiguous() for key in ("q", "k", "v", "g", "beta")]
+    outs = [gdn.kda_decode(*step(t), S).unsqueeze(1) for t in range(6)]
+    outs.append(gdn.kda_decode(*step(slice(6, 8)), S))
+    torch.cuda.synchronize()
+    ro, rS = oracle.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(torch.cat(outs, 1).cpu().numpy(), ro, "o kda decode 64x64")
+    assert_parity(S.cpu().numpy(), rS, "S kda decode 64x64")
 
 
 def test_kda_in_place_zero_length_and_determinism():
