@@ -777,7 +777,7 @@ PROFILE_CASES = {
     "decode": ("decode_b64_h16", None, 5),
     "prefill_b4_h32_t2048": (None, 64, 3),   # the large prefill's structure on 2048 tokens
     "prefill_b4_h32_t8192": (None, 64, 3),   # the same on 8192 tokens (DRAM traffic, scaled by 4)
-    "headline": ("prefill_b1_h16_t512", 64, 3),
+    "prefill_b1_h16_t512": ("prefill_b1_h16_t512", 64, 3),
     "kda_b1_h16_t512": (None, None, 3),       # per-channel gate, headline shape
     "kda_b4_h32_t2048": (None, None, 3),      # per-channel gate, a large batch
     "kda_decode": (None, None, 5),            # per-channel gate, B64 H16 one token

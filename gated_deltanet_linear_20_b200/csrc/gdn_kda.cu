@@ -42,6 +42,11 @@
 //   [256,384) ZQ  : [Z | Y] of S hi x [K+;Q+] hi, then [Z | Y] of S hi x lo    (32 cols each)
 //   [384,448) P   : [K';Q'] x [K'' hi | K'' lo]   (lanes 0..63 used)
 //   [448,512) DO  : [Dl | Dl'] of X x [T hi | T lo], then [O | O'] of Dl x [Mq hi | Mq lo]
+// Once a thread has read its Z columns, the same 16 columns take its tokens'
+// X^T as a bf16 hi/lo pair (8 + 8 columns: the A operand of Dl = X T^T, read
+// from tensor memory), and once Dl is in, its tokens' Dl^T likewise (the A
+// operand of the state update and of the output product).  An MMA reads A from
+// tensor memory at about a third of the issue cost of a shared-memory A.
 #include "gdn_internal.h"
 #include "sm100.cuh"
 
@@ -57,6 +62,12 @@ constexpr int CHAIN_THREADS = 256, SIDE_THREADS = 256;
 constexpr int BAR_CHAIN = 1, BAR_SIDE = 2;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TM_S = 0, TM_SHI = 128, TM_SLO = 192, TM_ZQ = 256, TM_P = 384, TM_DO = 448;
+// X^T, then Dl^T, as hi/lo pairs in the Z columns: chain thread half ch (tokens
+// 16 ch .. 16 ch + 15) at TM_X + 16 ch (hi) and TM_X + 16 ch + 8 (lo)
+constexpr uint32_t TM_X = TM_ZQ;
+// The output product is issued by a second chain thread (warp 12), in parallel
+// with the state update from the chain leader.
+constexpr int OI_ISSUER = 384;
 
 // Shared memory (offsets from a 1024-byte aligned base).  K-major SW128 tiles
 // have 128-byte rows (64 bf16 along K) in 8-row groups 1024 B apart.
@@ -66,10 +77,7 @@ constexpr uint32_t SM_ZQB = 24576;     // [K+ hi; Q+ hi; K+ lo; Q+ lo] 128 rows,
 constexpr uint32_t SM_PA = 57344;      // [K'; Q'] hi (64 rows, boxes 8 KB apart), then lo at +16 KB
 constexpr uint32_t SM_PB = 90112;      // [K'' hi; K'' lo] 64 rows, boxes 8 KB apart
 constexpr uint32_t SM_KT = 106496;     // K~ = K o Lambda_last / Lambda, rows j, MN-major: hi (2 x 4 KB), lo at +8 KB
-constexpr uint32_t SM_XH = 122880;     // X^T hi rows dv (K = 32 tokens in the first 64 B of a row);
-constexpr uint32_t SM_XL = 139264;     //   X^T hi doubles as the fp32 [32][128] o staging tile
-constexpr uint32_t SM_DH = 155648;     // Dl^T hi / lo, rows dv
-constexpr uint32_t SM_DL = 172032;
+constexpr uint32_t SM_XH = 122880;     // the fp32 [32][128] o staging tile (16 KB)
 constexpr uint32_t SM_TM = 188416;     // [T hi; T lo] rows i (32 + 32), K = 32 tokens
 constexpr uint32_t SM_MQ = 196608;     // [Mq hi; Mq lo]
 constexpr int APAD = 36;               // solve row pitch (floats)
@@ -85,7 +93,7 @@ constexpr uint32_t SM_BAR = SM_GATES + GATE_BUFS * GATE_BYTES;
 constexpr uint32_t SM_MISC = SM_BAR + 256;
 constexpr uint32_t SMEM_USED = SM_MISC + 256;
 static_assert(SM_ZQB % 1024 == 0 && SM_PA % 1024 == 0 && SM_PB % 1024 == 0 && SM_KT % 1024 == 0 &&
-                  SM_XH % 1024 == 0 && SM_DH % 1024 == 0 && SM_TM % 1024 == 0 && SM_MQ % 1024 == 0,
+                  SM_XH % 1024 == 0 && SM_TM % 1024 == 0 && SM_MQ % 1024 == 0,
               "SW128 tiles need 1024-byte alignment");
 // the M = 128 reads of the [K';Q'] tiles run 8 KB past each 64-row box: they
 // must stay inside this CTA's shared memory (the rows read there are unused)
@@ -95,8 +103,9 @@ static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 // mbarriers (8 bytes each, offsets inside SM_BAR)
 constexpr uint32_t B_KQFULL = 0, B_VFULL = 8, B_P = 16, B_TMFULL = 24, B_TMFREE = 32,
                    B_OPFULL = 40, B_OPFREE = 48, B_ZQ = 56, B_DL = 64, B_SU = 72, B_OI = 80,
-                   B_CLEAN0 = 88, B_CLEAN1 = 96, B_GFULL = 104;  // B_GFULL: 4 barriers
-constexpr int NUM_BARS = 17;
+                   B_CLEAN0 = 88, B_CLEAN1 = 96, B_CLEAN2 = 104,
+                   B_GFULL = 112;  // B_GFULL: 4 barriers
+constexpr int NUM_BARS = 18;
 static_assert(8 * NUM_BARS <= 256, "barrier slots");
 __device__ __forceinline__ uint32_t gfull_off(int c) { return B_GFULL + 8u * uint32_t(c & 3); }
 __device__ __forceinline__ uint32_t gfull_parity(int c) { return uint32_t(c >> 2) & 1u; }
@@ -110,6 +119,17 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float EXP2_CLAMP = 126.f;
 
 __device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+// Two 8-column tensor-memory stores (a hi / lo pair), one wait.
+__device__ __forceinline__ void tmem_st8x2(uint32_t ta, const uint32_t (&a)[8], uint32_t tb,
+                                           const uint32_t (&b)[8]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%2,%3,%4,%5,%6,%7,%8,%9};\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%1], {%10,%11,%12,%13,%14,%15,%16,%17};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(ta), "r"(tb),
+      "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]),
+      "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3]), "r"(b[4]), "r"(b[5]), "r"(b[6]), "r"(b[7])
+      : "memory");
+}
 __device__ __forceinline__ float exp2c(float x) {
   return fast_exp2(fminf(fmaxf(x, -EXP2_CLAMP), EXP2_CLAMP));
 }
@@ -514,7 +534,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
         mma_commit(x.bar(B_ZQ));
       }
     }
-    // ---- X^T[dv][n] = beta_n (V[n][dv] - Z[dv][n]) (hi/lo -> shared memory)
+    // ---- X^T[dv][n] = beta_n (V[n][dv] - Z[dv][n]) (hi/lo -> this thread's Z columns)
     {
       bool ok = true;
       if (leader) {
@@ -535,13 +555,15 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
         const int n = n0 + e;
         xv[e] = G[G_B / 4 + n] * (__bfloat162float(V[n * D + dv]) - (za[e] + zb[e]));
       }
+      uint32_t xh[8], xl[8];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) store_split8(sb + SM_XH, sb + SM_XL, dv, 2 * ch + e, xv + 8 * e);
+      for (int e = 0; e < 8; ++e) split2_bf16(xv[2 * e], xv[2 * e + 1], xh[e], xl[e]);
+      tmem_st8x2(tlane + TM_X + 16 * ch, xh, tlane + TM_X + 16 * ch + 8, xl);
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     named_bar(BAR_CHAIN, CHAIN_THREADS);
-    // ---- Dl^T = X^T T^T: X hi x [T hi; T lo] (N=64), X lo x T hi (N=32); K = 32
+    // ---- Dl^T = X^T T^T: X hi x [T hi; T lo] (N=64), X lo x T hi (N=32); K = 32,
+    //      A from tensor memory (K step ks = the tokens of chain half ks)
     if (leader) {
       if (!last) issue_v(x, tv, c + 1, h, b);  // V(c) has been read
       if (lead_wait(x, x.bar(B_TMFULL), c & 1)) {
@@ -550,12 +572,10 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
         const uint64_t dt = sdesc_sw128(sb + SM_TM, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
-          mma_ss(x.tmem + TM_DO, sdesc_sw128(sb + SM_XH + 32 * ks, 16, 1024), sdesc_add(dt, 32 * ks),
-                 id64, ks > 0);
+          mma_ts(x.tmem + TM_DO, x.tmem + TM_X + 16 * ks, sdesc_add(dt, 32 * ks), id64, ks > 0);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
-          mma_ss(x.tmem + TM_DO, sdesc_sw128(sb + SM_XL + 32 * ks, 16, 1024), sdesc_add(dt, 32 * ks),
-                 id32, 1u);
+          mma_ts(x.tmem + TM_DO, x.tmem + TM_X + 16 * ks + 8, sdesc_add(dt, 32 * ks), id32, 1u);
         mma_commit(x.bar(B_DL));
       }
     }
@@ -565,43 +585,47 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
       tmem_ld16x2(tlane + TM_DO + n0, da, tlane + TM_DO + 32 + n0, db2);
 #pragma unroll
       for (int e = 0; e < 16; ++e) da[e] += db2[e];
+      // X^T has been consumed (Dl is complete): Dl^T takes its columns
+      uint32_t dh[8], dl[8];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) store_split8(sb + SM_DH, sb + SM_DL, dv, 2 * ch + e, da + 8 * e);
+      for (int e = 0; e < 8; ++e) split2_bf16(da[2 * e], da[2 * e + 1], dh[e], dl[e]);
+      tmem_st8x2(tlane + TM_X + 16 * ch, dh, tlane + TM_X + 16 * ch + 8, dl);
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     named_bar(BAR_CHAIN, CHAIN_THREADS);
-    // ---- S += Dl^T K~ (3 hi/lo products, N=128, B MN-major); then
-    //      O_intra = Dl^T Mq^T: Dl hi x [Mq hi; Mq lo] (N=64), Dl lo x Mq hi (N=32)
+    // ---- S += Dl^T K~ (3 hi/lo products, N=128, B MN-major; the chain leader)
+    //      and O_intra = Dl^T Mq^T: Dl hi x [Mq hi; Mq lo] (N=64), Dl lo x Mq hi
+    //      (N=32; a second issuer), A from tensor memory, committed separately
     if (leader && !*x.abort_flag) {
       tc_fence_after();
       const uint32_t idu = idesc_bf16(128, 128, 0, 1, 0);
 #pragma unroll
       for (int part = 0; part < 3; ++part) {
-        const uint32_t a = part == 2 ? SM_DL : SM_DH;
+        const uint32_t a = x.tmem + TM_X + (part == 2 ? 8 : 0);
         const uint32_t kb = part == 1 ? SM_KT + 8192 : SM_KT;
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
-          mma_ss(x.tmem + TM_S, sdesc_sw128(sb + a + 32 * ks, 16, 1024),
-                 sdesc_sw128(sb + kb + 2048 * ks, 4096, 1024), idu, 1u);
+          mma_ts(x.tmem + TM_S, a + 16 * ks, sdesc_sw128(sb + kb + 2048 * ks, 4096, 1024), idu, 1u);
       }
       mma_commit(x.bar(B_SU));
       mma_commit(x.bar(B_OPFREE));  // [K+;Q+] (read by the first product) and K~ consumed
+    }
+    if (threadIdx.x == OI_ISSUER && !*x.abort_flag) {
+      tc_fence_after();
       const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0), id32 = idesc_bf16(128, 32, 0, 0, 0);
       const uint64_t dm = sdesc_sw128(sb + SM_MQ, 16, 1024);
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks)
-        mma_ss(x.tmem + TM_DO, sdesc_sw128(sb + SM_DH + 32 * ks, 16, 1024), sdesc_add(dm, 32 * ks), id64,
-               ks > 0);
+        mma_ts(x.tmem + TM_DO, x.tmem + TM_X + 16 * ks, sdesc_add(dm, 32 * ks), id64, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < 2; ++ks)
-        mma_ss(x.tmem + TM_DO, sdesc_sw128(sb + SM_DL + 32 * ks, 16, 1024), sdesc_add(dm, 32 * ks), id32,
-               1u);
+        mma_ts(x.tmem + TM_DO, x.tmem + TM_X + 16 * ks + 8, sdesc_add(dm, 32 * ks), id32, 1u);
       mma_commit(x.bar(B_OI));
-      mma_commit(x.bar(B_TMFREE));  // T and Mq consumed
+      mma_commit(x.bar(B_TMFREE));  // T and Mq consumed (T by Dl, which has completed)
     }
-    // ---- o[t][dv] = Y[dv][t] + O_intra[dv][t] (both halves), staged fp32 in the
-    //      X^T hi region (free: the residual product has completed), one TMA store
+    // ---- o[t][dv] = Y[dv][t] + O_intra[dv][t] (both halves), staged fp32 in
+    //      shared memory (the previous tile's store has read it: the leader
+    //      waited before this tile's X agreement), one TMA store
     if (!rs.wait(x, x.bar(B_OI), c & 1)) return;
     {
       float ya[16], yb[16], oa[16], ob[16];
@@ -703,8 +727,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     side_role(x, &tm_q, &tm_k, p, b, h, ntiles);
 
   // each MMA-issuing thread waits (bounded) for its own products in flight
-  if (tid == 0 || tid == 128) {
-    const uint32_t bc = x.bar(tid == 0 ? B_CLEAN0 : B_CLEAN1);
+  if (tid == 0 || tid == 128 || tid == OI_ISSUER) {
+    const uint32_t bc = x.bar(tid == 0 ? B_CLEAN0 : (tid == 128 ? B_CLEAN1 : B_CLEAN2));
     mma_commit(bc);
     mbar_wait_bounded(bc, 0, WAIT_LIMIT_NS / 4);
   }
