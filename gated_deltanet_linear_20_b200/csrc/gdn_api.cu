@@ -587,15 +587,16 @@ int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
     return GDN_ERR_ALIAS;
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
-  CUtensorMap tq{}, tk{}, tv{}, to{};
+  CUtensorMap tq{}, tk{}, tv{}, to{}, tg{};
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  if (!encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
+  if (!encode_act(&tg, g, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, kHeadDim, 32) ||
+      !encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
       !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
       !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, kHeadDim, 32) ||
       !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, kHeadDim, 32))
     return GDN_ERR_LAUNCH;
   gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status};
-  return gdn::launch_kda_prefill(tq, tk, tv, to, a, static_cast<cudaStream_t>(stream)) == 0
+  return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK
              : GDN_ERR_LAUNCH;
 }

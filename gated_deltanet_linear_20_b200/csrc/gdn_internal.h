@@ -104,7 +104,8 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
 // tq, tk: bf16 q, k boxes of 64 features x 32 tokens (SW128); tv: bf16 v, tv:
 // 128 x 32 unswizzled; to: fp32 o, 128 x 32.  T > 0 and B*H > 0.
 int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& to, const KdaArgs& a, cudaStream_t stream);
+                       const CUtensorMap& to, const CUtensorMap& tg, const KdaArgs& a,
+                       cudaStream_t stream);
 int launch_decode(const DecodeArgs& a, cudaStream_t stream);
 // Second pass of the segmented schedule (a.nseg > 1).
 int launch_segment_fix(const PrefillArgs& a, cudaStream_t stream);

@@ -74,10 +74,12 @@ constexpr int OI_ISSUER = 384;
 constexpr uint32_t SM_KQ = 0;          // raw [K dk0-63 | Q dk0-63 | K dk64-127 | Q dk64-127], 4 KB boxes
 constexpr uint32_t SM_V = 16384;       // raw V [32 tokens][128] bf16
 constexpr uint32_t SM_ZQB = 24576;     // [K+ hi; Q+ hi; K+ lo; Q+ lo] 128 rows, boxes dk0-63 / dk64-127 16 KB apart
-constexpr uint32_t SM_PA = 57344;      // [K'; Q'] hi (64 rows, boxes 8 KB apart), then lo at +16 KB
+constexpr uint32_t SM_PA = 57344;      // [K' hi; Q' hi; K' lo; Q' lo] 128 rows, boxes 16 KB apart
 constexpr uint32_t SM_PB = 90112;      // [K'' hi; K'' lo] 64 rows, boxes 8 KB apart
 constexpr uint32_t SM_KT = 106496;     // K~ = K o Lambda_last / Lambda, rows j, MN-major: hi (2 x 4 KB), lo at +8 KB
 constexpr uint32_t SM_XH = 122880;     // the fp32 [32][128] o staging tile (16 KB)
+constexpr uint32_t SM_G0 = 139264;     // g tiles [32 tokens][128] fp32, two buffers (tile c in c & 1)
+constexpr uint32_t SM_G1 = 155648;
 constexpr uint32_t SM_TM = 188416;     // [T hi; T lo] rows i (32 + 32), K = 32 tokens
 constexpr uint32_t SM_MQ = 196608;     // [Mq hi; Mq lo]
 constexpr int APAD = 36;               // solve row pitch (floats)
@@ -93,27 +95,28 @@ constexpr uint32_t SM_BAR = SM_GATES + GATE_BUFS * GATE_BYTES;
 constexpr uint32_t SM_MISC = SM_BAR + 256;
 constexpr uint32_t SMEM_USED = SM_MISC + 256;
 static_assert(SM_ZQB % 1024 == 0 && SM_PA % 1024 == 0 && SM_PB % 1024 == 0 && SM_KT % 1024 == 0 &&
-                  SM_XH % 1024 == 0 && SM_TM % 1024 == 0 && SM_MQ % 1024 == 0,
+                  SM_XH % 1024 == 0 && SM_TM % 1024 == 0 && SM_MQ % 1024 == 0 && SM_G0 % 1024 == 0 &&
+                  SM_G1 % 1024 == 0,
               "SW128 tiles need 1024-byte alignment");
-// the M = 128 reads of the [K';Q'] tiles run 8 KB past each 64-row box: they
-// must stay inside this CTA's shared memory (the rows read there are unused)
-static_assert(SM_PA + 32768 + 8192 <= SM_KT, "P operand over-read stays in the operand region");
+static_assert(SM_PA + 32768 <= SM_PB && SM_G1 + 16384 <= SM_TM, "operand regions");
 static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 
 // mbarriers (8 bytes each, offsets inside SM_BAR)
 constexpr uint32_t B_KQFULL = 0, B_VFULL = 8, B_P = 16, B_TMFULL = 24, B_TMFREE = 32,
                    B_OPFULL = 40, B_OPFREE = 48, B_ZQ = 56, B_DL = 64, B_SU = 72, B_OI = 80,
-                   B_CLEAN0 = 88, B_CLEAN1 = 96, B_CLEAN2 = 104,
-                   B_GFULL = 112;  // B_GFULL: 4 barriers
-constexpr int NUM_BARS = 18;
+                   B_CLEAN0 = 88, B_CLEAN1 = 96, B_CLEAN2 = 104, B_GLD = 112,  // B_GLD: 2 barriers
+                   B_GFULL = 128;  // B_GFULL: 4 barriers
+constexpr int NUM_BARS = 20;
 static_assert(8 * NUM_BARS <= 256, "barrier slots");
 __device__ __forceinline__ uint32_t gfull_off(int c) { return B_GFULL + 8u * uint32_t(c & 3); }
 __device__ __forceinline__ uint32_t gfull_parity(int c) { return uint32_t(c >> 2) & 1u; }
 constexpr uint32_t M_TMEM = 0, M_ABORT = 4, M_KQ_ISSUED = 12, M_KQ_SEEN = 16, M_V_ISSUED = 20,
-                   M_V_SEEN = 24, M_FLAG_CHAIN = 32, M_FLAG_SIDE = 40;
+                   M_V_SEEN = 24, M_FLAG_CHAIN = 32, M_FLAG_SIDE = 40, M_G_ISSUED = 48,
+                   M_G_SEEN = 52;
 
 constexpr uint32_t KQ_TX_BYTES = 4 * 4096;
 constexpr uint32_t V_TX_BYTES = NT * D * 2;
+constexpr uint32_t G_TX_BYTES = NT * D * 4;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float EXP2_CLAMP = 126.f;
@@ -133,17 +136,15 @@ __device__ __forceinline__ void tmem_st8x2(uint32_t ta, const uint32_t (&a)[8], 
 __device__ __forceinline__ float exp2c(float x) {
   return fast_exp2(fminf(fmaxf(x, -EXP2_CLAMP), EXP2_CLAMP));
 }
-// Byte offset of element (row r, column d) of a K-major SW128 tile whose
-// 64-column boxes are `box` bytes apart.
-__device__ __forceinline__ uint32_t kmaj_off(int r, int d, uint32_t box) {
-  return uint32_t(d >> 6) * box + sw128_off(r, (d & 63) >> 3) + uint32_t(d & 7) * 2u;
+// 32-bit shared-memory store / load at a register address plus a constant offset.
+template <uint32_t OFF>
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.b32 [%0+%2], %1;" ::"r"(addr), "r"(v), "n"(OFF) : "memory");
 }
-__device__ __forceinline__ void st_shared_b32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t ld_shared_b32(uint32_t addr) {
+template <uint32_t OFF>
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   uint32_t v;
-  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  asm volatile("ld.shared.b32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF) : "memory");
   return v;
 }
 
@@ -217,12 +218,20 @@ __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int
   *x.misc(M_V_ISSUED) = c + 1;
 }
 
+// g of tile c ([32 tokens][128] fp32; tokens past T read as 0) into buffer c & 1
+__device__ __forceinline__ void issue_g(const Ctx& x, const CUtensorMap* tg, int c, int h, int b) {
+  const uint32_t bar = x.bar(B_GLD + 8u * uint32_t(c & 1));
+  mbar_arrive_expect_tx(bar, G_TX_BYTES);
+  tma_load_4d(x.sb + ((c & 1) ? SM_G1 : SM_G0), tg, bar, 0, h, c * NT, b);
+  *x.misc(M_G_ISSUED) = c + 1;
+}
+
 // ============================================================== side role
 // Thread kt: channel pair cp = kt % 64 (channels 2cp, 2cp+1) and token quarter
 // qt = kt / 64 (tokens 8qt .. 8qt+7 of the tile) for the gates and operands;
 // TMEM lane quarter (warp % 4) and column half for the masks.
 __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
-                          const KdaArgs& p, int b, int h, int ntiles) {
+                          const CUtensorMap* tg, const KdaArgs& p, int b, int h, int ntiles) {
   const int kt = threadIdx.x - 128;
   const int warp = threadIdx.x >> 5;
   const int lq = warp & 3;
@@ -232,21 +241,35 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
   const uint32_t sb = x.sb;
   const int cp = kt & 63, qt = kt >> 6;
   const int d0 = 2 * cp;
+  // This thread's element (row 8 qt + t, columns d0, d0 + 1) of a K-major SW128
+  // tile whose 64-column boxes are `bx` bytes apart sits at tile_off(bx) +
+  // row_off(t): rows 8 qt .. 8 qt + 7 form one 8-row group, so the swizzle
+  // involves only t and d0's 16-byte chunk; row r + 32 m lies 4096 m bytes on.
+  const uint32_t cix = uint32_t((d0 & 63) >> 3);
+  const auto tile_off = [&](uint32_t bx) {
+    return uint32_t(d0 >> 6) * bx + uint32_t(qt) * 1024u + uint32_t(d0 & 7) * 2u;
+  };
+  const auto row_off = [&](int t) { return uint32_t(t) * 128u + ((cix ^ uint32_t(t)) << 4); };
   float* sA = reinterpret_cast<float*>(x.sm + SM_A);
   float* sT = reinterpret_cast<float*>(x.sm + SM_TF);
   float* sX = reinterpret_cast<float*>(x.sm + SM_X);
   RoleSync rs{BAR_SIDE, SIDE_THREADS, M_FLAG_SIDE, leader, 0};
+  // beta of token kt of the next tile, loaded one tile ahead (kt < 32)
+  float beta_next = 0.f;
+  if (kt < NT && kt < p.T) beta_next = __ldg(p.beta + (size_t(b) * p.T + kt) * p.H + h);
 
   for (int c = 0; c < ntiles; ++c) {
-    // ---- 1. gates: g of this thread's 8 tokens x 2 channels, cumulative sums
-    //      (log2 units) across the tile, beta, and Lambda_last per channel
+    // ---- 1. gates: g of this thread's 8 tokens x 2 channels (from the tile's
+    //      TMA buffer), cumulative sums (log2 units) across the tile, beta, and
+    //      Lambda_last per channel
     float gm[8][2];
     {
+      if (!rs.wait(x, x.bar(B_GLD + 8u * uint32_t(c & 1)), (c >> 1) & 1)) return;
+      if (leader) *x.misc(M_G_SEEN) = c + 1;
+      const float* sg = reinterpret_cast<const float*>(x.sm + ((c & 1) ? SM_G1 : SM_G0));
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        const int tok = c * NT + 8 * qt + t;
-        float2 g2 = make_float2(0.f, 0.f);
-        if (tok < p.T) g2 = __ldg(reinterpret_cast<const float2*>(p.g + ((size_t(b) * p.T + tok) * p.H + h) * D + d0));
+        const float2 g2 = *reinterpret_cast<const float2*>(sg + (8 * qt + t) * D + d0);
         gm[t][0] = g2.x * LOG2E;
         gm[t][1] = g2.y * LOG2E;
       }
@@ -256,13 +279,15 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
         gm[t][1] += gm[t - 1][1];
       }
       *reinterpret_cast<float2*>(sX + qt * 128 + d0) = make_float2(gm[7][0], gm[7][1]);
-      float* G = x.gates(c);
       if (kt < NT) {
-        const int tok = c * NT + kt;
-        G[G_B / 4 + kt] = tok < p.T ? __ldg(p.beta + (size_t(b) * p.T + tok) * p.H + h) : 0.f;
+        x.gates(c)[G_B / 4 + kt] = beta_next;
+        const int tok = (c + 1) * NT + kt;
+        beta_next = tok < p.T ? __ldg(p.beta + (size_t(b) * p.T + tok) * p.H + h) : 0.f;
       }
     }
     named_bar(BAR_SIDE, SIDE_THREADS);
+    // every thread has read g(c): its buffer takes g(c + 2)
+    if (leader && c + 2 < ntiles) issue_g(x, tg, c + 2, h, b);
     float gref[2], glast[2];
     {
       float pre[2] = {0.f, 0.f}, tot[2] = {0.f, 0.f}, half[2] = {0.f, 0.f};
@@ -297,11 +322,24 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
     {
       if (!rs.wait(x, x.bar(B_KQFULL), c & 1)) return;
       if (leader) *x.misc(M_KQ_SEEN) = c + 1;
+      // per channel: Lambda_r (from the tile start) and Lambda_last / Lambda_r,
+      // so that K+ = K' Lambda_r, Q+ = Q' Lambda_r and K~ = K'' Lambda_last / Lambda_r
+      // take two exponentials per token and channel instead of four (products
+      // capped at 2^126 like the exponents: no inf where g > 0 grows the state)
+      float lr[2], llr[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        lr[e] = exp2c(gref[e]);
+        llr[e] = exp2c(glast[e] - gref[e]);
+      }
+      constexpr float CAP = 8.5070592e37f;  // 2^126
+      const uint32_t kq_t = sb + SM_KQ + tile_off(8192u);  // K rows r; Q rows r at +4096
+      const uint32_t pa_t = sb + SM_PA + tile_off(16384u);  // rows r, 32 + r, 64 + r, 96 + r
+      const uint32_t pb_t = sb + SM_PB + tile_off(8192u);   // rows r, 32 + r
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        const int r = 8 * qt + t;
-        const uint32_t ko = SM_KQ + kmaj_off(r, d0, 8192u), qo = ko + 4096u;
-        const uint32_t kw = ld_shared_b32(sb + ko), qw = ld_shared_b32(sb + qo);
+        const uint32_t ro = row_off(t);
+        const uint32_t kw = lds32<0>(kq_t + ro), qw = lds32<4096>(kq_t + ro);
         const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw));
         const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw));
         const float kv[2] = {kf.x, kf.y}, qv[2] = {qf.x, qf.y};
@@ -310,8 +348,8 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
         for (int e = 0; e < 2; ++e) {
           const float ep = exp2c(gm[t][e] - gref[e]);   // Lambda_t / Lambda_r
           const float em = exp2c(gref[e] - gm[t][e]);   // Lambda_r / Lambda_t
-          const float eplus = exp2c(gm[t][e]);          // Lambda_t (from the tile start)
-          const float etil = exp2c(glast[e] - gm[t][e]);  // Lambda_last / Lambda_t
+          const float eplus = fminf(ep * lr[e], CAP);   // Lambda_t (from the tile start)
+          const float etil = fminf(em * llr[e], CAP);   // Lambda_last / Lambda_t
           k1[e] = kv[e] * ep;
           q1[e] = qv[e] * ep;
           k2[e] = kv[e] * em;
@@ -320,57 +358,69 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
           kt2[t][e] = kv[e] * etil;
         }
         uint32_t hi, lo;
-        split2_bf16(k1[0], k1[1], hi, lo);  // K' row r
-        st_shared_b32(sb + SM_PA + kmaj_off(r, d0, 8192u), hi);
-        st_shared_b32(sb + SM_PA + 16384u + kmaj_off(r, d0, 8192u), lo);
-        split2_bf16(q1[0], q1[1], hi, lo);  // Q' row 32 + r
-        st_shared_b32(sb + SM_PA + kmaj_off(32 + r, d0, 8192u), hi);
-        st_shared_b32(sb + SM_PA + 16384u + kmaj_off(32 + r, d0, 8192u), lo);
+        split2_bf16(k1[0], k1[1], hi, lo);  // K' hi row r, lo row 64 + r
+        sts32<0>(pa_t + ro, hi);
+        sts32<8192>(pa_t + ro, lo);
+        split2_bf16(q1[0], q1[1], hi, lo);  // Q' hi row 32 + r, lo row 96 + r
+        sts32<4096>(pa_t + ro, hi);
+        sts32<12288>(pa_t + ro, lo);
         split2_bf16(k2[0], k2[1], hi, lo);  // K'' hi row r, lo row 32 + r
-        st_shared_b32(sb + SM_PB + kmaj_off(r, d0, 8192u), hi);
-        st_shared_b32(sb + SM_PB + kmaj_off(32 + r, d0, 8192u), lo);
+        sts32<0>(pb_t + ro, hi);
+        sts32<4096>(pb_t + ro, lo);
       }
     }
     fence_proxy_async_smem();
     named_bar(BAR_SIDE, SIDE_THREADS);  // the raw tile is read; the P operands are in place
-    // ---- 3. P = [K';Q'] [K'' hi | K'' lo]^T + [K';Q'] lo K'' hi^T  (M=128: rows 0..63 used)
+    // ---- 3. P = [K' hi; Q' hi; K' lo; Q' lo] [K'' hi | K'' lo]^T  (M=128, N=64):
+    //      lanes 0..63 hold hi x hi | hi x lo, lanes 64..127 lo x hi | (unused lo x lo)
     {
       bool ok = true;
       if (leader) {
         if (c + 1 < ntiles) issue_kq(x, tq, tk, c + 1, h, b);
         tc_fence_after();
-        const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0), id32 = idesc_bf16(128, 32, 0, 0, 0);
+        const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0);
         const uint64_t da = sdesc_sw128(sb + SM_PA, 16, 1024), db = sdesc_sw128(sb + SM_PB, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-          mma_ss(x.tmem + TM_P, sdesc_add(da, off), sdesc_add(db, off), id64, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-          mma_ss(x.tmem + TM_P, sdesc_add(da, 16384 + off), sdesc_add(db, off), id32, 1u);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(x.tmem + TM_P, sdesc_add(da, (kk >> 2) * 16384 + (kk & 3) * 32),
+                 sdesc_add(db, (kk >> 2) * 8192 + (kk & 3) * 32), id64, kk > 0);
         mma_commit(x.bar(B_P));
         ok = lead_wait(x, x.bar(B_P), c & 1);
       }
       if (!rs.agree(x, ok)) return;
     }
     // ---- 4. masks: rows 0..31 (K') -> A = strict_tril(beta_i P_ij) (fp32, for the
-    //      solve); rows 32..63 (Q') -> Mq = tril(P_ij) (registers); lanes 64..127 unused
+    //      solve); rows 32..63 (Q') -> Mq = tril(P_ij) (registers).  The lo x hi
+    //      terms of row i sit in lane 64 + i (K') or 96 + i (Q'): those warps pass
+    //      them through shared memory (the A and T scratch, rewritten only after)
     float mq[16];
     {
       const float* G = x.gates(c);
+      const int i = threadIdx.x & 31;
+      float* xch = (lq & 1) ? sT : sA;
+      if (lq >= 2) {
+        float pl[16];
+        tmem_ld16(tlane + TM_P + 16 * hf, pl);
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4)
+          *reinterpret_cast<float4*>(xch + i * APAD + 16 * hf + 4 * e4) =
+              make_float4(pl[4 * e4], pl[4 * e4 + 1], pl[4 * e4 + 2], pl[4 * e4 + 3]);
+      }
+      named_bar(BAR_SIDE, SIDE_THREADS);
       if (lq < 2) {
         float pa[16], pb[16];
         tmem_ld16x2(tlane + TM_P + 16 * hf, pa, tlane + TM_P + 32 + 16 * hf, pb);
-        const int i = threadIdx.x & 31;
         const float bi = (lq == 0) ? G[G_B / 4 + i] : 1.f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int j = 16 * hf + e;
-          const float v = bi * (pa[e] + pb[e]);
-          mq[e] = (lq == 0 ? j < i : j <= i) ? v : 0.f;
+        for (int e4 = 0; e4 < 4; ++e4) {
+          const float4 l = ld4(xch + i * APAD + 16 * hf + 4 * e4);
+          const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 16 * hf + 4 * e4 + e;
+            const float v = bi * ((pa[4 * e4 + e] + lv[e]) + pb[4 * e4 + e]);
+            mq[4 * e4 + e] = (lq == 0 ? j < i : j <= i) ? v : 0.f;
+          }
         }
         if (lq == 0) {
 #pragma unroll
@@ -454,19 +504,23 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
     // ---- 7. the chain's operand tiles, once its state update of the previous
     //      tile (the last reader of both) has completed: [K+;Q+] hi/lo and K~ hi/lo
     if (c > 0 && !rs.wait(x, x.bar(B_OPFREE), (c - 1) & 1)) return;
+    {
+      const uint32_t zq_t = sb + SM_ZQB + tile_off(16384u);  // rows r, 32 + r, 64 + r, 96 + r
+      const uint32_t kt_t = sb + SM_KT + tile_off(4096u);    // rows j, 64-column blocks 4 KB apart
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int r = 8 * qt + t;
-      uint32_t hi, lo;
-      split2_bf16(kp[t][0], kp[t][1], hi, lo);
-      st_shared_b32(sb + SM_ZQB + kmaj_off(r, d0, 16384u), hi);
-      st_shared_b32(sb + SM_ZQB + kmaj_off(64 + r, d0, 16384u), lo);
-      split2_bf16(qp[t][0], qp[t][1], hi, lo);
-      st_shared_b32(sb + SM_ZQB + kmaj_off(32 + r, d0, 16384u), hi);
-      st_shared_b32(sb + SM_ZQB + kmaj_off(96 + r, d0, 16384u), lo);
-      split2_bf16(kt2[t][0], kt2[t][1], hi, lo);  // rows j, 64-column blocks 4 KB apart
-      st_shared_b32(sb + SM_KT + kmaj_off(r, d0, 4096u), hi);
-      st_shared_b32(sb + SM_KT + 8192u + kmaj_off(r, d0, 4096u), lo);
+      for (int t = 0; t < 8; ++t) {
+        const uint32_t ro = row_off(t);
+        uint32_t hi, lo;
+        split2_bf16(kp[t][0], kp[t][1], hi, lo);
+        sts32<0>(zq_t + ro, hi);
+        sts32<8192>(zq_t + ro, lo);
+        split2_bf16(qp[t][0], qp[t][1], hi, lo);
+        sts32<4096>(zq_t + ro, hi);
+        sts32<12288>(zq_t + ro, lo);
+        split2_bf16(kt2[t][0], kt2[t][1], hi, lo);
+        sts32<0>(kt_t + ro, hi);
+        sts32<8192>(kt_t + ro, lo);
+      }
     }
     fence_proxy_async_smem();
     named_bar(BAR_SIDE, SIDE_THREADS);
@@ -685,7 +739,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                       const KdaArgs p) {
+                       const __grid_constant__ CUtensorMap tm_g, const KdaArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -705,6 +759,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_o);
+    prefetch_tmap(&tm_g);
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(x.sb + SM_BAR + 8 * i, 1);
     fence_mbar_init();
     for (int i = 0; i < 16; ++i) reinterpret_cast<volatile int*>(sm + SM_MISC)[i] = 0;
@@ -720,11 +775,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (tid == 0) {
     issue_kq(x, &tm_q, &tm_k, 0, h, b);
     issue_v(x, &tm_v, 0, h, b);
+    issue_g(x, &tm_g, 0, h, b);
+    if (ntiles > 1) issue_g(x, &tm_g, 1, h, b);
   }
   if (warp < 4 || warp >= 12)
     chain_role(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
   else
-    side_role(x, &tm_q, &tm_k, p, b, h, ntiles);
+    side_role(x, &tm_q, &tm_k, &tm_g, p, b, h, ntiles);
 
   // each MMA-issuing thread waits (bounded) for its own products in flight
   if (tid == 0 || tid == 128 || tid == OI_ISSUER) {
@@ -742,6 +799,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (kq_issued > kq_seen) mbar_wait_bounded(x.bar(B_KQFULL), (kq_issued - 1) & 1, WAIT_LIMIT_NS / 4);
     const int v_issued = *x.misc(M_V_ISSUED), v_seen = *x.misc(M_V_SEEN);
     if (v_issued > v_seen) mbar_wait_bounded(x.bar(B_VFULL), (v_issued - 1) & 1, WAIT_LIMIT_NS / 4);
+    // g tiles: up to two in flight, tile i on barrier i & 1 with parity (i >> 1) & 1
+    const int g_issued = *x.misc(M_G_ISSUED), g_seen = *x.misc(M_G_SEEN);
+    for (int i = g_seen; i < g_issued; ++i)
+      mbar_wait_bounded(x.bar(B_GLD + 8u * uint32_t(i & 1)), uint32_t(i >> 1) & 1u, WAIT_LIMIT_NS / 4);
   }
   __syncthreads();
   tc_fence_after();
@@ -751,12 +812,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace
 
 int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& to, const KdaArgs& a, cudaStream_t stream) {
+                       const CUtensorMap& to, const CUtensorMap& tg, const KdaArgs& a,
+                       cudaStream_t stream) {
   const int chains = a.B * a.H;
   if (chains == 0 || a.T == 0) return -1;
   const uint32_t smem = SMEM_USED + 1024;
   if (!ensure_smem_attr(reinterpret_cast<const void*>(kda_prefill_kernel), 15, int(smem))) return -1;
-  kda_prefill_kernel<<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, a);
+  kda_prefill_kernel<<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, tg, a);
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 
