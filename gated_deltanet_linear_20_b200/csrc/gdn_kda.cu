@@ -73,40 +73,52 @@ constexpr int OI_ISSUER = 384;
 // have 128-byte rows (64 bf16 along K) in 8-row groups 1024 B apart.
 constexpr uint32_t SM_KQ = 0;          // raw [K dk0-63 | Q dk0-63 | K dk64-127 | Q dk64-127], 4 KB boxes
 constexpr uint32_t SM_V = 16384;       // raw V [32 tokens][128] bf16
-constexpr uint32_t SM_ZQB = 24576;     // [K+ hi; Q+ hi; K+ lo; Q+ lo] 128 rows, boxes dk0-63 / dk64-127 16 KB apart
+// The chain's operand tiles (ZQB: [K+;Q+], KT: K~) are double-buffered (tile c
+// in buffer c & 1), so the side writes them as soon as it derives them; the
+// solve's scratch (A, T, the exchange area) lives in the P operand region,
+// which is dead from P's completion to the next tile's operands.
+constexpr uint32_t SM_ZQB0 = 24576;    // [K+ hi; Q+ hi; K+ lo; Q+ lo] 128 rows, boxes dk0-63 / dk64-127 16 KB apart
 constexpr uint32_t SM_PA = 57344;      // [K' hi; Q' hi; K' lo; Q' lo] 128 rows, boxes 16 KB apart
 constexpr uint32_t SM_PB = 90112;      // [K'' hi; K'' lo] 64 rows, boxes 8 KB apart
-constexpr uint32_t SM_KT = 106496;     // K~ = K o Lambda_last / Lambda, rows j, MN-major: hi (2 x 4 KB), lo at +8 KB
+constexpr uint32_t SM_KT0 = 106496;    // K~ = K o Lambda_last / Lambda, rows j, MN-major: hi (2 x 4 KB), lo at +8 KB
 constexpr uint32_t SM_XH = 122880;     // the fp32 [32][128] o staging tile (16 KB)
-constexpr uint32_t SM_G0 = 139264;     // g tiles [32 tokens][128] fp32, two buffers (tile c in c & 1)
-constexpr uint32_t SM_G1 = 155648;
-constexpr uint32_t SM_TM = 188416;     // [T hi; T lo] rows i (32 + 32), K = 32 tokens
-constexpr uint32_t SM_MQ = 196608;     // [Mq hi; Mq lo]
+constexpr uint32_t SM_G = 139264;      // g tile [32 tokens][128] fp32
+constexpr uint32_t SM_ZQB1 = 155648;
+constexpr uint32_t SM_KT1 = 188416;
+constexpr uint32_t SM_TM = 204800;     // [T hi; T lo] rows i (32 + 32), K = 32 tokens
+constexpr uint32_t SM_MQ = 212992;     // [Mq hi; Mq lo]
 constexpr int APAD = 36;               // solve row pitch (floats)
-constexpr uint32_t SM_A = 204800;      // A fp32 [32][APAD]
+constexpr uint32_t SM_A = SM_PA;                   // A fp32 [32][APAD]
 constexpr uint32_t SM_TF = SM_A + 32 * APAD * 4;   // T fp32 [32][APAD]
 constexpr uint32_t SM_X = SM_TF + 32 * APAD * 4;   // exchange: per-quarter channel sums [4][128],
                                                    // then the solve's [16][16] product
-constexpr uint32_t SM_GATES = SM_X + 4 * 128 * 4;
+constexpr uint32_t SM_GATES = SM_MQ + 8192;
 constexpr uint32_t GATE_BYTES = 640;   // beta [32], Lambda_last [128]
 constexpr uint32_t G_B = 0, G_LC = 128;
 constexpr int GATE_BUFS = 4;
 constexpr uint32_t SM_BAR = SM_GATES + GATE_BUFS * GATE_BYTES;
 constexpr uint32_t SM_MISC = SM_BAR + 256;
 constexpr uint32_t SMEM_USED = SM_MISC + 256;
-static_assert(SM_ZQB % 1024 == 0 && SM_PA % 1024 == 0 && SM_PB % 1024 == 0 && SM_KT % 1024 == 0 &&
-                  SM_XH % 1024 == 0 && SM_TM % 1024 == 0 && SM_MQ % 1024 == 0 && SM_G0 % 1024 == 0 &&
-                  SM_G1 % 1024 == 0,
+static_assert(SM_ZQB0 % 1024 == 0 && SM_ZQB1 % 1024 == 0 && SM_PA % 1024 == 0 && SM_PB % 1024 == 0 &&
+                  SM_KT0 % 1024 == 0 && SM_KT1 % 1024 == 0 && SM_XH % 1024 == 0 && SM_TM % 1024 == 0 &&
+                  SM_MQ % 1024 == 0 && SM_G % 1024 == 0,
               "SW128 tiles need 1024-byte alignment");
-static_assert(SM_PA + 32768 <= SM_PB && SM_G1 + 16384 <= SM_TM, "operand regions");
+static_assert(SM_ZQB0 + 32768 <= SM_PA && SM_PA + 32768 <= SM_PB && SM_PB + 16384 <= SM_KT0 &&
+                  SM_KT0 + 16384 <= SM_XH && SM_XH + 16384 <= SM_G && SM_G + 16384 <= SM_ZQB1 &&
+                  SM_ZQB1 + 32768 <= SM_KT1 && SM_KT1 + 16384 <= SM_TM && SM_TM + 8192 <= SM_MQ,
+              "operand regions");
+static_assert(SM_X + 4 * 128 * 4 <= SM_PA + 32768, "solve scratch inside the P operand region");
 static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
+__device__ __forceinline__ uint32_t zqb_buf(int c) { return (c & 1) ? SM_ZQB1 : SM_ZQB0; }
+__device__ __forceinline__ uint32_t kt_buf(int c) { return (c & 1) ? SM_KT1 : SM_KT0; }
 
 // mbarriers (8 bytes each, offsets inside SM_BAR)
+// B_OPFULL, B_OPFREE: one per operand buffer (tile c: + 8 (c & 1), parity (c >> 1) & 1)
 constexpr uint32_t B_KQFULL = 0, B_VFULL = 8, B_P = 16, B_TMFULL = 24, B_TMFREE = 32,
-                   B_OPFULL = 40, B_OPFREE = 48, B_ZQ = 56, B_DL = 64, B_SU = 72, B_OI = 80,
-                   B_CLEAN0 = 88, B_CLEAN1 = 96, B_CLEAN2 = 104, B_GLD = 112,  // B_GLD: 2 barriers
-                   B_GFULL = 128;  // B_GFULL: 4 barriers
-constexpr int NUM_BARS = 20;
+                   B_OPFULL = 40, B_OPFREE = 56, B_ZQ = 72, B_DL = 80, B_SU = 88, B_OI = 96,
+                   B_CLEAN0 = 104, B_CLEAN1 = 112, B_CLEAN2 = 120, B_GLD = 128,
+                   B_GFULL = 136;  // B_GFULL: 4 barriers
+constexpr int NUM_BARS = 21;
 static_assert(8 * NUM_BARS <= 256, "barrier slots");
 __device__ __forceinline__ uint32_t gfull_off(int c) { return B_GFULL + 8u * uint32_t(c & 3); }
 __device__ __forceinline__ uint32_t gfull_parity(int c) { return uint32_t(c >> 2) & 1u; }
@@ -218,11 +230,12 @@ __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int
   *x.misc(M_V_ISSUED) = c + 1;
 }
 
-// g of tile c ([32 tokens][128] fp32; tokens past T read as 0) into buffer c & 1
+// g of tile c ([32 tokens][128] fp32; tokens past T read as 0), issued once
+// every side thread has read tile c - 1's
 __device__ __forceinline__ void issue_g(const Ctx& x, const CUtensorMap* tg, int c, int h, int b) {
-  const uint32_t bar = x.bar(B_GLD + 8u * uint32_t(c & 1));
+  const uint32_t bar = x.bar(B_GLD);
   mbar_arrive_expect_tx(bar, G_TX_BYTES);
-  tma_load_4d(x.sb + ((c & 1) ? SM_G1 : SM_G0), tg, bar, 0, h, c * NT, b);
+  tma_load_4d(x.sb + SM_G, tg, bar, 0, h, c * NT, b);
   *x.misc(M_G_ISSUED) = c + 1;
 }
 
@@ -264,9 +277,9 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
     //      Lambda_last per channel
     float gm[8][2];
     {
-      if (!rs.wait(x, x.bar(B_GLD + 8u * uint32_t(c & 1)), (c >> 1) & 1)) return;
+      if (!rs.wait(x, x.bar(B_GLD), c & 1)) return;
       if (leader) *x.misc(M_G_SEEN) = c + 1;
-      const float* sg = reinterpret_cast<const float*>(x.sm + ((c & 1) ? SM_G1 : SM_G0));
+      const float* sg = reinterpret_cast<const float*>(x.sm + SM_G);
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
         const float2 g2 = *reinterpret_cast<const float2*>(sg + (8 * qt + t) * D + d0);
@@ -286,8 +299,8 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
       }
     }
     named_bar(BAR_SIDE, SIDE_THREADS);
-    // every thread has read g(c): its buffer takes g(c + 2)
-    if (leader && c + 2 < ntiles) issue_g(x, tg, c + 2, h, b);
+    // every thread has read g(c): the buffer takes g(c + 1)
+    if (leader && c + 1 < ntiles) issue_g(x, tg, c + 1, h, b);
     float gref[2], glast[2];
     {
       float pre[2] = {0.f, 0.f}, tot[2] = {0.f, 0.f}, half[2] = {0.f, 0.f};
@@ -315,13 +328,18 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
     named_bar(BAR_SIDE, SIDE_THREADS);  // gates complete; the exchange area is free again
     if (leader) mbar_arrive(x.bar(gfull_off(c)));
 
-    // ---- 2. the decayed operands of this thread's 8 tokens x 2 channels: the
-    //      P operands go to shared memory now; K+, Q+, K~ stay in registers
-    //      until the chain has released their tiles
-    float kp[8][2], qp[8][2], kt2[8][2];
+    // ---- 2. the decayed operands of this thread's 8 tokens x 2 channels, to
+    //      shared memory: the P operands, and the chain's [K+;Q+] and K~ into
+    //      buffer c & 1 once the chain's state update of tile c - 2 (their last
+    //      reader) has completed
     {
-      if (!rs.wait(x, x.bar(B_KQFULL), c & 1)) return;
-      if (leader) *x.misc(M_KQ_SEEN) = c + 1;
+      bool ok = true;
+      if (leader) {
+        ok = lead_wait(x, x.bar(B_KQFULL), c & 1) &&
+             (c < 2 || lead_wait(x, x.bar(B_OPFREE + 8u * uint32_t(c & 1)), ((c - 2) >> 1) & 1));
+        if (ok) *x.misc(M_KQ_SEEN) = c + 1;
+      }
+      if (!rs.agree(x, ok)) return;
       // per channel: Lambda_r (from the tile start) and Lambda_last / Lambda_r,
       // so that K+ = K' Lambda_r, Q+ = Q' Lambda_r and K~ = K'' Lambda_last / Lambda_r
       // take two exponentials per token and channel instead of four (products
@@ -336,6 +354,8 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
       const uint32_t kq_t = sb + SM_KQ + tile_off(8192u);  // K rows r; Q rows r at +4096
       const uint32_t pa_t = sb + SM_PA + tile_off(16384u);  // rows r, 32 + r, 64 + r, 96 + r
       const uint32_t pb_t = sb + SM_PB + tile_off(8192u);   // rows r, 32 + r
+      const uint32_t zq_t = sb + zqb_buf(c) + tile_off(16384u);  // rows r, 32 + r, 64 + r, 96 + r
+      const uint32_t kt_t = sb + kt_buf(c) + tile_off(4096u);    // rows j, 64-column blocks 4 KB apart
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
         const uint32_t ro = row_off(t);
@@ -343,7 +363,7 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
         const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw));
         const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw));
         const float kv[2] = {kf.x, kf.y}, qv[2] = {qf.x, qf.y};
-        float k1[2], q1[2], k2[2];
+        float k1[2], q1[2], k2[2], kp[2], qp[2], kt2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const float ep = exp2c(gm[t][e] - gref[e]);   // Lambda_t / Lambda_r
@@ -353,9 +373,9 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
           k1[e] = kv[e] * ep;
           q1[e] = qv[e] * ep;
           k2[e] = kv[e] * em;
-          kp[t][e] = kv[e] * eplus;
-          qp[t][e] = qv[e] * eplus;
-          kt2[t][e] = kv[e] * etil;
+          kp[e] = kv[e] * eplus;
+          qp[e] = qv[e] * eplus;
+          kt2[e] = kv[e] * etil;
         }
         uint32_t hi, lo;
         split2_bf16(k1[0], k1[1], hi, lo);  // K' hi row r, lo row 64 + r
@@ -367,10 +387,20 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
         split2_bf16(k2[0], k2[1], hi, lo);  // K'' hi row r, lo row 32 + r
         sts32<0>(pb_t + ro, hi);
         sts32<4096>(pb_t + ro, lo);
+        split2_bf16(kp[0], kp[1], hi, lo);  // K+ hi row r, lo row 64 + r
+        sts32<0>(zq_t + ro, hi);
+        sts32<8192>(zq_t + ro, lo);
+        split2_bf16(qp[0], qp[1], hi, lo);  // Q+ hi row 32 + r, lo row 96 + r
+        sts32<4096>(zq_t + ro, hi);
+        sts32<12288>(zq_t + ro, lo);
+        split2_bf16(kt2[0], kt2[1], hi, lo);  // K~ rows j: hi, lo 8 KB on
+        sts32<0>(kt_t + ro, hi);
+        sts32<8192>(kt_t + ro, lo);
       }
     }
     fence_proxy_async_smem();
-    named_bar(BAR_SIDE, SIDE_THREADS);  // the raw tile is read; the P operands are in place
+    named_bar(BAR_SIDE, SIDE_THREADS);  // the raw tile is read; every operand is in place
+    if (leader) mbar_arrive(x.bar(B_OPFULL + 8u * uint32_t(c & 1)));
     // ---- 3. P = [K' hi; Q' hi; K' lo; Q' lo] [K'' hi | K'' lo]^T  (M=128, N=64):
     //      lanes 0..63 hold hi x hi | hi x lo, lanes 64..127 lo x hi | (unused lo x lo)
     {
@@ -501,30 +531,6 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
     fence_proxy_async_smem();
     named_bar(BAR_SIDE, SIDE_THREADS);
     if (leader) mbar_arrive(x.bar(B_TMFULL));
-    // ---- 7. the chain's operand tiles, once its state update of the previous
-    //      tile (the last reader of both) has completed: [K+;Q+] hi/lo and K~ hi/lo
-    if (c > 0 && !rs.wait(x, x.bar(B_OPFREE), (c - 1) & 1)) return;
-    {
-      const uint32_t zq_t = sb + SM_ZQB + tile_off(16384u);  // rows r, 32 + r, 64 + r, 96 + r
-      const uint32_t kt_t = sb + SM_KT + tile_off(4096u);    // rows j, 64-column blocks 4 KB apart
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const uint32_t ro = row_off(t);
-        uint32_t hi, lo;
-        split2_bf16(kp[t][0], kp[t][1], hi, lo);
-        sts32<0>(zq_t + ro, hi);
-        sts32<8192>(zq_t + ro, lo);
-        split2_bf16(qp[t][0], qp[t][1], hi, lo);
-        sts32<4096>(zq_t + ro, hi);
-        sts32<12288>(zq_t + ro, lo);
-        split2_bf16(kt2[t][0], kt2[t][1], hi, lo);
-        sts32<0>(kt_t + ro, hi);
-        sts32<8192>(kt_t + ro, lo);
-      }
-    }
-    fence_proxy_async_smem();
-    named_bar(BAR_SIDE, SIDE_THREADS);
-    if (leader) mbar_arrive(x.bar(B_OPFULL));
   }
 }
 
@@ -573,9 +579,9 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
     const int n0 = 16 * ch;  // this thread's tokens of the tile
     // ---- [Z|Y] = S_c [K+;Q+]^T: S hi x [hi rows; lo rows] (N=128), S lo x hi rows (N=64)
     if (leader) {
-      if (lead_wait(x, x.bar(B_OPFULL), c & 1)) {
+      if (lead_wait(x, x.bar(B_OPFULL + 8u * uint32_t(c & 1)), (c >> 1) & 1)) {
         tc_fence_after();
-        const uint64_t db = sdesc_sw128(sb + SM_ZQB, 16, 1024);
+        const uint64_t db = sdesc_sw128(sb + zqb_buf(c), 16, 1024);
         const uint32_t id128 = idesc_bf16(128, 128, 0, 0, 0), id64 = idesc_bf16(128, 64, 0, 0, 0);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -656,13 +662,13 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
 #pragma unroll
       for (int part = 0; part < 3; ++part) {
         const uint32_t a = x.tmem + TM_X + (part == 2 ? 8 : 0);
-        const uint32_t kb = part == 1 ? SM_KT + 8192 : SM_KT;
+        const uint32_t kb = kt_buf(c) + (part == 1 ? 8192u : 0u);
 #pragma unroll
         for (int ks = 0; ks < 2; ++ks)
           mma_ts(x.tmem + TM_S, a + 16 * ks, sdesc_sw128(sb + kb + 2048 * ks, 4096, 1024), idu, 1u);
       }
       mma_commit(x.bar(B_SU));
-      mma_commit(x.bar(B_OPFREE));  // [K+;Q+] (read by the first product) and K~ consumed
+      mma_commit(x.bar(B_OPFREE + 8u * uint32_t(c & 1)));  // [K+;Q+] (read by [Z|Y]) and K~ consumed
     }
     if (threadIdx.x == OI_ISSUER && !*x.abort_flag) {
       tc_fence_after();
@@ -776,7 +782,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     issue_kq(x, &tm_q, &tm_k, 0, h, b);
     issue_v(x, &tm_v, 0, h, b);
     issue_g(x, &tm_g, 0, h, b);
-    if (ntiles > 1) issue_g(x, &tm_g, 1, h, b);
   }
   if (warp < 4 || warp >= 12)
     chain_role(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
@@ -799,10 +804,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (kq_issued > kq_seen) mbar_wait_bounded(x.bar(B_KQFULL), (kq_issued - 1) & 1, WAIT_LIMIT_NS / 4);
     const int v_issued = *x.misc(M_V_ISSUED), v_seen = *x.misc(M_V_SEEN);
     if (v_issued > v_seen) mbar_wait_bounded(x.bar(B_VFULL), (v_issued - 1) & 1, WAIT_LIMIT_NS / 4);
-    // g tiles: up to two in flight, tile i on barrier i & 1 with parity (i >> 1) & 1
     const int g_issued = *x.misc(M_G_ISSUED), g_seen = *x.misc(M_G_SEEN);
-    for (int i = g_seen; i < g_issued; ++i)
-      mbar_wait_bounded(x.bar(B_GLD + 8u * uint32_t(i & 1)), uint32_t(i >> 1) & 1u, WAIT_LIMIT_NS / 4);
+    if (g_issued > g_seen) mbar_wait_bounded(x.bar(B_GLD), (g_issued - 1) & 1, WAIT_LIMIT_NS / 4);
   }
   __syncthreads();
   tc_fence_after();
