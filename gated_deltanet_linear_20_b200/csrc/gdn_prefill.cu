@@ -272,12 +272,15 @@ __device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int
 //   T_IJ = -sum_{K=J}^{I-1} At_IK T_KJ            (I > J),
 // computed by distance d = I - J = 1, 2, 3 after one pass that forms all six
 // At blocks.  A thread owns 1 x 4 strips of outputs; each dot product is split
-// over two accumulators; all loop bounds are compile-time.
+// over two accumulators; all loop bounds are compile-time.  The strip and block
+// loops stay rolled (only the 16-term dot products are unrolled): the per-tile
+// code path is long enough for instruction fetch to show, and on B200 this form
+// ran the 128-chain prefill ~4% faster than the fully unrolled one.
 __device__ __forceinline__ int at_index(int I, int K) { return (I * (I - 1)) / 2 + K; }  // 0..5
 
 __device__ __forceinline__ void solve_at_blocks(int kt, const float* sA, const float* sTf, float* sAt) {
   // 6 blocks x 16 rows x 4 strips = 384 strips
-#pragma unroll
+#pragma unroll 1
   for (int st = kt; st < 384; st += SIDE_THREADS) {
     const int blk = st >> 6, r = (st >> 2) & 15, c4 = st & 3;
     const int I = blk < 1 ? 1 : (blk < 3 ? 2 : 3);
@@ -302,12 +305,12 @@ __device__ __forceinline__ void solve_at_blocks(int kt, const float* sA, const f
 template <int d>
 __device__ __forceinline__ void solve_distance(int kt, const float* sAt, float* sTf) {
   constexpr int NSTRIP = (4 - d) * 64;
-#pragma unroll
+#pragma unroll 1
   for (int st = kt; st < NSTRIP; st += SIDE_THREADS) {
     const int J = st >> 6, r = (st >> 2) & 15, c4 = st & 3;
     const int I = J + d;
     float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
-#pragma unroll
+#pragma unroll 1
     for (int K = J; K < I; ++K) {
       const float* atrow = sAt + at_index(I, K) * AT_BLOCK + r * AT_PITCH;  // At_IK row r
       const float* tcol = sTf + (K * 16) * APAD + J * 16 + 4 * c4;    // T_KJ rows, cols 4c4..
