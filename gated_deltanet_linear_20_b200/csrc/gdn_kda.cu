@@ -277,8 +277,12 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
     //      Lambda_last per channel
     float gm[8][2];
     {
-      if (!rs.wait(x, x.bar(B_GLD), c & 1)) return;
-      if (leader) *x.misc(M_G_SEEN) = c + 1;
+      // tile 0's g is waited for here, every later tile's in the agreement that
+      // ends the previous tile
+      if (c == 0) {
+        if (!rs.wait(x, x.bar(B_GLD), 0)) return;
+        if (leader) *x.misc(M_G_SEEN) = 1;
+      }
       const float* sg = reinterpret_cast<const float*>(x.sm + SM_G);
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
@@ -325,8 +329,6 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
         *reinterpret_cast<float2*>(G + G_LC / 4 + d0) = make_float2(exp2c(tot[0]), exp2c(tot[1]));
       }
     }
-    named_bar(BAR_SIDE, SIDE_THREADS);  // gates complete; the exchange area is free again
-    if (leader) mbar_arrive(x.bar(gfull_off(c)));
 
     // ---- 2. the decayed operands of this thread's 8 tokens x 2 channels, to
     //      shared memory: the P operands, and the chain's [K+;Q+] and K~ into
@@ -339,7 +341,10 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
              (c < 2 || lead_wait(x, x.bar(B_OPFREE + 8u * uint32_t(c & 1)), ((c - 2) >> 1) & 1));
         if (ok) *x.misc(M_KQ_SEEN) = c + 1;
       }
+      // (this agreement also closes the gates: every thread has written its
+      // gate entries and read the exchange area, which the operands overwrite)
       if (!rs.agree(x, ok)) return;
+      if (leader) mbar_arrive(x.bar(gfull_off(c)));
       // per channel: Lambda_r (from the tile start) and Lambda_last / Lambda_r,
       // so that K+ = K' Lambda_r, Q+ = Q' Lambda_r and K~ = K'' Lambda_last / Lambda_r
       // take two exponentials per token and channel instead of four (products
@@ -515,10 +520,14 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
       }
       sT[(16 + r) * APAD + cc] = -(a0 + a1);
     }
-    named_bar(BAR_SIDE, SIDE_THREADS);
-    // ---- 6. hand T and Mq to the chain once it is done with the previous tile's
-    //      (its output product, the last reader, has completed)
-    if (c > 0 && !rs.wait(x, x.bar(B_TMFREE), (c - 1) & 1)) return;
+    // ---- 6. hand T and Mq to the chain once T is complete and the chain is done
+    //      with the previous tile's (its output product, the last reader, has
+    //      completed): one agreement
+    {
+      bool ok = true;
+      if (leader && c > 0) ok = lead_wait(x, x.bar(B_TMFREE), (c - 1) & 1);
+      if (!rs.agree(x, ok)) return;
+    }
     if (kt < 4 * NT) {  // T: row i = kt / 4, 8 columns each
       const int i = kt >> 2, cc = kt & 3;
       store_split8(sb + SM_TM, sb + SM_TM + 4096, i, cc, sT + i * APAD + 8 * cc);
@@ -529,7 +538,15 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
       for (int e = 0; e < 2; ++e) store_split8(sb + SM_MQ, sb + SM_MQ + 4096, i, 2 * hf + e, mq + 8 * e);
     }
     fence_proxy_async_smem();
-    named_bar(BAR_SIDE, SIDE_THREADS);
+    {
+      // T and Mq are in place, and the next tile's g has landed: one agreement
+      bool ok = true;
+      if (leader && c + 1 < ntiles) {
+        ok = lead_wait(x, x.bar(B_GLD), (c + 1) & 1);
+        if (ok) *x.misc(M_G_SEEN) = c + 2;
+      }
+      if (!rs.agree(x, ok)) return;
+    }
     if (leader) mbar_arrive(x.bar(B_TMFULL));
   }
 }
