@@ -375,7 +375,9 @@ __device__ __forceinline__ void side_norms(const Ctx& x, int kt, int c, const Pr
   }
 }
 
-template <int C, bool PRE>
+// CLOSE: end with a role-wide barrier and signal the gates' barrier; without
+// it the caller does both (in its next agreement).
+template <int C, bool PRE, bool CLOSE = true>
 __device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, float& g_next,
                                            float& b_next, const PrefillArgs& p, int b, int h,
                                            volatile float* s_part) {
@@ -425,8 +427,10 @@ __device__ __forceinline__ void side_gates(const Ctx& x, int kt, int c, int T, f
     }
     if (kt == last) G[G_GC / 4 + kt / C] = fast_exp2(gl);
   }
-  named_bar(BAR_SIDE, SIDE_THREADS);
-  if (kt == 0) mbar_arrive(x.bar(gfull_off(c)));
+  if constexpr (CLOSE) {
+    named_bar(BAR_SIDE, SIDE_THREADS);
+    if (kt == 0) mbar_arrive(x.bar(gfull_off(c)));
+  }
 }
 
 template <int DK>
@@ -642,7 +646,8 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       solve_distance<2>(kt, sAt, sTf);
       named_bar(BAR_SIDE, SIDE_THREADS);
       solve_distance<3>(kt, sAt, sTf);
-      named_bar(BAR_SIDE, SIDE_THREADS);
+      // (the role-wide barriers of the next tile's gates, or the hand-over's
+      // agreement, order these rows of T before the hand-over reads them)
     }
 
     // ---- gates of the next tile, while the chain is still on tile c-1 / c (with
@@ -654,11 +659,20 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
         side_norms(x, kt, c + 1, p);
         named_bar(BAR_SIDE, SIDE_THREADS);
       }
-      side_gates<C, PRE>(x, kt, c + 1, T, g_next, b_next, p, b, h, s_part);
+      side_gates<C, PRE, false>(x, kt, c + 1, T, g_next, b_next, p, b, h, s_part);
     }
 
-    // ---- hand T(c), Mq(c) to the chain once it is done with tile c-1's
-    if (c > 0 && !rs.wait(x, x.bar(B_TMFREE), (c - 1) & 1)) return;
+    // ---- hand T(c), Mq(c) to the chain once it is done with tile c-1's; the
+    //      same agreement closes the next tile's gates
+    {
+      bool ok = true;
+      if (leader) {
+        if (c > 0) ok = (*x.abort_flag == 0) && mbar_wait_bounded(x.bar(B_TMFREE), (c - 1) & 1, WAIT_LIMIT_NS);
+        if (!ok) x.fail();
+      }
+      if (!rs.agree(x, ok)) return;
+      if (leader && c + 1 < ntiles) mbar_arrive(x.bar(gfull_off(c + 1)));
+    }
     if (row < NT) {
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8)
@@ -672,13 +686,17 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
     named_bar(BAR_SIDE, SIDE_THREADS);
     if (leader) mbar_arrive(x.bar(B_TMFULL));
 
-    // ---- P(c+1), if it could not be started early
-    if (c + 1 < ntiles) {
-      if (!rs.wait(x, x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1)) return;
-      if (p_iss && p_issued == c + 1) {
+    // ---- P(c+1), if it could not be started early: its issuer waits for the
+    //      tile alone (a failed wait aborts the CTA; the next agreement sees it)
+    if (c + 1 < ntiles && p_iss && p_issued == c + 1) {
+      if (*x.abort_flag == 0 &&
+          mbar_wait_bounded(x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1, WAIT_LIMIT_NS)) {
+        tc_fence_after();
         *x.misc(M_KQ_SEEN) = c + 2;
         issue_p<DK>(x, c + 1);
         p_issued = c + 2;
+      } else {
+        x.fail();
       }
     }
   }
