@@ -287,6 +287,25 @@ def test_varlen_bad_offsets_are_reported_on_the_device():
     assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
 
 
+def test_varlen_malformed_offsets_leave_memory_before_the_snapshots_untouched():
+    """cu_seqlens [100, 0, 200] with snapshots: sequence 0 ends before it
+    starts.  Its own CTAs report GDN_ERR_SHAPE; sequence 1's snapshot slot base,
+    which counts sequence 0's snapshots, would come out negative, so sequence 1
+    takes no snapshots and nothing before the snapshot buffer is written."""
+    H, T = 2, 200
+    d = inputs.prefill_inputs(1, T, H, seed=91)
+    gdn = _gdn()
+    flat = lambda x: x[0].contiguous().to(DEV)
+    cu = torch.tensor([100, 0, 200], dtype=torch.int32, device=DEV)
+    guard = 2  # state-sized slots in front of the snapshot buffer
+    buf = torch.full((guard + 3, H, 128, 128), 7.0, dtype=torch.float32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gdn.prefill_varlen(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["g"]), flat(d["beta"]), cu,
+                       status=status, snap_every=64, snaps=buf[guard:])
+    assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
+    assert torch.all(buf[:guard] == 7.0), "memory before the snapshot buffer was written"
+
+
 def raw_qk(d, seed):
     """Un-normalised q, k (each token-head row scaled by a random factor in
     [0.2, 5]) and their fp64 L2-normalised versions."""
