@@ -84,7 +84,7 @@ constexpr uint32_t SM_MQL = 90112;
 constexpr uint32_t SM_TH = 98304;     // 8 KB: T rows i (64 x 64)
 constexpr uint32_t SM_TL = 106496;
 constexpr uint32_t SM_XH = 114688;    // 32 KB staging: the fp32 o tile [64 tokens][128]
-constexpr uint32_t SM_XL = 131072;    //   (and, with the Dl^T tiles, the 64 KB end state)
+constexpr uint32_t SM_XL = 131072;    //   (and, with the Dl^T tiles after them, the 64 KB end state)
 constexpr uint32_t SM_DH = 147456;    // 16 KB: Dl^T rows dv (128 x 64)
 constexpr uint32_t SM_DL = 163840;
 constexpr int APAD = 68;                      // row pitch (floats): conflict-free float4 rows
@@ -112,7 +112,7 @@ constexpr uint32_t SM_BAR = SM_GATES + GATE_BUFS * GATE_BYTES;
 constexpr uint32_t SM_MISC = SM_BAR + 256;    // TMEM slot, abort flags, scan scratch, counters
 constexpr uint32_t SMEM_USED = SM_MISC + 256;
 static_assert(SM_A >= SM_DL + 16384, "K-side scratch overlaps the residual tiles");
-static_assert(SM_DL + 16384 - SM_XH == 65536, "X^T and Dl^T tiles form the 64 KB end-state staging area");
+static_assert(SM_DL + 16384 - SM_XH == 65536, "o staging and Dl^T tiles form the 64 KB end-state staging area");
 static_assert(SMEM_USED + 1024 <= 232448, "shared memory budget");
 
 // mbarriers (8 bytes each, offsets inside SM_BAR)
@@ -458,11 +458,10 @@ __device__ __noinline__ void store_partial_tile(const float4* src, float* dst, i
 }
 
 // o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] of tile c.  This thread's 32
-// tokens (32 hf ..) of lane dv go into an fp32 [64 tokens][128] tile in the
-// X^T region, which is free between the state update and the next X epilogue;
-// the leader then stores the tile with TMA (tokens at or past T are dropped by
-// the copy) and waits for the copy to have read the tile before X^T is written
-// again.
+// tokens (32 hf ..) of lane dv go into the fp32 [64 tokens][128] o staging
+// tile; the leader then stores the tile with TMA (tokens at or past T are
+// dropped by the copy).  Before the next tile's staging is written the leader
+// waits for the copy to have read it (at the next tile's first agreement).
 // OBF: o is bf16 (tile rows of 256 B, stored through a bf16 view).
 template <bool OBF, int DVB>
 __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b, int h, int dv,
@@ -834,7 +833,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       {
         bool ok = true;
         if (leader) {
-          bulk_wait_read0();  // the previous tile's o store has read the X^T region
+          bulk_wait_read0();  // the previous tile's o store has read its staging tile
           ok = (*x.abort_flag == 0) && mbar_wait_bounded(x.bar(B_ZQ), sc & 1, WAIT_LIMIT_NS);
           if (ok && s == 0)
             ok = mbar_wait_bounded(x.bar(gfull_off(c)), gfull_parity(c), WAIT_LIMIT_NS);
@@ -1038,7 +1037,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
             }
           }
         } else if (final_chunk) {
-          // the end state goes out through the X^T / Dl^T region (64 KB, free once
+          // the end state goes out through the o staging / Dl^T region (64 KB, free once
           // the o store has read it): rows of 512 B whose 16-byte chunks are
           // XOR-swizzled by the row, then copied out row by row
           if (leader) bulk_wait_read0();
