@@ -379,3 +379,17 @@ def test_other_head_dims_size_the_overlap_checks(gdn):
     o = P + 0x50000000 - 0x8000
     assert gdn.raw_prefill(*prefill_args(o=o, Dk=64, Dv=256)) == -5
     assert gdn.raw_prefill(*prefill_args(o=o, Dk=64, Dv=64)) not in VALIDATION_CODES
+
+
+def test_plain_c_client_links_and_gets_the_documented_codes(gdn, tmp_path):
+    """tests/csrc/abi_c_client.c includes include/gdn.h as C99 (gcc, -Werror),
+    links the library and checks the device-free entry points and the
+    validation codes of the compute entry points."""
+    lib_dir = os.path.dirname(gdn.library_path)
+    exe = str(tmp_path / "abi_c_client")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "csrc", "abi_c_client.c"), "-L", lib_dir, "-lgdn_b200",
+                           "-Wl,-rpath," + lib_dir, "-o", exe])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "0 failure(s)" in r.stdout
