@@ -6,6 +6,8 @@
   exp(gamma_i - gamma_j) underflow to zero and the masked products must stay
   exact.  A second recipe alternates 32-token blocks of strong and weak decay,
   so that one chunk holds both underflowed and ordinary factors.
+* Growing states: positive log decays (g = 0.02 |logsigmoid(N(0, 1))|), with
+  the scalar gate and with a per-channel gate.
 * Un-normalised keys and queries without the fused norm: ||k|| drawn in
   [0.3, 1.4] per token and head, ||q|| in [0.5, 2].  beta ||k||^2 <= 1.96 keeps
   every factor (I - beta k k^T) a contraction along k, so the recurrence stays
@@ -125,3 +127,32 @@ def test_strong_decay_decode_burst_and_step():
     torch.cuda.synchronize()
     check(o.cpu().numpy(), ro, "o (burst)", design=False)
     check(S.cpu().numpy(), rS, "S (burst)", design=False)
+
+
+@pytest.mark.parametrize("segmented", [False, True], ids=["single", "segmented"])
+@pytest.mark.parametrize("chunk", [64, 16])
+def test_growing_state(chunk, segmented):
+    """Positive log decays (the API accepts g > 0, which grows the state):
+    g = 0.02 |logsigmoid(N(0, 1))|, so the state's decay factor grows to about
+    e^4 over the 300 tokens and the in-chunk factors exp(gamma_i - gamma_j)
+    exceed 1."""
+    d = inputs.prefill_inputs(2, 300, 3, seed=131, s0_std=0.05)
+    d["g"] = (d["g"].abs() * 0.02).contiguous()
+    o, S_T, ro, rS = run_both(d, chunk, segmented)
+    check(o, ro, "o (growing state)")
+    check(S_T, rS, "S_T (growing state)")
+
+
+def test_growing_state_per_channel_gate():
+    """The same with a per-channel gate (the KDA tensor-core kernel): positive
+    log decays of different sizes per key channel."""
+    d = inputs.kda_inputs(2, 300, 3, seed=137, s0_std=0.05)
+    d["g"] = (d["g"].abs() * 0.02).contiguous()
+    gdn = _gdn()
+    dd = {k: (v.to(DEV) if v is not None else None) for k, v in d.items()}
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.kda_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"], status=status)
+    assert gdn.query_status(status) == 0
+    ro, rS = oracle.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    check(o.cpu().numpy(), ro, "o (growing state, per-channel gate)")
+    check(S_T.cpu().numpy(), rS, "S_T (growing state, per-channel gate)")
