@@ -154,8 +154,10 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     ``qk_l2norm`` / ``q_scale`` (gdn_options) normalise q and k per token and
     head and scale q inside the kernel (gdn_prefill_ex).  ``o_bf16`` makes o
     bf16 (the fp32 value rounded to nearest even); it runs the single pass.
-    Dk, Dv may each be 64, 128 or 256: other than 128 x 128 the row-parallel
-    fp32 kernel runs (chunk, segments and the fused options do not apply)."""
+    Dk, Dv may each be 64, 128 or 256.  With Dk = 64 or 128 the chunked
+    tensor-core kernel runs (Dv = 256 on two CTAs per chain); with Dk = 256 the
+    row-parallel fp32 kernel.  Segments and the fused options apply at 128 x 128
+    only."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape
