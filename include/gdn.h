@@ -118,11 +118,12 @@ const char* gdn_status_str(int code);
  *   S_T  : final state, written (device; may equal S0)
  *   B, T, H : batch, tokens per sequence, heads; B*H == 0 or T == 0 are valid
  *             (T == 0 only writes S_T = S0, or zeros)
- *   Dk, Dv  : head dims, each 64, 128 or 256.  128 x 128 runs the chunked
- *             tensor-core kernel; every other pair runs the row-parallel fp32
- *             kernel (token by token, exact in the recurrence's order; chunk,
- *             workspace and schedule do not apply to it).  Other values:
- *             GDN_ERR_UNSUPPORTED
+ *   Dk, Dv  : head dims, each 64, 128 or 256.  Dk = 64 or 128 runs the
+ *             chunked tensor-core kernel (Dv = 256 on two CTAs per chain; the
+ *             segmented schedule only at 128 x 128); Dk = 256 runs the
+ *             row-parallel fp32 kernel (token by token, exact in the
+ *             recurrence's order; chunk, workspace and schedule do not apply
+ *             to it).  Other values: GDN_ERR_UNSUPPORTED
  *   chunk   : 16 or 64 -- tokens per chunk of the chunked form; the result is
  *             the same recurrence either way (up to rounding)
  *   status  : optional device int; a bounded device wait that gives up stores
