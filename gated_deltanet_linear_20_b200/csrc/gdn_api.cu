@@ -561,9 +561,21 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
 int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
                     const float* beta, const float* S0, float* o, float* S_T, int B, int T,
                     int H, int Dk, int Dv, int* status, void* stream) {
+  return gdn_kda_prefill_ex(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, nullptr, status, stream);
+}
+
+int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* S0, float* o, float* S_T, int B, int T,
+                       int H, int Dk, int Dv, const gdn_options* opts, int* status, void* stream) {
+  int qk_norm = 0, o_bf16 = 0;
+  float q_scale = 1.f;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
+  const bool fused = qk_norm || q_scale != 1.f;
   // the row kernel validates every argument; at 128 x 128 with tokens to process
-  // the chunked tensor-core kernel runs instead (same validation first)
+  // the chunked tensor-core kernel runs instead (same validation first); the
+  // fused options exist on the tensor-core kernel only
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (fused && (Dk != kHeadDim || Dv != kHeadDim)) return GDN_ERR_UNSUPPORTED;
   if (Dk != kHeadDim || Dv != kHeadDim || T == 0 || (long long)B * H == 0)
     return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, true, stream);
   const long long chains = (long long)B * H;
@@ -595,7 +607,7 @@ int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
       !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, kHeadDim, 32) ||
       !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, kHeadDim, 32))
     return GDN_ERR_LAUNCH;
-  gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status};
+  gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status, qk_norm, q_scale};
   return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK
              : GDN_ERR_LAUNCH;
@@ -604,13 +616,24 @@ int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
 int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                    int* status, void* stream) {
+  return gdn_kda_decode_ex(q, k, v, g, beta, S, o, B, T, H, Dk, Dv, nullptr, status, stream);
+}
+
+int gdn_kda_decode_ex(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
+                      const gdn_options* opts, int* status, void* stream) {
   (void)status;  // the decode kernels have no device-side waits
+  int qk_norm = 0, o_bf16 = 0;
+  float q_scale = 1.f;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
+  const bool fused = qk_norm || q_scale != 1.f;
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (fused && (Dk != kHeadDim || Dv != kHeadDim)) return GDN_ERR_UNSUPPORTED;
   if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
   // Dk = Dv = 128 or 64: the streaming decode kernel; other head dims: the row
   // kernel (both read and write the state once per call)
   if (Dk == Dv && (Dk == kHeadDim || Dk == 64))
-    return decode_impl(q, k, v, g, beta, S, o, B, T, H, Dk, 0, 1.f, 0, true, 4, stream);
+    return decode_impl(q, k, v, g, beta, S, o, B, T, H, Dk, qk_norm, q_scale, 0, true, 4, stream);
   return rows_impl(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, true, stream);
 }
 

@@ -350,11 +350,17 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const unsigned grid_step = unsigned(heads * StepGeom<D>::CTAS_PER_HEAD);
   const unsigned grid_burst = unsigned(heads * CTAS_PER_HEAD);
   if (a.vector_gate) {
-    if (pre) return -1;  // the per-channel gate takes no fused options
-    if (a.T == 1)
-      decode_step_kernel<D, false, true><<<grid_step, WARPS * 32, 0, stream>>>(a);
-    else
-      decode_burst_kernel<false, true><<<grid_burst, WARPS * 32, 0, stream>>>(a);
+    if (a.T == 1) {
+      if (pre)
+        decode_step_kernel<D, true, true><<<grid_step, WARPS * 32, 0, stream>>>(a);
+      else
+        decode_step_kernel<D, false, true><<<grid_step, WARPS * 32, 0, stream>>>(a);
+    } else {
+      if (pre)
+        decode_burst_kernel<true, true><<<grid_burst, WARPS * 32, 0, stream>>>(a);
+      else
+        decode_burst_kernel<false, true><<<grid_burst, WARPS * 32, 0, stream>>>(a);
+    }
   } else if (a.T == 1) {
     if (pre)
       decode_step_kernel<D, true, false><<<grid_step, WARPS * 32, 0, stream>>>(a);

@@ -89,6 +89,8 @@ struct KdaArgs {
   float* S_T;         // may equal S0
   int B, T, H;
   int* status;        // may be null
+  int qk_norm;        // q, k L2-normalised per token and head in the kernel
+  float q_scale;      // q multiplied by this after the normalisation
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device

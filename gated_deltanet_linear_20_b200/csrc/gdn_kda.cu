@@ -243,6 +243,9 @@ __device__ __forceinline__ void issue_g(const Ctx& x, const CUtensorMap* tg, int
 // Thread kt: channel pair cp = kt % 64 (channels 2cp, 2cp+1) and token quarter
 // qt = kt / 64 (tokens 8qt .. 8qt+7 of the tile) for the gates and operands;
 // TMEM lane quarter (warp % 4) and column half for the masks.
+// PRE: q and k are L2-normalised per token and head (and q scaled) on the way
+// in, before any decay is applied.
+template <bool PRE>
 __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
                           const CUtensorMap* tg, const KdaArgs& p, int b, int h, int ntiles) {
   const int kt = threadIdx.x - 128;
@@ -345,6 +348,46 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
       // gate entries and read the exchange area, which the operands overwrite)
       if (!rs.agree(x, ok)) return;
       if (leader) mbar_arrive(x.bar(gfull_off(c)));
+      // with PRE, the per-token factors |k|^-1 and q_scale |q|^-1 of this
+      // thread's 8 tokens: sums of squares over the 64 threads of the token
+      // quarter (two warps: a shuffle reduction each, then the exchange area)
+      float kn[8], qn[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) kn[t] = qn[t] = 1.f;
+      if constexpr (PRE) {
+        if (p.qk_norm) {
+          const int half = (kt >> 5) & 1;
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const uint32_t ro = row_off(t);
+            const uint32_t kw = lds32<0>(sb + SM_KQ + tile_off(8192u) + ro);
+            const uint32_t qw = lds32<4096>(sb + SM_KQ + tile_off(8192u) + ro);
+            const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw));
+            const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw));
+            float sk = fmaf(kf.x, kf.x, kf.y * kf.y), sq = fmaf(qf.x, qf.x, qf.y * qf.y);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+              sk += __shfl_xor_sync(0xffffffffu, sk, off);
+              sq += __shfl_xor_sync(0xffffffffu, sq, off);
+            }
+            if ((kt & 31) == 0) {
+              sX[(qt * 2 + half) * 16 + 2 * t] = sk;
+              sX[(qt * 2 + half) * 16 + 2 * t + 1] = sq;
+            }
+          }
+          named_bar(BAR_SIDE, SIDE_THREADS);
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float sk = sX[(qt * 2) * 16 + 2 * t] + sX[(qt * 2 + 1) * 16 + 2 * t];
+            const float sq = sX[(qt * 2) * 16 + 2 * t + 1] + sX[(qt * 2 + 1) * 16 + 2 * t + 1];
+            kn[t] = rsqrtf(sk + 1e-6f);
+            qn[t] = rsqrtf(sq + 1e-6f) * p.q_scale;
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) qn[t] = p.q_scale;
+        }
+      }
       // per channel: Lambda_r (from the tile start) and Lambda_last / Lambda_r,
       // so that K+ = K' Lambda_r, Q+ = Q' Lambda_r and K~ = K'' Lambda_last / Lambda_r
       // take two exponentials per token and channel instead of four (products
@@ -367,7 +410,7 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
         const uint32_t kw = lds32<0>(kq_t + ro), qw = lds32<4096>(kq_t + ro);
         const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kw));
         const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw));
-        const float kv[2] = {kf.x, kf.y}, qv[2] = {qf.x, qf.y};
+        const float kv[2] = {kf.x * kn[t], kf.y * kn[t]}, qv[2] = {qf.x * qn[t], qf.y * qn[t]};
         float k1[2], q1[2], k2[2], kp[2], qp[2], kt2[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -759,6 +802,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
   }
 }
 
+template <bool PRE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -803,7 +847,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (warp < 4 || warp >= 12)
     chain_role(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
   else
-    side_role(x, &tm_q, &tm_k, &tm_g, p, b, h, ntiles);
+    side_role<PRE>(x, &tm_q, &tm_k, &tm_g, p, b, h, ntiles);
 
   // each MMA-issuing thread waits (bounded) for its own products in flight
   if (tid == 0 || tid == 128 || tid == OI_ISSUER) {
@@ -837,8 +881,13 @@ int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const int chains = a.B * a.H;
   if (chains == 0 || a.T == 0) return -1;
   const uint32_t smem = SMEM_USED + 1024;
-  if (!ensure_smem_attr(reinterpret_cast<const void*>(kda_prefill_kernel), 15, int(smem))) return -1;
-  kda_prefill_kernel<<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, tg, a);
+  if (a.qk_norm || a.q_scale != 1.f) {
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(kda_prefill_kernel<true>), 48, int(smem))) return -1;
+    kda_prefill_kernel<true><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, tg, a);
+  } else {
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(kda_prefill_kernel<false>), 15, int(smem))) return -1;
+    kda_prefill_kernel<false><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, tg, a);
+  }
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

@@ -64,10 +64,14 @@ _lib.gdn_kda_prefill.argtypes = [_vp] * 8 + [_ci] * 5 + [_vp, _vp]
 _lib.gdn_kda_prefill.restype = _ci
 _lib.gdn_kda_decode.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp]
 _lib.gdn_kda_decode.restype = _ci
+_lib.gdn_kda_prefill_ex.argtypes = [_vp] * 8 + [_ci] * 5 + [_vp, _vp, _vp]
+_lib.gdn_kda_prefill_ex.restype = _ci
+_lib.gdn_kda_decode_ex.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp, _vp]
+_lib.gdn_kda_decode_ex.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
-ABI_VERSION = 6
+ABI_VERSION = 7
 if _lib.gdn_abi_version() != ABI_VERSION:
     raise ImportError(f"libgdn_b200.so ABI {_lib.gdn_abi_version()} != binding ABI {ABI_VERSION}")
 
@@ -394,12 +398,15 @@ def query_status(status: torch.Tensor) -> int:
 def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                 beta: torch.Tensor, S0: Optional[torch.Tensor] = None, *,
                 o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
-                status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+                status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
+                q_scale: float = 1.0) -> Tuple[torch.Tensor, torch.Tensor]:
     """Per-channel-gate (KDA) prefill: returns (o [B,T,H,Dv] fp32, S_T [B,H,Dv,Dk] fp32).
 
     q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g [B,T,H,Dk] fp32 (log decay per key
     channel); beta [B,T,H] fp32; S0 [B,H,Dv,Dk] fp32 or None (zeros).  ``S_T``
-    may be ``S0`` (in place).  Launches on the current stream."""
+    may be ``S0`` (in place).  ``qk_l2norm`` / ``q_scale`` normalise q and k per
+    token and head and scale q inside the kernel (gdn_kda_prefill_ex; 128 x 128
+    only).  Launches on the current stream."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape
@@ -420,8 +427,13 @@ def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     if S_T is None:
         S_T = torch.empty((B, H, Dv, Dk), dtype=torch.float32, device=dev)
     _check(S_T, "S_T", torch.float32, (B, H, Dv, Dk), dev)
-    rc = _lib.gdn_kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                              _ptr(S_T), B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    opts = _options(qk_l2norm, q_scale)
+    if opts is None:
+        rc = _lib.gdn_kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                  _ptr(S_T), B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    else:
+        rc = _lib.gdn_kda_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                     _ptr(S_T), B, T, H, Dk, Dv, opts, _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_kda_prefill")
     return o, S_T
@@ -429,11 +441,13 @@ def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
 
 def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
-               status: Optional[torch.Tensor] = None) -> torch.Tensor:
+               status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
+               q_scale: float = 1.0) -> torch.Tensor:
     """Per-channel-gate (KDA) decode; S [B,H,Dv,Dk] fp32 is updated in place.
 
     One token: q, k [B,H,Dk], v [B,H,Dv], g [B,H,Dk], beta [B,H] -> o [B,H,Dv].
-    T tokens: the same with a T axis after B ([B,T,H,...]) -> o [B,T,H,Dv]."""
+    T tokens: the same with a T axis after B ([B,T,H,...]) -> o [B,T,H,Dv].
+    ``qk_l2norm`` / ``q_scale`` as for ``kda_prefill`` (gdn_kda_decode_ex)."""
     one = q.dim() == 3
     if one:
         q, k, v, g, beta = (x.unsqueeze(1) for x in (q, k, v, g, beta))
@@ -455,8 +469,13 @@ def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tenso
     if o is None:
         o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
     _check(o, "o", torch.float32, (B, T, H, Dv), dev)
-    rc = _lib.gdn_kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
-                             B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    opts = _options(qk_l2norm, q_scale)
+    if opts is None:
+        rc = _lib.gdn_kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                 B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
+    else:
+        rc = _lib.gdn_kda_decode_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                                    B, T, H, Dk, Dv, opts, _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_kda_decode")
     return o[:, 0] if one else o
@@ -502,3 +521,11 @@ def raw_kda_prefill(*args) -> int:
 
 def raw_kda_decode(*args) -> int:
     return int(_lib.gdn_kda_decode(*args))
+
+
+def raw_kda_prefill_ex(*args) -> int:
+    return int(_lib.gdn_kda_prefill_ex(*args))
+
+
+def raw_kda_decode_ex(*args) -> int:
+    return int(_lib.gdn_kda_decode_ex(*args))

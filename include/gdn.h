@@ -64,7 +64,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 6
+#define GDN_ABI_VERSION 7
 
 enum gdn_status_code {
   GDN_OK = 0,
@@ -82,7 +82,8 @@ enum gdn_status_code {
 /* Size of the library's built-in device scratch used by gdn_prefill_static_ws. */
 #define GDN_STATIC_WORKSPACE_BYTES (16u << 20)
 
-/* Optional pre-steps fused into the kernels (gdn_prefill_ex, gdn_decode_ex).
+/* Optional pre-steps fused into the kernels (gdn_prefill_ex, gdn_decode_ex,
+ * gdn_kda_prefill_ex, gdn_kda_decode_ex).
  *   size      : sizeof(gdn_options) (a smaller value is rejected)
  *   qk_l2norm : nonzero: q and k are L2-normalised per token and head before
  *               use, x^ = x / sqrt(sum_d x_d^2 + 1e-6), in fp32 from the bf16
@@ -310,6 +311,19 @@ int gdn_kda_prefill(const void* q, const void* k, const void* v, const float* g,
 int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                    int* status, void* stream);
+
+/* gdn_kda_prefill / gdn_kda_decode with options (gdn_options; NULL = none).
+ * qk_l2norm and q_scale are applied to each token's q and k before any decay,
+ * as in gdn_prefill_ex; they need Dk = Dv = 128 (else GDN_ERR_UNSUPPORTED).
+ * o_bf16 is not offered with the per-channel gate: a nonzero o_bf16 (or an
+ * invalid struct) returns GDN_ERR_UNSUPPORTED.  Everything else as for the
+ * calls without options. */
+int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float* g,
+                       const float* beta, const float* S0, float* o, float* S_T, int B, int T,
+                       int H, int Dk, int Dv, const gdn_options* opts, int* status, void* stream);
+int gdn_kda_decode_ex(const void* q, const void* k, const void* v, const float* g,
+                      const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
+                      const gdn_options* opts, int* status, void* stream);
 
 /* Synchronises `stream`, then reads the device status word written by the
  * kernels.  Returns GDN_OK, GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_NULL (status_dev is

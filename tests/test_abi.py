@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(gdn):
 
 
 def test_abi_version_and_status_strings(gdn):
-    assert gdn.abi_version() == 6
+    assert gdn.abi_version() == 7
     for code in range(-9, 1):
         s = gdn.status_str(code)
         assert s and s != "unknown status code"
@@ -393,3 +393,28 @@ def test_plain_c_client_links_and_gets_the_documented_codes(gdn, tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "0 failure(s)" in r.stdout
+
+
+def test_kda_options_validation(gdn):
+    """gdn_kda_prefill_ex / gdn_kda_decode_ex: the fused norm and q scale exist
+    at 128 x 128 only; o_bf16 and invalid structs are GDN_ERR_UNSUPPORTED; valid
+    options at 128 x 128 pass validation (then fail only for want of a device)."""
+    import ctypes as ct
+    good = gdn.Options(ct.sizeof(gdn.Options), 1, 0.5, 0)
+    bf16 = gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 1)
+    short = gdn.Options(4, 1, 1.0, 0)
+    a = kda_args()
+    ins = lambda args, o: args[:13] + [ct.byref(o)] + args[13:]
+    assert gdn.raw_kda_prefill_ex(*ins(a, good)) not in (0, -1, -2, -3, -4, -5)
+    assert gdn.raw_kda_prefill_ex(*ins(a, bf16)) == -4
+    assert gdn.raw_kda_prefill_ex(*ins(a, short)) == -4
+    assert gdn.raw_kda_prefill_ex(*ins(kda_args(Dk=64, Dv=64), good)) == -4
+    assert gdn.raw_kda_prefill_ex(*(a[:13] + [None] + a[13:])) not in (0, -1, -2, -3, -4, -5)
+    d = [P, P + 0x1000000, P + 0x2000000, P + 0x3000000, P + 0x3100000, P + 0x4000000,
+         P + 0x5000000, 4, 1, 2, 128, 128]
+    tail = [None, None]
+    assert gdn.raw_kda_decode_ex(*(d + [ct.byref(good)] + tail)) not in (0, -1, -2, -3, -4, -5)
+    assert gdn.raw_kda_decode_ex(*(d + [ct.byref(bf16)] + tail)) == -4
+    d64 = d[:10] + [64, 64]
+    assert gdn.raw_kda_decode_ex(*(d64 + [ct.byref(good)] + tail)) == -4
+    assert gdn.raw_kda_decode_ex(*(d64 + [None] + tail)) not in (0, -1, -2, -3, -4, -5)

@@ -230,3 +230,71 @@ def test_kda_prefill_then_decode_continue_one_state():
     ro, rS = oracle.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
     assert_parity(torch.cat([o1, o2], 1).cpu().numpy(), ro, "o prefill + decode")
     assert_parity(S.cpu().numpy(), rS, "S prefill + decode")
+
+
+def _raw_qk(d, seed):
+    """Un-normalised q, k (each token-head row scaled by a random factor in
+    [0.2, 5]) and their fp64 L2-normalised versions."""
+    rng = np.random.default_rng(seed)
+    out = {}
+    for key in ("q", "k"):
+        x = d[key].double()
+        scale = torch.from_numpy(rng.uniform(0.2, 5.0, size=x.shape[:-1] + (1,)))
+        raw = (x * scale).to(torch.bfloat16)
+        r64 = raw.double()
+        out[key] = raw
+        out[key + "_n"] = r64 / torch.sqrt((r64 * r64).sum(-1, keepdim=True) + 1e-6)
+    return out
+
+
+@pytest.mark.parametrize("norm,qs", [(True, 128 ** -0.5), (False, 0.5)], ids=["l2norm+scale", "scale"])
+def test_kda_fused_qk_norm_and_q_scale(norm, qs):
+    """The per-channel-gate prefill with q / k normalised and q scaled inside
+    the kernel (gdn_kda_prefill_ex) equals the oracle run on inputs normalised
+    in fp64 beforehand; T = 300 covers whole and ragged 32-token tiles."""
+    d = inputs.kda_inputs(2, 300, 3, seed=151, s0_std=0.05)
+    r = _raw_qk(d, 152) if norm else {"q": d["q"], "k": d["k"], "q_n": d["q"].double(), "k_n": d["k"].double()}
+    dd = to_dev(d)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gdn = _gdn()
+    o, S_T = gdn.kda_prefill(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], dd["S0"],
+                             status=status, qk_l2norm=norm, q_scale=qs)
+    assert gdn.query_status(status) == 0
+    ro, rS = oracle.kda_prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, "o (fused norm)")
+    assert_parity(S_T.cpu().numpy(), rS, "S_T (fused norm)")
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_kda_fused_qk_norm_in_decode(T):
+    d = inputs.kda_inputs(4, T, 8, seed=160 + T, s0_std=0.05)
+    r = _raw_qk(d, 161)
+    qs = 0.5
+    gdn = _gdn()
+    dd = to_dev(d)
+    S = dd["S0"].clone()
+    o = gdn.kda_decode(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], S,
+                       qk_l2norm=True, q_scale=qs)
+    torch.cuda.synchronize()
+    ro, rS = oracle.kda_prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o T={T}")
+    assert_parity(S.cpu().numpy(), rS, f"S T={T}")
+
+
+def test_kda_default_options_are_bitwise_the_plain_call():
+    """Default options through gdn_kda_prefill_ex run the same kernel as the
+    plain call: bitwise the same results."""
+    import ctypes as ct
+    gdn = _gdn()
+    d = to_dev(inputs.kda_inputs(2, 100, 3, seed=171, s0_std=0.02))
+    o1, S1 = gdn.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    o2 = torch.empty_like(o1)
+    S2 = torch.empty_like(S1)
+    opts = gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 0)
+    rc = gdn.raw_kda_prefill_ex(*[ct.c_void_p(t.data_ptr()) for t in (d["q"], d["k"], d["v"], d["g"],
+                                                                       d["beta"], d["S0"], o2, S2)],
+                                2, 100, 3, 128, 128, ct.byref(opts), None,
+                                ct.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
