@@ -509,6 +509,21 @@ def run_extras(args, dev, stream, flush, peaks, rank):
     e1.record(stream)
     torch.cuda.synchronize()
     t_warm = e0.elapsed_time(e1) / wd.decode_steps
+    # the same 256 steps captured once as a CUDA graph and replayed: no host launch
+    # between steps (each step still one kernel launch inside the graph)
+    graph = torch.cuda.CUDAGraph()
+    it[0] = 0
+    with torch.cuda.graph(graph):
+        for _ in range(wd.decode_steps):
+            dstep()
+    graph.replay()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_graph = e0.elapsed_time(e1) / wd.decode_steps
+    del graph
     traffic = committed_traffic("decode_b64_h16", DECODE_SOURCES)
     copy_us = copy_reference_us(wd.B * wd.H * STATE_BYTES, dev, flush, stream)
     out["decode_b64_h16"] = {
@@ -522,7 +537,11 @@ def run_extras(args, dev, stream, flush, peaks, rank):
         "frac_of_copy": round(copy_us / (t * 1e3), 4),
         "back_to_back_256_steps": {"us_per_step": round(t_warm * 1e3, 3),
                                    "state_GB_per_s": round(sb / (t_warm / 1e3) / 1e9, 1),
-                                   "l2": "warm: the 64 MiB state fits in the 126 MB L2"}}
+                                   "l2": "warm: the 64 MiB state fits in the 126 MB L2"},
+        "cuda_graph_256_steps": {"us_per_step": round(t_graph * 1e3, 3),
+                                 "state_GB_per_s": round(sb / (t_graph / 1e3) / 1e9, 1),
+                                 "l2": "warm, as back_to_back_256_steps",
+                                 "note": "256 steps captured once in a CUDA graph, replayed"}}
     del dd, S
     # a 4-token burst per sequence in one call (state read and written once)
     dt = gin.prefill_inputs(wd.B, 4, wd.H, seed=2500 + rank, s0_std=0.02, device=str(dev))
