@@ -255,11 +255,14 @@ int prefill_impl(const void* q, const void* k, const void* v, const float* g, co
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if (chunk != 16 && chunk != 64) return GDN_ERR_UNSUPPORTED;
   if (Dk != kHeadDim || Dv != kHeadDim) {
-    // other head dims: no fused options; Dk = 256 takes the row kernel (its fp32
-    // state and bf16 hi/lo copy alone would fill the 512 TMEM columns)
-    if (qk_norm || q_scale != 1.f || o_bf16) return GDN_ERR_UNSUPPORTED;
+    // other head dims: Dk = 64 or 128 run the chunked tensor-core kernel, with the
+    // fused options; Dk = 256 takes the row kernel (its fp32 state and bf16 hi/lo
+    // copy alone would fill the 512 TMEM columns), which has none
     if (!gdn::rows_head_dims_ok(Dk, Dv)) return GDN_ERR_UNSUPPORTED;
-    if (Dk == 256) return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, false, stream);
+    if (Dk == 256) {
+      if (qk_norm || q_scale != 1.f || o_bf16) return GDN_ERR_UNSUPPORTED;
+      return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, false, stream);
+    }
     allow_segments = false;  // the segmented schedule is built for 128 x 128 states
   }
   const long long chains = (long long)B * H;
@@ -373,7 +376,7 @@ const char* gdn_status_str(int code) {
     case GDN_ERR_NULL: return "a required pointer is NULL";
     case GDN_ERR_ALIGN: return "misaligned pointer (q/k/v/o/S need 16 bytes, g/beta 4 bytes)";
     case GDN_ERR_SHAPE: return "negative size or problem larger than 2^31-1 elements";
-    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options and packed sequences at 128 x 128 only; chunk 16 or 64; device sm_100)";
+    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options not with Dk = 256, nor in decode outside 64 x 64 and 128 x 128, nor in the per-channel-gate prefill outside 128 x 128, and no bf16 o with the per-channel gate; packed sequences at 128 x 128 only; chunk 16 or 64; device sm_100)";
     case GDN_ERR_ALIAS: return "output overlaps an input";
     case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
     case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
@@ -545,13 +548,14 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
   if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
   if (B < 0 || H < 0 || T < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || Dv != kHeadDim) {
-    // other head dims: no fused options; 64 x 64 streams through the decode
-    // kernel, the rest through the row kernel, the state in place
-    if (!gdn::rows_head_dims_ok(Dk, Dv) || qk_norm || q_scale != 1.f || o_bf16)
-      return GDN_ERR_UNSUPPORTED;
+    // other head dims: 64 x 64 streams through the decode kernel (with the fused
+    // options), the rest through the row kernel (without), the state in place
+    if (!gdn::rows_head_dims_ok(Dk, Dv)) return GDN_ERR_UNSUPPORTED;
     if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
     if (Dk == 64 && Dv == 64)
-      return decode_impl(q, k, v, g, beta, S, o, B, T, H, 64, 0, 1.f, 0, false, 4, stream);
+      return decode_impl(q, k, v, g, beta, S, o, B, T, H, 64, qk_norm, q_scale, o_bf16, false, 4,
+                         stream);
+    if (qk_norm || q_scale != 1.f || o_bf16) return GDN_ERR_UNSUPPORTED;
     return rows_impl(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, false, stream);
   }
   return decode_impl(q, k, v, g, beta, S, o, B, T, H, kHeadDim, qk_norm, q_scale, o_bf16, false,
@@ -628,7 +632,7 @@ int gdn_kda_decode_ex(const void* q, const void* k, const void* v, const float* 
   if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
   const bool fused = qk_norm || q_scale != 1.f;
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
-  if (fused && (Dk != kHeadDim || Dv != kHeadDim)) return GDN_ERR_UNSUPPORTED;
+  if (fused && !(Dk == Dv && (Dk == kHeadDim || Dk == 64))) return GDN_ERR_UNSUPPORTED;
   if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
   // Dk = Dv = 128 or 64: the streaming decode kernel; other head dims: the row
   // kernel (both read and write the state once per call)

@@ -337,13 +337,19 @@ int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const long long heads = (long long)a.B * a.H;
   if (heads == 0) return 0;
   const bool pre = a.qk_norm || a.q_scale != 1.f;
-  if (a.head_dim == 64) {  // the step kernel at any T; no fused options
-    if (pre) return -1;
+  if (a.head_dim == 64) {  // the step kernel at any T
     const unsigned grid = unsigned(heads * StepGeom<64>::CTAS_PER_HEAD);
-    if (a.vector_gate)
-      decode_step_kernel<64, false, true><<<grid, WARPS * 32, 0, stream>>>(a);
-    else
-      decode_step_kernel<64, false, false><<<grid, WARPS * 32, 0, stream>>>(a);
+    if (a.vector_gate) {
+      if (pre)
+        decode_step_kernel<64, true, true><<<grid, WARPS * 32, 0, stream>>>(a);
+      else
+        decode_step_kernel<64, false, true><<<grid, WARPS * 32, 0, stream>>>(a);
+    } else {
+      if (pre)
+        decode_step_kernel<64, true, false><<<grid, WARPS * 32, 0, stream>>>(a);
+      else
+        decode_step_kernel<64, false, false><<<grid, WARPS * 32, 0, stream>>>(a);
+    }
     return cudaGetLastError() == cudaSuccess ? 0 : -1;
   }
   if (a.head_dim != D) return -1;

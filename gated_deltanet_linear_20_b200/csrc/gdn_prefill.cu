@@ -336,9 +336,11 @@ __device__ __forceinline__ void solve_distance(int kt, const float* sAt, float* 
 // chain has released tile c-1's T and Mq, writes T(c), Mq(c).
 // |k_j|^-1 and q_scale |q_i|^-1 of tile c into its gate buffer (all side
 // threads; with normalisation off, just 1 and q_scale).  Thread t sums the
-// squares of half a row of [K; Q] (64 bf16 in one 128-byte SW128 row: the
-// chunk order of the swizzle does not matter for a sum) and the two halves
-// meet by a shuffle.  x^ = x / sqrt(sum x^2 + 1e-6).
+// squares of half a row of [K; Q] (Dk = 128: the 64 bf16 of one 128-byte SW128
+// row; Dk = 64: half of the row's one 128-byte line; the chunk order of the
+// swizzle does not matter for a sum) and the two halves meet by a shuffle.
+// x^ = x / sqrt(sum x^2 + 1e-6).
+template <int DK>
 __device__ __forceinline__ void side_norms(const Ctx& x, int kt, int c, const PrefillArgs& p) {
   float* G = x.gates(c);
   if (!p.qk_norm) {
@@ -350,11 +352,14 @@ __device__ __forceinline__ void side_norms(const Ctx& x, int kt, int c, const Pr
   }
   const int r = kt >> 1, hf = kt & 1;  // row of [K; Q] (0..63 K, 64..127 Q), dk half
   const int rr = r & (NT - 1);
+  // Dk = 128: half hf is the box of dk 64 hf ..; Dk = 64: the 16-byte chunks
+  // 4 hf .. 4 hf + 3 of the row's line
   const uint32_t row = x.sb + ((c & 1) ? SM_KQ1 : SM_KQ0) + (r < NT ? 0u : 8192u) +
-                       (hf ? 16384u : 0u) + uint32_t(rr >> 3) * 1024u + uint32_t(rr & 7) * 128u;
+                       (DK == 128 ? (hf ? 16384u : 0u) : 64u * uint32_t(hf)) +
+                       uint32_t(rr >> 3) * 1024u + uint32_t(rr & 7) * 128u;
   float ss = 0.f;
 #pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {
+  for (int ch = 0; ch < DK / 16; ++ch) {
     uint32_t w[4];
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
@@ -462,7 +467,7 @@ __device__ __noinline__ void store_partial_tile(const float4* src, float* dst, i
 // tile; the leader then stores the tile with TMA (tokens at or past T are
 // dropped by the copy).  Before the next tile's staging is written the leader
 // waits for the copy to have read it (at the next tile's first agreement).
-// OBF: o is bf16 (tile rows of 256 B, stored through a bf16 view).
+// OBF: o is bf16 (tile rows of 2 DVB bytes, stored through a bf16 view).
 template <bool OBF, int DVB>
 __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b, int h, int dv,
                                              int hf, int c, bool leader) {
@@ -483,9 +488,10 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
       for (int e = 0; e < 4; ++e) {
         const int n = 32 * hf + 16 * q + 4 * e4 + e;  // token within the tile
         const float ov = fmaf(gv[e], y[4 * e4 + e], oi[4 * e4 + e]);
+        if (!own) continue;
         if constexpr (OBF)
-          so16[n * D] = __float2bfloat16_rn(ov);
-        else if (own)
+          so16[n * DVB] = __float2bfloat16_rn(ov);
+        else
           so[n * DVB] = ov;
       }
     }
@@ -538,7 +544,7 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
   if constexpr (PRE) {
     if (p.qk_norm && !rs.wait(x, x.bar(B_FULL0), 0)) return;  // the norms read tile 0
-    side_norms(x, kt, 0, p);
+    side_norms<DK>(x, kt, 0, p);
     named_bar(BAR_SIDE, SIDE_THREADS);
   }
   side_gates<C, PRE>(x, kt, 0, T, g_next, b_next, p, b, h, s_part);
@@ -655,7 +661,7 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       if constexpr (PRE) {
         if (p.qk_norm && !rs.wait(x, x.bar(((c + 1) & 1) ? B_FULL1 : B_FULL0), ((c + 1) >> 1) & 1))
           return;
-        side_norms(x, kt, c + 1, p);
+        side_norms<DK>(x, kt, c + 1, p);
         named_bar(BAR_SIDE, SIDE_THREADS);
       }
       side_gates<C, PRE, false>(x, kt, c + 1, T, g_next, b_next, p, b, h, s_part);
@@ -1284,19 +1290,34 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   };
   const bool obf = a.o_bf16 != 0;
   bool ok;
-  if (a.Dk != D || a.Dv != D) {  // plain calls only: no fused options at other head dims
-    if (pre || obf) return -1;
-    const bool c64 = chunk == 64;
-    if (a.Dk == D)  // Dv = 64 (Dv = 256 runs the 128 x 128 kernel on two CTAs per chain)
-      ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 128, 128>, 0)
-                                : go(prefill_kernel<16, false, false, 128, 128>, 1))
-                         : (c64 ? go(prefill_kernel<64, false, false, 128, 64>, 9)
-                                : go(prefill_kernel<16, false, false, 128, 64>, 10));
+  if (a.Dk == D && a.dv_box == D && a.Dv != D) {
+    // Dv = 256: the 128 x 128 kernels on two CTAs per chain (rows dv0 .. dv0 + 127)
+    if (chunk == 64)
+      ok = obf ? (pre ? go(prefill_kernel<64, true, true, 128, 128>, 5) : go(prefill_kernel<64, false, true, 128, 128>, 6))
+               : (pre ? go(prefill_kernel<64, true, false, 128, 128>, 3) : go(prefill_kernel<64, false, false, 128, 128>, 0));
     else
-      ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 64, 128>, 11)
-                                : go(prefill_kernel<16, false, false, 64, 128>, 12))
-                         : (c64 ? go(prefill_kernel<64, false, false, 64, 64>, 13)
-                                : go(prefill_kernel<16, false, false, 64, 64>, 14));
+      ok = obf ? (pre ? go(prefill_kernel<16, true, true, 128, 128>, 7) : go(prefill_kernel<16, false, true, 128, 128>, 8))
+               : (pre ? go(prefill_kernel<16, true, false, 128, 128>, 4) : go(prefill_kernel<16, false, false, 128, 128>, 1));
+  } else if (a.Dk != D || a.Dv != D) {
+    // Dk = 64 or Dv = 64: the pre-steps are always compiled in (with none
+    // requested their factors are exactly 1, so the result is the plain one);
+    // bf16 o is a separate instantiation
+    const bool c64 = chunk == 64;
+    if (a.Dk == D)  // Dv = 64
+      ok = obf ? (c64 ? go(prefill_kernel<64, true, true, 128, 64>, 49)
+                      : go(prefill_kernel<16, true, true, 128, 64>, 50))
+               : (c64 ? go(prefill_kernel<64, true, false, 128, 64>, 9)
+                      : go(prefill_kernel<16, true, false, 128, 64>, 10));
+    else if (a.dv_box == D)  // Dk = 64, Dv = 128
+      ok = obf ? (c64 ? go(prefill_kernel<64, true, true, 64, 128>, 51)
+                      : go(prefill_kernel<16, true, true, 64, 128>, 52))
+               : (c64 ? go(prefill_kernel<64, true, false, 64, 128>, 11)
+                      : go(prefill_kernel<16, true, false, 64, 128>, 12));
+    else  // Dk = Dv = 64
+      ok = obf ? (c64 ? go(prefill_kernel<64, true, true, 64, 64>, 53)
+                      : go(prefill_kernel<16, true, true, 64, 64>, 54))
+               : (c64 ? go(prefill_kernel<64, true, false, 64, 64>, 13)
+                      : go(prefill_kernel<16, true, false, 64, 64>, 14));
   } else if (chunk == 64) {
     if (obf)
       ok = pre ? go(prefill_kernel<64, true, true, 128, 128>, 5) : go(prefill_kernel<64, false, true, 128, 128>, 6);

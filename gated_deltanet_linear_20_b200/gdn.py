@@ -160,8 +160,8 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
     bf16 (the fp32 value rounded to nearest even); it runs the single pass.
     Dk, Dv may each be 64, 128 or 256.  With Dk = 64 or 128 the chunked
     tensor-core kernel runs (Dv = 256 on two CTAs per chain); with Dk = 256 the
-    row-parallel fp32 kernel.  Segments and the fused options apply at 128 x 128
-    only."""
+    row-parallel fp32 kernel.  Segments apply at 128 x 128 only; the fused
+    options on the tensor-core kernel (not with Dk = 256)."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape
@@ -322,7 +322,9 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     """One decode step; S [B,H,Dv,Dk] fp32 is updated in place.  Returns o [B,H,Dv]
     (fp32, or bf16 with ``o_bf16``).
 
-    q, k [B,H,Dk] bf16; v [B,H,Dv] bf16; g, beta [B,H] fp32."""
+    q, k [B,H,Dk] bf16; v [B,H,Dv] bf16; g, beta [B,H] fp32.  The fused options
+    (``qk_l2norm``, ``q_scale``, ``o_bf16``; gdn_decode_ex) need Dk = Dv = 128
+    or 64."""
     if q.dim() != 3:
         raise ValueError("q must be [B,H,Dk]")
     B, H, Dk = q.shape
@@ -360,7 +362,8 @@ def decode_tokens(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Te
     place (read and written once).  Returns o [B,T,H,Dv] (fp32, or bf16 with
     ``o_bf16``).
 
-    q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g, beta [B,T,H] fp32."""
+    q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g, beta [B,T,H] fp32.  The fused
+    options need Dk = Dv = 128 or 64."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape
@@ -447,7 +450,8 @@ def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tenso
 
     One token: q, k [B,H,Dk], v [B,H,Dv], g [B,H,Dk], beta [B,H] -> o [B,H,Dv].
     T tokens: the same with a T axis after B ([B,T,H,...]) -> o [B,T,H,Dv].
-    ``qk_l2norm`` / ``q_scale`` as for ``kda_prefill`` (gdn_kda_decode_ex)."""
+    ``qk_l2norm`` / ``q_scale`` as for ``kda_prefill`` (gdn_kda_decode_ex; 128 x 128
+    or 64 x 64)."""
     one = q.dim() == 3
     if one:
         q, k, v, g, beta = (x.unsqueeze(1) for x in (q, k, v, g, beta))

@@ -40,7 +40,10 @@
  *     GDN_ERR_NULL         a required pointer is NULL
  *     GDN_ERR_ALIGN        q/k/v/o/S pointers must be 16-byte aligned, g/beta 4-byte
  *     GDN_ERR_SHAPE        a size is negative or the problem exceeds 2^31-1 elements
- *     GDN_ERR_UNSUPPORTED  a head dim not in {64, 128, 256}; fused options or
+ *     GDN_ERR_UNSUPPORTED  a head dim not in {64, 128, 256}; fused options where
+ *                          the kernel serving the head dims has none (prefill
+ *                          with Dk = 256; decode outside 64 x 64 and 128 x 128;
+ *                          the per-channel-gate prefill outside 128 x 128);
  *                          packed sequences at head dims other than 128 x 128;
  *                          chunk not in {16, 64}; or the current device is not
  *                          compute capability 10.0
@@ -178,7 +181,8 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
 /* gdn_prefill_ws with options (gdn_options above; NULL = none); with a NULL
  * workspace it runs the single pass of gdn_prefill.  Invalid options (size
  * too small, q_scale NaN) return GDN_ERR_UNSUPPORTED, and so do non-default
- * options at head dims other than 128 x 128. */
+ * options with Dk = 256 (the row kernel; every head-dim pair with Dk = 64 or
+ * 128 runs the chunked tensor-core kernel, which has them). */
 int gdn_prefill_ex(const void* q, const void* k, const void* v, const float* g,
                    const float* beta, const float* S0, float* o, float* S_T, int B, int T, int H,
                    int Dk, int Dv, int chunk, void* workspace, size_t workspace_bytes,
@@ -269,7 +273,8 @@ int gdn_decode_tokens(const void* q, const void* k, const void* v, const float* 
                       int* status, void* stream);
 
 /* gdn_decode_tokens with options (gdn_options; NULL = none).  Non-default
- * options need Dk = Dv = 128 (else GDN_ERR_UNSUPPORTED). */
+ * options need Dk = Dv = 128 or Dk = Dv = 64, the dims the streaming decode
+ * kernels serve (else GDN_ERR_UNSUPPORTED). */
 int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
                   const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                   const gdn_options* opts, int* status, void* stream);
@@ -314,7 +319,8 @@ int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
 
 /* gdn_kda_prefill / gdn_kda_decode with options (gdn_options; NULL = none).
  * qk_l2norm and q_scale are applied to each token's q and k before any decay,
- * as in gdn_prefill_ex; they need Dk = Dv = 128 (else GDN_ERR_UNSUPPORTED).
+ * as in gdn_prefill_ex; they need Dk = Dv = 128 in the prefill, and 128 x 128
+ * or 64 x 64 in decode (else GDN_ERR_UNSUPPORTED).
  * o_bf16 is not offered with the per-channel gate: a nonzero o_bf16 (or an
  * invalid struct) returns GDN_ERR_UNSUPPORTED.  Everything else as for the
  * calls without options. */

@@ -78,9 +78,12 @@ int main(void) {
   opts.qk_l2norm = 1;
   opts.q_scale = 1.f;
   opts.o_bf16 = 0;
-  check(gdn_decode_ex(q, k, v, g, beta, S, o, 4, 1, 2, 64, 64, &opts, NULL, NULL) ==
+  check(gdn_decode_ex(q, k, v, g, beta, S, o, 4, 1, 2, 64, 128, &opts, NULL, NULL) ==
             GDN_ERR_UNSUPPORTED,
-        "decode_ex: fused options at 64 x 64 are GDN_ERR_UNSUPPORTED");
+        "decode_ex: fused options at 64 x 128 (row kernel) are GDN_ERR_UNSUPPORTED");
+  check(gdn_prefill_ex(q, k, v, g, beta, NULL, o, S, 1, 64, 2, 256, 256, 64, NULL, 0, &opts, NULL,
+                       NULL) == GDN_ERR_UNSUPPORTED,
+        "prefill_ex: fused options with Dk = 256 (row kernel) are GDN_ERR_UNSUPPORTED");
   opts.size = 4;
   check(gdn_decode_ex(q, k, v, g, beta, S, o, 4, 1, 2, 128, 128, &opts, NULL, NULL) ==
             GDN_ERR_UNSUPPORTED,

@@ -363,14 +363,29 @@ def test_other_head_dims_pass_validation(gdn, dk, dv):
     assert gdn.raw_kda_decode(*kd) not in VALIDATION_CODES + (0,)
 
 
-def test_other_head_dims_reject_fused_options(gdn):
-    """The fused q/k norm, q scale and bf16 o exist on the 128 x 128 kernels only."""
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 256)])
+def test_fused_options_pass_validation_on_the_tensor_core_dims(gdn, dk, dv):
+    """Prefill with Dk = 64 or 128 runs the chunked tensor-core kernel, which has
+    the fused q/k norm, q scale and bf16 o: valid options pass validation (and
+    then fail only for want of a device)."""
+    import ctypes as ct
+    for opts in (gdn.Options(ct.sizeof(gdn.Options), 1, 0.5, 0), gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 1)):
+        a = prefill_args(Dk=dk, Dv=dv)
+        assert gdn.raw_prefill_ex(*(a[:14] + [None, 0, ct.byref(opts)] + a[14:])) not in VALIDATION_CODES + (0,)
+
+
+def test_row_kernel_dims_reject_fused_options(gdn):
+    """The row kernel (prefill with Dk = 256; decode outside 64 x 64 and
+    128 x 128) has no fused options; the 64 x 64 decode has them."""
     import ctypes as ct
     opts = gdn.Options(ct.sizeof(gdn.Options), 1, 1.0, 0)
-    a = prefill_args(Dk=64, Dv=64)
+    a = prefill_args(Dk=256, Dv=256)
     assert gdn.raw_prefill_ex(*(a[:14] + [None, 0, ct.byref(opts)] + a[14:])) == -4
-    d = decode_tokens_args(Dk=256, Dv=256)
-    assert gdn.raw_decode_ex(*(d[:12] + [ct.byref(opts)] + d[12:])) == -4
+    for dk, dv in ((256, 256), (64, 128), (128, 64)):
+        d = decode_tokens_args(Dk=dk, Dv=dv)
+        assert gdn.raw_decode_ex(*(d[:12] + [ct.byref(opts)] + d[12:])) == -4
+    d = decode_tokens_args(Dk=64, Dv=64)
+    assert gdn.raw_decode_ex(*(d[:12] + [ct.byref(opts)] + d[12:])) not in VALIDATION_CODES + (0,)
 
 
 def test_other_head_dims_size_the_overlap_checks(gdn):
@@ -397,8 +412,9 @@ def test_plain_c_client_links_and_gets_the_documented_codes(gdn, tmp_path):
 
 def test_kda_options_validation(gdn):
     """gdn_kda_prefill_ex / gdn_kda_decode_ex: the fused norm and q scale exist
-    at 128 x 128 only; o_bf16 and invalid structs are GDN_ERR_UNSUPPORTED; valid
-    options at 128 x 128 pass validation (then fail only for want of a device)."""
+    at 128 x 128 in the prefill, and at 128 x 128 and 64 x 64 in decode; o_bf16
+    and invalid structs are GDN_ERR_UNSUPPORTED; valid options where they exist
+    pass validation (then fail only for want of a device)."""
     import ctypes as ct
     good = gdn.Options(ct.sizeof(gdn.Options), 1, 0.5, 0)
     bf16 = gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 1)
@@ -416,5 +432,7 @@ def test_kda_options_validation(gdn):
     assert gdn.raw_kda_decode_ex(*(d + [ct.byref(good)] + tail)) not in (0, -1, -2, -3, -4, -5)
     assert gdn.raw_kda_decode_ex(*(d + [ct.byref(bf16)] + tail)) == -4
     d64 = d[:10] + [64, 64]
-    assert gdn.raw_kda_decode_ex(*(d64 + [ct.byref(good)] + tail)) == -4
+    assert gdn.raw_kda_decode_ex(*(d64 + [ct.byref(good)] + tail)) not in (0, -1, -2, -3, -4, -5)
     assert gdn.raw_kda_decode_ex(*(d64 + [None] + tail)) not in (0, -1, -2, -3, -4, -5)
+    d64x128 = d[:10] + [64, 128]
+    assert gdn.raw_kda_decode_ex(*(d64x128 + [ct.byref(good)] + tail)) == -4

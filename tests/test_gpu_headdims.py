@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from gated_deltanet_linear_20_b200 import inputs
-from tests.test_gpu_parity import DEV, assert_parity, to_dev
+from tests.test_gpu_parity import DEV, assert_parity, raw_qk, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -177,9 +177,109 @@ def test_tensor_core_head_dims_many_chains_sampled():
         assert_parity(S_T[b, h], rS[b, h], f"S_T chain {c}")
 
 
-def test_other_head_dims_reject_fused_options_on_gpu():
+def test_row_kernel_dims_reject_fused_options_on_gpu():
+    """Dk = 256 (the row kernel) has no fused options; nor has decode outside
+    64 x 64 and 128 x 128."""
     gdn = _gdn()
-    d = to_dev(inputs.prefill_inputs(1, 16, 2, 64, 64, seed=22))
+    d = to_dev(inputs.prefill_inputs(1, 16, 2, 256, 256, seed=22))
     with pytest.raises(gdn.GDNError) as e:
         gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], qk_l2norm=True)
     assert e.value.code == gdn.GDN_ERR_UNSUPPORTED
+    e2 = to_dev(inputs.prefill_inputs(2, 1, 2, 64, 128, seed=23, s0_std=0.02))
+    with pytest.raises(gdn.GDNError) as e:
+        gdn.decode_tokens(e2["q"], e2["k"], e2["v"], e2["g"], e2["beta"], e2["S0"].clone(), q_scale=0.5)
+    assert e.value.code == gdn.GDN_ERR_UNSUPPORTED
+
+
+TC_DIMS = [(64, 64), (64, 128), (128, 64), (128, 256)]
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+@pytest.mark.parametrize("dk,dv", TC_DIMS, ids=[f"{a}x{b}" for a, b in TC_DIMS])
+def test_fused_options_tensor_core_head_dims(dk, dv, chunk):
+    """q / k L2 normalisation and the q scale fused into the tensor-core kernel
+    at the other head dims equal the oracle run on inputs normalised in fp64
+    beforehand; bf16 o is the fp32 o rounded to nearest even, bit for bit, with
+    the same end state.  T = 150 leaves a ragged last tile."""
+    gdn = _gdn()
+    d = inputs.prefill_inputs(2, 150, 3, dk, dv, seed=400 + dk + dv + chunk, s0_std=0.05)
+    r = raw_qk(d, 401 + dk + dv)
+    qs = dk ** -0.5
+    dd = to_dev(d)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.prefill(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], dd["S0"],
+                         chunk=chunk, qk_l2norm=True, q_scale=qs, status=status)
+    assert gdn.query_status(status) == 0
+    ro, rS = oracle.prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"], d["beta"],
+                            d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o (fused norm) {dk}x{dv}")
+    assert_parity(S_T.cpu().numpy(), rS, f"S_T (fused norm) {dk}x{dv}")
+    o16, S16 = gdn.prefill(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], dd["S0"],
+                           chunk=chunk, qk_l2norm=True, q_scale=qs, o_bf16=True, status=status)
+    assert gdn.query_status(status) == 0
+    assert o16.dtype == torch.bfloat16
+    assert torch.equal(o16, o.to(torch.bfloat16))
+    assert torch.equal(S16, S_T)
+
+
+@pytest.mark.parametrize("dk,dv", TC_DIMS, ids=[f"{a}x{b}" for a, b in TC_DIMS])
+def test_default_options_are_bitwise_the_plain_call_at_other_head_dims(dk, dv):
+    """Default options through gdn_prefill_ex give bitwise the plain call's
+    results (at these dims the plain call runs the kernel with the pre-steps
+    compiled in, their factors exactly 1)."""
+    import ctypes as ct
+    gdn = _gdn()
+    B, T, H = 2, 130, 3
+    d = to_dev(inputs.prefill_inputs(B, T, H, dk, dv, seed=420 + dk + dv, s0_std=0.02))
+    o1, S1 = gdn.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], segmented=False)
+    o2 = torch.empty_like(o1)
+    S2 = torch.empty_like(S1)
+    opts = gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 0)
+    rc = gdn.raw_prefill_ex(*[ct.c_void_p(t.data_ptr()) for t in (d["q"], d["k"], d["v"], d["g"],
+                                                                    d["beta"], d["S0"], o2, S2)],
+                            B, T, H, dk, dv, 64, None, ct.c_size_t(0), ct.byref(opts), None,
+                            ct.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert rc == 0 and torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_fused_options_in_decode_64(T):
+    """The 64 x 64 streaming decode with q / k normalised and q scaled in the
+    kernel equals the oracle on fp64-normalised inputs; its bf16 o is the fp32
+    o rounded, bit for bit."""
+    gdn = _gdn()
+    d = inputs.prefill_inputs(4, T, 8, 64, 64, seed=440 + T, s0_std=0.05)
+    r = raw_qk(d, 441)
+    qs = 0.5
+    dd = to_dev(d)
+    S = dd["S0"].clone()
+    o = gdn.decode_tokens(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], S,
+                          qk_l2norm=True, q_scale=qs)
+    torch.cuda.synchronize()
+    ro, rS = oracle.prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"], d["beta"],
+                            d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o T={T}")
+    assert_parity(S.cpu().numpy(), rS, f"S T={T}")
+    S2 = dd["S0"].clone()
+    o16 = gdn.decode_tokens(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], S2,
+                            qk_l2norm=True, q_scale=qs, o_bf16=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, o.to(torch.bfloat16)) and torch.equal(S2, S)
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_kda_fused_options_in_decode_64(T):
+    gdn = _gdn()
+    d = inputs.kda_inputs(4, T, 8, 64, 64, seed=450 + T, s0_std=0.05)
+    r = raw_qk(d, 451)
+    qs = 0.5
+    dd = to_dev(d)
+    S = dd["S0"].clone()
+    o = gdn.kda_decode(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], S,
+                       qk_l2norm=True, q_scale=qs)
+    torch.cuda.synchronize()
+    ro, rS = oracle.kda_prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"],
+                                d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o T={T}")
+    assert_parity(S.cpu().numpy(), rS, f"S T={T}")
