@@ -376,7 +376,7 @@ const char* gdn_status_str(int code) {
     case GDN_ERR_NULL: return "a required pointer is NULL";
     case GDN_ERR_ALIGN: return "misaligned pointer (q/k/v/o/S need 16 bytes, g/beta 4 bytes)";
     case GDN_ERR_SHAPE: return "negative size or problem larger than 2^31-1 elements";
-    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options not with Dk = 256, nor in decode outside 64 x 64 and 128 x 128, nor in the per-channel-gate prefill outside 128 x 128, and no bf16 o with the per-channel gate; packed sequences at 128 x 128 only; chunk 16 or 64; device sm_100)";
+    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options not with Dk = 256, nor in decode outside 64 x 64 and 128 x 128, nor in the per-channel-gate prefill outside 128 x 128, and no bf16 o with the per-channel gate; packed sequences not with Dk = 256; chunk 16 or 64; device sm_100)";
     case GDN_ERR_ALIAS: return "output overlaps an input";
     case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
     case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
@@ -437,11 +437,15 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
                        int chunk, float* snaps, int snap_every, int n_snaps, int* status,
                        void* stream) {
   if (N < 0 || total_T < 0 || H < 0 || n_snaps < 0) return GDN_ERR_SHAPE;
-  if (Dk != kHeadDim || Dv != kHeadDim || (chunk != 16 && chunk != 64)) return GDN_ERR_UNSUPPORTED;
+  // the chunked tensor-core kernel's head dims: Dk 64 or 128, Dv 64, 128 or 256
+  if ((Dk != 64 && Dk != kHeadDim) || !gdn::rows_head_dims_ok(Dk, Dv) ||
+      (chunk != 16 && chunk != 64))
+    return GDN_ERR_UNSUPPORTED;
   if (snaps && (snap_every <= 0 || snap_every % 64 != 0)) return GDN_ERR_UNSUPPORTED;
   const long long chains = (long long)N * H;
-  const long long act = (long long)total_T * H * kHeadDim;
-  if (act > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL) return GDN_ERR_SHAPE;
+  const long long act_k = (long long)total_T * H * Dk, act_v = (long long)total_T * H * Dv;
+  if (act_k > 0x7fffffffLL || act_v > 0x7fffffffLL || chains * Dk * Dv > 0x7fffffffLL)
+    return GDN_ERR_SHAPE;
   if (chains == 0) return GDN_OK;
   if (!S_T || !cu_seqlens) return GDN_ERR_NULL;
   if (total_T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
@@ -449,48 +453,51 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
   if (total_T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
                       !aligned(g, 4) || !aligned(beta, 4)))
     return GDN_ERR_ALIGN;
-  const size_t act_bf16 = size_t(act) * 2, act_f32 = size_t(act) * 4;
+  const size_t act_bf16 = size_t(act_k) * 2, v_bf16 = size_t(act_v) * 2, act_f32 = size_t(act_v) * 4;
   const size_t gate_bytes = size_t(total_T) * H * 4;
-  const size_t state_bytes = size_t(chains) * kHeadDim * kHeadDim * 4, cu_bytes = size_t(N + 1) * 4;
+  const size_t state_bytes = size_t(chains) * Dk * Dv * 4, cu_bytes = size_t(N + 1) * 4;
   if (total_T > 0 && (overlaps(o, act_f32, q, act_bf16) || overlaps(o, act_f32, k, act_bf16) ||
-                      overlaps(o, act_f32, v, act_bf16) || overlaps(o, act_f32, g, gate_bytes) ||
+                      overlaps(o, act_f32, v, v_bf16) || overlaps(o, act_f32, g, gate_bytes) ||
                       overlaps(o, act_f32, beta, gate_bytes) || overlaps(o, act_f32, S0, state_bytes) ||
                       overlaps(o, act_f32, S_T, state_bytes) || overlaps(o, act_f32, cu_seqlens, cu_bytes)))
     return GDN_ERR_ALIAS;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
   if (overlaps(S_T, state_bytes, cu_seqlens, cu_bytes)) return GDN_ERR_ALIAS;
   if (total_T > 0 && (overlaps(S_T, state_bytes, q, act_bf16) || overlaps(S_T, state_bytes, k, act_bf16) ||
-                      overlaps(S_T, state_bytes, v, act_bf16) || overlaps(S_T, state_bytes, g, gate_bytes) ||
+                      overlaps(S_T, state_bytes, v, v_bf16) || overlaps(S_T, state_bytes, g, gate_bytes) ||
                       overlaps(S_T, state_bytes, beta, gate_bytes)))
     return GDN_ERR_ALIAS;
   if (snaps) {
-    const size_t snap_bytes = size_t(n_snaps) * H * kHeadDim * kHeadDim * 4;
+    const size_t snap_bytes = size_t(n_snaps) * H * Dk * Dv * 4;
     if (!aligned(snaps, 16)) return GDN_ERR_ALIGN;
     if ((total_T > 0 && overlaps(snaps, snap_bytes, o, act_f32)) ||
         overlaps(snaps, snap_bytes, S_T, state_bytes) || overlaps(snaps, snap_bytes, S0, state_bytes) ||
         overlaps(snaps, snap_bytes, cu_seqlens, cu_bytes) ||
         (total_T > 0 && (overlaps(snaps, snap_bytes, q, act_bf16) || overlaps(snaps, snap_bytes, k, act_bf16) ||
-                         overlaps(snaps, snap_bytes, v, act_bf16) || overlaps(snaps, snap_bytes, g, gate_bytes) ||
+                         overlaps(snaps, snap_bytes, v, v_bf16) || overlaps(snaps, snap_bytes, g, gate_bytes) ||
                          overlaps(snaps, snap_bytes, beta, gate_bytes))))
       return GDN_ERR_ALIAS;
   }
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
 
-  // B = N chains of sequences, T = total_T: the views are [1][total_T][H][128]
+  // B = N chains of sequences, T = total_T: the views are [1][total_T][H][Dk or Dv]
+  const int dv_box = Dv < kHeadDim ? Dv : kHeadDim;
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
                      H,      status, 1,      (total_T + 63) / 64, 1, nullptr, nullptr, nullptr,
                      cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, 0, 1.f, 0,
-                     kHeadDim, kHeadDim, 1, kHeadDim};
+                     Dk,     Dv,   Dv / dv_box, dv_box};
   CUtensorMap tq{}, tk{}, tv{}, to{};
-  const int Tv = total_T > 0 ? total_T : 1;  // a valid (never read) view when every sequence is empty
+  // a valid (never read) view when every sequence is empty: S_T holds at least
+  // one token's worth of any of these rows (Dk Dv >= Dk, Dv)
+  const int Tv = total_T > 0 ? total_T : 1;
   const void* qv = total_T > 0 ? q : S_T;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  if (!encode_act(&tq, qv, 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
-      !encode_act(&tk, total_T > 0 ? k : S_T, 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2) ||
-      !encode_act(&tv, total_T > 0 ? v : S_T, 1, Tv, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2) ||
-      !encode_act(&to, total_T > 0 ? static_cast<const void*>(o) : S_T, 1, Tv, H, 128,
-                  CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4))
+  if (!encode_act(&tq, qv, 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, Dk) ||
+      !encode_act(&tk, total_T > 0 ? k : S_T, 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, Dk) ||
+      !encode_act(&tv, total_T > 0 ? v : S_T, 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv) ||
+      !encode_act(&to, total_T > 0 ? static_cast<const void*>(o) : S_T, 1, Tv, H, dv_box,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, Dv))
     return GDN_ERR_LAUNCH;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   return gdn::launch_prefill(tq, tk, tv, to, to, a, chunk, st) == 0 ? GDN_OK : GDN_ERR_LAUNCH;

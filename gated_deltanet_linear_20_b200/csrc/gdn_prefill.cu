@@ -195,6 +195,7 @@ struct Ctx {
   const CUtensorMap* tmo;  // TMA view of odst: [B][T][H][128] fp32, box 64 tokens x 128
   float* sdst;         // destination of the end state rows owned by this CTA
   int dv0;             // first state row (value channel) owned by this CTA
+  int dvw;             // value channels per head (Dv): o's row width, the state's rows
   __device__ __forceinline__ uint32_t bar(uint32_t off) const { return sb + SM_BAR + off; }
   __device__ __forceinline__ float* gates(int c) const {
     return reinterpret_cast<float*>(sm + SM_GATES + (c % GATE_BUFS) * GATE_BYTES);
@@ -450,15 +451,16 @@ __device__ __forceinline__ void issue_p(const Ctx& x, int c) {
   mma_commit(x.bar(B_PFULL));
 }
 
-// Copies rows 0 .. nvalid-1 of the staged fp32 o tile (rows of 128 floats) to
-// dst (row r at dst + r H 128), thread ct of the chain role taking every
+// Copies rows 0 .. nvalid-1 of the staged fp32 o tile (rows of DVB floats) to
+// dst (row r at dst + r rowstride), thread ct of the chain role taking every
 // CHAIN_THREADS-th 16-byte chunk.  Kept out of line: it runs only for the last
 // tile of a packed sequence.
-__device__ __noinline__ void store_partial_tile(const float4* src, float* dst, int H, int nvalid,
-                                                int ct) {
-  for (int i = ct; i < nvalid * (D / 4); i += CHAIN_THREADS) {
-    const int r = i / (D / 4), j = i % (D / 4);
-    reinterpret_cast<float4*>(dst + size_t(r) * H * D)[j] = src[i];
+template <int DVB>
+__device__ __noinline__ void store_partial_tile(const float4* src, float* dst, size_t rowstride,
+                                                int nvalid, int ct) {
+  for (int i = ct; i < nvalid * (DVB / 4); i += CHAIN_THREADS) {
+    const int r = i / (DVB / 4), j = i % (DVB / 4);
+    reinterpret_cast<float4*>(dst + size_t(r) * rowstride)[j] = src[i];
   }
 }
 
@@ -508,9 +510,9 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
   } else if constexpr (!OBF) {
     // last tile of a packed sequence (packed calls take fp32 o only): the rows
     // past it belong to the next sequence, so only the valid rows are copied out
-    store_partial_tile(reinterpret_cast<const float4*>(x.sm + SM_XH),
-                       x.odst + ((size_t(b) * x.tmap + ts) * x.H + h) * D, x.H, x.tend - ts,
-                       hf * 128 + dv);
+    store_partial_tile<DVB>(reinterpret_cast<const float4*>(x.sm + SM_XH),
+                            x.odst + ((size_t(b) * x.tmap + ts) * x.H + h) * x.dvw + x.dv0,
+                            size_t(x.H) * x.dvw, x.tend - ts, hf * 128 + dv);
   }
 }
 
@@ -707,13 +709,17 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
-// Copies columns col0 .. col0+63 of this lane's state row (fp32, TMEM) to
-// dst_row + col0.  Out of line: it runs only at snapshot tile ends.
-__device__ __noinline__ void snapshot_row(uint32_t tlane, int col0, float* dst_row) {
+// Copies columns col0 .. col0 + 32 NQ - 1 of this lane's state row (fp32,
+// TMEM) to dst_row + col0 (own: the lane holds one of the CTA's rows; the
+// loads are warp-wide either way).  Out of line: it runs only at snapshot tile
+// ends.
+template <int NQ>
+__device__ __noinline__ void snapshot_row(uint32_t tlane, int col0, float* dst_row, bool own) {
 #pragma unroll 1
-  for (int q = 0; q < 2; ++q) {
+  for (int q = 0; q < NQ; ++q) {
     float v[32];
     tmem_ld32(tlane + TM_S + col0 + 32 * q, v);
+    if (!own) continue;
 #pragma unroll
     for (int e = 0; e < 8; ++e)
       reinterpret_cast<float4*>(dst_row + col0 + 32 * q)[e] =
@@ -1024,22 +1030,28 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           gnext = x.gates(c + 1)[G_GC / 4];
         }
         if (final_chunk && (DK != D || DVB != D)) {
-          // other head dims: this thread's columns of its own row, straight to HBM
-          if (DVB == D || dv < DVB) {
-            float4* dst = reinterpret_cast<float4*>(x.sdst + size_t(dv) * DK + SCOLS * ch);
+          // other head dims: this thread's columns of its own row, straight to HBM,
+          // and into the last snapshot slot when the packed sequence ends on one
+          // (the loads are warp-wide; lanes past the CTA's rows store nothing)
+          const bool own = DVB == D || dv < DVB;
+          float4* dst = reinterpret_cast<float4*>(x.sdst + size_t(dv) * DK + SCOLS * ch);
+          float4* sdst = nullptr;
+          const int stiles = *x.misc(M_SNAP_TILES);
+          if (stiles && (x.tend - x.tok0) % (stiles * NT) == 0)
+            sdst = reinterpret_cast<float4*>(
+                *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR) +
+                size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * x.dvw * DK + size_t(dv) * DK +
+                SCOLS * ch);
 #pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-              float v[32];
-              tmem_ld32(tlane + TM_S + SCOLS * ch + 32 * q, v);
+          for (int q = 0; q < NQ; ++q) {
+            float v[32];
+            tmem_ld32(tlane + TM_S + SCOLS * ch + 32 * q, v);
+            if (!own) continue;
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                dst[8 * q + e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {  // keep the warp's TMEM loads convergent
-              float v[32];
-              tmem_ld32(tlane + TM_S + SCOLS * ch + 32 * q, v);
+            for (int e = 0; e < 8; ++e) {
+              const float4 w = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+              dst[8 * q + e] = w;
+              if (sdst) sdst[8 * q + e] = w;
             }
           }
         } else if (final_chunk) {
@@ -1067,7 +1079,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
             // the sequence ends on a snapshot boundary: its last snapshot is S_T
             float* snap = *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR);
             copy_staged_state(x.sm + SM_XH,
-                              snap + size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * D * D,
+                              snap + size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * x.dvw * DK,
                               ch * 128 + dv);
           }
         } else {
@@ -1076,7 +1088,9 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
             const int stiles = *x.misc(M_SNAP_TILES);
             if (stiles && (c + 1) % stiles == 0) {
               float* snap = *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR);
-              snapshot_row(tlane, 64 * ch, snap + (size_t((c + 1) / stiles - 1) * x.H * D + dv) * D);
+              snapshot_row<NQ>(tlane, SCOLS * ch,
+                               snap + size_t((c + 1) / stiles - 1) * x.H * x.dvw * DK + size_t(dv) * DK,
+                               DVB == D || dv < DVB);
             }
           }
           // this thread's DK / 2 columns, 32 at a time: load, split, store hi / lo /
@@ -1151,6 +1165,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   x.tend = p.T;
   x.tmap = p.T;
   x.dv0 = dv0;
+  x.dvw = p.Dv;
   int ntiles = total_tiles;
   if (p.cu_seqlens) {
     // packed sequences: chain = n H + h walks tokens [cu[n], cu[n+1]) of views with B = 1
@@ -1163,10 +1178,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     x.tend = end;
     b = 0;
     ntiles = (end - start + NT - 1) / NT;
-    if (ntiles == 0) {  // empty sequence: S_T = S0 (or zeros)
-      const float4* src = p.S0 ? reinterpret_cast<const float4*>(p.S0 + cstate) : nullptr;
-      float4* dst = reinterpret_cast<float4*>(p.S_T + cstate);
-      for (int i = tid; i < D * D / 4; i += NTHREADS)
+    if (ntiles == 0) {  // empty sequence: S_T = S0 (or zeros), this CTA's rows
+      const size_t off = cstate + size_t(dv0) * DK;
+      const float4* src = p.S0 ? reinterpret_cast<const float4*>(p.S0 + off) : nullptr;
+      float4* dst = reinterpret_cast<float4*>(p.S_T + off);
+      for (int i = tid; i < p.dv_box * DK / 4; i += NTHREADS)
         dst[i] = src ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
       return;
     }
@@ -1212,7 +1228,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (p.status) atomicExch(p.status, GDN_ERR_SHAPE);
       } else {
         *reinterpret_cast<float* volatile*>(sm + SM_MISC + M_SNAP_PTR) =
-            p.snaps + (size_t(base) * p.H + h) * D * D;
+            p.snaps + (size_t(base) * p.H + h) * p.Dv * DK + size_t(dv0) * DK;
         *x.misc(M_SNAP_TILES) = p.snap_every / NT;
       }
     }

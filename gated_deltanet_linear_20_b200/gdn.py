@@ -234,7 +234,8 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     With ``snap_every`` (a multiple of 64) it also returns the state snapshots
     [n_snaps,H,Dv,Dk] (after every snap_every tokens of each sequence, sequence
     by sequence); ``snaps`` may be given preallocated, else its size is read
-    from cu_seqlens (one device-to-host copy)."""
+    from cu_seqlens (one device-to-host copy).  Dk 64 or 128, Dv 64, 128 or
+    256 (the chunked tensor-core kernel)."""
     if q.dim() != 3:
         raise ValueError("q must be [total_T,H,Dk]")
     total_T, H, Dk = q.shape

@@ -44,7 +44,7 @@
  *                          the kernel serving the head dims has none (prefill
  *                          with Dk = 256; decode outside 64 x 64 and 128 x 128;
  *                          the per-channel-gate prefill outside 128 x 128);
- *                          packed sequences at head dims other than 128 x 128;
+ *                          packed sequences with Dk = 256;
  *                          chunk not in {16, 64}; or the current device is not
  *                          compute capability 10.0
  *     GDN_ERR_ALIAS        o or S_T overlaps an input, or o overlaps the state
@@ -170,8 +170,9 @@ size_t gdn_prefill_workspace_bytes(int B, int T, int H, int Dk, int Dv, int chun
  *                sequence whose slots would pass it, or that follows a
  *                sequence with invalid offsets, gets none, and GDN_ERR_SHAPE
  *                goes to *status.
- * Dk, Dv must be 128 (packed sequences run on the chunked tensor-core kernel
- * only).  chunk, status, stream and the other rules as for gdn_prefill. */
+ * Dk must be 64 or 128 and Dv 64, 128 or 256: packed sequences run on the
+ * chunked tensor-core kernel only (not on the Dk = 256 row kernel).  chunk,
+ * status, stream and the other rules as for gdn_prefill. */
 int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
                        const float* beta, const float* S0, float* o, float* S_T,
                        const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,

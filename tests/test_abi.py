@@ -162,7 +162,8 @@ def varlen_args(**over):
 
 
 @pytest.mark.parametrize("over,code", [
-    (dict(N=-1), -3), (dict(total_T=-1), -3), (dict(Dk=64), -4), (dict(chunk=8), -4),
+    (dict(N=-1), -3), (dict(total_T=-1), -3), (dict(Dk=256), -4), (dict(Dv=32), -4),
+    (dict(chunk=8), -4),
     (dict(cu=None), -1), (dict(S_T=None), -1), (dict(q=None), -1),
     (dict(cu=P + 0x60000002), -2), (dict(o=P + 0x40000008), -2),
     (dict(o=P + 0x60000000 - 64), -5),          # o runs into cu_seqlens
@@ -176,6 +177,21 @@ def varlen_args(**over):
 ], ids=lambda x: str(x))
 def test_prefill_varlen_rejects_bad_arguments(gdn, over, code):
     assert gdn.raw_prefill_varlen(*varlen_args(**over)) == code
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 256), (64, 256)])
+def test_prefill_varlen_other_head_dims_pass_validation(gdn, dk, dv):
+    """Packed sequences run on the chunked tensor-core kernel at every Dk of 64
+    or 128: valid calls pass validation (then fail only for want of a device)."""
+    assert gdn.raw_prefill_varlen(*varlen_args(Dk=dk, Dv=dv)) not in VALIDATION_CODES + (0,)
+
+
+def test_prefill_varlen_overlap_checks_follow_the_head_dims(gdn):
+    """3 sequences x 2 heads of 128 x 256 fp32 states take 768 KiB: an S_T that
+    starts 768 KiB - 16 B before cu_seqlens runs into it, at 128 x 128 it does not."""
+    s_t = P + 0x60000000 - 6 * 128 * 256 * 4 + 16
+    assert gdn.raw_prefill_varlen(*varlen_args(S_T=s_t, Dk=128, Dv=256)) == -5
+    assert gdn.raw_prefill_varlen(*varlen_args(S_T=s_t)) not in VALIDATION_CODES + (0,)
 
 
 def test_prefill_varlen_no_sequences_is_a_noop(gdn):

@@ -10,6 +10,7 @@ fp32 kernel.  The contract and the
 """
 from __future__ import annotations
 
+import numpy as np
 import pytest
 import torch
 
@@ -283,3 +284,71 @@ def test_kda_fused_options_in_decode_64(T):
                                 d["beta"], d["S0"])
     assert_parity(o.cpu().numpy(), ro, f"o T={T}")
     assert_parity(S.cpu().numpy(), rS, f"S T={T}")
+
+
+def _packed(lengths, H, dk, dv, seed, s0_std=None):
+    """Packed inputs of sequences of the given lengths at head dims dk x dv:
+    per-sequence draws of the seeded generator, concatenated along tokens."""
+    seqs = [inputs.prefill_inputs(1, L, H, dk, dv, seed=seed + i, s0_std=s0_std)
+            for i, L in enumerate(lengths)]
+    cat = lambda key: torch.cat([d[key][0] for d in seqs], 0)
+    S0 = torch.cat([d["S0"] for d in seqs], 0) if s0_std else None
+    cu = torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32)
+    return seqs, dict(q=cat("q"), k=cat("k"), v=cat("v"), g=cat("g"), beta=cat("beta"), S0=S0, cu=cu)
+
+
+VARLEN_DIMS = [(64, 64), (64, 128), (128, 64), (128, 256), (64, 256)]
+
+
+@pytest.mark.parametrize("chunk", [64, 16])
+@pytest.mark.parametrize("dk,dv", VARLEN_DIMS, ids=[f"{a}x{b}" for a, b in VARLEN_DIMS])
+def test_varlen_packed_sequences_other_head_dims(dk, dv, chunk):
+    """Packed sequences of mixed lengths (empty, 1 token, ragged, tile-aligned)
+    at the tensor-core head dims, each against the oracle run on that sequence
+    alone; an empty sequence's S_T is its S0."""
+    lengths = [130, 0, 1, 64, 77]
+    H = 2
+    seqs, pk = _packed(lengths, H, dk, dv, seed=500 + dk + dv, s0_std=0.05)
+    gdn = _gdn()
+    dd = to_dev(pk)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"], dd["S0"],
+                                chunk=chunk, status=status)
+    assert gdn.query_status(status) == 0
+    o, S_T = o.cpu().numpy(), S_T.cpu().numpy()
+    cu = pk["cu"].numpy()
+    for n, d in enumerate(seqs):
+        ro, rS = oracle.prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+        if lengths[n]:
+            assert_parity(o[cu[n]:cu[n + 1]], ro[0], f"o seq {n} (len {lengths[n]})")
+        assert_parity(S_T[n], rS[0], f"S_T seq {n} (len {lengths[n]})")
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 256), (64, 128)], ids=["64x64", "128x256", "64x128"])
+def test_varlen_state_snapshots_other_head_dims(dk, dv):
+    """Snapshots after every 64 tokens of each sequence equal the oracle's state
+    on that prefix (a sequence of 128 tokens ends on a snapshot: its last one is
+    its S_T); the outputs equal those of the call without snapshots."""
+    lengths = [130, 64, 0, 128]
+    H = 2
+    seqs, pk = _packed(lengths, H, dk, dv, seed=530 + dk + dv, s0_std=0.05)
+    gdn = _gdn()
+    dd = to_dev(pk)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T, snaps = gdn.prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"],
+                                       dd["S0"], status=status, snap_every=64)
+    assert gdn.query_status(status) == 0
+    assert tuple(snaps.shape) == (sum(L // 64 for L in lengths), H, dv, dk)
+    sn = snaps.cpu().numpy()
+    slot = 0
+    for n, d in enumerate(seqs):
+        for j in range(1, lengths[n] // 64 + 1):
+            t = 64 * j
+            cut = lambda x: x[:, :t]
+            _, rS = oracle.prefill(cut(d["q"]), cut(d["k"]), cut(d["v"]), cut(d["g"]), cut(d["beta"]),
+                                   d["S0"])
+            assert_parity(sn[slot], rS[0], f"snapshot {j} of seq {n} (t={t})")
+            slot += 1
+    o2, S2 = gdn.prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"], dd["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(S_T, S2)
