@@ -138,7 +138,8 @@ constexpr uint32_t M_TMEM = 0, M_ABORT = 4, M_PART = 8, M_KQ_ISSUED = 12, M_KQ_S
                    M_V_ISSUED = 20, M_V_SEEN = 24, M_FLAG_CHAIN = 32,
                    M_FLAG_SIDE = 40,  // two verdict slots per role
                    M_SNAP_TILES = 48,  // tiles between state snapshots (0: none)
-                   M_SNAP_PTR = 56;    // this chain's first snapshot slot (8 bytes)
+                   M_SNAP_PTR = 56,    // this chain's first snapshot slot (8 bytes)
+                   M_OROW = 64;        // o's row width (Dv), set at start
 static_assert(M_SNAP_PTR + 8 <= 64, "misc slots (the first 64 bytes are cleared at start)");
 static_assert(8 * NUM_BARS <= 256, "barrier slots");
 
@@ -195,7 +196,6 @@ struct Ctx {
   const CUtensorMap* tmo;  // TMA view of odst: [B][T][H][128] fp32, box 64 tokens x 128
   float* sdst;         // destination of the end state rows owned by this CTA
   int dv0;             // first state row (value channel) owned by this CTA
-  int dvw;             // value channels per head (Dv): o's row width, the state's rows
   __device__ __forceinline__ uint32_t bar(uint32_t off) const { return sb + SM_BAR + off; }
   __device__ __forceinline__ float* gates(int c) const {
     return reinterpret_cast<float*>(sm + SM_GATES + (c % GATE_BUFS) * GATE_BYTES);
@@ -470,7 +470,7 @@ __device__ __noinline__ void store_partial_tile(const float4* src, float* dst, s
 // dropped by the copy).  Before the next tile's staging is written the leader
 // waits for the copy to have read it (at the next tile's first agreement).
 // OBF: o is bf16 (tile rows of 2 DVB bytes, stored through a bf16 view).
-template <bool OBF, int DVB>
+template <bool OBF, int DVB, bool PK>
 __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b, int h, int dv,
                                              int hf, int c, bool leader) {
   const float* G = x.gates(c);
@@ -507,12 +507,12 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
       tma_store_4d(x.tmo, x.sb + SM_XH, x.dv0, h, ts, b);
       bulk_commit();
     }
-  } else if constexpr (!OBF) {
+  } else if constexpr (!OBF && PK) {
     // last tile of a packed sequence (packed calls take fp32 o only): the rows
     // past it belong to the next sequence, so only the valid rows are copied out
     store_partial_tile<DVB>(reinterpret_cast<const float4*>(x.sm + SM_XH),
-                            x.odst + ((size_t(b) * x.tmap + ts) * x.H + h) * x.dvw + x.dv0,
-                            size_t(x.H) * x.dvw, x.tend - ts, hf * 128 + dv);
+                            x.odst + ((size_t(b) * x.tmap + ts) * x.H + h) * *x.misc(M_OROW) + x.dv0,
+                            size_t(x.H) * *x.misc(M_OROW), x.tend - ts, hf * 128 + dv);
   }
 }
 
@@ -709,12 +709,23 @@ __device__ void kside_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
-// Copies columns col0 .. col0 + 32 NQ - 1 of this lane's state row (fp32,
-// TMEM) to dst_row + col0 (own: the lane holds one of the CTA's rows; the
-// loads are warp-wide either way).  Out of line: it runs only at snapshot tile
-// ends.
+// Copies columns col0 .. col0+63 of this lane's state row (fp32, TMEM) to
+// dst_row + col0.  Out of line: it runs only at snapshot tile ends.
+__device__ __noinline__ void snapshot_row(uint32_t tlane, int col0, float* dst_row) {
+#pragma unroll 1
+  for (int q = 0; q < 2; ++q) {
+    float v[32];
+    tmem_ld32(tlane + TM_S + col0 + 32 * q, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      reinterpret_cast<float4*>(dst_row + col0 + 32 * q)[e] =
+          make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+  }
+}
+// The same for the other head dims: NQ groups of 32 columns (own: the lane
+// holds one of the CTA's rows; the loads are warp-wide either way).
 template <int NQ>
-__device__ __noinline__ void snapshot_row(uint32_t tlane, int col0, float* dst_row, bool own) {
+__device__ __noinline__ void snapshot_row_n(uint32_t tlane, int col0, float* dst_row, bool own) {
 #pragma unroll 1
   for (int q = 0; q < NQ; ++q) {
     float v[32];
@@ -768,7 +779,7 @@ __device__ __forceinline__ void issue_zq(const Ctx& x, uint32_t kq, int s) {
 }
 
 // ============================================================== chain
-template <int C, bool OBF, int DK, int DVB>
+template <int C, bool OBF, int DK, int DVB, bool PK>
 __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
                            const CUtensorMap* tv, const PrefillArgs& p, int chain, int b, int h,
                            int ntiles) {
@@ -1015,7 +1026,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       // ---- the last tile: o first (its staging area then holds the end state)
       if (last_tile && s == NSUB - 1) {
         if (!rs.wait(x, x.bar(B_OI), sc & 1)) return;
-        output_drain<OBF, DVB>(x, tlane, b, h, dv, ch, c, leader);
+        output_drain<OBF, DVB, PK>(x, tlane, b, h, dv, ch, c, leader);
       }
 
       // ---- S_out now sits in TMEM: refresh its hi/lo copy, and pre-scale it by
@@ -1036,11 +1047,11 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           const bool own = DVB == D || dv < DVB;
           float4* dst = reinterpret_cast<float4*>(x.sdst + size_t(dv) * DK + SCOLS * ch);
           float4* sdst = nullptr;
-          const int stiles = *x.misc(M_SNAP_TILES);
+          const int stiles = PK ? *x.misc(M_SNAP_TILES) : 0;
           if (stiles && (x.tend - x.tok0) % (stiles * NT) == 0)
             sdst = reinterpret_cast<float4*>(
                 *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR) +
-                size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * x.dvw * DK + size_t(dv) * DK +
+                size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * p.Dv * DK + size_t(dv) * DK +
                 SCOLS * ch);
 #pragma unroll
           for (int q = 0; q < NQ; ++q) {
@@ -1074,23 +1085,26 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           }
           named_bar(BAR_CHAIN, CHAIN_THREADS);
           copy_staged_state(x.sm + SM_XH, x.sdst, ch * 128 + dv);
-          const int stiles = *x.misc(M_SNAP_TILES);
+          const int stiles = PK ? *x.misc(M_SNAP_TILES) : 0;
           if (stiles && (x.tend - x.tok0) % (stiles * NT) == 0) {
             // the sequence ends on a snapshot boundary: its last snapshot is S_T
             float* snap = *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR);
             copy_staged_state(x.sm + SM_XH,
-                              snap + size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * x.dvw * DK,
+                              snap + size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * p.Dv * D,
                               ch * 128 + dv);
           }
         } else {
           // at a snapshot tile end, the state itself first goes to its slot
-          if (s == NSUB - 1) {
+          if (PK && s == NSUB - 1) {
             const int stiles = *x.misc(M_SNAP_TILES);
             if (stiles && (c + 1) % stiles == 0) {
               float* snap = *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR);
-              snapshot_row<NQ>(tlane, SCOLS * ch,
-                               snap + size_t((c + 1) / stiles - 1) * x.H * x.dvw * DK + size_t(dv) * DK,
-                               DVB == D || dv < DVB);
+              if constexpr (DK == D && DVB == D)
+                snapshot_row(tlane, 64 * ch, snap + (size_t((c + 1) / stiles - 1) * x.H * p.Dv + dv) * D);
+              else
+                snapshot_row_n<NQ>(tlane, SCOLS * ch,
+                                   snap + size_t((c + 1) / stiles - 1) * x.H * p.Dv * DK + size_t(dv) * DK,
+                                   DVB == D || dv < DVB);
             }
           }
           // this thread's DK / 2 columns, 32 at a time: load, split, store hi / lo /
@@ -1116,7 +1130,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
       if (s == NSUB - 1 && !last_tile) {
         tc_fence_before();
         if (!rs.wait(x, x.bar(B_OI), sc & 1)) return;
-        output_drain<OBF, DVB>(x, tlane, b, h, dv, ch, c, leader);
+        output_drain<OBF, DVB, PK>(x, tlane, b, h, dv, ch, c, leader);
       }
       tc_fence_before();
       if (!rs.check(x)) return;
@@ -1124,7 +1138,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
   }
 }
 
-template <int C, bool PRE, bool OBF, int DK, int DVB>
+template <int C, bool PRE, bool OBF, int DK, int DVB, bool PK = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -1165,9 +1179,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   x.tend = p.T;
   x.tmap = p.T;
   x.dv0 = dv0;
-  x.dvw = p.Dv;
   int ntiles = total_tiles;
-  if (p.cu_seqlens) {
+  if (PK) {
     // packed sequences: chain = n H + h walks tokens [cu[n], cu[n+1]) of views with B = 1
     const int start = __ldg(p.cu_seqlens + b), end = __ldg(p.cu_seqlens + b + 1);
     if (start < 0 || end < start || end > p.T) {
@@ -1208,7 +1221,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(x.sb + SM_BAR + 8 * i, 1);
     fence_mbar_init();
     for (int i = 0; i < 16; ++i) reinterpret_cast<volatile int*>(sm + SM_MISC)[i] = 0;
-    if (p.snaps && p.cu_seqlens) {
+    if (PK) *reinterpret_cast<volatile int*>(sm + SM_MISC + M_OROW) = p.Dv;
+    if (PK && p.snaps) {
       // first snapshot slot of this sequence: one per snap_every tokens of
       // every earlier sequence; an invalid earlier entry (its own CTAs report
       // it) leaves this sequence without snapshots rather than with a slot
@@ -1246,7 +1260,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // for this grid to complete before it reads anything this grid writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (warp < 4 || warp >= 12)
-    chain_role<C, OBF, DK, DVB>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
+    chain_role<C, OBF, DK, DVB, PK>(x, &tm_q, &tm_k, &tm_v, p, chain, b, h, ntiles);
   else
     kside_role<C, PRE, DK, DVB>(x, &tm_q, &tm_k, &tm_v, p, b, h, ntiles);
 
@@ -1306,7 +1320,21 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   };
   const bool obf = a.o_bf16 != 0;
   bool ok;
-  if (a.Dk == D && a.dv_box == D && a.Dv != D) {
+  if (a.cu_seqlens) {
+    // packed sequences (fp32 o, no pre-steps): their own instantiations, so that the
+    // dense kernels carry none of the per-sequence paths
+    const bool c64 = chunk == 64;
+    if (a.Dk == D)
+      ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 128, 128, true>, 55)
+                                : go(prefill_kernel<16, false, false, 128, 128, true>, 56))
+                         : (c64 ? go(prefill_kernel<64, false, false, 128, 64, true>, 57)
+                                : go(prefill_kernel<16, false, false, 128, 64, true>, 58));
+    else
+      ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 64, 128, true>, 59)
+                                : go(prefill_kernel<16, false, false, 64, 128, true>, 60))
+                         : (c64 ? go(prefill_kernel<64, false, false, 64, 64, true>, 61)
+                                : go(prefill_kernel<16, false, false, 64, 64, true>, 62));
+  } else if (a.Dk == D && a.dv_box == D && a.Dv != D) {
     // Dv = 256: the 128 x 128 kernels on two CTAs per chain (rows dv0 .. dv0 + 127)
     if (chunk == 64)
       ok = obf ? (pre ? go(prefill_kernel<64, true, true, 128, 128>, 5) : go(prefill_kernel<64, false, true, 128, 128>, 6))
