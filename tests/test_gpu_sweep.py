@@ -8,7 +8,10 @@ under a second.  What the sweep varies, per entry point:
     gate strength (logsigmoid(N(mu, 1)), mu in {-3, 0, 2});
   * gdn_kda_prefill: B, H, T, with or without S0, the same gate strengths;
   * gdn_decode_tokens / gdn_kda_decode: B, H, T in 1 .. 6, head dims 64 / 128;
-  * gdn_prefill_varlen: 1 .. 5 packed sequences of 0 .. 200 tokens.
+  * gdn_prefill_varlen: 1 .. 5 packed sequences of 0 .. 200 tokens, at 128 x 128
+    and at the other tensor-core head dims;
+  * the fused options (q/k L2 norm with a q scale, bf16 o) at the tensor-core
+    head dims, prefill and decode.
 """
 from __future__ import annotations
 
@@ -18,7 +21,7 @@ import torch
 
 import oracle
 from gated_deltanet_linear_20_b200 import inputs
-from tests.test_gpu_parity import DEV, assert_parity, to_dev
+from tests.test_gpu_parity import DEV, assert_parity, raw_qk, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -124,6 +127,75 @@ def test_varlen_sweep(case):
     o, S_T = gdn.prefill_varlen(cat("q").to(DEV), cat("k").to(DEV), cat("v").to(DEV), cat("g").to(DEV),
                                 cat("beta").to(DEV), cu.to(DEV), S0.to(DEV) if S0 is not None else None,
                                 chunk=c["chunk"], status=status)
+    assert gdn.query_status(status) == 0
+    o = o.cpu().numpy()
+    S_T = S_T.cpu().numpy()
+    t0 = 0
+    for n, (L, s) in enumerate(zip(c["lengths"], seqs)):
+        ro, rS = oracle.prefill(s["q"], s["k"], s["v"], s["g"], s["beta"], s["S0"])
+        if L:
+            assert_parity(o[t0:t0 + L], ro[0], f"o of sequence {n}")
+        assert_parity(S_T[n:n + 1], rS, f"S_T of sequence {n}")
+        t0 += L
+
+
+TC_DIMS = ((64, 64), (64, 128), (128, 64), (128, 128), (128, 256))
+
+OPTION_CASES = _draw(16, 31, lambda r, i: dict(
+    B=int(r.integers(1, 3)), H=int(r.integers(1, 4)), T=int(r.integers(1, 201)),
+    chunk=int(r.choice([16, 64])), dims=TC_DIMS[int(r.integers(0, len(TC_DIMS)))],
+    bf16=bool(r.integers(0, 2)), seed=900 + i))
+
+
+@pytest.mark.parametrize("case", OPTION_CASES, ids=lambda c: "B{B}H{H}T{T}c{chunk}_{d[0]}x{d[1]}{o}".format(
+    d=c["dims"], o="_bf16" if c["bf16"] else "", **{k: v for k, v in c.items() if k not in ("dims", "bf16")}))
+def test_fused_options_sweep(case):
+    """The fused q/k norm and q scale (and bf16 o) in the tensor-core prefill at
+    a drawn head-dim pair, against the oracle on fp64-normalised inputs; bf16 o
+    within one bf16 ulp of the oracle plus the fp32 path's tolerance."""
+    c = case
+    dk, dv = c["dims"]
+    d = inputs.prefill_inputs(c["B"], c["T"], c["H"], dk, dv, seed=c["seed"], s0_std=0.05)
+    r = raw_qk(d, c["seed"] + 1)
+    qs = dk ** -0.5
+    dd = to_dev(d)
+    gdn = _gdn()
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.prefill(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], dd["S0"],
+                         chunk=c["chunk"], qk_l2norm=True, q_scale=qs, o_bf16=c["bf16"], status=status)
+    assert gdn.query_status(status) == 0
+    ro, rS = oracle.prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"], d["beta"], d["S0"])
+    if c["bf16"]:
+        got = o.float().cpu().numpy().astype(np.float64)
+        ref = np.asarray(ro, dtype=np.float64)
+        rms = float(np.sqrt(np.mean(ref ** 2)))
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -7 + 1e-2 * rms)
+    else:
+        assert_parity(o.cpu().numpy(), ro, "o")
+    assert_parity(S_T.cpu().numpy(), rS, "S_T")
+
+
+VARLEN_DIM_CASES = _draw(10, 13, lambda r, i: dict(
+    lengths=[int(x) for x in r.integers(0, 161, size=int(r.integers(1, 5)))], H=int(r.integers(1, 3)),
+    chunk=int(r.choice([16, 64])), dims=TC_DIMS[int(r.integers(0, len(TC_DIMS)))], seed=950 + 10 * i))
+
+
+@pytest.mark.parametrize("case", VARLEN_DIM_CASES, ids=lambda c: "L{}_H{}_c{}_{}x{}".format(
+    "-".join(map(str, c["lengths"])), c["H"], c["chunk"], *c["dims"]))
+def test_varlen_head_dims_sweep(case):
+    """Packed sequences at a drawn tensor-core head-dim pair, with carried
+    states, each sequence against the oracle run on it alone."""
+    c = case
+    dk, dv = c["dims"]
+    seqs = [inputs.prefill_inputs(1, L, c["H"], dk, dv, seed=c["seed"] + n, s0_std=0.05)
+            for n, L in enumerate(c["lengths"])]
+    cat = lambda key: torch.cat([s[key][0] for s in seqs], 0)
+    S0 = torch.cat([s["S0"] for s in seqs], 0)
+    cu = torch.tensor([0] + list(np.cumsum(c["lengths"])), dtype=torch.int32)
+    gdn = _gdn()
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.prefill_varlen(cat("q").to(DEV), cat("k").to(DEV), cat("v").to(DEV), cat("g").to(DEV),
+                                cat("beta").to(DEV), cu.to(DEV), S0.to(DEV), chunk=c["chunk"], status=status)
     assert gdn.query_status(status) == 0
     o = o.cpu().numpy()
     S_T = S_T.cpu().numpy()
