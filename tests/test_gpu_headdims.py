@@ -352,3 +352,29 @@ def test_varlen_state_snapshots_other_head_dims(dk, dv):
     o2, S2 = gdn.prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"], dd["S0"])
     torch.cuda.synchronize()
     assert torch.equal(o, o2) and torch.equal(S_T, S2)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 256)], ids=["64x64", "128x256"])
+def test_varlen_snapshot_bounds_other_head_dims(dk, dv):
+    """Snapshot slots at other head dims stay inside the buffer: malformed
+    offsets (a sequence ending before it starts) leave the slots in front of the
+    buffer untouched, and a buffer one slot short leaves the slot after it
+    untouched; both report GDN_ERR_SHAPE."""
+    H, T = 2, 200
+    d = inputs.prefill_inputs(1, T, H, dk, dv, seed=560 + dk + dv)
+    gdn = _gdn()
+    flat = lambda x: x[0].contiguous().to(DEV)
+    args = [flat(d[key]) for key in ("q", "k", "v", "g", "beta")]
+    guard = 2
+    buf = torch.full((guard + 3 + guard, H, dv, dk), 7.0, dtype=torch.float32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    bad = torch.tensor([100, 0, 200], dtype=torch.int32, device=DEV)
+    gdn.prefill_varlen(*args, bad, status=status, snap_every=64, snaps=buf[guard:guard + 3])
+    assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
+    assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + 3:] == 7.0)
+    # 200 tokens need 3 slots; give 2
+    status.zero_()
+    ok = torch.tensor([0, 200], dtype=torch.int32, device=DEV)
+    gdn.prefill_varlen(*args, ok, status=status, snap_every=64, snaps=buf[guard:guard + 2])
+    assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
+    assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + 2:] == 7.0)
