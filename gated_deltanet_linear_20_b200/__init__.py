@@ -13,7 +13,7 @@ fallback: calling into the binding without the built library raises.
 Head dims 64, 128 and 256 (Dk != Dv allowed) are accepted.  Prefill with
 Dk = 64 or 128 runs the chunked tensor-core kernel, with Dk = 256 the
 row-parallel fp32 kernel; the per-channel-gate prefill runs its own chunked
-tensor-core kernel at 128 x 128; decode at 128 x 128 and 64 x 64 streams the
+tensor-core kernel with Dk = 128 (any Dv); decode at 128 x 128 and 64 x 64 streams the
 state through the decode kernels, at other dims through the row kernel.
 
 The binding is imported lazily so that ``inputs`` (the seeded input

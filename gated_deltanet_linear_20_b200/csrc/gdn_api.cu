@@ -376,7 +376,7 @@ const char* gdn_status_str(int code) {
     case GDN_ERR_NULL: return "a required pointer is NULL";
     case GDN_ERR_ALIGN: return "misaligned pointer (q/k/v/o/S need 16 bytes, g/beta 4 bytes)";
     case GDN_ERR_SHAPE: return "negative size or problem larger than 2^31-1 elements";
-    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options not with Dk = 256, nor in decode outside 64 x 64 and 128 x 128, nor in the per-channel-gate prefill outside 128 x 128, and no bf16 o with the per-channel gate; packed sequences not with Dk = 256; chunk 16 or 64; device sm_100)";
+    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options not with Dk = 256, nor in decode outside 64 x 64 and 128 x 128, nor in the per-channel-gate prefill with Dk other than 128, and no bf16 o with the per-channel gate; packed sequences not with Dk = 256; chunk 16 or 64; device sm_100)";
     case GDN_ERR_ALIAS: return "output overlaps an input";
     case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
     case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
@@ -582,27 +582,27 @@ int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float*
   float q_scale = 1.f;
   if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
   const bool fused = qk_norm || q_scale != 1.f;
-  // the row kernel validates every argument; at 128 x 128 with tokens to process
-  // the chunked tensor-core kernel runs instead (same validation first); the
-  // fused options exist on the tensor-core kernel only
+  // the row kernel validates every argument; with Dk = 128 (Dv = 64, 128 or 256)
+  // and tokens to process the chunked tensor-core kernel runs instead (same
+  // validation first); the fused options exist on the tensor-core kernel only
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
-  if (fused && (Dk != kHeadDim || Dv != kHeadDim)) return GDN_ERR_UNSUPPORTED;
-  if (Dk != kHeadDim || Dv != kHeadDim || T == 0 || (long long)B * H == 0)
+  const bool tc = Dk == kHeadDim && (Dv == 64 || Dv == kHeadDim || Dv == 2 * kHeadDim);
+  if (fused && !tc) return GDN_ERR_UNSUPPORTED;
+  if (!tc || T == 0 || (long long)B * H == 0)
     return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, true, stream);
   const long long chains = (long long)B * H;
-  if (chains * T * kHeadDim > 0x7fffffffLL || chains * kHeadDim * kHeadDim > 0x7fffffffLL)
-    return GDN_ERR_SHAPE;
+  if (chains * T * Dv > 0x7fffffffLL || chains * kHeadDim * Dv > 0x7fffffffLL) return GDN_ERR_SHAPE;
   if (!S_T || !q || !k || !v || !g || !beta || !o) return GDN_ERR_NULL;
   if (!aligned(S_T, 16) || (S0 && !aligned(S0, 16)) || !aligned(q, 16) || !aligned(k, 16) ||
       !aligned(v, 16) || !aligned(g, 16) || !aligned(o, 16) || !aligned(beta, 4))
     return GDN_ERR_ALIGN;
   const size_t toks = size_t(chains) * T;
-  const size_t act_bf16 = toks * kHeadDim * 2, o_bytes = toks * kHeadDim * 4;
+  const size_t act_bf16 = toks * kHeadDim * 2, v_bf16 = toks * Dv * 2, o_bytes = toks * Dv * 4;
   const size_t g_bytes = toks * kHeadDim * 4, beta_bytes = toks * 4;
-  const size_t state_bytes = size_t(chains) * kHeadDim * kHeadDim * 4;
+  const size_t state_bytes = size_t(chains) * kHeadDim * Dv * 4;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
   const void* ins[5] = {q, k, v, g, beta};
-  const size_t in_bytes[5] = {act_bf16, act_bf16, act_bf16, g_bytes, beta_bytes};
+  const size_t in_bytes[5] = {act_bf16, act_bf16, v_bf16, g_bytes, beta_bytes};
   for (int i = 0; i < 5; ++i)
     if (overlaps(o, o_bytes, ins[i], in_bytes[i]) || overlaps(S_T, state_bytes, ins[i], in_bytes[i]))
       return GDN_ERR_ALIAS;
@@ -611,14 +611,15 @@ int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float*
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
   CUtensorMap tq{}, tk{}, tv{}, to{}, tg{};
+  const int dv_box = Dv < kHeadDim ? Dv : kHeadDim;  // the rows one CTA owns
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   if (!encode_act(&tg, g, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, kHeadDim, 32) ||
       !encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
       !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
-      !encode_act(&tv, v, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, kHeadDim, 32) ||
-      !encode_act(&to, o, B, T, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, kHeadDim, 32))
+      !encode_act(&tv, v, B, T, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv, 32) ||
+      !encode_act(&to, o, B, T, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, Dv, 32))
     return GDN_ERR_LAUNCH;
-  gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status, qk_norm, q_scale};
+  gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status, qk_norm, q_scale, Dv};
   return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK
              : GDN_ERR_LAUNCH;

@@ -85,12 +85,13 @@ struct RowArgs {
 struct KdaArgs {
   const float* g;     // [B][T][H][128] natural-log decays per key channel
   const float* beta;  // [B][T][H]
-  const float* S0;    // [B][H][128][128] or null (zeros)
+  const float* S0;    // [B][H][Dv][128] or null (zeros)
   float* S_T;         // may equal S0
   int B, T, H;
   int* status;        // may be null
   int qk_norm;        // q, k L2-normalised per token and head in the kernel
   float q_scale;      // q multiplied by this after the normalisation
+  int Dv;             // 64, 128 or 256 (Dk is 128)
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device
@@ -103,8 +104,9 @@ bool ensure_smem_attr(const void* func, int slot, int bytes);
 int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                    const CUtensorMap& to, const CUtensorMap& tf, const PrefillArgs& a, int chunk,
                    cudaStream_t stream);
-// tq, tk: bf16 q, k boxes of 64 features x 32 tokens (SW128); tv: bf16 v, tv:
-// 128 x 32 unswizzled; to: fp32 o, 128 x 32.  T > 0 and B*H > 0.
+// tq, tk: bf16 q, k boxes of 64 features x 32 tokens (SW128); tv: bf16 v, and
+// to: fp32 o, boxes of min(Dv, 128) features x 32 tokens, unswizzled; tg: fp32
+// g, 128 x 32.  T > 0 and B*H > 0; Dk = 128, a.Dv 64, 128 or 256.
 int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const CUtensorMap& to, const CUtensorMap& tg, const KdaArgs& a,
                        cudaStream_t stream);

@@ -2,8 +2,8 @@
 // cores (sm_100a): 32-token TMA tiles, tcgen05 MMAs accumulating in tensor
 // memory, the fp32 state carried from chunk to chunk in tensor memory.
 //
-// Recurrence (per sequence b, head h; S in R^{Dv x Dk}, Dk = Dv = 128; g_t a
-// vector of natural-log decays over the key channels):
+// Recurrence (per sequence b, head h; S in R^{Dv x Dk}, Dk = 128, Dv = 64, 128
+// or 256; g_t a vector of natural-log decays over the key channels):
 //   S_t = S_{t-1} diag(exp(g_t)) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t.
 // The ROCmFPX gated-delta-net prefill note (bittide.aicompass.dev article
 // d2880479, opening post) names KDA among the cases its chunked kernel left to
@@ -23,8 +23,9 @@
 // 32-token chunk: exact while a channel's decay over 16 tokens stays above
 // e^-87 (the fp32 range); beyond that the exponents are clamped (no inf/NaN).
 //
-// One CTA of 512 threads owns one (b, h) chain; two roles hand off through
-// mbarriers:
+// One CTA of 512 threads owns one (b, h) chain (with Dv = 256, two CTAs own
+// 128 rows of its state each; with Dv = 64, lanes 64..127 of the state stay
+// zero); two roles hand off through mbarriers:
 //   * chain (warps 0-3, 12-15): S_c [K+;Q+]^T, X, Dl = X T^T, the state update
 //     and the output product, their epilogues, and the o store;
 //   * side (warps 4-11), one chunk ahead: the gates (per-channel cumulative
@@ -72,7 +73,7 @@ constexpr int OI_ISSUER = 384;
 // Shared memory (offsets from a 1024-byte aligned base).  K-major SW128 tiles
 // have 128-byte rows (64 bf16 along K) in 8-row groups 1024 B apart.
 constexpr uint32_t SM_KQ = 0;          // raw [K dk0-63 | Q dk0-63 | K dk64-127 | Q dk64-127], 4 KB boxes
-constexpr uint32_t SM_V = 16384;       // raw V [32 tokens][128] bf16
+constexpr uint32_t SM_V = 16384;       // raw V [32 tokens][DVB] bf16 (the CTA's rows)
 // The chain's operand tiles (ZQB: [K+;Q+], KT: K~) are double-buffered (tile c
 // in buffer c & 1), so the side writes them as soon as it derives them; the
 // solve's scratch (A, T, the exchange area) lives in the P operand region,
@@ -81,7 +82,7 @@ constexpr uint32_t SM_ZQB0 = 24576;    // [K+ hi; Q+ hi; K+ lo; Q+ lo] 128 rows,
 constexpr uint32_t SM_PA = 57344;      // [K' hi; Q' hi; K' lo; Q' lo] 128 rows, boxes 16 KB apart
 constexpr uint32_t SM_PB = 90112;      // [K'' hi; K'' lo] 64 rows, boxes 8 KB apart
 constexpr uint32_t SM_KT0 = 106496;    // K~ = K o Lambda_last / Lambda, rows j, MN-major: hi (2 x 4 KB), lo at +8 KB
-constexpr uint32_t SM_XH = 122880;     // the fp32 [32][128] o staging tile (16 KB)
+constexpr uint32_t SM_XH = 122880;     // the fp32 [32][DVB] o staging tile (up to 16 KB)
 constexpr uint32_t SM_G = 139264;      // g tile [32 tokens][128] fp32
 constexpr uint32_t SM_ZQB1 = 155648;
 constexpr uint32_t SM_KT1 = 188416;
@@ -127,7 +128,6 @@ constexpr uint32_t M_TMEM = 0, M_ABORT = 4, M_KQ_ISSUED = 12, M_KQ_SEEN = 16, M_
                    M_G_SEEN = 52;
 
 constexpr uint32_t KQ_TX_BYTES = 4 * 4096;
-constexpr uint32_t V_TX_BYTES = NT * D * 2;
 constexpr uint32_t G_TX_BYTES = NT * D * 4;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr float LOG2E = 1.4426950408889634f;
@@ -223,10 +223,12 @@ __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, co
   tma_load_4d(x.sb + SM_KQ + 12288, tq, bar, 64, h, t0, b);
   *x.misc(M_KQ_ISSUED) = c + 1;
 }
-__device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b) {
+// V rows dv0 .. dv0 + DVB - 1 of tile c ([32 tokens][DVB] bf16)
+template <int DVB>
+__device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b, int dv0) {
   const uint32_t bar = x.bar(B_VFULL);
-  mbar_arrive_expect_tx(bar, V_TX_BYTES);
-  tma_load_4d(x.sb + SM_V, tv, bar, 0, h, c * NT, b);
+  mbar_arrive_expect_tx(bar, uint32_t(NT * DVB * 2));
+  tma_load_4d(x.sb + SM_V, tv, bar, dv0, h, c * NT, b);
   *x.misc(M_V_ISSUED) = c + 1;
 }
 
@@ -595,8 +597,13 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
 }
 
 // ============================================================== chain role
+// DVB: rows of the state this CTA owns (64 or 128); DV2: two CTAs per chain
+// (Dv = 256), this one owning rows dv0 = 128 (blockIdx & 1) ..
+template <int DVB, bool DV2>
 __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMap* tmo,
                            const KdaArgs& p, int chain, int b, int h, int ntiles) {
+  constexpr int DVW = DV2 ? 2 * D : DVB;  // Dv: rows of the chain's state
+  const int dv0 = DV2 ? D * (int(blockIdx.x) & 1) : 0;
   const int warp = threadIdx.x >> 5;
   const int lq = warp & 3;
   const int ch = (warp >= 12) ? 1 : 0;  // column half
@@ -605,14 +612,16 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
   const uint32_t tlane = x.tmem + (uint32_t(lq * 32) << 16);
   const uint32_t sb = x.sb;
   RoleSync rs{BAR_CHAIN, CHAIN_THREADS, M_FLAG_CHAIN, leader, 0};
-  const size_t cstate = size_t(chain) * D * D;
+  const size_t cstate = size_t(chain) * DVW * D + size_t(dv0) * D;  // this CTA's first row
+  const bool own = DVB == D || dv < DVB;  // the lane holds one of the CTA's rows
 
   // ---- initial state (row dv of S0, or zeros): hi/lo copy, and the fp32 copy
   //      pre-scaled, column by column, by the decay of the first tile
   if (!rs.wait(x, x.bar(gfull_off(0)), gfull_parity(0))) return;
   {
     const float* LC = x.gates(0) + G_LC / 4;
-    const float4* src = p.S0 ? reinterpret_cast<const float4*>(p.S0 + cstate + size_t(dv) * D) : nullptr;
+    const float4* src =
+        (p.S0 && own) ? reinterpret_cast<const float4*>(p.S0 + cstate + size_t(dv) * D) : nullptr;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int col = 64 * ch + 32 * q;
@@ -673,7 +682,8 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const int n = n0 + e;
-        xv[e] = G[G_B / 4 + n] * (__bfloat162float(V[n * D + dv]) - (za[e] + zb[e]));
+        const float vn = own ? __bfloat162float(V[n * DVB + dv]) : 0.f;
+        xv[e] = G[G_B / 4 + n] * (vn - (za[e] + zb[e]));
       }
       uint32_t xh[8], xl[8];
 #pragma unroll
@@ -685,7 +695,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
     // ---- Dl^T = X^T T^T: X hi x [T hi; T lo] (N=64), X lo x T hi (N=32); K = 32,
     //      A from tensor memory (K step ks = the tokens of chain half ks)
     if (leader) {
-      if (!last) issue_v(x, tv, c + 1, h, b);  // V(c) has been read
+      if (!last) issue_v<DVB>(x, tv, c + 1, h, b, dv0);  // V(c) has been read
       if (lead_wait(x, x.bar(B_TMFULL), c & 1)) {
         tc_fence_after();
         const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0), id32 = idesc_bf16(128, 32, 0, 0, 0);
@@ -752,14 +762,16 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
       tmem_ld16x2(tlane + TM_ZQ + 32 + n0, ya, tlane + TM_ZQ + 96 + n0, yb);
       tmem_ld16x2(tlane + TM_DO + n0, oa, tlane + TM_DO + 32 + n0, ob);
       float* so = reinterpret_cast<float*>(x.sm + SM_XH) + dv;
+      if (own) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) so[(n0 + e) * D] = (ya[e] + yb[e]) + (oa[e] + ob[e]);
+        for (int e = 0; e < 16; ++e) so[(n0 + e) * DVB] = (ya[e] + yb[e]) + (oa[e] + ob[e]);
+      }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     named_bar(BAR_CHAIN, CHAIN_THREADS);
     if (leader) {
-      tma_store_4d(tmo, sb + SM_XH, 0, h, c * NT, b);
+      tma_store_4d(tmo, sb + SM_XH, dv0, h, c * NT, b);
       bulk_commit();
     }
     // ---- state epilogue: the update has completed (its commit preceded the
@@ -795,6 +807,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
       for (int q = 0; q < 2; ++q) {
         float v[32];
         tmem_ld32(tlane + TM_S + 64 * ch + 32 * q, v);
+        if (!own) continue;
 #pragma unroll
         for (int e = 0; e < 8; ++e) dst[8 * q + e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
       }
@@ -802,7 +815,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
   }
 }
 
-template <bool PRE>
+template <bool PRE, int DVB, bool DV2>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -812,7 +825,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                            ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
-  const int chain = blockIdx.x;
+  const int chain = DV2 ? int(blockIdx.x) >> 1 : int(blockIdx.x);
   const int b = chain / p.H, h = chain - (chain / p.H) * p.H;
   const int ntiles = (p.T + NT - 1) / NT;
 
@@ -841,11 +854,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   x.tmem = *reinterpret_cast<volatile uint32_t*>(sm + SM_MISC + M_TMEM);
   if (tid == 0) {
     issue_kq(x, &tm_q, &tm_k, 0, h, b);
-    issue_v(x, &tm_v, 0, h, b);
+    issue_v<DVB>(x, &tm_v, 0, h, b, DV2 ? D * (int(blockIdx.x) & 1) : 0);
     issue_g(x, &tm_g, 0, h, b);
   }
   if (warp < 4 || warp >= 12)
-    chain_role(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
+    chain_role<DVB, DV2>(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
   else
     side_role<PRE>(x, &tm_q, &tm_k, &tm_g, p, b, h, ntiles);
 
@@ -881,13 +894,25 @@ int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
   const int chains = a.B * a.H;
   if (chains == 0 || a.T == 0) return -1;
   const uint32_t smem = SMEM_USED + 1024;
-  if (a.qk_norm || a.q_scale != 1.f) {
-    if (!ensure_smem_attr(reinterpret_cast<const void*>(kda_prefill_kernel<true>), 48, int(smem))) return -1;
-    kda_prefill_kernel<true><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, tg, a);
-  } else {
-    if (!ensure_smem_attr(reinterpret_cast<const void*>(kda_prefill_kernel<false>), 15, int(smem))) return -1;
-    kda_prefill_kernel<false><<<chains, NTHREADS, smem, stream>>>(tq, tk, tv, to, tg, a);
-  }
+  const bool pre = a.qk_norm || a.q_scale != 1.f;
+  auto go = [&](auto kernel, int slot, int ctas) {
+    if (!ensure_smem_attr(reinterpret_cast<const void*>(kernel), slot, int(smem))) return false;
+    kernel<<<ctas, NTHREADS, smem, stream>>>(tq, tk, tv, to, tg, a);
+    return true;
+  };
+  bool ok;
+  if (a.Dv == D)
+    ok = pre ? go(kda_prefill_kernel<true, 128, false>, 48, chains)
+             : go(kda_prefill_kernel<false, 128, false>, 15, chains);
+  else if (a.Dv == 2 * D)  // two CTAs per chain
+    ok = pre ? go(kda_prefill_kernel<true, 128, true>, 63, 2 * chains)
+             : go(kda_prefill_kernel<false, 128, true>, 40, 2 * chains);
+  else if (a.Dv == 64)
+    ok = pre ? go(kda_prefill_kernel<true, 64, false>, 41, chains)
+             : go(kda_prefill_kernel<false, 64, false>, 42, chains);
+  else
+    return -1;
+  if (!ok) return -1;
   return cudaGetLastError() == cudaSuccess ? 0 : -1;
 }
 

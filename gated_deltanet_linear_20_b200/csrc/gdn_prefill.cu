@@ -1047,12 +1047,14 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           const bool own = DVB == D || dv < DVB;
           float4* dst = reinterpret_cast<float4*>(x.sdst + size_t(dv) * DK + SCOLS * ch);
           float4* sdst = nullptr;
-          const int stiles = PK ? *x.misc(M_SNAP_TILES) : 0;
-          if (stiles && (x.tend - x.tok0) % (stiles * NT) == 0)
-            sdst = reinterpret_cast<float4*>(
-                *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR) +
-                size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * p.Dv * DK + size_t(dv) * DK +
-                SCOLS * ch);
+          if constexpr (PK) {
+            const int stiles = *x.misc(M_SNAP_TILES);
+            if (stiles && (x.tend - x.tok0) % (stiles * NT) == 0)
+              sdst = reinterpret_cast<float4*>(
+                  *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR) +
+                  size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * p.Dv * DK + size_t(dv) * DK +
+                  SCOLS * ch);
+          }
 #pragma unroll
           for (int q = 0; q < NQ; ++q) {
             float v[32];
@@ -1085,13 +1087,15 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMa
           }
           named_bar(BAR_CHAIN, CHAIN_THREADS);
           copy_staged_state(x.sm + SM_XH, x.sdst, ch * 128 + dv);
-          const int stiles = PK ? *x.misc(M_SNAP_TILES) : 0;
-          if (stiles && (x.tend - x.tok0) % (stiles * NT) == 0) {
-            // the sequence ends on a snapshot boundary: its last snapshot is S_T
-            float* snap = *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR);
-            copy_staged_state(x.sm + SM_XH,
-                              snap + size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * p.Dv * D,
-                              ch * 128 + dv);
+          if constexpr (PK) {
+            const int stiles = *x.misc(M_SNAP_TILES);
+            if (stiles && (x.tend - x.tok0) % (stiles * NT) == 0) {
+              // the sequence ends on a snapshot boundary: its last snapshot is S_T
+              float* snap = *reinterpret_cast<float* volatile*>(x.sm + SM_MISC + M_SNAP_PTR);
+              copy_staged_state(x.sm + SM_XH,
+                                snap + size_t((x.tend - x.tok0) / (stiles * NT) - 1) * x.H * p.Dv * D,
+                                ch * 128 + dv);
+            }
           }
         } else {
           // at a snapshot tile end, the state itself first goes to its slot

@@ -409,8 +409,9 @@ def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g [B,T,H,Dk] fp32 (log decay per key
     channel); beta [B,T,H] fp32; S0 [B,H,Dv,Dk] fp32 or None (zeros).  ``S_T``
     may be ``S0`` (in place).  ``qk_l2norm`` / ``q_scale`` normalise q and k per
-    token and head and scale q inside the kernel (gdn_kda_prefill_ex; 128 x 128
-    only).  Launches on the current stream."""
+    token and head and scale q inside the kernel (gdn_kda_prefill_ex; Dk = 128).
+    Dk = 128 runs the chunked tensor-core kernel (Dv 64, 128 or 256); Dk = 64 or
+    256 the row kernel.  Launches on the current stream."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape

@@ -43,7 +43,7 @@
  *     GDN_ERR_UNSUPPORTED  a head dim not in {64, 128, 256}; fused options where
  *                          the kernel serving the head dims has none (prefill
  *                          with Dk = 256; decode outside 64 x 64 and 128 x 128;
- *                          the per-channel-gate prefill outside 128 x 128);
+ *                          the per-channel-gate prefill with Dk other than 128);
  *                          packed sequences with Dk = 256;
  *                          chunk not in {16, 64}; or the current device is not
  *                          compute capability 10.0
@@ -286,10 +286,11 @@ int gdn_decode_ex(const void* q, const void* k, const void* v, const float* g,
  * d2880479, lists among the cases its fused kernel left to the old path):
  *     S_t = S_{t-1} diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
  *     o_t = S_t q_t
- * for t = 1..T of each of the B*H chains.  At Dk = Dv = 128 it runs chunked on
- * the tensor cores (32-token chunks; every derived operand as a bf16 hi/lo
- * pair; exact up to rounding while a key channel's decay over 16 tokens stays
- * above e^-87, the fp32 range); other head dims run token by token in fp32.
+ * for t = 1..T of each of the B*H chains.  With Dk = 128 (Dv 64, 128 or 256)
+ * it runs chunked on the tensor cores (32-token chunks; every derived operand
+ * as a bf16 hi/lo pair; exact up to rounding while a key channel's decay over
+ * 16 tokens stays above e^-87, the fp32 range; Dv = 256 on two CTAs per
+ * chain); Dk = 64 or 256 run token by token in fp32.
  *   q, k [B][T][H][Dk] bf16; v [B][T][H][Dv] bf16 (device, 16-byte aligned)
  *   g    [B][T][H][Dk] fp32, natural-log decays (device, 16-byte aligned;
  *        g > 0 is accepted and grows the state)
@@ -320,8 +321,8 @@ int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
 
 /* gdn_kda_prefill / gdn_kda_decode with options (gdn_options; NULL = none).
  * qk_l2norm and q_scale are applied to each token's q and k before any decay,
- * as in gdn_prefill_ex; they need Dk = Dv = 128 in the prefill, and 128 x 128
- * or 64 x 64 in decode (else GDN_ERR_UNSUPPORTED).
+ * as in gdn_prefill_ex; they need Dk = 128 in the prefill (any Dv), and
+ * 128 x 128 or 64 x 64 in decode (else GDN_ERR_UNSUPPORTED).
  * o_bf16 is not offered with the per-channel gate: a nonzero o_bf16 (or an
  * invalid struct) returns GDN_ERR_UNSUPPORTED.  Everything else as for the
  * calls without options. */

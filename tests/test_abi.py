@@ -428,7 +428,7 @@ def test_plain_c_client_links_and_gets_the_documented_codes(gdn, tmp_path):
 
 def test_kda_options_validation(gdn):
     """gdn_kda_prefill_ex / gdn_kda_decode_ex: the fused norm and q scale exist
-    at 128 x 128 in the prefill, and at 128 x 128 and 64 x 64 in decode; o_bf16
+    with Dk = 128 in the prefill, and at 128 x 128 and 64 x 64 in decode; o_bf16
     and invalid structs are GDN_ERR_UNSUPPORTED; valid options where they exist
     pass validation (then fail only for want of a device)."""
     import ctypes as ct
@@ -441,6 +441,8 @@ def test_kda_options_validation(gdn):
     assert gdn.raw_kda_prefill_ex(*ins(a, bf16)) == -4
     assert gdn.raw_kda_prefill_ex(*ins(a, short)) == -4
     assert gdn.raw_kda_prefill_ex(*ins(kda_args(Dk=64, Dv=64), good)) == -4
+    for dv in (64, 256):  # Dk = 128: the tensor-core kernel, with the options
+        assert gdn.raw_kda_prefill_ex(*ins(kda_args(Dv=dv), good)) not in (0, -1, -2, -3, -4, -5)
     assert gdn.raw_kda_prefill_ex(*(a[:13] + [None] + a[13:])) not in (0, -1, -2, -3, -4, -5)
     d = [P, P + 0x1000000, P + 0x2000000, P + 0x3000000, P + 0x3100000, P + 0x4000000,
          P + 0x5000000, 4, 1, 2, 128, 128]

@@ -97,7 +97,7 @@ def test_decode_64_b64_h16_steps():
     assert torch.equal(o, o2) and torch.equal(S, S2), "not bitwise run-to-run"
 
 
-@pytest.mark.parametrize("dk,dv", [(64, 64), (256, 256), (128, 64), (64, 256)], ids=lambda x: str(x))
+@pytest.mark.parametrize("dk,dv", [(64, 64), (256, 256), (128, 64), (64, 256), (128, 256)], ids=lambda x: str(x))
 def test_kda_other_head_dims(dk, dv):
     d = inputs.kda_inputs(2, 50, 3, dk, dv, seed=dk + 2 * dv, s0_std=0.05)
     dd = to_dev(d)
@@ -378,3 +378,32 @@ def test_varlen_snapshot_bounds_other_head_dims(dk, dv):
     gdn.prefill_varlen(*args, ok, status=status, snap_every=64, snaps=buf[guard:guard + 2])
     assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
     assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + 2:] == 7.0)
+
+
+@pytest.mark.parametrize("dv", [64, 256])
+def test_kda_tensor_core_prefill_other_value_dims(dv):
+    """The per-channel-gate prefill at Dk = 128 with Dv = 64 (lanes 64..127 of
+    the state stay zero) or Dv = 256 (two CTAs per chain) on the chunked
+    tensor-core kernel: whole and ragged 32-token tiles, carried state, strong
+    and weak decays, with and without the fused q/k norm and q scale."""
+    gdn = _gdn()
+    for T, g_mean, norm in ((100, 0.0, False), (33, 2.0, True), (64, -3.0, False)):
+        d = inputs.kda_inputs(2, T, 3, 128, dv, seed=600 + dv + T, g_mean=g_mean, s0_std=0.05)
+        r = raw_qk(d, 601 + T) if norm else {"q": d["q"], "k": d["k"], "q_n": d["q"].double(),
+                                               "k_n": d["k"].double()}
+        qs = 128 ** -0.5 if norm else 1.0
+        dd = to_dev(d)
+        status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        o, S_T = gdn.kda_prefill(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], dd["S0"],
+                                 status=status, qk_l2norm=norm, q_scale=qs)
+        assert gdn.query_status(status) == 0
+        ro, rS = oracle.kda_prefill((r["q_n"] * qs).float(), r["k_n"].float(), d["v"], d["g"], d["beta"],
+                                    d["S0"])
+        assert_parity(o.cpu().numpy(), ro, f"o kda 128x{dv} T={T}")
+        assert_parity(S_T.cpu().numpy(), rS, f"S_T kda 128x{dv} T={T}")
+    # in place and deterministic
+    S = dd["S0"].clone()
+    o1, _ = gdn.kda_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], S, S_T=S)
+    o2, S2 = gdn.kda_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S, S2)
