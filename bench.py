@@ -666,7 +666,8 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
     """The per-channel gate (KDA): prefill at 128 x 128 on the chunked
     tensor-core kernel (32-token chunks; HBM roofline, with the tensor fraction
     of the same chunk-GEMM FLOP count as the scalar gate beside it), at the
-    512-token single-sequence shape and a large batch; and the batched decode
+    512-token single-sequence shape and a large batch, and at 128 x 256 (two
+    CTAs per chain) at the 512-token shape; and the batched decode
     step at 128 x 128 and 64 x 64 on the streaming decode kernel (HBM
     roofline)."""
     from gated_deltanet_linear_20_b200 import gdn
@@ -690,6 +691,23 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
             "tensor_frac": round(fl / (t / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
             "gate": f"per channel, logsigmoid(N({g_mean},1))"}
         del d, o, sT
+    # Dk = 128 with Dv = 256 (two CTAs per chain) at the 512-token shape
+    B, T, H, Dv = 1, 512, 16, 2 * D
+    d = gin.kda_inputs(B, T, H, D, Dv, seed=5100 + rank, device=str(dev))
+    o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
+    sT = torch.empty((B, H, Dv, D), dtype=torch.float32, device=dev)
+    ms = time_steps(lambda: gdn.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], None,
+                                            o=o, S_T=sT), steps, 3, flush, stream)
+    t = statistics.mean(ms)
+    # q, k, g over Dk = 128; v bf16 and o fp32 over Dv; beta; S_T once
+    nb = B * T * H * (2 * D * 2 + D * 4 + 4 + Dv * 2 + Dv * 4) + B * H * Dv * D * 4
+    out["kda_prefill_b1_h16_t512_dk128_dv256"] = {
+        "tokens_per_s": round(B * T / (t / 1e3), 1), "ms": round(t, 5),
+        "kernel": "chunked tcgen05, chunk 32, two CTAs per chain",
+        "roofline": {"bound": "hbm", "achieved": round(nb / (t / 1e3) / 1e9, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}}
+    del d, o, sT
     # decode: one token for 64 x 16 heads, state in place, L2 flushed per step
     B, H = 64, 16
     for Dh in (D, 64):
