@@ -227,7 +227,7 @@ struct StepGeom {
 };
 
 template <int DH, bool PRE, bool VG>
-__global__ void __launch_bounds__(WARPS * 32) decode_step_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(WARPS * 32, 7) decode_step_kernel(const DecodeArgs a) {
   using G = StepGeom<DH>;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
