@@ -81,7 +81,7 @@ __device__ __forceinline__ Tok<VG> load_tok(const DecodeArgs& a, size_t tok, int
 // d_i = beta (v_i - (S_i diag(alpha)) . k), so the row dot products take the
 // decayed k and q, and o_i = (S_i diag(alpha)) . q + d_i (k . q).
 template <bool PRE, bool VG>
-__global__ void __launch_bounds__(WARPS * 32) decode_burst_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(WARPS * 32, VG ? 1 : 5) decode_burst_kernel(const DecodeArgs a) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.x / CTAS_PER_HEAD;  // b * H + h
