@@ -81,7 +81,7 @@ __device__ __forceinline__ Tok<VG> load_tok(const DecodeArgs& a, size_t tok, int
 // d_i = beta (v_i - (S_i diag(alpha)) . k), so the row dot products take the
 // decayed k and q, and o_i = (S_i diag(alpha)) . q + d_i (k . q).
 template <bool PRE, bool VG>
-__global__ void __launch_bounds__(WARPS * 32, VG ? 1 : 5) decode_burst_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(WARPS * 32, VG ? 4 : 5) decode_burst_kernel(const DecodeArgs a) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int head = blockIdx.x / CTAS_PER_HEAD;  // b * H + h
@@ -135,20 +135,21 @@ __global__ void __launch_bounds__(WARPS * 32, VG ? 1 : 5) decode_burst_kernel(co
       for (int e = 0; e < 16; ++e) q[e] *= a.q_scale;
     }
 
-    // sc: the decay of each of the lane's columns; kd, qd: k and q as the row
-    // dot products take them (decayed per column with VG; the scalar decay is
-    // applied to the dot products instead)
-    float sc[16], kd[16], qd[16];
+    // VG: the state is decayed in place, column by column (S <- S diag(alpha)),
+    // before the row dot products; the scalar decay is applied to the dot
+    // products and folded into the update instead
+    if constexpr (VG) {
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      if constexpr (VG) {
-        sc[e] = expf(reinterpret_cast<const float*>(cur.gv)[e]);
-        kd[e] = sc[e] * k[e];
-        qd[e] = sc[e] * q[e];
-      } else {
-        sc[e] = alpha;
-        kd[e] = k[e];
-        qd[e] = q[e];
+      for (int e4 = 0; e4 < 4; ++e4) {
+        const float4 gv = cur.gv[e4];
+        const float c0 = expf(gv.x), c1 = expf(gv.y), c2 = expf(gv.z), c3 = expf(gv.w);
+#pragma unroll
+        for (int i = 0; i < RG; ++i) {
+          s[i][e4].x *= c0;
+          s[i][e4].y *= c1;
+          s[i][e4].z *= c2;
+          s[i][e4].w *= c3;
+        }
       }
     }
     const float a_row = VG ? 1.f : alpha;
@@ -158,8 +159,8 @@ __global__ void __launch_bounds__(WARPS * 32, VG ? 1 : 5) decode_burst_kernel(co
     for (int e = 0; e < 16; ++e) kq = fmaf(k[e], q[e], kq);
 #pragma unroll
     for (int i = 0; i < RG; ++i) {
-      sk[i] = dot4(s[i][0], kd) + dot4(s[i][1], kd + 4) + dot4(s[i][2], kd + 8) + dot4(s[i][3], kd + 12);
-      sq[i] = dot4(s[i][0], qd) + dot4(s[i][1], qd + 4) + dot4(s[i][2], qd + 8) + dot4(s[i][3], qd + 12);
+      sk[i] = dot4(s[i][0], k) + dot4(s[i][1], k + 4) + dot4(s[i][2], k + 8) + dot4(s[i][3], k + 12);
+      sq[i] = dot4(s[i][0], q) + dot4(s[i][1], q + 4) + dot4(s[i][2], q + 8) + dot4(s[i][3], q + 12);
     }
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) {
@@ -175,10 +176,17 @@ __global__ void __launch_bounds__(WARPS * 32, VG ? 1 : 5) decode_burst_kernel(co
       const float d = beta * (v[4 * i + sub] - a_row * sk[i]);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        s[i][e].x = fmaf(sc[4 * e], s[i][e].x, d * k[4 * e]);
-        s[i][e].y = fmaf(sc[4 * e + 1], s[i][e].y, d * k[4 * e + 1]);
-        s[i][e].z = fmaf(sc[4 * e + 2], s[i][e].z, d * k[4 * e + 2]);
-        s[i][e].w = fmaf(sc[4 * e + 3], s[i][e].w, d * k[4 * e + 3]);
+        if constexpr (VG) {  // already decayed
+          s[i][e].x = fmaf(d, k[4 * e], s[i][e].x);
+          s[i][e].y = fmaf(d, k[4 * e + 1], s[i][e].y);
+          s[i][e].z = fmaf(d, k[4 * e + 2], s[i][e].z);
+          s[i][e].w = fmaf(d, k[4 * e + 3], s[i][e].w);
+        } else {
+          s[i][e].x = fmaf(alpha, s[i][e].x, d * k[4 * e]);
+          s[i][e].y = fmaf(alpha, s[i][e].y, d * k[4 * e + 1]);
+          s[i][e].z = fmaf(alpha, s[i][e].z, d * k[4 * e + 2]);
+          s[i][e].w = fmaf(alpha, s[i][e].w, d * k[4 * e + 3]);
+        }
       }
       if ((lane & 7) == 0) {
         const float ov = fmaf(a_row, sq[i], d * kq);
