@@ -667,7 +667,7 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
     tensor-core kernel (32-token chunks; HBM roofline, with the tensor fraction
     of the same chunk-GEMM FLOP count as the scalar gate beside it), at the
     512-token single-sequence shape and a large batch, and at 128 x 256 (two
-    CTAs per chain) at the 512-token shape; and the batched decode
+    CTAs per chain) at the 512-token shape; a 4-token decode burst; and the batched decode
     step at 128 x 128 and 64 x 64 on the streaming decode kernel (HBM
     roofline)."""
     from gated_deltanet_linear_20_b200 import gdn
@@ -737,6 +737,19 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
         out[key].update(same_bytes_copy_us=round(copy_us, 3),
                         frac_of_copy=round(copy_us / (t * 1e3), 4))
         del d, S, o, tok
+    # a 4-token burst per sequence in one call (state read and written once)
+    d = gin.kda_inputs(B, 4, H, seed=6100 + rank, s0_std=0.02, device=str(dev))
+    S = d["S0"].clone()
+    o = torch.empty((B, 4, H, D), dtype=torch.float32, device=dev)
+    ms = time_steps(lambda: gdn.kda_decode(d["q"], d["k"], d["v"], d["g"], d["beta"], S, o=o),
+                    32, 5, flush, stream)
+    t = statistics.mean(ms)
+    out["kda_decode_b64_h16_t4"] = {
+        "us_per_call": round(t * 1e3, 3), "tokens_per_s": round(B * 4 / (t / 1e3), 1),
+        "state_GB_per_s": round(B * H * 2 * STATE_BYTES / (t / 1e3) / 1e9, 1),
+        "kernel": "burst", "l2": "flushed before every call",
+        "note": "4 tokens per sequence per call; the state crosses HBM once per call"}
+    del d, S, o
     torch.cuda.empty_cache()
     return out
 
