@@ -298,3 +298,18 @@ def test_kda_default_options_are_bitwise_the_plain_call():
     assert rc == 0
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+@pytest.mark.parametrize("T", [8, 33])
+def test_kda_decode_long_bursts(T):
+    """Per-channel-gate decode bursts of T tokens in one call (the state read
+    and written once) against the oracle, o at every token and the end state."""
+    d = inputs.kda_inputs(16, T, 4, seed=170 + T, s0_std=0.05, g_mean=-1.0)
+    dd = to_dev(d)
+    gdn = _gdn()
+    S = dd["S0"].clone()
+    o = gdn.kda_decode(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], S)
+    torch.cuda.synchronize()
+    ro, rS = oracle.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    assert_parity(o.cpu().numpy(), ro, f"o kda burst T={T}")
+    assert_parity(S.cpu().numpy(), rS, f"S kda burst T={T}")
