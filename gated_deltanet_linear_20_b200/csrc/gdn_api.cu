@@ -376,7 +376,7 @@ const char* gdn_status_str(int code) {
     case GDN_ERR_NULL: return "a required pointer is NULL";
     case GDN_ERR_ALIGN: return "misaligned pointer (q/k/v/o/S need 16 bytes, g/beta 4 bytes)";
     case GDN_ERR_SHAPE: return "negative size or problem larger than 2^31-1 elements";
-    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options not with Dk = 256, nor in decode outside 64 x 64 and 128 x 128, nor in the per-channel-gate prefill with Dk other than 128, and no bf16 o with the per-channel gate; packed sequences not with Dk = 256; chunk 16 or 64; device sm_100)";
+    case GDN_ERR_UNSUPPORTED: return "unsupported configuration (head dims in {64, 128, 256}; fused options not with Dk = 256, nor in decode outside 64 x 64 and 128 x 128, nor in the per-channel-gate prefill with Dk other than 128; packed sequences not with Dk = 256; chunk 16 or 64; device sm_100)";
     case GDN_ERR_ALIAS: return "output overlaps an input";
     case GDN_ERR_LAUNCH: return "CUDA launch or runtime query failed";
     case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
@@ -580,14 +580,15 @@ int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float*
                        int H, int Dk, int Dv, const gdn_options* opts, int* status, void* stream) {
   int qk_norm = 0, o_bf16 = 0;
   float q_scale = 1.f;
-  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
-  const bool fused = qk_norm || q_scale != 1.f;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
+  const bool fused = qk_norm || q_scale != 1.f || o_bf16;
   // the row kernel validates every argument; with Dk = 128 (Dv = 64, 128 or 256)
   // and tokens to process the chunked tensor-core kernel runs instead (same
   // validation first); the fused options exist on the tensor-core kernel only
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   const bool tc = Dk == kHeadDim && (Dv == 64 || Dv == kHeadDim || Dv == 2 * kHeadDim);
   if (fused && !tc) return GDN_ERR_UNSUPPORTED;
+  if (o_bf16 && T == 0) o_bf16 = 0;  // no o is written
   if (!tc || T == 0 || (long long)B * H == 0)
     return rows_impl(q, k, v, g, beta, S0, o, S_T, B, T, H, Dk, Dv, true, stream);
   const long long chains = (long long)B * H;
@@ -597,7 +598,8 @@ int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float*
       !aligned(v, 16) || !aligned(g, 16) || !aligned(o, 16) || !aligned(beta, 4))
     return GDN_ERR_ALIGN;
   const size_t toks = size_t(chains) * T;
-  const size_t act_bf16 = toks * kHeadDim * 2, v_bf16 = toks * Dv * 2, o_bytes = toks * Dv * 4;
+  const size_t act_bf16 = toks * kHeadDim * 2, v_bf16 = toks * Dv * 2,
+               o_bytes = toks * Dv * (o_bf16 ? 2 : 4);
   const size_t g_bytes = toks * kHeadDim * 4, beta_bytes = toks * 4;
   const size_t state_bytes = size_t(chains) * kHeadDim * Dv * 4;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
@@ -617,9 +619,10 @@ int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float*
       !encode_act(&tq, q, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
       !encode_act(&tk, k, B, T, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
       !encode_act(&tv, v, B, T, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv, 32) ||
-      !encode_act(&to, o, B, T, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, Dv, 32))
+      !encode_act(&to, o, B, T, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, o_bf16 ? bf : f32,
+                  o_bf16 ? 2 : 4, Dv, 32))
     return GDN_ERR_LAUNCH;
-  gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status, qk_norm, q_scale, Dv};
+  gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status, qk_norm, q_scale, Dv, o_bf16};
   return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK
              : GDN_ERR_LAUNCH;
@@ -637,15 +640,16 @@ int gdn_kda_decode_ex(const void* q, const void* k, const void* v, const float* 
   (void)status;  // the decode kernels have no device-side waits
   int qk_norm = 0, o_bf16 = 0;
   float q_scale = 1.f;
-  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
-  const bool fused = qk_norm || q_scale != 1.f;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
+  const bool fused = qk_norm || q_scale != 1.f || o_bf16;
   if (B < 0 || T < 0 || H < 0) return GDN_ERR_SHAPE;
   if (fused && !(Dk == Dv && (Dk == kHeadDim || Dk == 64))) return GDN_ERR_UNSUPPORTED;
   if ((long long)B * H > 0 && !S) return GDN_ERR_NULL;
   // Dk = Dv = 128 or 64: the streaming decode kernel; other head dims: the row
   // kernel (both read and write the state once per call)
   if (Dk == Dv && (Dk == kHeadDim || Dk == 64))
-    return decode_impl(q, k, v, g, beta, S, o, B, T, H, Dk, qk_norm, q_scale, 0, true, 4, stream);
+    return decode_impl(q, k, v, g, beta, S, o, B, T, H, Dk, qk_norm, q_scale, o_bf16, true, 4,
+                       stream);
   return rows_impl(q, k, v, g, beta, S, o, S, B, T, H, Dk, Dv, true, stream);
 }
 

@@ -92,6 +92,7 @@ struct KdaArgs {
   int qk_norm;        // q, k L2-normalised per token and head in the kernel
   float q_scale;      // q multiplied by this after the normalisation
   int Dv;             // 64, 128 or 256 (Dk is 128)
+  int o_bf16;         // o written as bf16
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device

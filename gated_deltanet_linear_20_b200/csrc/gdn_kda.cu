@@ -82,7 +82,7 @@ constexpr uint32_t SM_ZQB0 = 24576;    // [K+ hi; Q+ hi; K+ lo; Q+ lo] 128 rows,
 constexpr uint32_t SM_PA = 57344;      // [K' hi; Q' hi; K' lo; Q' lo] 128 rows, boxes 16 KB apart
 constexpr uint32_t SM_PB = 90112;      // [K'' hi; K'' lo] 64 rows, boxes 8 KB apart
 constexpr uint32_t SM_KT0 = 106496;    // K~ = K o Lambda_last / Lambda, rows j, MN-major: hi (2 x 4 KB), lo at +8 KB
-constexpr uint32_t SM_XH = 122880;     // the fp32 [32][DVB] o staging tile (up to 16 KB)
+constexpr uint32_t SM_XH = 122880;     // the [32][DVB] o staging tile, fp32 or bf16 (up to 16 KB)
 constexpr uint32_t SM_G = 139264;      // g tile [32 tokens][128] fp32
 constexpr uint32_t SM_ZQB1 = 155648;
 constexpr uint32_t SM_KT1 = 188416;
@@ -598,8 +598,9 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
 
 // ============================================================== chain role
 // DVB: rows of the state this CTA owns (64 or 128); DV2: two CTAs per chain
-// (Dv = 256), this one owning rows dv0 = 128 (blockIdx & 1) ..
-template <int DVB, bool DV2>
+// (Dv = 256), this one owning rows dv0 = 128 (blockIdx & 1) ..; OBF: o is
+// bf16 (the fp32 value rounded to nearest even, through a bf16 TMA view)
+template <int DVB, bool DV2, bool OBF>
 __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMap* tmo,
                            const KdaArgs& p, int chain, int b, int h, int ntiles) {
   constexpr int DVW = DV2 ? 2 * D : DVB;  // Dv: rows of the chain's state
@@ -761,10 +762,17 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
       float ya[16], yb[16], oa[16], ob[16];
       tmem_ld16x2(tlane + TM_ZQ + 32 + n0, ya, tlane + TM_ZQ + 96 + n0, yb);
       tmem_ld16x2(tlane + TM_DO + n0, oa, tlane + TM_DO + 32 + n0, ob);
-      float* so = reinterpret_cast<float*>(x.sm + SM_XH) + dv;
       if (own) {
+        if constexpr (OBF) {
+          __nv_bfloat16* so = reinterpret_cast<__nv_bfloat16*>(x.sm + SM_XH) + dv;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) so[(n0 + e) * DVB] = (ya[e] + yb[e]) + (oa[e] + ob[e]);
+          for (int e = 0; e < 16; ++e)
+            so[(n0 + e) * DVB] = __float2bfloat16_rn((ya[e] + yb[e]) + (oa[e] + ob[e]));
+        } else {
+          float* so = reinterpret_cast<float*>(x.sm + SM_XH) + dv;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) so[(n0 + e) * DVB] = (ya[e] + yb[e]) + (oa[e] + ob[e]);
+        }
       }
     }
     fence_proxy_async_smem();
@@ -815,7 +823,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
   }
 }
 
-template <bool PRE, int DVB, bool DV2>
+template <bool PRE, int DVB, bool DV2, bool OBF = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -858,7 +866,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     issue_g(x, &tm_g, 0, h, b);
   }
   if (warp < 4 || warp >= 12)
-    chain_role<DVB, DV2>(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
+    chain_role<DVB, DV2, OBF>(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
   else
     side_role<PRE>(x, &tm_q, &tm_k, &tm_g, p, b, h, ntiles);
 
@@ -901,7 +909,18 @@ int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     return true;
   };
   bool ok;
-  if (a.Dv == D)
+  if (a.o_bf16) {
+    // bf16 o: the pre-step instantiations (with none requested their factors are
+    // exactly 1, so o is the fp32 call's o rounded)
+    if (a.Dv == D)
+      ok = go(kda_prefill_kernel<true, 128, false, true>, 43, chains);
+    else if (a.Dv == 2 * D)
+      ok = go(kda_prefill_kernel<true, 128, true, true>, 44, 2 * chains);
+    else if (a.Dv == 64)
+      ok = go(kda_prefill_kernel<true, 64, false, true>, 45, chains);
+    else
+      return -1;
+  } else if (a.Dv == D)
     ok = pre ? go(kda_prefill_kernel<true, 128, false>, 48, chains)
              : go(kda_prefill_kernel<false, 128, false>, 15, chains);
   else if (a.Dv == 2 * D)  // two CTAs per chain

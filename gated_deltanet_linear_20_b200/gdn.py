@@ -403,15 +403,17 @@ def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
                 beta: torch.Tensor, S0: Optional[torch.Tensor] = None, *,
                 o: Optional[torch.Tensor] = None, S_T: Optional[torch.Tensor] = None,
                 status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
-                q_scale: float = 1.0) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Per-channel-gate (KDA) prefill: returns (o [B,T,H,Dv] fp32, S_T [B,H,Dv,Dk] fp32).
+                q_scale: float = 1.0, o_bf16: bool = False) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-channel-gate (KDA) prefill: returns (o [B,T,H,Dv] fp32, or bf16 with
+    ``o_bf16``, S_T [B,H,Dv,Dk] fp32).
 
     q, k [B,T,H,Dk] bf16; v [B,T,H,Dv] bf16; g [B,T,H,Dk] fp32 (log decay per key
     channel); beta [B,T,H] fp32; S0 [B,H,Dv,Dk] fp32 or None (zeros).  ``S_T``
     may be ``S0`` (in place).  ``qk_l2norm`` / ``q_scale`` normalise q and k per
-    token and head and scale q inside the kernel (gdn_kda_prefill_ex; Dk = 128).
-    Dk = 128 runs the chunked tensor-core kernel (Dv 64, 128 or 256); Dk = 64 or
-    256 the row kernel.  Launches on the current stream."""
+    token and head and scale q inside the kernel, and ``o_bf16`` writes o as bf16
+    (gdn_kda_prefill_ex; Dk = 128).  Dk = 128 runs the chunked tensor-core kernel
+    (Dv 64, 128 or 256); Dk = 64 or 256 the row kernel.  Launches on the current
+    stream."""
     if q.dim() != 4:
         raise ValueError("q must be [B,T,H,Dk]")
     B, T, H, Dk = q.shape
@@ -426,13 +428,14 @@ def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     _check(beta, "beta", torch.float32, (B, T, H), dev)
     if S0 is not None:
         _check(S0, "S0", torch.float32, (B, H, Dv, Dk), dev)
+    o_dtype = torch.bfloat16 if o_bf16 else torch.float32
     if o is None:
-        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
-    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
+        o = torch.empty((B, T, H, Dv), dtype=o_dtype, device=dev)
+    _check(o, "o", o_dtype, (B, T, H, Dv), dev)
     if S_T is None:
         S_T = torch.empty((B, H, Dv, Dk), dtype=torch.float32, device=dev)
     _check(S_T, "S_T", torch.float32, (B, H, Dv, Dk), dev)
-    opts = _options(qk_l2norm, q_scale)
+    opts = _options(qk_l2norm, q_scale, o_bf16)
     if opts is None:
         rc = _lib.gdn_kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
                                   _ptr(S_T), B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))
@@ -447,13 +450,13 @@ def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
 def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
                status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
-               q_scale: float = 1.0) -> torch.Tensor:
+               q_scale: float = 1.0, o_bf16: bool = False) -> torch.Tensor:
     """Per-channel-gate (KDA) decode; S [B,H,Dv,Dk] fp32 is updated in place.
 
     One token: q, k [B,H,Dk], v [B,H,Dv], g [B,H,Dk], beta [B,H] -> o [B,H,Dv].
     T tokens: the same with a T axis after B ([B,T,H,...]) -> o [B,T,H,Dv].
-    ``qk_l2norm`` / ``q_scale`` as for ``kda_prefill`` (gdn_kda_decode_ex; 128 x 128
-    or 64 x 64)."""
+    ``qk_l2norm`` / ``q_scale`` / ``o_bf16`` as for ``kda_prefill``
+    (gdn_kda_decode_ex; 128 x 128 or 64 x 64)."""
     one = q.dim() == 3
     if one:
         q, k, v, g, beta = (x.unsqueeze(1) for x in (q, k, v, g, beta))
@@ -472,10 +475,11 @@ def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tenso
     _check(g, "g", torch.float32, (B, T, H, Dk), dev)
     _check(beta, "beta", torch.float32, (B, T, H), dev)
     _check(S, "S", torch.float32, (B, H, Dv, Dk), dev)
+    o_dtype = torch.bfloat16 if o_bf16 else torch.float32
     if o is None:
-        o = torch.empty((B, T, H, Dv), dtype=torch.float32, device=dev)
-    _check(o, "o", torch.float32, (B, T, H, Dv), dev)
-    opts = _options(qk_l2norm, q_scale)
+        o = torch.empty((B, T, H, Dv), dtype=o_dtype, device=dev)
+    _check(o, "o", o_dtype, (B, T, H, Dv), dev)
+    opts = _options(qk_l2norm, q_scale, o_bf16)
     if opts is None:
         rc = _lib.gdn_kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
                                  B, T, H, Dk, Dv, _ptr(status), _stream_handle(dev))

@@ -321,10 +321,10 @@ int gdn_kda_decode(const void* q, const void* k, const void* v, const float* g,
 
 /* gdn_kda_prefill / gdn_kda_decode with options (gdn_options; NULL = none).
  * qk_l2norm and q_scale are applied to each token's q and k before any decay,
- * as in gdn_prefill_ex; they need Dk = 128 in the prefill (any Dv), and
- * 128 x 128 or 64 x 64 in decode (else GDN_ERR_UNSUPPORTED).
- * o_bf16 is not offered with the per-channel gate: a nonzero o_bf16 (or an
- * invalid struct) returns GDN_ERR_UNSUPPORTED.  Everything else as for the
+ * as in gdn_prefill_ex, and o_bf16 writes o as bf16 (the fp32 value rounded
+ * to nearest even; o then needs B*T*H*Dv*2 bytes); they need Dk = 128 in the
+ * prefill (any Dv), and 128 x 128 or 64 x 64 in decode (else
+ * GDN_ERR_UNSUPPORTED, as for an invalid struct).  Everything else as for the
  * calls without options. */
 int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float* g,
                        const float* beta, const float* S0, float* o, float* S_T, int B, int T,

@@ -427,10 +427,11 @@ def test_plain_c_client_links_and_gets_the_documented_codes(gdn, tmp_path):
 
 
 def test_kda_options_validation(gdn):
-    """gdn_kda_prefill_ex / gdn_kda_decode_ex: the fused norm and q scale exist
-    with Dk = 128 in the prefill, and at 128 x 128 and 64 x 64 in decode; o_bf16
-    and invalid structs are GDN_ERR_UNSUPPORTED; valid options where they exist
-    pass validation (then fail only for want of a device)."""
+    """gdn_kda_prefill_ex / gdn_kda_decode_ex: the fused norm, q scale and bf16
+    o exist with Dk = 128 in the prefill, and at 128 x 128 and 64 x 64 in
+    decode; elsewhere, and for invalid structs, GDN_ERR_UNSUPPORTED; valid
+    options where they exist pass validation (then fail only for want of a
+    device)."""
     import ctypes as ct
     good = gdn.Options(ct.sizeof(gdn.Options), 1, 0.5, 0)
     bf16 = gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 1)
@@ -438,7 +439,8 @@ def test_kda_options_validation(gdn):
     a = kda_args()
     ins = lambda args, o: args[:13] + [ct.byref(o)] + args[13:]
     assert gdn.raw_kda_prefill_ex(*ins(a, good)) not in (0, -1, -2, -3, -4, -5)
-    assert gdn.raw_kda_prefill_ex(*ins(a, bf16)) == -4
+    assert gdn.raw_kda_prefill_ex(*ins(a, bf16)) not in (0, -1, -2, -3, -4, -5)
+    assert gdn.raw_kda_prefill_ex(*ins(kda_args(Dk=64, Dv=64), bf16)) == -4
     assert gdn.raw_kda_prefill_ex(*ins(a, short)) == -4
     assert gdn.raw_kda_prefill_ex(*ins(kda_args(Dk=64, Dv=64), good)) == -4
     for dv in (64, 256):  # Dk = 128: the tensor-core kernel, with the options
@@ -448,7 +450,8 @@ def test_kda_options_validation(gdn):
          P + 0x5000000, 4, 1, 2, 128, 128]
     tail = [None, None]
     assert gdn.raw_kda_decode_ex(*(d + [ct.byref(good)] + tail)) not in (0, -1, -2, -3, -4, -5)
-    assert gdn.raw_kda_decode_ex(*(d + [ct.byref(bf16)] + tail)) == -4
+    assert gdn.raw_kda_decode_ex(*(d + [ct.byref(bf16)] + tail)) not in (0, -1, -2, -3, -4, -5)
+    assert gdn.raw_kda_decode_ex(*(d[:10] + [64, 128] + [ct.byref(bf16)] + tail)) == -4
     d64 = d[:10] + [64, 64]
     assert gdn.raw_kda_decode_ex(*(d64 + [ct.byref(good)] + tail)) not in (0, -1, -2, -3, -4, -5)
     assert gdn.raw_kda_decode_ex(*(d64 + [None] + tail)) not in (0, -1, -2, -3, -4, -5)

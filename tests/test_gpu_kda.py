@@ -313,3 +313,34 @@ def test_kda_decode_long_bursts(T):
     ro, rS = oracle.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
     assert_parity(o.cpu().numpy(), ro, f"o kda burst T={T}")
     assert_parity(S.cpu().numpy(), rS, f"S kda burst T={T}")
+
+
+
+@pytest.mark.parametrize("dv", [128, 64, 256])
+def test_kda_bf16_o_is_the_fp32_o_rounded(dv):
+    """o_bf16 in the per-channel-gate prefill stores the fp32 call's o rounded
+    to nearest even, bit for bit, with an identical end state (T = 100: whole
+    and ragged 32-token tiles); with the fused norm too at 128 x 128."""
+    gdn = _gdn()
+    d = to_dev(inputs.kda_inputs(2, 100, 3, 128, dv, seed=180 + dv, s0_std=0.05))
+    for kw in ({}, dict(qk_l2norm=True, q_scale=0.25)) if dv == 128 else ({},):
+        o32, S32 = gdn.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], **kw)
+        o16, S16 = gdn.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"], o_bf16=True, **kw)
+        torch.cuda.synchronize()
+        assert o16.dtype == torch.bfloat16
+        assert torch.equal(o16, o32.to(torch.bfloat16)), f"dv={dv} {kw}"
+        assert torch.equal(S16, S32), f"dv={dv} {kw}"
+
+
+@pytest.mark.parametrize("D,T", [(128, 1), (128, 5), (64, 1), (64, 3)])
+def test_kda_bf16_o_in_decode(D, T):
+    gdn = _gdn()
+    d = to_dev(inputs.kda_inputs(8, T, 4, D, D, seed=190 + D + T, s0_std=0.05))
+    S32 = d["S0"].clone()
+    S16 = d["S0"].clone()
+    args = [d[key] for key in ("q", "k", "v", "g", "beta")]
+    o32 = gdn.kda_decode(*args, S32)
+    o16 = gdn.kda_decode(*args, S16, o_bf16=True)
+    torch.cuda.synchronize()
+    assert o16.dtype == torch.bfloat16
+    assert torch.equal(o16, o32.to(torch.bfloat16)) and torch.equal(S16, S32)
