@@ -667,7 +667,8 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
     tensor-core kernel (32-token chunks; HBM roofline, with the tensor fraction
     of the same chunk-GEMM FLOP count as the scalar gate beside it), at the
     512-token single-sequence shape and a large batch, and at 128 x 256 (two
-    CTAs per chain) at the 512-token shape; a 4-token decode burst; and the batched decode
+    CTAs per chain) at the 512-token shape; 32 packed sequences of mixed lengths;
+    a 4-token decode burst; and the batched decode
     step at 128 x 128 and 64 x 64 on the streaming decode kernel (HBM
     roofline)."""
     from gated_deltanet_linear_20_b200 import gdn
@@ -708,6 +709,26 @@ def run_kda_extras(dev, stream, flush, peaks, rank, steps):
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}}
     del d, o, sT
+    # packed sequences of mixed lengths (one pass per sequence and head)
+    rng = np.random.default_rng(4000 + rank)
+    lens = rng.integers(64, 2049, size=32)
+    seqs = [gin.kda_inputs(1, int(L), 16, seed=5200 + 37 * rank + i, device=str(dev))
+            for i, L in enumerate(lens)]
+    pk = {key: torch.cat([d[key][0] for d in seqs], 0) for key in ("q", "k", "v", "g", "beta")}
+    del seqs
+    cu = torch.tensor([0] + np.cumsum(lens).tolist(), dtype=torch.int32, device=dev)
+    ms = time_steps(lambda: gdn.kda_prefill_varlen(pk["q"], pk["k"], pk["v"], pk["g"], pk["beta"],
+                                                   cu), steps, 3, flush, stream)
+    t = statistics.mean(ms)
+    ntok = int(lens.sum())
+    nb = kda_prefill_bytes(1, ntok, 16, False) + (len(lens) - 1) * 16 * STATE_BYTES
+    out["kda_prefill_varlen_32seq_h16"] = {
+        "tokens": ntok, "lengths": "32 sequences, seeded uniform 64..2048",
+        "tokens_per_s": round(ntok / (t / 1e3), 1), "ms": round(t, 4),
+        "kernel": "chunked tcgen05, chunk 32, one pass per sequence and head",
+        "hbm_frac": round(nb / (t / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
+    del pk, cu
+    torch.cuda.empty_cache()
     # decode: one token for 64 x 16 heads, state in place, L2 flushed per step
     B, H = 64, 16
     for Dh in (D, 64):

@@ -22,12 +22,13 @@ generator) can be used without loading the CUDA library.
 from __future__ import annotations
 
 __all__ = ["prefill", "decode_step", "decode_tokens", "prefill_varlen", "kda_prefill",
-           "kda_decode", "abi_version", "status_str", "query_status", "GDNError"]
+           "kda_prefill_varlen", "kda_decode", "abi_version", "status_str", "query_status",
+           "GDNError"]
 
 
 def __getattr__(name):
     if name in ("prefill", "decode_step", "decode_tokens", "prefill_varlen", "kda_prefill",
-                "kda_decode", "abi_version", "status_str", "query_status", "GDNError",
+                "kda_prefill_varlen", "kda_decode", "abi_version", "status_str", "query_status", "GDNError",
                 "library_path"):
         import importlib
         return getattr(importlib.import_module(__name__ + ".gdn"), name)

@@ -353,9 +353,9 @@ int static_workspace(void** out) {
 
 namespace gdn {
 bool ensure_smem_attr(const void* func, int slot, int bytes) {
-  static std::atomic<uint64_t> done[64];  // bit d: device d, per kernel slot
+  static std::atomic<uint64_t> done[96];  // bit d: device d, per kernel slot
   int dev = 0;
-  if (slot < 0 || slot >= 64 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+  if (slot < 0 || slot >= 96 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
     return false;
   const uint64_t bit = uint64_t(1) << dev;
   if (done[slot].load(std::memory_order_acquire) & bit) return true;
@@ -623,6 +623,60 @@ int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float*
                   o_bf16 ? 2 : 4, Dv, 32))
     return GDN_ERR_LAUNCH;
   gdn::KdaArgs a{g, beta, S0, S_T, B, T, H, status, qk_norm, q_scale, Dv, o_bf16};
+  return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
+             ? GDN_OK
+             : GDN_ERR_LAUNCH;
+}
+
+int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* S0, float* o, float* S_T,
+                           const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
+                           int* status, void* stream) {
+  if (N < 0 || total_T < 0 || H < 0) return GDN_ERR_SHAPE;
+  if (Dk != kHeadDim || (Dv != 64 && Dv != kHeadDim && Dv != 2 * kHeadDim)) return GDN_ERR_UNSUPPORTED;
+  const long long chains = (long long)N * H;
+  if ((long long)total_T * H * Dv > 0x7fffffffLL || (long long)total_T * H * kHeadDim > 0x7fffffffLL ||
+      chains * kHeadDim * Dv > 0x7fffffffLL)
+    return GDN_ERR_SHAPE;
+  if (chains == 0) return GDN_OK;
+  if (!S_T || !cu_seqlens) return GDN_ERR_NULL;
+  if (total_T > 0 && (!q || !k || !v || !g || !beta || !o)) return GDN_ERR_NULL;
+  if (!aligned(S_T, 16) || (S0 && !aligned(S0, 16)) || !aligned(cu_seqlens, 4)) return GDN_ERR_ALIGN;
+  if (total_T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(g, 16) ||
+                      !aligned(o, 16) || !aligned(beta, 4)))
+    return GDN_ERR_ALIGN;
+  const size_t toks = size_t(total_T) * H;
+  const size_t act_bf16 = toks * kHeadDim * 2, v_bf16 = toks * Dv * 2, o_bytes = toks * Dv * 4;
+  const size_t g_bytes = toks * kHeadDim * 4, beta_bytes = toks * 4;
+  const size_t state_bytes = size_t(chains) * kHeadDim * Dv * 4, cu_bytes = size_t(N + 1) * 4;
+  if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
+  if (overlaps(S_T, state_bytes, cu_seqlens, cu_bytes)) return GDN_ERR_ALIAS;
+  if (total_T > 0) {
+    const void* ins[6] = {q, k, v, g, beta, cu_seqlens};
+    const size_t in_bytes[6] = {act_bf16, act_bf16, v_bf16, g_bytes, beta_bytes, cu_bytes};
+    for (int i = 0; i < 6; ++i)
+      if (overlaps(o, o_bytes, ins[i], in_bytes[i]) ||
+          (i < 5 && overlaps(S_T, state_bytes, ins[i], in_bytes[i])))
+        return GDN_ERR_ALIAS;
+    if (overlaps(o, o_bytes, S_T, state_bytes) || overlaps(o, o_bytes, S0, state_bytes))
+      return GDN_ERR_ALIAS;
+  }
+  const int dev_ok = check_device();
+  if (dev_ok != GDN_OK) return dev_ok;
+  // the views are [1][total_T][H][..]; with every sequence empty they are one
+  // never-read token of S_T (which holds at least Dk Dv >= Dk, Dv floats)
+  const int Tv = total_T > 0 ? total_T : 1;
+  const auto pick = [&](const void* a) { return total_T > 0 ? a : static_cast<const void*>(S_T); };
+  CUtensorMap tq{}, tk{}, tv{}, to{}, tg{};
+  const int dv_box = Dv < kHeadDim ? Dv : kHeadDim;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  if (!encode_act(&tg, pick(g), 1, Tv, H, 128, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, kHeadDim, 32) ||
+      !encode_act(&tq, pick(q), 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
+      !encode_act(&tk, pick(k), 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
+      !encode_act(&tv, pick(v), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv, 32) ||
+      !encode_act(&to, pick(o), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, Dv, 32))
+    return GDN_ERR_LAUNCH;
+  gdn::KdaArgs a{g, beta, S0, S_T, N, total_T, H, status, 0, 1.f, Dv, 0, cu_seqlens, o};
   return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK
              : GDN_ERR_LAUNCH;

@@ -93,6 +93,8 @@ struct KdaArgs {
   float q_scale;      // q multiplied by this after the normalisation
   int Dv;             // 64, 128 or 256 (Dk is 128)
   int o_bf16;         // o written as bf16
+  const int* cu_seqlens = nullptr;  // packed sequences: [B + 1] token offsets (views with B = 1)
+  float* o = nullptr;               // o (fp32), for the packed last tile's row copy
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device

@@ -212,11 +212,12 @@ __device__ __forceinline__ bool lead_wait(const Ctx& x, uint32_t bar, uint32_t p
   return false;
 }
 
+// tb: the token coordinate of tile 0 (a packed sequence's first token, else 0)
 __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
-                                         int c, int h, int b) {
+                                         int c, int h, int b, int tb) {
   const uint32_t bar = x.bar(B_KQFULL);
   mbar_arrive_expect_tx(bar, KQ_TX_BYTES);
-  const int t0 = c * NT;
+  const int t0 = tb + c * NT;
   tma_load_4d(x.sb + SM_KQ + 0, tk, bar, 0, h, t0, b);
   tma_load_4d(x.sb + SM_KQ + 4096, tq, bar, 0, h, t0, b);
   tma_load_4d(x.sb + SM_KQ + 8192, tk, bar, 64, h, t0, b);
@@ -225,19 +226,20 @@ __device__ __forceinline__ void issue_kq(const Ctx& x, const CUtensorMap* tq, co
 }
 // V rows dv0 .. dv0 + DVB - 1 of tile c ([32 tokens][DVB] bf16)
 template <int DVB>
-__device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b, int dv0) {
+__device__ __forceinline__ void issue_v(const Ctx& x, const CUtensorMap* tv, int c, int h, int b, int dv0,
+                                        int tb) {
   const uint32_t bar = x.bar(B_VFULL);
   mbar_arrive_expect_tx(bar, uint32_t(NT * DVB * 2));
-  tma_load_4d(x.sb + SM_V, tv, bar, dv0, h, c * NT, b);
+  tma_load_4d(x.sb + SM_V, tv, bar, dv0, h, tb + c * NT, b);
   *x.misc(M_V_ISSUED) = c + 1;
 }
 
 // g of tile c ([32 tokens][128] fp32; tokens past T read as 0), issued once
 // every side thread has read tile c - 1's
-__device__ __forceinline__ void issue_g(const Ctx& x, const CUtensorMap* tg, int c, int h, int b) {
+__device__ __forceinline__ void issue_g(const Ctx& x, const CUtensorMap* tg, int c, int h, int b, int tb) {
   const uint32_t bar = x.bar(B_GLD);
   mbar_arrive_expect_tx(bar, G_TX_BYTES);
-  tma_load_4d(x.sb + SM_G, tg, bar, 0, h, c * NT, b);
+  tma_load_4d(x.sb + SM_G, tg, bar, 0, h, tb + c * NT, b);
   *x.misc(M_G_ISSUED) = c + 1;
 }
 
@@ -246,10 +248,13 @@ __device__ __forceinline__ void issue_g(const Ctx& x, const CUtensorMap* tg, int
 // qt = kt / 64 (tokens 8qt .. 8qt+7 of the tile) for the gates and operands;
 // TMEM lane quarter (warp % 4) and column half for the masks.
 // PRE: q and k are L2-normalised per token and head (and q scaled) on the way
-// in, before any decay is applied.
-template <bool PRE>
+// in, before any decay is applied.  PK: a packed sequence (tokens tb .. tend - 1
+// of the views): tokens of the next sequence in its last tile are made padding
+// (g = beta = 0, an exact identity).
+template <bool PRE, bool PK>
 __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap* tk,
-                          const CUtensorMap* tg, const KdaArgs& p, int b, int h, int ntiles) {
+                          const CUtensorMap* tg, const KdaArgs& p, int b, int h, int ntiles, int tb,
+                          int tend) {
   const int kt = threadIdx.x - 128;
   const int warp = threadIdx.x >> 5;
   const int lq = warp & 3;
@@ -274,7 +279,7 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
   RoleSync rs{BAR_SIDE, SIDE_THREADS, M_FLAG_SIDE, leader, 0};
   // beta of token kt of the next tile, loaded one tile ahead (kt < 32)
   float beta_next = 0.f;
-  if (kt < NT && kt < p.T) beta_next = __ldg(p.beta + (size_t(b) * p.T + kt) * p.H + h);
+  if (kt < NT && tb + kt < tend) beta_next = __ldg(p.beta + (size_t(b) * p.T + tb + kt) * p.H + h);
 
   for (int c = 0; c < ntiles; ++c) {
     // ---- 1. gates: g of this thread's 8 tokens x 2 channels (from the tile's
@@ -291,9 +296,14 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
       const float* sg = reinterpret_cast<const float*>(x.sm + SM_G);
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        const float2 g2 = *reinterpret_cast<const float2*>(sg + (8 * qt + t) * D + d0);
-        gm[t][0] = g2.x * LOG2E;
-        gm[t][1] = g2.y * LOG2E;
+        float2 g2 = *reinterpret_cast<const float2*>(sg + (8 * qt + t) * D + d0);
+        if constexpr (PK) {
+          if (tb + c * NT + 8 * qt + t >= tend) g2 = make_float2(0.f, 0.f);
+        }
+        // rounded products (never contracted into the sums below): the packed
+        // instantiation, which selects g first, then rounds exactly as this one
+        gm[t][0] = __fmul_rn(g2.x, LOG2E);
+        gm[t][1] = __fmul_rn(g2.y, LOG2E);
       }
 #pragma unroll
       for (int t = 1; t < 8; ++t) {
@@ -303,13 +313,13 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
       *reinterpret_cast<float2*>(sX + qt * 128 + d0) = make_float2(gm[7][0], gm[7][1]);
       if (kt < NT) {
         x.gates(c)[G_B / 4 + kt] = beta_next;
-        const int tok = (c + 1) * NT + kt;
-        beta_next = tok < p.T ? __ldg(p.beta + (size_t(b) * p.T + tok) * p.H + h) : 0.f;
+        const int tok = tb + (c + 1) * NT + kt;
+        beta_next = tok < tend ? __ldg(p.beta + (size_t(b) * p.T + tok) * p.H + h) : 0.f;
       }
     }
     named_bar(BAR_SIDE, SIDE_THREADS);
     // every thread has read g(c): the buffer takes g(c + 1)
-    if (leader && c + 1 < ntiles) issue_g(x, tg, c + 1, h, b);
+    if (leader && c + 1 < ntiles) issue_g(x, tg, c + 1, h, b, tb);
     float gref[2], glast[2];
     {
       float pre[2] = {0.f, 0.f}, tot[2] = {0.f, 0.f}, half[2] = {0.f, 0.f};
@@ -456,7 +466,7 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
     {
       bool ok = true;
       if (leader) {
-        if (c + 1 < ntiles) issue_kq(x, tq, tk, c + 1, h, b);
+        if (c + 1 < ntiles) issue_kq(x, tq, tk, c + 1, h, b, tb);
         tc_fence_after();
         const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0);
         const uint64_t da = sdesc_sw128(sb + SM_PA, 16, 1024), db = sdesc_sw128(sb + SM_PB, 16, 1024);
@@ -600,9 +610,9 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
 // DVB: rows of the state this CTA owns (64 or 128); DV2: two CTAs per chain
 // (Dv = 256), this one owning rows dv0 = 128 (blockIdx & 1) ..; OBF: o is
 // bf16 (the fp32 value rounded to nearest even, through a bf16 TMA view)
-template <int DVB, bool DV2, bool OBF>
+template <int DVB, bool DV2, bool OBF, bool PK>
 __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMap* tmo,
-                           const KdaArgs& p, int chain, int b, int h, int ntiles) {
+                           const KdaArgs& p, int chain, int b, int h, int ntiles, int tb, int tend) {
   constexpr int DVW = DV2 ? 2 * D : DVB;  // Dv: rows of the chain's state
   const int dv0 = DV2 ? D * (int(blockIdx.x) & 1) : 0;
   const int warp = threadIdx.x >> 5;
@@ -696,7 +706,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
     // ---- Dl^T = X^T T^T: X hi x [T hi; T lo] (N=64), X lo x T hi (N=32); K = 32,
     //      A from tensor memory (K step ks = the tokens of chain half ks)
     if (leader) {
-      if (!last) issue_v<DVB>(x, tv, c + 1, h, b, dv0);  // V(c) has been read
+      if (!last) issue_v<DVB>(x, tv, c + 1, h, b, dv0, tb);  // V(c) has been read
       if (lead_wait(x, x.bar(B_TMFULL), c & 1)) {
         tc_fence_after();
         const uint32_t id64 = idesc_bf16(128, 64, 0, 0, 0), id32 = idesc_bf16(128, 32, 0, 0, 0);
@@ -778,9 +788,23 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
     fence_proxy_async_smem();
     tc_fence_before();
     named_bar(BAR_CHAIN, CHAIN_THREADS);
-    if (leader) {
-      tma_store_4d(tmo, sb + SM_XH, dv0, h, c * NT, b);
-      bulk_commit();
+    if (!PK || tb + (c + 1) * NT <= tend || tend == p.T) {
+      // a whole tile, or the view's own end clips it
+      if (leader) {
+        tma_store_4d(tmo, sb + SM_XH, dv0, h, tb + c * NT, b);
+        bulk_commit();
+      }
+    } else if constexpr (PK && !OBF) {
+      // the last tile of a packed sequence: the rows past it are the next
+      // sequence's, so only the valid rows are copied out, 16 bytes at a time
+      const int nvalid = tend - (tb + c * NT);
+      const float4* src = reinterpret_cast<const float4*>(x.sm + SM_XH);
+      float* dst = p.o + (size_t(tb + c * NT) * p.H + h) * DVW + dv0;
+      const int ct = (warp >= 12 ? 128 : 0) + lq * 32 + (threadIdx.x & 31);  // 0 .. 255
+      for (int i = ct; i < nvalid * (DVB / 4); i += CHAIN_THREADS) {
+        const int r = i / (DVB / 4), j = i % (DVB / 4);
+        reinterpret_cast<float4*>(dst + size_t(r) * p.H * DVW)[j] = src[i];
+      }
     }
     // ---- state epilogue: the update has completed (its commit preceded the
     //      output product's); refresh hi/lo and pre-scale by the next tile's
@@ -823,7 +847,7 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
   }
 }
 
-template <bool PRE, int DVB, bool DV2, bool OBF = false>
+template <bool PRE, int DVB, bool DV2, bool OBF = false, bool PK = false>
 __global__ void __launch_bounds__(NTHREADS, 1)
     kda_prefill_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -834,8 +858,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int chain = DV2 ? int(blockIdx.x) >> 1 : int(blockIdx.x);
-  const int b = chain / p.H, h = chain - (chain / p.H) * p.H;
-  const int ntiles = (p.T + NT - 1) / NT;
+  int b = chain / p.H;
+  const int h = chain - (chain / p.H) * p.H;
+  int ntiles = (p.T + NT - 1) / NT;
+  int tb = 0, tend = p.T;  // this chain's tokens in the views
+  if constexpr (PK) {
+    // packed sequences: chain n H + h walks tokens [cu[n], cu[n+1]) of views with B = 1
+    tb = __ldg(p.cu_seqlens + b);
+    tend = __ldg(p.cu_seqlens + b + 1);
+    if (tb < 0 || tend < tb || tend > p.T) {
+      if (tid == 0 && p.status) atomicExch(p.status, GDN_ERR_SHAPE);
+      return;
+    }
+    b = 0;
+    ntiles = (tend - tb + NT - 1) / NT;
+    if (ntiles == 0) {  // an empty sequence: S_T = S0 (or zeros), this CTA's rows
+      const int rows = DVB;
+      const size_t off = size_t(chain) * (DV2 ? 2 * D : DVB) * D +
+                         size_t(DV2 ? D * (int(blockIdx.x) & 1) : 0) * D;
+      const float4* src = p.S0 ? reinterpret_cast<const float4*>(p.S0 + off) : nullptr;
+      float4* dst = reinterpret_cast<float4*>(p.S_T + off);
+      for (int i = tid; i < rows * D / 4; i += NTHREADS)
+        dst[i] = src ? src[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      return;
+    }
+  }
 
   Ctx x;
   x.sm = sm;
@@ -861,14 +908,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   x.tmem = *reinterpret_cast<volatile uint32_t*>(sm + SM_MISC + M_TMEM);
   if (tid == 0) {
-    issue_kq(x, &tm_q, &tm_k, 0, h, b);
-    issue_v<DVB>(x, &tm_v, 0, h, b, DV2 ? D * (int(blockIdx.x) & 1) : 0);
-    issue_g(x, &tm_g, 0, h, b);
+    issue_kq(x, &tm_q, &tm_k, 0, h, b, tb);
+    issue_v<DVB>(x, &tm_v, 0, h, b, DV2 ? D * (int(blockIdx.x) & 1) : 0, tb);
+    issue_g(x, &tm_g, 0, h, b, tb);
   }
   if (warp < 4 || warp >= 12)
-    chain_role<DVB, DV2, OBF>(x, &tm_v, &tm_o, p, chain, b, h, ntiles);
+    chain_role<DVB, DV2, OBF, PK>(x, &tm_v, &tm_o, p, chain, b, h, ntiles, tb, tend);
   else
-    side_role<PRE>(x, &tm_q, &tm_k, &tm_g, p, b, h, ntiles);
+    side_role<PRE, PK>(x, &tm_q, &tm_k, &tm_g, p, b, h, ntiles, tb, tend);
 
   // each MMA-issuing thread waits (bounded) for its own products in flight
   if (tid == 0 || tid == 128 || tid == OI_ISSUER) {
@@ -900,7 +947,7 @@ int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        const CUtensorMap& to, const CUtensorMap& tg, const KdaArgs& a,
                        cudaStream_t stream) {
   const int chains = a.B * a.H;
-  if (chains == 0 || a.T == 0) return -1;
+  if (chains == 0 || (a.T == 0 && !a.cu_seqlens)) return -1;
   const uint32_t smem = SMEM_USED + 1024;
   const bool pre = a.qk_norm || a.q_scale != 1.f;
   auto go = [&](auto kernel, int slot, int ctas) {
@@ -909,7 +956,16 @@ int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     return true;
   };
   bool ok;
-  if (a.o_bf16) {
+  if (a.cu_seqlens) {  // packed sequences (fp32 o, no pre-steps)
+    if (a.Dv == D)
+      ok = go(kda_prefill_kernel<false, 128, false, false, true>, 64, chains);
+    else if (a.Dv == 2 * D)
+      ok = go(kda_prefill_kernel<false, 128, true, false, true>, 65, 2 * chains);
+    else if (a.Dv == 64)
+      ok = go(kda_prefill_kernel<false, 64, false, false, true>, 66, chains);
+    else
+      return -1;
+  } else if (a.o_bf16) {
     // bf16 o: the pre-step instantiations (with none requested their factors are
     // exactly 1, so o is the fp32 call's o rounded)
     if (a.Dv == D)

@@ -68,10 +68,12 @@ _lib.gdn_kda_prefill_ex.argtypes = [_vp] * 8 + [_ci] * 5 + [_vp, _vp, _vp]
 _lib.gdn_kda_prefill_ex.restype = _ci
 _lib.gdn_kda_decode_ex.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp, _vp]
 _lib.gdn_kda_decode_ex.restype = _ci
+_lib.gdn_kda_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 5 + [_vp, _vp]
+_lib.gdn_kda_prefill_varlen.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
-ABI_VERSION = 7
+ABI_VERSION = 8
 if _lib.gdn_abi_version() != ABI_VERSION:
     raise ImportError(f"libgdn_b200.so ABI {_lib.gdn_abi_version()} != binding ABI {ABI_VERSION}")
 
@@ -447,6 +449,49 @@ def kda_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tens
     return o, S_T
 
 
+def kda_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
+                       beta: torch.Tensor, cu_seqlens: torch.Tensor,
+                       S0: Optional[torch.Tensor] = None, *, o: Optional[torch.Tensor] = None,
+                       S_T: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-channel-gate prefill of N packed sequences (gdn_kda_prefill_varlen):
+    q, k [total_T,H,128] bf16; v [total_T,H,Dv] bf16 (Dv 64, 128 or 256);
+    g [total_T,H,128] fp32; beta [total_T,H] fp32; cu_seqlens int32 [N+1] on
+    the device.  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,128] fp32)."""
+    if q.dim() != 3:
+        raise ValueError("q must be [total_T,H,Dk]")
+    total_T, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("gdn.kda_prefill_varlen runs on CUDA tensors only (no CPU path)")
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+        raise ValueError("cu_seqlens must be [N+1]")
+    N = cu_seqlens.numel() - 1
+    _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+    _check(q, "q", torch.bfloat16, (total_T, H, Dk), dev)
+    _check(k, "k", torch.bfloat16, (total_T, H, Dk), dev)
+    _check(v, "v", torch.bfloat16, (total_T, H, Dv), dev)
+    _check(g, "g", torch.float32, (total_T, H, Dk), dev)
+    _check(beta, "beta", torch.float32, (total_T, H), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (N, H, Dv, Dk), dev)
+    if o is None:
+        o = torch.empty((total_T, H, Dv), dtype=torch.float32, device=dev)
+    _check(o, "o", torch.float32, (total_T, H, Dv), dev)
+    if S_T is None:
+        S_T = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=dev)
+    _check(S_T, "S_T", torch.float32, (N, H, Dv, Dk), dev)
+    if status is not None:
+        _check(status, "status", torch.int32, (1,), dev)
+    rc = _lib.gdn_kda_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                     _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk, Dv,
+                                     _ptr(status), _stream_handle(dev))
+    if rc != GDN_OK:
+        raise GDNError(rc, "gdn_kda_prefill_varlen")
+    return o, S_T
+
+
 def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,
                beta: torch.Tensor, S: torch.Tensor, *, o: Optional[torch.Tensor] = None,
                status: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
@@ -539,3 +584,7 @@ def raw_kda_prefill_ex(*args) -> int:
 
 def raw_kda_decode_ex(*args) -> int:
     return int(_lib.gdn_kda_decode_ex(*args))
+
+
+def raw_kda_prefill_varlen(*args) -> int:
+    return int(_lib.gdn_kda_prefill_varlen(*args))

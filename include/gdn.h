@@ -67,7 +67,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 7
+#define GDN_ABI_VERSION 8
 
 enum gdn_status_code {
   GDN_OK = 0,
@@ -332,6 +332,26 @@ int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float*
 int gdn_kda_decode_ex(const void* q, const void* k, const void* v, const float* g,
                       const float* beta, float* S, float* o, int B, int T, int H, int Dk, int Dv,
                       const gdn_options* opts, int* status, void* stream);
+
+/* gdn_kda_prefill for N sequences of different lengths packed along the token
+ * axis, as in gdn_prefill_varlen: sequence n is tokens cu_seqlens[n] ..
+ * cu_seqlens[n+1]-1 of the packed arrays, each (sequence, head) one chain of
+ * the per-channel-gate recurrence.
+ *   q, k, g [total_T][H][128]; v, o [total_T][H][Dv]; beta [total_T][H]
+ *   (types and alignment as for gdn_kda_prefill; o fp32)
+ *   S0, S_T [N][H][Dv][128] fp32 (S0 may be NULL; S_T may equal S0)
+ *   cu_seqlens : device int[N+1], 0 = cu_seqlens[0] <= ... <= cu_seqlens[N] =
+ *                total_T.  Offsets out of order or past total_T are detected
+ *                on the device: GDN_ERR_SHAPE goes to *status and that
+ *                sequence's outputs are not written.  Empty sequences are
+ *                allowed (S_T = S0, or zeros).
+ * Dk must be 128 and Dv 64, 128 or 256 (the chunked tensor-core kernel, one
+ * CTA per chain, two with Dv = 256); no options.  Returns GDN_OK, a negative
+ * code for invalid arguments (nothing is launched), as for gdn_kda_prefill. */
+int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
+                           const float* beta, const float* S0, float* o, float* S_T,
+                           const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
+                           int* status, void* stream);
 
 /* Synchronises `stream`, then reads the device status word written by the
  * kernels.  Returns GDN_OK, GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_NULL (status_dev is

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(gdn):
 
 
 def test_abi_version_and_status_strings(gdn):
-    assert gdn.abi_version() == 7
+    assert gdn.abi_version() == 8
     for code in range(-9, 1):
         s = gdn.status_str(code)
         assert s and s != "unknown status code"
@@ -457,3 +457,38 @@ def test_kda_options_validation(gdn):
     assert gdn.raw_kda_decode_ex(*(d64 + [None] + tail)) not in (0, -1, -2, -3, -4, -5)
     d64x128 = d[:10] + [64, 128]
     assert gdn.raw_kda_decode_ex(*(d64x128 + [ct.byref(good)] + tail)) == -4
+
+
+def kda_varlen_args(**over):
+    # N=3 sequences, total_T=200, H=2, Dk=128: q/k 100 KiB each, g 200 KiB, o 200 KiB (Dv 128)
+    a = dict(q=P, k=P + 0x1000000, v=P + 0x2000000, g=P + 0x3000000, beta=P + 0x3100000,
+             S0=None, o=P + 0x5000000, S_T=P + 0x6000000, cu=P + 0x7000000, N=3, total_T=200,
+             H=2, Dk=128, Dv=128, status=None, stream=None)
+    a.update(over)
+    return [a[k] for k in ("q", "k", "v", "g", "beta", "S0", "o", "S_T", "cu", "N", "total_T",
+                           "H", "Dk", "Dv", "status", "stream")]
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(N=-1), -3), (dict(total_T=-1), -3), (dict(H=-1), -3),
+    (dict(Dk=64, Dv=64), -4), (dict(Dk=256), -4), (dict(Dv=32), -4),
+    (dict(cu=None), -1), (dict(S_T=None), -1), (dict(q=None), -1), (dict(g=None), -1),
+    (dict(cu=P + 0x7000002), -2), (dict(g=P + 0x3000004), -2), (dict(o=P + 0x5000008), -2),
+    (dict(S_T=P + 0x6000008), -2),
+    (dict(S0=P + 0x6000000 + 0x1000), -5),         # S0 partly overlaps S_T
+    (dict(o=P + 0x3000000 + 0x100), -5),           # o over g
+    (dict(o=P + 0x7000000 - 64), -5),              # o runs into cu_seqlens
+    (dict(S_T=P + 0x7000000 - 64 * 1024), -5),     # S_T runs into cu_seqlens
+    (dict(S_T=P + 0x2000000 + 0x40), -5),          # S_T over v
+], ids=lambda x: str(x))
+def test_kda_prefill_varlen_rejects_bad_arguments(gdn, over, code):
+    assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(**over)) == code
+
+
+@pytest.mark.parametrize("dv", [64, 128, 256])
+def test_kda_prefill_varlen_valid_calls_pass_validation(gdn, dv):
+    """Dk = 128 with Dv 64, 128 or 256 passes validation (the call then fails
+    only for want of a device); no sequences or no heads is a no-op."""
+    assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(Dv=dv)) not in VALIDATION_CODES + (0,)
+    assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(N=0, q=None, S_T=None)) == 0
+    assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(H=0, cu=None)) == 0

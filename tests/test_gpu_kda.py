@@ -344,3 +344,81 @@ def test_kda_bf16_o_in_decode(D, T):
     torch.cuda.synchronize()
     assert o16.dtype == torch.bfloat16
     assert torch.equal(o16, o32.to(torch.bfloat16)) and torch.equal(S16, S32)
+
+
+def _kda_packed(lengths, H, dv, seed, s0_std=None):
+    """Packed per-channel-gate inputs: per-sequence draws of the seeded
+    generator, concatenated along tokens."""
+    seqs = [inputs.kda_inputs(1, L, H, Dv=dv, seed=seed + i, s0_std=s0_std)
+            for i, L in enumerate(lengths)]
+    cat = lambda key: torch.cat([d[key][0] for d in seqs], 0)
+    S0 = torch.cat([d["S0"] for d in seqs], 0) if s0_std else None
+    cu = torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32)
+    return seqs, dict(q=cat("q"), k=cat("k"), v=cat("v"), g=cat("g"), beta=cat("beta"), S0=S0, cu=cu)
+
+
+@pytest.mark.parametrize("dv,s0", [(128, None), (128, 0.05), (64, 0.05), (256, 0.05)],
+                         ids=["128_zero_state", "128", "64", "256"])
+def test_kda_varlen_packed_sequences(dv, s0):
+    """Packed sequences of mixed lengths (empty, 1 token, ragged, exact 32-token
+    tiles; a ragged sequence last, ending at the end of the packed arrays), each
+    against the oracle run on that sequence alone; an empty sequence's S_T is
+    its S0 (or zeros)."""
+    lengths = [130, 0, 1, 32, 77, 33, 31, 45]
+    H = 2
+    seqs, pk = _kda_packed(lengths, H, dv, seed=700 + dv, s0_std=s0)
+    gdn = _gdn()
+    dd = to_dev(pk)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.kda_prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"],
+                                    dd["S0"], status=status)
+    assert gdn.query_status(status) == 0
+    o, S_T = o.cpu().numpy(), S_T.cpu().numpy()
+    cu = pk["cu"].numpy()
+    for n, d in enumerate(seqs):
+        if lengths[n]:
+            ro, rS = oracle.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+            assert_parity(o[cu[n]:cu[n + 1]], ro[0], f"o seq {n} (len {lengths[n]})")
+            assert_parity(S_T[n], rS[0], f"S_T seq {n} (len {lengths[n]})")
+        elif s0:
+            np.testing.assert_array_equal(S_T[n], d["S0"][0].numpy())
+        else:
+            np.testing.assert_array_equal(S_T[n], 0.0)
+
+
+def test_kda_varlen_equal_lengths_match_the_dense_call():
+    """Equal lengths packed = the dense [B][T][H] call, bitwise: the tokens of
+    the next sequence in a last tile enter as padding (g = beta = 0), which
+    contributes exact zeros, as the zero fill past T does in the dense call."""
+    B, T, H = 3, 150, 4
+    d = to_dev(inputs.kda_inputs(B, T, H, seed=8, s0_std=0.05))
+    gdn = _gdn()
+    o1, S1 = gdn.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+    cu = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=DEV)
+    flat = lambda x: x.reshape(B * T, *x.shape[2:]).contiguous()
+    o2, S2 = gdn.kda_prefill_varlen(flat(d["q"]), flat(d["k"]), flat(d["v"]), flat(d["g"]),
+                                    flat(d["beta"]), cu, d["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(o1.reshape(B * T, H, 128), o2) and torch.equal(S1, S2)
+
+
+def test_kda_varlen_bad_offsets_are_reported_on_the_device():
+    _, pk = _kda_packed([40, 40], 2, 128, seed=3)
+    gdn = _gdn()
+    dd = to_dev(pk)
+    bad = torch.tensor([0, 50, 30], dtype=torch.int32, device=DEV)  # out of order
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gdn.kda_prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], bad, status=status)
+    assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
+
+
+def test_kda_varlen_all_sequences_empty_copy_the_state():
+    H = 3
+    S0 = torch.randn(2, H, 128, 128, device=DEV)
+    e = lambda *s, dt=torch.bfloat16: torch.empty(*s, dtype=dt, device=DEV)
+    cu = torch.zeros(3, dtype=torch.int32, device=DEV)
+    gdn = _gdn()
+    o, S_T = gdn.kda_prefill_varlen(e(0, H, 128), e(0, H, 128), e(0, H, 128),
+                                    e(0, H, 128, dt=torch.float32), e(0, H, dt=torch.float32), cu, S0)
+    torch.cuda.synchronize()
+    assert o.shape == (0, H, 128) and torch.equal(S_T, S0)
