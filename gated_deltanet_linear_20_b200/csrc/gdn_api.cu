@@ -631,9 +631,10 @@ int gdn_kda_prefill_ex(const void* q, const void* k, const void* v, const float*
 int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, const float* S0, float* o, float* S_T,
                            const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
-                           int* status, void* stream) {
-  if (N < 0 || total_T < 0 || H < 0) return GDN_ERR_SHAPE;
+                           float* snaps, int snap_every, int n_snaps, int* status, void* stream) {
+  if (N < 0 || total_T < 0 || H < 0 || n_snaps < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || (Dv != 64 && Dv != kHeadDim && Dv != 2 * kHeadDim)) return GDN_ERR_UNSUPPORTED;
+  if (snaps && (snap_every <= 0 || snap_every % 32 != 0)) return GDN_ERR_UNSUPPORTED;
   const long long chains = (long long)N * H;
   if ((long long)total_T * H * Dv > 0x7fffffffLL || (long long)total_T * H * kHeadDim > 0x7fffffffLL ||
       chains * kHeadDim * Dv > 0x7fffffffLL)
@@ -661,6 +662,17 @@ int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const fl
     if (overlaps(o, o_bytes, S_T, state_bytes) || overlaps(o, o_bytes, S0, state_bytes))
       return GDN_ERR_ALIAS;
   }
+  if (snaps) {
+    const size_t snap_bytes = size_t(n_snaps) * H * kHeadDim * Dv * 4;
+    if (!aligned(snaps, 16)) return GDN_ERR_ALIGN;
+    const void* others[8] = {q, k, v, g, beta, o, S_T, S0};
+    const size_t other_bytes[8] = {act_bf16, act_bf16, v_bf16, g_bytes, beta_bytes, o_bytes,
+                                   state_bytes, state_bytes};
+    for (int i = 0; i < 8; ++i)
+      if ((i >= 6 || total_T > 0) && overlaps(snaps, snap_bytes, others[i], other_bytes[i]))
+        return GDN_ERR_ALIAS;
+    if (overlaps(snaps, snap_bytes, cu_seqlens, cu_bytes)) return GDN_ERR_ALIAS;
+  }
   const int dev_ok = check_device();
   if (dev_ok != GDN_OK) return dev_ok;
   // the views are [1][total_T][H][..]; with every sequence empty they are one
@@ -676,7 +688,8 @@ int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const fl
       !encode_act(&tv, pick(v), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv, 32) ||
       !encode_act(&to, pick(o), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, Dv, 32))
     return GDN_ERR_LAUNCH;
-  gdn::KdaArgs a{g, beta, S0, S_T, N, total_T, H, status, 0, 1.f, Dv, 0, cu_seqlens, o};
+  gdn::KdaArgs a{g,  beta, S0, S_T,        N, total_T, H,     status, 0, 1.f, Dv, 0, cu_seqlens,
+                 o,  snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0};
   return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK
              : GDN_ERR_LAUNCH;

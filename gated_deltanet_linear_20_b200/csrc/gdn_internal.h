@@ -95,6 +95,9 @@ struct KdaArgs {
   int o_bf16;         // o written as bf16
   const int* cu_seqlens = nullptr;  // packed sequences: [B + 1] token offsets (views with B = 1)
   float* o = nullptr;               // o (fp32), for the packed last tile's row copy
+  float* snaps = nullptr;           // packed sequences: state snapshots, or null
+  int snap_every = 0;               // tokens between snapshots (a multiple of 32)
+  int n_snaps = 0;                  // slots in snaps
 };
 
 // Sets the dynamic shared-memory limit of `func` to `bytes` once per device

@@ -610,9 +610,12 @@ __device__ void side_role(const Ctx& x, const CUtensorMap* tq, const CUtensorMap
 // DVB: rows of the state this CTA owns (64 or 128); DV2: two CTAs per chain
 // (Dv = 256), this one owning rows dv0 = 128 (blockIdx & 1) ..; OBF: o is
 // bf16 (the fp32 value rounded to nearest even, through a bf16 TMA view)
+// snap (PK only; null: none): this CTA's first snapshot row, slot j (j = 1, 2, ..)
+// taking the state after j * stiles tiles
 template <int DVB, bool DV2, bool OBF, bool PK>
 __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMap* tmo,
-                           const KdaArgs& p, int chain, int b, int h, int ntiles, int tb, int tend) {
+                           const KdaArgs& p, int chain, int b, int h, int ntiles, int tb, int tend,
+                           float* snap, int stiles) {
   constexpr int DVW = DV2 ? 2 * D : DVB;  // Dv: rows of the chain's state
   const int dv0 = DV2 ? D * (int(blockIdx.x) & 1) : 0;
   const int warp = threadIdx.x >> 5;
@@ -810,6 +813,13 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
     //      output product's); refresh hi/lo and pre-scale by the next tile's
     //      decay per column, or store S_T
     if (!rs.wait(x, x.bar(B_SU), c & 1)) return;
+    // the state after this tile goes to a snapshot slot every stiles tiles (a
+    // last tile that the sequence ends inside is no boundary)
+    float* snap_row = nullptr;
+    if constexpr (PK) {
+      if (snap && own && (c + 1) % stiles == 0 && (c + 1) * NT <= tend - tb)
+        snap_row = snap + (size_t((c + 1) / stiles - 1) * p.H * DVW + dv) * D;
+    }
     if (!last) {
       if (!rs.wait(x, x.bar(gfull_off(c + 1)), gfull_parity(c + 1))) return;
       const float* LC = x.gates(c + 1) + G_LC / 4;
@@ -818,6 +828,13 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
         const int col = 64 * ch + 32 * q;
         float v[32];
         tmem_ld32(tlane + TM_S + col, v);
+        if constexpr (PK) {
+          if (snap_row) {
+            float4* sd = reinterpret_cast<float4*>(snap_row + col);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sd[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          }
+        }
         uint32_t hi[16], lo[16], u[32];
 #pragma unroll
         for (int e = 0; e < 16; ++e) split2_bf16(v[2 * e], v[2 * e + 1], hi[e], lo[e]);
@@ -842,6 +859,13 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
         if (!own) continue;
 #pragma unroll
         for (int e = 0; e < 8; ++e) dst[8 * q + e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        if constexpr (PK) {
+          if (snap_row) {  // the sequence ends on a snapshot boundary: that slot is S_T
+            float4* sd = reinterpret_cast<float4*>(snap_row + 64 * ch + 32 * q);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sd[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+          }
+        }
       }
     }
   }
@@ -862,6 +886,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int h = chain - (chain / p.H) * p.H;
   int ntiles = (p.T + NT - 1) / NT;
   int tb = 0, tend = p.T;  // this chain's tokens in the views
+  float* snap = nullptr;   // this CTA's first snapshot row (packed sequences)
+  int stiles = 1;
   if constexpr (PK) {
     // packed sequences: chain n H + h walks tokens [cu[n], cu[n+1]) of views with B = 1
     tb = __ldg(p.cu_seqlens + b);
@@ -872,6 +898,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     b = 0;
     ntiles = (tend - tb + NT - 1) / NT;
+    if (p.snaps) {
+      // first snapshot slot of this sequence: one per snap_every tokens of every
+      // earlier sequence; an invalid earlier entry (its own CTAs report it)
+      // leaves this sequence without snapshots
+      int base = 0;
+      bool offsets_ok = true;
+      for (int m = 0; m < chain / p.H; ++m) {
+        const int s0 = __ldg(p.cu_seqlens + m), s1 = __ldg(p.cu_seqlens + m + 1);
+        if (s0 < 0 || s1 < s0 || s1 > p.T) {
+          offsets_ok = false;
+          break;
+        }
+        base += (s1 - s0) / p.snap_every;
+      }
+      if (!offsets_ok || base + (tend - tb) / p.snap_every > p.n_snaps) {
+        if (tid == 0 && p.status) atomicExch(p.status, GDN_ERR_SHAPE);
+      } else {
+        snap = p.snaps + (size_t(base) * p.H + h) * (DV2 ? 2 * D : DVB) * D +
+               size_t(DV2 ? D * (int(blockIdx.x) & 1) : 0) * D;
+        stiles = p.snap_every / NT;
+      }
+    }
     if (ntiles == 0) {  // an empty sequence: S_T = S0 (or zeros), this CTA's rows
       const int rows = DVB;
       const size_t off = size_t(chain) * (DV2 ? 2 * D : DVB) * D +
@@ -913,7 +961,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     issue_g(x, &tm_g, 0, h, b, tb);
   }
   if (warp < 4 || warp >= 12)
-    chain_role<DVB, DV2, OBF, PK>(x, &tm_v, &tm_o, p, chain, b, h, ntiles, tb, tend);
+    chain_role<DVB, DV2, OBF, PK>(x, &tm_v, &tm_o, p, chain, b, h, ntiles, tb, tend, snap, stiles);
   else
     side_role<PRE, PK>(x, &tm_q, &tm_k, &tm_g, p, b, h, ntiles, tb, tend);
 

@@ -68,7 +68,7 @@ _lib.gdn_kda_prefill_ex.argtypes = [_vp] * 8 + [_ci] * 5 + [_vp, _vp, _vp]
 _lib.gdn_kda_prefill_ex.restype = _ci
 _lib.gdn_kda_decode_ex.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp, _vp]
 _lib.gdn_kda_decode_ex.restype = _ci
-_lib.gdn_kda_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 5 + [_vp, _vp]
+_lib.gdn_kda_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 5 + [_vp, _ci, _ci, _vp, _vp]
 _lib.gdn_kda_prefill_varlen.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
@@ -453,11 +453,14 @@ def kda_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: tor
                        beta: torch.Tensor, cu_seqlens: torch.Tensor,
                        S0: Optional[torch.Tensor] = None, *, o: Optional[torch.Tensor] = None,
                        S_T: Optional[torch.Tensor] = None,
-                       status: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+                       status: Optional[torch.Tensor] = None, snap_every: int = 0,
+                       snaps: Optional[torch.Tensor] = None):
     """Per-channel-gate prefill of N packed sequences (gdn_kda_prefill_varlen):
     q, k [total_T,H,128] bf16; v [total_T,H,Dv] bf16 (Dv 64, 128 or 256);
     g [total_T,H,128] fp32; beta [total_T,H] fp32; cu_seqlens int32 [N+1] on
-    the device.  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,128] fp32)."""
+    the device.  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,128] fp32), and
+    with ``snap_every`` (a multiple of 32) the state snapshots as in
+    ``prefill_varlen``."""
     if q.dim() != 3:
         raise ValueError("q must be [total_T,H,Dk]")
     total_T, H, Dk = q.shape
@@ -484,12 +487,23 @@ def kda_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: tor
     _check(S_T, "S_T", torch.float32, (N, H, Dv, Dk), dev)
     if status is not None:
         _check(status, "status", torch.int32, (1,), dev)
+    n_snaps = 0
+    if snap_every:
+        if snaps is None:
+            lens = (cu_seqlens[1:] - cu_seqlens[:-1]).cpu()
+            n_snaps = int((lens // int(snap_every)).sum())
+            snaps = torch.empty((n_snaps, H, Dv, Dk), dtype=torch.float32, device=dev)
+        n_snaps = snaps.shape[0]
+        _check(snaps, "snaps", torch.float32, (n_snaps, H, Dv, Dk), dev)
+    else:
+        snaps = None
     rc = _lib.gdn_kda_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
                                      _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk, Dv,
-                                     _ptr(status), _stream_handle(dev))
+                                     _ptr(snaps), int(snap_every), n_snaps, _ptr(status),
+                                     _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_kda_prefill_varlen")
-    return o, S_T
+    return (o, S_T) if snaps is None else (o, S_T, snaps)
 
 
 def kda_decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.Tensor,

@@ -345,13 +345,17 @@ int gdn_kda_decode_ex(const void* q, const void* k, const void* v, const float* 
  *                on the device: GDN_ERR_SHAPE goes to *status and that
  *                sequence's outputs are not written.  Empty sequences are
  *                allowed (S_T = S0, or zeros).
+ *   snaps, snap_every, n_snaps : optional state snapshots, laid out and
+ *                bounded as in gdn_prefill_varlen ([Dv][128] per slot), except
+ *                that snap_every is a positive multiple of 32 (the kernel's
+ *                chunk); NULL snaps: none.
  * Dk must be 128 and Dv 64, 128 or 256 (the chunked tensor-core kernel, one
  * CTA per chain, two with Dv = 256); no options.  Returns GDN_OK, a negative
  * code for invalid arguments (nothing is launched), as for gdn_kda_prefill. */
 int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, const float* S0, float* o, float* S_T,
                            const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
-                           int* status, void* stream);
+                           float* snaps, int snap_every, int n_snaps, int* status, void* stream);
 
 /* Synchronises `stream`, then reads the device status word written by the
  * kernels.  Returns GDN_OK, GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_NULL (status_dev is

@@ -463,10 +463,10 @@ def kda_varlen_args(**over):
     # N=3 sequences, total_T=200, H=2, Dk=128: q/k 100 KiB each, g 200 KiB, o 200 KiB (Dv 128)
     a = dict(q=P, k=P + 0x1000000, v=P + 0x2000000, g=P + 0x3000000, beta=P + 0x3100000,
              S0=None, o=P + 0x5000000, S_T=P + 0x6000000, cu=P + 0x7000000, N=3, total_T=200,
-             H=2, Dk=128, Dv=128, status=None, stream=None)
+             H=2, Dk=128, Dv=128, snaps=None, snap_every=0, n_snaps=0, status=None, stream=None)
     a.update(over)
     return [a[k] for k in ("q", "k", "v", "g", "beta", "S0", "o", "S_T", "cu", "N", "total_T",
-                           "H", "Dk", "Dv", "status", "stream")]
+                           "H", "Dk", "Dv", "snaps", "snap_every", "n_snaps", "status", "stream")]
 
 
 @pytest.mark.parametrize("over,code", [
@@ -480,6 +480,12 @@ def kda_varlen_args(**over):
     (dict(o=P + 0x7000000 - 64), -5),              # o runs into cu_seqlens
     (dict(S_T=P + 0x7000000 - 64 * 1024), -5),     # S_T runs into cu_seqlens
     (dict(S_T=P + 0x2000000 + 0x40), -5),          # S_T over v
+    (dict(n_snaps=-1), -3),
+    (dict(snaps=P + 0x8000000, snap_every=48, n_snaps=2), -4),    # not a multiple of 32
+    (dict(snaps=P + 0x8000000, snap_every=0, n_snaps=2), -4),
+    (dict(snaps=P + 0x8000008, snap_every=32, n_snaps=2), -2),
+    (dict(snaps=P + 0x6000000, snap_every=32, n_snaps=2), -5),    # snapshots over S_T
+    (dict(snaps=P + 0x7000000 - 1024, snap_every=32, n_snaps=1), -5),  # into cu_seqlens
 ], ids=lambda x: str(x))
 def test_kda_prefill_varlen_rejects_bad_arguments(gdn, over, code):
     assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(**over)) == code
@@ -490,5 +496,7 @@ def test_kda_prefill_varlen_valid_calls_pass_validation(gdn, dv):
     """Dk = 128 with Dv 64, 128 or 256 passes validation (the call then fails
     only for want of a device); no sequences or no heads is a no-op."""
     assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(Dv=dv)) not in VALIDATION_CODES + (0,)
+    assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(
+        Dv=dv, snaps=P + 0x8000000, snap_every=32, n_snaps=6)) not in VALIDATION_CODES + (0,)
     assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(N=0, q=None, S_T=None)) == 0
     assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(H=0, cu=None)) == 0

@@ -422,3 +422,60 @@ def test_kda_varlen_all_sequences_empty_copy_the_state():
                                     e(0, H, 128, dt=torch.float32), e(0, H, dt=torch.float32), cu, S0)
     torch.cuda.synchronize()
     assert o.shape == (0, H, 128) and torch.equal(S_T, S0)
+
+
+@pytest.mark.parametrize("dv,snap_every", [(128, 32), (128, 64), (256, 96), (64, 32)],
+                         ids=["128_every32", "128_every64", "256_every96", "64_every32"])
+def test_kda_varlen_state_snapshots(dv, snap_every):
+    """Snapshots after every snap_every tokens of each sequence equal the oracle's
+    state on that prefix (a sequence ending on a boundary: its last snapshot is
+    S_T); the outputs are unchanged by taking them."""
+    lengths = [200, 64, 0, 129, 96, 31]
+    H = 2
+    seqs, pk = _kda_packed(lengths, H, dv, seed=760 + dv + snap_every, s0_std=0.05)
+    gdn = _gdn()
+    dd = to_dev(pk)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T, snaps = gdn.kda_prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"],
+                                           dd["S0"], status=status, snap_every=snap_every)
+    assert gdn.query_status(status) == 0
+    assert snaps.shape[0] == sum(L // snap_every for L in lengths)
+    snaps = snaps.cpu().numpy()
+    slot = 0
+    for n, d in enumerate(seqs):
+        for j in range(1, lengths[n] // snap_every + 1):
+            t = j * snap_every
+            cut = lambda x: x[:, :t]
+            _, rS = oracle.kda_prefill(cut(d["q"]), cut(d["k"]), cut(d["v"]), cut(d["g"]),
+                                       cut(d["beta"]), d["S0"])
+            assert_parity(snaps[slot], rS[0], f"snapshot {j} of seq {n} (t={t})")
+            slot += 1
+    o2, S2 = gdn.kda_prefill_varlen(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"], dd["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(o.cpu(), o2.cpu()) and torch.equal(S_T.cpu(), S2.cpu())
+
+
+@pytest.mark.parametrize("dv", [128, 256])
+def test_kda_varlen_snapshot_bounds(dv):
+    """Snapshot slots stay inside the buffer: malformed offsets (a sequence
+    ending before it starts) leave the slots in front of the buffer untouched,
+    and a buffer one slot short leaves the slot after it untouched; both report
+    GDN_ERR_SHAPE."""
+    H, T = 2, 200
+    d = inputs.kda_inputs(1, T, H, Dv=dv, seed=780 + dv)
+    gdn = _gdn()
+    flat = lambda x: x[0].contiguous().to(DEV)
+    args = [flat(d[key]) for key in ("q", "k", "v", "g", "beta")]
+    guard = 2
+    buf = torch.full((guard + 3 + guard, H, dv, 128), 7.0, dtype=torch.float32, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    bad = torch.tensor([100, 0, 200], dtype=torch.int32, device=DEV)
+    gdn.kda_prefill_varlen(*args, bad, status=status, snap_every=64, snaps=buf[guard:guard + 3])
+    assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
+    assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + 3:] == 7.0)
+    # 200 tokens need 3 slots of 64; give 2
+    status.zero_()
+    ok = torch.tensor([0, 200], dtype=torch.int32, device=DEV)
+    gdn.kda_prefill_varlen(*args, ok, status=status, snap_every=64, snaps=buf[guard:guard + 2])
+    assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
+    assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + 2:] == 7.0)
