@@ -94,6 +94,15 @@ int main(void) {
   check(gdn_kda_prefill(q, k, v, g, beta, NULL, o, S, 1, 64, 2, 100, 128, NULL, NULL) ==
             GDN_ERR_UNSUPPORTED,
         "kda_prefill: Dk = 100 is GDN_ERR_UNSUPPORTED");
+  check(gdn_kda_prefill_varlen(q, k, v, g, beta, NULL, o, S, (const int*)beta, 1, 64, 2, 64, 64,
+                               NULL, 0, 0, NULL, NULL) == GDN_ERR_UNSUPPORTED,
+        "kda_prefill_varlen: Dk = 64 is GDN_ERR_UNSUPPORTED");
+  check(gdn_kda_prefill_varlen(q, k, v, g, beta, NULL, o, S, NULL, 1, 64, 2, 128, 128, NULL, 0, 0,
+                               NULL, NULL) == GDN_ERR_NULL,
+        "kda_prefill_varlen: NULL cu_seqlens is GDN_ERR_NULL");
+  check(gdn_kda_prefill_varlen(q, k, v, g, beta, NULL, o, S, (const int*)beta, 1, 64, 2, 128, 128,
+                               S, 48, 1, NULL, NULL) == GDN_ERR_UNSUPPORTED,
+        "kda_prefill_varlen: snapshots every 48 tokens are GDN_ERR_UNSUPPORTED");
 
   check(gdn_query_status(NULL, NULL) == GDN_ERR_NULL, "query_status: NULL word is GDN_ERR_NULL");
 
