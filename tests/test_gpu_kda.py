@@ -479,3 +479,28 @@ def test_kda_varlen_snapshot_bounds(dv):
     gdn.kda_prefill_varlen(*args, ok, status=status, snap_every=64, snaps=buf[guard:guard + 2])
     assert gdn.query_status(status) == gdn.GDN_ERR_SHAPE
     assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + 2:] == 7.0)
+
+
+def test_kda_varlen_benchmark_workload_sampled_chains():
+    """The packed benchmark workload (32 sequences of seeded uniform 64..2048
+    tokens, 16 heads), drawn on the device as the benchmark draws it; four
+    (sequence, head) chains, the longest sequence among them, checked against
+    the oracle on their own slices."""
+    rng = np.random.default_rng(4000)
+    lens = rng.integers(64, 2049, size=32)
+    seqs = [inputs.kda_inputs(1, int(L), 16, seed=5200 + i, device=DEV) for i, L in enumerate(lens)]
+    pk = {key: torch.cat([d[key][0] for d in seqs], 0) for key in ("q", "k", "v", "g", "beta")}
+    del seqs
+    cu_h = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    cu = torch.from_numpy(cu_h).to(DEV)
+    gdn = _gdn()
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.kda_prefill_varlen(pk["q"], pk["k"], pk["v"], pk["g"], pk["beta"], cu, status=status)
+    assert gdn.query_status(status) == 0
+    longest = int(np.argmax(lens))
+    for n, h in ((0, 0), (longest, 7), (17, 15), (31, 3)):
+        t0, t1 = int(cu_h[n]), int(cu_h[n + 1])
+        sl = lambda x: x[t0:t1, h:h + 1].unsqueeze(0).cpu()
+        ro, rS = oracle.kda_prefill(sl(pk["q"]), sl(pk["k"]), sl(pk["v"]), sl(pk["g"]), sl(pk["beta"]))
+        assert_parity(o[t0:t1, h:h + 1].unsqueeze(0).cpu().numpy(), ro, f"o seq {n} head {h}")
+        assert_parity(S_T[n:n + 1, h:h + 1].cpu().numpy(), rS, f"S_T seq {n} head {h}")
