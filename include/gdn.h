@@ -350,16 +350,19 @@ int gdn_kda_decode_ex(const void* q, const void* k, const void* v, const float* 
  *                that snap_every is a positive multiple of 32 (the kernel's
  *                chunk); NULL snaps: none.
  * Dk must be 128 and Dv 64, 128 or 256 (the chunked tensor-core kernel, one
- * CTA per chain, two with Dv = 256); no options.  Returns GDN_OK, a negative
- * code for invalid arguments (nothing is launched), as for gdn_kda_prefill. */
+ * CTA per chain, two with Dv = 256); no options.  N*H == 0 is a no-op.
+ * status: optional device int; GDN_ERR_SHAPE (offsets, snapshot slots) or
+ * GDN_ERR_DEVICE_TIMEOUT (a bounded wait gave up) is stored there.  Returns
+ * GDN_OK, or a negative code for invalid arguments (nothing is launched). */
 int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const float* g,
                            const float* beta, const float* S0, float* o, float* S_T,
                            const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
                            float* snaps, int snap_every, int n_snaps, int* status, void* stream);
 
 /* Synchronises `stream`, then reads the device status word written by the
- * kernels.  Returns GDN_OK, GDN_ERR_DEVICE_TIMEOUT, GDN_ERR_NULL (status_dev is
- * NULL) or GDN_ERR_LAUNCH (the synchronisation or copy failed). */
+ * kernels.  Returns the word (GDN_OK, GDN_ERR_DEVICE_TIMEOUT, or GDN_ERR_SHAPE
+ * from the packed-sequence calls), GDN_ERR_NULL (status_dev is NULL) or
+ * GDN_ERR_LAUNCH (the synchronisation or copy failed). */
 int gdn_query_status(const int* status_dev, void* stream);
 
 #ifdef __cplusplus
