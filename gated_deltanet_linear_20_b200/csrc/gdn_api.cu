@@ -436,6 +436,18 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
                        const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
                        int chunk, float* snaps, int snap_every, int n_snaps, int* status,
                        void* stream) {
+  return gdn_prefill_varlen_ex(q, k, v, g, beta, S0, o, S_T, cu_seqlens, N, total_T, H, Dk, Dv,
+                               chunk, snaps, snap_every, n_snaps, nullptr, status, stream);
+}
+
+int gdn_prefill_varlen_ex(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* S0, float* o, float* S_T,
+                          const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
+                          int chunk, float* snaps, int snap_every, int n_snaps,
+                          const gdn_options* opts, int* status, void* stream) {
+  int qk_norm = 0, o_bf16 = 0;
+  float q_scale = 1.f;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
   if (N < 0 || total_T < 0 || H < 0 || n_snaps < 0) return GDN_ERR_SHAPE;
   // the chunked tensor-core kernel's head dims: Dk 64 or 128, Dv 64, 128 or 256
   if ((Dk != 64 && Dk != kHeadDim) || !gdn::rows_head_dims_ok(Dk, Dv) ||
@@ -485,7 +497,7 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
   const int dv_box = Dv < kHeadDim ? Dv : kHeadDim;
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
                      H,      status, 1,      (total_T + 63) / 64, 1, nullptr, nullptr, nullptr,
-                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, 0, 1.f, 0,
+                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, qk_norm, q_scale, 0,
                      Dk,     Dv,   Dv / dv_box, dv_box};
   CUtensorMap tq{}, tk{}, tv{}, to{};
   // a valid (never read) view when every sequence is empty: S_T holds at least
@@ -632,6 +644,18 @@ int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const fl
                            const float* beta, const float* S0, float* o, float* S_T,
                            const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
                            float* snaps, int snap_every, int n_snaps, int* status, void* stream) {
+  return gdn_kda_prefill_varlen_ex(q, k, v, g, beta, S0, o, S_T, cu_seqlens, N, total_T, H, Dk, Dv,
+                                   snaps, snap_every, n_snaps, nullptr, status, stream);
+}
+
+int gdn_kda_prefill_varlen_ex(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, const float* S0, float* o, float* S_T,
+                              const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
+                              float* snaps, int snap_every, int n_snaps, const gdn_options* opts,
+                              int* status, void* stream) {
+  int qk_norm = 0, o_bf16 = 0;
+  float q_scale = 1.f;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
   if (N < 0 || total_T < 0 || H < 0 || n_snaps < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || (Dv != 64 && Dv != kHeadDim && Dv != 2 * kHeadDim)) return GDN_ERR_UNSUPPORTED;
   if (snaps && (snap_every <= 0 || snap_every % 32 != 0)) return GDN_ERR_UNSUPPORTED;
@@ -688,7 +712,7 @@ int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const fl
       !encode_act(&tv, pick(v), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv, 32) ||
       !encode_act(&to, pick(o), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, Dv, 32))
     return GDN_ERR_LAUNCH;
-  gdn::KdaArgs a{g,  beta, S0, S_T,        N, total_T, H,     status, 0, 1.f, Dv, 0, cu_seqlens,
+  gdn::KdaArgs a{g,  beta, S0, S_T,        N, total_T, H,     status, qk_norm, q_scale, Dv, 0, cu_seqlens,
                  o,  snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0};
   return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK

@@ -1004,13 +1004,16 @@ int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     return true;
   };
   bool ok;
-  if (a.cu_seqlens) {  // packed sequences (fp32 o, no pre-steps)
+  if (a.cu_seqlens) {  // packed sequences (fp32 o; the pre-steps on request)
     if (a.Dv == D)
-      ok = go(kda_prefill_kernel<false, 128, false, false, true>, 64, chains);
+      ok = pre ? go(kda_prefill_kernel<true, 128, false, false, true>, 75, chains)
+               : go(kda_prefill_kernel<false, 128, false, false, true>, 64, chains);
     else if (a.Dv == 2 * D)
-      ok = go(kda_prefill_kernel<false, 128, true, false, true>, 65, 2 * chains);
+      ok = pre ? go(kda_prefill_kernel<true, 128, true, false, true>, 76, 2 * chains)
+               : go(kda_prefill_kernel<false, 128, true, false, true>, 65, 2 * chains);
     else if (a.Dv == 64)
-      ok = go(kda_prefill_kernel<false, 64, false, false, true>, 66, chains);
+      ok = pre ? go(kda_prefill_kernel<true, 64, false, false, true>, 77, chains)
+               : go(kda_prefill_kernel<false, 64, false, false, true>, 66, chains);
     else
       return -1;
   } else if (a.o_bf16) {

@@ -1325,19 +1325,32 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   const bool obf = a.o_bf16 != 0;
   bool ok;
   if (a.cu_seqlens) {
-    // packed sequences (fp32 o, no pre-steps): their own instantiations, so that the
-    // dense kernels carry none of the per-sequence paths
+    // packed sequences (fp32 o; the pre-steps on request): their own
+    // instantiations, so that the dense kernels carry none of the per-sequence paths
     const bool c64 = chunk == 64;
-    if (a.Dk == D)
-      ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 128, 128, true>, 55)
-                                : go(prefill_kernel<16, false, false, 128, 128, true>, 56))
-                         : (c64 ? go(prefill_kernel<64, false, false, 128, 64, true>, 57)
-                                : go(prefill_kernel<16, false, false, 128, 64, true>, 58));
-    else
-      ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 64, 128, true>, 59)
-                                : go(prefill_kernel<16, false, false, 64, 128, true>, 60))
-                         : (c64 ? go(prefill_kernel<64, false, false, 64, 64, true>, 61)
-                                : go(prefill_kernel<16, false, false, 64, 64, true>, 62));
+    if (!pre) {
+      if (a.Dk == D)
+        ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 128, 128, true>, 55)
+                                  : go(prefill_kernel<16, false, false, 128, 128, true>, 56))
+                           : (c64 ? go(prefill_kernel<64, false, false, 128, 64, true>, 57)
+                                  : go(prefill_kernel<16, false, false, 128, 64, true>, 58));
+      else
+        ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 64, 128, true>, 59)
+                                  : go(prefill_kernel<16, false, false, 64, 128, true>, 60))
+                           : (c64 ? go(prefill_kernel<64, false, false, 64, 64, true>, 61)
+                                  : go(prefill_kernel<16, false, false, 64, 64, true>, 62));
+    } else {
+      if (a.Dk == D)
+        ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, true, false, 128, 128, true>, 67)
+                                  : go(prefill_kernel<16, true, false, 128, 128, true>, 68))
+                           : (c64 ? go(prefill_kernel<64, true, false, 128, 64, true>, 69)
+                                  : go(prefill_kernel<16, true, false, 128, 64, true>, 70));
+      else
+        ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, true, false, 64, 128, true>, 71)
+                                  : go(prefill_kernel<16, true, false, 64, 128, true>, 72))
+                           : (c64 ? go(prefill_kernel<64, true, false, 64, 64, true>, 73)
+                                  : go(prefill_kernel<16, true, false, 64, 64, true>, 74));
+    }
   } else if (a.Dk == D && a.dv_box == D && a.Dv != D) {
     // Dv = 256: the 128 x 128 kernels on two CTAs per chain (rows dv0 .. dv0 + 127)
     if (chunk == 64)

@@ -70,6 +70,10 @@ _lib.gdn_kda_decode_ex.argtypes = [_vp] * 7 + [_ci] * 5 + [_vp, _vp, _vp]
 _lib.gdn_kda_decode_ex.restype = _ci
 _lib.gdn_kda_prefill_varlen.argtypes = [_vp] * 9 + [_ci] * 5 + [_vp, _ci, _ci, _vp, _vp]
 _lib.gdn_kda_prefill_varlen.restype = _ci
+_lib.gdn_prefill_varlen_ex.argtypes = [_vp] * 9 + [_ci] * 6 + [_vp, _ci, _ci, _vp, _vp, _vp]
+_lib.gdn_prefill_varlen_ex.restype = _ci
+_lib.gdn_kda_prefill_varlen_ex.argtypes = [_vp] * 9 + [_ci] * 5 + [_vp, _ci, _ci, _vp, _vp, _vp]
+_lib.gdn_kda_prefill_varlen_ex.restype = _ci
 _lib.gdn_query_status.argtypes = [_vp, _vp]
 _lib.gdn_query_status.restype = _ci
 
@@ -229,7 +233,8 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
                    chunk: int = 64, *, o: Optional[torch.Tensor] = None,
                    S_T: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
                    snap_every: int = 0,
-                   snaps: Optional[torch.Tensor] = None):
+                   snaps: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
+                   q_scale: float = 1.0):
     """Prefill of N packed sequences: q, k [total_T,H,Dk] bf16; v [total_T,H,Dv] bf16;
     g, beta [total_T,H] fp32; cu_seqlens int32 [N+1] on the device (offsets of
     the sequences).  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,Dk] fp32).
@@ -237,7 +242,8 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     [n_snaps,H,Dv,Dk] (after every snap_every tokens of each sequence, sequence
     by sequence); ``snaps`` may be given preallocated, else its size is read
     from cu_seqlens (one device-to-host copy).  Dk 64 or 128, Dv 64, 128 or
-    256 (the chunked tensor-core kernel)."""
+    256 (the chunked tensor-core kernel).  ``qk_l2norm`` / ``q_scale`` apply the
+    fused pre-steps of ``prefill`` (gdn_prefill_varlen_ex)."""
     if q.dim() != 3:
         raise ValueError("q must be [total_T,H,Dk]")
     total_T, H, Dk = q.shape
@@ -274,10 +280,17 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
         _check(snaps, "snaps", torch.float32, (n_snaps, H, Dv, Dk), dev)
     else:
         snaps = None
-    rc = _lib.gdn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                                 _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk, Dv, int(chunk),
-                                 _ptr(snaps), int(snap_every), n_snaps, _ptr(status),
-                                 _stream_handle(dev))
+    opts = _options(qk_l2norm, q_scale)
+    if opts is None:
+        rc = _lib.gdn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                     _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk, Dv,
+                                     int(chunk), _ptr(snaps), int(snap_every), n_snaps,
+                                     _ptr(status), _stream_handle(dev))
+    else:
+        rc = _lib.gdn_prefill_varlen_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                        _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk,
+                                        Dv, int(chunk), _ptr(snaps), int(snap_every), n_snaps,
+                                        opts, _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_prefill_varlen")
     return (o, S_T) if snaps is None else (o, S_T, snaps)
@@ -454,13 +467,14 @@ def kda_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: tor
                        S0: Optional[torch.Tensor] = None, *, o: Optional[torch.Tensor] = None,
                        S_T: Optional[torch.Tensor] = None,
                        status: Optional[torch.Tensor] = None, snap_every: int = 0,
-                       snaps: Optional[torch.Tensor] = None):
+                       snaps: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
+                       q_scale: float = 1.0):
     """Per-channel-gate prefill of N packed sequences (gdn_kda_prefill_varlen):
     q, k [total_T,H,128] bf16; v [total_T,H,Dv] bf16 (Dv 64, 128 or 256);
     g [total_T,H,128] fp32; beta [total_T,H] fp32; cu_seqlens int32 [N+1] on
     the device.  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,128] fp32), and
     with ``snap_every`` (a multiple of 32) the state snapshots as in
-    ``prefill_varlen``."""
+    ``prefill_varlen``.  ``qk_l2norm`` / ``q_scale`` as in ``kda_prefill``."""
     if q.dim() != 3:
         raise ValueError("q must be [total_T,H,Dk]")
     total_T, H, Dk = q.shape
@@ -497,10 +511,17 @@ def kda_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: tor
         _check(snaps, "snaps", torch.float32, (n_snaps, H, Dv, Dk), dev)
     else:
         snaps = None
-    rc = _lib.gdn_kda_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
-                                     _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk, Dv,
-                                     _ptr(snaps), int(snap_every), n_snaps, _ptr(status),
-                                     _stream_handle(dev))
+    opts = _options(qk_l2norm, q_scale)
+    if opts is None:
+        rc = _lib.gdn_kda_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
+                                         _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk,
+                                         Dv, _ptr(snaps), int(snap_every), n_snaps, _ptr(status),
+                                         _stream_handle(dev))
+    else:
+        rc = _lib.gdn_kda_prefill_varlen_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                            _ptr(S0), _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N,
+                                            total_T, H, Dk, Dv, _ptr(snaps), int(snap_every),
+                                            n_snaps, opts, _ptr(status), _stream_handle(dev))
     if rc != GDN_OK:
         raise GDNError(rc, "gdn_kda_prefill_varlen")
     return (o, S_T) if snaps is None else (o, S_T, snaps)
@@ -602,3 +623,11 @@ def raw_kda_decode_ex(*args) -> int:
 
 def raw_kda_prefill_varlen(*args) -> int:
     return int(_lib.gdn_kda_prefill_varlen(*args))
+
+
+def raw_prefill_varlen_ex(*args) -> int:
+    return int(_lib.gdn_prefill_varlen_ex(*args))
+
+
+def raw_kda_prefill_varlen_ex(*args) -> int:
+    return int(_lib.gdn_kda_prefill_varlen_ex(*args))

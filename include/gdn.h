@@ -179,6 +179,16 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
                        int chunk, float* snaps, int snap_every, int n_snaps, int* status,
                        void* stream);
 
+/* gdn_prefill_varlen with options (gdn_options; NULL = none): qk_l2norm
+ * and q_scale as in gdn_prefill_ex, applied to every token of every packed
+ * sequence.  o_bf16 is not offered on packed sequences (GDN_ERR_UNSUPPORTED,
+ * as for an invalid struct).  Everything else as for gdn_prefill_varlen. */
+int gdn_prefill_varlen_ex(const void* q, const void* k, const void* v, const float* g,
+                          const float* beta, const float* S0, float* o, float* S_T,
+                          const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
+                          int chunk, float* snaps, int snap_every, int n_snaps,
+                          const gdn_options* opts, int* status, void* stream);
+
 /* gdn_prefill_ws with options (gdn_options above; NULL = none); with a NULL
  * workspace it runs the single pass of gdn_prefill.  Invalid options (size
  * too small, q_scale NaN) return GDN_ERR_UNSUPPORTED, and so do non-default
@@ -358,6 +368,15 @@ int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const fl
                            const float* beta, const float* S0, float* o, float* S_T,
                            const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
                            float* snaps, int snap_every, int n_snaps, int* status, void* stream);
+
+/* gdn_kda_prefill_varlen with options: qk_l2norm and q_scale as in
+ * gdn_kda_prefill_ex; o_bf16 is GDN_ERR_UNSUPPORTED here.  Everything else as
+ * for gdn_kda_prefill_varlen. */
+int gdn_kda_prefill_varlen_ex(const void* q, const void* k, const void* v, const float* g,
+                              const float* beta, const float* S0, float* o, float* S_T,
+                              const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
+                              float* snaps, int snap_every, int n_snaps,
+                              const gdn_options* opts, int* status, void* stream);
 
 /* Synchronises `stream`, then reads the device status word written by the
  * kernels.  Returns the word (GDN_OK, GDN_ERR_DEVICE_TIMEOUT, or GDN_ERR_SHAPE

@@ -500,3 +500,32 @@ def test_kda_prefill_varlen_valid_calls_pass_validation(gdn, dv):
         Dv=dv, snaps=P + 0x8000000, snap_every=32, n_snaps=6)) not in VALIDATION_CODES + (0,)
     assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(N=0, q=None, S_T=None)) == 0
     assert gdn.raw_kda_prefill_varlen(*kda_varlen_args(H=0, cu=None)) == 0
+
+
+def test_packed_calls_take_the_pre_step_options(gdn):
+    """gdn_prefill_varlen_ex and gdn_kda_prefill_varlen_ex accept qk_l2norm and
+    q_scale (the call then fails only for want of a device), reject o_bf16, a
+    short struct and a NaN scale (GDN_ERR_UNSUPPORTED), and validate every other
+    argument as the calls without options do."""
+    import ctypes as ct
+    good = ct.byref(gdn.Options(ct.sizeof(gdn.Options), 1, 0.5, 0))
+    bad = [ct.byref(gdn.Options(ct.sizeof(gdn.Options), 1, 1.0, 1)),
+           ct.byref(gdn.Options(4, 1, 1.0)),
+           ct.byref(gdn.Options(ct.sizeof(gdn.Options), 0, float("nan")))]
+    with_opts = lambda a, o: a[:18] + [o] + a[18:]
+    for dk, dv in ((128, 128), (64, 64), (128, 256)):
+        a = varlen_args(Dk=dk, Dv=dv)
+        assert gdn.raw_prefill_varlen_ex(*with_opts(a, good)) not in VALIDATION_CODES + (0,)
+        assert gdn.raw_prefill_varlen_ex(*with_opts(a, None)) not in VALIDATION_CODES + (0,)
+        for o in bad:
+            assert gdn.raw_prefill_varlen_ex(*with_opts(a, o)) == -4
+    assert gdn.raw_prefill_varlen_ex(*with_opts(varlen_args(N=-1), good)) == -3
+    assert gdn.raw_prefill_varlen_ex(*with_opts(varlen_args(S_T=P + 0x10000000), good)) == -5
+    kwith = lambda a, o: a[:17] + [o] + a[17:]
+    for dv in (64, 128, 256):
+        a = kda_varlen_args(Dv=dv)
+        assert gdn.raw_kda_prefill_varlen_ex(*kwith(a, good)) not in VALIDATION_CODES + (0,)
+        for o in bad:
+            assert gdn.raw_kda_prefill_varlen_ex(*kwith(a, o)) == -4
+    assert gdn.raw_kda_prefill_varlen_ex(*kwith(kda_varlen_args(Dk=64, Dv=64), good)) == -4
+    assert gdn.raw_kda_prefill_varlen_ex(*kwith(kda_varlen_args(cu=None), good)) == -1

@@ -504,3 +504,74 @@ def test_kda_varlen_benchmark_workload_sampled_chains():
         ro, rS = oracle.kda_prefill(sl(pk["q"]), sl(pk["k"]), sl(pk["v"]), sl(pk["g"]), sl(pk["beta"]))
         assert_parity(o[t0:t1, h:h + 1].unsqueeze(0).cpu().numpy(), ro, f"o seq {n} head {h}")
         assert_parity(S_T[n:n + 1, h:h + 1].cpu().numpy(), rS, f"S_T seq {n} head {h}")
+
+
+@pytest.mark.parametrize("dv", [128, 64, 256])
+def test_kda_varlen_fused_qk_norm_and_q_scale(dv):
+    """Packed per-channel-gate sequences with q / k normalised and q scaled in
+    the kernel (gdn_kda_prefill_varlen_ex) equal the oracle run per sequence on
+    inputs normalised in fp64 beforehand; snapshots are taken on the way."""
+    lengths = [130, 0, 1, 64, 77]
+    H, qs = 2, 0.5
+    seqs, pk = _kda_packed(lengths, H, dv, seed=800 + dv, s0_std=0.05)
+    r = _raw_qk(pk, 801 + dv)
+    dd = to_dev(pk)
+    gdn = _gdn()
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T, snaps = gdn.kda_prefill_varlen(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"],
+                                           dd["cu"], dd["S0"], status=status, snap_every=64,
+                                           qk_l2norm=True, q_scale=qs)
+    assert gdn.query_status(status) == 0
+    o, S_T, snaps = o.cpu().numpy(), S_T.cpu().numpy(), snaps.cpu().numpy()
+    cu = pk["cu"].numpy()
+    slot = 0
+    for n, d in enumerate(seqs):
+        t0, t1 = int(cu[n]), int(cu[n + 1])
+        sl = lambda x, t=t1: x[t0:t].unsqueeze(0)
+        if lengths[n]:
+            ro, rS = oracle.kda_prefill((sl(r["q_n"]) * qs).float(), sl(r["k_n"]).float(), d["v"], d["g"],
+                                        d["beta"], d["S0"])
+            assert_parity(o[t0:t1], ro[0], f"o seq {n} (fused norm)")
+            assert_parity(S_T[n], rS[0], f"S_T seq {n} (fused norm)")
+        for j in range(1, lengths[n] // 64 + 1):
+            te = t0 + 64 * j
+            _, rS = oracle.kda_prefill((sl(r["q_n"], te) * qs).float(), sl(r["k_n"], te).float(),
+                                       d["v"][:, :64 * j], d["g"][:, :64 * j], d["beta"][:, :64 * j], d["S0"])
+            assert_parity(snaps[slot], rS[0], f"snapshot {j} of seq {n} (fused norm)")
+            slot += 1
+    assert slot == snaps.shape[0]
+
+
+@pytest.mark.parametrize("dk,dv,chunk", [(128, 128, 64), (128, 128, 16), (64, 64, 64), (128, 256, 64)],
+                         ids=["128x128_c64", "128x128_c16", "64x64", "128x256"])
+def test_scalar_varlen_fused_qk_norm_and_q_scale(dk, dv, chunk):
+    """Packed scalar-gate sequences with q / k normalised and q scaled in the
+    kernel (gdn_prefill_varlen_ex) equal the oracle run per sequence on inputs
+    normalised in fp64 beforehand."""
+    lengths = [130, 0, 1, 64, 77]
+    H, qs = 2, 0.5
+    seqs = [inputs.prefill_inputs(1, L, H, dk, dv, seed=820 + i, s0_std=0.05)
+            for i, L in enumerate(lengths)]
+    cat = lambda key: torch.cat([d[key][0] for d in seqs], 0)
+    pk = dict(q=cat("q"), k=cat("k"), v=cat("v"), g=cat("g"), beta=cat("beta"),
+              S0=torch.cat([d["S0"] for d in seqs], 0),
+              cu=torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32))
+    r = _raw_qk(pk, 830 + dk + dv)
+    dd = to_dev(pk)
+    gdn = _gdn()
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = gdn.prefill_varlen(r["q"].to(DEV), r["k"].to(DEV), dd["v"], dd["g"], dd["beta"], dd["cu"],
+                                dd["S0"], chunk=chunk, status=status, qk_l2norm=True, q_scale=qs)
+    assert gdn.query_status(status) == 0
+    o, S_T = o.cpu().numpy(), S_T.cpu().numpy()
+    cu = pk["cu"].numpy()
+    for n, d in enumerate(seqs):
+        t0, t1 = int(cu[n]), int(cu[n + 1])
+        if not lengths[n]:
+            np.testing.assert_array_equal(S_T[n], d["S0"][0].numpy())
+            continue
+        sl = lambda x: x[t0:t1].unsqueeze(0)
+        ro, rS = oracle.prefill((sl(r["q_n"]) * qs).float(), sl(r["k_n"]).float(), d["v"], d["g"],
+                                d["beta"], d["S0"])
+        assert_parity(o[t0:t1], ro[0], f"o seq {n} (fused norm)")
+        assert_parity(S_T[n], rS[0], f"S_T seq {n} (fused norm)")
