@@ -447,7 +447,7 @@ int gdn_prefill_varlen_ex(const void* q, const void* k, const void* v, const flo
                           const gdn_options* opts, int* status, void* stream) {
   int qk_norm = 0, o_bf16 = 0;
   float q_scale = 1.f;
-  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
   if (N < 0 || total_T < 0 || H < 0 || n_snaps < 0) return GDN_ERR_SHAPE;
   // the chunked tensor-core kernel's head dims: Dk 64 or 128, Dv 64, 128 or 256
   if ((Dk != 64 && Dk != kHeadDim) || !gdn::rows_head_dims_ok(Dk, Dv) ||
@@ -465,13 +465,14 @@ int gdn_prefill_varlen_ex(const void* q, const void* k, const void* v, const flo
   if (total_T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
                       !aligned(g, 4) || !aligned(beta, 4)))
     return GDN_ERR_ALIGN;
-  const size_t act_bf16 = size_t(act_k) * 2, v_bf16 = size_t(act_v) * 2, act_f32 = size_t(act_v) * 4;
+  const size_t act_bf16 = size_t(act_k) * 2, v_bf16 = size_t(act_v) * 2;
+  const size_t o_bytes = size_t(act_v) * (o_bf16 ? 2 : 4);
   const size_t gate_bytes = size_t(total_T) * H * 4;
   const size_t state_bytes = size_t(chains) * Dk * Dv * 4, cu_bytes = size_t(N + 1) * 4;
-  if (total_T > 0 && (overlaps(o, act_f32, q, act_bf16) || overlaps(o, act_f32, k, act_bf16) ||
-                      overlaps(o, act_f32, v, v_bf16) || overlaps(o, act_f32, g, gate_bytes) ||
-                      overlaps(o, act_f32, beta, gate_bytes) || overlaps(o, act_f32, S0, state_bytes) ||
-                      overlaps(o, act_f32, S_T, state_bytes) || overlaps(o, act_f32, cu_seqlens, cu_bytes)))
+  if (total_T > 0 && (overlaps(o, o_bytes, q, act_bf16) || overlaps(o, o_bytes, k, act_bf16) ||
+                      overlaps(o, o_bytes, v, v_bf16) || overlaps(o, o_bytes, g, gate_bytes) ||
+                      overlaps(o, o_bytes, beta, gate_bytes) || overlaps(o, o_bytes, S0, state_bytes) ||
+                      overlaps(o, o_bytes, S_T, state_bytes) || overlaps(o, o_bytes, cu_seqlens, cu_bytes)))
     return GDN_ERR_ALIAS;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
   if (overlaps(S_T, state_bytes, cu_seqlens, cu_bytes)) return GDN_ERR_ALIAS;
@@ -482,7 +483,7 @@ int gdn_prefill_varlen_ex(const void* q, const void* k, const void* v, const flo
   if (snaps) {
     const size_t snap_bytes = size_t(n_snaps) * H * Dk * Dv * 4;
     if (!aligned(snaps, 16)) return GDN_ERR_ALIGN;
-    if ((total_T > 0 && overlaps(snaps, snap_bytes, o, act_f32)) ||
+    if ((total_T > 0 && overlaps(snaps, snap_bytes, o, o_bytes)) ||
         overlaps(snaps, snap_bytes, S_T, state_bytes) || overlaps(snaps, snap_bytes, S0, state_bytes) ||
         overlaps(snaps, snap_bytes, cu_seqlens, cu_bytes) ||
         (total_T > 0 && (overlaps(snaps, snap_bytes, q, act_bf16) || overlaps(snaps, snap_bytes, k, act_bf16) ||
@@ -497,7 +498,7 @@ int gdn_prefill_varlen_ex(const void* q, const void* k, const void* v, const flo
   const int dv_box = Dv < kHeadDim ? Dv : kHeadDim;
   gdn::PrefillArgs a{g,      beta, S0,      o,       S_T,     N,      total_T,
                      H,      status, 1,      (total_T + 63) / 64, 1, nullptr, nullptr, nullptr,
-                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, qk_norm, q_scale, 0,
+                     cu_seqlens, snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0, qk_norm, q_scale, o_bf16,
                      Dk,     Dv,   Dv / dv_box, dv_box};
   CUtensorMap tq{}, tk{}, tv{}, to{};
   // a valid (never read) view when every sequence is empty: S_T holds at least
@@ -509,7 +510,7 @@ int gdn_prefill_varlen_ex(const void* q, const void* k, const void* v, const flo
       !encode_act(&tk, total_T > 0 ? k : S_T, 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, Dk) ||
       !encode_act(&tv, total_T > 0 ? v : S_T, 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv) ||
       !encode_act(&to, total_T > 0 ? static_cast<const void*>(o) : S_T, 1, Tv, H, dv_box,
-                  CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, Dv))
+                  CU_TENSOR_MAP_SWIZZLE_NONE, o_bf16 ? bf : f32, o_bf16 ? 2 : 4, Dv))
     return GDN_ERR_LAUNCH;
   const cudaStream_t st = static_cast<cudaStream_t>(stream);
   return gdn::launch_prefill(tq, tk, tv, to, to, a, chunk, st) == 0 ? GDN_OK : GDN_ERR_LAUNCH;
@@ -655,7 +656,7 @@ int gdn_kda_prefill_varlen_ex(const void* q, const void* k, const void* v, const
                               int* status, void* stream) {
   int qk_norm = 0, o_bf16 = 0;
   float q_scale = 1.f;
-  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16) || o_bf16) return GDN_ERR_UNSUPPORTED;
+  if (!read_options(opts, &qk_norm, &q_scale, &o_bf16)) return GDN_ERR_UNSUPPORTED;
   if (N < 0 || total_T < 0 || H < 0 || n_snaps < 0) return GDN_ERR_SHAPE;
   if (Dk != kHeadDim || (Dv != 64 && Dv != kHeadDim && Dv != 2 * kHeadDim)) return GDN_ERR_UNSUPPORTED;
   if (snaps && (snap_every <= 0 || snap_every % 32 != 0)) return GDN_ERR_UNSUPPORTED;
@@ -671,7 +672,7 @@ int gdn_kda_prefill_varlen_ex(const void* q, const void* k, const void* v, const
                       !aligned(o, 16) || !aligned(beta, 4)))
     return GDN_ERR_ALIGN;
   const size_t toks = size_t(total_T) * H;
-  const size_t act_bf16 = toks * kHeadDim * 2, v_bf16 = toks * Dv * 2, o_bytes = toks * Dv * 4;
+  const size_t act_bf16 = toks * kHeadDim * 2, v_bf16 = toks * Dv * 2, o_bytes = toks * Dv * (o_bf16 ? 2 : 4);
   const size_t g_bytes = toks * kHeadDim * 4, beta_bytes = toks * 4;
   const size_t state_bytes = size_t(chains) * kHeadDim * Dv * 4, cu_bytes = size_t(N + 1) * 4;
   if (S0 && S0 != S_T && overlaps(S0, state_bytes, S_T, state_bytes)) return GDN_ERR_ALIAS;
@@ -710,9 +711,10 @@ int gdn_kda_prefill_varlen_ex(const void* q, const void* k, const void* v, const
       !encode_act(&tq, pick(q), 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
       !encode_act(&tk, pick(k), 1, Tv, H, 64, CU_TENSOR_MAP_SWIZZLE_128B, bf, 2, kHeadDim, 32) ||
       !encode_act(&tv, pick(v), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, bf, 2, Dv, 32) ||
-      !encode_act(&to, pick(o), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, f32, 4, Dv, 32))
+      !encode_act(&to, pick(o), 1, Tv, H, dv_box, CU_TENSOR_MAP_SWIZZLE_NONE, o_bf16 ? bf : f32,
+                  o_bf16 ? 2 : 4, Dv, 32))
     return GDN_ERR_LAUNCH;
-  gdn::KdaArgs a{g,  beta, S0, S_T,        N, total_T, H,     status, qk_norm, q_scale, Dv, 0, cu_seqlens,
+  gdn::KdaArgs a{g,  beta, S0, S_T,        N, total_T, H,     status, qk_norm, q_scale, Dv, o_bf16, cu_seqlens,
                  o,  snaps, snaps ? snap_every : 0, snaps ? n_snaps : 0};
   return gdn::launch_kda_prefill(tq, tk, tv, to, tg, a, static_cast<cudaStream_t>(stream)) == 0
              ? GDN_OK

@@ -94,7 +94,7 @@ struct KdaArgs {
   int Dv;             // 64, 128 or 256 (Dk is 128)
   int o_bf16;         // o written as bf16
   const int* cu_seqlens = nullptr;  // packed sequences: [B + 1] token offsets (views with B = 1)
-  float* o = nullptr;               // o (fp32), for the packed last tile's row copy
+  float* o = nullptr;               // o (fp32, or bf16 with o_bf16): the packed last tile's row copy
   float* snaps = nullptr;           // packed sequences: state snapshots, or null
   int snap_every = 0;               // tokens between snapshots (a multiple of 32)
   int n_snaps = 0;                  // slots in snaps

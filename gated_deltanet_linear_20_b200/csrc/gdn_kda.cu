@@ -808,6 +808,17 @@ __device__ void chain_role(const Ctx& x, const CUtensorMap* tv, const CUtensorMa
         const int r = i / (DVB / 4), j = i % (DVB / 4);
         reinterpret_cast<float4*>(dst + size_t(r) * p.H * DVW)[j] = src[i];
       }
+    } else if constexpr (PK && OBF) {
+      // the same for bf16 o (rows of DVB bf16: DVB / 8 chunks of 16 bytes)
+      const int nvalid = tend - (tb + c * NT);
+      const uint4* src = reinterpret_cast<const uint4*>(x.sm + SM_XH);
+      __nv_bfloat16* dst =
+          reinterpret_cast<__nv_bfloat16*>(p.o) + (size_t(tb + c * NT) * p.H + h) * DVW + dv0;
+      const int ct = (warp >= 12 ? 128 : 0) + lq * 32 + (threadIdx.x & 31);
+      for (int i = ct; i < nvalid * (DVB / 8); i += CHAIN_THREADS) {
+        const int r = i / (DVB / 8), j = i % (DVB / 8);
+        reinterpret_cast<uint4*>(dst + size_t(r) * p.H * DVW)[j] = src[i];
+      }
     }
     // ---- state epilogue: the update has completed (its commit preceded the
     //      output product's); refresh hi/lo and pre-scale by the next tile's
@@ -1004,7 +1015,16 @@ int launch_kda_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
     return true;
   };
   bool ok;
-  if (a.cu_seqlens) {  // packed sequences (fp32 o; the pre-steps on request)
+  if (a.cu_seqlens && a.o_bf16) {  // packed sequences, bf16 o (pre-step instantiations)
+    if (a.Dv == D)
+      ok = go(kda_prefill_kernel<true, 128, false, true, true>, 86, chains);
+    else if (a.Dv == 2 * D)
+      ok = go(kda_prefill_kernel<true, 128, true, true, true>, 87, 2 * chains);
+    else if (a.Dv == 64)
+      ok = go(kda_prefill_kernel<true, 64, false, true, true>, 88, chains);
+    else
+      return -1;
+  } else if (a.cu_seqlens) {  // packed sequences (fp32 o; the pre-steps on request)
     if (a.Dv == D)
       ok = pre ? go(kda_prefill_kernel<true, 128, false, false, true>, 75, chains)
                : go(kda_prefill_kernel<false, 128, false, false, true>, 64, chains);

@@ -464,6 +464,16 @@ __device__ __noinline__ void store_partial_tile(const float4* src, float* dst, s
   }
 }
 
+// The same for a bf16 staging tile (rows of DVB bf16, DVB / 8 chunks of 16 bytes).
+template <int DVB>
+__device__ __noinline__ void store_partial_tile_bf16(const uint4* src, __nv_bfloat16* dst,
+                                                     size_t rowstride, int nvalid, int ct) {
+  for (int i = ct; i < nvalid * (DVB / 8); i += CHAIN_THREADS) {
+    const int r = i / (DVB / 8), j = i % (DVB / 8);
+    reinterpret_cast<uint4*>(dst + size_t(r) * rowstride)[j] = src[i];
+  }
+}
+
 // o[t][dv] = Gamma_t Y[dv][t] + O_intra[dv][t] of tile c.  This thread's 32
 // tokens (32 hf ..) of lane dv go into the fp32 [64 tokens][128] o staging
 // tile; the leader then stores the tile with TMA (tokens at or past T are
@@ -508,11 +518,16 @@ __device__ __forceinline__ void output_drain(const Ctx& x, uint32_t tlane, int b
       bulk_commit();
     }
   } else if constexpr (!OBF && PK) {
-    // last tile of a packed sequence (packed calls take fp32 o only): the rows
-    // past it belong to the next sequence, so only the valid rows are copied out
+    // last tile of a packed sequence: the rows past it belong to the next
+    // sequence, so only the valid rows are copied out
     store_partial_tile<DVB>(reinterpret_cast<const float4*>(x.sm + SM_XH),
                             x.odst + ((size_t(b) * x.tmap + ts) * x.H + h) * *x.misc(M_OROW) + x.dv0,
                             size_t(x.H) * *x.misc(M_OROW), x.tend - ts, hf * 128 + dv);
+  } else if constexpr (OBF && PK) {
+    store_partial_tile_bf16<DVB>(
+        reinterpret_cast<const uint4*>(x.sm + SM_XH),
+        reinterpret_cast<__nv_bfloat16*>(x.odst) + ((size_t(b) * x.tmap + ts) * x.H + h) * *x.misc(M_OROW) + x.dv0,
+        size_t(x.H) * *x.misc(M_OROW), x.tend - ts, hf * 128 + dv);
   }
 }
 
@@ -1325,10 +1340,10 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
   const bool obf = a.o_bf16 != 0;
   bool ok;
   if (a.cu_seqlens) {
-    // packed sequences (fp32 o; the pre-steps on request): their own
+    // packed sequences (the pre-steps and bf16 o on request): their own
     // instantiations, so that the dense kernels carry none of the per-sequence paths
     const bool c64 = chunk == 64;
-    if (!pre) {
+    if (!pre && !obf) {
       if (a.Dk == D)
         ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, false, false, 128, 128, true>, 55)
                                   : go(prefill_kernel<16, false, false, 128, 128, true>, 56))
@@ -1339,6 +1354,19 @@ int launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorM
                                   : go(prefill_kernel<16, false, false, 64, 128, true>, 60))
                            : (c64 ? go(prefill_kernel<64, false, false, 64, 64, true>, 61)
                                   : go(prefill_kernel<16, false, false, 64, 64, true>, 62));
+    } else if (obf) {
+      // bf16 o: the pre-step instantiations (with no pre-step requested their
+      // factors are exactly 1)
+      if (a.Dk == D)
+        ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, true, true, 128, 128, true>, 78)
+                                  : go(prefill_kernel<16, true, true, 128, 128, true>, 79))
+                           : (c64 ? go(prefill_kernel<64, true, true, 128, 64, true>, 80)
+                                  : go(prefill_kernel<16, true, true, 128, 64, true>, 81));
+      else
+        ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, true, true, 64, 128, true>, 82)
+                                  : go(prefill_kernel<16, true, true, 64, 128, true>, 83))
+                           : (c64 ? go(prefill_kernel<64, true, true, 64, 64, true>, 84)
+                                  : go(prefill_kernel<16, true, true, 64, 64, true>, 85));
     } else {
       if (a.Dk == D)
         ok = a.dv_box == D ? (c64 ? go(prefill_kernel<64, true, false, 128, 128, true>, 67)

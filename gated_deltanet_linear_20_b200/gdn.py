@@ -234,7 +234,7 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
                    S_T: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
                    snap_every: int = 0,
                    snaps: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
-                   q_scale: float = 1.0):
+                   q_scale: float = 1.0, o_bf16: bool = False):
     """Prefill of N packed sequences: q, k [total_T,H,Dk] bf16; v [total_T,H,Dv] bf16;
     g, beta [total_T,H] fp32; cu_seqlens int32 [N+1] on the device (offsets of
     the sequences).  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,Dk] fp32).
@@ -243,7 +243,8 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     by sequence); ``snaps`` may be given preallocated, else its size is read
     from cu_seqlens (one device-to-host copy).  Dk 64 or 128, Dv 64, 128 or
     256 (the chunked tensor-core kernel).  ``qk_l2norm`` / ``q_scale`` apply the
-    fused pre-steps of ``prefill`` (gdn_prefill_varlen_ex)."""
+    fused pre-steps of ``prefill`` and ``o_bf16`` writes o as bf16
+    (gdn_prefill_varlen_ex)."""
     if q.dim() != 3:
         raise ValueError("q must be [total_T,H,Dk]")
     total_T, H, Dk = q.shape
@@ -262,9 +263,10 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
     _check(beta, "beta", torch.float32, (total_T, H), dev)
     if S0 is not None:
         _check(S0, "S0", torch.float32, (N, H, Dv, Dk), dev)
+    o_dtype = torch.bfloat16 if o_bf16 else torch.float32
     if o is None:
-        o = torch.empty((total_T, H, Dv), dtype=torch.float32, device=dev)
-    _check(o, "o", torch.float32, (total_T, H, Dv), dev)
+        o = torch.empty((total_T, H, Dv), dtype=o_dtype, device=dev)
+    _check(o, "o", o_dtype, (total_T, H, Dv), dev)
     if S_T is None:
         S_T = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=dev)
     _check(S_T, "S_T", torch.float32, (N, H, Dv, Dk), dev)
@@ -280,7 +282,7 @@ def prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: torch.T
         _check(snaps, "snaps", torch.float32, (n_snaps, H, Dv, Dk), dev)
     else:
         snaps = None
-    opts = _options(qk_l2norm, q_scale)
+    opts = _options(qk_l2norm, q_scale, o_bf16)
     if opts is None:
         rc = _lib.gdn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
                                      _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk, Dv,
@@ -468,13 +470,14 @@ def kda_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: tor
                        S_T: Optional[torch.Tensor] = None,
                        status: Optional[torch.Tensor] = None, snap_every: int = 0,
                        snaps: Optional[torch.Tensor] = None, qk_l2norm: bool = False,
-                       q_scale: float = 1.0):
+                       q_scale: float = 1.0, o_bf16: bool = False):
     """Per-channel-gate prefill of N packed sequences (gdn_kda_prefill_varlen):
     q, k [total_T,H,128] bf16; v [total_T,H,Dv] bf16 (Dv 64, 128 or 256);
     g [total_T,H,128] fp32; beta [total_T,H] fp32; cu_seqlens int32 [N+1] on
-    the device.  Returns (o [total_T,H,Dv] fp32, S_T [N,H,Dv,128] fp32), and
+    the device.  Returns (o [total_T,H,Dv] fp32 or bf16, S_T [N,H,Dv,128] fp32), and
     with ``snap_every`` (a multiple of 32) the state snapshots as in
-    ``prefill_varlen``.  ``qk_l2norm`` / ``q_scale`` as in ``kda_prefill``."""
+    ``prefill_varlen``.  ``qk_l2norm``, ``q_scale`` and ``o_bf16`` as in
+    ``kda_prefill``."""
     if q.dim() != 3:
         raise ValueError("q must be [total_T,H,Dk]")
     total_T, H, Dk = q.shape
@@ -493,9 +496,10 @@ def kda_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: tor
     _check(beta, "beta", torch.float32, (total_T, H), dev)
     if S0 is not None:
         _check(S0, "S0", torch.float32, (N, H, Dv, Dk), dev)
+    o_dtype = torch.bfloat16 if o_bf16 else torch.float32
     if o is None:
-        o = torch.empty((total_T, H, Dv), dtype=torch.float32, device=dev)
-    _check(o, "o", torch.float32, (total_T, H, Dv), dev)
+        o = torch.empty((total_T, H, Dv), dtype=o_dtype, device=dev)
+    _check(o, "o", o_dtype, (total_T, H, Dv), dev)
     if S_T is None:
         S_T = torch.empty((N, H, Dv, Dk), dtype=torch.float32, device=dev)
     _check(S_T, "S_T", torch.float32, (N, H, Dv, Dk), dev)
@@ -511,7 +515,7 @@ def kda_prefill_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, g: tor
         _check(snaps, "snaps", torch.float32, (n_snaps, H, Dv, Dk), dev)
     else:
         snaps = None
-    opts = _options(qk_l2norm, q_scale)
+    opts = _options(qk_l2norm, q_scale, o_bf16)
     if opts is None:
         rc = _lib.gdn_kda_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0),
                                          _ptr(o), _ptr(S_T), _ptr(cu_seqlens), N, total_T, H, Dk,

@@ -181,8 +181,9 @@ int gdn_prefill_varlen(const void* q, const void* k, const void* v, const float*
 
 /* gdn_prefill_varlen with options (gdn_options; NULL = none): qk_l2norm
  * and q_scale as in gdn_prefill_ex, applied to every token of every packed
- * sequence.  o_bf16 is not offered on packed sequences (GDN_ERR_UNSUPPORTED,
- * as for an invalid struct).  Everything else as for gdn_prefill_varlen. */
+ * sequence, and o_bf16 writes o as bf16 (the fp32 value rounded to nearest
+ * even; o then needs total_T*H*Dv*2 bytes).  Everything else as for
+ * gdn_prefill_varlen. */
 int gdn_prefill_varlen_ex(const void* q, const void* k, const void* v, const float* g,
                           const float* beta, const float* S0, float* o, float* S_T,
                           const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
@@ -369,9 +370,8 @@ int gdn_kda_prefill_varlen(const void* q, const void* k, const void* v, const fl
                            const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,
                            float* snaps, int snap_every, int n_snaps, int* status, void* stream);
 
-/* gdn_kda_prefill_varlen with options: qk_l2norm and q_scale as in
- * gdn_kda_prefill_ex; o_bf16 is GDN_ERR_UNSUPPORTED here.  Everything else as
- * for gdn_kda_prefill_varlen. */
+/* gdn_kda_prefill_varlen with options: qk_l2norm, q_scale and o_bf16 as in
+ * gdn_kda_prefill_ex.  Everything else as for gdn_kda_prefill_varlen. */
 int gdn_kda_prefill_varlen_ex(const void* q, const void* k, const void* v, const float* g,
                               const float* beta, const float* S0, float* o, float* S_T,
                               const int* cu_seqlens, int N, int total_T, int H, int Dk, int Dv,

@@ -503,14 +503,13 @@ def test_kda_prefill_varlen_valid_calls_pass_validation(gdn, dv):
 
 
 def test_packed_calls_take_the_pre_step_options(gdn):
-    """gdn_prefill_varlen_ex and gdn_kda_prefill_varlen_ex accept qk_l2norm and
-    q_scale (the call then fails only for want of a device), reject o_bf16, a
+    """gdn_prefill_varlen_ex and gdn_kda_prefill_varlen_ex accept qk_l2norm,
+    q_scale and o_bf16 (the call then fails only for want of a device), reject a
     short struct and a NaN scale (GDN_ERR_UNSUPPORTED), and validate every other
-    argument as the calls without options do."""
+    argument as the calls without options do (o sized by its element type)."""
     import ctypes as ct
-    good = ct.byref(gdn.Options(ct.sizeof(gdn.Options), 1, 0.5, 0))
-    bad = [ct.byref(gdn.Options(ct.sizeof(gdn.Options), 1, 1.0, 1)),
-           ct.byref(gdn.Options(4, 1, 1.0)),
+    good = ct.byref(gdn.Options(ct.sizeof(gdn.Options), 1, 0.5, 1))
+    bad = [ct.byref(gdn.Options(4, 1, 1.0)),
            ct.byref(gdn.Options(ct.sizeof(gdn.Options), 0, float("nan")))]
     with_opts = lambda a, o: a[:18] + [o] + a[18:]
     for dk, dv in ((128, 128), (64, 64), (128, 256)):
@@ -529,3 +528,8 @@ def test_packed_calls_take_the_pre_step_options(gdn):
             assert gdn.raw_kda_prefill_varlen_ex(*kwith(a, o)) == -4
     assert gdn.raw_kda_prefill_varlen_ex(*kwith(kda_varlen_args(Dk=64, Dv=64), good)) == -4
     assert gdn.raw_kda_prefill_varlen_ex(*kwith(kda_varlen_args(cu=None), good)) == -1
+    # 200 tokens x 2 heads x 128: o runs 200 KiB as fp32, 100 KiB as bf16
+    plain = ct.byref(gdn.Options(ct.sizeof(gdn.Options), 0, 1.0, 0))
+    o = P + 0x7000000 - 128 * 1024                # 128 KiB before cu_seqlens
+    assert gdn.raw_kda_prefill_varlen_ex(*kwith(kda_varlen_args(o=o), plain)) == -5
+    assert gdn.raw_kda_prefill_varlen_ex(*kwith(kda_varlen_args(o=o), good)) not in VALIDATION_CODES + (0,)

@@ -575,3 +575,37 @@ def test_scalar_varlen_fused_qk_norm_and_q_scale(dk, dv, chunk):
                                 d["beta"], d["S0"])
         assert_parity(o[t0:t1], ro[0], f"o seq {n} (fused norm)")
         assert_parity(S_T[n], rS[0], f"S_T seq {n} (fused norm)")
+
+
+@pytest.mark.parametrize("gate,dims", [("kda", (128, 128)), ("kda", (128, 256)), ("kda", (128, 64)),
+                                       ("scalar", (128, 128)), ("scalar", (64, 64)),
+                                       ("scalar", (128, 256))],
+                         ids=["kda_128", "kda_256", "kda_64", "scalar_128x128", "scalar_64x64",
+                              "scalar_128x256"])
+def test_varlen_bf16_o_is_the_fp32_o_rounded(gate, dims):
+    """Packed sequences with bf16 o (the ragged last tile of each sequence
+    copied out as bf16 rows) give the fp32 call's o rounded to nearest even,
+    bit for bit, and the same S_T and snapshots."""
+    dk, dv = dims
+    lengths = [130, 0, 1, 64, 77, 33]
+    H = 2
+    if gate == "kda":
+        seqs, pk = _kda_packed(lengths, H, dv, seed=900 + dv, s0_std=0.05)
+        call, every = _gdn().kda_prefill_varlen, 64
+    else:
+        seqs = [inputs.prefill_inputs(1, L, H, dk, dv, seed=910 + i, s0_std=0.05)
+                for i, L in enumerate(lengths)]
+        cat = lambda key: torch.cat([d[key][0] for d in seqs], 0)
+        pk = dict(q=cat("q"), k=cat("k"), v=cat("v"), g=cat("g"), beta=cat("beta"),
+                  S0=torch.cat([d["S0"] for d in seqs], 0),
+                  cu=torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32))
+        call, every = _gdn().prefill_varlen, 64
+    dd = to_dev(pk)
+    args = (dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"], dd["S0"])
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o32, S32, sn32 = call(*args, status=status, snap_every=every)
+    o16, S16, sn16 = call(*args, status=status, snap_every=every, o_bf16=True)
+    assert _gdn().query_status(status) == 0
+    assert o16.dtype == torch.bfloat16
+    assert torch.equal(o16, o32.to(torch.bfloat16))
+    assert torch.equal(S16, S32) and torch.equal(sn16, sn32)
