@@ -854,6 +854,7 @@ PROFILE_CASES = {
     "kda_b1_h16_t512": (None, None, 3),       # per-channel gate, headline shape
     "kda_b4_h32_t2048": (None, None, 3),      # per-channel gate, a large batch
     "kda_decode": (None, None, 5),            # per-channel gate, B64 H16 one token
+    "kda_varlen_32seq_h16": (None, None, 3),  # per-channel gate, the packed 32-sequence workload
 }
 
 
@@ -863,7 +864,17 @@ def run_profile_case(name):
     from gated_deltanet_linear_20_b200 import gdn
     dev = torch.device("cuda", 0)
     wname, chunk, calls = PROFILE_CASES[name]
-    if name.startswith("kda"):
+    if name == "kda_varlen_32seq_h16":
+        # the packed workload of the benchmark's extras (rank 0's draw)
+        lens = np.random.default_rng(4000).integers(64, 2049, size=32)
+        seqs = [gin.kda_inputs(1, int(L), 16, seed=5200 + i, device=str(dev))
+                for i, L in enumerate(lens)]
+        pk = {key: torch.cat([d[key][0] for d in seqs], 0) for key in ("q", "k", "v", "g", "beta")}
+        del seqs
+        cu = torch.tensor([0] + np.cumsum(lens).tolist(), dtype=torch.int32, device=dev)
+        for _ in range(calls):
+            gdn.kda_prefill_varlen(pk["q"], pk["k"], pk["v"], pk["g"], pk["beta"], cu)
+    elif name.startswith("kda"):
         B, T, H = {"kda_b1_h16_t512": (1, 512, 16), "kda_b4_h32_t2048": (4, 2048, 32),
                    "kda_decode": (64, calls, 16)}[name]
         d = gin.kda_inputs(B, T, H, seed=0, g_mean=2.0 if B == 4 else 0.0,
