@@ -892,7 +892,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                            ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
-  const int chain = DV2 ? int(blockIdx.x) >> 1 : int(blockIdx.x);
+  int chain = DV2 ? int(blockIdx.x) >> 1 : int(blockIdx.x);
   int b = chain / p.H;
   const int h = chain - (chain / p.H) * p.H;
   int ntiles = (p.T + NT - 1) / NT;
@@ -900,6 +900,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   float* snap = nullptr;   // this CTA's first snapshot row (packed sequences)
   int stiles = 1;
   if constexpr (PK) {
+    // longest sequences first: CTAs start in index order, so slot r of the
+    // grid takes the sequence of rank r by (length descending, index), a
+    // bijection whatever the offsets hold; the shorter chains then fill the
+    // SMs the long ones leave.  Up to one sequence per thread (else index order).
+    if (p.B <= NTHREADS) {
+      int* lens = reinterpret_cast<int*>(sm + SM_G);  // scratch: g(0) is not issued yet
+      for (int i = tid; i < p.B; i += NTHREADS)
+        lens[i] = __ldg(p.cu_seqlens + i + 1) - __ldg(p.cu_seqlens + i);
+      __syncthreads();
+      if (tid < p.B) {
+        const int L = lens[tid];
+        int rank = 0;
+        for (int m = 0; m < p.B; ++m) {
+          const int Lm = lens[m];
+          rank += (Lm > L || (Lm == L && m < tid)) ? 1 : 0;
+        }
+        if (rank == b) lens[NTHREADS] = tid;
+      }
+      __syncthreads();
+      b = lens[NTHREADS];
+      chain = b * p.H + h;
+    }
     // packed sequences: chain n H + h walks tokens [cu[n], cu[n+1]) of views with B = 1
     tb = __ldg(p.cu_seqlens + b);
     tend = __ldg(p.cu_seqlens + b + 1);
