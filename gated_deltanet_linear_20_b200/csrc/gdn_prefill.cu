@@ -1183,6 +1183,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     frun = j >= p.nseg;
     seg = frun ? j - p.nseg + 1 : j;
   }
+  if constexpr (PK) {
+    // longest sequences first: CTAs start in index order, so slot n H + h of the
+    // grid takes the sequence of rank n by (length descending, index), a
+    // bijection whatever the offsets hold; the shorter chains then fill the SMs
+    // the long ones leave.  Up to one sequence per thread (else index order).
+    if (p.B <= NTHREADS) {
+      int* lens = reinterpret_cast<int*>(sm + SM_A);  // scratch: the solve has not started
+      for (int i = tid; i < p.B; i += NTHREADS)
+        lens[i] = __ldg(p.cu_seqlens + i + 1) - __ldg(p.cu_seqlens + i);
+      __syncthreads();
+      const int r = chain / p.H;
+      if (tid < p.B) {
+        const int L = lens[tid];
+        int rank = 0;
+        for (int m = 0; m < p.B; ++m) {
+          const int Lm = lens[m];
+          rank += (Lm > L || (Lm == L && m < tid)) ? 1 : 0;
+        }
+        if (rank == r) lens[NTHREADS] = tid;
+      }
+      __syncthreads();
+      chain = lens[NTHREADS] * p.H + (chain - r * p.H);
+    }
+  }
   int b = chain / p.H;
   const int h = chain - b * p.H;
   const size_t cstate = size_t(chain) * p.Dv * DK;  // this chain's state
