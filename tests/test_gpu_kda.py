@@ -609,3 +609,37 @@ def test_varlen_bf16_o_is_the_fp32_o_rounded(gate, dims):
     assert o16.dtype == torch.bfloat16
     assert torch.equal(o16, o32.to(torch.bfloat16))
     assert torch.equal(S16, S32) and torch.equal(sn16, sn32)
+
+
+@pytest.mark.parametrize("gate", ["kda", "scalar"])
+def test_varlen_many_sequences_keep_index_order(gate):
+    """More sequences than a CTA has threads (520, of 0..40 tokens, one head):
+    the longest-first ordering is skipped and every sequence still matches the
+    oracle run on it alone."""
+    rng = np.random.default_rng(950)
+    lengths = [int(x) for x in rng.integers(0, 41, size=520)]
+    if gate == "kda":
+        seqs, pk = _kda_packed(lengths, 1, 128, seed=960, s0_std=0.05)
+    else:
+        seqs = [inputs.prefill_inputs(1, L, 1, seed=960 + i, s0_std=0.05) for i, L in enumerate(lengths)]
+        cat = lambda key: torch.cat([d[key][0] for d in seqs], 0)
+        pk = dict(q=cat("q"), k=cat("k"), v=cat("v"), g=cat("g"), beta=cat("beta"),
+                  S0=torch.cat([d["S0"] for d in seqs], 0),
+                  cu=torch.tensor([0] + list(np.cumsum(lengths)), dtype=torch.int32))
+    dd = to_dev(pk)
+    gdn = _gdn()
+    call = gdn.kda_prefill_varlen if gate == "kda" else gdn.prefill_varlen
+    ref = oracle.kda_prefill if gate == "kda" else oracle.prefill
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o, S_T = call(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu"], dd["S0"], status=status)
+    assert gdn.query_status(status) == 0
+    o, S_T = o.cpu().numpy(), S_T.cpu().numpy()
+    cu = pk["cu"].numpy()
+    for n in range(0, 520, 7):
+        d = seqs[n]
+        if not lengths[n]:
+            np.testing.assert_array_equal(S_T[n], d["S0"][0].numpy())
+            continue
+        ro, rS = ref(d["q"], d["k"], d["v"], d["g"], d["beta"], d["S0"])
+        assert_parity(o[cu[n]:cu[n + 1]], ro[0], f"o seq {n} (len {lengths[n]})")
+        assert_parity(S_T[n], rS[0], f"S_T seq {n} (len {lengths[n]})")
