@@ -361,7 +361,8 @@ int gdn_kda_decode_ex(const void* q, const void* k, const void* v, const float* 
  *                that snap_every is a positive multiple of 32 (the kernel's
  *                chunk); NULL snaps: none.
  * Dk must be 128 and Dv 64, 128 or 256 (the chunked tensor-core kernel, one
- * CTA per chain, two with Dv = 256); no options.  N*H == 0 is a no-op.
+ * CTA per chain, two with Dv = 256); options through the _ex call below.
+ * N*H == 0 is a no-op.
  * status: optional device int; GDN_ERR_SHAPE (offsets, snapshot slots) or
  * GDN_ERR_DEVICE_TIMEOUT (a bounded wait gave up) is stored there.  Returns
  * GDN_OK, or a negative code for invalid arguments (nothing is launched). */
